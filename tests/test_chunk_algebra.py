@@ -1,0 +1,157 @@
+"""fp64 check of the chunkwise equations the CUDA kernels implement (CPU only).
+
+The pages say a chunkwise algorithm with diagonal-plus-low-rank structure
+exists ("Kimi Linear acaba de superar a la atencion completa...", the section
+on the chunk training algorithm and the DPLR transition) but print no
+equations.  The chunk form below is derived by unrolling the per-token step of
+"Kimi Delta Attention: la atencion lineal detras de Kimi K2 y Qwen3" (section
+"Como funciona Kimi Delta Attention paso a paso"), and this file proves it
+equals the token recurrence (the oracle) to fp64 rounding -- including the
+16-token sub-chunk reference points used to keep every exponential factor in
+range, the blocked inversion of (I + A), partial last chunks and h0 != 0.
+It is written in numpy, shares nothing with the CUDA sources and imports only
+the oracle.
+
+Per chunk of C tokens (padded with g = 0, beta = 0, k = q = v = 0), with
+G_i = sum_{j <= i} g_j (inclusive, restarting at the chunk):
+  A_ij   = beta_i sum_c k_ic k_jc e^{G_ic - G_jc}          (i > j)
+  Aqk_ij = scale  sum_c q_ic k_jc e^{G_ic - G_jc}          (i >= j)
+  T      = (I + A)^{-1}
+  W      = T diag(beta) (K * e^G),   Ut = T diag(beta) V
+  U      = Ut - W S,   O = scale (Q * e^G) S + Aqk U
+  S'     = Diag(e^{G_last}) S + (K * e^{G_last - G})^T U
+"""
+import numpy as np
+import pytest
+
+import oracle
+
+C, SC = 64, 16
+
+
+def blocked_unit_lower_inverse(A, sc=SC):
+    """(I + A)^{-1} for strictly lower A: invert the sc x sc diagonal blocks by
+    forward substitution, then fill block (p, r) as
+    -T_pp * sum_{r <= m < p} A_pm T_mr, block-row by block-row."""
+    n = A.shape[0]
+    nb = n // sc
+    T = np.zeros_like(A)
+    for p in range(nb):
+        s = slice(p * sc, (p + 1) * sc)
+        Ab = A[s, s]
+        Tb = np.eye(sc)
+        for i in range(sc):
+            for c in range(i):
+                Tb[i, c] = -sum(Ab[i, j] * Tb[j, c] for j in range(c, i))
+        T[s, s] = Tb
+    for p in range(1, nb):
+        sp = slice(p * sc, (p + 1) * sc)
+        for r in range(p - 1, -1, -1):
+            sr = slice(r * sc, (r + 1) * sc)
+            acc = np.zeros((sc, sc))
+            for m in range(r, p):
+                sm = slice(m * sc, (m + 1) * sc)
+                acc += A[sp, sm] @ T[sm, sr]
+            T[sp, sr] = -T[sp, sp] @ acc
+    return T
+
+
+def chunk_intra(qc, kc, vc, gc, bc, scale):
+    """Intra-chunk quantities for one padded chunk (C rows)."""
+    G = np.cumsum(gc, axis=0)
+    f = (np.arange(C) // SC) * SC
+    Kin = kc * np.exp(G - G[f])          # every factor <= 1
+    Qin = qc * np.exp(G - G[f])
+    Akk = np.zeros((C, C))
+    Aqk = np.zeros((C, C))
+    for p in range(C // SC):
+        fp = p * SC
+        n = fp + SC
+        Kvar = kc[:n] * np.exp(G[fp] - G[:n])   # <= 1 before fp, >= 1 (<= 15 tokens) after
+        rows = slice(fp, n)
+        Akk[rows, :n] = Kin[rows] @ Kvar.T
+        Aqk[rows, :n] = Qin[rows] @ Kvar.T
+    A = np.tril(Akk, -1) * bc[:, None]
+    Aqk = np.tril(Aqk, 0) * scale
+    T = blocked_unit_lower_inverse(A)
+    W = T @ (bc[:, None] * kc * np.exp(G))
+    Ut = T @ (bc[:, None] * vc)
+    QG = scale * qc * np.exp(G)
+    KGl = kc * np.exp(G[-1] - G)
+    return dict(G=G, A=A, T=T, W=W, Ut=Ut, Aqk=Aqk, QG=QG, KGl=KGl, gam=np.exp(G[-1]))
+
+
+def chunk_forward(q, k, v, g, b, h0, scale):
+    """One (sequence, head): q,k [L,dk], v [L,dv], g [L,dk], b [L]."""
+    L, dk = k.shape
+    dv = v.shape[1]
+    S = h0.copy()
+    out = np.zeros((L, dv))
+    for s0 in range(0, L, C):
+        n = min(C, L - s0)
+        pad = lambda x: np.concatenate([x[s0:s0 + n], np.zeros((C - n,) + x.shape[1:])])
+        I = chunk_intra(pad(q), pad(k), pad(v), pad(g), pad(b), scale)
+        U = I["Ut"] - I["W"] @ S
+        O = I["QG"] @ S + I["Aqk"] @ U
+        S = I["gam"][:, None] * S + I["KGl"].T @ U
+        out[s0:s0 + n] = O[:n]
+    return out, S
+
+
+def _inputs(rng, L, dk, dv, gate_shift=0.0):
+    q = rng.standard_normal((L, dk)); q /= np.linalg.norm(q, axis=1, keepdims=True)
+    k = rng.standard_normal((L, dk)); k /= np.linalg.norm(k, axis=1, keepdims=True)
+    v = rng.standard_normal((L, dv))
+    g = -np.log1p(np.exp(rng.standard_normal((L, dk)) + gate_shift))
+    b = 1.0 / (1.0 + np.exp(-rng.standard_normal(L)))
+    return q, k, v, g, b
+
+
+@pytest.mark.parametrize("L", [1, 15, 64, 100, 193, 256])
+def test_chunk_form_equals_token_recurrence(L):
+    rng = np.random.default_rng(100 + L)
+    dk, dv, scale = 16, 12, 0.25
+    q, k, v, g, b = _inputs(rng, L, dk, dv)
+    h0 = 0.5 * rng.standard_normal((dk, dv))
+    out, hT = chunk_forward(q, k, v, g, b, h0, scale)
+    o_ref, h_ref = oracle.fwd(q[None, :, None], k[None, :, None], v[None, :, None],
+                              g[None, :, None], b[None, :, None], scale, h0=h0[None, None])
+    np.testing.assert_allclose(out, o_ref[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(hT, h_ref[0, 0], rtol=0, atol=1e-12)
+
+
+def test_fast_decay_stays_finite_and_exact():
+    """Mean per-token decay about e^-3.1 (gate shift +3): the sub-chunk
+    references keep every factor finite; the result still matches."""
+    rng = np.random.default_rng(3)
+    L, dk, dv, scale = 160, 16, 8, 0.25
+    q, k, v, g, b = _inputs(rng, L, dk, dv, gate_shift=3.0)
+    out, hT = chunk_forward(q, k, v, g, b, np.zeros((dk, dv)), scale)
+    assert np.all(np.isfinite(out)) and np.all(np.isfinite(hT))
+    o_ref, h_ref = oracle.fwd(q[None, :, None], k[None, :, None], v[None, :, None],
+                              g[None, :, None], b[None, :, None], scale)
+    np.testing.assert_allclose(out, o_ref[0, :, 0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(hT, h_ref[0, 0], rtol=0, atol=1e-12)
+
+
+def test_blocked_inverse():
+    rng = np.random.default_rng(4)
+    A = np.tril(rng.standard_normal((C, C)) * 0.3, -1)
+    T = blocked_unit_lower_inverse(A)
+    np.testing.assert_allclose(T @ (np.eye(C) + A), np.eye(C), rtol=0, atol=1e-10)
+    np.testing.assert_array_equal(np.triu(T, 1), 0.0)
+    np.testing.assert_array_equal(np.diag(T), 1.0)
+
+
+def test_chunk_is_one_affine_map():
+    """Each chunk maps S -> M S + Bm with M = Diag(e^{G_last}) - KGl^T W and
+    Bm = KGl^T Ut (the form a sequence-parallel scan would compose)."""
+    rng = np.random.default_rng(5)
+    dk, dv, scale = 8, 6, 0.3
+    q, k, v, g, b = _inputs(rng, C, dk, dv)
+    I = chunk_intra(q, k, v, g, b, scale)
+    M = np.diag(I["gam"]) - I["KGl"].T @ I["W"]
+    Bm = I["KGl"].T @ I["Ut"]
+    S0 = rng.standard_normal((dk, dv))
+    _, S1 = chunk_forward(q, k, v, g, b, S0, scale)
+    np.testing.assert_allclose(M @ S0 + Bm, S1, rtol=0, atol=1e-12)
