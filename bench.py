@@ -1,0 +1,432 @@
+#!/usr/bin/env python
+"""Throughput of the KDA hot path on B200: chunkwise prefill tokens/s (with
+tensor-core and HBM fractions) and decode-step state GB/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+One step = one chunkwise forward (cumulative decay, intra-chunk transform,
+state propagation, output) over the batched-prefill workload B=8, H=32,
+T=8192, dk=dv=128, bf16 q/k/v/out with fp32 gates and state, seeded synthetic
+inputs (3.2 GB per step, larger than L2).  The decode workload (N=256, H=32,
+d=128, 1000 chained steps) is timed in the same run and reported under
+"decode".  Multi-GPU: one process per GPU under torchrun; every rank runs the
+same workload on its own GPU with no collective on the data path (weak
+scaling); the timed region is bracketed by barriers and the max over ranks is
+reported.  `--impl reference` times the fp64 CPU oracle on a bounded sample of
+the same workload instead (rank 0 only).
+"""
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+import workloads as W  # noqa: E402
+
+METRIC = "KDA fwd tokens/sec (H=32,d=128,bf16) + % TC peak; decode-step state GB/s vs HBM"
+CHUNK = 64
+BYTES_PER_HEAD_TOKEN = 1540        # q,k,v,out bf16 (4*256) + log_alpha fp32 (512) + beta (4)
+FLOP_PER_HEAD_TOKEN = 2 * CHUNK * (3 * 128 + 2 * 128) + 6 * 128 * 128   # 180,224 at C=64, d=128
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained"), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "source": "fallback"}
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.3)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[4:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        pmax = max(r[2] for r in rows)
+        loaded = [r for r in rows if r[2] >= 0.5 * pmax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in loaded for i, v in enumerate(r[3][1:5])
+                          if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in loaded),
+                "sm_max_mhz": max(r[1] for r in loaded), "power_w_max": pmax,
+                "samples": len(loaded), "reasons": reasons}
+
+
+# ----------------------------------------------------------------------------
+# distributed plumbing
+# ----------------------------------------------------------------------------
+def dist_setup():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=600))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return ws, rank, local
+
+
+def barrier(ws):
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, ws):
+    if ws == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------
+# oracle timing (CPU baseline / reference arm)
+# ----------------------------------------------------------------------------
+def oracle_sample(inp_host, cfg, heads):
+    """Oracle on batch entry 0 and the first `heads` heads of the workload."""
+    import oracle
+    sl = lambda x: x[0:1, :, :heads].contiguous()
+    t = time.perf_counter()
+    oracle.fwd(sl(inp_host["q"]), sl(inp_host["k"]), sl(inp_host["v"]), sl(inp_host["log_alpha"]),
+               sl(inp_host["beta"]), inp_host["scale"], return_state=True)
+    dt = time.perf_counter() - t
+    head_tokens = cfg.T * heads
+    return dt, head_tokens, oracle.threads()
+
+
+def host_sample_inputs(cfg, heads):
+    """The same seeded workload generated on the host, restricted to batch 0
+    and `heads` heads (the generator is the one the GPU run uses, on CPU)."""
+    small = W.PrefillConfig(cfg.name, 1, cfg.T, heads, cfg.dk, cfg.dv, cfg.io_dtype, cfg.seed,
+                            cfg.gate_shift, cfg.h0_std)
+    return W.make_prefill(small, "cpu")
+
+
+def run_reference(args, ws, rank):
+    cfg = W.BATCHED
+    if rank != 0:
+        return
+    heads = 4
+    inp = host_sample_inputs(cfg, heads)
+    for _ in range(args.warmup):
+        oracle_sample(inp, cfg, heads)
+    times = []
+    threads = 1
+    for _ in range(args.steps):
+        dt, ht, threads = oracle_sample(inp, cfg, heads)
+        times.append(dt)
+    total = sum(times)
+    value = cfg.T * heads * args.steps / total / cfg.H     # tokens/s at H=32 equivalent
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * total / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": workload_config(cfg),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"batch entry 0, heads 0..{heads - 1}, all {cfg.T} tokens per "
+                                   f"step ({cfg.T * heads} head-tokens); tokens/s = head-tokens/s / {cfg.H}"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def workload_config(cfg):
+    return {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv,
+            "chunk": CHUNK, "io": cfg.io_dtype, "gates_state": "fp32",
+            "l2": "inputs larger than L2 (3.2 GB read per step)",
+            "parallelism": "independent replica per GPU (weak scaling, no collective)"}
+
+
+# ----------------------------------------------------------------------------
+# the GPU arm
+# ----------------------------------------------------------------------------
+def time_region(fn, steps, stream):
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        fn()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1)
+
+
+def run_prefill(args, ws, rank, kda, peaks):
+    cfg = W.BATCHED
+    inp = W.make_prefill(cfg, "cuda")
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
+    hT = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
+                      h0=inp["h0"], out=out, hT=hT, impl=args.prefill_impl)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    kda.profiler_read(reset=True)
+    kda.profiler_enable(True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier(ws)
+        torch.cuda.synchronize()
+        ms = time_region(step, args.steps, stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+    kda.profiler_enable(False)
+    stats = kda.profiler_read(reset=True)
+    ms_max = max_over_ranks(ms, ws)
+    tokens = cfg.B * cfg.T * args.steps * ws
+    value = tokens / (ms_max / 1e3)
+    head_tokens_per_step = cfg.B * cfg.T * cfg.H
+    launches = sum(v[0] for v in stats.values())
+    # dominant kernel = largest share of event time
+    kern = max(stats.items(), key=lambda kv: kv[1][2])
+    kname, (kl, ktimed, kms) = kern
+    k_ms_per_step = kms / args.steps
+    k_ms_per_launch = kms / max(1, ktimed)
+    launches_per_step = ktimed / args.steps
+    algo_bytes_step = BYTES_PER_HEAD_TOKEN * head_tokens_per_step
+    algo_flop_step = FLOP_PER_HEAD_TOKEN * head_tokens_per_step
+    path_gbs = algo_bytes_step / (ms_max / args.steps / 1e3) / 1e9
+    path_tflops = algo_flop_step / (ms_max / args.steps / 1e3) / 1e12
+    kbytes = kernel_algorithmic_bytes(kname, cfg) / max(1.0, launches_per_step)
+    roof = {"kernel": kname, "bound": "hbm", "achieved": kbytes / (k_ms_per_launch / 1e3) / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s",
+            "frac": None, "traffic": None, "launches_per_step": launches_per_step,
+            "ms_per_launch": k_ms_per_launch, "share_of_step": k_ms_per_step / (ms_max / args.steps),
+            "algorithmic_bytes_per_launch": kbytes, "peak_source": peaks["source"] + " (burst copy)"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    res = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": workload_config(cfg),
+        "prefill_impl": args.prefill_impl,
+        "tc_frac": path_tflops / (peaks["bf16_tflops"]),
+        "hbm_frac": path_gbs / peaks["hbm_gbs"],
+        "path": {"algorithmic_GBps": path_gbs, "algorithmic_TFLOPs": path_tflops,
+                 "bytes_per_head_token": BYTES_PER_HEAD_TOKEN,
+                 "flop_per_head_token": FLOP_PER_HEAD_TOKEN,
+                 "peaks": {"hbm_gbs": peaks["hbm_gbs"], "bf16_tflops": peaks["bf16_tflops"],
+                           "source": peaks["source"]}},
+        "roofline": roof,
+        "kernels": {k: {"launches": v[0], "ms": v[2]} for k, v in stats.items() if v[0]},
+        "gpu_launches": launches,
+        "clocks": clk.summary(),
+    }
+    return res, inp, step, (out, hT)
+
+
+def kernel_algorithmic_bytes(kname, cfg):
+    """Minimal bytes the named kernel must move for one step of the workload."""
+    ht = cfg.B * cfg.T * cfg.H
+    chunks = cfg.B * math.ceil(cfg.T / CHUNK) * cfg.H
+    dk, dv = cfg.dk, cfg.dv
+    io = 2 if cfg.io_dtype == "bf16" else 4
+    qkvgb = ht * ((2 * dk + dv) * io + dk * 4 + 4)
+    if kname == "chunk_prep_simt":       # reads q,k,v,g,beta; writes fp32 W,Ut,Aqk,QG,KG,gamma
+        return qkvgb + chunks * 4 * (CHUNK * (3 * dk + dv + CHUNK) + dk)
+    if kname == "chunk_state_simt":      # reads the fp32 workspace (Ut once, the rest per dv tile)
+        tiles = dv // 32
+        per_chunk = 4 * (CHUNK * dv + tiles * (CHUNK * 3 * dk + CHUNK * CHUNK + dk))
+        return chunks * per_chunk + ht * dv * io + cfg.B * cfg.H * dk * dv * 4
+    if kname == "chunk_prep_tc":
+        return qkvgb + chunks * TC_WS_BYTES_PER_CHUNK
+    if kname == "chunk_state_tc":
+        return chunks * TC_WS_BYTES_PER_CHUNK + ht * dv * io + cfg.B * cfg.H * dk * dv * 4
+    return BYTES_PER_HEAD_TOKEN * ht
+
+
+TC_WS_BYTES_PER_CHUNK = 72 * 1024 + 512
+
+
+def run_decode(args, ws, rank, kda, peaks):
+    cfg = W.DECODE
+    gen = W.decode_generator(cfg, "cuda")
+    S = W.make_decode_state(cfg, gen, "cuda")
+    steps_in = [W.make_decode_step(cfg, gen, "cuda") for _ in range(cfg.steps)]
+    out = torch.empty((cfg.N, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
+    scale = 1.0 / math.sqrt(cfg.dk)
+    stream = torch.cuda.current_stream()
+
+    def run_all():
+        for x in steps_in:
+            kda.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, scale, out=out)
+
+    for x in steps_in[:3]:
+        kda.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], S, scale, out=out)
+    torch.cuda.synchronize()
+    kda.profiler_read(reset=True)
+    kda.profiler_enable(True)
+    barrier(ws)
+    torch.cuda.synchronize()
+    ms = time_region(run_all, 1, stream)
+    barrier(ws)
+    kda.profiler_enable(False)
+    stats = kda.profiler_read(reset=True)
+    ms = max_over_ranks(ms, ws)
+    per_head = 2 * cfg.dk * cfg.dv * 4 + 2 * cfg.dk * 2 + cfg.dv * 2 + cfg.dk * 4 + 4 + cfg.dv * 2
+    bytes_step = per_head * cfg.N * cfg.H
+    launches, timed, kms = stats["decode_step"]
+    gbs = bytes_step / (kms / max(1, timed) / 1e3) / 1e9
+    return {
+        "workload": cfg.name, "steps_chained": cfg.steps, "ms_per_step": ms / cfg.steps,
+        "tokens_per_s": cfg.N * cfg.steps * ws / (ms / 1e3),
+        "state_GBps": bytes_step * cfg.steps * ws / (ms / 1e3) / 1e9,
+        "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": gbs,
+                     "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "traffic": None, "algorithmic_bytes_per_launch": bytes_step,
+                     "ms_per_launch": kms / max(1, timed)},
+        "gpu_launches": launches,
+    }
+
+
+def run_e2e(args, ws, kda, inp, bufs, steps):
+    """Same metric through the public API with host (pinned) buffers: every
+    step copies its inputs host->device and its output device->host."""
+    cfg = W.BATCHED
+    names = ("q", "k", "v", "log_alpha", "beta")
+    host = {n: inp[n].to("cpu").pin_memory() for n in names}
+    dev = {n: torch.empty_like(inp[n]) for n in names}
+    out, hT = bufs
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    stream = torch.cuda.current_stream()
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        kda.chunk_fwd(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], inp["scale"],
+                      out=out, hT=hT, impl=args.prefill_impl)
+        out_h.copy_(out, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = time_region(step, steps, stream)
+    barrier(ws)
+    ms = max_over_ranks(ms, ws)
+    h2d = sum(host[n].numel() * host[n].element_size() for n in names)
+    d2h = out_h.numel() * out_h.element_size()
+    return {"value": cfg.B * cfg.T * steps * ws / (ms / 1e3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--prefill-impl", choices=["auto", "simt", "tensorcore"], default="auto")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+
+    ws, rank, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            run_reference(args, ws, rank)
+            return
+        if not torch.cuda.is_available():
+            raise SystemExit("bench.py needs a CUDA device for the kda arm")
+        from gated_delta_rule_75_b200 import build
+        if rank == 0:
+            build.build()
+        barrier(ws)
+        import gated_delta_rule_75_b200 as kda
+        peaks = load_peaks()
+        res, inp, step, bufs = run_prefill(args, ws, rank, kda, peaks)
+        if not args.no_e2e:
+            res["e2e"] = run_e2e(args, ws, kda, inp, bufs, steps=min(args.steps, 3))
+        del inp
+        torch.cuda.empty_cache()
+        if not args.no_decode:
+            res["decode"] = run_decode(args, ws, rank, kda, peaks)
+            res["gpu_launches"] += 0   # decode launches are reported inside "decode"
+        if rank == 0 and not args.no_cpu:
+            cfg = W.BATCHED
+            heads = 8
+            hinp = host_sample_inputs(cfg, heads)
+            dt, ht, thr = oracle_sample(hinp, cfg, heads)
+            res["cpu_baseline"] = {"value": ht / dt / cfg.H, "unit": "tokens/s", "cores": thr,
+                                   "kind": "oracle",
+                                   "sample": f"batch entry 0, heads 0..{heads - 1}, all {cfg.T} "
+                                             f"tokens ({ht} head-tokens, {dt:.1f} s); tokens/s = "
+                                             f"head-tokens/s / {cfg.H}"}
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if ws > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,184 @@
+"""Python binding of libkda.so, the B200 (sm_100a) Kimi Delta Attention library.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in ``include/kda.h``.  Torch supplies device
+memory and the current stream.  There is no CPU fallback: if the shared
+library is missing or fails to load, every call raises.
+
+    out, hT = chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None)
+    out     = recurrent_step(q, k, v, log_alpha, beta, state, scale)   # state in place
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = ["chunk_fwd", "recurrent_step", "KDAError", "library_path", "version",
+           "profiler_enable", "profiler_read",
+           "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
+           "KDA_ERR_NO_MEMORY", "KDA_ERR_TIMEOUT"]
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_NO_MEMORY, \
+    KDA_ERR_TIMEOUT = range(6)
+_IO = {torch.float32: 0, torch.bfloat16: 1}
+_IMPL = {"auto": 0, "simt": 1, "tensorcore": 2}
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
+
+_lib = None
+
+
+class _KernelStat(ctypes.Structure):
+    _fields_ = [("name", ctypes.c_char_p), ("launches", ctypes.c_int64),
+                ("timed_launches", ctypes.c_int64), ("total_ms", ctypes.c_double)]
+
+
+def _load():
+    """Load libkda.so (once).  Raises if it is missing: there is no fallback."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(library_path):
+        raise ImportError(f"{library_path} is not built; run "
+                          "`python -m gated_delta_rule_75_b200.build`")
+    lib = ctypes.CDLL(library_path)
+    vp, i64 = ctypes.c_void_p, ctypes.c_int64
+    lib.kda_chunk_fwd_ex.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                     ctypes.c_float, ctypes.c_int, ctypes.c_int, vp]
+    lib.kda_chunk_fwd_ex.restype = ctypes.c_int
+    lib.kda_chunk_fwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64,
+                                  ctypes.c_float, ctypes.c_int, vp]
+    lib.kda_chunk_fwd.restype = ctypes.c_int
+    lib.kda_recurrent_step.argtypes = [vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                       ctypes.c_float, ctypes.c_int, vp]
+    lib.kda_recurrent_step.restype = ctypes.c_int
+    lib.kda_status_string.argtypes = [ctypes.c_int]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_version.argtypes = []
+    lib.kda_version.restype = ctypes.c_int
+    lib.kda_profiler_enable.argtypes = [ctypes.c_int]
+    lib.kda_profiler_enable.restype = None
+    lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
+    lib.kda_profiler_read.restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_load().kda_status_string(status).decode()} (status {status})")
+
+
+def version() -> int:
+    return int(_load().kda_version())
+
+
+def profiler_enable(on: bool = True) -> None:
+    """Record CUDA events on the launching stream around each library kernel."""
+    _load().kda_profiler_enable(1 if on else 0)
+
+
+def profiler_read(reset: bool = True) -> dict:
+    """{kernel name: (launches, timed launches, total event ms)}; waits for the
+    recorded events.  Launches are counted whether or not timing is on."""
+    lib = _load()
+    arr = (_KernelStat * 32)()
+    n = lib.kda_profiler_read(arr, 32, 1 if reset else 0)
+    if n < 0:
+        raise RuntimeError("kda_profiler_read: an event could not be read")
+    return {arr[i].name.decode(): (int(arr[i].launches), int(arr[i].timed_launches),
+                                   float(arr[i].total_ms)) for i in range(n)}
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, dtype, shape, device):
+    if t.dtype != dtype:
+        raise TypeError(f"{name}: dtype {t.dtype}, expected {dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name}: shape {tuple(t.shape)}, expected {tuple(shape)}")
+    if t.device != device:
+        raise ValueError(f"{name}: on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name}: must be contiguous")
+
+
+def _stream(device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None, out=None,
+              hT=None, output_final_state=True, impl="auto"):
+    """Chunkwise KDA prefill (C ABI ``kda_chunk_fwd_ex``).
+
+    q, k [B,T,H,dk] and v [B,T,H,dv] in fp32 or bf16; log_alpha [B,T,H,dk] and
+    beta [B,T,H] fp32; h0 [N,H,dk,dv] fp32 or None.  With ``cu_seqlens`` (int32,
+    N+1 entries, on the device) B must be 1 and N sequences are packed along T.
+    Returns (out [B,T,H,dv] in the I/O dtype, hT [N,H,dk,dv] fp32 or None).
+    """
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    io = q.dtype
+    if io not in _IO:
+        raise TypeError(f"unsupported I/O dtype {io}")
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv))):
+        _check(t, name, io, shp, dev)
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H, dk), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    if cu_seqlens is not None:
+        if B != 1:
+            raise ValueError("cu_seqlens needs a leading axis of 1")
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be a 1-D int32 tensor on the same device")
+        N = cu_seqlens.numel() - 1
+        n_arg, T_arg = N, T
+    else:
+        N = B
+        n_arg, T_arg = B, T
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=io, device=dev)
+    else:
+        _check(out, "out", io, (B, T, H, dv), dev)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    elif hT is not None:
+        _check(hT, "hT", torch.float32, (N, H, dk, dv), dev)
+    st = _load().kda_chunk_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0),
+                               _ptr(out), _ptr(hT), _ptr(cu_seqlens), n_arg, T_arg, H, dk, dv,
+                               float(scale), _IO[io], _IMPL[impl], _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd")
+    return out, hT
+
+
+def recurrent_step(q, k, v, log_alpha, beta, state, scale, out=None):
+    """One decode token per sequence (C ABI ``kda_recurrent_step``); ``state``
+    [N,H,dk,dv] fp32 is updated in place.  Returns out [N,H,dv]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    io = q.dtype
+    if io not in _IO:
+        raise TypeError(f"unsupported I/O dtype {io}")
+    _check(q, "q", io, (N, H, dk), dev)
+    _check(k, "k", io, (N, H, dk), dev)
+    _check(v, "v", io, (N, H, dv), dev)
+    _check(log_alpha, "log_alpha", torch.float32, (N, H, dk), dev)
+    _check(beta, "beta", torch.float32, (N, H), dev)
+    _check(state, "state", torch.float32, (N, H, dk, dv), dev)
+    if out is None:
+        out = torch.empty((N, H, dv), dtype=io, device=dev)
+    else:
+        _check(out, "out", io, (N, H, dv), dev)
+    st = _load().kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                 _ptr(state), _ptr(out), N, H, dk, dv, float(scale), _IO[io],
+                                 _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_recurrent_step")
+    return out

@@ -1,0 +1,217 @@
+// C ABI of the KDA library: argument checks, workspace, dispatch.
+#include <cuda_runtime.h>
+
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+
+#include "kda.h"
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+static bool debug_mode()
+{
+    static const bool on = [] {
+        const char* s = std::getenv("KDA_DEBUG");
+        return s != nullptr && s[0] == '1';
+    }();
+    return on;
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+static bool head_ok(int64_t d) { return d == 64 || d == 128; }
+
+// Library-owned, per-device CUDA memory pool for stream-ordered workspace.
+// Memory freed with cudaFreeAsync stays cached in the pool (release threshold
+// set to the maximum), so repeated calls do not go back to the driver.
+static cudaMemPool_t workspace_pool(int dev)
+{
+    static std::mutex mu;
+    static cudaMemPool_t pools[64] = {};
+    if (dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (pools[dev] == nullptr) {
+        cudaMemPoolProps props;
+        std::memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t p = nullptr;
+        if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return nullptr;
+        uint64_t thr = ~0ull;
+        cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &thr);
+        pools[dev] = p;
+    }
+    return pools[dev];
+}
+
+// Workspace budget per call (bytes); heads are processed in groups that fit.
+static int64_t workspace_budget()
+{
+    static const int64_t b = [] {
+        const char* s = std::getenv("KDA_WORKSPACE_MB");
+        int64_t mb = s ? std::atoll(s) : 4096;
+        if (mb < 64) mb = 64;
+        return mb << 20;
+    }();
+    return b;
+}
+
+static kda_status_t from_cuda(cudaError_t e)
+{
+    if (e == cudaSuccess) return KDA_OK;
+    if (e == cudaErrorMemoryAllocation) return KDA_ERR_NO_MEMORY;
+    return KDA_ERR_CUDA;
+}
+
+// Stream-ordered allocation that is always released on scope exit.
+struct StreamBuffer {
+    void* ptr = nullptr;
+    cudaStream_t st = nullptr;
+    cudaError_t alloc(size_t bytes, cudaStream_t s) {
+        st = s;
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e) return e;
+        cudaMemPool_t pool = workspace_pool(dev);
+        if (!pool) return cudaErrorMemoryAllocation;
+        return cudaMallocFromPoolAsync(&ptr, bytes, pool, s);
+    }
+    ~StreamBuffer() {
+        if (ptr) cudaFreeAsync(ptr, st);
+    }
+};
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+const char* kda_status_string(kda_status_t s)
+{
+    switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARG: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+    case KDA_ERR_CUDA: return "CUDA error";
+    case KDA_ERR_NO_MEMORY: return "workspace allocation failed";
+    case KDA_ERR_TIMEOUT: return "device-side wait timed out";
+    }
+    return "unknown status";
+}
+
+int kda_version(void) { return 100; }
+
+kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, float* state,
+                                void* out, int64_t N, int64_t H, int64_t dk, int64_t dv,
+                                float scale, kda_io_dtype_t io_dtype, cudaStream_t stream)
+{
+    if (N < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
+    if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (N == 0 || H == 0) return KDA_OK;
+    const void* ptrs[] = {q, k, v, log_alpha, beta, state, out};
+    for (const void* p : ptrs)
+        if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (out == q || out == k || out == v || out == state) return KDA_ERR_INVALID_ARG;
+    cudaError_t e = launch_decode(io_dtype, (int)dk, (int)dv, q, k, v, log_alpha, beta, state,
+                                  out, N * H, scale, stream);
+    if (e == cudaSuccess && debug_mode()) e = cudaStreamSynchronize(stream);
+    return from_cuda(e);
+}
+
+kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta, const float* h0,
+                              void* out, float* hT, const int32_t* cu_seqlens, int64_t B,
+                              int64_t T, int64_t H, int64_t dk, int64_t dv, float scale,
+                              kda_io_dtype_t io_dtype, kda_prefill_impl_t impl,
+                              cudaStream_t stream)
+{
+    if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
+    if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (impl != KDA_PREFILL_AUTO && impl != KDA_PREFILL_SIMT && impl != KDA_PREFILL_TENSORCORE)
+        return KDA_ERR_INVALID_ARG;
+    if (impl == KDA_PREFILL_TENSORCORE)
+        return KDA_ERR_UNSUPPORTED;   // tensor-core kernels are added separately
+    if (cu_seqlens != nullptr && B < 1) return KDA_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return KDA_OK;
+    const int64_t T_total = cu_seqlens ? T : B * T;
+    if (T_total > 0) {
+        const void* ptrs[] = {q, k, v, log_alpha, beta, out};
+        for (const void* p : ptrs)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        if (out == q || out == k || out == v || out == log_alpha || out == beta)
+            return KDA_ERR_INVALID_ARG;
+    }
+    if ((h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0))
+        return KDA_ERR_INVALID_ARG;
+    // every index must fit the kernels' 64-bit arithmetic and 32-bit grid limits
+    if (T_total > (int64_t(1) << 40) || H > 65535) return KDA_ERR_UNSUPPORTED;
+
+    PrefillArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
+    a.out = out; a.hT = hT; a.H = H; a.dk = (int)dk; a.dv = (int)dv; a.scale = scale;
+    a.io = io_dtype;
+    SeqInfo& si = a.si;
+    si.cu = cu_seqlens;
+    si.chunk_off = nullptr;
+    si.N = B;
+    si.T_seq = cu_seqlens ? 0 : T;
+    si.T_total = T_total;
+    si.nct = cu_seqlens ? 0 : (T + kChunk - 1) / kChunk;
+    si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
+
+    // workspace: [256 B header | chunk offsets | per-(chunk, head) blocks]
+    const int64_t blk_bytes = simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
+    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 255) / 256 * 256 : 0;
+    const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1);
+    int64_t Hg = (workspace_budget() - 256 - off_bytes) / per_head;
+    if (Hg < 1) Hg = 1;
+    if (Hg > H) Hg = H;
+    const int64_t ws_bytes = 256 + off_bytes + Hg * per_head;
+
+    StreamBuffer buf;
+    cudaError_t e = buf.alloc((size_t)ws_bytes, stream);
+    if (e) return from_cuda(e);
+    char* base = static_cast<char*>(buf.ptr);
+    int* err_flag = reinterpret_cast<int*>(base);
+    if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
+    if (cu_seqlens) {
+        int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 256);
+        if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, chunk_off, err_flag, stream)))
+            return from_cuda(e);
+        si.chunk_off = chunk_off;
+    }
+    float* ws = reinterpret_cast<float*>(base + 256 + off_bytes);
+    e = run_prefill_simt(a, ws, Hg, stream);
+    if (e) return from_cuda(e);
+    if (debug_mode()) {
+        int flag = 0;
+        if ((e = cudaMemcpyAsync(&flag, err_flag, sizeof(int), cudaMemcpyDeviceToHost, stream)))
+            return from_cuda(e);
+        if ((e = cudaStreamSynchronize(stream))) return from_cuda(e);
+        if (flag) return KDA_ERR_INVALID_ARG;
+    }
+    return KDA_OK;
+}
+
+kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* h0, void* out, float* hT,
+                           const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                           int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
+                           cudaStream_t stream)
+{
+    return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, h0, out, hT, cu_seqlens, B, T, H, dk, dv,
+                            scale, io_dtype, KDA_PREFILL_AUTO, stream);
+}
+
+}  // extern "C"

@@ -1,0 +1,117 @@
+// Internal declarations shared by the KDA library's translation units.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// Where the tokens of each sequence live, and how chunks are numbered.
+// Chunks are numbered sequence after sequence: sequence n owns global chunks
+// [chunk_start(n), chunk_start(n+1)).  Without cu_seqlens every sequence has
+// T_seq tokens and nct = ceil(T_seq / 64) chunks; with cu_seqlens the
+// per-sequence chunk offsets are computed on the device (chunk_off, N+1
+// entries) from the clamped offsets.
+struct SeqInfo {
+    const int32_t* cu;          // device, N+1 entries, or nullptr
+    const int64_t* chunk_off;   // device, N+1 entries (only with cu)
+    int64_t N;                  // number of sequences
+    int64_t T_seq;              // tokens per sequence (fixed-length case)
+    int64_t T_total;            // packed token count (B*T, or T with cu)
+    int64_t nct;                // chunks per sequence (fixed-length case)
+    int64_t chunks_upper;       // upper bound on the number of chunks (grid size)
+
+#ifdef __CUDACC__
+    __device__ __forceinline__ int64_t chunk_start(int64_t n) const {
+        return cu ? chunk_off[n] : n * nct;
+    }
+    // Map a global chunk index to (sequence, first token, length); false when
+    // the index is past the last chunk.
+    __device__ __forceinline__ bool locate(int64_t gc, int64_t& n, int64_t& t0,
+                                           int64_t& len) const {
+        if (cu == nullptr) {
+            n = gc / nct;
+            if (n >= N) return false;
+            const int64_t c = gc - n * nct;
+            const int64_t bos = n * T_seq;
+            t0 = bos + c * 64;
+            len = bos + T_seq - t0;
+            len = len > 64 ? 64 : len;
+            return len > 0;
+        }
+        if (gc >= chunk_off[N]) return false;
+        int64_t lo = 0, hi = N;                  // chunk_off[lo] <= gc < chunk_off[hi]
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if (chunk_off[mid] <= gc) lo = mid; else hi = mid;
+        }
+        n = lo;
+        int64_t a = cu[n], b = cu[n + 1];
+        a = a < 0 ? 0 : (a > T_total ? T_total : a);
+        b = b < a ? a : (b > T_total ? T_total : b);
+        t0 = a + (gc - chunk_off[n]) * 64;
+        len = b - t0;
+        len = len > 64 ? 64 : len;
+        return len > 0;
+    }
+#endif
+};
+
+struct PrefillArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    const float* h0;
+    void* out;
+    float* hT;
+    SeqInfo si;
+    int64_t H;
+    int dk, dv;
+    float scale;
+    kda_io_dtype_t io;
+};
+
+// Kernel identities for launch counting and timing (kda_profiler.cu).
+enum KernelId {
+    K_CHUNK_OFFSETS = 0,
+    K_PREP_SIMT,
+    K_STATE_SIMT,
+    K_DECODE,
+    K_PREP_TC,
+    K_STATE_TC,
+    K_KERNEL_COUNT
+};
+
+// Opened around every kernel launch: counts it and, while the profiler is
+// enabled, records start/stop CUDA events on the launching stream.
+class LaunchScope {
+public:
+    LaunchScope(cudaStream_t st, KernelId id);
+    ~LaunchScope();
+    LaunchScope(const LaunchScope&) = delete;
+    LaunchScope& operator=(const LaunchScope&) = delete;
+
+private:
+    cudaStream_t st_;
+    KernelId id_;
+    void* start_ = nullptr;
+    void* stop_ = nullptr;
+};
+
+// kda_decode.cu
+cudaError_t launch_decode(kda_io_dtype_t io, int dk, int dv, const void* q, const void* k,
+                          const void* v, const float* g, const float* b, float* state, void* out,
+                          int64_t NH, float scale, cudaStream_t st);
+
+// kda_chunk_simt.cu
+int64_t simt_ws_floats_per_chunk(int dk, int dv);
+cudaError_t run_prefill_simt(const PrefillArgs& a, float* ws, int64_t Hg, cudaStream_t st);
+
+// kda_seqinfo.cu
+cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total,
+                                 int64_t* chunk_off, int* err_flag, cudaStream_t st);
+
+}  // namespace kda

@@ -1,0 +1,56 @@
+// Per-sequence chunk offsets for packed variable-length batches.
+//
+// One CTA scans the N sequence lengths (clamped into [0, T]) and writes
+// chunk_off[n] = sum_{m<n} ceil(L_m / 64), n = 0..N.  It also checks the
+// offsets (cu[0] == 0, non-decreasing, cu[N] == T) and sets bit 0 of
+// *err_flag when they are malformed; the kernels that follow only ever use
+// clamped offsets, so a malformed array cannot cause an out-of-bounds access.
+#include <cub/block/block_scan.cuh>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+
+namespace kda {
+
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads)
+chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
+                     int64_t* __restrict__ chunk_off, int* __restrict__ err)
+{
+    using Scan = cub::BlockScan<int64_t, kScanThreads>;
+    __shared__ typename Scan::TempStorage tmp;
+    __shared__ int64_t carry;
+    if (threadIdx.x == 0) {
+        carry = 0;
+        if (cu[0] != 0 || cu[N] != T_total) atomicOr(err, 1);
+    }
+    __syncthreads();
+    for (int64_t base = 0; base < N; base += kScanThreads) {
+        const int64_t n = base + threadIdx.x;
+        int64_t nc = 0;
+        if (n < N) {
+            int64_t bos, eos;
+            seq_range(cu, n, 0, T_total, bos, eos);
+            nc = (eos - bos + kChunk - 1) / kChunk;
+            if (cu[n + 1] < cu[n]) atomicOr(err, 1);
+        }
+        int64_t excl, total;
+        Scan(tmp).ExclusiveSum(nc, excl, total);
+        if (n < N) chunk_off[n] = carry + excl;
+        __syncthreads();
+        if (threadIdx.x == 0) carry += total;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) chunk_off[N] = carry;
+}
+
+cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total,
+                                 int64_t* chunk_off, int* err_flag, cudaStream_t st)
+{
+    LaunchScope scope(st, K_CHUNK_OFFSETS);
+    chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, chunk_off, err_flag);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

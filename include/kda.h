@@ -1,0 +1,170 @@
+/*
+ * kda.h -- C ABI of the B200 (sm_100a) Kimi Delta Attention library (libkda.so).
+ *
+ * The operation ("Kimi Delta Attention: la atencion lineal detras de Kimi K2 y
+ * Qwen3", section "Como funciona Kimi Delta Attention paso a paso", the
+ * per-token step and the flowchart after it): for every sequence and head, with
+ * a state S of shape dk x dv, and for every token t in order,
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *     o_t = scale * S_t^T q_t,          alpha_t = exp(log_alpha_t)  (per key channel)
+ *
+ * i.e. decay the state per key channel, predict vhat = S~^T k_t, write the
+ * beta-scaled error along k_t, then read with the query.  The page keeps the
+ * state as (d_v, d_k) and reads S q; this library keeps S as [dk][dv] (dv
+ * innermost) and reads S^T q -- the same arithmetic.
+ *
+ * Conventions shared by every entry point
+ *  - All tensor pointers are DEVICE pointers, contiguous, last dimension
+ *    innermost, 16-byte aligned.  The caller owns all of them.
+ *  - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument
+ *    errors are detected on the host and returned before anything is launched;
+ *    a failed launch returns KDA_ERR_CUDA.  No entry point synchronises the
+ *    device unless KDA_DEBUG=1 is set in the environment, in which case the
+ *    call synchronises `stream` at the end and also reports device-side input
+ *    errors (malformed cu_seqlens) as KDA_ERR_INVALID_ARG.
+ *  - q and k are expected to be L2-normalised per (token, head) by the caller
+ *    (the delta rule is only stable for normalised keys, as the same page notes
+ *    in its warning on key normalisation); the kernels do not renormalise.
+ *  - `scale` multiplies q once, at the read (configurations use 1/sqrt(dk)).
+ *  - log_alpha is the natural log of the per-channel decay, finite and <= 0.
+ *    The tensor-core prefill path additionally assumes that, within each
+ *    64-token chunk, no key channel decays by more than e^-80 over 16
+ *    consecutive tokens (its exponential factors are referenced to 16-token
+ *    sub-chunk starts and would leave the fp32 range beyond that); the SIMT
+ *    paths have no such limit.
+ *  - Supported head sizes: dk, dv in {64, 128}.  Anything else returns
+ *    KDA_ERR_UNSUPPORTED.
+ */
+#ifndef KDA_H_
+#define KDA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad shape, bad cu_seqlens (debug) */
+    KDA_ERR_UNSUPPORTED = 2,   /* head size or dtype not implemented */
+    KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
+    KDA_ERR_NO_MEMORY = 4,     /* workspace could not be allocated */
+    KDA_ERR_TIMEOUT = 5        /* reserved: a bounded device-side wait gave up */
+} kda_status_t;
+
+typedef enum {
+    KDA_IO_F32 = 0,            /* q, k, v, out are fp32 */
+    KDA_IO_BF16 = 1            /* q, k, v, out are bf16 (gates, beta and states stay fp32) */
+} kda_io_dtype_t;
+
+typedef enum {
+    KDA_PREFILL_AUTO = 0,      /* tensor cores for bf16 with dk = dv = 128, SIMT otherwise */
+    KDA_PREFILL_SIMT = 1,      /* fp32 SIMT chunk kernels (any supported shape / dtype) */
+    KDA_PREFILL_TENSORCORE = 2 /* tcgen05 chunk kernels; bf16, dk = dv = 128 only */
+} kda_prefill_impl_t;
+
+/*
+ * kda_chunk_fwd -- chunkwise-parallel prefill (64-token chunks).
+ *
+ * The chunkwise form is the exact reformulation of the token recurrence that
+ * "Kimi Linear acaba de superar a la atencion completa en sus propios
+ * terminos" (sections on the chunk training algorithm and the
+ * diagonal-plus-low-rank transition) says the method uses; it returns the
+ * token recurrence's result up to rounding.  Per chunk: cumulative log-decay,
+ * intra-chunk WY/UT transform (T = (I + A)^{-1}), state propagation across
+ * chunks with the state kept in fp32, and the output.
+ *
+ *  q, k        [B, T, H, dk]  io_dtype
+ *  v           [B, T, H, dv]  io_dtype
+ *  log_alpha   [B, T, H, dk]  fp32
+ *  beta        [B, T, H]      fp32
+ *  h0          [N, H, dk, dv] fp32 initial states, or NULL for zeros
+ *  out         [B, T, H, dv]  io_dtype, written; must not alias any input
+ *  hT          [N, H, dk, dv] fp32 final states, or NULL (not written); may alias h0
+ *  cu_seqlens  NULL, or a DEVICE array of B+1 int32 offsets.  Then the B
+ *              sequences are packed along T (q, k, v, log_alpha, beta, out have
+ *              a leading axis of 1), cu_seqlens[0] = 0, non-decreasing,
+ *              cu_seqlens[B] = T, and N = B.  Empty sequences are allowed
+ *              (their hT equals h0).  Offsets are clamped into [0, T] on the
+ *              device, so a malformed array never causes an out-of-bounds
+ *              access (its results are then unspecified; KDA_DEBUG=1 reports it).
+ *              With NULL, every one of the N = B sequences has length T.
+ * Memory: the call allocates stream-ordered workspace from a library-owned
+ * CUDA memory pool (bounded, reused across calls); KDA_ERR_NO_MEMORY if that
+ * fails.  T = 0 is a no-op apart from hT = h0.
+ */
+KDA_API kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v,
+                           const float* log_alpha, const float* beta,
+                           const float* h0, void* out, float* hT,
+                           const int32_t* cu_seqlens,
+                           int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                           float scale, kda_io_dtype_t io_dtype, cudaStream_t stream);
+
+/* Same as kda_chunk_fwd with an explicit choice of implementation. */
+KDA_API kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
+                              const float* log_alpha, const float* beta,
+                              const float* h0, void* out, float* hT,
+                              const int32_t* cu_seqlens,
+                              int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                              float scale, kda_io_dtype_t io_dtype,
+                              kda_prefill_impl_t impl, cudaStream_t stream);
+
+/*
+ * kda_recurrent_step -- one decode token per sequence, the per-token step
+ * itself, with the state updated in place (HBM-bound: each (sequence, head)
+ * state is read once and written once).
+ *
+ *  q, k        [N, H, dk]  io_dtype
+ *  v           [N, H, dv]  io_dtype
+ *  log_alpha   [N, H, dk]  fp32
+ *  beta        [N, H]      fp32
+ *  state       [N, H, dk, dv] fp32, read and overwritten
+ *  out         [N, H, dv]  io_dtype
+ * No workspace is used.  N = 0 is a no-op.
+ */
+KDA_API kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta,
+                                float* state, void* out,
+                                int64_t N, int64_t H, int64_t dk, int64_t dv,
+                                float scale, kda_io_dtype_t io_dtype, cudaStream_t stream);
+
+/*
+ * Launch accounting of the library's own kernels (no counterpart on the
+ * pages; it exists so throughput can be attributed per kernel).  Every
+ * launch is counted.  While enabled, each launch is also bracketed by CUDA
+ * events recorded on its own stream.  kda_profiler_read() waits for the
+ * recorded events, fills up to max_entries stats (one per kernel, in a fixed
+ * order), optionally resets the counters, and returns the number of entries,
+ * or -1 if an event could not be read.
+ */
+typedef struct {
+    const char* name;          /* static string */
+    int64_t launches;          /* launches since the last reset */
+    int64_t timed_launches;    /* launches recorded while the profiler was on */
+    double total_ms;           /* summed event time of the timed launches */
+} kda_kernel_stat_t;
+
+KDA_API void kda_profiler_enable(int on);
+KDA_API int kda_profiler_read(kda_kernel_stat_t* out, int max_entries, int reset);
+
+/* Static, NUL-terminated description of a status code. */
+KDA_API const char* kda_status_string(kda_status_t status);
+
+/* Library version as major*10000 + minor*100 + patch. */
+KDA_API int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H_ */

@@ -1,0 +1,157 @@
+"""GPU parity of the chunkwise prefill (kda_chunk_fwd through the C ABI)
+against the fp64 oracle, element by element, on seeded inputs: ragged tails,
+several chunks, every supported head size, packed variable-length batches,
+continuation across calls, the empty case, and the full-size workloads
+(all pairs for the 16-head prefill; sampled pairs for the larger ones)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import workloads as W
+from kda_testutil import TOL, host, oracle_pairs, oracle_prefill, rel
+
+pytestmark = pytest.mark.gpu
+
+IMPLS = ["simt"]
+
+
+@pytest.fixture(scope="module")
+def kda(cuda_ok):
+    from gated_delta_rule_75_b200 import build
+    build.build()
+    import gated_delta_rule_75_b200 as kda
+    return kda
+
+
+def run(kda, inp, impl="auto"):
+    out, hT = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                            inp["scale"], h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], impl=impl)
+    torch.cuda.synchronize()
+    return out, hT
+
+
+def check_full(kda, cfg, impl="auto"):
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = run(kda, inp, impl)
+    ro, rh = oracle_prefill(inp)
+    eo, eh = rel(out, ro), rel(hT, rh)
+    tol = TOL[cfg.io_dtype]
+    assert eo <= tol and eh <= tol, (cfg.name, impl, eo, eh)
+    return eo, eh
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_tiny_fp32_workload(kda, impl):
+    """B=1, H=2, T=256, dk=dv=64, fp32 I/O, h0 = 0, seed 0."""
+    check_full(kda, W.TINY, impl)
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_head_sizes_ragged_tail(kda, dk, dv, io):
+    cfg = W.small_prefill(B=2, T=150, H=3, dk=dk, dv=dv, io_dtype=io, seed=dk + dv, h0_std=0.05)
+    check_full(kda, cfg, "simt")
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("impl", IMPLS)
+def test_packed_variable_lengths(kda, io, impl):
+    lens = [1, 63, 64, 65, 0, 130, 200, 7]
+    cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype=io, seed=7, h0_std=0.05, lengths=lens)
+    check_full(kda, cfg, impl)
+
+
+@pytest.mark.parametrize("impl", IMPLS)
+def test_packed_equals_separate_calls(kda, impl):
+    lens = [70, 1, 129]
+    cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype="f32", seed=8, h0_std=0.05, lengths=lens)
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = run(kda, inp, impl)
+    cu = [0] + list(np.cumsum(lens))
+    for n in range(len(lens)):
+        sub = {k: (v[:, cu[n]:cu[n + 1]] if k in ("q", "k", "v", "log_alpha", "beta") else v)
+               for k, v in inp.items()}
+        sub = {k: (v.contiguous() if isinstance(v, torch.Tensor) else v) for k, v in sub.items()}
+        sub["h0"] = inp["h0"][n:n + 1].contiguous()
+        sub["cu_seqlens"] = None
+        o1, h1 = run(kda, sub, impl)
+        assert rel(o1, host(out[:, cu[n]:cu[n + 1]]).double().numpy()) <= 1e-6
+        assert rel(h1, host(hT[n:n + 1]).double().numpy()) <= 1e-6
+
+
+@pytest.mark.parametrize("t1", [64, 100])
+@pytest.mark.parametrize("impl", IMPLS)
+def test_continuation_across_calls(kda, t1, impl):
+    """[0, t1) then [t1, T) with h0 = hT of the first call equals one pass
+    (on and off a chunk boundary): the state layout survives the hand-over."""
+    cfg = W.small_prefill(B=1, T=256, H=2, dk=128, dv=128, io_dtype="f32", seed=9, h0_std=0.05)
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = run(kda, inp, impl)
+    a = {k: (v[:, :t1].contiguous() if k in ("q", "k", "v", "log_alpha", "beta") else v)
+         for k, v in inp.items()}
+    o1, h1 = run(kda, a, impl)
+    b = {k: (v[:, t1:].contiguous() if k in ("q", "k", "v", "log_alpha", "beta") else v)
+         for k, v in inp.items()}
+    b["h0"] = h1
+    o2, h2 = run(kda, b, impl)
+    ro, rh = oracle_prefill(inp)
+    assert rel(torch.cat([o1, o2], dim=1), ro) <= TOL["f32"]
+    assert rel(h2, rh) <= TOL["f32"]
+
+
+def test_empty_sequence_passes_state_through(kda):
+    cfg = W.small_prefill(B=3, T=0, H=2, dk=64, dv=64, io_dtype="f32", seed=1, h0_std=0.1)
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = run(kda, inp)
+    assert out.numel() == 0
+    torch.testing.assert_close(hT, inp["h0"], rtol=0, atol=0)
+
+
+def test_zero_initial_state_when_h0_absent(kda):
+    cfg = W.small_prefill(B=1, T=80, H=1, dk=64, dv=64, io_dtype="f32", seed=2)
+    inp = W.make_prefill(cfg, "cuda")
+    o1, h1 = run(kda, inp)
+    inp["h0"] = torch.zeros(1, 1, 64, 64, device="cuda")
+    o2, h2 = run(kda, inp)
+    torch.testing.assert_close(o1, o2, rtol=0, atol=0)
+    torch.testing.assert_close(h1, h2, rtol=0, atol=0)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("impl", ["auto"])
+def test_single_head_group_prefill_full(kda, impl):
+    """B=1, H=16, T=4096, d=128, bf16, h0 ~ N(0, 0.02^2): every output and state."""
+    check_full(kda, W.SINGLE, impl)
+
+
+@pytest.mark.slow
+def test_batched_prefill_sampled_pairs(kda):
+    """B=8, H=32, T=8192, bf16 (the benchmark workload, same launch): four
+    (batch, head) pairs compared in full against the oracle."""
+    cfg = W.BATCHED
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = run(kda, inp)
+    rng = np.random.default_rng(cfg.seed)
+    pairs = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(4)]
+    res = oracle_pairs(inp, pairs)
+    for (n, h), ((b, t0, t1), ro, rh) in zip(pairs, res):
+        assert rel(out[b, t0:t1, h], ro) <= TOL["bf16"], (n, h)
+        assert rel(hT[n, h], rh) <= TOL["bf16"], (n, h)
+
+
+@pytest.mark.slow
+def test_long_context_varlen_sampled_pairs(kda):
+    """16 packed sequences, 2^20 tokens, H=32, bf16: four (sequence, head)
+    pairs (the longest and the shortest sequence among them) in full."""
+    cfg = W.varlen_config()
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = run(kda, inp)
+    L = np.array(cfg.lengths)
+    rng = np.random.default_rng(cfg.seed)
+    seqs = [int(L.argmax()), int(L.argmin()), int(rng.integers(cfg.N)), int(rng.integers(cfg.N))]
+    pairs = [(n, int(rng.integers(cfg.H))) for n in seqs]
+    res = oracle_pairs(inp, pairs)
+    for (n, h), ((b, t0, t1), ro, rh) in zip(pairs, res):
+        assert rel(out[0, t0:t1, h], ro) <= TOL["bf16"], (n, h)
+        assert rel(hT[n, h], rh) <= TOL["bf16"], (n, h)
