@@ -145,22 +145,22 @@ def max_over_ranks(x, ws):
 # ----------------------------------------------------------------------------
 # oracle timing (CPU baseline / reference arm)
 # ----------------------------------------------------------------------------
-def oracle_sample(inp_host, cfg, heads):
-    """Oracle on batch entry 0 and the first `heads` heads of the workload."""
+def oracle_sample(inp_host, cfg, heads, batch=1):
+    """Oracle on the first `batch` batch entries and `heads` heads of the workload."""
     import oracle
-    sl = lambda x: x[0:1, :, :heads].contiguous()
+    sl = lambda x: x[0:batch, :, :heads].contiguous()
     t = time.perf_counter()
     oracle.fwd(sl(inp_host["q"]), sl(inp_host["k"]), sl(inp_host["v"]), sl(inp_host["log_alpha"]),
                sl(inp_host["beta"]), inp_host["scale"], return_state=True)
     dt = time.perf_counter() - t
-    head_tokens = cfg.T * heads
+    head_tokens = cfg.T * heads * batch
     return dt, head_tokens, oracle.threads()
 
 
-def host_sample_inputs(cfg, heads):
-    """The same seeded workload generated on the host, restricted to batch 0
-    and `heads` heads (the generator is the one the GPU run uses, on CPU)."""
-    small = W.PrefillConfig(cfg.name, 1, cfg.T, heads, cfg.dk, cfg.dv, cfg.io_dtype, cfg.seed,
+def host_sample_inputs(cfg, heads, batch=1):
+    """The same seeded workload generated on the host, restricted to `batch`
+    batch entries and `heads` heads (the generator the GPU run uses, on CPU)."""
+    small = W.PrefillConfig(cfg.name, batch, cfg.T, heads, cfg.dk, cfg.dv, cfg.io_dtype, cfg.seed,
                             cfg.gate_shift, cfg.h0_std)
     return W.make_prefill(small, "cpu")
 
@@ -307,6 +307,8 @@ TC_WS_BYTES_PER_CHUNK = 72 * 1024 + 512
 
 def run_decode(args, ws, rank, kda, peaks):
     cfg = W.DECODE
+    if args.decode_steps != cfg.steps:
+        cfg = W.DecodeConfig(cfg.name, cfg.N, cfg.H, cfg.dk, cfg.dv, args.decode_steps, cfg.seed)
     gen = W.decode_generator(cfg, "cuda")
     S = W.make_decode_state(cfg, gen, "cuda")
     steps_in = [W.make_decode_step(cfg, gen, "cuda") for _ in range(cfg.steps)]
@@ -386,6 +388,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="restrict the run (profiling of one kernel family)")
+    ap.add_argument("--decode-steps", type=int, default=W.DECODE.steps)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 
@@ -402,24 +407,28 @@ def main():
         barrier(ws)
         import gated_delta_rule_75_b200 as kda
         peaks = load_peaks()
+        if args.only == "decode":
+            res = {"decode": run_decode(args, ws, rank, kda, peaks)}
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res, inp, step, bufs = run_prefill(args, ws, rank, kda, peaks)
-        if not args.no_e2e:
+        if not args.no_e2e and args.only == "all":
             res["e2e"] = run_e2e(args, ws, kda, inp, bufs, steps=min(args.steps, 3))
-        del inp
+        del inp, bufs
         torch.cuda.empty_cache()
-        if not args.no_decode:
+        if not args.no_decode and args.only == "all":
             res["decode"] = run_decode(args, ws, rank, kda, peaks)
-            res["gpu_launches"] += 0   # decode launches are reported inside "decode"
-        if rank == 0 and not args.no_cpu:
+        if rank == 0 and not args.no_cpu and args.only == "all":
             cfg = W.BATCHED
-            heads = 8
-            hinp = host_sample_inputs(cfg, heads)
-            dt, ht, thr = oracle_sample(hinp, cfg, heads)
+            heads, batch = cfg.H, 2
+            hinp = host_sample_inputs(cfg, heads, batch)
+            dt, ht, thr = oracle_sample(hinp, cfg, heads, batch)
             res["cpu_baseline"] = {"value": ht / dt / cfg.H, "unit": "tokens/s", "cores": thr,
                                    "kind": "oracle",
-                                   "sample": f"batch entry 0, heads 0..{heads - 1}, all {cfg.T} "
-                                             f"tokens ({ht} head-tokens, {dt:.1f} s); tokens/s = "
-                                             f"head-tokens/s / {cfg.H}"}
+                                   "sample": f"{batch} of the {cfg.B} sequences, all {heads} heads, "
+                                             f"all {cfg.T} tokens ({ht} head-tokens, {dt:.1f} s "
+                                             f"wall); tokens/s = head-tokens/s / {cfg.H}"}
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:

@@ -22,6 +22,7 @@ static bool debug_mode()
 }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 static bool head_ok(int64_t d) { return d == 64 || d == 128; }
 
@@ -117,9 +118,10 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0 || H == 0) return KDA_OK;
-    const void* ptrs[] = {q, k, v, log_alpha, beta, state, out};
+    const void* ptrs[] = {q, k, v, log_alpha, state, out};
     for (const void* p : ptrs)
         if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
     if (out == q || out == k || out == v || out == state) return KDA_ERR_INVALID_ARG;
     cudaError_t e = launch_decode(io_dtype, (int)dk, (int)dv, q, k, v, log_alpha, beta, state,
                                   out, N * H, scale, stream);
@@ -145,9 +147,10 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     if (B == 0 || H == 0) return KDA_OK;
     const int64_t T_total = cu_seqlens ? T : B * T;
     if (T_total > 0) {
-        const void* ptrs[] = {q, k, v, log_alpha, beta, out};
+        const void* ptrs[] = {q, k, v, log_alpha, out};
         for (const void* p : ptrs)
             if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
         if (out == q || out == k || out == v || out == log_alpha || out == beta)
             return KDA_ERR_INVALID_ARG;
     }
@@ -187,7 +190,8 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 256);
-        if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, chunk_off, err_flag, stream)))
+        if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off,
+                                          err_flag, stream)))
             return from_cuda(e);
         si.chunk_off = chunk_off;
     }

@@ -179,7 +179,7 @@ chunk_state_simt_kernel(const float* __restrict__ ws, const float* __restrict__ 
     const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
     int64_t bos, eos;
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
-    const int64_t nchunks = (eos - bos + C - 1) / C;
+    const int64_t nchunks = si.chunk_count(n, eos - bos);
     const int64_t gc0 = si.chunk_start(n);
 
     for (int e = tid; e < DK * TW; e += blockDim.x) {

@@ -26,6 +26,14 @@ struct SeqInfo {
     __device__ __forceinline__ int64_t chunk_start(int64_t n) const {
         return cu ? chunk_off[n] : n * nct;
     }
+    // Chunks of sequence n that have workspace slots: ceil(len/64), capped by
+    // the (capped) device offsets when cu_seqlens is malformed.
+    __device__ __forceinline__ int64_t chunk_count(int64_t n, int64_t len) const {
+        const int64_t c = (len + 63) / 64;
+        if (!cu) return c;
+        const int64_t slots = chunk_off[n + 1] - chunk_off[n];
+        return c < slots ? c : slots;
+    }
     // Map a global chunk index to (sequence, first token, length); false when
     // the index is past the last chunk.
     __device__ __forceinline__ bool locate(int64_t gc, int64_t& n, int64_t& t0,
@@ -111,7 +119,7 @@ int64_t simt_ws_floats_per_chunk(int dk, int dv);
 cudaError_t run_prefill_simt(const PrefillArgs& a, float* ws, int64_t Hg, cudaStream_t st);
 
 // kda_seqinfo.cu
-cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total,
+cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
                                  int64_t* chunk_off, int* err_flag, cudaStream_t st);
 
 }  // namespace kda

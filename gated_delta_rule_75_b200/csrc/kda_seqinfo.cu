@@ -1,10 +1,12 @@
 // Per-sequence chunk offsets for packed variable-length batches.
 //
 // One CTA scans the N sequence lengths (clamped into [0, T]) and writes
-// chunk_off[n] = sum_{m<n} ceil(L_m / 64), n = 0..N.  It also checks the
-// offsets (cu[0] == 0, non-decreasing, cu[N] == T) and sets bit 0 of
-// *err_flag when they are malformed; the kernels that follow only ever use
-// clamped offsets, so a malformed array cannot cause an out-of-bounds access.
+// chunk_off[n] = min(cap, sum_{m<n} ceil(L_m / 64)), n = 0..N, where cap is
+// the number of chunk slots the workspace holds.  For well-formed offsets the
+// sum never reaches past floor(T/64) + N = cap; for malformed ones (checked
+// here: cu[0] == 0, non-decreasing, cu[N] == T; bit 0 of *err_flag is set
+// otherwise) the cap keeps every chunk index the later kernels derive inside
+// the workspace, so a malformed array cannot cause an out-of-bounds access.
 #include <cub/block/block_scan.cuh>
 
 #include "kda_common.cuh"
@@ -15,7 +17,7 @@ namespace kda {
 constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads)
-chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
+chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total, int64_t cap,
                      int64_t* __restrict__ chunk_off, int* __restrict__ err)
 {
     using Scan = cub::BlockScan<int64_t, kScanThreads>;
@@ -37,19 +39,22 @@ chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
         }
         int64_t excl, total;
         Scan(tmp).ExclusiveSum(nc, excl, total);
-        if (n < N) chunk_off[n] = carry + excl;
+        if (n < N) chunk_off[n] = (carry + excl) < cap ? (carry + excl) : cap;
         __syncthreads();
         if (threadIdx.x == 0) carry += total;
         __syncthreads();
     }
-    if (threadIdx.x == 0) chunk_off[N] = carry;
+    if (threadIdx.x == 0) {
+        if (carry > cap) atomicOr(err, 1);
+        chunk_off[N] = carry < cap ? carry : cap;
+    }
 }
 
-cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total,
+cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
                                  int64_t* chunk_off, int* err_flag, cudaStream_t st)
 {
     LaunchScope scope(st, K_CHUNK_OFFSETS);
-    chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, chunk_off, err_flag);
+    chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, cap, chunk_off, err_flag);
     return cudaGetLastError();
 }
 

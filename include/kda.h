@@ -16,7 +16,8 @@
  *
  * Conventions shared by every entry point
  *  - All tensor pointers are DEVICE pointers, contiguous, last dimension
- *    innermost, 16-byte aligned.  The caller owns all of them.
+ *    innermost, 16-byte aligned (beta and cu_seqlens: 4-byte aligned).  The
+ *    caller owns all of them.
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument
  *    errors are detected on the host and returned before anything is launched;
  *    a failed launch returns KDA_ERR_CUDA.  No entry point synchronises the

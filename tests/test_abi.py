@@ -70,6 +70,7 @@ def test_prefill_argument_errors(lib):
     assert _fwd(lib, T=-5) == kda.KDA_ERR_INVALID_ARG
     assert _fwd(lib, q=None) == kda.KDA_ERR_INVALID_ARG
     assert _fwd(lib, b=None) == kda.KDA_ERR_INVALID_ARG
+    assert _fwd(lib, b=FAKE + 66) == kda.KDA_ERR_INVALID_ARG         # beta not 4-byte aligned
     assert _fwd(lib, q=FAKE + 2) == kda.KDA_ERR_INVALID_ARG          # misaligned
     assert _fwd(lib, out=FAKE) == kda.KDA_ERR_INVALID_ARG            # out aliases q
     assert _fwd(lib, h0=FAKE + 8) == kda.KDA_ERR_INVALID_ARG         # misaligned h0
@@ -89,6 +90,7 @@ def test_decode_argument_errors(lib):
     assert _step(lib, s=None) == kda.KDA_ERR_INVALID_ARG
     assert _step(lib, out=FAKE + 80) == kda.KDA_ERR_INVALID_ARG      # out aliases state
     assert _step(lib, v=FAKE + 40) == kda.KDA_ERR_INVALID_ARG        # misaligned
+    assert _step(lib, b=FAKE + 66) == kda.KDA_ERR_INVALID_ARG        # beta not 4-byte aligned
     assert _step(lib, N=0) == kda.KDA_OK
 
 

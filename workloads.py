@@ -124,6 +124,8 @@ def _unit_rows(x: torch.Tensor) -> torch.Tensor:
 def _fill_normal(shape, gen, device, block=1 << 26):
     """N(0,1) fp32 of `shape`, drawn in slabs along the first axis to bound temporaries."""
     out = torch.empty(shape, dtype=torch.float32, device=device)
+    if out.numel() == 0:
+        return out
     flat = out.view(shape[0], -1)
     rows_per = max(1, block // max(1, flat.shape[1]))
     for r in range(0, flat.shape[0], rows_per):
