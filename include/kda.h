@@ -121,6 +121,44 @@ KDA_API kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* 
                               kda_prefill_impl_t impl, cudaStream_t stream);
 
 /*
+ * kda_chunk_fwd_noalloc -- the chunkwise prefill for callers that cannot
+ * allocate device memory.  The pages have no counterpart to this entry point.
+ *
+ * Some hosts reserve all GPU memory at start-up and forbid allocation
+ * afterwards (serving engines that carve the device into their own pools,
+ * plugin interfaces that pass a plugin its tensors but no allocator); for
+ * them a library that calls cudaMalloc or a pool allocator mid-request can
+ * fail or stall.  This call takes the same arguments as kda_chunk_fwd and runs
+ * the fp32 SIMT chunk kernels (any supported dtype and head size), but keeps
+ * its intermediate data in a fixed scratch array compiled into the library
+ * (KDA_NOALLOC_SCRATCH_BYTES per GPU, held from the first load of the
+ * library's kernels on that GPU until the process exits), so it allocates
+ * nothing.  The caller still owns and passes every input and output.
+ *
+ * Limits and rules:
+ *  - the problem must fit: with blk = 4*(64*(3*dk + dv + 64) + dk) bytes per
+ *    (chunk, head) and C = number of chunk slots (B*ceil(T/64), or
+ *    floor(T/64) + B with cu_seqlens), it needs 256 + (cu_seqlens ?
+ *    round_up(8*(B+1), 256) : 0) + blk*C bytes for one head at a time (heads
+ *    then run in groups that fit).  Otherwise KDA_ERR_UNSUPPORTED is returned
+ *    before anything is launched (for dk = dv = 128 that is about 29,000
+ *    chunk-tokens per call);
+ *  - every call on a GPU shares the one scratch array, which keeps the last
+ *    call's contents: calls whose GPU work overlaps (unordered streams) race on
+ *    it, so the caller must order them;
+ *  - the first call on each device looks up the array's device address with
+ *    that device current; make that first call before any stream capture.
+ */
+#define KDA_NOALLOC_SCRATCH_BYTES (64u << 20)
+KDA_API kda_status_t kda_chunk_fwd_noalloc(const void* q, const void* k, const void* v,
+                                           const float* log_alpha, const float* beta,
+                                           const float* h0, void* out, float* hT,
+                                           const int32_t* cu_seqlens,
+                                           int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                                           float scale, kda_io_dtype_t io_dtype,
+                                           cudaStream_t stream);
+
+/*
  * kda_recurrent_step -- one decode token per sequence, the per-token step
  * itself, with the state updated in place (HBM-bound: each (sequence, head)
  * state is read once and written once).
