@@ -215,8 +215,17 @@ def time_region(fn, steps, stream):
     return e0.elapsed_time(e1)
 
 
-def run_prefill(args, ws, rank, kda, peaks):
+def prefill_config(args):
     cfg = W.BATCHED
+    if args.shape:
+        B, T, H = (int(x) for x in args.shape.split(","))
+        cfg = W.PrefillConfig(f"prefill_B{B}_H{H}_T{T}_d128_bf16", B, T, H, 128, 128, "bf16",
+                              seed=cfg.seed, gate_shift=cfg.gate_shift)
+    return cfg
+
+
+def run_prefill(args, ws, rank, kda, peaks):
+    cfg = prefill_config(args)
     inp = W.make_prefill(cfg, "cuda")
     out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
     hT = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device="cuda")
@@ -351,7 +360,7 @@ def run_decode(args, ws, rank, kda, peaks):
 def run_e2e(args, ws, kda, inp, bufs, steps):
     """Same metric through the public API with host (pinned) buffers: every
     step copies its inputs host->device and its output device->host."""
-    cfg = W.BATCHED
+    cfg = prefill_config(args)
     names = ("q", "k", "v", "log_alpha", "beta")
     host = {n: inp[n].to("cpu").pin_memory() for n in names}
     dev = {n: torch.empty_like(inp[n]) for n in names}
@@ -391,6 +400,8 @@ def main():
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="restrict the run (profiling of one kernel family)")
     ap.add_argument("--decode-steps", type=int, default=W.DECODE.steps)
+    ap.add_argument("--shape", default="", help="B,T,H override of the prefill workload "
+                    "(profiling of a smaller case; the default is the benchmark workload)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
 

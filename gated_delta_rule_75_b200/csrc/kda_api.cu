@@ -141,8 +141,9 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (impl != KDA_PREFILL_AUTO && impl != KDA_PREFILL_SIMT && impl != KDA_PREFILL_TENSORCORE)
         return KDA_ERR_INVALID_ARG;
-    if (impl == KDA_PREFILL_TENSORCORE)
-        return KDA_ERR_UNSUPPORTED;   // tensor-core kernels are added separately
+    const bool tc_shape = io_dtype == KDA_IO_BF16 && dk == 128 && dv == 128;
+    if (impl == KDA_PREFILL_TENSORCORE && !tc_shape) return KDA_ERR_UNSUPPORTED;
+    const bool use_tc = impl == KDA_PREFILL_TENSORCORE || (impl == KDA_PREFILL_AUTO && tc_shape);
     if (cu_seqlens != nullptr && B < 1) return KDA_ERR_INVALID_ARG;
     if (B == 0 || H == 0) return KDA_OK;
     const int64_t T_total = cu_seqlens ? T : B * T;
@@ -173,14 +174,15 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     si.nct = cu_seqlens ? 0 : (T + kChunk - 1) / kChunk;
     si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
 
-    // workspace: [256 B header | chunk offsets | per-(chunk, head) blocks]
-    const int64_t blk_bytes = simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
-    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 255) / 256 * 256 : 0;
+    // workspace: [1 KiB header (error word) | chunk offsets | per-(chunk, head) blocks]
+    const int64_t blk_bytes = use_tc ? tc_ws_bytes_per_chunk()
+                                     : simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
+    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 1023) / 1024 * 1024 : 0;
     const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1);
-    int64_t Hg = (workspace_budget() - 256 - off_bytes) / per_head;
+    int64_t Hg = (workspace_budget() - 1024 - off_bytes) / per_head;
     if (Hg < 1) Hg = 1;
     if (Hg > H) Hg = H;
-    const int64_t ws_bytes = 256 + off_bytes + Hg * per_head;
+    const int64_t ws_bytes = 1024 + off_bytes + Hg * per_head;
 
     StreamBuffer buf;
     cudaError_t e = buf.alloc((size_t)ws_bytes, stream);
@@ -189,21 +191,23 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     int* err_flag = reinterpret_cast<int*>(base);
     if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
     if (cu_seqlens) {
-        int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 256);
+        int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
         if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off,
                                           err_flag, stream)))
             return from_cuda(e);
         si.chunk_off = chunk_off;
     }
-    float* ws = reinterpret_cast<float*>(base + 256 + off_bytes);
-    e = run_prefill_simt(a, ws, Hg, stream);
+    unsigned char* ws = reinterpret_cast<unsigned char*>(base + 1024 + off_bytes);
+    e = use_tc ? run_prefill_tc(a, ws, Hg, err_flag, stream)
+               : run_prefill_simt(a, reinterpret_cast<float*>(ws), Hg, stream);
     if (e) return from_cuda(e);
     if (debug_mode()) {
         int flag = 0;
         if ((e = cudaMemcpyAsync(&flag, err_flag, sizeof(int), cudaMemcpyDeviceToHost, stream)))
             return from_cuda(e);
         if ((e = cudaStreamSynchronize(stream))) return from_cuda(e);
-        if (flag) return KDA_ERR_INVALID_ARG;
+        if (flag & kErrTimeoutMask) return KDA_ERR_TIMEOUT;
+        if (flag & kErrSeqlens) return KDA_ERR_INVALID_ARG;
     }
     return KDA_OK;
 }

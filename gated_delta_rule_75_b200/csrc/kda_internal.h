@@ -118,6 +118,16 @@ cudaError_t launch_decode(kda_io_dtype_t io, int dk, int dv, const void* q, cons
 int64_t simt_ws_floats_per_chunk(int dk, int dv);
 cudaError_t run_prefill_simt(const PrefillArgs& a, float* ws, int64_t Hg, cudaStream_t st);
 
+// kda_chunk_tc.cu (bf16, dk = dv = 128)
+int64_t tc_ws_bytes_per_chunk();
+cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, int* err,
+                           cudaStream_t st);
+
+// Device error word bits (workspace header): malformed cu_seqlens, and bounded
+// waits that gave up in the tensor-core kernels.
+constexpr int kErrSeqlens = 1 << 0;
+constexpr int kErrTimeoutMask = 0x3e;
+
 // kda_seqinfo.cu
 cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
                                  int64_t* chunk_off, int* err_flag, cudaStream_t st);

@@ -4,6 +4,9 @@ import sys
 import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+# every library call in the tests synchronises and reports device-side errors
+# (malformed offsets, a bounded wait that gave up) as a status code
+os.environ.setdefault("KDA_DEBUG", "1")
 if ROOT not in sys.path:
     sys.path.insert(0, ROOT)
 

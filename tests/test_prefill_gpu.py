@@ -13,7 +13,7 @@ from kda_testutil import TOL, host, oracle_pairs, oracle_prefill, rel
 
 pytestmark = pytest.mark.gpu
 
-IMPLS = ["simt"]
+IMPLS = ["simt", "tensorcore"]        # tensor cores: bf16 with dk = dv = 128 only
 
 
 @pytest.fixture(scope="module")
@@ -41,10 +41,38 @@ def check_full(kda, cfg, impl="auto"):
     return eo, eh
 
 
+def test_tiny_fp32_workload(kda):
+    """B=1, H=2, T=256, dk=dv=64, fp32 I/O, h0 = 0, seed 0 (SIMT path)."""
+    check_full(kda, W.TINY, "simt")
+    check_full(kda, W.TINY, "auto")
+
+
 @pytest.mark.parametrize("impl", IMPLS)
-def test_tiny_fp32_workload(kda, impl):
-    """B=1, H=2, T=256, dk=dv=64, fp32 I/O, h0 = 0, seed 0."""
-    check_full(kda, W.TINY, impl)
+@pytest.mark.parametrize("T", [1, 64, 150, 300])
+def test_bf16_d128_ragged(kda, impl, T):
+    """bf16, dk = dv = 128, h0 != 0, lengths below, at and across chunk boundaries."""
+    cfg = W.small_prefill(B=2, T=T, H=3, dk=128, dv=128, io_dtype="bf16", seed=T, h0_std=0.02)
+    check_full(kda, cfg, impl)
+
+
+@pytest.mark.parametrize("shift", [3.0, -4.0])
+def test_tensorcore_fast_and_slow_decay(kda, shift):
+    """Mean per-token decay e^-3.1 (fast) and e^-0.02 (slow): the sub-chunk
+    references keep the tensor-core factors in range; parity holds."""
+    cfg = W.small_prefill(B=1, T=256, H=2, dk=128, dv=128, io_dtype="bf16", seed=4,
+                          gate_shift=shift, h0_std=0.02)
+    check_full(kda, cfg, "tensorcore")
+
+
+def test_tensorcore_refuses_unsupported_shapes(kda):
+    cfg = W.small_prefill(B=1, T=64, H=1, dk=64, dv=64, io_dtype="bf16", seed=1)
+    inp = W.make_prefill(cfg, "cuda")
+    with pytest.raises(kda.KDAError):
+        run(kda, inp, "tensorcore")
+    cfg = W.small_prefill(B=1, T=64, H=1, dk=128, dv=128, io_dtype="f32", seed=1)
+    inp = W.make_prefill(cfg, "cuda")
+    with pytest.raises(kda.KDAError):
+        run(kda, inp, "tensorcore")
 
 
 @pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64), (128, 128)])
@@ -54,18 +82,17 @@ def test_head_sizes_ragged_tail(kda, dk, dv, io):
     check_full(kda, cfg, "simt")
 
 
-@pytest.mark.parametrize("io", ["f32", "bf16"])
-@pytest.mark.parametrize("impl", IMPLS)
+@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "simt"), ("bf16", "tensorcore")])
 def test_packed_variable_lengths(kda, io, impl):
     lens = [1, 63, 64, 65, 0, 130, 200, 7]
     cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype=io, seed=7, h0_std=0.05, lengths=lens)
     check_full(kda, cfg, impl)
 
 
-@pytest.mark.parametrize("impl", IMPLS)
-def test_packed_equals_separate_calls(kda, impl):
+@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "tensorcore")])
+def test_packed_equals_separate_calls(kda, io, impl):
     lens = [70, 1, 129]
-    cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype="f32", seed=8, h0_std=0.05, lengths=lens)
+    cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype=io, seed=8, h0_std=0.05, lengths=lens)
     inp = W.make_prefill(cfg, "cuda")
     out, hT = run(kda, inp, impl)
     cu = [0] + list(np.cumsum(lens))
@@ -76,16 +103,17 @@ def test_packed_equals_separate_calls(kda, impl):
         sub["h0"] = inp["h0"][n:n + 1].contiguous()
         sub["cu_seqlens"] = None
         o1, h1 = run(kda, sub, impl)
+        # the same per-sequence chunk arithmetic either way: equal to rounding noise
         assert rel(o1, host(out[:, cu[n]:cu[n + 1]]).double().numpy()) <= 1e-6
         assert rel(h1, host(hT[n:n + 1]).double().numpy()) <= 1e-6
 
 
 @pytest.mark.parametrize("t1", [64, 100])
-@pytest.mark.parametrize("impl", IMPLS)
-def test_continuation_across_calls(kda, t1, impl):
+@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "tensorcore")])
+def test_continuation_across_calls(kda, t1, io, impl):
     """[0, t1) then [t1, T) with h0 = hT of the first call equals one pass
     (on and off a chunk boundary): the state layout survives the hand-over."""
-    cfg = W.small_prefill(B=1, T=256, H=2, dk=128, dv=128, io_dtype="f32", seed=9, h0_std=0.05)
+    cfg = W.small_prefill(B=1, T=256, H=2, dk=128, dv=128, io_dtype=io, seed=9, h0_std=0.05)
     inp = W.make_prefill(cfg, "cuda")
     out, hT = run(kda, inp, impl)
     a = {k: (v[:, :t1].contiguous() if k in ("q", "k", "v", "log_alpha", "beta") else v)
@@ -96,8 +124,8 @@ def test_continuation_across_calls(kda, t1, impl):
     b["h0"] = h1
     o2, h2 = run(kda, b, impl)
     ro, rh = oracle_prefill(inp)
-    assert rel(torch.cat([o1, o2], dim=1), ro) <= TOL["f32"]
-    assert rel(h2, rh) <= TOL["f32"]
+    assert rel(torch.cat([o1, o2], dim=1), ro) <= TOL[io]
+    assert rel(h2, rh) <= TOL[io]
 
 
 def test_empty_sequence_passes_state_through(kda):
