@@ -304,14 +304,14 @@ def kernel_algorithmic_bytes(kname, cfg):
         tiles = dv // 32
         per_chunk = 4 * (CHUNK * dv + tiles * (CHUNK * 3 * dk + CHUNK * CHUNK + dk))
         return chunks * per_chunk + ht * dv * io + cfg.B * cfg.H * dk * dv * 4
-    if kname == "chunk_prep_tc":
-        return qkvgb + chunks * TC_WS_BYTES_PER_CHUNK
-    if kname == "chunk_state_tc":
-        return chunks * TC_WS_BYTES_PER_CHUNK + ht * dv * io + cfg.B * cfg.H * dk * dv * 4
+    if kname == "chunk_prep_tc":         # reads q,k,g,beta; writes the operand image
+        return ht * (2 * dk * io + dk * 4 + 4) + chunks * TC_WS_BYTES_PER_CHUNK
+    if kname == "chunk_state_tc":        # reads the image and v; writes out and hT
+        return chunks * TC_WS_BYTES_PER_CHUNK + ht * 2 * dv * io + cfg.B * cfg.H * dk * dv * 4
     return BYTES_PER_HEAD_TOKEN * ht
 
 
-TC_WS_BYTES_PER_CHUNK = 72 * 1024 + 512
+TC_WS_BYTES_PER_CHUNK = 66560         # per (chunk, head) operand image of the tensor-core path
 
 
 def run_decode(args, ws, rank, kda, peaks):

@@ -57,7 +57,7 @@ def build(force: bool = False, verbose: bool = False) -> str:
     if failed:
         raise RuntimeError("nvcc failed:\n" + "\n".join(failed))
     tmp = LIB + f".tmp{os.getpid()}"
-    subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs, "-lcuda"], check=True)
+    subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)
     return LIB
 

@@ -4,35 +4,37 @@
 // step of "Kimi Delta Attention: la atencion lineal detras de Kimi K2 y
 // Qwen3", section "Como funciona Kimi Delta Attention paso a paso"; the
 // chunkwise DPLR form is the one "Kimi Linear acaba de superar a la atencion
-// completa en sus propios terminos" says the method trains with):
+// completa en sus propios terminos" says the method trains with), with
+// T' = (I + A)^{-1} diag(beta):
 //
 //   A_ij   = beta_i sum_c k_ic k_jc e^{G_ic - G_jc}   (i > j)
 //   Aqk_ij = scale  sum_c q_ic k_jc e^{G_ic - G_jc}   (i >= j)
-//   T = (I + A)^{-1},  W = T diag(beta)(K e^G)
-//   U = T diag(beta) V - W S,  O = scale (Q e^G) S + Aqk U,
+//   W = T' (K e^G),  U = T' V - W S,  O = scale (Q e^G) S + Aqk U,
 //   S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U
 //
-// Kernel `chunk_prep_tc` (one CTA per (chunk, head), steps a and b):
-//   cumulative decay in fp32; the products behind A and Aqk as tcgen05 MMAs
-//   whose exponential factors are referenced to 16-token sub-chunk starts
-//   (every factor <= 1 except e^{G_f - G_j} inside a sub-chunk, bounded by 16
-//   tokens of decay); T by blocked forward substitution in fp32; W = T (beta K
-//   e^G) as a tcgen05 MMA.  It writes one operand image per (chunk, head),
-//   already in the 128B-swizzled shared-memory layout the state kernel's MMAs
-//   read, so the state kernel moves it with one bulk copy.
+// Kernel `chunk_prep_tc` (one CTA per (chunk, head), steps a and b): TMA loads
+//   k and q (128B-swizzled) and log_alpha; cumulative decay in the log2 domain;
+//   the products behind A and Aqk as tcgen05 MMAs whose exponential factors are
+//   referenced to 16-token sub-chunk starts (every factor <= 1 except
+//   e^{G_f - G_j} inside a sub-chunk, bounded by 16 tokens of decay); the
+//   diagonal 16x16 blocks of (I + A)^{-1} by fp32 forward substitution and the
+//   off-diagonal blocks by tf32 mma.sync block products; W = T' (K e^G) as a
+//   tcgen05 MMA.  It writes one operand image per (chunk, head), already in the
+//   128B-swizzled shared-memory layout the state kernel's MMAs read.
 // Kernel `chunk_state_tc` (one CTA per (sequence, head), steps c and d): walks
 //   the chunks in order with S^T (dv x dk, fp32) resident in tensor memory and
-//   a bf16 copy in shared memory as the MMA operand; images are double-buffered
-//   with cp.async.bulk.  Per chunk:
-//     U^T = (beta V)^T T^T + S^T (-W)^T      (MMA0 + MMA1a, fp32 in TMEM)
-//     O^T = S^T (scale Q e^G)^T               (MMA1b)
-//     [O^T | S^T] += U^T [Aqk^T | K e^{G_last - G}]   (MMA2, N = 64 + 128)
+//   a bf16 copy in shared memory as the MMA operand; each chunk's image (bulk
+//   copy) and its v tile (TMA) are double-buffered.  Per chunk:
+//     U^T = V^T T'^T + S^T (-W)^T             (fp32 in TMEM)
+//     O^T = S^T (scale Q e^G)^T
+//     [O^T | S^T] += U^T [Aqk^T | K e^{G_last - G}]   (one MMA, N = 64 + 128)
 //   then O goes to HBM, S^T is copied to bf16 for the next chunk and scaled by
 //   the next chunk's e^{G_last} in TMEM.
-// Every wait on an mbarrier is bounded; on a timeout the CTA records the fact
-// in the workspace error word, drains its own copies and frees its TMEM.
+// Every mbarrier wait is bounded; on a timeout the CTA records it in the
+// workspace error word, drains its own copies and frees its TMEM.
 #include "kda_common.cuh"
 #include "kda_internal.h"
+#include "kda_tma.cuh"
 #include "kda_umma.cuh"
 
 namespace kda {
@@ -43,18 +45,25 @@ namespace tc {
 
 constexpr int C = 64;
 constexpr int D = 128;     // dk = dv = 128
+constexpr float kLog2e = 1.4426950408889634f;
 
 // Operand image of one (chunk, head), byte offsets (all 1024-aligned).
-constexpr uint32_t IMG_W = 0;          // -W         K-major B: 64 token rows x 128 ch (2 K-blocks)
+constexpr uint32_t IMG_W = 0;          // -W          K-major B: 64 token rows x 128 ch (2 K-blocks)
 constexpr uint32_t IMG_QG = 16384;     // scale Q e^G K-major B: same shape
-constexpr uint32_t IMG_B2 = 32768;     // MN-major B, K = 64 token rows: [Aqk^T | K e^{Gl-G}] (3 x 64 cols)
-constexpr uint32_t IMG_V = 57344;      // (beta V)^T MN-major A: M = dv (2 blocks), K = 64 token rows
-constexpr uint32_t IMG_T = 73728;      // T K-major: 64 rows x 64
-constexpr uint32_t IMG_GAM = 81920;    // e^{G_last}, fp32 [128]
-constexpr uint32_t IMG_BYTES = 82944;
+constexpr uint32_t IMG_B2 = 32768;     // MN-major B, K = 64 token rows: [Aqk^T | K e^{Gl-G}] (3 x 64)
+constexpr uint32_t IMG_T = 57344;      // T' = T diag(beta), K-major: 64 rows x 64
+constexpr uint32_t IMG_GAM = 65536;    // e^{G_last}, fp32 [128]
+constexpr uint32_t IMG_BYTES = 66560;
 
 // Kvar rows: variant p holds key rows 0 .. 16p+15 referenced to token 16p.
 __device__ __constant__ int kVoff[4] = {0, 16, 48, 96};
+
+__device__ __forceinline__ float ex2(float x)
+{
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
 
 __device__ __forceinline__ void unpack8(uint4 u, float* f)
 {
@@ -85,30 +94,81 @@ __device__ __forceinline__ void ld8f(const float* p, float* f)
     f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+__device__ __forceinline__ uint32_t tf32(float x)
+{
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// acc (16x16, m16n8 fragments for the two 8-column halves) += X * Y, where X
+// and Y are 16x16 fp32 blocks in shared memory with a row pitch of 64 floats.
+__device__ __forceinline__ void mma16x16x16_tf32(float (&acc)[2][4], const float* X, const float* Y,
+                                                 int lane)
+{
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = tf32(X[g * 64 + 8 * ks + q]);
+        const uint32_t a1 = tf32(X[(g + 8) * 64 + 8 * ks + q]);
+        const uint32_t a2 = tf32(X[g * 64 + 8 * ks + q + 4]);
+        const uint32_t a3 = tf32(X[(g + 8) * 64 + 8 * ks + q + 4]);
+#pragma unroll
+        for (int nh = 0; nh < 2; ++nh) {
+            const uint32_t b0 = tf32(Y[(8 * ks + q) * 64 + 8 * nh + g]);
+            const uint32_t b1 = tf32(Y[(8 * ks + q + 4) * 64 + 8 * nh + g]);
+            asm volatile(
+                "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+                "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                : "+f"(acc[nh][0]), "+f"(acc[nh][1]), "+f"(acc[nh][2]), "+f"(acc[nh][3])
+                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        }
+    }
+}
+
+// Store a 16x16 accumulator (m16n8 fragments) scaled by `s` into a block with
+// a row pitch of 64 floats.
+__device__ __forceinline__ void store16x16(float* Z, const float (&acc)[2][4], float s, int lane)
+{
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        Z[g * 64 + 8 * nh + 2 * q] = s * acc[nh][0];
+        Z[g * 64 + 8 * nh + 2 * q + 1] = s * acc[nh][1];
+        Z[(g + 8) * 64 + 8 * nh + 2 * q] = s * acc[nh][2];
+        Z[(g + 8) * 64 + 8 * nh + 2 * q + 1] = s * acc[nh][3];
+    }
+}
+
 // ---------------------------------------------------------------------------
 // prep kernel shared memory (bytes from a 1024-aligned base)
 // ---------------------------------------------------------------------------
-constexpr uint32_t P_K = 0;            // MN-major [t][c] image of k, later beta K e^G   16 KB
-constexpr uint32_t P_G = 16384;        // fp32 G [64][128]; later T bf16 image            32 KB
-constexpr uint32_t P_KQ = 49152;       // K-major B: [Kin_p; Qin_p] x 4, one K-block     16 KB
-constexpr uint32_t P_KV = 65536;       // K-major A: Kvar rows (160), one K-block        20 KB
-constexpr uint32_t P_A = 49152;        // fp32 A [64][64] (aliases KQ after the strips)  16 KB
-constexpr uint32_t P_T = 65536;        // fp32 T [64][64] (aliases KV)                   16 KB
-constexpr uint32_t P_VEC = 86016;      // per-channel vectors: egf[4], eglf[4], dvec[6]  7 KB
+constexpr uint32_t P_K = 0;            // k, MN-major [t][c] image (TMA, swizzled); later K e^G   16 KB
+constexpr uint32_t P_Q = 16384;        // q, same layout (TMA); later the T' bf16 image           16 KB
+constexpr uint32_t P_G = 32768;        // fp32 log_alpha [64][128] (TMA), then G (log2 units)    32 KB
+constexpr uint32_t P_KQ = 65536;       // K-major B: [Kin_p; Qin_p] x 4, one K-block             16 KB
+constexpr uint32_t P_KV = 81920;       // K-major A: Kvar rows (160), one K-block                20 KB
+constexpr uint32_t P_A = 65536;        // fp32 A [64][64] (aliases KQ after the strips)          16 KB
+constexpr uint32_t P_T = 81920;        // fp32 T [64][64] (aliases KV)                           16 KB
+constexpr uint32_t P_VEC = 102400;     // per-channel vectors: egf[4], eglf[4], dvec[6]          7 KB
 constexpr uint32_t P_BETA = P_VEC + 14 * 512;
 constexpr uint32_t P_BYTES = P_BETA + 256;
 constexpr uint32_t P_SMEM = P_BYTES + 1024 + 64;
+constexpr uint32_t P_TX = 16384 + 16384 + 32768;   // bytes the input TMA loads deliver
+
+struct PrepMaps {
+    CUtensorMap k, q, g;
+};
 
 __global__ void __launch_bounds__(128)
-chunk_prep_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
-                     const __nv_bfloat16* __restrict__ v, const float* __restrict__ log_alpha,
-                     const float* __restrict__ beta, SeqInfo si, int64_t H, int64_t h_base,
-                     int64_t Hg, float scale, unsigned char* __restrict__ ws, int* __restrict__ err)
+chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
+                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
+                     unsigned char* __restrict__ ws, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar;
+    __shared__ uint64_t bar_in, bar;
     __shared__ uint32_t tmem_base;
 
     const int64_t gc = blockIdx.x;
@@ -125,156 +185,142 @@ chunk_prep_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
     float* dvec = eglf + 4 * D;                                   // [6][128]  e^{G_fp - G_fr}
     float* sB = reinterpret_cast<float*>(sm + P_BETA);
 
-    if (tid == 0) { mbar_init(&bar, 1); fence_mbar_init(); }
-    if (w == 0) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
-
-    // ---- load beta, g (fp32 rows) and k (MN-major image); rows >= len are zero
+    if (tid == 0) {
+        mbar_init(&bar_in, 1);
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        tma::expect_tx(&bar_in, P_TX);
+        const int32_t y = (int32_t)t0, x = (int32_t)(h * D);
+        tma::load_2d(sm + P_K, &maps.k, x, y, &bar_in);
+        tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_in);
+        tma::load_2d(sm + P_Q, &maps.q, x, y, &bar_in);
+        tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_in);
+        tma::load_2d(sm + P_G, &maps.g, x, y, &bar_in);
+    }
+    if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
     if (tid < C) sB[tid] = tid < len ? beta[(t0 + tid) * H + h] : 0.f;
-#pragma unroll 4
-    for (int i = 0; i < 16; ++i) {
-        const int e = tid + 128 * i, t = e >> 5, c4 = e & 31;
-        float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < len) x = *reinterpret_cast<const float4*>(log_alpha + ((t0 + t) * H + h) * D + 4 * c4);
-        *reinterpret_cast<float4*>(sG + t * D + 4 * c4) = x;
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = tid + 128 * i, t = e >> 4, ch = e & 15;
-        uint4 x = make_uint4(0, 0, 0, 0);
-        if (t < len) x = *reinterpret_cast<const uint4*>(k + ((t0 + t) * H + h) * D + 8 * ch);
-        *reinterpret_cast<uint4*>(sm + P_K + (ch >> 3) * 8192 + sw128_offset(t, (8 * ch) & 63)) = x;
-    }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
+    bool ok = __syncthreads_and(mbar_wait(&bar_in, 0, err, 1) ? 1 : 0);
 
-    // ---- (a) cumulative log-decay per channel; per-channel reference vectors
-    {
-        const int c = tid;
-        float run = 0.f;
-        for (int t = 0; t < C; ++t) { run += sG[t * D + c]; sG[t * D + c] = run; }
-        const float Gl = run;
-        float Gf[4];
+    if (ok) {
+        // ---- (a) cumulative log-decay per channel (log2 units); rows >= len add nothing
+        {
+            const int c = tid;
+            float run = 0.f;
+            for (int t = 0; t < C; ++t) {
+                if (t < len) run += kLog2e * sG[t * D + c];
+                sG[t * D + c] = run;
+            }
+            const float Gl = run;
+            float Gf[4];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            Gf[p] = sG[(16 * p) * D + c];
-            egf[p * D + c] = expf(Gf[p]);
-            eglf[p * D + c] = expf(Gl - Gf[p]);
+            for (int p = 0; p < 4; ++p) {
+                Gf[p] = sG[(16 * p) * D + c];
+                egf[p * D + c] = ex2(Gf[p]);
+                eglf[p * D + c] = ex2(Gl - Gf[p]);
+            }
+            int idx = 0;
+#pragma unroll
+            for (int p = 1; p < 4; ++p)
+#pragma unroll
+                for (int r = 0; r < p; ++r) dvec[(idx++) * D + c] = ex2(Gf[p] - Gf[r]);
+            reinterpret_cast<float*>(img + IMG_GAM)[c] = ex2(Gl);
         }
-        int idx = 0;
-#pragma unroll
-        for (int p = 1; p < 4; ++p)
-#pragma unroll
-            for (int r = 0; r < p; ++r) dvec[(idx++) * D + c] = expf(Gf[p] - Gf[r]);
-        reinterpret_cast<float*>(img + IMG_GAM)[c] = expf(Gl);
-    }
-    __syncthreads();
-
-    // ---- (beta V)^T image, straight to the workspace
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = tid + 128 * i, t = e >> 4, ch = e & 15;
-        float f[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        if (t < len) unpack8(*reinterpret_cast<const uint4*>(v + ((t0 + t) * H + h) * D + 8 * ch), f);
-        const float b = sB[t];
-#pragma unroll
-        for (int j = 0; j < 8; ++j) f[j] *= b;
-        *reinterpret_cast<uint4*>(img + IMG_V + (ch >> 3) * 8192 + sw128_offset(t, (8 * ch) & 63)) = pack8(f);
-    }
-
-    // ---- (b1) A / Aqk strips: two passes over channel halves
-    const int ch8 = tid & 7, tr = tid >> 3;
-    bool ok = true;
-    for (int hh = 0; hh < 2; ++hh) {
-        const int c0 = 64 * hh + 8 * ch8;
-#pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            const int t = 16 * p + tr;
-            float G8[8], Gf8[8], kk[8], qq[8], E1[8], R1[8];
-            ld8f(sG + t * D + c0, G8);
-            ld8f(sG + (16 * p) * D + c0, Gf8);
-            const uint32_t koff = P_K + hh * 8192 + sw128_offset(t, 8 * ch8);
-            unpack8(*reinterpret_cast<const uint4*>(sm + koff), kk);
-            if (t < len) unpack8(*reinterpret_cast<const uint4*>(q + ((t0 + t) * H + h) * D + c0), qq);
-            else {
-#pragma unroll
-                for (int j = 0; j < 8; ++j) qq[j] = 0.f;
-            }
-            float kin[8], qin[8], kd[8], tmp[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) {
-                E1[j] = expf(G8[j] - Gf8[j]);      // <= 1
-                R1[j] = expf(Gf8[j] - G8[j]);      // >= 1, at most 15 tokens of decay
-                kin[j] = kk[j] * E1[j];
-                qin[j] = scale * qq[j] * E1[j];
-                kd[j] = kk[j] * R1[j];
-            }
-            *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + tr, 8 * ch8)) = pack8(kin);
-            *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + 16 + tr, 8 * ch8)) = pack8(qin);
-            *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[p] + t, 8 * ch8)) = pack8(kd);
-#pragma unroll
-            for (int pp = p + 1; pp < 4; ++pp) {
-                const float* dv8 = dvec + ((pp * (pp - 1)) / 2 + p) * D + c0;
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * dv8[j];
-                *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pp] + t, 8 * ch8)) = pack8(tmp);
-            }
-            // scale Q e^G (K-major rows = tokens) and K e^{G_last - G} (MN-major rows = tokens)
-            const float* eg = egf + p * D + c0;
-            const float* egl = eglf + p * D + c0;
-#pragma unroll
-            for (int j = 0; j < 8; ++j) tmp[j] = qin[j] * eg[j];
-            *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
-#pragma unroll
-            for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * egl[j];
-            *reinterpret_cast<uint4*>(img + IMG_B2 + (1 + hh) * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
-            // beta K e^G replaces k in place (B operand of the W product)
-            const float b = sB[t];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) tmp[j] = b * kin[j] * eg[j];
-            *reinterpret_cast<uint4*>(sm + koff) = pack8(tmp);
-        }
-        fence_smem_to_async();
-        fence_before_sync();
         __syncthreads();
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t idesc = make_idesc_bf16(64, 32, false, false);
+
+        // ---- (b1) A / Aqk strips: operands built per channel half, MMAs accumulate
+        const int ch8 = tid & 7, tr = tid >> 3;
+        for (int hh = 0; hh < 2 && ok; ++hh) {
+            const int c0 = 64 * hh + 8 * ch8;
 #pragma unroll
-            for (int p = 0; p < 4; ++p)
+            for (int p = 0; p < 4; ++p) {
+                const int t = 16 * p + tr;
+                const bool live = t < len;
+                float G8[8], Gf8[8], kk[8], qq[8];
+                ld8f(sG + t * D + c0, G8);
+                ld8f(sG + (16 * p) * D + c0, Gf8);
+                const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
+                unpack8(*reinterpret_cast<const uint4*>(sm + P_K + off), kk);
+                unpack8(*reinterpret_cast<const uint4*>(sm + P_Q + off), qq);
+                float kin[8], qin[8], kd[8], tmp[8];
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) {
-                    const uint64_t ad = make_desc(smem_u32(sm + P_KV + kVoff[p] * 128 + ks * 32), 16, 1024);
-                    const uint64_t bd = make_desc(smem_u32(sm + P_KQ + 32 * p * 128 + ks * 32), 16, 1024);
-                    mma_bf16(tmem + 32 * p, ad, bd, idesc, (hh > 0 || ks > 0) ? 1u : 0u);
+                for (int j = 0; j < 8; ++j) {
+                    const float x = G8[j] - Gf8[j];
+                    const float e1 = ex2(x);          // <= 1
+                    const float r1 = ex2(-x);         // >= 1, at most 15 tokens of decay
+                    const float kv = live ? kk[j] : 0.f;
+                    kin[j] = kv * e1;
+                    qin[j] = live ? scale * qq[j] * e1 : 0.f;
+                    kd[j] = kv * r1;
                 }
-            commit(&bar);
+                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + tr, 8 * ch8)) = pack8(kin);
+                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + 16 + tr, 8 * ch8)) = pack8(qin);
+                *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[p] + t, 8 * ch8)) = pack8(kd);
+#pragma unroll
+                for (int pp = p + 1; pp < 4; ++pp) {
+                    const float* dv8 = dvec + ((pp * (pp - 1)) / 2 + p) * D + c0;
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * dv8[j];
+                    *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pp] + t, 8 * ch8)) = pack8(tmp);
+                }
+                const float* eg = egf + p * D + c0;
+                const float* egl = eglf + p * D + c0;
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tmp[j] = qin[j] * eg[j];
+                *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * egl[j];
+                *reinterpret_cast<uint4*>(img + IMG_B2 + (1 + hh) * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
+                // K e^G replaces k in place (B operand of W = T' (K e^G))
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tmp[j] = kin[j] * eg[j];
+                *reinterpret_cast<uint4*>(sm + P_K + off) = pack8(tmp);
+            }
+            fence_smem_to_async();
+            fence_before_sync();
+            __syncthreads();
+            if (tid == 0) {
+                fence_after_sync();
+                const uint32_t idesc = make_idesc_bf16(64, 32, false, false);
+#pragma unroll
+                for (int p = 0; p < 4; ++p)
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks) {
+                        const uint64_t ad = make_desc(smem_u32(sm + P_KV + kVoff[p] * 128 + ks * 32), 16, 1024);
+                        const uint64_t bd = make_desc(smem_u32(sm + P_KQ + 32 * p * 128 + ks * 32), 16, 1024);
+                        mma_bf16(tmem + 32 * p, ad, bd, idesc, (hh > 0 || ks > 0) ? 1u : 0u);
+                    }
+                commit(&bar);
+            }
+            ok = __syncthreads_and(mbar_wait(&bar, hh & 1, err, 2) ? 1 : 0);
+            fence_after_sync();
         }
-        ok = __syncthreads_and(mbar_wait(&bar, hh & 1, err, 1) ? 1 : 0) && ok;
-        fence_after_sync();
-        if (!ok) break;
     }
 
     float* sA = reinterpret_cast<float*>(sm + P_A);
     float* sT = reinterpret_cast<float*>(sm + P_T);
     if (ok) {
         // ---- extract A (fp32, for the inverse) and Aqk^T (bf16 image rows)
-        const bool act = l < 16;
         const int j = 16 * w + l;
+        float kp[4][16], qp[4][16];
 #pragma unroll
         for (int p = 0; p < 4; ++p) {
-            float kp[16], qp[16];
-            tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 32 * p, kp);
-            tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 32 * p + 16, qp);
-            tmem_wait_ld();
-            if (act) {
+            tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 32 * p, kp[p]);
+            tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 32 * p + 16, qp[p]);
+        }
+        tmem_wait_ld();
+        if (l < 16) {
+#pragma unroll
+            for (int p = 0; p < 4; ++p) {
                 float aq[16];
 #pragma unroll
                 for (int cc = 0; cc < 16; ++cc) {
                     const int i = 16 * p + cc;
-                    sA[i * C + j] = (j < i) ? sB[i] * kp[cc] : 0.f;
-                    aq[cc] = (j <= i) ? qp[cc] : 0.f;
+                    sA[i * C + j] = (j < i) ? sB[i] * kp[p][cc] : 0.f;
+                    aq[cc] = (j <= i) ? qp[p][cc] : 0.f;
                 }
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p + 8)) = pack8(aq + 8);
@@ -284,118 +330,111 @@ chunk_prep_tc_kernel(const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* _
         __syncthreads();
 
         // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
-        for (int e = tid; e < C * C; e += 128) sT[e] = 0.f;
-        __syncthreads();
         if (tid < C) {
             const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-            sT[(o + cc) * C + o + cc] = 1.f;
-            for (int r = cc + 1; r < 16; ++r) {
-                float acc = 0.f;
-                for (int m = cc; m < r; ++m) acc += sA[(o + r) * C + o + m] * sT[(o + m) * C + o + cc];
-                sT[(o + r) * C + o + cc] = -acc;
+            for (int r = 0; r < 16; ++r) {
+                float val = (r == cc) ? 1.f : 0.f;
+                if (r > cc) {
+                    float acc = 0.f;
+                    for (int m = cc; m < r; ++m) acc += sA[(o + r) * C + o + m] * sT[(o + m) * C + o + cc];
+                    val = -acc;
+                }
+                sT[(o + r) * C + o + cc] = val;
             }
         }
         __syncthreads();
-        // off-diagonal blocks by distance d: T_pr = -T_pp * sum_{r<=m<p} A_pm T_mr.
-        // X_pr = sum_m A_pm T_mr is parked in the (unused, zero) upper block (r, p) of sA.
+        // off-diagonal blocks by distance d (one warp per block):
+        //   X_pr = sum_{r<=m<p} A_pm T_mr  (parked in the unused upper block (r, p) of A),
+        //   T_pr = -T_pp X_pr
         for (int d = 1; d < 4; ++d) {
-            const int nb = 4 - d;
-            for (int e = tid; e < nb * 256; e += 128) {
-                const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                const int p = d + bi, r = bi;
-                float acc = 0.f;
+            const int r = w, p = w + d;
+            if (p < 4) {
+                float acc[2][4] = {};
                 for (int m = r; m < p; ++m)
-                    for (int x = 0; x < 16; ++x)
-                        acc += sA[(16 * p + rr) * C + 16 * m + x] * sT[(16 * m + x) * C + 16 * r + cc];
-                sA[(16 * r + rr) * C + 16 * p + cc] = acc;
-            }
-            __syncthreads();
-            for (int e = tid; e < nb * 256; e += 128) {
-                const int bi = e >> 8, rr = (e >> 4) & 15, cc = e & 15;
-                const int p = d + bi, r = bi;
-                float acc = 0.f;
-                for (int x = 0; x < 16; ++x)
-                    acc += sT[(16 * p + rr) * C + 16 * p + x] * sA[(16 * r + x) * C + 16 * p + cc];
-                sT[(16 * p + rr) * C + 16 * r + cc] = -acc;
+                    mma16x16x16_tf32(acc, sA + (16 * p) * C + 16 * m, sT + (16 * m) * C + 16 * r, l);
+                store16x16(sA + (16 * r) * C + 16 * p, acc, 1.f, l);
+                __syncwarp();
+                float acc2[2][4] = {};
+                mma16x16x16_tf32(acc2, sT + (16 * p) * C + 16 * p, sA + (16 * r) * C + 16 * p, l);
+                store16x16(sT + (16 * p) * C + 16 * r, acc2, -1.f, l);
             }
             __syncthreads();
         }
-        // T in bf16: K-major image (rows i, K = j) in shared memory and in the workspace
+        // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
         for (int e = tid; e < C * 8; e += 128) {
             const int i = e >> 3, cb = e & 7;
             float f[8];
             ld8f(sT + i * C + 8 * cb, f);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * sB[8 * cb + x] : 0.f;
             const uint4 u = pack8(f);
-            *reinterpret_cast<uint4*>(sm + P_G + sw128_offset(i, 8 * cb)) = u;
+            *reinterpret_cast<uint4*>(sm + P_Q + sw128_offset(i, 8 * cb)) = u;
             *reinterpret_cast<uint4*>(img + IMG_T + sw128_offset(i, 8 * cb)) = u;
         }
         fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
 
-        // ---- (b3) W = T (beta K e^G): M = 64 tokens, N = 128 channels, K = 64 tokens
+        // ---- (b3) W = T' (K e^G): M = 64 tokens, N = 128 channels, K = 64 tokens
         if (tid == 0) {
             fence_after_sync();
             const uint32_t idesc = make_idesc_bf16(64, 128, false, true);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = make_desc(smem_u32(sm + P_G + ks * 32), 16, 1024);
+                const uint64_t ad = make_desc(smem_u32(sm + P_Q + ks * 32), 16, 1024);
                 const uint64_t bd = make_desc(smem_u32(sm + P_K + ks * 2048), 8192, 1024);
-                mma_bf16(tmem + 128, ad, bd, idesc, ks > 0 ? 1u : 0u);
+                mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
             }
             commit(&bar);
         }
-        ok = __syncthreads_and(mbar_wait(&bar, 0, err, 2) ? 1 : 0);
+        ok = __syncthreads_and(mbar_wait(&bar, 0, err, 3) ? 1 : 0);
         fence_after_sync();
         if (ok) {
             const int i = 16 * w + l;
 #pragma unroll
-            for (int cb = 0; cb < 8; ++cb) {
-                float f[16];
-                tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 128 + 16 * cb, f);
+            for (int half = 0; half < 2; ++half) {
+                float f[4][16];
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb)
+                    tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 64 * half + 16 * cb, f[cb]);
                 tmem_wait_ld();
                 if (l < 16) {
+                    unsigned char* dst = img + IMG_W + half * 8192;
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) f[x] = -f[x];
-                    const int c = 16 * cb;
-                    unsigned char* dst = img + IMG_W + (c >> 6) * 8192;
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(i, c & 63)) = pack8(f);
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(i, (c & 63) + 8)) = pack8(f + 8);
+                    for (int cb = 0; cb < 4; ++cb) {
+#pragma unroll
+                        for (int x = 0; x < 16; ++x) f[cb][x] = -f[cb][x];
+                        *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
+                        *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
+                    }
                 }
             }
         }
+    } else {
+        // the input loads may still be in flight: let them land before leaving
+        mbar_wait(&bar_in, 0, nullptr, 0, 1u << 16);
     }
     fence_before_sync();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tmem, 256);
+    if (w == 0) tmem_dealloc(tmem, 128);
 }
 
 // ---------------------------------------------------------------------------
 // state kernel
 // ---------------------------------------------------------------------------
-constexpr uint32_t S_STAGE0 = 0;
-constexpr uint32_t S_STAGE1 = IMG_BYTES;
-constexpr uint32_t S_SBF = 2 * IMG_BYTES;           // S^T bf16, K-major A: 128 rows x 128 (2 K-blocks)
-constexpr uint32_t S_UBF = S_SBF + 32768;           // U^T bf16, K-major A: 128 rows x 64
+constexpr uint32_t STAGE_V = IMG_BYTES;                  // v tile, MN-major A (2 blocks of 8 KB)
+constexpr uint32_t STAGE_BYTES = IMG_BYTES + 16384;      // 81 KB
+constexpr uint32_t S_SBF = 2 * STAGE_BYTES;              // S^T bf16, K-major A: 128 rows x 128 (2 K-blocks)
+constexpr uint32_t S_UBF = S_SBF + 32768;                // U^T bf16, K-major A: 128 rows x 64
 constexpr uint32_t S_BYTES = S_UBF + 16384;
 constexpr uint32_t S_SMEM = S_BYTES + 1024;
 
-__device__ __forceinline__ void bulk_load(void* dst_smem, const void* src, uint32_t bytes, uint64_t* bar)
-{
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;"
-                 : : "r"(smem_u32(bar)), "r"(bytes) : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
-        :
-        : "r"(smem_u32(dst_smem)), "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
-
 template <bool kHasH0>
 __global__ void __launch_bounds__(128, 1)
-chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restrict__ h0,
-                      __nv_bfloat16* __restrict__ out, float* __restrict__ hT, SeqInfo si,
-                      int64_t H, int64_t h_base, int64_t Hg, int* __restrict__ err)
+chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constant__ CUtensorMap vmap,
+                      const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
+                      float* __restrict__ hT, SeqInfo si, int64_t H, int64_t h_base, int64_t Hg,
+                      int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -420,12 +459,22 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restr
             for (int c = 0; c < D; ++c) hTp[c * D + j] = kHasH0 ? h0p[c * D + j] : 0.f;
         return;
     }
-    auto image = [&](int64_t ch) { return ws + ((gc0 + ch) * Hg + hl) * (int64_t)IMG_BYTES; };
+    auto load_stage = [&](int64_t ch, int s) {          // one thread
+        unsigned char* st = sm + s * STAGE_BYTES;
+        fence_smem_to_async();
+        tma::expect_tx(&full[s], IMG_BYTES + 16384);
+        tma::load_bulk(st, ws + ((gc0 + ch) * Hg + hl) * (int64_t)IMG_BYTES, IMG_BYTES, &full[s]);
+        const int32_t y = (int32_t)(bos + ch * C), x = (int32_t)(h * D);
+        tma::load_2d(st + STAGE_V, &vmap, x, y, &full[s]);
+        tma::load_2d(st + STAGE_V + 8192, &vmap, x + 64, y, &full[s]);
+    };
 
     if (tid == 0) {
         mbar_init(&full[0], 1); mbar_init(&full[1], 1);
         mbar_init(&bar1, 1); mbar_init(&bar2, 1);
         fence_mbar_init();
+        load_stage(0, 0);
+        if (nch > 1) load_stage(1, 1);
     }
     if (w == 0) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
     fence_before_sync();
@@ -434,20 +483,14 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restr
     const uint32_t tmem = tmem_base;
     const uint32_t lane = (uint32_t)(32 * w) << 16;
     const uint32_t tU = tmem, tO = tmem + 64, tS = tmem + 128;
-    bool pending[2] = {false, false};
+    bool pending[2] = {true, nch > 1};
 
-    if (tid == 0) {
-        bulk_load(sm + S_STAGE0, image(0), IMG_BYTES, &full[0]);
-        if (nch > 1) bulk_load(sm + S_STAGE1, image(1), IMG_BYTES, &full[1]);
-    }
-    pending[0] = true;
-    pending[1] = nch > 1;
-    bool ok = __syncthreads_and(mbar_wait(&full[0], 0, err, 3) ? 1 : 0);
+    bool ok = __syncthreads_and(mbar_wait(&full[0], 0, err, 4) ? 1 : 0);
     if (ok) pending[0] = false;
 
     // initial state: bf16 copy (operand) and gamma_0-scaled fp32 in TMEM
     if (ok) {
-        const float* gam = reinterpret_cast<const float*>(sm + S_STAGE0 + IMG_GAM);
+        const float* gam = reinterpret_cast<const float*>(sm + IMG_GAM);
 #pragma unroll 1
         for (int cb = 0; cb < 8; ++cb) {
             float f[16];
@@ -468,18 +511,18 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restr
 
     for (int64_t ch = 0; ok && ch < nch; ++ch) {
         const int s = (int)(ch & 1);
-        unsigned char* st = sm + (s ? S_STAGE1 : S_STAGE0);
+        unsigned char* st = sm + s * STAGE_BYTES;
         const int64_t t0 = bos + ch * C;
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
         const uint32_t ph = (uint32_t)(ch & 1);
 
         if (tid == 0) {
             fence_after_sync();
-            // U^T = (beta V)^T T^T  (M = dv, N = 64, K = 64)
+            // U^T = V^T T'^T  (M = dv, N = 64, K = 64)
             const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tU, make_desc(smem_u32(st + IMG_V + ks * 2048), 8192, 1024),
+                mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
                          make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
             // U^T += S^T (-W)^T ; O^T = S^T (scale Q e^G)^T   (M = dv, N = 64, K = dk)
             const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
@@ -491,18 +534,21 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restr
             }
             commit(&bar1);
         }
-        ok = __syncthreads_and(mbar_wait(&bar1, ph, err, 4) ? 1 : 0);
+        ok = __syncthreads_and(mbar_wait(&bar1, ph, err, 5) ? 1 : 0);
         fence_after_sync();
         if (!ok) break;
 
         // U^T (fp32, TMEM) -> bf16 operand rows
+        {
+            float f[4][16];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float f[16];
-            tmem_ld16(tU + lane + 16 * cb, f);
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tU + lane + 16 * cb, f[cb]);
             tmem_wait_ld();
-            *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, 16 * cb)) = pack8(f);
-            *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, 16 * cb + 8)) = pack8(f + 8);
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, 16 * cb)) = pack8(f[cb]);
+                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, 16 * cb + 8)) = pack8(f[cb] + 8);
+            }
         }
         fence_smem_to_async();
         fence_before_sync();
@@ -523,47 +569,54 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restr
 
         // the stage is free again: prefetch chunk ch + 2 into it
         if (ch + 2 < nch) {
-            if (tid == 0) bulk_load(st, image(ch + 2), IMG_BYTES, &full[s]);
+            if (tid == 0) load_stage(ch + 2, s);
             pending[s] = true;
         }
         const bool last = (ch + 1 == nch);
         const float* gam_next = nullptr;
         if (!last) {
-            ok = __syncthreads_and(mbar_wait(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 3) ? 1 : 0);
+            ok = __syncthreads_and(mbar_wait(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 4) ? 1 : 0);
             if (!ok) break;
             pending[s ^ 1] = false;
-            gam_next = reinterpret_cast<const float*>(sm + (s ? S_STAGE0 : S_STAGE1) + IMG_GAM);
+            gam_next = reinterpret_cast<const float*>(sm + (s ^ 1) * STAGE_BYTES + IMG_GAM);
         }
 
         // output rows of this chunk
+        {
+            float f[4][16];
 #pragma unroll
-        for (int cb = 0; cb < 4; ++cb) {
-            float f[16];
-            tmem_ld16(tO + lane + 16 * cb, f);
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tO + lane + 16 * cb, f[cb]);
             tmem_wait_ld();
+            __nv_bfloat16* op = out + (t0 * H + h) * D + j;
 #pragma unroll
-            for (int x = 0; x < 16; ++x) {
-                const int t = 16 * cb + x;
-                if (t < len) out[((t0 + t) * H + h) * D + j] = __float2bfloat16_rn(f[x]);
-            }
+            for (int cb = 0; cb < 4; ++cb)
+#pragma unroll
+                for (int x = 0; x < 16; ++x)
+                    if (16 * cb + x < len) op[(int64_t)(16 * cb + x) * H * D] = __float2bfloat16_rn(f[cb][x]);
         }
         // next entry state: bf16 operand copy, then scaled by the next chunk's decay
 #pragma unroll 1
-        for (int cb = 0; cb < 8; ++cb) {
-            float f[16];
-            tmem_ld16(tS + lane + 16 * cb, f);
+        for (int half = 0; half < 2; ++half) {
+            float f[4][16];
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tS + lane + 64 * half + 16 * cb, f[cb]);
             tmem_wait_ld();
             if (last) {
                 if (hTp)
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) hTp[(16 * cb + x) * D + j] = f[x];
-            } else {
-                unsigned char* dst = sm + S_SBF + (cb >> 2) * 16384;
-                *reinterpret_cast<uint4*>(dst + sw128_offset(j, (16 * cb) & 63)) = pack8(f);
-                *reinterpret_cast<uint4*>(dst + sw128_offset(j, ((16 * cb) & 63) + 8)) = pack8(f + 8);
+                    for (int cb = 0; cb < 4; ++cb)
 #pragma unroll
-                for (int x = 0; x < 16; ++x) f[x] *= gam_next[16 * cb + x];
-                tmem_st16(tS + lane + 16 * cb, f);
+                        for (int x = 0; x < 16; ++x) hTp[(64 * half + 16 * cb + x) * D + j] = f[cb][x];
+            } else {
+                unsigned char* dst = sm + S_SBF + half * 16384;
+#pragma unroll
+                for (int cb = 0; cb < 4; ++cb) {
+                    *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f[cb]);
+                    *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f[cb] + 8);
+#pragma unroll
+                    for (int x = 0; x < 16; ++x) f[cb][x] *= gam_next[64 * half + 16 * cb + x];
+                    tmem_st16(tS + lane + 64 * half + 16 * cb, f[cb]);
+                }
             }
         }
         tmem_wait_st();
@@ -574,7 +627,10 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const float* __restr
     if (!ok) {
         // drain this CTA's own copies in flight before its shared memory goes away
         for (int s = 0; s < 2; ++s)
-            if (pending[s]) mbar_wait(&full[s], 0, nullptr, 0, 1u << 16), mbar_wait(&full[s], 1, nullptr, 0, 1u << 16);
+            if (pending[s]) {
+                mbar_wait(&full[s], 0, nullptr, 0, 1u << 16);
+                mbar_wait(&full[s], 1, nullptr, 0, 1u << 16);
+            }
     }
     fence_before_sync();
     __syncthreads();
@@ -598,14 +654,22 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     if ((e = cudaFuncSetAttribute(tc::chunk_state_tc_kernel<false>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::S_SMEM)))
         return e;
+    // [tokens][H * d] views of the inputs; rows past the end read as zeros
+    const uint64_t rows = (uint64_t)a.si.T_total, cols = (uint64_t)a.H * tc::D;
+    tc::PrepMaps maps;
+    CUtensorMap vmap;
+    if ((e = make_tensor_map_2d(&maps.k, a.k, true, cols, rows, cols * 2, 64, 64, true))) return e;
+    if ((e = make_tensor_map_2d(&maps.q, a.q, true, cols, rows, cols * 2, 64, 64, true))) return e;
+    if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 128, 64, false))) return e;
+    if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
+
     for (int64_t hb = 0; hb < a.H; hb += Hg) {
         const int64_t hg = (a.H - hb) < Hg ? (a.H - hb) : Hg;
         if (a.si.chunks_upper > 0) {
             dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
             LaunchScope scope(st, K_PREP_TC);
-            tc::chunk_prep_tc_kernel<<<gp, 128, tc::P_SMEM, st>>>(
-                (const __nv_bfloat16*)a.q, (const __nv_bfloat16*)a.k, (const __nv_bfloat16*)a.v,
-                a.log_alpha, a.beta, a.si, a.H, hb, Hg, a.scale, ws, err);
+            tc::chunk_prep_tc_kernel<<<gp, 128, tc::P_SMEM, st>>>(maps, a.beta, a.si, a.H, hb, Hg,
+                                                                 a.scale, ws, err);
             if ((e = cudaGetLastError())) return e;
         }
         dim3 gs((unsigned)a.si.N, (unsigned)hg);
@@ -613,10 +677,10 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
             LaunchScope scope(st, K_STATE_TC);
             if (a.h0)
                 tc::chunk_state_tc_kernel<true><<<gs, 128, tc::S_SMEM, st>>>(
-                    ws, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
+                    ws, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
             else
                 tc::chunk_state_tc_kernel<false><<<gs, 128, tc::S_SMEM, st>>>(
-                    ws, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
+                    ws, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
         }
         if ((e = cudaGetLastError())) return e;
     }
