@@ -102,21 +102,22 @@ __device__ __forceinline__ uint32_t tf32(float x)
 }
 
 // acc (16x16, m16n8 fragments for the two 8-column halves) += X * Y, where X
-// and Y are 16x16 fp32 blocks in shared memory with a row pitch of 64 floats.
+// and Y are 16x16 fp32 blocks in shared memory with a row pitch of P floats.
+template <int P>
 __device__ __forceinline__ void mma16x16x16_tf32(float (&acc)[2][4], const float* X, const float* Y,
                                                  int lane)
 {
     const int g = lane >> 2, q = lane & 3;
 #pragma unroll
     for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t a0 = tf32(X[g * 64 + 8 * ks + q]);
-        const uint32_t a1 = tf32(X[(g + 8) * 64 + 8 * ks + q]);
-        const uint32_t a2 = tf32(X[g * 64 + 8 * ks + q + 4]);
-        const uint32_t a3 = tf32(X[(g + 8) * 64 + 8 * ks + q + 4]);
+        const uint32_t a0 = tf32(X[g * P + 8 * ks + q]);
+        const uint32_t a1 = tf32(X[(g + 8) * P + 8 * ks + q]);
+        const uint32_t a2 = tf32(X[g * P + 8 * ks + q + 4]);
+        const uint32_t a3 = tf32(X[(g + 8) * P + 8 * ks + q + 4]);
 #pragma unroll
         for (int nh = 0; nh < 2; ++nh) {
-            const uint32_t b0 = tf32(Y[(8 * ks + q) * 64 + 8 * nh + g]);
-            const uint32_t b1 = tf32(Y[(8 * ks + q + 4) * 64 + 8 * nh + g]);
+            const uint32_t b0 = tf32(Y[(8 * ks + q) * P + 8 * nh + g]);
+            const uint32_t b1 = tf32(Y[(8 * ks + q + 4) * P + 8 * nh + g]);
             asm volatile(
                 "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
                 "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
@@ -127,40 +128,51 @@ __device__ __forceinline__ void mma16x16x16_tf32(float (&acc)[2][4], const float
 }
 
 // Store a 16x16 accumulator (m16n8 fragments) scaled by `s` into a block with
-// a row pitch of 64 floats.
+// a row pitch of P floats.
+template <int P>
 __device__ __forceinline__ void store16x16(float* Z, const float (&acc)[2][4], float s, int lane)
 {
     const int g = lane >> 2, q = lane & 3;
 #pragma unroll
     for (int nh = 0; nh < 2; ++nh) {
-        Z[g * 64 + 8 * nh + 2 * q] = s * acc[nh][0];
-        Z[g * 64 + 8 * nh + 2 * q + 1] = s * acc[nh][1];
-        Z[(g + 8) * 64 + 8 * nh + 2 * q] = s * acc[nh][2];
-        Z[(g + 8) * 64 + 8 * nh + 2 * q + 1] = s * acc[nh][3];
+        Z[g * P + 8 * nh + 2 * q] = s * acc[nh][0];
+        Z[g * P + 8 * nh + 2 * q + 1] = s * acc[nh][1];
+        Z[(g + 8) * P + 8 * nh + 2 * q] = s * acc[nh][2];
+        Z[(g + 8) * P + 8 * nh + 2 * q + 1] = s * acc[nh][3];
     }
 }
 
 // ---------------------------------------------------------------------------
 // prep kernel shared memory (bytes from a 1024-aligned base)
 // ---------------------------------------------------------------------------
+constexpr int PT = 256;                // threads
+constexpr int AP = 68;                 // row pitch (floats) of the fp32 A and T matrices
 constexpr uint32_t P_K = 0;            // k, MN-major [t][c] image (TMA, swizzled); later K e^G   16 KB
 constexpr uint32_t P_Q = 16384;        // q, same layout (TMA); later the T' bf16 image           16 KB
-constexpr uint32_t P_G = 32768;        // fp32 log_alpha [64][128] (TMA), then G (log2 units)    32 KB
+constexpr uint32_t P_G = 32768;        // fp32 log_alpha -> G: 4 swizzled slabs of 32 channels   32 KB
 constexpr uint32_t P_KQ = 65536;       // K-major B: [Kin_p; Qin_p] x 4, one K-block             16 KB
 constexpr uint32_t P_KV = 81920;       // K-major A: Kvar rows (160), one K-block                20 KB
-constexpr uint32_t P_A = 65536;        // fp32 A [64][64] (aliases KQ after the strips)          16 KB
-constexpr uint32_t P_T = 81920;        // fp32 T [64][64] (aliases KV)                           16 KB
+constexpr uint32_t P_A = 65536;        // fp32 A [64][68] (aliases KQ/KV after the strips)       17 KB
+constexpr uint32_t P_T = P_A + 64 * AP * 4;   // fp32 T [64][68]                                 17 KB
 constexpr uint32_t P_VEC = 102400;     // per-channel vectors: egf[4], eglf[4], dvec[6]          7 KB
 constexpr uint32_t P_BETA = P_VEC + 14 * 512;
 constexpr uint32_t P_BYTES = P_BETA + 256;
 constexpr uint32_t P_SMEM = P_BYTES + 1024 + 64;
 constexpr uint32_t P_TX = 16384 + 16384 + 32768;   // bytes the input TMA loads deliver
+static_assert(P_T + 64 * AP * 4 <= P_VEC, "A/T overlap the vectors");
+
+// Byte offset of G[t][c] in the four 128B-swizzled slabs of 32 fp32 channels.
+__device__ __forceinline__ uint32_t g_off(int t, int c)
+{
+    return (uint32_t)(c >> 5) * 8192u + (uint32_t)t * 128u +
+           ((uint32_t)(((c & 31) >> 2) ^ (t & 7)) << 4) + (uint32_t)(c & 3) * 4u;
+}
 
 struct PrepMaps {
     CUtensorMap k, q, g;
 };
 
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(PT, 2)
 chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
                      SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
                      unsigned char* __restrict__ ws, int* __restrict__ err)
@@ -177,13 +189,15 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     int64_t n, t0, len;
     if (!si.locate(gc, n, t0, len)) return;
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int sp = w & 3;                          // TMEM lane quarter of this warp
     unsigned char* img = ws + (gc * Hg + hl) * (int64_t)IMG_BYTES;
 
-    float* sG = reinterpret_cast<float*>(sm + P_G);
+    unsigned char* sGb = sm + P_G;
     float* egf = reinterpret_cast<float*>(sm + P_VEC);           // [4][128]  e^{G_f}
     float* eglf = egf + 4 * D;                                    // [4][128]  e^{G_last - G_f}
     float* dvec = eglf + 4 * D;                                   // [6][128]  e^{G_fp - G_fr}
     float* sB = reinterpret_cast<float*>(sm + P_BETA);
+    auto G = [&](int t, int c) -> float& { return *reinterpret_cast<float*>(sGb + g_off(t, c)); };
 
     if (tid == 0) {
         mbar_init(&bar_in, 1);
@@ -195,7 +209,8 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_in);
         tma::load_2d(sm + P_Q, &maps.q, x, y, &bar_in);
         tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_in);
-        tma::load_2d(sm + P_G, &maps.g, x, y, &bar_in);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
     }
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
     if (tid < C) sB[tid] = tid < len ? beta[(t0 + tid) * H + h] : 0.f;
@@ -206,42 +221,68 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     bool ok = __syncthreads_and(mbar_wait(&bar_in, 0, err, 1) ? 1 : 0);
 
     if (ok) {
-        // ---- (a) cumulative log-decay per channel (log2 units); rows >= len add nothing
+        // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
+        // Threads c and c + 128 scan tokens 0..31 and 32..63; the second half then
+        // adds the first half's total.
         {
-            const int c = tid;
+            const int c = tid & 127, part = tid >> 7, tb = 32 * part;
             float run = 0.f;
-            for (int t = 0; t < C; ++t) {
-                if (t < len) run += kLog2e * sG[t * D + c];
-                sG[t * D + c] = run;
+#pragma unroll 8
+            for (int x = 0; x < 32; ++x) {
+                const int t = tb + x;
+                float& gv = G(t, c);
+                run += (t < len) ? kLog2e * gv : 0.f;
+                gv = run;
             }
-            const float Gl = run;
-            float Gf[4];
-#pragma unroll
-            for (int p = 0; p < 4; ++p) {
-                Gf[p] = sG[(16 * p) * D + c];
-                egf[p * D + c] = ex2(Gf[p]);
-                eglf[p * D + c] = ex2(Gl - Gf[p]);
+            __syncthreads();
+            if (part == 1) {
+                const float base = G(31, c);
+#pragma unroll 8
+                for (int x = 0; x < 32; ++x) G(32 + x, c) += base;
             }
-            int idx = 0;
+            __syncthreads();
+            if (part == 0) {
+                const float Gl = G(63, c);
+                float Gf[4];
 #pragma unroll
-            for (int p = 1; p < 4; ++p)
+                for (int p = 0; p < 4; ++p) {
+                    Gf[p] = G(16 * p, c);
+                    egf[p * D + c] = ex2(Gf[p]);
+                    eglf[p * D + c] = ex2(Gl - Gf[p]);
+                }
+                int idx = 0;
 #pragma unroll
-                for (int r = 0; r < p; ++r) dvec[(idx++) * D + c] = ex2(Gf[p] - Gf[r]);
-            reinterpret_cast<float*>(img + IMG_GAM)[c] = ex2(Gl);
+                for (int p = 1; p < 4; ++p)
+#pragma unroll
+                    for (int r = 0; r < p; ++r) dvec[(idx++) * D + c] = ex2(Gf[p] - Gf[r]);
+                reinterpret_cast<float*>(img + IMG_GAM)[c] = ex2(Gl);
+            }
         }
         __syncthreads();
 
         // ---- (b1) A / Aqk strips: operands built per channel half, MMAs accumulate
-        const int ch8 = tid & 7, tr = tid >> 3;
+        const int ch8 = tid & 7, tr = (tid >> 3) & 15, pg = tid >> 7;
         for (int hh = 0; hh < 2 && ok; ++hh) {
             const int c0 = 64 * hh + 8 * ch8;
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
+            for (int pp = 0; pp < 2; ++pp) {
+                const int p = 2 * pg + pp;
                 const int t = 16 * p + tr;
                 const bool live = t < len;
                 float G8[8], Gf8[8], kk[8], qq[8];
-                ld8f(sG + t * D + c0, G8);
-                ld8f(sG + (16 * p) * D + c0, Gf8);
+                {
+                    const unsigned char* slab = sGb + (c0 >> 5) * 8192;
+                    const int q0 = (c0 & 31) >> 2;
+                    const float4 a = *reinterpret_cast<const float4*>(slab + t * 128 + ((q0 ^ (t & 7)) << 4));
+                    const float4 b = *reinterpret_cast<const float4*>(slab + t * 128 + (((q0 + 1) ^ (t & 7)) << 4));
+                    const int tf = 16 * p;
+                    const float4 fa = *reinterpret_cast<const float4*>(slab + tf * 128 + ((q0 ^ (tf & 7)) << 4));
+                    const float4 fb = *reinterpret_cast<const float4*>(slab + tf * 128 + (((q0 + 1) ^ (tf & 7)) << 4));
+                    G8[0] = a.x; G8[1] = a.y; G8[2] = a.z; G8[3] = a.w;
+                    G8[4] = b.x; G8[5] = b.y; G8[6] = b.z; G8[7] = b.w;
+                    Gf8[0] = fa.x; Gf8[1] = fa.y; Gf8[2] = fa.z; Gf8[3] = fa.w;
+                    Gf8[4] = fb.x; Gf8[5] = fb.y; Gf8[6] = fb.z; Gf8[7] = fb.w;
+                }
                 const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
                 unpack8(*reinterpret_cast<const uint4*>(sm + P_K + off), kk);
                 unpack8(*reinterpret_cast<const uint4*>(sm + P_Q + off), qq);
@@ -260,11 +301,14 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + 16 + tr, 8 * ch8)) = pack8(qin);
                 *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[p] + t, 8 * ch8)) = pack8(kd);
 #pragma unroll
-                for (int pp = p + 1; pp < 4; ++pp) {
-                    const float* dv8 = dvec + ((pp * (pp - 1)) / 2 + p) * D + c0;
+                for (int q2 = 1; q2 < 4; ++q2) {
+                    const int pv = p + q2;
+                    if (pv < 4) {
+                        const float* dv8 = dvec + ((pv * (pv - 1)) / 2 + p) * D + c0;
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * dv8[j];
-                    *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pp] + t, 8 * ch8)) = pack8(tmp);
+                        for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * dv8[j];
+                        *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pv] + t, 8 * ch8)) = pack8(tmp);
+                    }
                 }
                 const float* eg = egf + p * D + c0;
                 const float* egl = eglf + p * D + c0;
@@ -303,24 +347,27 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     float* sA = reinterpret_cast<float*>(sm + P_A);
     float* sT = reinterpret_cast<float*>(sm + P_T);
     if (ok) {
-        // ---- extract A (fp32, for the inverse) and Aqk^T (bf16 image rows)
-        const int j = 16 * w + l;
-        float kp[4][16], qp[4][16];
+        // ---- extract A (fp32, for the inverse) and Aqk^T (bf16 image rows);
+        // warps w and w + 4 share a TMEM lane quarter and take two strips each
+        const int j = 16 * sp + l;
+        float kp[2][16], qp[2][16];
 #pragma unroll
-        for (int p = 0; p < 4; ++p) {
-            tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 32 * p, kp[p]);
-            tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 32 * p + 16, qp[p]);
+        for (int x = 0; x < 2; ++x) {
+            const int p = 2 * (w >> 2) + x;
+            tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p, kp[x]);
+            tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p + 16, qp[x]);
         }
         tmem_wait_ld();
         if (l < 16) {
 #pragma unroll
-            for (int p = 0; p < 4; ++p) {
+            for (int x = 0; x < 2; ++x) {
+                const int p = 2 * (w >> 2) + x;
                 float aq[16];
 #pragma unroll
                 for (int cc = 0; cc < 16; ++cc) {
                     const int i = 16 * p + cc;
-                    sA[i * C + j] = (j < i) ? sB[i] * kp[p][cc] : 0.f;
-                    aq[cc] = (j <= i) ? qp[p][cc] : 0.f;
+                    sA[i * AP + j] = (j < i) ? sB[i] * kp[x][cc] : 0.f;
+                    aq[cc] = (j <= i) ? qp[x][cc] : 0.f;
                 }
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p + 8)) = pack8(aq + 8);
@@ -329,18 +376,20 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         fence_before_sync();
         __syncthreads();
 
-        // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution
+        // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution,
+        // one column per thread, held in registers
         if (tid < C) {
             const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+            float tcol[16];
+#pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float val = (r == cc) ? 1.f : 0.f;
-                if (r > cc) {
-                    float acc = 0.f;
-                    for (int m = cc; m < r; ++m) acc += sA[(o + r) * C + o + m] * sT[(o + m) * C + o + cc];
-                    val = -acc;
-                }
-                sT[(o + r) * C + o + cc] = val;
+                float acc = 0.f;
+#pragma unroll
+                for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
+                tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -acc);
             }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
         }
         __syncthreads();
         // off-diagonal blocks by distance d (one warp per block):
@@ -351,20 +400,20 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             if (p < 4) {
                 float acc[2][4] = {};
                 for (int m = r; m < p; ++m)
-                    mma16x16x16_tf32(acc, sA + (16 * p) * C + 16 * m, sT + (16 * m) * C + 16 * r, l);
-                store16x16(sA + (16 * r) * C + 16 * p, acc, 1.f, l);
+                    mma16x16x16_tf32<AP>(acc, sA + (16 * p) * AP + 16 * m, sT + (16 * m) * AP + 16 * r, l);
+                store16x16<AP>(sA + (16 * r) * AP + 16 * p, acc, 1.f, l);
                 __syncwarp();
                 float acc2[2][4] = {};
-                mma16x16x16_tf32(acc2, sT + (16 * p) * C + 16 * p, sA + (16 * r) * C + 16 * p, l);
-                store16x16(sT + (16 * p) * C + 16 * r, acc2, -1.f, l);
+                mma16x16x16_tf32<AP>(acc2, sT + (16 * p) * AP + 16 * p, sA + (16 * r) * AP + 16 * p, l);
+                store16x16<AP>(sT + (16 * p) * AP + 16 * r, acc2, -1.f, l);
             }
             __syncthreads();
         }
         // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
-        for (int e = tid; e < C * 8; e += 128) {
+        for (int e = tid; e < C * 8; e += PT) {
             const int i = e >> 3, cb = e & 7;
             float f[8];
-            ld8f(sT + i * C + 8 * cb, f);
+            ld8f(sT + i * AP + 8 * cb, f);
 #pragma unroll
             for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * sB[8 * cb + x] : 0.f;
             const uint4 u = pack8(f);
@@ -390,23 +439,20 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         ok = __syncthreads_and(mbar_wait(&bar, 0, err, 3) ? 1 : 0);
         fence_after_sync();
         if (ok) {
-            const int i = 16 * w + l;
+            const int i = 16 * sp + l, half = w >> 2;
+            float f[4][16];
 #pragma unroll
-            for (int half = 0; half < 2; ++half) {
-                float f[4][16];
+            for (int cb = 0; cb < 4; ++cb)
+                tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 64 * half + 16 * cb, f[cb]);
+            tmem_wait_ld();
+            if (l < 16) {
+                unsigned char* dst = img + IMG_W + half * 8192;
 #pragma unroll
-                for (int cb = 0; cb < 4; ++cb)
-                    tmem_ld16(tmem + ((uint32_t)(32 * w) << 16) + 64 * half + 16 * cb, f[cb]);
-                tmem_wait_ld();
-                if (l < 16) {
-                    unsigned char* dst = img + IMG_W + half * 8192;
+                for (int cb = 0; cb < 4; ++cb) {
 #pragma unroll
-                    for (int cb = 0; cb < 4; ++cb) {
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) f[cb][x] = -f[cb][x];
-                        *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
-                        *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
-                    }
+                    for (int x = 0; x < 16; ++x) f[cb][x] = -f[cb][x];
+                    *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
+                    *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
                 }
             }
         }
@@ -660,7 +706,7 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     CUtensorMap vmap;
     if ((e = make_tensor_map_2d(&maps.k, a.k, true, cols, rows, cols * 2, 64, 64, true))) return e;
     if ((e = make_tensor_map_2d(&maps.q, a.q, true, cols, rows, cols * 2, 64, 64, true))) return e;
-    if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 128, 64, false))) return e;
+    if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 32, 64, true))) return e;
     if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
 
     for (int64_t hb = 0; hb < a.H; hb += Hg) {
@@ -668,7 +714,7 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         if (a.si.chunks_upper > 0) {
             dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
             LaunchScope scope(st, K_PREP_TC);
-            tc::chunk_prep_tc_kernel<<<gp, 128, tc::P_SMEM, st>>>(maps, a.beta, a.si, a.H, hb, Hg,
+            tc::chunk_prep_tc_kernel<<<gp, tc::PT, tc::P_SMEM, st>>>(maps, a.beta, a.si, a.H, hb, Hg,
                                                                  a.scale, ws, err);
             if ((e = cudaGetLastError())) return e;
         }
