@@ -222,31 +222,39 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
 
     if (ok) {
         // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
-        // Threads c and c + 128 scan tokens 0..31 and 32..63; the second half then
-        // adds the first half's total.
+        // Threads c and c + 128 scan tokens 0..31 and 32..63 in registers; the second
+        // half then adds the first half's total and derives the per-channel vectors.
         {
             const int c = tid & 127, part = tid >> 7, tb = 32 * part;
+            const unsigned char* slab = sGb + (c >> 5) * 8192 + (c & 3) * 4;
+            const int q0 = (c & 31) >> 2;
+            float v[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+                v[x] = *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
             float run = 0.f;
-#pragma unroll 8
+#pragma unroll
             for (int x = 0; x < 32; ++x) {
-                const int t = tb + x;
-                float& gv = G(t, c);
-                run += (t < len) ? kLog2e * gv : 0.f;
-                gv = run;
+                run += (tb + x < len) ? kLog2e * v[x] : 0.f;
+                v[x] = run;
+            }
+            if (part == 0) {
+#pragma unroll
+                for (int x = 0; x < 32; ++x)
+                    *reinterpret_cast<float*>(const_cast<unsigned char*>(slab) + x * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
             }
             __syncthreads();
             if (part == 1) {
                 const float base = G(31, c);
-#pragma unroll 8
-                for (int x = 0; x < 32; ++x) G(32 + x, c) += base;
-            }
-            __syncthreads();
-            if (part == 0) {
-                const float Gl = G(63, c);
-                float Gf[4];
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    v[x] += base;
+                    *reinterpret_cast<float*>(const_cast<unsigned char*>(slab) + (32 + x) * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
+                }
+                const float Gl = v[31];
+                const float Gf[4] = {G(0, c), G(16, c), v[0], v[16]};
 #pragma unroll
                 for (int p = 0; p < 4; ++p) {
-                    Gf[p] = G(16 * p, c);
                     egf[p * D + c] = ex2(Gf[p]);
                     eglf[p * D + c] = ex2(Gl - Gf[p]);
                 }
@@ -304,14 +312,16 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 for (int q2 = 1; q2 < 4; ++q2) {
                     const int pv = p + q2;
                     if (pv < 4) {
-                        const float* dv8 = dvec + ((pv * (pv - 1)) / 2 + p) * D + c0;
+                        float dv8[8];
+                        ld8f(dvec + ((pv * (pv - 1)) / 2 + p) * D + c0, dv8);
 #pragma unroll
                         for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * dv8[j];
                         *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pv] + t, 8 * ch8)) = pack8(tmp);
                     }
                 }
-                const float* eg = egf + p * D + c0;
-                const float* egl = eglf + p * D + c0;
+                float eg[8], egl[8];
+                ld8f(egf + p * D + c0, eg);
+                ld8f(eglf + p * D + c0, egl);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) tmp[j] = qin[j] * eg[j];
                 *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
@@ -392,20 +402,36 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
         }
         __syncthreads();
-        // off-diagonal blocks by distance d (one warp per block):
-        //   X_pr = sum_{r<=m<p} A_pm T_mr  (parked in the unused upper block (r, p) of A),
-        //   T_pr = -T_pp X_pr
-        for (int d = 1; d < 4; ++d) {
-            const int r = w, p = w + d;
-            if (p < 4) {
+        // off-diagonal blocks, 32 x 32 recursion (X blocks are parked in the unused
+        // upper blocks of A):
+        //   level 1 (warps 0, 1): T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
+        //   level 2: X = A_21 T_1 (rows 2..3, cols 0..1), then T_21 = -T_2 X
+        {
+            auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
+            auto Tb = [&](int r, int c) { return sT + (16 * r) * AP + 16 * c; };
+            if (w < 2) {
+                const int p = 2 * w + 1, r = 2 * w;
                 float acc[2][4] = {};
-                for (int m = r; m < p; ++m)
-                    mma16x16x16_tf32<AP>(acc, sA + (16 * p) * AP + 16 * m, sT + (16 * m) * AP + 16 * r, l);
-                store16x16<AP>(sA + (16 * r) * AP + 16 * p, acc, 1.f, l);
+                mma16x16x16_tf32<AP>(acc, Ab(p, r), Tb(r, r), l);
+                store16x16<AP>(Ab(r, p), acc, 1.f, l);
                 __syncwarp();
                 float acc2[2][4] = {};
-                mma16x16x16_tf32<AP>(acc2, sT + (16 * p) * AP + 16 * p, sA + (16 * r) * AP + 16 * p, l);
-                store16x16<AP>(sT + (16 * p) * AP + 16 * r, acc2, -1.f, l);
+                mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
+                store16x16<AP>(Tb(p, r), acc2, -1.f, l);
+            }
+            __syncthreads();
+            if (w < 4) {
+                const int p = 2 + (w >> 1), r = w & 1;       // X_pr = sum_{m=r..1} A_pm T_mr
+                float acc[2][4] = {};
+                for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
+                store16x16<AP>(Ab(r, p), acc, 1.f, l);
+            }
+            __syncthreads();
+            if (w < 4) {
+                const int p = 2 + (w >> 1), r = w & 1;       // T_pr = -sum_{m=2..p} T_pm X_mr
+                float acc[2][4] = {};
+                for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
+                store16x16<AP>(Tb(p, r), acc, -1.f, l);
             }
             __syncthreads();
         }
@@ -475,8 +501,10 @@ constexpr uint32_t S_UBF = S_SBF + 32768;                // U^T bf16, K-major A:
 constexpr uint32_t S_BYTES = S_UBF + 16384;
 constexpr uint32_t S_SMEM = S_BYTES + 1024;
 
+constexpr int ST = 256;                                 // state-kernel threads
+
 template <bool kHasH0>
-__global__ void __launch_bounds__(128, 1)
+__global__ void __launch_bounds__(ST, 1)
 chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constant__ CUtensorMap vmap,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, SeqInfo si, int64_t H, int64_t h_base, int64_t Hg,
@@ -491,8 +519,9 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     const int64_t n = blockIdx.x;
     const int hl = blockIdx.y;
     const int64_t h = h_base + hl;
-    const int tid = threadIdx.x, w = tid >> 5;
-    const int j = tid;                                  // dv index = TMEM lane
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int sp = w & 3, half = w >> 2;                // TMEM lane quarter, column half
+    const int j = 32 * sp + l;                          // dv index = TMEM lane
     int64_t bos, eos;
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
     const int64_t nch = si.chunk_count(n, eos - bos);
@@ -502,7 +531,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 
     if (nch == 0) {                                      // empty sequence: hT = h0
         if (hTp)
-            for (int c = 0; c < D; ++c) hTp[c * D + j] = kHasH0 ? h0p[c * D + j] : 0.f;
+            for (int c = 64 * half; c < 64 * half + 64; ++c)
+                hTp[c * D + j] = kHasH0 ? h0p[c * D + j] : 0.f;
         return;
     }
     auto load_stage = [&](int64_t ch, int s) {          // one thread
@@ -522,38 +552,62 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         load_stage(0, 0);
         if (nch > 1) load_stage(1, 1);
     }
-    if (w == 0) { tmem_alloc(&tmem_base, 256); tmem_relinquish(); }
+    if (w == 0) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
-    const uint32_t lane = (uint32_t)(32 * w) << 16;
-    const uint32_t tU = tmem, tO = tmem + 64, tS = tmem + 128;
+    const uint32_t lane = (uint32_t)(32 * sp) << 16;
+    const uint32_t tU = tmem, tS = tmem + 256;
+    auto tO = [&](int64_t ch) { return tmem + 64 + 64 * (uint32_t)(ch & 1); };
     bool pending[2] = {true, nch > 1};
+
+    // U^T = V^T T'^T + S^T (-W)^T and O^T = S^T (scale Q e^G)^T for chunk ch (one thread)
+    auto issue_mma1 = [&](int64_t ch) {
+        unsigned char* st = sm + (ch & 1) * STAGE_BYTES;
+        fence_after_sync();
+        const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks)
+            mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
+                     make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
+        const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
+        const uint32_t to = tO(ch);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
+            mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, 1u);
+            mma_bf16(to, ad, make_desc(smem_u32(st + IMG_QG + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, ks > 0);
+        }
+        commit(&bar1);
+    };
 
     bool ok = __syncthreads_and(mbar_wait(&full[0], 0, err, 4) ? 1 : 0);
     if (ok) pending[0] = false;
 
-    // initial state: bf16 copy (operand) and gamma_0-scaled fp32 in TMEM
+    // initial state: bf16 copy (operand) and gamma_0-scaled fp32 in TMEM; this
+    // thread owns columns 64*half .. +63 of row j of S^T
     if (ok) {
         const float* gam = reinterpret_cast<const float*>(sm + IMG_GAM);
+        unsigned char* dst = sm + S_SBF + half * 16384;
 #pragma unroll 1
-        for (int cb = 0; cb < 8; ++cb) {
+        for (int cb = 0; cb < 4; ++cb) {
+            const int c0 = 64 * half + 16 * cb;
             float f[16];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) f[x] = kHasH0 ? h0p[(16 * cb + x) * D + j] : 0.f;
-            unsigned char* dst = sm + S_SBF + (cb >> 2) * 16384;
-            *reinterpret_cast<uint4*>(dst + sw128_offset(j, (16 * cb) & 63)) = pack8(f);
-            *reinterpret_cast<uint4*>(dst + sw128_offset(j, ((16 * cb) & 63) + 8)) = pack8(f + 8);
+            for (int x = 0; x < 16; ++x) f[x] = kHasH0 ? h0p[(c0 + x) * D + j] : 0.f;
+            *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f);
+            *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f + 8);
 #pragma unroll
-            for (int x = 0; x < 16; ++x) f[x] *= gam[16 * cb + x];
-            tmem_st16(tS + lane + 16 * cb, f);
+            for (int x = 0; x < 16; ++x) f[x] *= gam[c0 + x];
+            tmem_st16(tS + lane + c0, f);
         }
         tmem_wait_st();
     }
     fence_smem_to_async();
     fence_before_sync();
     __syncthreads();
+    if (ok && tid == 0) issue_mma1(0);
 
     for (int64_t ch = 0; ok && ch < nch; ++ch) {
         const int s = (int)(ch & 1);
@@ -561,39 +615,23 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         const int64_t t0 = bos + ch * C;
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
         const uint32_t ph = (uint32_t)(ch & 1);
+        const bool last = (ch + 1 == nch);
 
-        if (tid == 0) {
-            fence_after_sync();
-            // U^T = V^T T'^T  (M = dv, N = 64, K = 64)
-            const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
-                         make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
-            // U^T += S^T (-W)^T ; O^T = S^T (scale Q e^G)^T   (M = dv, N = 64, K = dk)
-            const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
-#pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
-                mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, 1u);
-                mma_bf16(tO, ad, make_desc(smem_u32(st + IMG_QG + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, ks > 0);
-            }
-            commit(&bar1);
-        }
         ok = __syncthreads_and(mbar_wait(&bar1, ph, err, 5) ? 1 : 0);
         fence_after_sync();
         if (!ok) break;
 
-        // U^T (fp32, TMEM) -> bf16 operand rows
+        // U^T (fp32, TMEM) -> bf16 operand rows; this thread: tokens 32*half .. +31
         {
-            float f[4][16];
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tU + lane + 16 * cb, f[cb]);
+            float f[2][16];
+            tmem_ld16(tU + lane + 32 * half, f[0]);
+            tmem_ld16(tU + lane + 32 * half + 16, f[1]);
             tmem_wait_ld();
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, 16 * cb)) = pack8(f[cb]);
-                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, 16 * cb + 8)) = pack8(f[cb] + 8);
+            for (int x = 0; x < 2; ++x) {
+                const int c = 32 * half + 16 * x;
+                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, c)) = pack8(f[x]);
+                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, c + 8)) = pack8(f[x] + 8);
             }
         }
         fence_smem_to_async();
@@ -601,12 +639,15 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         __syncthreads();
         if (tid == 0) {
             fence_after_sync();
-            // [O^T | S^T] += U^T [Aqk^T | K e^{Gl - G}]   (M = dv, N = 192, K = 64)
-            const uint32_t id2 = make_idesc_bf16(128, 192, false, true);
+            // O^T += U^T Aqk^T (N = 64) ; S^T += U^T (K e^{Gl - G}) (N = 128)
+            const uint32_t idO = make_idesc_bf16(128, 64, false, true);
+            const uint32_t idS = make_idesc_bf16(128, 128, false, true);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tO, make_desc(smem_u32(sm + S_UBF + ks * 32), 16, 1024),
-                         make_desc(smem_u32(st + IMG_B2 + ks * 2048), 8192, 1024), id2, 1u);
+            for (int ks = 0; ks < 4; ++ks) {
+                const uint64_t ad = make_desc(smem_u32(sm + S_UBF + ks * 32), 16, 1024);
+                mma_bf16(tO(ch), ad, make_desc(smem_u32(st + IMG_B2 + ks * 2048), 8192, 1024), idO, 1u);
+                mma_bf16(tS, ad, make_desc(smem_u32(st + IMG_B2 + 8192 + ks * 2048), 8192, 1024), idS, 1u);
+            }
             commit(&bar2);
         }
         ok = __syncthreads_and(mbar_wait(&bar2, ph, err, 5) ? 1 : 0);
@@ -618,7 +659,6 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             if (tid == 0) load_stage(ch + 2, s);
             pending[s] = true;
         }
-        const bool last = (ch + 1 == nch);
         const float* gam_next = nullptr;
         if (!last) {
             ok = __syncthreads_and(mbar_wait(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 4) ? 1 : 0);
@@ -627,22 +667,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             gam_next = reinterpret_cast<const float*>(sm + (s ^ 1) * STAGE_BYTES + IMG_GAM);
         }
 
-        // output rows of this chunk
-        {
-            float f[4][16];
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tO + lane + 16 * cb, f[cb]);
-            tmem_wait_ld();
-            __nv_bfloat16* op = out + (t0 * H + h) * D + j;
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb)
-#pragma unroll
-                for (int x = 0; x < 16; ++x)
-                    if (16 * cb + x < len) op[(int64_t)(16 * cb + x) * H * D] = __float2bfloat16_rn(f[cb][x]);
-        }
         // next entry state: bf16 operand copy, then scaled by the next chunk's decay
-#pragma unroll 1
-        for (int half = 0; half < 2; ++half) {
+        {
             float f[4][16];
 #pragma unroll
             for (int cb = 0; cb < 4; ++cb) tmem_ld16(tS + lane + 64 * half + 16 * cb, f[cb]);
@@ -659,16 +685,37 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
                 for (int cb = 0; cb < 4; ++cb) {
                     *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f[cb]);
                     *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f[cb] + 8);
+                    float g8[16];
+                    ld8f(gam_next + 64 * half + 16 * cb, g8);
+                    ld8f(gam_next + 64 * half + 16 * cb + 8, g8 + 8);
 #pragma unroll
-                    for (int x = 0; x < 16; ++x) f[cb][x] *= gam_next[64 * half + 16 * cb + x];
+                    for (int x = 0; x < 16; ++x) f[cb][x] *= g8[x];
                     tmem_st16(tS + lane + 64 * half + 16 * cb, f[cb]);
                 }
+                tmem_wait_st();
             }
         }
-        tmem_wait_st();
         fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
+        if (!last && tid == 0) issue_mma1(ch + 1);     // overlaps the output write below
+
+        // output rows of this chunk: tokens 32*half .. +31 of column j
+        {
+            float f[2][16];
+            tmem_ld16(tO(ch) + lane + 32 * half, f[0]);
+            tmem_ld16(tO(ch) + lane + 32 * half + 16, f[1]);
+            tmem_wait_ld();
+            __nv_bfloat16* op = out + (t0 * H + h) * D + j;
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int y = 0; y < 16; ++y) {
+                    const int t = 32 * half + 16 * x + y;
+                    if (t < len) op[(int64_t)t * H * D] = __float2bfloat16_rn(f[x][y]);
+                }
+        }
+        fence_before_sync();
     }
     if (!ok) {
         // drain this CTA's own copies in flight before its shared memory goes away
@@ -680,7 +727,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     }
     fence_before_sync();
     __syncthreads();
-    if (w == 0) tmem_dealloc(tmem, 256);
+    if (w == 0) tmem_dealloc(tmem, 512);
 }
 
 }  // namespace tc
@@ -722,10 +769,10 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         {
             LaunchScope scope(st, K_STATE_TC);
             if (a.h0)
-                tc::chunk_state_tc_kernel<true><<<gs, 128, tc::S_SMEM, st>>>(
+                tc::chunk_state_tc_kernel<true><<<gs, tc::ST, tc::S_SMEM, st>>>(
                     ws, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
             else
-                tc::chunk_state_tc_kernel<false><<<gs, 128, tc::S_SMEM, st>>>(
+                tc::chunk_state_tc_kernel<false><<<gs, tc::ST, tc::S_SMEM, st>>>(
                     ws, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
         }
         if ((e = cudaGetLastError())) return e;
