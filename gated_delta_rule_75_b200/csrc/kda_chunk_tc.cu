@@ -218,7 +218,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
-    bool ok = __syncthreads_and(mbar_wait(&bar_in, 0, err, 1) ? 1 : 0);
+    bool ok = block_wait(&bar_in, 0, err, 1);
 
     if (ok) {
         // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
@@ -268,70 +268,65 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         }
         __syncthreads();
 
-        // ---- (b1) A / Aqk strips: operands built per channel half, MMAs accumulate
-        const int ch8 = tid & 7, tr = (tid >> 3) & 15, pg = tid >> 7;
+        // ---- (b1) A / Aqk strips: operands built per channel half, MMAs accumulate.
+        // Thread (ch8, tr, p) handles rows 16p + tr and 16p + tr + 8 of channels
+        // c0 .. c0 + 7, so the sub-chunk's reference values are loaded once.
+        const int ch8 = tid & 7, tr = (tid >> 3) & 7, p = tid >> 6;
         for (int hh = 0; hh < 2 && ok; ++hh) {
             const int c0 = 64 * hh + 8 * ch8;
+            const unsigned char* slab = sGb + (c0 >> 5) * 8192;
+            const int q0 = (c0 & 31) >> 2;
+            float Gf8[8], eg[8], egl[8];
+            {
+                const int tf = 16 * p;
+                const float4 fa = *reinterpret_cast<const float4*>(slab + tf * 128 + (q0 << 4));
+                const float4 fb = *reinterpret_cast<const float4*>(slab + tf * 128 + ((q0 + 1) << 4));
+                Gf8[0] = fa.x; Gf8[1] = fa.y; Gf8[2] = fa.z; Gf8[3] = fa.w;
+                Gf8[4] = fb.x; Gf8[5] = fb.y; Gf8[6] = fb.z; Gf8[7] = fb.w;
+            }
+            ld8f(egf + p * D + c0, eg);
+            ld8f(eglf + p * D + c0, egl);
+            float kin[2][8], qin[2][8], kd[2][8];
 #pragma unroll
-            for (int pp = 0; pp < 2; ++pp) {
-                const int p = 2 * pg + pp;
-                const int t = 16 * p + tr;
+            for (int rr = 0; rr < 2; ++rr) {
+                const int t = 16 * p + tr + 8 * rr;
                 const bool live = t < len;
-                float G8[8], Gf8[8], kk[8], qq[8];
+                float G8[8], kk[8], qq[8];
                 {
-                    const unsigned char* slab = sGb + (c0 >> 5) * 8192;
-                    const int q0 = (c0 & 31) >> 2;
                     const float4 a = *reinterpret_cast<const float4*>(slab + t * 128 + ((q0 ^ (t & 7)) << 4));
                     const float4 b = *reinterpret_cast<const float4*>(slab + t * 128 + (((q0 + 1) ^ (t & 7)) << 4));
-                    const int tf = 16 * p;
-                    const float4 fa = *reinterpret_cast<const float4*>(slab + tf * 128 + ((q0 ^ (tf & 7)) << 4));
-                    const float4 fb = *reinterpret_cast<const float4*>(slab + tf * 128 + (((q0 + 1) ^ (tf & 7)) << 4));
                     G8[0] = a.x; G8[1] = a.y; G8[2] = a.z; G8[3] = a.w;
                     G8[4] = b.x; G8[5] = b.y; G8[6] = b.z; G8[7] = b.w;
-                    Gf8[0] = fa.x; Gf8[1] = fa.y; Gf8[2] = fa.z; Gf8[3] = fa.w;
-                    Gf8[4] = fb.x; Gf8[5] = fb.y; Gf8[6] = fb.z; Gf8[7] = fb.w;
                 }
                 const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
                 unpack8(*reinterpret_cast<const uint4*>(sm + P_K + off), kk);
                 unpack8(*reinterpret_cast<const uint4*>(sm + P_Q + off), qq);
-                float kin[8], qin[8], kd[8], tmp[8];
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
                     const float x = G8[j] - Gf8[j];
                     const float e1 = ex2(x);          // <= 1
                     const float r1 = ex2(-x);         // >= 1, at most 15 tokens of decay
                     const float kv = live ? kk[j] : 0.f;
-                    kin[j] = kv * e1;
-                    qin[j] = live ? scale * qq[j] * e1 : 0.f;
-                    kd[j] = kv * r1;
+                    kin[rr][j] = kv * e1;
+                    qin[rr][j] = live ? scale * qq[j] * e1 : 0.f;
+                    kd[rr][j] = kv * r1;
                 }
-                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + tr, 8 * ch8)) = pack8(kin);
-                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + 16 + tr, 8 * ch8)) = pack8(qin);
-                *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[p] + t, 8 * ch8)) = pack8(kd);
+                // operands of the strip MMAs first
+                const int ts = tr + 8 * rr;          // row within the sub-chunk
+                float tmp[8];
+                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + ts, 8 * ch8)) = pack8(kin[rr]);
+                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + 16 + ts, 8 * ch8)) = pack8(qin[rr]);
+                *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[p] + t, 8 * ch8)) = pack8(kd[rr]);
 #pragma unroll
-                for (int q2 = 1; q2 < 4; ++q2) {
-                    const int pv = p + q2;
-                    if (pv < 4) {
+                for (int pv = 1; pv < 4; ++pv) {
+                    if (pv > p) {
                         float dv8[8];
                         ld8f(dvec + ((pv * (pv - 1)) / 2 + p) * D + c0, dv8);
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * dv8[j];
+                        for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * dv8[j];
                         *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pv] + t, 8 * ch8)) = pack8(tmp);
                     }
                 }
-                float eg[8], egl[8];
-                ld8f(egf + p * D + c0, eg);
-                ld8f(eglf + p * D + c0, egl);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = qin[j] * eg[j];
-                *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = kd[j] * egl[j];
-                *reinterpret_cast<uint4*>(img + IMG_B2 + (1 + hh) * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
-                // K e^G replaces k in place (B operand of W = T' (K e^G))
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = kin[j] * eg[j];
-                *reinterpret_cast<uint4*>(sm + P_K + off) = pack8(tmp);
             }
             fence_smem_to_async();
             fence_before_sync();
@@ -340,16 +335,32 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 fence_after_sync();
                 const uint32_t idesc = make_idesc_bf16(64, 32, false, false);
 #pragma unroll
-                for (int p = 0; p < 4; ++p)
+                for (int pp = 0; pp < 4; ++pp)
 #pragma unroll
                     for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = make_desc(smem_u32(sm + P_KV + kVoff[p] * 128 + ks * 32), 16, 1024);
-                        const uint64_t bd = make_desc(smem_u32(sm + P_KQ + 32 * p * 128 + ks * 32), 16, 1024);
-                        mma_bf16(tmem + 32 * p, ad, bd, idesc, (hh > 0 || ks > 0) ? 1u : 0u);
+                        const uint64_t ad = make_desc(smem_u32(sm + P_KV + kVoff[pp] * 128 + ks * 32), 16, 1024);
+                        const uint64_t bd = make_desc(smem_u32(sm + P_KQ + 32 * pp * 128 + ks * 32), 16, 1024);
+                        mma_bf16(tmem + 32 * pp, ad, bd, idesc, (hh > 0 || ks > 0) ? 1u : 0u);
                     }
                 commit(&bar);
             }
-            ok = __syncthreads_and(mbar_wait(&bar, hh & 1, err, 2) ? 1 : 0);
+            // while the MMAs run: scale Q e^G, K e^{G_last - G} (image) and K e^G (in place)
+#pragma unroll
+            for (int rr = 0; rr < 2; ++rr) {
+                const int t = 16 * p + tr + 8 * rr;
+                const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
+                float tmp[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * eg[j];
+                *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * egl[j];
+                *reinterpret_cast<uint4*>(img + IMG_B2 + (1 + hh) * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) tmp[j] = kin[rr][j] * eg[j];
+                *reinterpret_cast<uint4*>(sm + P_K + off) = pack8(tmp);
+            }
+            ok = block_wait(&bar, hh & 1, err, 2) && ok;
             fence_after_sync();
         }
     }
@@ -462,7 +473,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             }
             commit(&bar);
         }
-        ok = __syncthreads_and(mbar_wait(&bar, 0, err, 3) ? 1 : 0);
+        ok = block_wait(&bar, 0, err, 3);
         fence_after_sync();
         if (ok) {
             const int i = 16 * sp + l, half = w >> 2;

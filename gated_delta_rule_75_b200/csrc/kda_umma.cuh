@@ -143,6 +143,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     return false;
 }
 
+// Block-wide wait: thread 0 polls `bar` (phase `parity`) with the iteration
+// limit of mbar_wait, the rest of the block sleeps in the barrier, and every
+// thread gets the same verdict.  The barrier orders the observed completion
+// (and the data it guards) before everything the block does next.
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, int* err, int err_bit)
+{
+    int ok = 1;
+    if (threadIdx.x == 0) ok = mbar_wait(bar, parity, err, err_bit) ? 1 : 0;
+    return __syncthreads_or(ok ? 0 : 1) == 0;
+}
+
 // TMEM allocation by one full warp; writes the base address to *dst (smem).
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst, uint32_t ncols)
 {
