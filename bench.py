@@ -154,7 +154,8 @@ def oracle_sample(inp_host, cfg, heads, batch=1):
                sl(inp_host["beta"]), inp_host["scale"], return_state=True)
     dt = time.perf_counter() - t
     head_tokens = cfg.T * heads * batch
-    return dt, head_tokens, oracle.threads()
+    # OpenMP runs over (sequence, head) pairs: no more threads than pairs do work
+    return dt, head_tokens, min(oracle.threads(), heads * batch)
 
 
 def host_sample_inputs(cfg, heads, batch=1):
@@ -169,7 +170,7 @@ def run_reference(args, ws, rank):
     cfg = W.BATCHED
     if rank != 0:
         return
-    heads = 4
+    heads = 16
     inp = host_sample_inputs(cfg, heads)
     for _ in range(args.warmup):
         oracle_sample(inp, cfg, heads)
@@ -270,6 +271,8 @@ def run_prefill(args, ws, rank, kda, peaks):
             "ms_per_launch": k_ms_per_launch, "share_of_step": k_ms_per_step / (ms_max / args.steps),
             "algorithmic_bytes_per_launch": kbytes, "peak_source": peaks["source"] + " (burst copy)"}
     roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = measured_traffic(kname, cfg.name)
+    roof["traffic_source"] = "profiles/dram_traffic.md (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -289,6 +292,39 @@ def run_prefill(args, ws, rank, kda, peaks):
         "clocks": clk.summary(),
     }
     return res, inp, step, (out, hT)
+
+
+KERNEL_SOURCE = {"chunk_prep_tc": "kda_chunk_tc.cu", "chunk_state_tc": "kda_chunk_tc.cu",
+                 "chunk_prep_simt": "kda_chunk_simt.cu", "chunk_state_simt": "kda_chunk_simt.cu",
+                 "decode_step": "kda_decode.cu"}
+
+
+def kernel_source_sha(kname):
+    import hashlib
+    f = KERNEL_SOURCE.get(kname)
+    if f is None:
+        return None
+    path = os.path.join(ROOT, "gated_delta_rule_75_b200", "csrc", f)
+    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+
+
+def measured_traffic(kname, workload):
+    """DRAM bytes (read + write) per launch of `kname` on `workload` from the
+    committed ncu table profiles/dram_traffic.md, or None when the table has no
+    row for this kernel source (the kernel changed since the capture)."""
+    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha(kname)
+    for line in open(path):
+        cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
+        if len(cells) >= 7 and cells[0] == kname and cells[1] == workload and cells[2] == sha:
+            try:
+                launches = float(cells[3])
+                return (float(cells[4]) + float(cells[5])) / launches
+            except ValueError:
+                return None
+    return None
 
 
 def kernel_algorithmic_bytes(kname, cfg):
@@ -351,7 +387,8 @@ def run_decode(args, ws, rank, kda, peaks):
         "state_GBps": bytes_step * cfg.steps * ws / (ms / 1e3) / 1e9,
         "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
-                     "traffic": None, "algorithmic_bytes_per_launch": bytes_step,
+                     "traffic": measured_traffic("decode_step", cfg.name),
+                     "algorithmic_bytes_per_launch": bytes_step,
                      "ms_per_launch": kms / max(1, timed)},
         "gpu_launches": launches,
     }

@@ -1,0 +1,79 @@
+"""GPU edge cases of the chunkwise prefill: heads processed in several
+workspace groups (forced small workspace budget, in a child process since the
+budget is read once per process), hT written over h0 in place, and malformed
+cu_seqlens (reported in debug mode; offsets are clamped on the device, so the
+call never reads or writes out of bounds)."""
+import os
+import subprocess
+import sys
+import textwrap
+
+import numpy as np
+import pytest
+import torch
+
+import workloads as W
+from kda_testutil import TOL, host, oracle_prefill, rel
+
+pytestmark = pytest.mark.gpu
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def kda(cuda_ok):
+    from gated_delta_rule_75_b200 import build
+    build.build()
+    import gated_delta_rule_75_b200 as kda
+    return kda
+
+
+@pytest.mark.parametrize("impl", ["simt", "tensorcore"])
+def test_head_groups_with_small_workspace(cuda_ok, impl):
+    """64 MiB budget: 512 chunks per head need about 34 MB (tensor cores) or
+    76 MB (SIMT), so the three heads run in separate groups."""
+    code = textwrap.dedent(f"""
+        import sys; sys.path.insert(0, {ROOT!r}); sys.path.insert(0, {os.path.join(ROOT, 'tests')!r})
+        import workloads as W, gated_delta_rule_75_b200 as kda, torch
+        from kda_testutil import TOL, oracle_prefill, rel
+        cfg = W.small_prefill(B=4, T=8192, H=3, dk=128, dv=128, io_dtype="bf16", seed=31, h0_std=0.02)
+        inp = W.make_prefill(cfg, "cuda")
+        out, hT = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                inp["scale"], h0=inp["h0"], impl={impl!r})
+        torch.cuda.synchronize()
+        ro, rh = oracle_prefill(inp)
+        eo, eh = rel(out, ro), rel(hT, rh)
+        print(eo, eh)
+        assert eo <= TOL["bf16"] and eh <= TOL["bf16"], (eo, eh)
+    """)
+    env = dict(os.environ, KDA_WORKSPACE_MB="64", KDA_DEBUG="1")
+    r = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                       timeout=600)
+    assert r.returncode == 0, r.stdout + r.stderr
+
+
+@pytest.mark.parametrize("impl,io", [("simt", "f32"), ("tensorcore", "bf16")])
+def test_final_state_written_over_initial_state(kda, impl, io):
+    cfg = W.small_prefill(B=2, T=130, H=2, dk=128, dv=128, io_dtype=io, seed=32, h0_std=0.05)
+    inp = W.make_prefill(cfg, "cuda")
+    ro, rh = oracle_prefill(inp)
+    state = inp["h0"].clone()
+    out, hT = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                            inp["scale"], h0=state, hT=state, impl=impl)
+    torch.cuda.synchronize()
+    assert hT.data_ptr() == state.data_ptr()
+    assert rel(out, ro) <= TOL[io] and rel(state, rh) <= TOL[io]
+
+
+@pytest.mark.parametrize("impl", ["simt", "tensorcore"])
+@pytest.mark.parametrize("cu", [[0, 100, 50, 200], [0, 200, 0, 200], [0, 64, 300, 200], [5, 64, 128, 200]])
+def test_malformed_offsets_are_reported_not_faulted(kda, impl, cu):
+    cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype="bf16", seed=33, lengths=[64, 64, 72])
+    inp = W.make_prefill(cfg, "cuda")
+    inp["cu_seqlens"] = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    with pytest.raises(kda.KDAError) as e:
+        kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
+                      cu_seqlens=inp["cu_seqlens"], impl=impl)
+    assert e.value.status == kda.KDA_ERR_INVALID_ARG
+    # the context is still healthy
+    x = torch.ones(4, device="cuda") * 2
+    assert float(x.sum()) == 8.0
