@@ -52,15 +52,34 @@ static cudaMemPool_t workspace_pool(int dev)
 }
 
 // Workspace budget per call (bytes); heads are processed in groups that fit.
+// KDA_WORKSPACE_MB fixes it; otherwise it is 60 % of the device memory that
+// was free when the library first ran on the device, but at least 4 GiB
+// (queried once per device: the query is too slow for every call).
 static int64_t workspace_budget()
 {
-    static const int64_t b = [] {
+    static const int64_t fixed = [] {
         const char* s = std::getenv("KDA_WORKSPACE_MB");
-        int64_t mb = s ? std::atoll(s) : 4096;
+        if (!s) return int64_t(0);
+        int64_t mb = std::atoll(s);
         if (mb < 64) mb = 64;
         return mb << 20;
     }();
-    return b;
+    if (fixed) return fixed;
+    static std::mutex mu;
+    static int64_t cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return int64_t(4) << 30;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        size_t free_b = 0, total_b = 0;
+        int64_t b = int64_t(4) << 30;
+        if (cudaMemGetInfo(&free_b, &total_b) == cudaSuccess) {
+            const int64_t f = (int64_t)(0.6 * (double)free_b);
+            if (f > b) b = f;
+        }
+        cached[dev] = b;
+    }
+    return cached[dev];
 }
 
 static kda_status_t from_cuda(cudaError_t e)
@@ -179,7 +198,8 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                                      : simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
     const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 1023) / 1024 * 1024 : 0;
     const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1);
-    int64_t Hg = (workspace_budget() - 1024 - off_bytes) / per_head;
+    const int64_t budget = workspace_budget() - 1024 - off_bytes;
+    int64_t Hg = budget / per_head;
     if (Hg < 1) Hg = 1;
     if (Hg > H) Hg = H;
     const int64_t ws_bytes = 1024 + off_bytes + Hg * per_head;

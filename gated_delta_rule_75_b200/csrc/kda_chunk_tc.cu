@@ -199,6 +199,8 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     float* sB = reinterpret_cast<float*>(sm + P_BETA);
     auto G = [&](int t, int c) -> float& { return *reinterpret_cast<float*>(sGb + g_off(t, c)); };
 
+    // beta first: its global latency overlaps the TMA loads and the TMEM allocation
+    const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
     if (tid == 0) {
         mbar_init(&bar_in, 1);
         mbar_init(&bar, 1);
@@ -213,12 +215,11 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
     }
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
-    if (tid < C) sB[tid] = tid < len ? beta[(t0 + tid) * H + h] : 0.f;
+    if (tid < C) sB[tid] = bval;
     fence_before_sync();
-    __syncthreads();
+    bool ok = block_wait(&bar_in, 0, err, 1);      // also the barrier for sB and the TMEM address
     fence_after_sync();
     const uint32_t tmem = tmem_base;
-    bool ok = block_wait(&bar_in, 0, err, 1);
 
     if (ok) {
         // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
@@ -383,11 +384,13 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 const int p = 2 * (w >> 2) + x;
-                float aq[16];
+                float aq[16], bt[16];
+                ld8f(sB + 16 * p, bt);
+                ld8f(sB + 16 * p + 8, bt + 8);
 #pragma unroll
                 for (int cc = 0; cc < 16; ++cc) {
                     const int i = 16 * p + cc;
-                    sA[i * AP + j] = (j < i) ? sB[i] * kp[x][cc] : 0.f;
+                    sA[i * AP + j] = (j < i) ? bt[cc] * kp[x][cc] : 0.f;
                     aq[cc] = (j <= i) ? qp[x][cc] : 0.f;
                 }
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
@@ -449,10 +452,11 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
         for (int e = tid; e < C * 8; e += PT) {
             const int i = e >> 3, cb = e & 7;
-            float f[8];
+            float f[8], bt[8];
             ld8f(sT + i * AP + 8 * cb, f);
+            ld8f(sB + 8 * cb, bt);
 #pragma unroll
-            for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * sB[8 * cb + x] : 0.f;
+            for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * bt[x] : 0.f;
             const uint4 u = pack8(f);
             *reinterpret_cast<uint4*>(sm + P_Q + sw128_offset(i, 8 * cb)) = u;
             *reinterpret_cast<uint4*>(img + IMG_T + sw128_offset(i, 8 * cb)) = u;
@@ -767,26 +771,30 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 32, 64, true))) return e;
     if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
 
+    auto launch_prep = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
+        if (a.si.chunks_upper <= 0) return cudaSuccess;
+        dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
+        LaunchScope scope(s, K_PREP_TC);
+        tc::chunk_prep_tc_kernel<<<gp, tc::PT, tc::P_SMEM, s>>>(maps, a.beta, a.si, a.H, hb, Hg,
+                                                               a.scale, w, err);
+        return cudaGetLastError();
+    };
+    auto launch_state = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
+        dim3 gs((unsigned)a.si.N, (unsigned)hg);
+        LaunchScope scope(s, K_STATE_TC);
+        if (a.h0)
+            tc::chunk_state_tc_kernel<true><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
+        else
+            tc::chunk_state_tc_kernel<false><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
+        return cudaGetLastError();
+    };
+
     for (int64_t hb = 0; hb < a.H; hb += Hg) {
         const int64_t hg = (a.H - hb) < Hg ? (a.H - hb) : Hg;
-        if (a.si.chunks_upper > 0) {
-            dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
-            LaunchScope scope(st, K_PREP_TC);
-            tc::chunk_prep_tc_kernel<<<gp, tc::PT, tc::P_SMEM, st>>>(maps, a.beta, a.si, a.H, hb, Hg,
-                                                                 a.scale, ws, err);
-            if ((e = cudaGetLastError())) return e;
-        }
-        dim3 gs((unsigned)a.si.N, (unsigned)hg);
-        {
-            LaunchScope scope(st, K_STATE_TC);
-            if (a.h0)
-                tc::chunk_state_tc_kernel<true><<<gs, tc::ST, tc::S_SMEM, st>>>(
-                    ws, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
-            else
-                tc::chunk_state_tc_kernel<false><<<gs, tc::ST, tc::S_SMEM, st>>>(
-                    ws, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
-        }
-        if ((e = cudaGetLastError())) return e;
+        if ((e = launch_prep(hb, hg, ws, st))) return e;
+        if ((e = launch_state(hb, hg, ws, st))) return e;
     }
     return cudaSuccess;
 }

@@ -77,3 +77,24 @@ def test_malformed_offsets_are_reported_not_faulted(kda, impl, cu):
     # the context is still healthy
     x = torch.ones(4, device="cuda") * 2
     assert float(x.sum()) == 8.0
+
+
+@pytest.mark.parametrize("H", [4, 6, 9])
+def test_many_heads_and_side_stream(kda, H):
+    """More heads, and the same call on a side stream gives identical results."""
+    cfg = W.small_prefill(B=2, T=300, H=H, dk=128, dv=128, io_dtype="bf16", seed=40 + H, h0_std=0.02)
+    inp = W.make_prefill(cfg, "cuda")
+    out, hT = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                            inp["scale"], h0=inp["h0"])
+    torch.cuda.synchronize()
+    ro, rh = oracle_prefill(inp)
+    assert rel(out, ro) <= TOL["bf16"] and rel(hT, rh) <= TOL["bf16"]
+    # and on a side stream, ordered after work queued there
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        out2 = torch.zeros_like(out)
+        out2, hT2 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                  inp["scale"], h0=inp["h0"], out=out2)
+    s.synchronize()
+    torch.testing.assert_close(out2, out, rtol=0, atol=0)
+    torch.testing.assert_close(hT2, hT, rtol=0, atol=0)
