@@ -56,6 +56,12 @@ def _load():
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_version.argtypes = []
     lib.kda_version.restype = ctypes.c_int
+    lib.kda_chunk_fwd_slots.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                        i64, i64, ctypes.c_float, ctypes.c_int, ctypes.c_int, vp]
+    lib.kda_chunk_fwd_slots.restype = ctypes.c_int
+    lib.kda_recurrent_step_slots.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                             i64, ctypes.c_float, ctypes.c_int, vp]
+    lib.kda_recurrent_step_slots.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -111,13 +117,17 @@ def _stream(device):
 
 
 def chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None, out=None,
-              hT=None, output_final_state=True, impl="auto"):
-    """Chunkwise KDA prefill (C ABI ``kda_chunk_fwd_ex``).
+              hT=None, output_final_state=True, impl="auto", state_pool=None, slots=None):
+    """Chunkwise KDA prefill (C ABI ``kda_chunk_fwd_ex``, or ``kda_chunk_fwd_slots``
+    when ``slots`` is given).
 
     q, k [B,T,H,dk] and v [B,T,H,dv] in fp32 or bf16; log_alpha [B,T,H,dk] and
     beta [B,T,H] fp32; h0 [N,H,dk,dv] fp32 or None.  With ``cu_seqlens`` (int32,
     N+1 entries, on the device) B must be 1 and N sequences are packed along T.
-    Returns (out [B,T,H,dv] in the I/O dtype, hT [N,H,dk,dv] fp32 or None).
+    With ``slots`` (int32 [N] on the device) and ``state_pool`` [P,H,dk,dv] fp32,
+    sequence n starts from and writes back to state_pool[slots[n]] (h0/hT unused).
+    Returns (out [B,T,H,dv] in the I/O dtype, hT [N,H,dk,dv] fp32 or None; with
+    slots: (out, state_pool)).
     """
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -139,12 +149,25 @@ def chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None, out=Non
     else:
         N = B
         n_arg, T_arg = B, T
-    if h0 is not None:
-        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
     if out is None:
         out = torch.empty((B, T, H, dv), dtype=io, device=dev)
     else:
         _check(out, "out", io, (B, T, H, dv), dev)
+    if slots is not None:
+        if state_pool is None or h0 is not None or hT is not None:
+            raise ValueError("slots go with state_pool (and without h0 / hT)")
+        _check(slots, "slots", torch.int32, (N,), dev)
+        P = state_pool.shape[0]
+        _check(state_pool, "state_pool", torch.float32, (P, H, dk, dv), dev)
+        st = _load().kda_chunk_fwd_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                         _ptr(state_pool), _ptr(slots), _ptr(out), _ptr(cu_seqlens),
+                                         n_arg, T_arg, P, H, dk, dv, float(scale), _IO[io],
+                                         _IMPL[impl], _stream(dev))
+        if st != KDA_OK:
+            raise KDAError(st, "kda_chunk_fwd_slots")
+        return out, state_pool
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
     if hT is None and output_final_state:
         hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
     elif hT is not None:
@@ -157,9 +180,11 @@ def chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None, out=Non
     return out, hT
 
 
-def recurrent_step(q, k, v, log_alpha, beta, state, scale, out=None):
+def recurrent_step(q, k, v, log_alpha, beta, state, scale, out=None, slots=None):
     """One decode token per sequence (C ABI ``kda_recurrent_step``); ``state``
-    [N,H,dk,dv] fp32 is updated in place.  Returns out [N,H,dv]."""
+    [N,H,dk,dv] fp32 is updated in place.  With ``slots`` (int32 [N] on the
+    device), ``state`` is a pool [P,H,dk,dv] and sequence n uses slot slots[n]
+    (``kda_recurrent_step_slots``).  Returns out [N,H,dv]."""
     N, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
@@ -171,11 +196,21 @@ def recurrent_step(q, k, v, log_alpha, beta, state, scale, out=None):
     _check(v, "v", io, (N, H, dv), dev)
     _check(log_alpha, "log_alpha", torch.float32, (N, H, dk), dev)
     _check(beta, "beta", torch.float32, (N, H), dev)
-    _check(state, "state", torch.float32, (N, H, dk, dv), dev)
     if out is None:
         out = torch.empty((N, H, dv), dtype=io, device=dev)
     else:
         _check(out, "out", io, (N, H, dv), dev)
+    if slots is not None:
+        _check(slots, "slots", torch.int32, (N,), dev)
+        P = state.shape[0]
+        _check(state, "state", torch.float32, (P, H, dk, dv), dev)
+        st = _load().kda_recurrent_step_slots(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha),
+                                              _ptr(beta), _ptr(state), _ptr(slots), _ptr(out),
+                                              N, P, H, dk, dv, float(scale), _IO[io], _stream(dev))
+        if st != KDA_OK:
+            raise KDAError(st, "kda_recurrent_step_slots")
+        return out
+    _check(state, "state", torch.float32, (N, H, dk, dv), dev)
     st = _load().kda_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                                  _ptr(state), _ptr(out), N, H, dk, dv, float(scale), _IO[io],
                                  _stream(dev))

@@ -128,12 +128,20 @@ const char* kda_status_string(kda_status_t s)
 
 int kda_version(void) { return 100; }
 
-kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
-                                const float* log_alpha, const float* beta, float* state,
-                                void* out, int64_t N, int64_t H, int64_t dk, int64_t dv,
-                                float scale, kda_io_dtype_t io_dtype, cudaStream_t stream)
+}  // extern "C"
+
+namespace kda {
+
+// Error word for debug-mode checks of the decode step (which has no workspace).
+static __device__ int g_decode_err;
+
+static kda_status_t recurrent_step_impl(const void* q, const void* k, const void* v,
+                                        const float* log_alpha, const float* beta, float* state,
+                                        const int32_t* slots, void* out, int64_t N, int64_t P,
+                                        int64_t H, int64_t dk, int64_t dv, float scale,
+                                        kda_io_dtype_t io_dtype, cudaStream_t stream)
 {
-    if (N < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (N < 0 || H < 0 || P < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0 || H == 0) return KDA_OK;
@@ -141,11 +149,60 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
     for (const void* p : ptrs)
         if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
     if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
+    if (slots && !aligned4(slots)) return KDA_ERR_INVALID_ARG;
     if (out == q || out == k || out == v || out == state) return KDA_ERR_INVALID_ARG;
-    cudaError_t e = launch_decode(io_dtype, (int)dk, (int)dv, q, k, v, log_alpha, beta, state,
-                                  out, N * H, scale, stream);
-    if (e == cudaSuccess && debug_mode()) e = cudaStreamSynchronize(stream);
+    DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.state = state;
+    a.out = out; a.N = N; a.H = H; a.P = slots ? P : N; a.dk = (int)dk; a.dv = (int)dv;
+    a.scale = scale; a.io = io_dtype; a.slots = slots; a.err = nullptr;
+    cudaError_t e = cudaSuccess;
+    if (debug_mode() && slots) {
+        void* ep = nullptr;
+        if ((e = cudaGetSymbolAddress(&ep, g_decode_err))) return from_cuda(e);
+        a.err = static_cast<int*>(ep);
+        if ((e = cudaMemsetAsync(a.err, 0, sizeof(int), stream))) return from_cuda(e);
+    }
+    e = launch_decode(a, stream);
+    if (e == cudaSuccess && debug_mode()) {
+        e = cudaStreamSynchronize(stream);
+        if (e == cudaSuccess && a.err) {
+            int flag = 0;
+            e = cudaMemcpy(&flag, a.err, sizeof(int), cudaMemcpyDeviceToHost);
+            if (e == cudaSuccess && flag) return KDA_ERR_INVALID_ARG;
+        }
+    }
     return from_cuda(e);
+}
+
+static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta, const float* h0,
+                                   void* out, float* hT, const int32_t* slots, int64_t P,
+                                   const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                                   int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
+                                   kda_prefill_impl_t impl, cudaStream_t stream);
+
+}  // namespace kda
+
+extern "C" {
+
+kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
+                                const float* log_alpha, const float* beta, float* state,
+                                void* out, int64_t N, int64_t H, int64_t dk, int64_t dv,
+                                float scale, kda_io_dtype_t io_dtype, cudaStream_t stream)
+{
+    return recurrent_step_impl(q, k, v, log_alpha, beta, state, nullptr, out, N, N, H, dk, dv,
+                               scale, io_dtype, stream);
+}
+
+kda_status_t kda_recurrent_step_slots(const void* q, const void* k, const void* v,
+                                      const float* log_alpha, const float* beta,
+                                      float* state_pool, const int32_t* slots, void* out,
+                                      int64_t N, int64_t P, int64_t H, int64_t dk, int64_t dv,
+                                      float scale, kda_io_dtype_t io_dtype, cudaStream_t stream)
+{
+    if (slots == nullptr) return KDA_ERR_INVALID_ARG;
+    return recurrent_step_impl(q, k, v, log_alpha, beta, state_pool, slots, out, N, P, H, dk,
+                               dv, scale, io_dtype, stream);
 }
 
 kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
@@ -154,6 +211,33 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                               int64_t T, int64_t H, int64_t dk, int64_t dv, float scale,
                               kda_io_dtype_t io_dtype, kda_prefill_impl_t impl,
                               cudaStream_t stream)
+{
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, h0, out, hT, nullptr, 0, cu_seqlens, B, T, H,
+                          dk, dv, scale, io_dtype, impl, stream);
+}
+
+kda_status_t kda_chunk_fwd_slots(const void* q, const void* k, const void* v,
+                                 const float* log_alpha, const float* beta, float* state_pool,
+                                 const int32_t* slots, void* out, const int32_t* cu_seqlens,
+                                 int64_t B, int64_t T, int64_t P, int64_t H, int64_t dk,
+                                 int64_t dv, float scale, kda_io_dtype_t io_dtype,
+                                 kda_prefill_impl_t impl, cudaStream_t stream)
+{
+    if (slots == nullptr || state_pool == nullptr || P < 0) return KDA_ERR_INVALID_ARG;
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, state_pool, out, state_pool, slots, P,
+                          cu_seqlens, B, T, H, dk, dv, scale, io_dtype, impl, stream);
+}
+
+}  // extern "C"
+
+namespace kda {
+
+static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta, const float* h0,
+                                   void* out, float* hT, const int32_t* slots, int64_t P,
+                                   const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                                   int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
+                                   kda_prefill_impl_t impl, cudaStream_t stream)
 {
     if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
@@ -175,6 +259,7 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
             return KDA_ERR_INVALID_ARG;
     }
     if ((h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return KDA_ERR_INVALID_ARG;
+    if (slots && !aligned4(slots)) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens && ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0))
         return KDA_ERR_INVALID_ARG;
     // every index must fit the kernels' 64-bit arithmetic and 32-bit grid limits
@@ -184,6 +269,9 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
     a.out = out; a.hT = hT; a.H = H; a.dk = (int)dk; a.dv = (int)dv; a.scale = scale;
     a.io = io_dtype;
+    a.slots = slots;
+    a.P = P;
+    a.err = nullptr;
     SeqInfo& si = a.si;
     si.cu = cu_seqlens;
     si.chunk_off = nullptr;
@@ -209,6 +297,7 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     if (e) return from_cuda(e);
     char* base = static_cast<char*>(buf.ptr);
     int* err_flag = reinterpret_cast<int*>(base);
+    a.err = err_flag;
     if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
@@ -231,6 +320,10 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
     }
     return KDA_OK;
 }
+
+}  // namespace kda
+
+extern "C" {
 
 kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const float* log_alpha,
                            const float* beta, const float* h0, void* out, float* hT,

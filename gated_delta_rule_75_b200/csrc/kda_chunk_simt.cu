@@ -158,10 +158,11 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(256)
-chunk_state_simt_kernel(const float* __restrict__ ws, const float* __restrict__ h0,
-                        T* __restrict__ out, float* __restrict__ hT, SeqInfo si,
-                        int64_t H, int64_t h_base, int64_t Hg)
+chunk_state_simt_kernel(const float* __restrict__ ws, PrefillArgs a, int64_t h_base, int64_t Hg)
 {
+    const SeqInfo& si = a.si;
+    const int64_t H = a.H;
+    T* __restrict__ out = (T*)a.out;
     constexpr int C = kChunk, TW = 32;
     extern __shared__ float smem[];
     float* sW = smem;                 // [C][DK]
@@ -182,9 +183,12 @@ chunk_state_simt_kernel(const float* __restrict__ ws, const float* __restrict__ 
     const int64_t nchunks = si.chunk_count(n, eos - bos);
     const int64_t gc0 = si.chunk_start(n);
 
+    const int64_t sidx = a.state_index(n, h);
+    const float* h0p = (a.h0 && sidx >= 0) ? a.h0 + sidx * DK * DV : nullptr;
+    float* hTp = (a.hT && sidx >= 0) ? a.hT + sidx * DK * DV : nullptr;
     for (int e = tid; e < DK * TW; e += blockDim.x) {
         const int c = e / TW, j = e % TW;
-        sS[e] = h0 ? h0[((n * H + h) * DK + c) * DV + j0 + j] : 0.f;
+        sS[e] = h0p ? h0p[c * DV + j0 + j] : 0.f;
     }
     for (int64_t ch = 0; ch < nchunks; ++ch) {
         const float* blk = ws + ((gc0 + ch) * Hg + hl) * SimtWs<DK, DV>::size;
@@ -224,10 +228,10 @@ chunk_state_simt_kernel(const float* __restrict__ ws, const float* __restrict__ 
         }
     }
     __syncthreads();
-    if (hT) {
+    if (hTp) {
         for (int e = tid; e < DK * TW; e += blockDim.x) {
             const int c = e / TW, j = e % TW;
-            hT[((n * H + h) * DK + c) * DV + j0 + j] = sS[e];
+            hTp[c * DV + j0 + j] = sS[e];
         }
     }
 }
@@ -258,8 +262,7 @@ static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaS
         dim3 gs((unsigned)a.si.N, (unsigned)hg, DV / 32);
         {
             LaunchScope scope(st, K_STATE_SIMT);
-            chunk_state_simt_kernel<T, DK, DV><<<gs, 256, smem_state, st>>>(
-                ws, a.h0, (T*)a.out, a.hT, a.si, a.H, hb, Hg);
+            chunk_state_simt_kernel<T, DK, DV><<<gs, 256, smem_state, st>>>(ws, a, hb, Hg);
         }
         if ((e = cudaGetLastError())) return e;
     }

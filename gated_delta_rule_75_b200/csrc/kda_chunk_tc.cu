@@ -523,7 +523,7 @@ __global__ void __launch_bounds__(ST, 1)
 chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constant__ CUtensorMap vmap,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, SeqInfo si, int64_t H, int64_t h_base, int64_t Hg,
-                      int* __restrict__ err)
+                      const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -541,13 +541,20 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
     const int64_t nch = si.chunk_count(n, eos - bos);
     const int64_t gc0 = si.chunk_start(n);
-    const float* h0p = kHasH0 ? h0 + (n * H + h) * (int64_t)D * D : nullptr;
-    float* hTp = hT ? hT + (n * H + h) * (int64_t)D * D : nullptr;
+    // state slot of this (sequence, head); -1: none (zero start, nothing stored)
+    int64_t sidx = n * H + h;
+    if (slots) {
+        const int64_t sl = slots[n];
+        sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
+        if (sl >= P && tid == 0 && err) atomicOr(err, 1);
+    }
+    const float* h0p = (kHasH0 && sidx >= 0) ? h0 + sidx * (int64_t)D * D : nullptr;
+    float* hTp = (hT && sidx >= 0) ? hT + sidx * (int64_t)D * D : nullptr;
 
     if (nch == 0) {                                      // empty sequence: hT = h0
         if (hTp)
             for (int c = 64 * half; c < 64 * half + 64; ++c)
-                hTp[c * D + j] = kHasH0 ? h0p[c * D + j] : 0.f;
+                hTp[c * D + j] = h0p ? h0p[c * D + j] : 0.f;
         return;
     }
     auto load_stage = [&](int64_t ch, int s) {          // one thread
@@ -610,7 +617,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             const int c0 = 64 * half + 16 * cb;
             float f[16];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) f[x] = kHasH0 ? h0p[(c0 + x) * D + j] : 0.f;
+            for (int x = 0; x < 16; ++x) f[x] = h0p ? h0p[(c0 + x) * D + j] : 0.f;
             *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f);
             *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f + 8);
 #pragma unroll
@@ -784,10 +791,10 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         LaunchScope scope(s, K_STATE_TC);
         if (a.h0)
             tc::chunk_state_tc_kernel<true><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
+                w, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err);
         else
             tc::chunk_state_tc_kernel<false><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, err);
+                w, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err);
         return cudaGetLastError();
     };
 

@@ -20,7 +20,8 @@ template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(256)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                   float* __restrict__ state, T* __restrict__ out, float scale)
+                   float* __restrict__ state, T* __restrict__ out, float scale,
+                   const int32_t* __restrict__ slots, int64_t H, int64_t P, int* __restrict__ err)
 {
     constexpr int TPR = DV / 4;        // threads per state row (float4 each)
     constexpr int RG = 256 / TPR;      // row groups
@@ -35,7 +36,20 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     const int c4 = tid % TPR;
     const int rg = tid / TPR;
 
-    float4* S4 = reinterpret_cast<float4*>(state + p * (int64_t)DK * DV);
+    // pooled states: sequence n owns state slot slots[n]; a negative slot means
+    // "no state" (output zeros); a slot past the pool is reported and skipped
+    int64_t sp = p;
+    if (slots) {
+        const int64_t n = p / H, h = p - n * H;
+        const int64_t sl = slots[n];
+        if (sl < 0 || sl >= P) {
+            if (sl >= P && tid == 0 && err) atomicOr(err, 1);
+            for (int j = tid; j < DV; j += 256) IO<T>::store(out, p * DV + j, 0.f);
+            return;
+        }
+        sp = sl * H + h;
+    }
+    float4* S4 = reinterpret_cast<float4*>(state + sp * (int64_t)DK * DV);
     float4 s[RPT];
 #pragma unroll
     for (int r = 0; r < RPT; ++r)                 // issue every state load first
@@ -91,35 +105,30 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
 }
 
 template <typename T, int DK, int DV>
-static cudaError_t launch_decode_t(const void* q, const void* k, const void* v, const float* g,
-                                   const float* b, float* state, void* out, int64_t NH,
-                                   float scale, cudaStream_t stream)
+static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream)
 {
     LaunchScope scope(stream, K_DECODE);
-    decode_step_kernel<T, DK, DV><<<(unsigned)NH, 256, 0, stream>>>(
-        (const T*)q, (const T*)k, (const T*)v, g, b, state, (T*)out, scale);
+    decode_step_kernel<T, DK, DV><<<(unsigned)(a.N * a.H), 256, 0, stream>>>(
+        (const T*)a.q, (const T*)a.k, (const T*)a.v, a.log_alpha, a.beta, a.state, (T*)a.out,
+        a.scale, a.slots, a.H, a.P, a.err);
     return cudaGetLastError();
 }
 
 template <typename T>
-static cudaError_t launch_decode_d(int dk, int dv, const void* q, const void* k, const void* v,
-                                   const float* g, const float* b, float* state, void* out,
-                                   int64_t NH, float scale, cudaStream_t st)
+static cudaError_t launch_decode_d(const DecodeArgs& a, cudaStream_t st)
 {
-    if (dk == 128 && dv == 128) return launch_decode_t<T, 128, 128>(q, k, v, g, b, state, out, NH, scale, st);
-    if (dk == 128 && dv == 64) return launch_decode_t<T, 128, 64>(q, k, v, g, b, state, out, NH, scale, st);
-    if (dk == 64 && dv == 128) return launch_decode_t<T, 64, 128>(q, k, v, g, b, state, out, NH, scale, st);
-    return launch_decode_t<T, 64, 64>(q, k, v, g, b, state, out, NH, scale, st);
+    if (a.dk == 128 && a.dv == 128) return launch_decode_t<T, 128, 128>(a, st);
+    if (a.dk == 128 && a.dv == 64) return launch_decode_t<T, 128, 64>(a, st);
+    if (a.dk == 64 && a.dv == 128) return launch_decode_t<T, 64, 128>(a, st);
+    return launch_decode_t<T, 64, 64>(a, st);
 }
 
-cudaError_t launch_decode(kda_io_dtype_t io, int dk, int dv, const void* q, const void* k,
-                          const void* v, const float* g, const float* b, float* state, void* out,
-                          int64_t NH, float scale, cudaStream_t st)
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st)
 {
     // one CTA per (sequence, head); grid.x is limited to 2^31-1
-    if (NH > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
-    if (io == KDA_IO_F32) return launch_decode_d<float>(dk, dv, q, k, v, g, b, state, out, NH, scale, st);
-    return launch_decode_d<__nv_bfloat16>(dk, dv, q, k, v, g, b, state, out, NH, scale, st);
+    if (a.N * a.H > 0x7fffffffLL) return cudaErrorInvalidConfiguration;
+    if (a.io == KDA_IO_F32) return launch_decode_d<float>(a, st);
+    return launch_decode_d<__nv_bfloat16>(a, st);
 }
 
 }  // namespace kda

@@ -80,6 +80,42 @@ struct PrefillArgs {
     int dk, dv;
     float scale;
     kda_io_dtype_t io;
+    // pooled states: when `slots` is set, sequence n's initial and final states
+    // live at index slots[n] of h0 / hT ([P, H, dk, dv]); a negative slot means
+    // zero initial state and no final state; slots >= P are reported and skipped
+    const int32_t* slots;
+    int64_t P;
+    int* err;
+
+#ifdef __CUDACC__
+    // Flat (slot, head) index of sequence n's state, or -1 when it has none.
+    __device__ __forceinline__ int64_t state_index(int64_t n, int64_t h) const {
+        if (!slots) return n * H + h;
+        const int64_t sl = slots[n];
+        if (sl < 0) return -1;
+        if (sl >= P) {
+            if (err) atomicOr(err, 1);
+            return -1;
+        }
+        return sl * H + h;
+    }
+#endif
+};
+
+struct DecodeArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    float* state;
+    void* out;
+    int64_t N, H, P;
+    int dk, dv;
+    float scale;
+    kda_io_dtype_t io;
+    const int32_t* slots;    // nullptr: state index = n * H + h
+    int* err;
 };
 
 // Kernel identities for launch counting and timing (kda_profiler.cu).
@@ -110,9 +146,7 @@ private:
 };
 
 // kda_decode.cu
-cudaError_t launch_decode(kda_io_dtype_t io, int dk, int dv, const void* q, const void* k,
-                          const void* v, const float* g, const float* b, float* state, void* out,
-                          int64_t NH, float scale, cudaStream_t st);
+cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 
 // kda_chunk_simt.cu
 int64_t simt_ws_floats_per_chunk(int dk, int dv);

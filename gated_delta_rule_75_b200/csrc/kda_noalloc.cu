@@ -88,6 +88,9 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
     a.out = out; a.hT = hT; a.H = H; a.dk = (int)dk; a.dv = (int)dv; a.scale = scale;
     a.io = io_dtype;
+    a.slots = nullptr;
+    a.P = 0;
+    a.err = nullptr;
     SeqInfo& si = a.si;
     si.cu = cu_seqlens;
     si.chunk_off = nullptr;
@@ -112,6 +115,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     char* base = static_cast<char*>(base_v);
     int* err_flag = reinterpret_cast<int*>(base);
+    a.err = err_flag;
     // the error word must start at zero; offsets and blocks are fully written
     // by the kernels before they are read
     if (cudaMemsetAsync(err_flag, 0, 256, stream) != cudaSuccess) return KDA_ERR_CUDA;

@@ -196,6 +196,44 @@ typedef struct {
 KDA_API void kda_profiler_enable(int on);
 KDA_API int kda_profiler_read(kda_kernel_stat_t* out, int max_entries, int reset);
 
+/*
+ * Pooled recurrent states for serving (continuous batching, prefix reuse,
+ * chunked prefill).  The pages single out the recurrent-state layout across
+ * chunked prefill, batched decode and prefix caching as what breaks in
+ * practice ("Kimi Linear acaba de superar a la atencion completa en sus
+ * propios terminos", section on serving reliability); these entry points keep
+ * every sequence's state in one caller-owned pool and address it by slot.
+ *
+ *  state_pool  [P, H, dk, dv] fp32, read and written in place
+ *  slots       DEVICE int32 [N]: sequence n uses pool slot slots[n].  A negative
+ *              slot means "no cached state": zero initial state, final state
+ *              not stored (decode: output row set to 0, nothing else touched).
+ *              Slots >= P are not accessed (reported as KDA_ERR_INVALID_ARG in
+ *              KDA_DEBUG mode).  Two sequences of one call must not share a
+ *              slot (their updates would race).
+ *
+ * kda_chunk_fwd_slots -- kda_chunk_fwd_ex with h0 = hT = state_pool[slots[n]];
+ *   a prefill that continues from, and returns to, the pool.  Splitting a
+ *   prompt into several calls (chunked prefill) gives the single-call result.
+ * kda_recurrent_step_slots -- kda_recurrent_step on pool slots; N is the number
+ *   of sequences in this step, P the pool size.
+ */
+KDA_API kda_status_t kda_chunk_fwd_slots(const void* q, const void* k, const void* v,
+                                         const float* log_alpha, const float* beta,
+                                         float* state_pool, const int32_t* slots, void* out,
+                                         const int32_t* cu_seqlens,
+                                         int64_t B, int64_t T, int64_t P, int64_t H,
+                                         int64_t dk, int64_t dv, float scale,
+                                         kda_io_dtype_t io_dtype, kda_prefill_impl_t impl,
+                                         cudaStream_t stream);
+
+KDA_API kda_status_t kda_recurrent_step_slots(const void* q, const void* k, const void* v,
+                                              const float* log_alpha, const float* beta,
+                                              float* state_pool, const int32_t* slots, void* out,
+                                              int64_t N, int64_t P, int64_t H, int64_t dk,
+                                              int64_t dv, float scale, kda_io_dtype_t io_dtype,
+                                              cudaStream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char* kda_status_string(kda_status_t status);
 
