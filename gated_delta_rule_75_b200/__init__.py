@@ -13,7 +13,8 @@ import os
 
 import torch
 
-__all__ = ["chunk_fwd", "recurrent_step", "KDAError", "library_path", "version",
+__all__ = ["chunk_fwd", "recurrent_step", "gdn_chunk_fwd", "gdn_recurrent_step", "KDAError",
+           "library_path", "version",
            "profiler_enable", "profiler_read",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
            "KDA_ERR_NO_MEMORY", "KDA_ERR_TIMEOUT"]
@@ -62,6 +63,10 @@ def _load():
     lib.kda_recurrent_step_slots.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
                                              i64, ctypes.c_float, ctypes.c_int, vp]
     lib.kda_recurrent_step_slots.restype = ctypes.c_int
+    lib.kda_gdn_chunk_fwd.argtypes = lib.kda_chunk_fwd_ex.argtypes
+    lib.kda_gdn_chunk_fwd.restype = ctypes.c_int
+    lib.kda_gdn_recurrent_step.argtypes = lib.kda_recurrent_step.argtypes
+    lib.kda_gdn_recurrent_step.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -178,6 +183,53 @@ def chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None, out=Non
     if st != KDA_OK:
         raise KDAError(st, "kda_chunk_fwd")
     return out, hT
+
+
+def gdn_chunk_fwd(q, k, v, log_a, beta, scale, h0=None, cu_seqlens=None, out=None, hT=None,
+                  output_final_state=True, impl="auto"):
+    """Gated DeltaNet prefill (C ABI ``kda_gdn_chunk_fwd``): as :func:`chunk_fwd`
+    with one gate per (token, head), log_a [B,T,H] fp32."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, io = q.device, q.dtype
+    if io not in _IO:
+        raise TypeError(f"unsupported I/O dtype {io}")
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv))):
+        _check(t, name, io, shp, dev)
+    _check(log_a, "log_a", torch.float32, (B, T, H), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    N = B if cu_seqlens is None else cu_seqlens.numel() - 1
+    if cu_seqlens is not None and (B != 1 or cu_seqlens.dtype != torch.int32):
+        raise ValueError("cu_seqlens needs int32 offsets and a leading axis of 1")
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, (N, H, dk, dv), dev)
+    out = torch.empty((B, T, H, dv), dtype=io, device=dev) if out is None else out
+    _check(out, "out", io, (B, T, H, dv), dev)
+    if hT is None and output_final_state:
+        hT = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    st = _load().kda_gdn_chunk_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(beta), _ptr(h0),
+                                   _ptr(out), _ptr(hT), _ptr(cu_seqlens), N, T, H, dk, dv,
+                                   float(scale), _IO[io], _IMPL[impl], _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_gdn_chunk_fwd")
+    return out, hT
+
+
+def gdn_recurrent_step(q, k, v, log_a, beta, state, scale, out=None):
+    """Gated DeltaNet decode step (C ABI ``kda_gdn_recurrent_step``); log_a [N,H]."""
+    N, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, io = q.device, q.dtype
+    _check(log_a, "log_a", torch.float32, (N, H), dev)
+    _check(beta, "beta", torch.float32, (N, H), dev)
+    _check(state, "state", torch.float32, (N, H, dk, dv), dev)
+    out = torch.empty((N, H, dv), dtype=io, device=dev) if out is None else out
+    st = _load().kda_gdn_recurrent_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_a), _ptr(beta),
+                                        _ptr(state), _ptr(out), N, H, dk, dv, float(scale),
+                                        _IO[io], _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_gdn_recurrent_step")
+    return out
 
 
 def recurrent_step(q, k, v, log_alpha, beta, state, scale, out=None, slots=None):

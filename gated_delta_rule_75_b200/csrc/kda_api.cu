@@ -139,15 +139,18 @@ static kda_status_t recurrent_step_impl(const void* q, const void* k, const void
                                         const float* log_alpha, const float* beta, float* state,
                                         const int32_t* slots, void* out, int64_t N, int64_t P,
                                         int64_t H, int64_t dk, int64_t dv, float scale,
-                                        kda_io_dtype_t io_dtype, cudaStream_t stream)
+                                        kda_io_dtype_t io_dtype, bool gate_scalar,
+                                        cudaStream_t stream)
 {
     if (N < 0 || H < 0 || P < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (N == 0 || H == 0) return KDA_OK;
-    const void* ptrs[] = {q, k, v, log_alpha, state, out};
+    const void* ptrs[] = {q, k, v, state, out};
     for (const void* p : ptrs)
         if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (log_alpha == nullptr || !(gate_scalar ? aligned4(log_alpha) : aligned16(log_alpha)))
+        return KDA_ERR_INVALID_ARG;
     if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
     if (slots && !aligned4(slots)) return KDA_ERR_INVALID_ARG;
     if (out == q || out == k || out == v || out == state) return KDA_ERR_INVALID_ARG;
@@ -155,6 +158,7 @@ static kda_status_t recurrent_step_impl(const void* q, const void* k, const void
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.state = state;
     a.out = out; a.N = N; a.H = H; a.P = slots ? P : N; a.dk = (int)dk; a.dv = (int)dv;
     a.scale = scale; a.io = io_dtype; a.slots = slots; a.err = nullptr;
+    a.gate_scalar = gate_scalar;
     cudaError_t e = cudaSuccess;
     if (debug_mode() && slots) {
         void* ep = nullptr;
@@ -179,7 +183,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
                                    void* out, float* hT, const int32_t* slots, int64_t P,
                                    const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
                                    int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
-                                   kda_prefill_impl_t impl, cudaStream_t stream);
+                                   kda_prefill_impl_t impl, bool gate_scalar, cudaStream_t stream);
 
 }  // namespace kda
 
@@ -191,7 +195,16 @@ kda_status_t kda_recurrent_step(const void* q, const void* k, const void* v,
                                 float scale, kda_io_dtype_t io_dtype, cudaStream_t stream)
 {
     return recurrent_step_impl(q, k, v, log_alpha, beta, state, nullptr, out, N, N, H, dk, dv,
-                               scale, io_dtype, stream);
+                               scale, io_dtype, false, stream);
+}
+
+kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const void* v,
+                                    const float* log_a, const float* beta, float* state,
+                                    void* out, int64_t N, int64_t H, int64_t dk, int64_t dv,
+                                    float scale, kda_io_dtype_t io_dtype, cudaStream_t stream)
+{
+    return recurrent_step_impl(q, k, v, log_a, beta, state, nullptr, out, N, N, H, dk, dv,
+                               scale, io_dtype, true, stream);
 }
 
 kda_status_t kda_recurrent_step_slots(const void* q, const void* k, const void* v,
@@ -202,7 +215,7 @@ kda_status_t kda_recurrent_step_slots(const void* q, const void* k, const void* 
 {
     if (slots == nullptr) return KDA_ERR_INVALID_ARG;
     return recurrent_step_impl(q, k, v, log_alpha, beta, state_pool, slots, out, N, P, H, dk,
-                               dv, scale, io_dtype, stream);
+                               dv, scale, io_dtype, false, stream);
 }
 
 kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
@@ -213,7 +226,17 @@ kda_status_t kda_chunk_fwd_ex(const void* q, const void* k, const void* v,
                               cudaStream_t stream)
 {
     return chunk_fwd_impl(q, k, v, log_alpha, beta, h0, out, hT, nullptr, 0, cu_seqlens, B, T, H,
-                          dk, dv, scale, io_dtype, impl, stream);
+                          dk, dv, scale, io_dtype, impl, false, stream);
+}
+
+kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v, const float* log_a,
+                               const float* beta, const float* h0, void* out, float* hT,
+                               const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                               int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
+                               kda_prefill_impl_t impl, cudaStream_t stream)
+{
+    return chunk_fwd_impl(q, k, v, log_a, beta, h0, out, hT, nullptr, 0, cu_seqlens, B, T, H,
+                          dk, dv, scale, io_dtype, impl, true, stream);
 }
 
 kda_status_t kda_chunk_fwd_slots(const void* q, const void* k, const void* v,
@@ -225,7 +248,7 @@ kda_status_t kda_chunk_fwd_slots(const void* q, const void* k, const void* v,
 {
     if (slots == nullptr || state_pool == nullptr || P < 0) return KDA_ERR_INVALID_ARG;
     return chunk_fwd_impl(q, k, v, log_alpha, beta, state_pool, out, state_pool, slots, P,
-                          cu_seqlens, B, T, H, dk, dv, scale, io_dtype, impl, stream);
+                          cu_seqlens, B, T, H, dk, dv, scale, io_dtype, impl, false, stream);
 }
 
 }  // extern "C"
@@ -237,7 +260,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
                                    void* out, float* hT, const int32_t* slots, int64_t P,
                                    const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
                                    int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
-                                   kda_prefill_impl_t impl, cudaStream_t stream)
+                                   kda_prefill_impl_t impl, bool gate_scalar, cudaStream_t stream)
 {
     if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
@@ -251,9 +274,11 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if (B == 0 || H == 0) return KDA_OK;
     const int64_t T_total = cu_seqlens ? T : B * T;
     if (T_total > 0) {
-        const void* ptrs[] = {q, k, v, log_alpha, out};
+        const void* ptrs[] = {q, k, v, out};
         for (const void* p : ptrs)
             if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        if (log_alpha == nullptr || !(gate_scalar ? aligned4(log_alpha) : aligned16(log_alpha)))
+            return KDA_ERR_INVALID_ARG;
         if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
         if (out == q || out == k || out == v || out == log_alpha || out == beta)
             return KDA_ERR_INVALID_ARG;
@@ -272,6 +297,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     a.slots = slots;
     a.P = P;
     a.err = nullptr;
+    a.gate_scalar = gate_scalar;
     SeqInfo& si = a.si;
     si.cu = cu_seqlens;
     si.chunk_off = nullptr;

@@ -52,7 +52,7 @@ __global__ void __launch_bounds__(256)
 chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const float* __restrict__ log_alpha, const float* __restrict__ beta,
                        SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
-                       float* __restrict__ ws)
+                       float* __restrict__ ws, int gate_scalar)
 {
     constexpr int C = kChunk;
     extern __shared__ float smem[];
@@ -77,7 +77,7 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
         const int64_t src = ((t0 + t) * H + h) * DK + c;
         sK[e] = ok ? IO<T>::load(k, src) : 0.f;
         sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
-        sG[e] = ok ? log_alpha[src] : 0.f;
+        sG[e] = ok ? log_alpha[gate_scalar ? (t0 + t) * H + h : src] : 0.f;
     }
     for (int e = tid; e < C * DV; e += blockDim.x) {
         const int t = e / DV, c = e % DV;
@@ -256,7 +256,7 @@ static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaS
             LaunchScope scope(st, K_PREP_SIMT);
             chunk_prep_simt_kernel<T, DK, DV><<<gp, 256, smem_prep, st>>>(
                 (const T*)a.q, (const T*)a.k, (const T*)a.v, a.log_alpha, a.beta, a.si, a.H, hb,
-                Hg, a.scale, ws);
+                Hg, a.scale, ws, a.gate_scalar ? 1 : 0);
             if ((e = cudaGetLastError())) return e;
         }
         dim3 gs((unsigned)a.si.N, (unsigned)hg, DV / 32);

@@ -155,8 +155,8 @@ constexpr uint32_t P_KV = 81920;       // K-major A: Kvar rows (160), one K-bloc
 constexpr uint32_t P_A = 65536;        // fp32 A [64][68] (aliases KQ/KV after the strips)       17 KB
 constexpr uint32_t P_T = P_A + 64 * AP * 4;   // fp32 T [64][68]                                 17 KB
 constexpr uint32_t P_VEC = 102400;     // per-channel vectors: egf[4], eglf[4], dvec[6]          7 KB
-constexpr uint32_t P_BETA = P_VEC + 14 * 512;
-constexpr uint32_t P_BYTES = P_BETA + 256;
+constexpr uint32_t P_BETA = P_VEC + 14 * 512;  // beta [64], then the scalar gates [64]
+constexpr uint32_t P_BYTES = P_BETA + 512;
 constexpr uint32_t P_SMEM = P_BYTES + 1024 + 64;
 constexpr uint32_t P_TX = 16384 + 16384 + 32768;   // bytes the input TMA loads deliver
 static_assert(P_T + 64 * AP * 4 <= P_VEC, "A/T overlap the vectors");
@@ -172,10 +172,11 @@ struct PrepMaps {
     CUtensorMap k, q, g;
 };
 
+template <bool kScalarGate>
 __global__ void __launch_bounds__(PT, 2)
 chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
-                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
-                     unsigned char* __restrict__ ws, int* __restrict__ err)
+                     const float* __restrict__ log_a, SeqInfo si, int64_t H, int64_t h_base,
+                     int64_t Hg, float scale, unsigned char* __restrict__ ws, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -201,21 +202,27 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
 
     // beta first: its global latency overlaps the TMA loads and the TMEM allocation
     const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
+    // Gated DeltaNet: one gate per (token, head), broadcast over the channels
+    const float gval = (kScalarGate && tid < len) ? log_a[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
+    float* sGs = sB + C;                           // [64] scalar gates (kScalarGate)
     if (tid == 0) {
         mbar_init(&bar_in, 1);
         mbar_init(&bar, 1);
         fence_mbar_init();
-        tma::expect_tx(&bar_in, P_TX);
+        tma::expect_tx(&bar_in, kScalarGate ? P_TX - 32768 : P_TX);
         const int32_t y = (int32_t)t0, x = (int32_t)(h * D);
         tma::load_2d(sm + P_K, &maps.k, x, y, &bar_in);
         tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_in);
         tma::load_2d(sm + P_Q, &maps.q, x, y, &bar_in);
         tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_in);
+        if (!kScalarGate) {
 #pragma unroll
-        for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
+            for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
+        }
     }
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
     if (tid < C) sB[tid] = bval;
+    if (kScalarGate && tid < C) sGs[tid] = gval;
     fence_before_sync();
     bool ok = block_wait(&bar_in, 0, err, 1);      // also the barrier for sB and the TMEM address
     fence_after_sync();
@@ -232,7 +239,8 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             float v[32];
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-                v[x] = *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
+                v[x] = kScalarGate ? sGs[tb + x]
+                                   : *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
             float run = 0.f;
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
@@ -760,7 +768,10 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
                            cudaStream_t st)
 {
     cudaError_t e;
-    if ((e = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel,
+    if ((e = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<false>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
+        return e;
+    if ((e = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<true>,
                                   cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
         return e;
     if ((e = cudaFuncSetAttribute(tc::chunk_state_tc_kernel<true>,
@@ -775,15 +786,21 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     CUtensorMap vmap;
     if ((e = make_tensor_map_2d(&maps.k, a.k, true, cols, rows, cols * 2, 64, 64, true))) return e;
     if ((e = make_tensor_map_2d(&maps.q, a.q, true, cols, rows, cols * 2, 64, 64, true))) return e;
-    if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 32, 64, true))) return e;
+    if (a.gate_scalar) maps.g = maps.k;        // unused: the gates are loaded per (token, head)
+    else if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 32, 64, true)))
+        return e;
     if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
 
     auto launch_prep = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
         if (a.si.chunks_upper <= 0) return cudaSuccess;
         dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
         LaunchScope scope(s, K_PREP_TC);
-        tc::chunk_prep_tc_kernel<<<gp, tc::PT, tc::P_SMEM, s>>>(maps, a.beta, a.si, a.H, hb, Hg,
-                                                               a.scale, w, err);
+        if (a.gate_scalar)
+            tc::chunk_prep_tc_kernel<true><<<gp, tc::PT, tc::P_SMEM, s>>>(
+                maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, a.scale, w, err);
+        else
+            tc::chunk_prep_tc_kernel<false><<<gp, tc::PT, tc::P_SMEM, s>>>(
+                maps, a.beta, nullptr, a.si, a.H, hb, Hg, a.scale, w, err);
         return cudaGetLastError();
     };
     auto launch_state = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {

@@ -21,7 +21,8 @@ __global__ void __launch_bounds__(256)
 decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                    const float* __restrict__ log_alpha, const float* __restrict__ beta,
                    float* __restrict__ state, T* __restrict__ out, float scale,
-                   const int32_t* __restrict__ slots, int64_t H, int64_t P, int* __restrict__ err)
+                   const int32_t* __restrict__ slots, int64_t H, int64_t P, int* __restrict__ err,
+                   int gate_scalar)
 {
     constexpr int TPR = DV / 4;        // threads per state row (float4 each)
     constexpr int RG = 256 / TPR;      // row groups
@@ -58,7 +59,7 @@ decode_step_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __
     for (int i = tid; i < DK; i += 256) {
         sk[i] = IO<T>::load(k, p * DK + i);
         sq[i] = scale * IO<T>::load(q, p * DK + i);
-        sa[i] = expf(log_alpha[p * DK + i]);
+        sa[i] = expf(gate_scalar ? log_alpha[p] : log_alpha[p * DK + i]);
     }
     for (int j = tid; j < DV; j += 256) sv[j] = IO<T>::load(v, p * DV + j);
     const float b = beta[p];
@@ -110,7 +111,7 @@ static cudaError_t launch_decode_t(const DecodeArgs& a, cudaStream_t stream)
     LaunchScope scope(stream, K_DECODE);
     decode_step_kernel<T, DK, DV><<<(unsigned)(a.N * a.H), 256, 0, stream>>>(
         (const T*)a.q, (const T*)a.k, (const T*)a.v, a.log_alpha, a.beta, a.state, (T*)a.out,
-        a.scale, a.slots, a.H, a.P, a.err);
+        a.scale, a.slots, a.H, a.P, a.err, a.gate_scalar ? 1 : 0);
     return cudaGetLastError();
 }
 

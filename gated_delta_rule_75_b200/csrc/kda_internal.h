@@ -86,6 +86,9 @@ struct PrefillArgs {
     const int32_t* slots;
     int64_t P;
     int* err;
+    // Gated DeltaNet form: one gate per (token, head), log_alpha [.., H],
+    // broadcast over the key channels
+    bool gate_scalar;
 
 #ifdef __CUDACC__
     // Flat (slot, head) index of sequence n's state, or -1 when it has none.
@@ -116,6 +119,7 @@ struct DecodeArgs {
     kda_io_dtype_t io;
     const int32_t* slots;    // nullptr: state index = n * H + h
     int* err;
+    bool gate_scalar;        // log_alpha [N, H] (one gate per head) instead of [N, H, dk]
 };
 
 // Kernel identities for launch counting and timing (kda_profiler.cu).

@@ -91,6 +91,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     a.slots = nullptr;
     a.P = 0;
     a.err = nullptr;
+    a.gate_scalar = false;
     SeqInfo& si = a.si;
     si.cu = cu_seqlens;
     si.chunk_off = nullptr;

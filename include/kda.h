@@ -197,6 +197,32 @@ KDA_API void kda_profiler_enable(int on);
 KDA_API int kda_profiler_read(kda_kernel_stat_t* out, int max_entries, int reset);
 
 /*
+ * Gated DeltaNet, the direct predecessor the pages compare KDA with ("Kimi
+ * Delta Attention: la atencion lineal detras de Kimi K2 y Qwen3", comparison
+ * table and FAQ; "Cos'e Kimi Delta Attention (KDA)?", section on per-channel
+ * gating): the same recurrence with ONE decay per (token, head),
+ * Diag(alpha_t) = a_t I.  Same arguments as kda_chunk_fwd_ex /
+ * kda_recurrent_step except the gate:
+ *  log_a   [B, T, H] (prefill) or [N, H] (decode) fp32, natural log, <= 0,
+ *          4-byte aligned.
+ * The same kernels run, with the gate broadcast over the key channels.
+ */
+KDA_API kda_status_t kda_gdn_chunk_fwd(const void* q, const void* k, const void* v,
+                                       const float* log_a, const float* beta,
+                                       const float* h0, void* out, float* hT,
+                                       const int32_t* cu_seqlens,
+                                       int64_t B, int64_t T, int64_t H, int64_t dk, int64_t dv,
+                                       float scale, kda_io_dtype_t io_dtype,
+                                       kda_prefill_impl_t impl, cudaStream_t stream);
+
+KDA_API kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const void* v,
+                                            const float* log_a, const float* beta,
+                                            float* state, void* out,
+                                            int64_t N, int64_t H, int64_t dk, int64_t dv,
+                                            float scale, kda_io_dtype_t io_dtype,
+                                            cudaStream_t stream);
+
+/*
  * Pooled recurrent states for serving (continuous batching, prefix reuse,
  * chunked prefill).  The pages single out the recurrent-state layout across
  * chunked prefill, batched decode and prefix caching as what breaks in

@@ -194,3 +194,11 @@ def small_prefill(B=1, T=200, H=2, dk=64, dv=64, io_dtype="f32", seed=0, gate_sh
         B, T = 1, int(sum(lengths))
     return PrefillConfig(f"small_B{B}_T{T}_H{H}_dk{dk}_dv{dv}_{io_dtype}", B, T, H, dk, dv,
                          io_dtype, seed, gate_shift, h0_std, lengths)
+
+
+def scalar_gates(B: int, T: int, H: int, seed: int, gate_shift: float = 0.0,
+                 device="cpu") -> torch.Tensor:
+    """Gated DeltaNet gates: log a = -softplus(N(0,1) + gate_shift), one per (token, head)."""
+    gen = _gen(seed + 1000, device)
+    x = torch.randn((B, T, H), generator=gen, device=device)
+    return -torch.nn.functional.softplus(x + gate_shift)
