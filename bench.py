@@ -196,10 +196,14 @@ def run_reference(args, ws, rank):
 
 
 def workload_config(cfg):
-    return {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv,
-            "chunk": CHUNK, "io": cfg.io_dtype, "gates_state": "fp32",
-            "l2": "inputs larger than L2 (3.2 GB read per step)",
-            "parallelism": "independent replica per GPU (weak scaling, no collective)"}
+    d = {"workload": cfg.name, "B": cfg.B, "T": cfg.T, "H": cfg.H, "dk": cfg.dk, "dv": cfg.dv,
+         "chunk": CHUNK, "io": cfg.io_dtype, "gates_state": "fp32",
+         "l2": f"inputs larger than L2 ({cfg.tokens * cfg.H * (BYTES_PER_HEAD_TOKEN - 256) / 1e9:.2f} "
+               f"GB read per step)",
+         "parallelism": "independent replica per GPU (weak scaling, no collective)"}
+    if cfg.lengths is not None:
+        d["sequence_lengths"] = cfg.lengths
+    return d
 
 
 # ----------------------------------------------------------------------------
@@ -217,7 +221,7 @@ def time_region(fn, steps, stream):
 
 
 def prefill_config(args):
-    cfg = W.BATCHED
+    cfg = {"batched": W.BATCHED, "single": W.SINGLE}.get(args.workload) or W.varlen_config()
     if args.shape:
         B, T, H = (int(x) for x in args.shape.split(","))
         cfg = W.PrefillConfig(f"prefill_B{B}_H{H}_T{T}_d128_bf16", B, T, H, 128, 128, "bf16",
@@ -229,12 +233,13 @@ def run_prefill(args, ws, rank, kda, peaks):
     cfg = prefill_config(args)
     inp = W.make_prefill(cfg, "cuda")
     out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
-    hT = torch.empty((cfg.B, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device="cuda")
+    hT = torch.empty((cfg.N, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device="cuda")
     stream = torch.cuda.current_stream()
 
     def step():
         kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
-                      h0=inp["h0"], out=out, hT=hT, impl=args.prefill_impl)
+                      h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], out=out, hT=hT,
+                      impl=args.prefill_impl)
 
     for _ in range(args.warmup):
         step()
@@ -330,7 +335,10 @@ def measured_traffic(kname, workload):
 def kernel_algorithmic_bytes(kname, cfg):
     """Minimal bytes the named kernel must move for one step of the workload."""
     ht = cfg.B * cfg.T * cfg.H
-    chunks = cfg.B * math.ceil(cfg.T / CHUNK) * cfg.H
+    if cfg.lengths is not None:
+        chunks = sum(math.ceil(L / CHUNK) for L in cfg.lengths) * cfg.H
+    else:
+        chunks = cfg.B * math.ceil(cfg.T / CHUNK) * cfg.H
     dk, dv = cfg.dk, cfg.dv
     io = 2 if cfg.io_dtype == "bf16" else 4
     qkvgb = ht * ((2 * dk + dv) * io + dk * 4 + 4)
@@ -339,11 +347,11 @@ def kernel_algorithmic_bytes(kname, cfg):
     if kname == "chunk_state_simt":      # reads the fp32 workspace (Ut once, the rest per dv tile)
         tiles = dv // 32
         per_chunk = 4 * (CHUNK * dv + tiles * (CHUNK * 3 * dk + CHUNK * CHUNK + dk))
-        return chunks * per_chunk + ht * dv * io + cfg.B * cfg.H * dk * dv * 4
+        return chunks * per_chunk + ht * dv * io + cfg.N * cfg.H * dk * dv * 4
     if kname == "chunk_prep_tc":         # reads q,k,g,beta; writes the operand image
         return ht * (2 * dk * io + dk * 4 + 4) + chunks * TC_WS_BYTES_PER_CHUNK
     if kname == "chunk_state_tc":        # reads the image and v; writes out and hT
-        return chunks * TC_WS_BYTES_PER_CHUNK + ht * 2 * dv * io + cfg.B * cfg.H * dk * dv * 4
+        return chunks * TC_WS_BYTES_PER_CHUNK + ht * 2 * dv * io + cfg.N * cfg.H * dk * dv * 4
     return BYTES_PER_HEAD_TOKEN * ht
 
 
@@ -394,6 +402,62 @@ def run_decode(args, ws, rank, kda, peaks):
     }
 
 
+def run_variants(args, ws, kda, peaks):
+    """The serving and Gated DeltaNet entry points on the benchmark shapes:
+    GDN prefill (one gate per token and head) on B=8, H=32, T=8192, and the
+    decode step on a pool of 512 state slots addressed through a shuffled slot
+    array (N=256 sequences, H=32, d=128)."""
+    res = {}
+    cfg = prefill_config(args)
+    inp = W.make_prefill(cfg, "cuda")
+    log_a = W.scalar_gates(cfg.B, cfg.T, cfg.H, seed=cfg.seed, gate_shift=cfg.gate_shift, device="cuda")
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=torch.bfloat16, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.gdn_chunk_fwd(inp["q"], inp["k"], inp["v"], log_a, inp["beta"], inp["scale"], out=out,
+                          output_final_state=False)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = max_over_ranks(time_region(step, args.steps, stream), ws)
+    res["gdn_prefill"] = {"workload": cfg.name.replace("prefill", "gdn_prefill"),
+                          "tokens_per_s": cfg.B * cfg.T * args.steps * ws / (ms / 1e3),
+                          "ms_per_step": ms / args.steps}
+    del inp, out, log_a
+    torch.cuda.empty_cache()
+
+    dcfg = W.DECODE
+    P = 2 * dcfg.N
+    gen = W.decode_generator(dcfg, "cuda")
+    pool = torch.randn((P, dcfg.H, dcfg.dk, dcfg.dv), generator=gen, device="cuda") * dcfg.state_std
+    slots = torch.randperm(P, generator=gen, device="cuda")[:dcfg.N].to(torch.int32)
+    nsteps = 200
+    xs = [W.make_decode_step(dcfg, gen, "cuda") for _ in range(nsteps)]
+    o = torch.empty((dcfg.N, dcfg.H, dcfg.dv), dtype=torch.bfloat16, device="cuda")
+    scale = 1.0 / math.sqrt(dcfg.dk)
+
+    def run_all():
+        for x in xs:
+            kda.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], pool, scale,
+                               out=o, slots=slots)
+
+    for x in xs[:3]:
+        kda.recurrent_step(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], pool, scale, out=o,
+                           slots=slots)
+    torch.cuda.synchronize()
+    barrier(ws)
+    ms = max_over_ranks(time_region(run_all, 1, stream), ws)
+    per_head = 2 * dcfg.dk * dcfg.dv * 4 + 2 * dcfg.dk * 2 + dcfg.dv * 2 + dcfg.dk * 4 + 4 + dcfg.dv * 2
+    res["slot_decode"] = {"workload": f"slot_decode_N{dcfg.N}_pool{P}_H{dcfg.H}_d128_bf16_x{nsteps}",
+                          "ms_per_step": ms / nsteps,
+                          "state_GBps": per_head * dcfg.N * dcfg.H * nsteps * ws / (ms / 1e3) / 1e9,
+                          "hbm_frac": per_head * dcfg.N * dcfg.H * nsteps / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+    return res
+
+
 def run_e2e(args, ws, kda, inp, bufs, steps):
     """Same metric through the public API with host (pinned) buffers: every
     step copies its inputs host->device and its output device->host."""
@@ -437,6 +501,9 @@ def main():
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="restrict the run (profiling of one kernel family)")
     ap.add_argument("--decode-steps", type=int, default=W.DECODE.steps)
+    ap.add_argument("--workload", choices=["batched", "single", "varlen"], default="batched",
+                    help="prefill workload: batched B=8,H=32,T=8192 (the benchmark), single "
+                         "B=1,H=16,T=4096, or varlen (16 packed sequences, 2^20 tokens, H=32)")
     ap.add_argument("--shape", default="", help="B,T,H override of the prefill workload "
                     "(profiling of a smaller case; the default is the benchmark workload)")
     args = ap.parse_args()
@@ -467,6 +534,8 @@ def main():
         torch.cuda.empty_cache()
         if not args.no_decode and args.only == "all":
             res["decode"] = run_decode(args, ws, rank, kda, peaks)
+            torch.cuda.empty_cache()
+            res["variants"] = run_variants(args, ws, kda, peaks)
         if rank == 0 and not args.no_cpu and args.only == "all":
             cfg = W.BATCHED
             heads, batch = cfg.H, 2

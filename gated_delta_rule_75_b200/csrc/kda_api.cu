@@ -289,6 +289,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         return KDA_ERR_INVALID_ARG;
     // every index must fit the kernels' 64-bit arithmetic and 32-bit grid limits
     if (T_total > (int64_t(1) << 40) || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if (B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;   // one state-kernel block per (seq, head, tile)
 
     PrefillArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
@@ -306,11 +307,14 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     si.T_total = T_total;
     si.nct = cu_seqlens ? 0 : (T + kChunk - 1) / kChunk;
     si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
+    si.order = nullptr;
 
     // workspace: [1 KiB header (error word) | chunk offsets | per-(chunk, head) blocks]
     const int64_t blk_bytes = use_tc ? tc_ws_bytes_per_chunk()
                                      : simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
-    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 1023) / 1024 * 1024 : 0;
+    // [chunk offsets (N+1 int64) | length order (N int32)] when sequences are packed
+    const bool ordered = cu_seqlens != nullptr && B <= kMaxOrderedSeqs;
+    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + (ordered ? B * 4 : 0) + 1023) / 1024 * 1024 : 0;
     const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1);
     const int64_t budget = workspace_budget() - 1024 - off_bytes;
     int64_t Hg = budget / per_head;
@@ -327,10 +331,12 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
-        if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off,
-                                          err_flag, stream)))
+        int32_t* order = ordered ? reinterpret_cast<int32_t*>(chunk_off + B + 1) : nullptr;
+        if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, order,
+                                      err_flag, stream)))
             return from_cuda(e);
         si.chunk_off = chunk_off;
+        si.order = order;
     }
     unsigned char* ws = reinterpret_cast<unsigned char*>(base + 1024 + off_bytes);
     e = use_tc ? run_prefill_tc(a, ws, Hg, err_flag, stream)

@@ -173,10 +173,14 @@ chunk_state_simt_kernel(const float* __restrict__ ws, PrefillArgs a, int64_t h_b
     float* sS = sU + C * TW;          // [DK][TW]
     float* sGam = sS + DK * TW;       // [DK]
 
-    const int64_t n = blockIdx.x;
-    const int hl = blockIdx.y;
+    // blocks run (tile, head)-innermost over sequences ranked longest first
+    const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
+    const int64_t tiles = DV / TW;
+    const int64_t bid = blockIdx.x;
+    const int64_t n = si.seq_of(bid / (hg * tiles));
+    const int hl = (int)((bid / tiles) % hg);
     const int64_t h = h_base + hl;
-    const int j0 = blockIdx.z * TW;
+    const int j0 = (int)(bid % tiles) * TW;
     const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
     int64_t bos, eos;
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
@@ -259,7 +263,7 @@ static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaS
                 Hg, a.scale, ws, a.gate_scalar ? 1 : 0);
             if ((e = cudaGetLastError())) return e;
         }
-        dim3 gs((unsigned)a.si.N, (unsigned)hg, DV / 32);
+        dim3 gs((unsigned)(a.si.N * hg * (DV / 32)));
         {
             LaunchScope scope(st, K_STATE_SIMT);
             chunk_state_simt_kernel<T, DK, DV><<<gs, 256, smem_state, st>>>(ws, a, hb, Hg);

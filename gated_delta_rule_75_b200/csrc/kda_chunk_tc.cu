@@ -507,7 +507,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         }
     } else {
         // the input loads may still be in flight: let them land before leaving
-        mbar_wait(&bar_in, 0, nullptr, 0, 1u << 16);
+        mbar_wait(&bar_in, 0, nullptr, 0, 200);
     }
     fence_before_sync();
     __syncthreads();
@@ -539,8 +539,10 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     __shared__ uint64_t full[2], bar1, bar2;
     __shared__ uint32_t tmem_base;
 
-    const int64_t n = blockIdx.x;
-    const int hl = blockIdx.y;
+    // blocks run heads-innermost over sequences ranked longest first
+    const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
+    const int64_t n = si.seq_of((int64_t)blockIdx.x / hg);
+    const int hl = (int)((int64_t)blockIdx.x % hg);
     const int64_t h = h_base + hl;
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3, half = w >> 2;                // TMEM lane quarter, column half
@@ -751,8 +753,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         // drain this CTA's own copies in flight before its shared memory goes away
         for (int s = 0; s < 2; ++s)
             if (pending[s]) {
-                mbar_wait(&full[s], 0, nullptr, 0, 1u << 16);
-                mbar_wait(&full[s], 1, nullptr, 0, 1u << 16);
+                mbar_wait(&full[s], 0, nullptr, 0, 200);
+                mbar_wait(&full[s], 1, nullptr, 0, 200);
             }
     }
     fence_before_sync();
@@ -804,7 +806,7 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         return cudaGetLastError();
     };
     auto launch_state = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
-        dim3 gs((unsigned)a.si.N, (unsigned)hg);
+        dim3 gs((unsigned)(a.si.N * hg));
         LaunchScope scope(s, K_STATE_TC);
         if (a.h0)
             tc::chunk_state_tc_kernel<true><<<gs, tc::ST, tc::S_SMEM, s>>>(

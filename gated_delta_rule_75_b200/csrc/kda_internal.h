@@ -21,8 +21,14 @@ struct SeqInfo {
     int64_t T_total;            // packed token count (B*T, or T with cu)
     int64_t nct;                // chunks per sequence (fixed-length case)
     int64_t chunks_upper;       // upper bound on the number of chunks (grid size)
+    const int32_t* order;       // device, N entries: sequences longest first, or nullptr
 
 #ifdef __CUDACC__
+    // Sequence handled by the r-th sequential chain: the longest sequences
+    // first when an order is known, so their chains start in the first wave.
+    __device__ __forceinline__ int64_t seq_of(int64_t r) const {
+        return order ? (int64_t)order[r] : r;
+    }
     __device__ __forceinline__ int64_t chunk_start(int64_t n) const {
         return cu ? chunk_off[n] : n * nct;
     }
@@ -168,6 +174,9 @@ constexpr int kErrTimeoutMask = 0x3e;
 
 // kda_seqinfo.cu
 cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
-                                 int64_t* chunk_off, int* err_flag, cudaStream_t st);
+                                 int64_t* chunk_off, int32_t* order, int* err_flag,
+                                 cudaStream_t st);
+// Sequences are ranked by length (for `order`) when there are at most this many.
+constexpr int64_t kMaxOrderedSeqs = 2048;
 
 }  // namespace kda

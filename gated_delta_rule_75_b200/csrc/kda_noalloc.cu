@@ -83,6 +83,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     if ((h0 && !a16(h0)) || (hT && !a16(hT))) return KDA_ERR_INVALID_ARG;
     if (cu_seqlens && !a4(cu_seqlens)) return KDA_ERR_INVALID_ARG;
     if (T_total > (int64_t(1) << 40) || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if (B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
 
     PrefillArgs a;
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
@@ -100,6 +101,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     si.T_total = T_total;
     si.nct = cu_seqlens ? 0 : (T + kChunk - 1) / kChunk;
     si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
+    si.order = nullptr;
 
     // scratch layout: [256 B error word | chunk offsets | per-(chunk, head) blocks];
     // at least one head's chunks must fit, heads then run in groups that fit
@@ -122,8 +124,8 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     if (cudaMemsetAsync(err_flag, 0, 256, stream) != cudaSuccess) return KDA_ERR_CUDA;
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 256);
-        if (launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, err_flag,
-                                 stream) != cudaSuccess)
+        if (launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, nullptr,
+                                 err_flag, stream) != cudaSuccess)
             return KDA_ERR_CUDA;
         si.chunk_off = chunk_off;
     }

@@ -18,7 +18,8 @@ constexpr int kScanThreads = 1024;
 
 __global__ void __launch_bounds__(kScanThreads)
 chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total, int64_t cap,
-                     int64_t* __restrict__ chunk_off, int* __restrict__ err)
+                     int64_t* __restrict__ chunk_off, int32_t* __restrict__ order,
+                     int* __restrict__ err)
 {
     using Scan = cub::BlockScan<int64_t, kScanThreads>;
     __shared__ typename Scan::TempStorage tmp;
@@ -48,13 +49,28 @@ chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
         if (carry > cap) atomicOr(err, 1);
         chunk_off[N] = carry < cap ? carry : cap;
     }
+    if (order == nullptr) return;
+    // rank sequences by chunk count, longest first (ties: lower index first):
+    // order[rank] = sequence
+    __syncthreads();
+    for (int64_t n = threadIdx.x; n < N; n += kScanThreads) {
+        const int64_t cn = chunk_off[n + 1] - chunk_off[n];
+        int64_t rank = 0;
+        for (int64_t m = 0; m < N; ++m) {
+            const int64_t cm = chunk_off[m + 1] - chunk_off[m];
+            rank += (cm > cn) || (cm == cn && m < n);
+        }
+        order[rank] = (int32_t)n;
+    }
 }
 
 cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
-                                 int64_t* chunk_off, int* err_flag, cudaStream_t st)
+                                 int64_t* chunk_off, int32_t* order, int* err_flag,
+                                 cudaStream_t st)
 {
     LaunchScope scope(st, K_CHUNK_OFFSETS);
-    chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, cap, chunk_off, err_flag);
+    chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, cap, chunk_off, order,
+                                                     err_flag);
     return cudaGetLastError();
 }
 

@@ -115,27 +115,30 @@ __device__ __forceinline__ void fence_mbar_init()
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
 }
 
-__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity)
+// One bounded wait on phase `parity` of `bar`: the thread is suspended by the
+// hardware until the phase completes or about `hint_ns` nanoseconds pass, so a
+// waiting warp issues almost nothing.  Returns whether the phase completed.
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity,
+                                              uint32_t hint_ns = 100000)
 {
     uint32_t ok;
     asm volatile(
         "{\n\t"
         ".reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.b32 %0, 1, 0, p;\n\t"
         "}\n"
         : "=r"(ok)
-        : "r"(smem_u32(bar)), "r"(parity)
+        : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
         : "memory");
     return ok != 0;
 }
 
 // Wait for phase `parity` of `bar` to complete, giving up after `limit`
-// polls: then bit `err_bit` is set in *err and false is returned.  Each poll
-// is a hardware try_wait, which returns after a bounded, implementation-defined
-// time, so the whole wait is bounded.
+// suspended polls (each at most ~0.1 ms, so about 2 s in all by default): then
+// bit `err_bit` is set in *err and false is returned.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* err, int err_bit,
-                                          uint32_t limit = (1u << 20))
+                                          uint32_t limit = 20000)
 {
     for (uint32_t i = 0; i < limit; ++i)
         if (mbar_try_wait(bar, parity)) return true;

@@ -37,6 +37,7 @@ def check_full(kda, cfg, impl="auto"):
     ro, rh = oracle_prefill(inp)
     eo, eh = rel(out, ro), rel(hT, rh)
     tol = TOL[cfg.io_dtype]
+    print(f"PARITY {cfg.name} impl={impl} out={eo:.3e} hT={eh:.3e} tol={tol:g}")
     assert eo <= tol and eh <= tol, (cfg.name, impl, eo, eh)
     return eo, eh
 
@@ -164,8 +165,9 @@ def test_batched_prefill_sampled_pairs(kda):
     pairs = [(int(rng.integers(cfg.B)), int(rng.integers(cfg.H))) for _ in range(4)]
     res = oracle_pairs(inp, pairs)
     for (n, h), ((b, t0, t1), ro, rh) in zip(pairs, res):
-        assert rel(out[b, t0:t1, h], ro) <= TOL["bf16"], (n, h)
-        assert rel(hT[n, h], rh) <= TOL["bf16"], (n, h)
+        eo, eh = rel(out[b, t0:t1, h], ro), rel(hT[n, h], rh)
+        print(f"PARITY {cfg.name} pair=({n},{h}) out={eo:.3e} hT={eh:.3e} tol=0.005")
+        assert eo <= TOL["bf16"] and eh <= TOL["bf16"], (n, h)
 
 
 @pytest.mark.slow
@@ -181,5 +183,6 @@ def test_long_context_varlen_sampled_pairs(kda):
     pairs = [(n, int(rng.integers(cfg.H))) for n in seqs]
     res = oracle_pairs(inp, pairs)
     for (n, h), ((b, t0, t1), ro, rh) in zip(pairs, res):
-        assert rel(out[0, t0:t1, h], ro) <= TOL["bf16"], (n, h)
-        assert rel(hT[n, h], rh) <= TOL["bf16"], (n, h)
+        eo, eh = rel(out[0, t0:t1, h], ro), rel(hT[n, h], rh)
+        print(f"PARITY {cfg.name} pair=({n},{h}) len={t1 - t0} out={eo:.3e} hT={eh:.3e} tol=0.005")
+        assert eo <= TOL["bf16"] and eh <= TOL["bf16"], (n, h)
