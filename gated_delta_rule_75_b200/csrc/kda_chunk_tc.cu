@@ -200,12 +200,8 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     float* sB = reinterpret_cast<float*>(sm + P_BETA);
     auto G = [&](int t, int c) -> float& { return *reinterpret_cast<float*>(sGb + g_off(t, c)); };
 
-    // beta first: its global latency overlaps the TMA loads and the TMEM allocation
-    const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
-    // Gated DeltaNet: one gate per (token, head), broadcast over the channels
-    const float gval = (kScalarGate && tid < len) ? log_a[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
     float* sGs = sB + C;                           // [64] scalar gates (kScalarGate)
-    if (tid == 0) {
+    if (tid == 0) {                                // the input loads go out first
         mbar_init(&bar_in, 1);
         mbar_init(&bar, 1);
         fence_mbar_init();
@@ -220,6 +216,9 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
         }
     }
+    // beta (and the scalar gates) meanwhile: their latency overlaps the TMA loads
+    const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
+    const float gval = (kScalarGate && tid < len) ? log_a[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
     if (tid < C) sB[tid] = bval;
     if (kScalarGate && tid < C) sGs[tid] = gval;
@@ -227,6 +226,16 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     bool ok = block_wait(&bar_in, 0, err, 1);      // also the barrier for sB and the TMEM address
     fence_after_sync();
     const uint32_t tmem = tmem_base;
+    if (ok && len < C) {
+        // a partial chunk: tokens past its end (next sequence or zero fill) read as zero
+        for (int e = tid; e < (C - (int)len) * 16; e += PT) {
+            const int t = (int)len + (e >> 4), ch = e & 15;
+            const uint32_t off = (ch >> 3) * 8192 + sw128_offset(t, (8 * ch) & 63);
+            *reinterpret_cast<uint4*>(sm + P_K + off) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sm + P_Q + off) = make_uint4(0, 0, 0, 0);
+        }
+        __syncthreads();
+    }
 
     if (ok) {
         // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
@@ -295,11 +304,13 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             }
             ld8f(egf + p * D + c0, eg);
             ld8f(eglf + p * D + c0, egl);
+            float egs[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) egs[j] = scale * eg[j];
             float kin[2][8], qin[2][8], kd[2][8];
 #pragma unroll
             for (int rr = 0; rr < 2; ++rr) {
                 const int t = 16 * p + tr + 8 * rr;
-                const bool live = t < len;
                 float G8[8], kk[8], qq[8];
                 {
                     const float4 a = *reinterpret_cast<const float4*>(slab + t * 128 + ((q0 ^ (t & 7)) << 4));
@@ -315,10 +326,9 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                     const float x = G8[j] - Gf8[j];
                     const float e1 = ex2(x);          // <= 1
                     const float r1 = ex2(-x);         // >= 1, at most 15 tokens of decay
-                    const float kv = live ? kk[j] : 0.f;
-                    kin[rr][j] = kv * e1;
-                    qin[rr][j] = live ? scale * qq[j] * e1 : 0.f;
-                    kd[rr][j] = kv * r1;
+                    kin[rr][j] = kk[j] * e1;
+                    qin[rr][j] = qq[j] * e1;          // `scale` is applied to Aqk and Q e^G later
+                    kd[rr][j] = kk[j] * r1;
                 }
                 // operands of the strip MMAs first
                 const int ts = tr + 8 * rr;          // row within the sub-chunk
@@ -360,7 +370,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
                 float tmp[8];
 #pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * eg[j];
+                for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * egs[j];
                 *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * egl[j];
@@ -399,7 +409,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 for (int cc = 0; cc < 16; ++cc) {
                     const int i = 16 * p + cc;
                     sA[i * AP + j] = (j < i) ? bt[cc] * kp[x][cc] : 0.f;
-                    aq[cc] = (j <= i) ? qp[x][cc] : 0.f;
+                    aq[cc] = (j <= i) ? scale * qp[x][cc] : 0.f;
                 }
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
                 *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p + 8)) = pack8(aq + 8);
@@ -476,7 +486,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         // ---- (b3) W = T' (K e^G): M = 64 tokens, N = 128 channels, K = 64 tokens
         if (tid == 0) {
             fence_after_sync();
-            const uint32_t idesc = make_idesc_bf16(64, 128, false, true);
+            const uint32_t idesc = make_idesc_bf16(64, 128, false, true, true);   // -T' (K e^G)
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = make_desc(smem_u32(sm + P_Q + ks * 32), 16, 1024);
@@ -498,8 +508,6 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 unsigned char* dst = img + IMG_W + half * 8192;
 #pragma unroll
                 for (int cb = 0; cb < 4; ++cb) {
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) f[cb][x] = -f[cb][x];
                     *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
                     *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
                 }
