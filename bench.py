@@ -352,6 +352,9 @@ def kernel_algorithmic_bytes(kname, cfg):
         return ht * (2 * dk * io + dk * 4 + 4) + chunks * TC_WS_BYTES_PER_CHUNK
     if kname == "chunk_state_tc":        # reads the image and v; writes out and hT
         return chunks * TC_WS_BYTES_PER_CHUNK + ht * 2 * dv * io + cfg.N * cfg.H * dk * dv * 4
+    if kname == "chunk_state_seg_tc":    # value walk (image, v) + map walk (image), per step;
+        # the per-segment (M, B) matrices they write are not counted
+        return 2 * chunks * TC_WS_BYTES_PER_CHUNK + ht * dv * io
     return BYTES_PER_HEAD_TOKEN * ht
 
 
@@ -494,7 +497,8 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
-    ap.add_argument("--prefill-impl", choices=["auto", "simt", "tensorcore"], default="auto")
+    ap.add_argument("--prefill-impl", choices=["auto", "simt", "tensorcore", "tensorcore_chain",
+                                               "tensorcore_segmented"], default="auto")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")

@@ -7,6 +7,8 @@ library is missing or fails to load, every call raises.
 
     out, hT = chunk_fwd(q, k, v, log_alpha, beta, scale, h0=None, cu_seqlens=None)
     out     = recurrent_step(q, k, v, log_alpha, beta, state, scale)   # state in place
+    maps, offs = chunk_fwd_segmap(q, k, v, log_alpha, beta)            # context parallelism
+    start   = affine_prefix(maps, offs, h0)
 """
 import ctypes
 import os
@@ -14,6 +16,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "recurrent_step", "gdn_chunk_fwd", "gdn_recurrent_step", "KDAError",
+           "chunk_fwd_segmap", "affine_prefix",
            "library_path", "version",
            "profiler_enable", "profiler_read",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -22,7 +25,8 @@ __all__ = ["chunk_fwd", "recurrent_step", "gdn_chunk_fwd", "gdn_recurrent_step",
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_NO_MEMORY, \
     KDA_ERR_TIMEOUT = range(6)
 _IO = {torch.float32: 0, torch.bfloat16: 1}
-_IMPL = {"auto": 0, "simt": 1, "tensorcore": 2}
+_IMPL = {"auto": 0, "simt": 1, "tensorcore": 2, "tensorcore_chain": 3,
+         "tensorcore_segmented": 4}
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 
@@ -67,6 +71,11 @@ def _load():
     lib.kda_gdn_chunk_fwd.restype = ctypes.c_int
     lib.kda_gdn_recurrent_step.argtypes = lib.kda_recurrent_step.argtypes
     lib.kda_gdn_recurrent_step.restype = ctypes.c_int
+    lib.kda_chunk_fwd_segmap.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64,
+                                         i64, ctypes.c_int, vp]
+    lib.kda_chunk_fwd_segmap.restype = ctypes.c_int
+    lib.kda_affine_prefix.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp]
+    lib.kda_affine_prefix.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -268,4 +277,65 @@ def recurrent_step(q, k, v, log_alpha, beta, state, scale, out=None, slots=None)
                                  _stream(dev))
     if st != KDA_OK:
         raise KDAError(st, "kda_recurrent_step")
+    return out
+
+
+def chunk_fwd_segmap(q, k, v, log_alpha, beta, cu_seqlens=None, maps=None, offs=None):
+    """Affine map of every (sequence, head) of a prefill input (C ABI
+    ``kda_chunk_fwd_segmap``): for any entry state S0 the final state is
+    maps[n, h] @ S0 + offs[n, h].  Inputs as for :func:`chunk_fwd`.  Returns
+    (maps [N,H,dk,dk], offs [N,H,dk,dv]), fp32."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, io = q.device, q.dtype
+    if io not in _IO:
+        raise TypeError(f"unsupported I/O dtype {io}")
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv))):
+        _check(t, name, io, shp, dev)
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H, dk), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    if cu_seqlens is not None:
+        if B != 1 or cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev:
+            raise ValueError("cu_seqlens needs int32 offsets on the device and a leading axis of 1")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    if maps is None:
+        maps = torch.empty((N, H, dk, dk), dtype=torch.float32, device=dev)
+    if offs is None:
+        offs = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev)
+    _check(maps, "maps", torch.float32, (N, H, dk, dk), dev)
+    _check(offs, "offs", torch.float32, (N, H, dk, dv), dev)
+    st = _load().kda_chunk_fwd_segmap(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                      _ptr(maps), _ptr(offs), _ptr(cu_seqlens), N, T, H, dk, dv,
+                                      _IO[io], _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_fwd_segmap")
+    return maps, offs
+
+
+def affine_prefix(maps, offs, h0=None, out=None):
+    """State after consecutive affine maps (C ABI ``kda_affine_prefix``).
+
+    maps [S, ..., dk, dk] and offs [S, ..., dk, dv] fp32 hold S segments in
+    order (segment-major); h0 [..., dk, dv] fp32 or None (zeros).  Returns
+    out [..., dk, dv] = M_{S-1}(...(M_0 h0 + B_0)...) + B_{S-1}."""
+    nseg = maps.shape[0]
+    lead = tuple(offs.shape[1:-2])
+    dk, dv = offs.shape[-2], offs.shape[-1]
+    dev = offs.device
+    NH = 1
+    for x in lead:
+        NH *= x
+    _check(maps, "maps", torch.float32, (nseg,) + lead + (dk, dk), dev)
+    _check(offs, "offs", torch.float32, (nseg,) + lead + (dk, dv), dev)
+    if h0 is not None:
+        _check(h0, "h0", torch.float32, lead + (dk, dv), dev)
+    if out is None:
+        out = torch.empty(lead + (dk, dv), dtype=torch.float32, device=dev)
+    _check(out, "out", torch.float32, lead + (dk, dv), dev)
+    st = _load().kda_affine_prefix(_ptr(maps), _ptr(offs), _ptr(h0), _ptr(out), nseg, NH, dk, dv,
+                                   _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_affine_prefix")
     return out

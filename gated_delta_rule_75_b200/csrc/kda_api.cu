@@ -183,7 +183,8 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
                                    void* out, float* hT, const int32_t* slots, int64_t P,
                                    const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
                                    int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
-                                   kda_prefill_impl_t impl, bool gate_scalar, cudaStream_t stream);
+                                   kda_prefill_impl_t impl, bool gate_scalar, cudaStream_t stream,
+                                   float* maps = nullptr, float* offs = nullptr);
 
 }  // namespace kda
 
@@ -255,32 +256,93 @@ kda_status_t kda_chunk_fwd_slots(const void* q, const void* k, const void* v,
 
 namespace kda {
 
+// Streaming multiprocessors of the current device (queried once per device).
+static int64_t sm_count()
+{
+    static std::mutex mu;
+    static int cached[64] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+    std::lock_guard<std::mutex> lock(mu);
+    if (cached[dev] == 0) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+            n = 148;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
+// Segment plan of the tensor-core state walk.  A chain per (sequence, head)
+// runs one CTA per SM at most, so with fewer chains than about a quarter of
+// the SMs the walk is latency-bound on its longest chain; cutting the chains
+// into segments costs about three walks' worth of work (value, map, final) but
+// runs them side by side.  The plan aims at about one segment-CTA per SM.
+static SegPlan plan_segments(const SeqInfo& si, int64_t H, kda_prefill_impl_t impl)
+{
+    SegPlan p;
+    std::memset(&p, 0, sizeof(p));
+    if (impl == KDA_PREFILL_TENSORCORE_CHAIN || si.chunks_upper <= 0) return p;
+    const bool force = impl == KDA_PREFILL_TENSORCORE_SEGMENTED;
+    const int64_t sms = sm_count();
+    const int64_t chains = si.N * H;
+    if (!force && chains * 4 > sms) return p;
+    if (si.cu == nullptr) {
+        int64_t per_chain = sms / chains;
+        if (per_chain < 2) per_chain = 2;
+        const int64_t len = (si.nct + per_chain - 1) / per_chain;
+        const int64_t nseg = (si.nct + len - 1) / len;
+        if (!force && nseg < 4) return p;
+        p.len = len;
+        p.nseg = nseg;
+        p.upper = si.N * nseg;
+    } else {
+        int64_t total = sms / H;                 // segments wanted over all sequences
+        if (total < 2 * si.N) total = 2 * si.N;
+        const int64_t len = (si.chunks_upper + total - 1) / total;
+        if (!force && si.chunks_upper < 4 * len * si.N) return p;
+        p.len = len;
+        p.nseg = 0;
+        p.upper = (si.chunks_upper + len - 1) / len + si.N;
+    }
+    return p;
+}
+
 static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
                                    const float* log_alpha, const float* beta, const float* h0,
                                    void* out, float* hT, const int32_t* slots, int64_t P,
                                    const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
                                    int64_t dk, int64_t dv, float scale, kda_io_dtype_t io_dtype,
-                                   kda_prefill_impl_t impl, bool gate_scalar, cudaStream_t stream)
+                                   kda_prefill_impl_t impl, bool gate_scalar, cudaStream_t stream,
+                                   float* maps, float* offs)
 {
+    // segmap mode: each (sequence, head)'s affine map instead of outputs
+    const bool segmap = maps != nullptr || offs != nullptr;
     if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (impl != KDA_PREFILL_AUTO && impl != KDA_PREFILL_SIMT && impl != KDA_PREFILL_TENSORCORE)
+    if (impl < KDA_PREFILL_AUTO || impl > KDA_PREFILL_TENSORCORE_SEGMENTED)
         return KDA_ERR_INVALID_ARG;
     const bool tc_shape = io_dtype == KDA_IO_BF16 && dk == 128 && dv == 128;
-    if (impl == KDA_PREFILL_TENSORCORE && !tc_shape) return KDA_ERR_UNSUPPORTED;
-    const bool use_tc = impl == KDA_PREFILL_TENSORCORE || (impl == KDA_PREFILL_AUTO && tc_shape);
+    const bool tc_forced = impl != KDA_PREFILL_AUTO && impl != KDA_PREFILL_SIMT;
+    if (tc_forced && !tc_shape) return KDA_ERR_UNSUPPORTED;
+    const bool use_tc = tc_forced || (impl == KDA_PREFILL_AUTO && tc_shape);
     if (cu_seqlens != nullptr && B < 1) return KDA_ERR_INVALID_ARG;
+    if (segmap) {
+        if (maps == nullptr || offs == nullptr || !aligned16(maps) || !aligned16(offs))
+            return KDA_ERR_INVALID_ARG;
+        if (maps == offs) return KDA_ERR_INVALID_ARG;
+    }
     if (B == 0 || H == 0) return KDA_OK;
     const int64_t T_total = cu_seqlens ? T : B * T;
     if (T_total > 0) {
-        const void* ptrs[] = {q, k, v, out};
+        const void* ptrs[] = {q, k, v, segmap ? (const void*)maps : out};
         for (const void* p : ptrs)
             if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
         if (log_alpha == nullptr || !(gate_scalar ? aligned4(log_alpha) : aligned16(log_alpha)))
             return KDA_ERR_INVALID_ARG;
         if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
-        if (out == q || out == k || out == v || out == log_alpha || out == beta)
+        if (!segmap && (out == q || out == k || out == v || out == log_alpha || out == beta))
             return KDA_ERR_INVALID_ARG;
     }
     if ((h0 && !aligned16(h0)) || (hT && !aligned16(hT))) return KDA_ERR_INVALID_ARG;
@@ -292,6 +354,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if (B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;   // one state-kernel block per (seq, head, tile)
 
     PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
     a.out = out; a.hT = hT; a.H = H; a.dk = (int)dk; a.dv = (int)dv; a.scale = scale;
     a.io = io_dtype;
@@ -299,6 +362,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     a.P = P;
     a.err = nullptr;
     a.gate_scalar = gate_scalar;
+    a.tc_what = 0;
     SeqInfo& si = a.si;
     si.cu = cu_seqlens;
     si.chunk_off = nullptr;
@@ -309,18 +373,55 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
     si.order = nullptr;
 
-    // workspace: [1 KiB header (error word) | chunk offsets | per-(chunk, head) blocks]
-    const int64_t blk_bytes = use_tc ? tc_ws_bytes_per_chunk()
-                                     : simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
-    // [chunk offsets (N+1 int64) | length order (N int32)] when sequences are packed
-    const bool ordered = cu_seqlens != nullptr && B <= kMaxOrderedSeqs;
-    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + (ordered ? B * 4 : 0) + 1023) / 1024 * 1024 : 0;
-    const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1);
-    const int64_t budget = workspace_budget() - 1024 - off_bytes;
+    // segment plan (tensor-core path): the segment-parallel walk, or in
+    // segmap mode one segment per sequence written to the caller's buffers
+    SegPlan& plan = a.seg;
+    std::memset(&plan, 0, sizeof(plan));
+    if (use_tc && segmap) {
+        a.tc_what = 1;
+        plan.len = int64_t(1) << 40;
+        plan.nseg = 1;
+        plan.upper = B;
+        plan.maps = maps;
+        plan.offs = offs;
+        plan.hstride = H;
+        plan.abs_head = true;
+    } else if (use_tc) {
+        plan = plan_segments(si, H, impl);
+        if (plan.upper > 0x7fffffffLL / H) std::memset(&plan, 0, sizeof(plan));
+    }
+    const bool seg_table = use_tc && !segmap && plan.len > 0 && cu_seqlens != nullptr;
+
+    // workspace: [1 KiB header (error word) | chunk offsets (+ length order,
+    // + segment offsets) | per head group: per-(chunk, head) blocks, segment
+    // buffers | SIMT segmap extras]
+    const int64_t blk_bytes =
+        use_tc ? tc_ws_bytes_per_chunk()
+               : simt_ws_floats_per_chunk((int)dk, (int)(segmap && dk > dv ? dk : dv)) *
+                     (int64_t)sizeof(float);
+    const bool ordered = cu_seqlens != nullptr && B <= kMaxOrderedSeqs && !seg_table;
+    const int64_t off_bytes =
+        cu_seqlens ? ((B + 1) * 8 + (ordered ? B * 4 : 0) + (seg_table ? (B + 1) * 8 : 0) + 1023) /
+                         1024 * 1024
+                   : 0;
+    const int64_t seg_bytes = (use_tc && !segmap) ? tc_seg_bytes_per_head(plan) : 0;
+    const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1) + seg_bytes;
+    // SIMT segmap: zero values [T, H, dk], scratch outputs [T, H, max(dk, dv)],
+    // identity initial states [N, H, dk, dk]
+    const int64_t es = io_dtype == KDA_IO_BF16 ? 2 : 4;
+    int64_t extra = 0, ex_v0 = 0, ex_out = 0, ex_eye = 0;
+    if (segmap && !use_tc) {
+        const int64_t dm = dk > dv ? dk : dv;
+        ex_v0 = 0;
+        ex_out = (T_total * H * dk * es + 1023) / 1024 * 1024;
+        ex_eye = ex_out + (T_total * H * dm * es + 1023) / 1024 * 1024;
+        extra = ex_eye + B * H * dk * dk * 4;
+    }
+    const int64_t budget = workspace_budget() - 1024 - off_bytes - extra;
     int64_t Hg = budget / per_head;
     if (Hg < 1) Hg = 1;
     if (Hg > H) Hg = H;
-    const int64_t ws_bytes = 1024 + off_bytes + Hg * per_head;
+    const int64_t ws_bytes = 1024 + off_bytes + Hg * per_head + (extra ? extra + 1024 : 0);
 
     StreamBuffer buf;
     cudaError_t e = buf.alloc((size_t)ws_bytes, stream);
@@ -332,15 +433,37 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
         int32_t* order = ordered ? reinterpret_cast<int32_t*>(chunk_off + B + 1) : nullptr;
+        int64_t* seg_off = seg_table ? chunk_off + B + 1 : nullptr;
         if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, order,
-                                      err_flag, stream)))
+                                      err_flag, plan.len, plan.upper, seg_off, stream)))
             return from_cuda(e);
         si.chunk_off = chunk_off;
         si.order = order;
+        plan.seg_off = seg_off;
     }
     unsigned char* ws = reinterpret_cast<unsigned char*>(base + 1024 + off_bytes);
-    e = use_tc ? run_prefill_tc(a, ws, Hg, err_flag, stream)
-               : run_prefill_simt(a, reinterpret_cast<float*>(ws), Hg, stream);
+    if (use_tc) {
+        e = run_prefill_tc(a, ws, Hg, err_flag, stream);
+    } else if (!segmap) {
+        e = run_prefill_simt(a, reinterpret_cast<float*>(ws), Hg, stream);
+    } else {
+        // B: the final states from zero; M: from the identity with zero values
+        char* ex = reinterpret_cast<char*>(
+            (reinterpret_cast<uintptr_t>(ws) + Hg * per_head + 1023) & ~uintptr_t(1023));
+        void* v0 = ex + ex_v0;
+        void* scratch = ex + ex_out;
+        float* eye = reinterpret_cast<float*>(ex + ex_eye);
+        PrefillArgs b = a;
+        b.out = scratch; b.h0 = nullptr; b.hT = offs;
+        e = run_prefill_simt(b, reinterpret_cast<float*>(ws), Hg, stream);
+        if (!e) e = cudaMemsetAsync(v0, 0, (size_t)(T_total * H * dk * es), stream);
+        if (!e) e = launch_fill_identity(eye, B * H, (int)dk, stream);
+        if (!e) {
+            PrefillArgs m = a;
+            m.v = v0; m.dv = (int)dk; m.out = scratch; m.h0 = eye; m.hT = maps;
+            e = run_prefill_simt(m, reinterpret_cast<float*>(ws), Hg, stream);
+        }
+    }
     if (e) return from_cuda(e);
     if (debug_mode()) {
         int flag = 0;
@@ -365,6 +488,56 @@ kda_status_t kda_chunk_fwd(const void* q, const void* k, const void* v, const fl
 {
     return kda_chunk_fwd_ex(q, k, v, log_alpha, beta, h0, out, hT, cu_seqlens, B, T, H, dk, dv,
                             scale, io_dtype, KDA_PREFILL_AUTO, stream);
+}
+
+}  // extern "C"
+
+extern "C" {
+
+kda_status_t kda_chunk_fwd_segmap(const void* q, const void* k, const void* v,
+                                  const float* log_alpha, const float* beta, float* maps,
+                                  float* offs, const int32_t* cu_seqlens, int64_t B, int64_t T,
+                                  int64_t H, int64_t dk, int64_t dv, kda_io_dtype_t io_dtype,
+                                  cudaStream_t stream)
+{
+    if (maps == nullptr || offs == nullptr) return KDA_ERR_INVALID_ARG;
+    if (B < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (B > 0 && H > 0 && (cu_seqlens ? T : B * T) == 0) {
+        // no tokens: M = I, B = 0 for every sequence
+        if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+        if (!aligned16(maps) || !aligned16(offs)) return KDA_ERR_INVALID_ARG;
+        cudaError_t e = cudaMemsetAsync(offs, 0, (size_t)(B * H * dk * dv * 4), stream);
+        if (!e) e = launch_fill_identity(maps, B * H, (int)dk, stream);
+        return from_cuda(e);
+    }
+    return chunk_fwd_impl(q, k, v, log_alpha, beta, nullptr, nullptr, nullptr, nullptr, 0,
+                          cu_seqlens, B, T, H, dk, dv, 1.f, io_dtype, KDA_PREFILL_AUTO, false,
+                          stream, maps, offs);
+}
+
+kda_status_t kda_affine_prefix(const float* maps, const float* offs, const float* h0,
+                               float* out, int64_t nseg, int64_t NH, int64_t dk, int64_t dv,
+                               cudaStream_t stream)
+{
+    if (nseg < 0 || NH < 0) return KDA_ERR_INVALID_ARG;
+    if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (NH == 0) return KDA_OK;
+    if (NH > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+    if (out == nullptr || !aligned16(out)) return KDA_ERR_INVALID_ARG;
+    if (h0 && !aligned16(h0)) return KDA_ERR_INVALID_ARG;
+    if (nseg > 0) {
+        if (maps == nullptr || offs == nullptr || !aligned16(maps) || !aligned16(offs))
+            return KDA_ERR_INVALID_ARG;
+        if ((const void*)maps == (const void*)out || (const void*)offs == (const void*)out)
+            return KDA_ERR_INVALID_ARG;
+    }
+    PrefixArgs p;
+    std::memset(&p, 0, sizeof(p));
+    p.maps = maps; p.offs = offs; p.h0 = h0; p.starts = nullptr; p.out = out;
+    p.seg_off = nullptr; p.nseg = nseg; p.N = 1; p.H = NH; p.h_base = 0; p.hg = NH;
+    p.hstride = NH; p.abs_head = true; p.slots = nullptr; p.P = 0;
+    p.dk = (int)dk; p.dv = (int)dv; p.err = nullptr;
+    return from_cuda(launch_affine_prefix(p, stream));
 }
 
 }  // extern "C"

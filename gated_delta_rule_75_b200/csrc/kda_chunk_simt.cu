@@ -246,13 +246,16 @@ static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaS
     constexpr int C = kChunk;
     const size_t smem_prep = sizeof(float) * (size_t)(C * (3 * DK + DV) + 2 * C * C + C);
     const size_t smem_state = sizeof(float) * (size_t)(3 * C * DK + C * C + C * 32 + DK * 32 + DK);
-    cudaError_t e;
-    if ((e = cudaFuncSetAttribute(chunk_prep_simt_kernel<T, DK, DV>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_prep)))
-        return e;
-    if ((e = cudaFuncSetAttribute(chunk_state_simt_kernel<T, DK, DV>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state)))
-        return e;
+    static std::atomic<uint64_t> attrs_done{0};
+    cudaError_t e = once_per_device(attrs_done, [&] {
+        cudaError_t r = cudaFuncSetAttribute(chunk_prep_simt_kernel<T, DK, DV>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             (int)smem_prep);
+        if (r) return r;
+        return cudaFuncSetAttribute(chunk_state_simt_kernel<T, DK, DV>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_state);
+    });
+    if (e) return e;
     for (int64_t hb = 0; hb < a.H; hb += Hg) {
         const int64_t hg = (a.H - hb) < Hg ? (a.H - hb) : Hg;
         if (a.si.chunks_upper > 0) {

@@ -32,6 +32,8 @@
 //   the next chunk's e^{G_last} in TMEM.
 // Every mbarrier wait is bounded; on a timeout the CTA records it in the
 // workspace error word, drains its own copies and frees its TMEM.
+#include <cstring>
+
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_tma.cuh"
@@ -534,31 +536,58 @@ constexpr uint32_t S_SMEM = S_BYTES + 1024;
 
 constexpr int ST = 256;                                 // state-kernel threads
 
-template <bool kHasH0>
+// What one CTA walks (kMode):
+//   WALK_SEQ   a whole sequence from h0 (or zero): outputs and the final state;
+//   WALK_VALUE one segment from a zero state: its final state is the segment's
+//              offset B (no outputs);
+//   WALK_MAP   one segment from the identity, with V = 0 (no v loads, no
+//              V T'^T product): its final state is the segment's map M;
+//   WALK_FINAL one segment from its entry state (SegPlan::starts): outputs, and
+//              the final state when it is the sequence's last segment.
+enum { WALK_SEQ = 0, WALK_VALUE = 1, WALK_MAP = 2, WALK_FINAL = 3 };
+
+template <bool kHasH0, int kMode>
 __global__ void __launch_bounds__(ST, 1)
 chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constant__ CUtensorMap vmap,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, SeqInfo si, int64_t H, int64_t h_base, int64_t Hg,
-                      const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err)
+                      const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err,
+                      const __grid_constant__ SegPlan sp)
 {
+    constexpr bool kOut = kMode == WALK_SEQ || kMode == WALK_FINAL;   // outputs written
+    constexpr bool kV = kMode != WALK_MAP;                            // v tiles used
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t full[2], bar1, bar2;
     __shared__ uint32_t tmem_base;
 
-    // blocks run heads-innermost over sequences ranked longest first
+    // blocks run heads-innermost over sequences ranked longest first (or over
+    // segments in order)
     const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
-    const int64_t n = si.seq_of((int64_t)blockIdx.x / hg);
     const int hl = (int)((int64_t)blockIdx.x % hg);
     const int64_t h = h_base + hl;
+    int64_t n, g = 0, sg = 0, nsg = 1;
+    if constexpr (kMode == WALK_SEQ) {
+        n = si.seq_of((int64_t)blockIdx.x / hg);
+    } else {
+        g = (int64_t)blockIdx.x / hg;
+        if (!sp.locate(g, si.N, n, sg, nsg)) return;
+    }
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
-    const int sp = w & 3, half = w >> 2;                // TMEM lane quarter, column half
-    const int j = 32 * sp + l;                          // dv index = TMEM lane
+    const int qt = w & 3, half = w >> 2;                // TMEM lane quarter, column half
+    const int j = 32 * qt + l;                          // dv index = TMEM lane
     int64_t bos, eos;
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
-    const int64_t nch = si.chunk_count(n, eos - bos);
-    const int64_t gc0 = si.chunk_start(n);
+    int64_t nch = si.chunk_count(n, eos - bos);
+    int64_t gc0 = si.chunk_start(n);
+    if constexpr (kMode != WALK_SEQ) {                  // this segment's chunks
+        const int64_t c0 = sg * sp.len;
+        nch -= c0;
+        nch = nch < 0 ? 0 : (nch > sp.len ? sp.len : nch);
+        gc0 += c0;
+        bos += c0 * C;
+    }
     // state slot of this (sequence, head); -1: none (zero start, nothing stored)
     int64_t sidx = n * H + h;
     if (slots) {
@@ -566,23 +595,41 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
         if (sl >= P && tid == 0 && err) atomicOr(err, 1);
     }
-    const float* h0p = (kHasH0 && sidx >= 0) ? h0 + sidx * (int64_t)D * D : nullptr;
-    float* hTp = (hT && sidx >= 0) ? hT + sidx * (int64_t)D * D : nullptr;
+    const int64_t sbuf = (g * sp.hstride + (sp.abs_head ? h : (int64_t)hl)) * (int64_t)D * D;
+    const float* h0p = nullptr;
+    float* hTp = nullptr;
+    if constexpr (kMode == WALK_SEQ) {
+        h0p = (kHasH0 && sidx >= 0) ? h0 + sidx * (int64_t)D * D : nullptr;
+        hTp = (hT && sidx >= 0) ? hT + sidx * (int64_t)D * D : nullptr;
+    } else if constexpr (kMode == WALK_VALUE) {
+        hTp = sp.offs + sbuf;
+    } else if constexpr (kMode == WALK_MAP) {
+        hTp = sp.maps + sbuf;
+    } else {
+        h0p = sp.starts + sbuf;
+        hTp = (sg + 1 == nsg && hT && sidx >= 0) ? hT + sidx * (int64_t)D * D : nullptr;
+    }
+    // entry state element (row c of S, column j)
+    auto s_init = [&](int c) -> float {
+        if constexpr (kMode == WALK_MAP) return c == j ? 1.f : 0.f;
+        else return h0p ? h0p[c * D + j] : 0.f;
+    };
 
-    if (nch == 0) {                                      // empty sequence: hT = h0
+    if (nch == 0) {                                      // nothing to walk: final = entry state
         if (hTp)
-            for (int c = 64 * half; c < 64 * half + 64; ++c)
-                hTp[c * D + j] = h0p ? h0p[c * D + j] : 0.f;
+            for (int c = 64 * half; c < 64 * half + 64; ++c) hTp[c * D + j] = s_init(c);
         return;
     }
     auto load_stage = [&](int64_t ch, int s) {          // one thread
         unsigned char* st = sm + s * STAGE_BYTES;
         fence_smem_to_async();
-        tma::expect_tx(&full[s], IMG_BYTES + 16384);
+        tma::expect_tx(&full[s], kV ? IMG_BYTES + 16384 : IMG_BYTES);
         tma::load_bulk(st, ws + ((gc0 + ch) * Hg + hl) * (int64_t)IMG_BYTES, IMG_BYTES, &full[s]);
-        const int32_t y = (int32_t)(bos + ch * C), x = (int32_t)(h * D);
-        tma::load_2d(st + STAGE_V, &vmap, x, y, &full[s]);
-        tma::load_2d(st + STAGE_V + 8192, &vmap, x + 64, y, &full[s]);
+        if constexpr (kV) {
+            const int32_t y = (int32_t)(bos + ch * C), x = (int32_t)(h * D);
+            tma::load_2d(st + STAGE_V, &vmap, x, y, &full[s]);
+            tma::load_2d(st + STAGE_V + 8192, &vmap, x + 64, y, &full[s]);
+        }
     };
 
     if (tid == 0) {
@@ -597,7 +644,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
-    const uint32_t lane = (uint32_t)(32 * sp) << 16;
+    const uint32_t lane = (uint32_t)(32 * qt) << 16;
     const uint32_t tU = tmem, tS = tmem + 256;
     auto tO = [&](int64_t ch) { return tmem + 64 + 64 * (uint32_t)(ch & 1); };
     bool pending[2] = {true, nch > 1};
@@ -606,18 +653,22 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     auto issue_mma1 = [&](int64_t ch) {
         unsigned char* st = sm + (ch & 1) * STAGE_BYTES;
         fence_after_sync();
-        const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
+        if constexpr (kV) {
+            const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
-        for (int ks = 0; ks < 4; ++ks)
-            mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
-                     make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
+            for (int ks = 0; ks < 4; ++ks)
+                mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
+                         make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
+        }
         const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
         const uint32_t to = tO(ch);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks) {
             const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
-            mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, 1u);
-            mma_bf16(to, ad, make_desc(smem_u32(st + IMG_QG + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, ks > 0);
+            mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1,
+                     (kV || ks > 0) ? 1u : 0u);
+            if constexpr (kOut)
+                mma_bf16(to, ad, make_desc(smem_u32(st + IMG_QG + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, ks > 0);
         }
         commit(&bar1);
     };
@@ -635,7 +686,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             const int c0 = 64 * half + 16 * cb;
             float f[16];
 #pragma unroll
-            for (int x = 0; x < 16; ++x) f[x] = h0p ? h0p[(c0 + x) * D + j] : 0.f;
+            for (int x = 0; x < 16; ++x) f[x] = s_init(c0 + x);
             *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f);
             *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f + 8);
 #pragma unroll
@@ -685,7 +736,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const uint64_t ad = make_desc(smem_u32(sm + S_UBF + ks * 32), 16, 1024);
-                mma_bf16(tO(ch), ad, make_desc(smem_u32(st + IMG_B2 + ks * 2048), 8192, 1024), idO, 1u);
+                if constexpr (kOut)
+                    mma_bf16(tO(ch), ad, make_desc(smem_u32(st + IMG_B2 + ks * 2048), 8192, 1024), idO, 1u);
                 mma_bf16(tS, ad, make_desc(smem_u32(st + IMG_B2 + 8192 + ks * 2048), 8192, 1024), idS, 1u);
             }
             commit(&bar2);
@@ -741,7 +793,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         if (!last && tid == 0) issue_mma1(ch + 1);     // overlaps the output write below
 
         // output rows of this chunk: tokens 32*half .. +31 of column j
-        {
+        if constexpr (kOut) {
             float f[2][16];
             tmem_ld16(tO(ch) + lane + 32 * half, f[0]);
             tmem_ld16(tO(ch) + lane + 32 * half + 16, f[1]);
@@ -774,22 +826,37 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 
 int64_t tc_ws_bytes_per_chunk() { return tc::IMG_BYTES; }
 
+int64_t tc_seg_bytes_per_head(const SegPlan& p)
+{
+    return p.len > 0 ? p.upper * 3 * (int64_t)tc::D * tc::D * (int64_t)sizeof(float) : 0;
+}
+
+template <bool kHasH0, int kMode>
+static cudaError_t set_state_smem()
+{
+    return cudaFuncSetAttribute(tc::chunk_state_tc_kernel<kHasH0, kMode>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::S_SMEM);
+}
+
 cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, int* err,
                            cudaStream_t st)
 {
-    cudaError_t e;
-    if ((e = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
-        return e;
-    if ((e = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
-        return e;
-    if ((e = cudaFuncSetAttribute(tc::chunk_state_tc_kernel<true>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::S_SMEM)))
-        return e;
-    if ((e = cudaFuncSetAttribute(tc::chunk_state_tc_kernel<false>,
-                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::S_SMEM)))
-        return e;
+    static std::atomic<uint64_t> attrs_done{0};
+    cudaError_t e = once_per_device(attrs_done, [] {
+        cudaError_t r;
+        if ((r = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<false>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
+            return r;
+        if ((r = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<true>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
+            return r;
+        if ((r = set_state_smem<true, tc::WALK_SEQ>())) return r;
+        if ((r = set_state_smem<false, tc::WALK_SEQ>())) return r;
+        if ((r = set_state_smem<false, tc::WALK_VALUE>())) return r;
+        if ((r = set_state_smem<false, tc::WALK_MAP>())) return r;
+        return set_state_smem<false, tc::WALK_FINAL>();
+    });
+    if (e) return e;
     // [tokens][H * d] views of the inputs; rows past the end read as zeros
     const uint64_t rows = (uint64_t)a.si.T_total, cols = (uint64_t)a.H * tc::D;
     tc::PrepMaps maps;
@@ -813,22 +880,70 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
                 maps, a.beta, nullptr, a.si, a.H, hb, Hg, a.scale, w, err);
         return cudaGetLastError();
     };
+    SegPlan none;
+    memset(&none, 0, sizeof(none));
     auto launch_state = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
         dim3 gs((unsigned)(a.si.N * hg));
         LaunchScope scope(s, K_STATE_TC);
         if (a.h0)
-            tc::chunk_state_tc_kernel<true><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err);
+            tc::chunk_state_tc_kernel<true, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
         else
-            tc::chunk_state_tc_kernel<false><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err);
+            tc::chunk_state_tc_kernel<false, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
         return cudaGetLastError();
     };
+    // one walk over every segment of the plan (grid: segment bound x heads)
+    auto launch_walk = [&](int mode, const SegPlan& sp, int64_t hb, int64_t hg, unsigned char* w,
+                           cudaStream_t s) -> cudaError_t {
+        if (sp.upper <= 0) return cudaSuccess;
+        dim3 gs((unsigned)(sp.upper * hg));
+        LaunchScope scope(s, mode == tc::WALK_FINAL ? K_STATE_TC : K_STATE_SEG_TC);
+        __nv_bfloat16* o = (__nv_bfloat16*)a.out;
+        if (mode == tc::WALK_VALUE)
+            tc::chunk_state_tc_kernel<false, tc::WALK_VALUE><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+        else if (mode == tc::WALK_MAP)
+            tc::chunk_state_tc_kernel<false, tc::WALK_MAP><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+        else
+            tc::chunk_state_tc_kernel<false, tc::WALK_FINAL><<<gs, tc::ST, tc::S_SMEM, s>>>(
+                w, vmap, nullptr, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+        return cudaGetLastError();
+    };
+
+    // segment buffers sit after the operand images of one head group
+    SegPlan sp = a.seg;
+    if (a.tc_what == 0 && sp.len > 0) {
+        const int64_t mat = (int64_t)tc::D * tc::D;
+        float* segbuf = reinterpret_cast<float*>(
+            ws + Hg * (a.si.chunks_upper > 0 ? a.si.chunks_upper : 1) * (int64_t)tc::IMG_BYTES);
+        sp.maps = segbuf;
+        sp.offs = segbuf + sp.upper * Hg * mat;
+        sp.starts = segbuf + 2 * sp.upper * Hg * mat;
+        sp.hstride = Hg;
+        sp.abs_head = false;
+    }
 
     for (int64_t hb = 0; hb < a.H; hb += Hg) {
         const int64_t hg = (a.H - hb) < Hg ? (a.H - hb) : Hg;
         if ((e = launch_prep(hb, hg, ws, st))) return e;
-        if ((e = launch_state(hb, hg, ws, st))) return e;
+        if (a.tc_what == 1) {                  // each sequence's (M, B) into the caller's buffers
+            if ((e = launch_walk(tc::WALK_VALUE, sp, hb, hg, ws, st))) return e;
+            if ((e = launch_walk(tc::WALK_MAP, sp, hb, hg, ws, st))) return e;
+        } else if (sp.len > 0) {               // segment-parallel walk
+            if ((e = launch_walk(tc::WALK_VALUE, sp, hb, hg, ws, st))) return e;
+            if ((e = launch_walk(tc::WALK_MAP, sp, hb, hg, ws, st))) return e;
+            PrefixArgs pa;
+            pa.maps = sp.maps; pa.offs = sp.offs; pa.h0 = a.h0; pa.starts = sp.starts;
+            pa.out = nullptr; pa.seg_off = sp.seg_off; pa.nseg = sp.nseg; pa.N = a.si.N;
+            pa.H = a.H; pa.h_base = hb; pa.hg = hg; pa.hstride = Hg; pa.abs_head = false;
+            pa.slots = a.slots; pa.P = a.P; pa.dk = tc::D; pa.dv = tc::D; pa.err = err;
+            if ((e = launch_affine_prefix(pa, st))) return e;
+            if ((e = launch_walk(tc::WALK_FINAL, sp, hb, hg, ws, st))) return e;
+        } else {
+            if ((e = launch_state(hb, hg, ws, st))) return e;
+        }
     }
     return cudaSuccess;
 }

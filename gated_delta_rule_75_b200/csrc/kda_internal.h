@@ -3,6 +3,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 #include "kda.h"
 
 namespace kda {
@@ -72,6 +74,51 @@ struct SeqInfo {
 #endif
 };
 
+// Segment-parallel walk of the state chains (tensor-core path).  The chunks of
+// each sequence are cut into segments of `len` chunks.  A segment maps its
+// entry state affinely, S -> M S + B, so each segment's M (walk from the
+// identity with V = 0) and B (walk from zero) are computed independently, the
+// entry states follow from a short sequential composition, and a last walk per
+// segment writes the outputs.  Buffers hold one dk x dk (maps) or dk x dv
+// (offs, starts) fp32 matrix per (segment, head), at (g * hstride + head) where
+// head is the index within the head group (or the absolute head when
+// abs_head is set).
+struct SegPlan {
+    int64_t len;              // chunks per segment; 0: segmentation off
+    int64_t nseg;             // segments per sequence (fixed-length batches)
+    int64_t upper;            // bound on the number of segments (grid, buffers)
+    const int64_t* seg_off;   // device [N+1]: first segment of each sequence (packed), or nullptr
+    float* maps;
+    float* offs;
+    float* starts;
+    int64_t hstride;
+    bool abs_head;
+
+#ifdef __CUDACC__
+    // Segment g -> (sequence n, index s within it, segments of n); false past the end.
+    __device__ __forceinline__ bool locate(int64_t g, int64_t N, int64_t& n, int64_t& s,
+                                           int64_t& count) const {
+        if (seg_off == nullptr) {
+            n = g / nseg;
+            if (n >= N) return false;
+            s = g - n * nseg;
+            count = nseg;
+            return true;
+        }
+        if (g >= seg_off[N]) return false;
+        int64_t lo = 0, hi = N;                  // seg_off[lo] <= g < seg_off[hi]
+        while (hi - lo > 1) {
+            const int64_t mid = (lo + hi) >> 1;
+            if (seg_off[mid] <= g) lo = mid; else hi = mid;
+        }
+        n = lo;
+        s = g - seg_off[n];
+        count = seg_off[n + 1] - seg_off[n];
+        return true;
+    }
+#endif
+};
+
 struct PrefillArgs {
     const void* q;
     const void* k;
@@ -95,6 +142,12 @@ struct PrefillArgs {
     // Gated DeltaNet form: one gate per (token, head), log_alpha [.., H],
     // broadcast over the key channels
     bool gate_scalar;
+    // tensor-core path: segment-parallel state walk (len == 0: one chain per
+    // (sequence, head)); the buffers are placed by run_prefill_tc
+    SegPlan seg;
+    // what the tensor-core state walks produce: outputs and final states (0),
+    // or only each sequence's affine map, into seg.maps / seg.offs (1)
+    int tc_what;
 
 #ifdef __CUDACC__
     // Flat (slot, head) index of sequence n's state, or -1 when it has none.
@@ -128,6 +181,22 @@ struct DecodeArgs {
     bool gate_scalar;        // log_alpha [N, H] (one gate per head) instead of [N, H, dk]
 };
 
+// Runs `f` (a per-device setup such as raising a kernel's shared-memory
+// limit) once per device: the bit of the current device in `done` is set after
+// the first success.  Devices past 63 run it every time.
+template <typename F>
+inline cudaError_t once_per_device(std::atomic<uint64_t>& done, F f)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = (dev >= 0 && dev < 64) ? (uint64_t(1) << dev) : 0;
+    if (bit && (done.load(std::memory_order_acquire) & bit)) return cudaSuccess;
+    e = f();
+    if (e == cudaSuccess && bit) done.fetch_or(bit, std::memory_order_release);
+    return e;
+}
+
 // Kernel identities for launch counting and timing (kda_profiler.cu).
 enum KernelId {
     K_CHUNK_OFFSETS = 0,
@@ -136,6 +205,9 @@ enum KernelId {
     K_DECODE,
     K_PREP_TC,
     K_STATE_TC,
+    K_STATE_SEG_TC,
+    K_AFFINE_PREFIX,
+    K_FILL,
     K_KERNEL_COUNT
 };
 
@@ -164,6 +236,8 @@ cudaError_t run_prefill_simt(const PrefillArgs& a, float* ws, int64_t Hg, cudaSt
 
 // kda_chunk_tc.cu (bf16, dk = dv = 128)
 int64_t tc_ws_bytes_per_chunk();
+// Workspace bytes per head for the segment buffers of a plan.
+int64_t tc_seg_bytes_per_head(const SegPlan& p);
 cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, int* err,
                            cudaStream_t st);
 
@@ -172,10 +246,35 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
 constexpr int kErrSeqlens = 1 << 0;
 constexpr int kErrTimeoutMask = 0x3e;
 
-// kda_seqinfo.cu
+// kda_seqinfo.cu.  With seg_off set, also the first segment of each sequence
+// for segments of seg_len chunks (at least one per sequence), capped at seg_cap.
 cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
                                  int64_t* chunk_off, int32_t* order, int* err_flag,
+                                 int64_t seg_len, int64_t seg_cap, int64_t* seg_off,
                                  cudaStream_t st);
+
+// kda_segscan.cu.  Entry states of consecutive segments: for every chain
+// (sequence n, head h of the group h_base .. h_base + hg - 1) with segments
+// s = 0 .. count-1 (count from seg_off, else nseg), X_0 = h0 (or zero),
+// X_{s+1} = M_s X_s + B_s.  starts (nullable) receives every X_s, out
+// (nullable) the state after the last segment at the chain's state index.
+struct PrefixArgs {
+    const float* maps;       // [(base(n) + s) * hstride + head][dk][dk]
+    const float* offs;       // [(base(n) + s) * hstride + head][dk][dv]
+    const float* h0;         // nullable; at the chain's state index
+    float* starts;           // nullable; indexed like offs
+    float* out;              // nullable; at the chain's state index
+    const int64_t* seg_off;  // nullable: nseg segments per sequence
+    int64_t nseg, N, H, h_base, hg, hstride;
+    bool abs_head;           // buffer head index = h (else h - h_base)
+    const int32_t* slots;    // pooled states, as in PrefillArgs
+    int64_t P;
+    int dk, dv;
+    int* err;
+};
+cudaError_t launch_affine_prefix(const PrefixArgs& p, cudaStream_t st);
+// count consecutive d x d identity matrices at dst.
+cudaError_t launch_fill_identity(float* dst, int64_t count, int d, cudaStream_t st);
 // Sequences are ranked by length (for `order`) when there are at most this many.
 constexpr int64_t kMaxOrderedSeqs = 2048;
 

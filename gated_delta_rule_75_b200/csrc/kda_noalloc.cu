@@ -125,7 +125,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 256);
         if (launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, nullptr,
-                                 err_flag, stream) != cudaSuccess)
+                                 err_flag, 0, 0, nullptr, stream) != cudaSuccess)
             return KDA_ERR_CUDA;
         si.chunk_off = chunk_off;
     }

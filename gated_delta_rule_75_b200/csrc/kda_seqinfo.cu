@@ -7,6 +7,11 @@
 // here: cu[0] == 0, non-decreasing, cu[N] == T; bit 0 of *err_flag is set
 // otherwise) the cap keeps every chunk index the later kernels derive inside
 // the workspace, so a malformed array cannot cause an out-of-bounds access.
+//
+// For the segment-parallel state walk it also writes seg_off[n], the first
+// segment of sequence n when every sequence's chunk slots are cut into
+// segments of seg_len chunks (an empty sequence still gets one segment, which
+// carries its initial state through), capped at seg_cap like the chunk offsets.
 #include <cub/block/block_scan.cuh>
 
 #include "kda_common.cuh"
@@ -19,7 +24,8 @@ constexpr int kScanThreads = 1024;
 __global__ void __launch_bounds__(kScanThreads)
 chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total, int64_t cap,
                      int64_t* __restrict__ chunk_off, int32_t* __restrict__ order,
-                     int* __restrict__ err)
+                     int* __restrict__ err, int64_t seg_len, int64_t seg_cap,
+                     int64_t* __restrict__ seg_off)
 {
     using Scan = cub::BlockScan<int64_t, kScanThreads>;
     __shared__ typename Scan::TempStorage tmp;
@@ -49,6 +55,26 @@ chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
         if (carry > cap) atomicOr(err, 1);
         chunk_off[N] = carry < cap ? carry : cap;
     }
+    if (seg_off != nullptr) {
+        __syncthreads();
+        if (threadIdx.x == 0) carry = 0;
+        __syncthreads();
+        for (int64_t base = 0; base < N; base += kScanThreads) {
+            const int64_t n = base + threadIdx.x;
+            int64_t ns = 0;
+            if (n < N) {
+                const int64_t c = chunk_off[n + 1] - chunk_off[n];
+                ns = c > 0 ? (c + seg_len - 1) / seg_len : 1;
+            }
+            int64_t excl, total;
+            Scan(tmp).ExclusiveSum(ns, excl, total);
+            if (n < N) seg_off[n] = (carry + excl) < seg_cap ? (carry + excl) : seg_cap;
+            __syncthreads();
+            if (threadIdx.x == 0) carry += total;
+            __syncthreads();
+        }
+        if (threadIdx.x == 0) seg_off[N] = carry < seg_cap ? carry : seg_cap;
+    }
     if (order == nullptr) return;
     // rank sequences by chunk count, longest first (ties: lower index first):
     // order[rank] = sequence
@@ -66,11 +92,13 @@ chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
 
 cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, int64_t cap,
                                  int64_t* chunk_off, int32_t* order, int* err_flag,
+                                 int64_t seg_len, int64_t seg_cap, int64_t* seg_off,
                                  cudaStream_t st)
 {
+    if (seg_off != nullptr && seg_len < 1) return cudaErrorInvalidValue;
     LaunchScope scope(st, K_CHUNK_OFFSETS);
     chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, cap, chunk_off, order,
-                                                     err_flag);
+                                                     err_flag, seg_len, seg_cap, seg_off);
     return cudaGetLastError();
 }
 

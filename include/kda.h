@@ -68,10 +68,22 @@ typedef enum {
     KDA_IO_BF16 = 1            /* q, k, v, out are bf16 (gates, beta and states stay fp32) */
 } kda_io_dtype_t;
 
+/*
+ * Tensor-core state walk.  Each (sequence, head) pair is a sequential chain of
+ * chunks.  When there are too few chains to fill the GPU (few sequences and
+ * heads), the library cuts every chain into segments that are walked in
+ * parallel: a segment maps its entry state affinely (S -> M S + B, the
+ * recurrence being linear in S), so each segment's M and B are computed
+ * independently, the entry states follow from a short composition, and a last
+ * parallel walk writes the outputs.  AUTO and TENSORCORE choose between the
+ * two by the chain count; the last two values force one or the other.
+ */
 typedef enum {
     KDA_PREFILL_AUTO = 0,      /* tensor cores for bf16 with dk = dv = 128, SIMT otherwise */
     KDA_PREFILL_SIMT = 1,      /* fp32 SIMT chunk kernels (any supported shape / dtype) */
-    KDA_PREFILL_TENSORCORE = 2 /* tcgen05 chunk kernels; bf16, dk = dv = 128 only */
+    KDA_PREFILL_TENSORCORE = 2, /* tcgen05 chunk kernels; bf16, dk = dv = 128 only */
+    KDA_PREFILL_TENSORCORE_CHAIN = 3,     /* tcgen05, one chain per (sequence, head) */
+    KDA_PREFILL_TENSORCORE_SEGMENTED = 4  /* tcgen05, segment-parallel walk */
 } kda_prefill_impl_t;
 
 /*
@@ -259,6 +271,54 @@ KDA_API kda_status_t kda_recurrent_step_slots(const void* q, const void* k, cons
                                               int64_t N, int64_t P, int64_t H, int64_t dk,
                                               int64_t dv, float scale, kda_io_dtype_t io_dtype,
                                               cudaStream_t stream);
+
+/*
+ * Context parallelism: one long sequence split across GPUs (or across calls).
+ *
+ * The recurrence is linear in the state, so a run of tokens maps any entry
+ * state S to M S + B (M: dk x dk, B: dk x dv).  Splitting a sequence into
+ * consecutive pieces, each holder computes its piece's (M, B); the entry state
+ * of piece r is then the composition of pieces 0 .. r-1 applied to h0, and a
+ * plain kda_chunk_fwd of piece r from that state gives exactly the outputs and
+ * final state of the unsplit sequence (up to rounding).  The pages run the
+ * method at contexts of about a million tokens ("Kimi Linear acaba de superar
+ * a la atencion completa en sus propios terminos", sections on decode timing
+ * at 1M tokens and on the open release); the split itself is not on the pages
+ * and follows from the linearity of the step.  The exchange between GPUs is
+ * left to the caller (an all-gather of (M, B), 2 * 64 KiB per head at d = 128).
+ *
+ * kda_chunk_fwd_segmap -- (M, B) of every (sequence, head) of a prefill input.
+ *  q, k, v, log_alpha, beta, cu_seqlens, B, T, H, dk, dv, io_dtype: as for
+ *              kda_chunk_fwd (no output, no scale)
+ *  maps        [N, H, dk, dk] fp32, written: M of each (sequence, head)
+ *  offs        [N, H, dk, dv] fp32, written: B (the final state from a zero
+ *              entry state)
+ *  Both 16-byte aligned, not aliasing the inputs.  An empty sequence gives
+ *  M = I, B = 0.  bf16 with dk = dv = 128 runs on the tensor cores (M and B
+ *  carry the bf16-operand rounding of that path), anything else on the fp32
+ *  SIMT kernels.  Allocates workspace like kda_chunk_fwd.
+ *
+ * kda_affine_prefix -- apply nseg consecutive maps to initial states.
+ *  maps        [nseg, NH, dk, dk] fp32 (segment-major: segment s of chain i
+ *              at s * NH + i)
+ *  offs        [nseg, NH, dk, dv] fp32
+ *  h0          [NH, dk, dv] fp32, or NULL for zeros
+ *  out         [NH, dk, dv] fp32, written: M_{nseg-1}(...(M_0 h0 + B_0)...) +
+ *              B_{nseg-1}; may alias h0, must not alias maps or offs.
+ *  nseg = 0 copies h0 (or zeros).  fp32 FMA arithmetic on the device; all
+ *  pointers 16-byte aligned; dk, dv in {64, 128}.  Allocates nothing.
+ */
+KDA_API kda_status_t kda_chunk_fwd_segmap(const void* q, const void* k, const void* v,
+                                          const float* log_alpha, const float* beta,
+                                          float* maps, float* offs,
+                                          const int32_t* cu_seqlens,
+                                          int64_t B, int64_t T, int64_t H, int64_t dk,
+                                          int64_t dv, kda_io_dtype_t io_dtype,
+                                          cudaStream_t stream);
+
+KDA_API kda_status_t kda_affine_prefix(const float* maps, const float* offs, const float* h0,
+                                       float* out, int64_t nseg, int64_t NH, int64_t dk,
+                                       int64_t dv, cudaStream_t stream);
 
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char* kda_status_string(kda_status_t status);

@@ -11,6 +11,12 @@ read with the values the GPU sees):
   section "Como funciona Kimi Delta Attention paso a paso": decay, predict,
   beta-scaled error, correct, read).
 * :func:`step` -- one decode step, state updated in place (same update, one token).
+* :func:`segment_map` -- the affine map S -> M S + B of a run of tokens.  The
+  step is linear in S, so M is the state that the same tokens reach from the
+  identity with zero values and B the state they reach from zero; both are
+  computed with :func:`fwd`.  (The pages do not state this split; it follows
+  from the step's linearity and is pinned against dense transition products.)
+* :func:`compose` -- X_r of consecutive maps: X_0 = h0, X_{s+1} = M_s X_s + B_s.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, reductions to simpler published rules and brute-force matrix products.
@@ -110,6 +116,31 @@ def step(q, k, v, log_alpha, beta, state, scale):
     if rc != 0:
         raise RuntimeError(f"oracle failed rc={rc}")
     return out, S
+
+
+def segment_map(q, k, v, log_alpha, beta, cu_seqlens=None):
+    """(M [N,H,dk,dk], B [N,H,dk,dv]) of every (sequence, head): for any entry
+    state S0 the state after the tokens is M @ S0 + B.  Inputs as for fwd."""
+    q, k, v, g, b = (_f64(x) for x in (q, k, v, log_alpha, beta))
+    dk = q.shape[-1]
+    N = q.shape[0] if cu_seqlens is None else len(np.asarray(
+        cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens)) - 1
+    H = q.shape[2]
+    _, Bm = fwd(q, k, v, g, b, 1.0, h0=None, cu_seqlens=cu_seqlens)
+    eye = np.broadcast_to(np.eye(dk), (N, H, dk, dk)).copy()
+    v0 = np.zeros(q.shape[:3] + (dk,))
+    _, M = fwd(q, k, v0, g, b, 1.0, h0=eye, cu_seqlens=cu_seqlens)
+    return M, Bm
+
+
+def compose(maps, offs, h0=None):
+    """State after applying maps[0], maps[1], ... in order to h0 (zeros if None):
+    X <- maps[s] @ X + offs[s].  maps [S,...,dk,dk], offs [S,...,dk,dv]."""
+    maps, offs = _f64(maps), _f64(offs)
+    X = np.zeros(offs.shape[1:]) if h0 is None else _f64(h0).copy()
+    for s in range(maps.shape[0]):
+        X = maps[s] @ X + offs[s]
+    return X
 
 
 def rel_l2(x, ref):

@@ -98,3 +98,82 @@ def test_partitions():
     assert a == [[0, 1], [2, 3]]          # loads 101 and 100
     with pytest.raises(ValueError):
         head_range(4, 2, 2)
+
+
+class _OracleOps:
+    """Per-rank compute of the context-parallel split done by the fp64 oracle
+    (CPU), so the gloo test checks the orchestration: pieces, exchange order,
+    composition."""
+
+    def segmap(self, q, k, v, g, b):
+        import oracle
+        M, Bm = oracle.segment_map(q, k, v, g, b)
+        return torch.from_numpy(M), torch.from_numpy(Bm)
+
+    def prefix(self, maps, offs, h0):
+        import oracle
+        return torch.from_numpy(oracle.compose(maps, offs, h0))
+
+    def forward(self, q, k, v, g, b, scale, h0):
+        import oracle
+        out, hT = oracle.fwd(q, k, v, g, b, scale, h0=h0)
+        return torch.from_numpy(out), torch.from_numpy(hT)
+
+
+def _cp_worker(rank, world, port, result_q):
+    import sys
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        import oracle
+        import workloads as W
+        from gated_delta_rule_75_b200.context_parallel import (chunk_fwd_context_parallel,
+                                                               token_range)
+        cfg = W.small_prefill(B=2, T=150, H=2, dk=8, dv=6, io_dtype="f32", seed=9, h0_std=0.1)
+        inp = W.make_prefill(cfg, "cpu")
+        t0, t1 = token_range(150, world, rank, align=16)
+        sl = lambda x: x[:, t0:t1].contiguous()
+        out, hT = chunk_fwd_context_parallel(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]),
+                                             sl(inp["log_alpha"]), sl(inp["beta"]), inp["scale"],
+                                             h0=inp["h0"], ops=_OracleOps())
+        full_out, full_hT = oracle.fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
+                                       inp["beta"], inp["scale"], h0=inp["h0"])
+        ok = np.allclose(out.numpy(), full_out[:, t0:t1], rtol=0, atol=1e-11)
+        if rank == world - 1:
+            ok &= np.allclose(hT.numpy(), full_hT, rtol=0, atol=1e-11)
+        result_q.put((rank, bool(ok)))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_context_parallel_gloo(world):
+    """A sequence split across `world` ranks reproduces the single-pass
+    outputs and final state (compute by the oracle, exchange over gloo)."""
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_cp_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(timeout=120)
+    codes = [p.exitcode for p in procs]
+    results = dict(q.get(timeout=5) for _ in range(world))
+    assert codes == [0] * world, codes
+    assert results == {r: True for r in range(world)}, results
+
+
+def test_token_range():
+    from gated_delta_rule_75_b200.context_parallel import token_range
+    for T in (0, 1, 63, 64, 150, 4096, 4097):
+        for world in (1, 2, 3, 8):
+            rs = [token_range(T, world, r) for r in range(world)]
+            assert rs[0][0] == 0 and rs[-1][1] == T
+            assert all(rs[i][1] == rs[i + 1][0] for i in range(world - 1))
+            assert all(a % 64 == 0 or a == T for a, _ in rs)
+    with pytest.raises(ValueError):
+        token_range(10, 2, 2)

@@ -339,3 +339,54 @@ def test_rel_l2_metric():
     a = np.array([3.0, 4.0])
     assert oracle.rel_l2(a, a) == 0.0
     assert math.isclose(oracle.rel_l2(np.array([3.0, 4.0 + 0.5]), a), 0.1, rel_tol=1e-15)
+
+
+# --------------------------------------------------------------------------
+# P-affine: segment maps (context parallelism) from the linearity of the step
+# --------------------------------------------------------------------------
+def test_segment_map_is_dense_transition_product():
+    """oracle.segment_map gives M = M_T..M_1 and B = sum_t M_T..M_{t+1} b_t k_t v_t^T
+    with the dense M_t = (I - b_t k_t k_t^T) Diag(alpha_t): a map built with the
+    wrong start (not the identity), with the values left in, or transposed
+    disagrees."""
+    rng = np.random.default_rng(21)
+    N, T, H, dk, dv = 2, 9, 2, 6, 4
+    q, k, v, g, b, _, cu = _rand_inputs(rng, N, T, H, dk, dv, unit_keys=False)
+    M, Bm = oracle.segment_map(q, k, v, g, b, cu_seqlens=cu)
+    for n in range(N):
+        for h in range(H):
+            P = np.eye(dk)
+            Bref = np.zeros((dk, dv))
+            for t in range(cu[n], cu[n + 1]):
+                kt = k[0, t, h][:, None]
+                Mt = (np.eye(dk) - b[0, t, h] * kt @ kt.T) @ np.diag(np.exp(g[0, t, h]))
+                P = Mt @ P
+                Bref = Mt @ Bref + b[0, t, h] * np.outer(k[0, t, h], v[0, t, h])
+            np.testing.assert_allclose(M[n, h], P, rtol=0, atol=1e-13)
+            np.testing.assert_allclose(Bm[n, h], Bref, rtol=0, atol=1e-13)
+    assert not np.allclose(M[0, 0], M[0, 0].T)        # not symmetric: a transpose would show
+
+
+@pytest.mark.parametrize("cuts", [(0, 80), (17, 80), (64, 128), (1, 2, 79)])
+def test_composed_segment_maps_reproduce_the_sequence(cuts):
+    """Pieces [c_i, c_{i+1}) run from the composed entry states give the
+    single-pass outputs and final state (what a context-parallel split returns)."""
+    rng = np.random.default_rng(22)
+    T, H, dk, dv, scale = 80, 2, 8, 6, 0.3
+    q, k, v, g, b, h0, _ = _rand_inputs(rng, 1, T, H, dk, dv)
+    out, hT = oracle.fwd(q, k, v, g, b, scale, h0=h0)
+    bounds = sorted(set((0,) + tuple(cuts) + (T,)))
+    sl = lambda x, a, c: x[:, a:c]
+    pieces = list(zip(bounds[:-1], bounds[1:]))
+    maps, offs = zip(*(oracle.segment_map(sl(q, a, c), sl(k, a, c), sl(v, a, c), sl(g, a, c),
+                                          sl(b, a, c)) for a, c in pieces))
+    outs = []
+    for r, (a, c) in enumerate(pieces):
+        X = oracle.compose(np.stack(maps[:r]), np.stack(offs[:r]), h0) if r else h0
+        o, S = oracle.fwd(sl(q, a, c), sl(k, a, c), sl(v, a, c), sl(g, a, c), sl(b, a, c),
+                          scale, h0=X)
+        outs.append(o)
+    np.testing.assert_allclose(np.concatenate(outs, axis=1), out, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(S, hT, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(oracle.compose(np.stack(maps), np.stack(offs), h0), hT,
+                               rtol=0, atol=1e-12)
