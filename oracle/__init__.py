@@ -17,6 +17,12 @@ read with the values the GPU sees):
   computed with :func:`fwd`.  (The pages do not state this split; it follows
   from the step's linearity and is pinned against dense transition products.)
 * :func:`compose` -- X_r of consecutive maps: X_0 = h0, X_{s+1} = M_s X_s + B_s.
+* :func:`bwd`  -- gradients of sum(dout * out) + sum(dhT * hT) with respect to
+  q, k, v, log_alpha, beta and h0: reverse-mode differentiation of the same
+  per-token step, token by token backwards (the pages say the chunk algorithm
+  is what the method trains with; the gradient itself is not on the pages and
+  is pinned by finite differences and by torch autograd of a separately
+  written recurrence).
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, reductions to simpler published rules and brute-force matrix products.
@@ -44,6 +50,9 @@ def _load():
         lib.kda_oracle_step.argtypes = [dp, dp, dp, dp, dp, dp, dp,
                                         i64, i64, i64, i64, ctypes.c_double]
         lib.kda_oracle_step.restype = ctypes.c_int
+        lib.kda_oracle_bwd.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp, dp,
+                                       i64p, i64, i64, i64, i64, ctypes.c_double]
+        lib.kda_oracle_bwd.restype = ctypes.c_int
         lib.kda_oracle_threads.argtypes = []
         lib.kda_oracle_threads.restype = ctypes.c_int
         _lib = lib
@@ -116,6 +125,39 @@ def step(q, k, v, log_alpha, beta, state, scale):
     if rc != 0:
         raise RuntimeError(f"oracle failed rc={rc}")
     return out, S
+
+
+def bwd(q, k, v, log_alpha, beta, scale, dout, h0=None, dhT=None, cu_seqlens=None):
+    """fp64 gradients.  Shapes as for fwd; dout [B,T,H,dv]; dhT [N,H,dk,dv] or
+    None (zero).  Returns (dq, dk, dv, dlog_alpha, dbeta, dh0) as fp64 arrays."""
+    q, k, v, g, b, do = (_f64(x) for x in (q, k, v, log_alpha, beta, dout))
+    h0, dhT = _f64(h0), _f64(dhT)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    if cu_seqlens is None:
+        cu = np.arange(B + 1, dtype=np.int64) * T
+    else:
+        if B != 1:
+            raise ValueError("packed sequences need batch axis 1")
+        cu = np.ascontiguousarray(np.asarray(
+            cu_seqlens.cpu() if hasattr(cu_seqlens, "cpu") else cu_seqlens, dtype=np.int64))
+    N = cu.shape[0] - 1
+    if cu[0] != 0 or cu[-1] != B * T:
+        raise ValueError("cu_seqlens must start at 0 and end at the packed length")
+    if do.shape != (B, T, H, dv):
+        raise ValueError(f"dout shape {do.shape} != {(B, T, H, dv)}")
+    for name, x in (("h0", h0), ("dhT", dhT)):
+        if x is not None and x.shape != (N, H, dk, dv):
+            raise ValueError(f"{name} shape {x.shape} != {(N, H, dk, dv)}")
+    dq = np.zeros_like(q); dk_ = np.zeros_like(k); dv_ = np.zeros_like(v)
+    dg = np.zeros_like(g); db = np.zeros_like(b); dh0 = np.zeros((N, H, dk, dv))
+    rc = _load().kda_oracle_bwd(_p(q), _p(k), _p(v), _p(g), _p(b), _p(h0), _p(do), _p(dhT),
+                                _p(dq), _p(dk_), _p(dv_), _p(dg), _p(db), _p(dh0),
+                                cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)),
+                                N, H, dk, dv, float(scale))
+    if rc != 0:
+        raise RuntimeError(f"oracle failed rc={rc}")
+    return dq, dk_, dv_, dg, db, dh0
 
 
 def segment_map(q, k, v, log_alpha, beta, cu_seqlens=None):

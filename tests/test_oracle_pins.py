@@ -390,3 +390,72 @@ def test_composed_segment_maps_reproduce_the_sequence(cuts):
     np.testing.assert_allclose(S, hT, rtol=0, atol=1e-12)
     np.testing.assert_allclose(oracle.compose(np.stack(maps), np.stack(offs), h0), hT,
                                rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# P-grad: the backward pass (training)
+# --------------------------------------------------------------------------
+def _loss(q, k, v, g, b, h0, cu, scale, dout, dhT):
+    out, hT = oracle.fwd(q, k, v, g, b, scale, h0=h0, cu_seqlens=cu)
+    return float(np.sum(out * dout) + np.sum(hT * dhT))
+
+
+def test_backward_matches_finite_differences():
+    """Central differences of sum(dout*out) + sum(dhT*hT) for every input
+    element; the second sequence crosses the oracle's 64-token replay block."""
+    rng = np.random.default_rng(31)
+    lens, H, dk, dv, scale = [4, 67], 1, 3, 2, 0.7
+    T = sum(lens)
+    q, k, v, g, b, _, _ = _rand_inputs(rng, 1, T, H, dk, dv)
+    h0 = 0.5 * rng.standard_normal((2, H, dk, dv))
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    dout = rng.standard_normal((1, T, H, dv))
+    dhT = rng.standard_normal((2, H, dk, dv))
+    grads = oracle.bwd(q, k, v, g, b, scale, dout, h0=h0, dhT=dhT, cu_seqlens=cu)
+    inputs = [q, k, v, g, b, h0]
+    eps = 1e-6
+    for x, gx in zip(inputs, grads):
+        fd = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            old = x[idx]
+            x[idx] = old + eps
+            lp = _loss(*inputs, cu, scale, dout, dhT)
+            x[idx] = old - eps
+            lm = _loss(*inputs, cu, scale, dout, dhT)
+            x[idx] = old
+            fd[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(gx, fd, rtol=1e-6, atol=1e-7)
+
+
+def test_backward_matches_autograd_of_a_plain_recurrence():
+    """torch autograd (fp64) through a separately written dense-matrix form of
+    the step, S_t = (I - b k k^T) Diag(alpha) S_{t-1} + b k v^T, o = scale S^T q."""
+    torch = pytest.importorskip("torch")
+    rng = np.random.default_rng(32)
+    lens, H, dk, dv, scale = [150, 0, 70], 2, 8, 6, 0.35
+    T = sum(lens)
+    q, k, v, g, b, _, _ = _rand_inputs(rng, 1, T, H, dk, dv)
+    h0 = 0.3 * rng.standard_normal((3, H, dk, dv))
+    cu = np.concatenate([[0], np.cumsum(lens)])
+    dout = rng.standard_normal((1, T, H, dv))
+    dhT = rng.standard_normal((3, H, dk, dv))
+    ts = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (q, k, v, g, b, h0)]
+    tq, tk, tv, tg, tb, th0 = ts
+    loss = 0.0
+    eye = torch.eye(dk, dtype=torch.float64)
+    for n in range(3):
+        for h in range(H):
+            S = th0[n, h]
+            for t in range(cu[n], cu[n + 1]):
+                kt = tk[0, t, h][:, None]
+                M = (eye - tb[0, t, h] * kt @ kt.T) @ torch.diag(torch.exp(tg[0, t, h]))
+                S = M @ S + tb[0, t, h] * kt @ tv[0, t, h][None, :]
+                o = scale * S.T @ tq[0, t, h]
+                loss = loss + (o * torch.from_numpy(dout[0, t, h])).sum()
+            loss = loss + (S * torch.from_numpy(dhT[n, h])).sum()
+    loss.backward()
+    grads = oracle.bwd(q, k, v, g, b, scale, dout, h0=h0, dhT=dhT, cu_seqlens=cu)
+    for t, gx in zip(ts, grads):
+        np.testing.assert_allclose(gx, t.grad.numpy(), rtol=1e-10, atol=1e-11)
