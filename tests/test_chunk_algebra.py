@@ -155,3 +155,110 @@ def test_chunk_is_one_affine_map():
     S0 = rng.standard_normal((dk, dv))
     _, S1 = chunk_forward(q, k, v, g, b, S0, scale)
     np.testing.assert_allclose(M @ S0 + Bm, S1, rtol=0, atol=1e-12)
+
+
+# --------------------------------------------------------------------------
+# Backward of the chunk equations (what the backward kernels compute)
+# --------------------------------------------------------------------------
+def chunk_backward_one(qc, kc, vc, gc, bc, S, dO, dSn, scale):
+    """Gradients of one padded chunk from its entry state S, the output
+    gradient dO and the gradient dSn of its exit state.  Pairwise
+    exponentials e^{G_ic - G_jc} (no sub-chunk references), as the fp32
+    backward kernels take them.  Returns (dq, dk, dv, dg, db, dS)."""
+    G = np.cumsum(gc, axis=0)
+    Ex = np.exp(G[:, None, :] - G[None, :, :])                 # [i, j, c]
+    Pkk = kc[:, None, :] * kc[None, :, :] * Ex                  # k_ic k_jc e^{..}
+    Pqk = scale * qc[:, None, :] * kc[None, :, :] * Ex
+    low = np.tril(np.ones((C, C)), -1)
+    lowd = np.tril(np.ones((C, C)), 0)
+    Ap = Pkk.sum(-1) * low                                     # A' (i > j)
+    A = bc[:, None] * Ap
+    Aqk = Pqk.sum(-1) * lowd
+    T = np.linalg.inv(np.eye(C) + A)
+    Tp = T * bc[None, :]                                       # T' = T diag(beta)
+    KG = kc * np.exp(G)
+    W = Tp @ KG
+    R = vc - KG @ S
+    E = Tp @ R
+    Khat = kc * np.exp(G[-1] - G)
+    QGs = scale * qc * np.exp(G)
+    gam = np.exp(G[-1])
+    # state side
+    dE = Aqk.T @ dO + Khat @ dSn
+    dS = QGs.T @ dO + gam[:, None] * dSn - W.T @ dE
+    dR = Tp.T @ dE
+    dv = dR.copy()
+    dKG = -dR @ S.T
+    dTp = dE @ R.T
+    dQGs = dO @ S.T
+    dAqk = (dO @ E.T) * lowd
+    dKhat = E @ dSn.T
+    dq = scale * np.exp(G) * dQGs
+    dG = QGs * dQGs
+    dk = np.exp(G[-1] - G) * dKhat
+    dGl = (dKhat * Khat).sum(0) + gam * (S * dSn).sum(1)
+    dG -= dKhat * Khat
+    dk += np.exp(G) * dKG
+    dG += KG * dKG
+    # T' = T diag(beta), T = (I + A)^{-1}, A = diag(beta) A'
+    dT = dTp * bc[None, :]
+    db = (T * dTp).sum(0)
+    dA = -(T.T @ dT @ T.T) * low
+    db += (dA * Ap).sum(1)
+    dAp = bc[:, None] * dA
+    # pairwise products
+    dk += np.einsum("ij,ijc->ic", dAp, kc[None, :, :] * Ex)
+    dk += np.einsum("ij,ijc->jc", dAp, kc[:, None, :] * Ex)
+    dG += np.einsum("ij,ijc->ic", dAp, Pkk) - np.einsum("ij,ijc->jc", dAp, Pkk)
+    dq += np.einsum("ij,ijc->ic", dAqk, scale * kc[None, :, :] * Ex)
+    dk += np.einsum("ij,ijc->jc", dAqk, scale * qc[:, None, :] * Ex)
+    dG += np.einsum("ij,ijc->ic", dAqk, Pqk) - np.einsum("ij,ijc->jc", dAqk, Pqk)
+    dG[-1] += dGl
+    dg = np.cumsum(dG[::-1], axis=0)[::-1]                     # G = cumsum(g)
+    return dq, dk, dv, dg, db, dS
+
+
+def chunk_backward(q, k, v, g, b, h0, dout, dhT, scale):
+    """One (sequence, head): forward walk for the entry states, then the
+    chunks in reverse with the state gradient carried between them."""
+    L, dk_ = k.shape
+    dv_ = v.shape[1]
+    starts = list(range(0, L, C))
+    pad = lambda x, s0, n: np.concatenate([x[s0:s0 + n], np.zeros((C - n,) + x.shape[1:])])
+    S = h0.copy()
+    entry = []
+    for s0 in starts:
+        n = min(C, L - s0)
+        I = chunk_intra(pad(q, s0, n), pad(k, s0, n), pad(v, s0, n), pad(g, s0, n),
+                        pad(b, s0, n), scale)
+        entry.append(S)
+        U = I["Ut"] - I["W"] @ S
+        S = I["gam"][:, None] * S + I["KGl"].T @ U
+    grads = [np.zeros_like(x) for x in (q, k, v, g, b)]
+    dS = dhT.copy()
+    for ci in range(len(starts) - 1, -1, -1):
+        s0 = starts[ci]
+        n = min(C, L - s0)
+        r = chunk_backward_one(pad(q, s0, n), pad(k, s0, n), pad(v, s0, n), pad(g, s0, n),
+                               pad(b, s0, n), entry[ci], pad(dout, s0, n), dS, scale)
+        for gx, part in zip(grads, r[:5]):
+            gx[s0:s0 + n] = part[:n]
+        dS = r[5]
+    return (*grads, dS)
+
+
+@pytest.mark.parametrize("L", [1, 64, 100, 193])
+def test_chunk_backward_equals_oracle(L):
+    rng = np.random.default_rng(40 + L)
+    dk, dv, scale = 8, 6, 0.4
+    q, k, v, g, b = _inputs(rng, L, dk, dv)
+    h0 = 0.3 * rng.standard_normal((dk, dv))
+    dout = rng.standard_normal((L, dv))
+    dhT = rng.standard_normal((dk, dv))
+    got = chunk_backward(q, k, v, g, b, h0, dout, dhT, scale)
+    sh = lambda x: x[None, :, None]
+    ref = oracle.bwd(sh(q), sh(k), sh(v), sh(g), b[None, :, None], scale, sh(dout),
+                     h0=h0[None, None], dhT=dhT[None, None])
+    ref = [r[0, :, 0] for r in ref[:5]] + [ref[5][0, 0]]
+    for a, r in zip(got, ref):
+        np.testing.assert_allclose(a, r, rtol=1e-9, atol=1e-10)
