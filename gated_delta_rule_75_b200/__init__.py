@@ -16,7 +16,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "recurrent_step", "gdn_chunk_fwd", "gdn_recurrent_step", "KDAError",
-           "chunk_fwd_segmap", "affine_prefix",
+           "chunk_fwd_segmap", "affine_prefix", "chunk_bwd",
            "library_path", "version",
            "profiler_enable", "profiler_read",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -76,6 +76,9 @@ def _load():
     lib.kda_chunk_fwd_segmap.restype = ctypes.c_int
     lib.kda_affine_prefix.argtypes = [vp, vp, vp, vp, i64, i64, i64, i64, vp]
     lib.kda_affine_prefix.restype = ctypes.c_int
+    lib.kda_chunk_bwd.argtypes = [vp] * 15 + [i64, i64, i64, i64, i64, ctypes.c_float,
+                                              ctypes.c_int, vp]
+    lib.kda_chunk_bwd.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -339,3 +342,44 @@ def affine_prefix(maps, offs, h0=None, out=None):
     if st != KDA_OK:
         raise KDAError(st, "kda_affine_prefix")
     return out
+
+
+def chunk_bwd(q, k, v, log_alpha, beta, scale, dout, h0=None, dhT=None, cu_seqlens=None,
+              need_dh0=True):
+    """Gradients of sum(dout * out) + sum(dhT * hT) for the prefill
+    :func:`chunk_fwd` computes on the same inputs (C ABI ``kda_chunk_bwd``).
+    dout [B,T,H,dv] in the I/O dtype; dhT [N,H,dk,dv] fp32 or None.  Returns
+    (dq, dk, dv in the I/O dtype; dlog_alpha, dbeta, dh0 in fp32; dh0 is None
+    when need_dh0 is False)."""
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev, io = q.device, q.dtype
+    if io not in _IO:
+        raise TypeError(f"unsupported I/O dtype {io}")
+    for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
+                         ("dout", dout, (B, T, H, dv))):
+        _check(t, name, io, shp, dev)
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H, dk), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    if cu_seqlens is not None:
+        if B != 1 or cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev:
+            raise ValueError("cu_seqlens needs int32 offsets on the device and a leading axis of 1")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    for name, t in (("h0", h0), ("dhT", dhT)):
+        if t is not None:
+            _check(t, name, torch.float32, (N, H, dk, dv), dev)
+    dq = torch.empty_like(q)
+    dk_ = torch.empty_like(k)
+    dv_ = torch.empty_like(v)
+    dg = torch.empty_like(log_alpha)
+    db = torch.empty_like(beta)
+    dh0 = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if need_dh0 else None
+    st = _load().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0),
+                               _ptr(dout), _ptr(dhT), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg),
+                               _ptr(db), _ptr(dh0), _ptr(cu_seqlens), N, T, H, dk, dv,
+                               float(scale), _IO[io], _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_chunk_bwd")
+    return dq, dk_, dv_, dg, db, dh0

@@ -541,3 +541,90 @@ kda_status_t kda_affine_prefix(const float* maps, const float* offs, const float
 }
 
 }  // extern "C"
+
+extern "C" {
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* h0, const void* dout, const float* dhT,
+                           void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
+                           float* dh0, const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                           int64_t dk_, int64_t dv_, float scale, kda_io_dtype_t io_dtype,
+                           cudaStream_t stream)
+{
+    if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
+    if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
+    if (!head_ok(dk_) || !head_ok(dv_)) return KDA_ERR_UNSUPPORTED;
+    if (cu_seqlens != nullptr && B < 1) return KDA_ERR_INVALID_ARG;
+    if (B == 0 || H == 0) return KDA_OK;
+    const int64_t T_total = cu_seqlens ? T : B * T;
+    if (T_total > 0) {
+        const void* ptrs[] = {q, k, v, dout, dq, dk, dv, log_alpha, dlog_alpha};
+        for (const void* p : ptrs)
+            if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        if (beta == nullptr || !aligned4(beta) || dbeta == nullptr || !aligned4(dbeta))
+            return KDA_ERR_INVALID_ARG;
+        // outputs must not alias inputs (or one another)
+        const void* outs[] = {dq, dk, dv, dlog_alpha, dbeta};
+        const void* ins[] = {q, k, v, log_alpha, beta, dout};
+        for (const void* o : outs)
+            for (const void* i : ins)
+                if (o == i) return KDA_ERR_INVALID_ARG;
+        for (int a = 0; a < 5; ++a)
+            for (int c = a + 1; c < 5; ++c)
+                if (outs[a] == outs[c]) return KDA_ERR_INVALID_ARG;
+    }
+    if ((h0 && !aligned16(h0)) || (dhT && !aligned16(dhT)) || (dh0 && !aligned16(dh0)))
+        return KDA_ERR_INVALID_ARG;
+    if (cu_seqlens && !aligned4(cu_seqlens)) return KDA_ERR_INVALID_ARG;
+    if (T_total > (int64_t(1) << 40) || H > 65535) return KDA_ERR_UNSUPPORTED;
+    if (B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
+
+    BackwardArgs b;
+    std::memset(&b, 0, sizeof(b));
+    b.q = q; b.k = k; b.v = v; b.log_alpha = log_alpha; b.beta = beta; b.h0 = h0;
+    b.dout = dout; b.dhT = dhT; b.dq = dq; b.dk = dk; b.dv = dv; b.dlog_alpha = dlog_alpha;
+    b.dbeta = dbeta; b.dh0 = dh0; b.H = H; b.dk_ = (int)dk_; b.dv_ = (int)dv_; b.scale = scale;
+    b.io = io_dtype;
+    SeqInfo& si = b.si;
+    si.cu = cu_seqlens;
+    si.chunk_off = nullptr;
+    si.N = B;
+    si.T_seq = cu_seqlens ? 0 : T;
+    si.T_total = T_total;
+    si.nct = cu_seqlens ? 0 : (T + kChunk - 1) / kChunk;
+    si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
+    si.order = nullptr;
+
+    // workspace: [1 KiB header (error word) | chunk offsets | per-(chunk, head) backward blocks]
+    const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 1023) / 1024 * 1024 : 0;
+    const int64_t per_head = bwd_ws_floats_per_chunk((int)dk_, (int)dv_) * (int64_t)sizeof(float) *
+                             (si.chunks_upper > 0 ? si.chunks_upper : 1);
+    int64_t Hg = (workspace_budget() - 1024 - off_bytes) / per_head;
+    if (Hg < 1) Hg = 1;
+    if (Hg > H) Hg = H;
+    StreamBuffer buf;
+    cudaError_t e = buf.alloc((size_t)(1024 + off_bytes + Hg * per_head), stream);
+    if (e) return from_cuda(e);
+    char* base = static_cast<char*>(buf.ptr);
+    int* err_flag = reinterpret_cast<int*>(base);
+    if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
+    if (cu_seqlens) {
+        int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
+        if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, nullptr,
+                                      err_flag, 0, 0, nullptr, stream)))
+            return from_cuda(e);
+        si.chunk_off = chunk_off;
+    }
+    e = run_backward_simt(b, reinterpret_cast<float*>(base + 1024 + off_bytes), Hg, stream);
+    if (e) return from_cuda(e);
+    if (debug_mode()) {
+        int flag = 0;
+        if ((e = cudaMemcpyAsync(&flag, err_flag, sizeof(int), cudaMemcpyDeviceToHost, stream)))
+            return from_cuda(e);
+        if ((e = cudaStreamSynchronize(stream))) return from_cuda(e);
+        if (flag & kErrSeqlens) return KDA_ERR_INVALID_ARG;
+    }
+    return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,584 @@
+// Chunkwise backward pass of KDA, fp32 SIMT kernels.
+//
+// "Kimi Linear acaba de superar a la atencion completa en sus propios
+// terminos" (section on the chunk training algorithm over the
+// diagonal-plus-low-rank transition) says the chunk form exists for training;
+// the pages print no gradient.  The gradients below differentiate the chunk
+// equations (listed at the top of kda_chunk_simt.cu) in reverse; they are
+// checked in fp64 against the oracle's token-by-token reverse mode.  Per chunk,
+// with entry state S, exit-state gradient dS' and output gradient dO:
+//
+//   E  = U = T'(V - K_G S)          R  = V - K_G S      (T' = T diag(beta), K_G = K e^G)
+//   dE = Aqk^T dO + Khat dS'        dR = T'^T dE        (Khat = K e^{G_last - G})
+//   dS = Q_G^T dO + Diag(e^{G_last}) dS' - W^T dE       (Q_G = scale Q e^G, W = T' K_G)
+//   dV = dR,  dK_G = -dR S^T,  dQ_G = dO S^T,  dKhat = E dS'^T
+//   dT' = dE R^T,  dAqk = dO E^T (lower),  dbeta += colsum(T o dT'),
+//   dA = -T^T (dT' diag(beta)) T^T (strictly lower),  dbeta += rowsum(dA o A'),
+//   dA' = diag(beta) dA, then the pairwise products
+//   A'_ij = sum_c k_ic k_jc e^{G_ic - G_jc} and Aqk_ij = scale sum_c q_ic k_jc e^{G_ic - G_jc}
+//   give dk, dq and dG; G = cumsum(g) turns dG into dlog_alpha by a reverse cumsum.
+//
+// Kernels (all fp32, one (chunk, head) block of BwdWs floats each):
+//   prep (kBwd)      the prefill prep, also saving T, A' and K e^G
+//   walk (kBwd)      forward walk per (sequence, head, 32 columns), saving every entry state
+//   bwd_state        reverse walk per (sequence, head, 32 columns): dE, dS across chunks,
+//                    saving every exit-state gradient; dh0 at the start
+//   bwd_dense1       per (chunk, head): E, R, dE, dR (dv written), sum_v S dS'
+//   bwd_dense2       per (chunk, head, product): dK_G, dQ_G, dKhat, dT', dAqk
+//   bwd_param        per (chunk, head): dbeta, dA, the pairwise terms, dq, dk, dlog_alpha
+#include <cstring>
+
+#include "kda_chunk_simt.cuh"
+
+namespace kda {
+
+constexpr int kBT = 256;          // threads of every backward kernel
+constexpr int kTW = 32;           // dv columns per walk tile / dense tile
+
+// ---------------------------------------------------------------------------
+// reverse walk: per (sequence, head, 32-column tile)
+// ---------------------------------------------------------------------------
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kBT)
+chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
+{
+    using BW = BwdWs<DK, DV>;
+    using SW = SimtWs<DK, DV>;
+    constexpr int C = kChunk;
+    const SeqInfo& si = b.si;
+    const int64_t H = b.H;
+    extern __shared__ float smem[];
+    float* sW = smem;                 // [C][DK]
+    float* sQG = sW + C * DK;         // [C][DK]
+    float* sKh = sQG + C * DK;        // [C][DK]
+    float* sAqk = sKh + C * DK;       // [C][C]
+    float* sdO = sAqk + C * C;        // [C][32]
+    float* sdE = sdO + C * kTW;       // [C][32]
+    float* sdS = sdE + C * kTW;       // [DK][32]
+    float* sGam = sdS + DK * kTW;     // [DK]
+
+    const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
+    const int64_t tiles = DV / kTW;
+    const int64_t bid = blockIdx.x;
+    const int64_t n = bid / (hg * tiles);
+    const int hl = (int)((bid / tiles) % hg);
+    const int64_t h = h_base + hl;
+    const int j0 = (int)(bid % tiles) * kTW;
+    const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
+    int64_t bos, eos;
+    seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
+    const int64_t nchunks = si.chunk_count(n, eos - bos);
+    const int64_t gc0 = si.chunk_start(n);
+    const int64_t sidx = n * H + h;
+    const T* __restrict__ dout = (const T*)b.dout;
+
+    for (int e = tid; e < DK * kTW; e += kBT) {
+        const int c = e / kTW, j = e % kTW;
+        sdS[e] = b.dhT ? b.dhT[sidx * DK * DV + c * DV + j0 + j] : 0.f;
+    }
+    for (int64_t ch = nchunks - 1; ch >= 0; --ch) {
+        float* blk = ws + ((gc0 + ch) * Hg + hl) * BW::size;
+        const int64_t t0 = bos + ch * C;
+        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+        __syncthreads();
+        for (int e = tid; e < C * DK; e += kBT) {
+            sW[e] = blk[SW::W + e];
+            sQG[e] = blk[SW::QG + e];
+            sKh[e] = blk[SW::KG + e];
+        }
+        for (int e = tid; e < C * C; e += kBT) sAqk[e] = blk[SW::Aqk + e];
+        for (int c = tid; c < DK; c += kBT) sGam[c] = blk[SW::Gam + c];
+        for (int e = tid; e < C * kTW; e += kBT) {
+            const int t = e / kTW, j = e % kTW;
+            sdO[e] = t < len ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+        }
+        for (int e = tid; e < DK * kTW; e += kBT)          // gradient of this chunk's exit state
+            blk[BW::dSx + (e / kTW) * DV + j0 + (e % kTW)] = sdS[e];
+        __syncthreads();
+        // dE = Aqk^T dO + Khat dS'
+        for (int t = wrp; t < C; t += 8) {
+            float acc = 0.f;
+            for (int s = t; s < C; ++s) acc += sAqk[s * C + t] * sdO[s * kTW + lane];
+            for (int c = 0; c < DK; ++c) acc += sKh[t * DK + c] * sdS[c * kTW + lane];
+            sdE[t * kTW + lane] = acc;
+        }
+        __syncthreads();
+        // dS = Diag(e^{G_last}) dS' + Q_G^T dO - W^T dE
+        for (int c = wrp; c < DK; c += 8) {
+            float acc = sGam[c] * sdS[c * kTW + lane];
+            for (int t = 0; t < C; ++t)
+                acc += sQG[t * DK + c] * sdO[t * kTW + lane] - sW[t * DK + c] * sdE[t * kTW + lane];
+            sdS[c * kTW + lane] = acc;
+        }
+    }
+    __syncthreads();
+    if (b.dh0)
+        for (int e = tid; e < DK * kTW; e += kBT)
+            b.dh0[sidx * DK * DV + (e / kTW) * DV + j0 + (e % kTW)] = sdS[e];
+}
+
+// acc[r] += sum_k A[(row0 + 8 r) * lda + k] * B[k * 32 + lane] (A rows read as
+// 16-byte broadcasts, B columns one per lane), r < 8, K a multiple of 4.
+__device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int lda, int row0,
+                                          const float* B, int K, int lane)
+{
+    for (int k = 0; k < K; k += 4) {
+        const float b0 = B[k * kTW + lane], b1 = B[(k + 1) * kTW + lane];
+        const float b2 = B[(k + 2) * kTW + lane], b3 = B[(k + 3) * kTW + lane];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const float4 a = *reinterpret_cast<const float4*>(A + (row0 + 8 * r) * lda + k);
+            acc[r] += a.x * b0 + a.y * b1 + a.z * b2 + a.w * b3;
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// dense pass 1: per (chunk, head)
+// ---------------------------------------------------------------------------
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kBT)
+chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
+{
+    using BW = BwdWs<DK, DV>;
+    using SW = SimtWs<DK, DV>;
+    constexpr int C = kChunk;
+    const SeqInfo& si = b.si;
+    const int64_t H = b.H;
+    extern __shared__ __align__(16) float smem[];
+    float* sW = smem;                 // [C][DK]
+    float* sKG = sW + C * DK;         // [C][DK]   K e^G
+    float* sKh = sKG + C * DK;        // [C][DK]   K e^{G_last - G}
+    float* sAqk = sKh + C * DK;       // [C][C]
+    float* sT = sAqk + C * C;         // [C][C]
+    float* sS = sT + C * C;           // [DK][32]
+    float* sdSn = sS + DK * kTW;      // [DK][32]
+    float* sdO = sdSn + DK * kTW;     // [C][32]
+    float* sdE = sdO + C * kTW;       // [C][32]
+    float* sB = sdE + C * kTW;        // [C]
+
+    const int64_t gc = blockIdx.x;
+    const int hl = blockIdx.y;
+    const int64_t h = h_base + hl;
+    int64_t n, t0, len64;
+    if (!si.locate(gc, n, t0, len64)) return;
+    const int len = (int)len64;
+    const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
+    float* blk = ws + (gc * Hg + hl) * BW::size;
+    const T* __restrict__ dout = (const T*)b.dout;
+    const T* __restrict__ v = (const T*)b.v;
+    T* __restrict__ dv = (T*)b.dv;
+
+    for (int e = tid; e < C * DK; e += kBT) {
+        sW[e] = blk[SW::W + e];
+        sKG[e] = blk[BW::KGm + e];
+        sKh[e] = blk[SW::KG + e];
+    }
+    for (int e = tid; e < C * C; e += kBT) {
+        sAqk[e] = blk[SW::Aqk + e];
+        sT[e] = blk[BW::Tm + e];
+    }
+    for (int t = tid; t < C; t += kBT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
+    float glS = 0.f;                                  // thread c < DK: sum_v S[c][v] dS'[c][v]
+
+    for (int j0 = 0; j0 < DV; j0 += kTW) {
+        __syncthreads();
+        for (int e = tid; e < DK * kTW; e += kBT) {
+            const int c = e / kTW, j = e % kTW;
+            sS[e] = blk[BW::Sx + c * DV + j0 + j];
+            sdSn[e] = blk[BW::dSx + c * DV + j0 + j];
+        }
+        for (int e = tid; e < C * kTW; e += kBT) {
+            const int t = e / kTW, j = e % kTW;
+            sdO[e] = t < len ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+        }
+        __syncthreads();
+        if (tid < DK)
+            for (int j = 0; j < kTW; ++j) glS += sS[tid * kTW + j] * sdSn[tid * kTW + j];
+        // rows w, w+8, ..., w+56 of this warp; column j0 + lane
+        float e8[8], r8[8], de8[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) { e8[r] = 0.f; r8[r] = 0.f; de8[r] = 0.f; }
+        rows8_mac(e8, sW, DK, wrp, sS, DK, lane);      // W S
+        rows8_mac(r8, sKG, DK, wrp, sS, DK, lane);     // K_G S
+        rows8_mac(de8, sKh, DK, wrp, sdSn, DK, lane);  // Khat dS'
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int t = wrp + 8 * r;
+            const float ut = blk[SW::Ut + t * DV + j0 + lane];
+            const float vt = t < len ? IO<T>::load(v, ((t0 + t) * H + h) * DV + j0 + lane) : 0.f;
+            e8[r] = ut - e8[r];
+            r8[r] = vt - r8[r];
+            float acc = 0.f;                            // Aqk^T dO
+            for (int s = t; s < C; ++s) acc += sAqk[s * C + t] * sdO[s * kTW + lane];
+            de8[r] += acc;
+            sdE[t * kTW + lane] = de8[r];
+            blk[BW::E + t * DV + j0 + lane] = e8[r];
+            blk[BW::R + t * DV + j0 + lane] = r8[r];
+            blk[BW::dE + t * DV + j0 + lane] = de8[r];
+        }
+        __syncthreads();
+        // dR = diag(beta) T^T dE  (T lower: T[s][t] != 0 only for s >= t)
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const int t = wrp + 8 * r;
+            float acc = 0.f;
+            for (int s = t; s < C; ++s) acc += sT[s * C + t] * sdE[s * kTW + lane];
+            acc *= sB[t];
+            blk[BW::dR + t * DV + j0 + lane] = acc;
+            if (t < len) IO<T>::store(dv, ((t0 + t) * H + h) * DV + j0 + lane, acc);
+        }
+    }
+    if (tid < DK) blk[BW::dGlS + tid] = glS;
+}
+
+// ---------------------------------------------------------------------------
+// dense pass 2: out[i][m] = sign * sum_v A[i][v] B[m][v], per (chunk, head, product)
+//   0: dK_G = -dR S^T   1: dQ_G = dO S^T   2: dKhat = E dS'^T   (m < DK)
+//   3: dT'  =  dE R^T   4: dAqk = dO E^T (kept for m <= i)       (m < C)
+// ---------------------------------------------------------------------------
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kBT)
+chunk_bwd_dense2_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
+{
+    using BW = BwdWs<DK, DV>;
+    constexpr int C = kChunk;
+    constexpr int P = kTW + 1;        // padded pitch: 16 consecutive rows hit distinct banks
+    const SeqInfo& si = b.si;
+    const int64_t H = b.H;
+    __shared__ float sA[C * P];
+    __shared__ float sBm[DK * P];
+
+    const int64_t gc = blockIdx.x;
+    const int hl = blockIdx.y;
+    const int job = blockIdx.z;
+    const int64_t h = h_base + hl;
+    int64_t n, t0, len64;
+    if (!si.locate(gc, n, t0, len64)) return;
+    const int len = (int)len64;
+    const int tid = threadIdx.x;
+    float* blk = ws + (gc * Hg + hl) * BW::size;
+    const T* __restrict__ dout = (const T*)b.dout;
+
+    const bool a_is_dO = job == 1 || job == 4;
+    const float* Ag = job == 0 ? blk + BW::dR : job == 2 ? blk + BW::E : job == 3 ? blk + BW::dE : nullptr;
+    const float* Bg = (job == 0 || job == 1) ? blk + BW::Sx : job == 2 ? blk + BW::dSx
+                    : job == 3 ? blk + BW::R : blk + BW::E;
+    const int M = job < 3 ? DK : C;                   // rows of B
+    const float sign = job == 0 ? -1.f : 1.f;
+    float* out = blk + (job == 0 ? BW::dKG : job == 1 ? BW::dQG : job == 2 ? BW::dKh
+                        : job == 3 ? BW::dTp : BW::dAqk);
+
+    // thread tile: rows ti + 16 r (r < 4), columns tm + 16 q (q < M / 16)
+    const int ti = tid >> 4, tm = tid & 15;
+    float acc[4][DK / 16];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int q = 0; q < DK / 16; ++q) acc[r][q] = 0.f;
+    const int nq = M / 16;
+
+    for (int v0 = 0; v0 < DV; v0 += kTW) {
+        __syncthreads();
+        for (int e = tid; e < C * kTW; e += kBT) {
+            const int i = e / kTW, j = e % kTW;
+            float x;
+            if (a_is_dO) x = i < len ? IO<T>::load(dout, ((t0 + i) * H + h) * DV + v0 + j) : 0.f;
+            else x = Ag[i * DV + v0 + j];
+            sA[i * P + j] = x;
+        }
+        for (int e = tid; e < M * kTW; e += kBT) {
+            const int m = e / kTW, j = e % kTW;
+            sBm[m * P + j] = Bg[m * DV + v0 + j];
+        }
+        __syncthreads();
+        for (int j = 0; j < kTW; ++j) {
+            float a[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) a[r] = sA[(ti + 16 * r) * P + j];
+#pragma unroll
+            for (int q = 0; q < DK / 16; ++q) {
+                if (q < nq) {
+                    const float bb = sBm[(tm + 16 * q) * P + j];
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) acc[r][q] += a[r] * bb;
+                }
+            }
+        }
+    }
+    const int ld = job < 3 ? DK : C;
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+        for (int q = 0; q < DK / 16; ++q)
+            if (q < nq) {
+                const int i = ti + 16 * r, m = tm + 16 * q;
+                float x = sign * acc[r][q];
+                if (job == 4 && m > i) x = 0.f;
+                out[i * ld + m] = x;
+            }
+}
+
+// ---------------------------------------------------------------------------
+// parameter gradients: per (chunk, head)
+// ---------------------------------------------------------------------------
+template <typename T, int DK, int DV>
+__global__ void __launch_bounds__(kBT)
+chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
+{
+    using BW = BwdWs<DK, DV>;
+    using SW = SimtWs<DK, DV>;
+    constexpr int C = kChunk;
+    const SeqInfo& si = b.si;
+    const int64_t H = b.H;
+    extern __shared__ __align__(16) float smem[];
+    float* sK = smem;                 // [C][DK]
+    float* sQ = sK + C * DK;          // [C][DK]
+    float* sG = sQ + C * DK;          // [C][DK]  cumulative log-decay
+    float* sdG = sG + C * DK;         // [C][DK]
+    float* sT = sdG + C * DK;         // [C][C]
+    float* sAp = sT + C * C;          // [C][C]   A', then dA' = diag(beta) dA
+    float* sdT = sAp + C * C;         // [C][C]   dT', then dT = dT' diag(beta)
+    float* sX = sdT + C * C;          // [C][C]   dT T^T, then dA
+    float* sdAqk = sX + C * C;        // [C][C]
+    float* sB = sdAqk + C * C;        // [C]
+    float* sdB = sB + C;              // [C]
+
+    const int64_t gc = blockIdx.x;
+    const int hl = blockIdx.y;
+    const int64_t h = h_base + hl;
+    int64_t n, t0, len64;
+    if (!si.locate(gc, n, t0, len64)) return;
+    const int len = (int)len64;
+    const int tid = threadIdx.x;
+    float* blk = ws + (gc * Hg + hl) * BW::size;
+    const T* __restrict__ q = (const T*)b.q;
+    const T* __restrict__ k = (const T*)b.k;
+    const float scale = b.scale;
+
+    for (int e = tid; e < C * DK; e += kBT) {
+        const int t = e / DK, c = e % DK;
+        const bool ok = t < len;
+        const int64_t src = ((t0 + t) * H + h) * DK + c;
+        sK[e] = ok ? IO<T>::load(k, src) : 0.f;
+        sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
+        sG[e] = ok ? b.log_alpha[src] : 0.f;
+    }
+    for (int e = tid; e < C * C; e += kBT) {
+        sT[e] = blk[BW::Tm + e];
+        sAp[e] = blk[BW::Ap + e];
+        sdT[e] = blk[BW::dTp + e];
+        sdAqk[e] = blk[BW::dAqk + e];
+    }
+    for (int t = tid; t < C; t += kBT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
+    __syncthreads();
+    if (tid < DK) {                                   // G = cumsum(g) per channel
+        float run = 0.f;
+        for (int t = 0; t < C; ++t) { run += sG[t * DK + tid]; sG[t * DK + tid] = run; }
+    }
+    // dbeta_i = sum_r T[r][i] dT'[r][i]
+    if (tid < C) {
+        float acc = 0.f;
+        for (int r = tid; r < C; ++r) acc += sT[r * C + tid] * sdT[r * C + tid];
+        sdB[tid] = acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += kBT) sdT[e] *= sB[e % C];   // dT = dT' diag(beta)
+    __syncthreads();
+    // X = dT T^T:  X[r][j] = sum_m dT[r][m] T[j][m]  (T[j][m] = 0 for m > j)
+    for (int e = tid; e < C * C; e += kBT) {
+        const int r = e / C, j = e % C;
+        float acc = 0.f;
+        for (int m = 0; m <= j; ++m) acc += sdT[r * C + m] * sT[j * C + m];
+        sX[e] = acc;
+    }
+    __syncthreads();
+    // dA[i][j] = -sum_r T[r][i] X[r][j]  (i > j; T[r][i] = 0 for r < i)
+    float dA[16];
+    for (int u = 0; u < 16; ++u) {
+        const int e = tid + kBT * u, i = e / C, j = e % C;
+        float acc = 0.f;
+        if (j < i)
+            for (int r = i; r < C; ++r) acc += sT[r * C + i] * sX[r * C + j];
+        dA[u] = -acc;
+    }
+    __syncthreads();
+    for (int u = 0; u < 16; ++u) sX[tid + kBT * u] = dA[u];
+    __syncthreads();
+    // dbeta_i += sum_{j<i} dA[i][j] A'[i][j];  dA' = diag(beta) dA
+    if (tid < C) {
+        float acc = 0.f;
+        for (int j = 0; j < tid; ++j) acc += sX[tid * C + j] * sAp[tid * C + j];
+        sdB[tid] += acc;
+    }
+    __syncthreads();
+    for (int e = tid; e < C * C; e += kBT) sAp[e] = sB[e / C] * sX[e];
+    __syncthreads();
+
+    // pairwise products and elementwise terms, element (i, c)
+    const float* dKG = blk + BW::dKG;
+    const float* dQG = blk + BW::dQG;
+    const float* dKh = blk + BW::dKh;
+    const float* gam = blk + SW::Gam;
+    for (int e = tid; e < C * DK; e += kBT) {
+        const int i = e / DK, c = e % DK;
+        const float gi = sG[e], ki = sK[e], qi = sQ[e];
+        float dk = 0.f, dq = 0.f, dg = 0.f;
+        for (int j = 0; j < C; ++j) {
+            const float kj = sK[j * DK + c], gj = sG[j * DK + c];
+            if (j < i) {
+                const float ex = expf(gi - gj);
+                const float x = sAp[i * C + j] * ex;
+                const float y = scale * sdAqk[i * C + j] * ex;
+                dk += x * kj;
+                dq += y * kj;
+                dg += (x * ki + y * qi) * kj;
+            } else if (j > i) {
+                const float ex = expf(gj - gi);
+                const float x = sAp[j * C + i] * ex;
+                const float y = scale * sdAqk[j * C + i] * ex;
+                const float qj = sQ[j * DK + c];
+                dk += x * kj + y * qj;
+                dg -= (x * kj + y * qj) * ki;
+            } else {
+                const float y = scale * sdAqk[i * C + i];
+                dq += y * ki;
+                dk += y * qi;
+            }
+        }
+        const float eg = expf(gi), egl = expf(sG[(C - 1) * DK + c] - gi);
+        dq += scale * eg * dQG[e];
+        dg += scale * qi * eg * dQG[e];
+        dk += egl * dKh[e] + eg * dKG[e];
+        dg += ki * eg * dKG[e] - ki * egl * dKh[e];
+        sdG[e] = dg;
+        if (i < len) {
+            const int64_t dst = ((t0 + i) * H + h) * DK + c;
+            IO<T>::store((T*)b.dq, dst, dq);
+            IO<T>::store((T*)b.dk, dst, dk);
+        }
+    }
+    __syncthreads();
+    // dG_last = sum_i dKhat o Khat + e^{G_last} sum_v S dS'; dlog_alpha = reverse cumsum of dG
+    if (tid < DK) {
+        const int c = tid;
+        const float gl = sG[(C - 1) * DK + c];
+        float acc = gam[c] * blk[BW::dGlS + c];
+        for (int i = 0; i < C; ++i) acc += dKh[i * DK + c] * sK[i * DK + c] * expf(gl - sG[i * DK + c]);
+        float run = acc;
+        for (int i = C - 1; i >= 0; --i) {
+            run += sdG[i * DK + c];
+            if (i < len) b.dlog_alpha[((t0 + i) * H + h) * DK + c] = run;
+        }
+    }
+    if (tid < len) b.dbeta[(t0 + tid) * H + h] = sdB[tid];
+}
+
+template <int DK, int DV>
+constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kChunk + 2 * kChunk * kTW + DK * kTW + DK); }
+template <int DK, int DV>
+constexpr size_t bwd_dense1_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + 2 * kChunk * kChunk + 2 * DK * kTW + 2 * kChunk * kTW + kChunk); }
+template <int DK, int DV>
+constexpr size_t bwd_param_smem() { return sizeof(float) * (size_t)(4 * kChunk * DK + 5 * kChunk * kChunk + 2 * kChunk); }
+
+template <typename T, int DK, int DV>
+static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaStream_t st)
+{
+    static std::atomic<uint64_t> attrs_done{0};
+    cudaError_t e = once_per_device(attrs_done, [] {
+        const int mx = cudaFuncAttributeMaxDynamicSharedMemorySize;
+        cudaError_t r;
+        if ((r = cudaFuncSetAttribute(chunk_prep_simt_kernel<T, DK, DV, true>, (cudaFuncAttribute)mx,
+                                      (int)simt_prep_smem<DK, DV>())))
+            return r;
+        if ((r = cudaFuncSetAttribute(chunk_state_simt_kernel<T, DK, DV, true>, (cudaFuncAttribute)mx,
+                                      (int)simt_state_smem<DK, DV>())))
+            return r;
+        if ((r = cudaFuncSetAttribute(chunk_bwd_state_kernel<T, DK, DV>, (cudaFuncAttribute)mx,
+                                      (int)bwd_state_smem<DK, DV>())))
+            return r;
+        if ((r = cudaFuncSetAttribute(chunk_bwd_dense1_kernel<T, DK, DV>, (cudaFuncAttribute)mx,
+                                      (int)bwd_dense1_smem<DK, DV>())))
+            return r;
+        return cudaFuncSetAttribute(chunk_bwd_param_kernel<T, DK, DV>, (cudaFuncAttribute)mx,
+                                    (int)bwd_param_smem<DK, DV>());
+    });
+    if (e) return e;
+    const SeqInfo& si = b.si;
+    // the forward pieces see the same inputs through a PrefillArgs view
+    PrefillArgs a;
+    memset(&a, 0, sizeof(a));
+    a.q = b.q; a.k = b.k; a.v = b.v; a.log_alpha = b.log_alpha; a.beta = b.beta; a.h0 = b.h0;
+    a.out = nullptr; a.hT = nullptr; a.si = si; a.H = b.H; a.dk = DK; a.dv = DV;
+    a.scale = b.scale; a.io = b.io; a.slots = nullptr; a.P = 0; a.err = nullptr;
+    a.gate_scalar = false;
+    for (int64_t hb = 0; hb < b.H; hb += Hg) {
+        const int64_t hg = (b.H - hb) < Hg ? (b.H - hb) : Hg;
+        const dim3 gchunk((unsigned)si.chunks_upper, (unsigned)hg);
+        if (si.chunks_upper > 0) {
+            LaunchScope scope(st, K_PREP_SIMT);
+            chunk_prep_simt_kernel<T, DK, DV, true><<<gchunk, 256, simt_prep_smem<DK, DV>(), st>>>(
+                (const T*)b.q, (const T*)b.k, (const T*)b.v, b.log_alpha, b.beta, si, b.H, hb, Hg,
+                b.scale, ws, 0);
+            if ((e = cudaGetLastError())) return e;
+        }
+        const dim3 gwalk((unsigned)(si.N * hg * (DV / kTW)));
+        {
+            LaunchScope scope(st, K_STATE_SIMT);
+            chunk_state_simt_kernel<T, DK, DV, true><<<gwalk, 256, simt_state_smem<DK, DV>(), st>>>(
+                ws, a, hb, Hg);
+            if ((e = cudaGetLastError())) return e;
+        }
+        {
+            LaunchScope scope(st, K_BWD_STATE);
+            chunk_bwd_state_kernel<T, DK, DV><<<gwalk, kBT, bwd_state_smem<DK, DV>(), st>>>(ws, b, hb, Hg);
+            if ((e = cudaGetLastError())) return e;
+        }
+        if (si.chunks_upper > 0) {
+            {
+                LaunchScope scope(st, K_BWD_DENSE1);
+                chunk_bwd_dense1_kernel<T, DK, DV><<<gchunk, kBT, bwd_dense1_smem<DK, DV>(), st>>>(
+                    ws, b, hb, Hg);
+                if ((e = cudaGetLastError())) return e;
+            }
+            {
+                LaunchScope scope(st, K_BWD_DENSE2);
+                const dim3 g5((unsigned)si.chunks_upper, (unsigned)hg, 5);
+                chunk_bwd_dense2_kernel<T, DK, DV><<<g5, kBT, 0, st>>>(ws, b, hb, Hg);
+                if ((e = cudaGetLastError())) return e;
+            }
+            {
+                LaunchScope scope(st, K_BWD_PARAM);
+                chunk_bwd_param_kernel<T, DK, DV><<<gchunk, kBT, bwd_param_smem<DK, DV>(), st>>>(
+                    ws, b, hb, Hg);
+                if ((e = cudaGetLastError())) return e;
+            }
+        }
+    }
+    return cudaSuccess;
+}
+
+template <typename T>
+static cudaError_t run_bwd_d(const BackwardArgs& b, float* ws, int64_t Hg, cudaStream_t st)
+{
+    if (b.dk_ == 128 && b.dv_ == 128) return run_bwd_t<T, 128, 128>(b, ws, Hg, st);
+    if (b.dk_ == 128 && b.dv_ == 64) return run_bwd_t<T, 128, 64>(b, ws, Hg, st);
+    if (b.dk_ == 64 && b.dv_ == 128) return run_bwd_t<T, 64, 128>(b, ws, Hg, st);
+    return run_bwd_t<T, 64, 64>(b, ws, Hg, st);
+}
+
+int64_t bwd_ws_floats_per_chunk(int dk, int dv)
+{
+    if (dk == 128 && dv == 128) return BwdWs<128, 128>::size;
+    if (dk == 128 && dv == 64) return BwdWs<128, 64>::size;
+    if (dk == 64 && dv == 128) return BwdWs<64, 128>::size;
+    return BwdWs<64, 64>::size;
+}
+
+cudaError_t run_backward_simt(const BackwardArgs& b, float* ws, int64_t Hg, cudaStream_t st)
+{
+    if (b.io == KDA_IO_F32) return run_bwd_d<float>(b, ws, Hg, st);
+    return run_bwd_d<__nv_bfloat16>(b, ws, Hg, st);
+}
+
+}  // namespace kda

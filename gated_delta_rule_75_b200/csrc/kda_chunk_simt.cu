@@ -22,230 +22,21 @@
 // taken pairwise (e^{G_i - G_j}), so this path has no limit on the decay rate.
 // It is the reference-quality GPU path: fp32 I/O and the bisection baseline of
 // the tensor-core kernels.
-#include "kda_common.cuh"
-#include "kda_internal.h"
+#include "kda_chunk_simt.cuh"
 
 namespace kda {
-
-// Workspace block of one (chunk, head), in floats.
-template <int DK, int DV>
-struct SimtWs {
-    static constexpr int64_t W = 0;
-    static constexpr int64_t Ut = W + kChunk * DK;
-    static constexpr int64_t Aqk = Ut + kChunk * DV;
-    static constexpr int64_t QG = Aqk + kChunk * kChunk;
-    static constexpr int64_t KG = QG + kChunk * DK;
-    static constexpr int64_t Gam = KG + kChunk * DK;
-    static constexpr int64_t size = Gam + DK;
-};
 
 int64_t simt_ws_floats_per_chunk(int dk, int dv)
 {
     return (int64_t)kChunk * (3 * dk + dv + kChunk) + dk;
 }
 
-// ---------------------------------------------------------------------------
-// step a + b: cumulative log-decay and intra-chunk transform
-// ---------------------------------------------------------------------------
-template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(256)
-chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
-                       const float* __restrict__ log_alpha, const float* __restrict__ beta,
-                       SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
-                       float* __restrict__ ws, int gate_scalar)
-{
-    constexpr int C = kChunk;
-    extern __shared__ float smem[];
-    float* sK = smem;                 // [C][DK]
-    float* sQ = sK + C * DK;          // [C][DK], later beta K e^G
-    float* sV = sQ + C * DK;          // [C][DV], later beta V
-    float* sG = sV + C * DV;          // [C][DK]
-    float* sA = sG + C * DK;          // [C][C]
-    float* sT = sA + C * C;           // [C][C]
-    float* sB = sT + C * C;           // [C]
-
-    const int64_t gc = blockIdx.x;
-    const int hl = blockIdx.y;
-    const int64_t h = h_base + hl;
-    int64_t n, t0, len;
-    if (!si.locate(gc, n, t0, len)) return;
-    const int tid = threadIdx.x;
-
-    for (int e = tid; e < C * DK; e += blockDim.x) {
-        const int t = e / DK, c = e % DK;
-        const bool ok = t < len;
-        const int64_t src = ((t0 + t) * H + h) * DK + c;
-        sK[e] = ok ? IO<T>::load(k, src) : 0.f;
-        sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
-        sG[e] = ok ? log_alpha[gate_scalar ? (t0 + t) * H + h : src] : 0.f;
-    }
-    for (int e = tid; e < C * DV; e += blockDim.x) {
-        const int t = e / DV, c = e % DV;
-        sV[e] = t < len ? IO<T>::load(v, ((t0 + t) * H + h) * DV + c) : 0.f;
-    }
-    for (int t = tid; t < C; t += blockDim.x) sB[t] = t < len ? beta[(t0 + t) * H + h] : 0.f;
-    __syncthreads();
-
-    // (a) inclusive cumulative sum of log-decay per channel within the chunk
-    if (tid < DK) {
-        float run = 0.f;
-        for (int t = 0; t < C; ++t) { run += sG[t * DK + tid]; sG[t * DK + tid] = run; }
-    }
-    __syncthreads();
-
-    // (b1) A (strictly lower, beta-weighted) and Aqk (lower incl. diagonal)
-    for (int pidx = tid; pidx < C * C; pidx += blockDim.x) {
-        const int i = pidx / C, j = pidx % C;
-        float kk = 0.f, qk = 0.f;
-        if (j <= i) {
-            for (int cc = 0; cc < DK; ++cc) {
-                const int c = (cc + j) % DK;        // rotate to spread banks
-                const float e = expf(sG[i * DK + c] - sG[j * DK + c]);
-                const float kj = sK[j * DK + c] * e;
-                kk += sK[i * DK + c] * kj;
-                qk += sQ[i * DK + c] * kj;
-            }
-        }
-        sA[pidx] = (j < i) ? sB[i] * kk : 0.f;
-        sT[pidx] = (j <= i) ? scale * qk : 0.f;   // Aqk parked in sT for now
-    }
-    __syncthreads();
-
-    float* blk = ws + (gc * Hg + hl) * SimtWs<DK, DV>::size;
-    for (int e = tid; e < C * C; e += blockDim.x) blk[SimtWs<DK, DV>::Aqk + e] = sT[e];
-    // Q e^G (scaled), K e^{G_last - G}, e^{G_last}
-    for (int e = tid; e < C * DK; e += blockDim.x) {
-        const int c = e % DK;
-        const float G = sG[e], Gl = sG[(C - 1) * DK + c];
-        blk[SimtWs<DK, DV>::QG + e] = scale * sQ[e] * expf(G);
-        blk[SimtWs<DK, DV>::KG + e] = sK[e] * expf(Gl - G);
-    }
-    for (int c = tid; c < DK; c += blockDim.x) blk[SimtWs<DK, DV>::Gam + c] = expf(sG[(C - 1) * DK + c]);
-    __syncthreads();
-
-    // (b2) T = (I + A)^{-1}: column c by forward substitution
-    if (tid < C) {
-        const int c = tid;
-        for (int i = 0; i < C; ++i) sT[i * C + c] = (i == c) ? 1.f : 0.f;
-        for (int i = c + 1; i < C; ++i) {
-            float acc = 0.f;
-            for (int j = c; j < i; ++j) acc += sA[i * C + j] * sT[j * C + c];
-            sT[i * C + c] = -acc;
-        }
-    }
-    // beta K e^G into sQ, beta V in place
-    for (int e = tid; e < C * DK; e += blockDim.x) sQ[e] = sB[e / DK] * sK[e] * expf(sG[e]);
-    for (int e = tid; e < C * DV; e += blockDim.x) sV[e] *= sB[e / DV];
-    __syncthreads();
-
-    // (b3) W = T (beta K e^G), Ut = T (beta V)
-    for (int e = tid; e < C * DK; e += blockDim.x) {
-        const int i = e / DK, c = e % DK;
-        float acc = 0.f;
-        for (int j = 0; j <= i; ++j) acc += sT[i * C + j] * sQ[j * DK + c];
-        blk[SimtWs<DK, DV>::W + e] = acc;
-    }
-    for (int e = tid; e < C * DV; e += blockDim.x) {
-        const int i = e / DV, c = e % DV;
-        float acc = 0.f;
-        for (int j = 0; j <= i; ++j) acc += sT[i * C + j] * sV[j * DV + c];
-        blk[SimtWs<DK, DV>::Ut + e] = acc;
-    }
-}
-
-// ---------------------------------------------------------------------------
-// steps c + d: sequential state propagation and output, per 32-column dv tile
-// ---------------------------------------------------------------------------
-template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(256)
-chunk_state_simt_kernel(const float* __restrict__ ws, PrefillArgs a, int64_t h_base, int64_t Hg)
-{
-    const SeqInfo& si = a.si;
-    const int64_t H = a.H;
-    T* __restrict__ out = (T*)a.out;
-    constexpr int C = kChunk, TW = 32;
-    extern __shared__ float smem[];
-    float* sW = smem;                 // [C][DK]
-    float* sQG = sW + C * DK;         // [C][DK]
-    float* sKG = sQG + C * DK;        // [C][DK]
-    float* sAqk = sKG + C * DK;       // [C][C]
-    float* sU = sAqk + C * C;         // [C][TW]
-    float* sS = sU + C * TW;          // [DK][TW]
-    float* sGam = sS + DK * TW;       // [DK]
-
-    // blocks run (tile, head)-innermost over sequences ranked longest first
-    const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
-    const int64_t tiles = DV / TW;
-    const int64_t bid = blockIdx.x;
-    const int64_t n = si.seq_of(bid / (hg * tiles));
-    const int hl = (int)((bid / tiles) % hg);
-    const int64_t h = h_base + hl;
-    const int j0 = (int)(bid % tiles) * TW;
-    const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
-    int64_t bos, eos;
-    seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
-    const int64_t nchunks = si.chunk_count(n, eos - bos);
-    const int64_t gc0 = si.chunk_start(n);
-
-    const int64_t sidx = a.state_index(n, h);
-    const float* h0p = (a.h0 && sidx >= 0) ? a.h0 + sidx * DK * DV : nullptr;
-    float* hTp = (a.hT && sidx >= 0) ? a.hT + sidx * DK * DV : nullptr;
-    for (int e = tid; e < DK * TW; e += blockDim.x) {
-        const int c = e / TW, j = e % TW;
-        sS[e] = h0p ? h0p[c * DV + j0 + j] : 0.f;
-    }
-    for (int64_t ch = 0; ch < nchunks; ++ch) {
-        const float* blk = ws + ((gc0 + ch) * Hg + hl) * SimtWs<DK, DV>::size;
-        const int64_t t0 = bos + ch * C;
-        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-        __syncthreads();
-        for (int e = tid; e < C * DK; e += blockDim.x) {
-            sW[e] = blk[SimtWs<DK, DV>::W + e];
-            sQG[e] = blk[SimtWs<DK, DV>::QG + e];
-            sKG[e] = blk[SimtWs<DK, DV>::KG + e];
-        }
-        for (int e = tid; e < C * C; e += blockDim.x) sAqk[e] = blk[SimtWs<DK, DV>::Aqk + e];
-        for (int e = tid; e < C * TW; e += blockDim.x)
-            sU[e] = blk[SimtWs<DK, DV>::Ut + (e / TW) * DV + j0 + (e % TW)];
-        for (int c = tid; c < DK; c += blockDim.x) sGam[c] = blk[SimtWs<DK, DV>::Gam + c];
-        __syncthreads();
-        // U = Ut - W S
-        for (int t = wrp; t < C; t += 8) {
-            float acc = 0.f;
-            for (int c = 0; c < DK; ++c) acc += sW[t * DK + c] * sS[c * TW + lane];
-            sU[t * TW + lane] -= acc;
-        }
-        __syncthreads();
-        // O = scale (Q e^G) S + Aqk U   (uses the entry state)
-        for (int t = wrp; t < len; t += 8) {
-            float acc = 0.f;
-            for (int c = 0; c < DK; ++c) acc += sQG[t * DK + c] * sS[c * TW + lane];
-            for (int s = 0; s <= t; ++s) acc += sAqk[t * C + s] * sU[s * TW + lane];
-            IO<T>::store(out, ((t0 + t) * H + h) * DV + j0 + lane, acc);
-        }
-        __syncthreads();
-        // S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U
-        for (int c = wrp; c < DK; c += 8) {
-            float acc = sGam[c] * sS[c * TW + lane];
-            for (int t = 0; t < C; ++t) acc += sKG[t * DK + c] * sU[t * TW + lane];
-            sS[c * TW + lane] = acc;
-        }
-    }
-    __syncthreads();
-    if (hTp) {
-        for (int e = tid; e < DK * TW; e += blockDim.x) {
-            const int c = e / TW, j = e % TW;
-            hTp[c * DV + j0 + j] = sS[e];
-        }
-    }
-}
-
 template <typename T, int DK, int DV>
 static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaStream_t st)
 {
     constexpr int C = kChunk;
-    const size_t smem_prep = sizeof(float) * (size_t)(C * (3 * DK + DV) + 2 * C * C + C);
-    const size_t smem_state = sizeof(float) * (size_t)(3 * C * DK + C * C + C * 32 + DK * 32 + DK);
+    const size_t smem_prep = simt_prep_smem<DK, DV>();
+    const size_t smem_state = simt_state_smem<DK, DV>();
     static std::atomic<uint64_t> attrs_done{0};
     cudaError_t e = once_per_device(attrs_done, [&] {
         cudaError_t r = cudaFuncSetAttribute(chunk_prep_simt_kernel<T, DK, DV>,

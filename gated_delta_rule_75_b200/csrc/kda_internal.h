@@ -164,6 +164,29 @@ struct PrefillArgs {
 #endif
 };
 
+// Backward pass (chunkwise gradients), fp32 SIMT kernels.
+struct BackwardArgs {
+    const void* q;
+    const void* k;
+    const void* v;
+    const float* log_alpha;
+    const float* beta;
+    const float* h0;          // nullable: zero initial state
+    const void* dout;         // [.., H, dv] io dtype
+    const float* dhT;         // nullable: zero gradient of the final state
+    void* dq;                 // [.., H, dk] io dtype
+    void* dk;
+    void* dv;                 // [.., H, dv] io dtype
+    float* dlog_alpha;        // [.., H, dk]
+    float* dbeta;             // [.., H]
+    float* dh0;               // nullable
+    SeqInfo si;
+    int64_t H;
+    int dk_, dv_;
+    float scale;
+    kda_io_dtype_t io;
+};
+
 struct DecodeArgs {
     const void* q;
     const void* k;
@@ -208,6 +231,10 @@ enum KernelId {
     K_STATE_SEG_TC,
     K_AFFINE_PREFIX,
     K_FILL,
+    K_BWD_STATE,
+    K_BWD_DENSE1,
+    K_BWD_DENSE2,
+    K_BWD_PARAM,
     K_KERNEL_COUNT
 };
 
@@ -233,6 +260,10 @@ cudaError_t launch_decode(const DecodeArgs& a, cudaStream_t st);
 // kda_chunk_simt.cu
 int64_t simt_ws_floats_per_chunk(int dk, int dv);
 cudaError_t run_prefill_simt(const PrefillArgs& a, float* ws, int64_t Hg, cudaStream_t st);
+
+// kda_chunk_bwd.cu
+int64_t bwd_ws_floats_per_chunk(int dk, int dv);
+cudaError_t run_backward_simt(const BackwardArgs& b, float* ws, int64_t Hg, cudaStream_t st);
 
 // kda_chunk_tc.cu (bf16, dk = dv = 128)
 int64_t tc_ws_bytes_per_chunk();

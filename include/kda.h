@@ -273,6 +273,41 @@ KDA_API kda_status_t kda_recurrent_step_slots(const void* q, const void* k, cons
                                               cudaStream_t stream);
 
 /*
+ * kda_chunk_bwd -- gradients of the chunkwise prefill (training).
+ *
+ * "Kimi Linear acaba de superar a la atencion completa en sus propios
+ * terminos" (section on the chunk training algorithm) says the method trains
+ * with the chunk form; the pages give no gradient.  This returns the exact
+ * gradients (up to rounding) of L = sum(dout * out) + sum(dhT * hT) for the
+ * forward kda_chunk_fwd computes on the same arguments, obtained by
+ * differentiating the chunk equations in reverse: a forward walk recomputes
+ * every chunk's entry state, a reverse walk carries dL/dS back across chunks,
+ * and per-chunk kernels form the parameter gradients.  All arithmetic is fp32
+ * on the SIMT cores (no tensor cores yet).
+ *
+ *  q, k, v, log_alpha, beta, h0, cu_seqlens, B, T, H, dk, dv, scale, io_dtype:
+ *              exactly as passed to kda_chunk_fwd
+ *  dout        [B, T, H, dv]  io_dtype: gradient of out
+ *  dhT         [N, H, dk, dv] fp32 gradient of hT, or NULL (zero)
+ *  dq, dk      [B, T, H, dk]  io_dtype, written
+ *  dv          [B, T, H, dv]  io_dtype, written
+ *  dlog_alpha  [B, T, H, dk]  fp32, written
+ *  dbeta       [B, T, H]      fp32, written
+ *  dh0         [N, H, dk, dv] fp32, written, or NULL (not computed)
+ * Outputs must not alias the inputs or one another.  Alignment, varlen rules
+ * and supported shapes as for kda_chunk_fwd.  Workspace: about 600 KB per
+ * (64-token chunk, head) at dk = dv = 128 from the library pool; heads run in
+ * groups that fit the workspace budget.
+ */
+KDA_API kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta, const float* h0,
+                                   const void* dout, const float* dhT,
+                                   void* dq, void* dk, void* dv, float* dlog_alpha,
+                                   float* dbeta, float* dh0, const int32_t* cu_seqlens,
+                                   int64_t B, int64_t T, int64_t H, int64_t dk_, int64_t dv_,
+                                   float scale, kda_io_dtype_t io_dtype, cudaStream_t stream);
+
+/*
  * Context parallelism: one long sequence split across GPUs (or across calls).
  *
  * The recurrence is linear in the state, so a run of tokens maps any entry
