@@ -405,6 +405,88 @@ def run_decode(args, ws, rank, kda, peaks):
     }
 
 
+def bwd_kernel_flops(kname, cfg):
+    """fp32 flops the named backward kernel evaluates per step (the chunk
+    equations it implements, triangles counted once), per SIMT unit count."""
+    C, dk, dv = CHUNK, cfg.dk, cfg.dv
+    if cfg.lengths is not None:
+        chunks = sum(math.ceil(L / C) for L in cfg.lengths) * cfg.H
+    else:
+        chunks = cfg.B * math.ceil(cfg.T / C) * cfg.H
+    tri = C * (C + 1) / 2
+    per = {
+        "chunk_prep_simt": tri * dk * 4 + C ** 3 / 3 + tri * (dk + dv) * 2,
+        "chunk_state_simt": 4 * C * dk * dv + tri * dv * 2,
+        "bwd_state": 6 * C * dk * dv + tri * dv * 2,
+        "bwd_dense1": 6 * C * dk * dv + 2 * tri * dv * 2,
+        "bwd_dense2": 6 * C * dk * dv + 4 * C * C * dv,
+        "bwd_param": 2 * C ** 3 + C * C * dk * 10,
+    }
+    return per.get(kname, 0.0) * chunks
+
+
+def fp32_alu_peak(clocks):
+    """fp32 FMA peak: 148 SMs x 128 fp32 lanes x 2 flop x the SM clock."""
+    mhz = (clocks or {}).get("sm_max_mhz") or 1965.0
+    return 148 * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def run_backward(args, ws, kda, peaks):
+    """The chunkwise backward (kda_chunk_bwd) on the prefill workload: random
+    bf16 output gradients and fp32 final-state gradients, all six gradients
+    written every step."""
+    cfg = prefill_config(args)
+    inp = W.make_prefill(cfg, "cuda")
+    gen = torch.Generator(device="cuda").manual_seed(cfg.seed + 77)
+    dout = torch.randn((cfg.B, cfg.T, cfg.H, cfg.dv), generator=gen, device="cuda").to(torch.bfloat16)
+    dhT = torch.randn((cfg.N, cfg.H, cfg.dk, cfg.dv), generator=gen, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
+                      dout, h0=inp["h0"], dhT=dhT, cu_seqlens=inp["cu_seqlens"])
+
+    steps = max(1, min(args.steps, args.bwd_steps))
+    for _ in range(min(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    kda.profiler_read(reset=True)
+    kda.profiler_enable(True)
+    with ClockSampler(torch.cuda.current_device()) as clk:
+        barrier(ws)
+        torch.cuda.synchronize()
+        ms = time_region(step, steps, stream)
+        torch.cuda.synchronize()
+        barrier(ws)
+    kda.profiler_enable(False)
+    stats = kda.profiler_read(reset=True)
+    ms = max_over_ranks(ms, ws)
+    clocks = clk.summary()
+    peak = fp32_alu_peak(clocks)
+    kern = max(stats.items(), key=lambda kv: kv[1][2])
+    kname, (kl, ktimed, kms) = kern
+    kflop = bwd_kernel_flops(kname, cfg) / max(1.0, ktimed / steps)
+    k_ms = kms / max(1, ktimed)
+    total_flop = sum(bwd_kernel_flops(k, cfg) for k in stats)
+    res = {
+        "workload": cfg.name.replace("prefill", "backward"), "steps": steps,
+        "ms_per_step": ms / steps, "tokens_per_s": cfg.B * cfg.T * steps * ws / (ms / 1e3),
+        "dtype": "f32 arithmetic, bf16 I/O",
+        "path_TFLOPs": total_flop / (ms / steps / 1e3) / 1e12,
+        "roofline": {"kernel": kname, "bound": "alu", "achieved": kflop / (k_ms / 1e3) / 1e12,
+                     "peak": peak, "unit": "TFLOP/s",
+                     "frac": kflop / (k_ms / 1e3) / 1e12 / peak, "traffic": None,
+                     "ms_per_launch": k_ms, "share_of_step": kms / steps / (ms / steps),
+                     "peak_source": "derived: 148 SMs x 128 fp32 lanes x 2 x max SM clock"},
+        "kernels": {k: {"launches": v[0], "ms": v[2]} for k, v in stats.items() if v[0]},
+        "gpu_launches": sum(v[0] for v in stats.values()),
+        "clocks": clocks,
+    }
+    del inp, dout, dhT
+    torch.cuda.empty_cache()
+    return res
+
+
 def run_variants(args, ws, kda, peaks):
     """The serving and Gated DeltaNet entry points on the benchmark shapes:
     GDN prefill (one gate per token and head) on B=8, H=32, T=8192, and the
@@ -502,7 +584,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--bwd-steps", type=int, default=3,
+                    help="timed steps of the backward leg (at most --steps)")
+    ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
                     help="restrict the run (profiling of one kernel family)")
     ap.add_argument("--decode-steps", type=int, default=W.DECODE.steps)
     ap.add_argument("--workload", choices=["batched", "single", "varlen"], default="batched",
@@ -531,6 +616,11 @@ def main():
             if rank == 0:
                 print(json.dumps(res), flush=True)
             return
+        if args.only == "backward":
+            res = {"backward": run_backward(args, ws, kda, peaks)}
+            if rank == 0:
+                print(json.dumps(res), flush=True)
+            return
         res, inp, step, bufs = run_prefill(args, ws, rank, kda, peaks)
         if not args.no_e2e and args.only == "all":
             res["e2e"] = run_e2e(args, ws, kda, inp, bufs, steps=min(args.steps, 3))
@@ -540,6 +630,9 @@ def main():
             res["decode"] = run_decode(args, ws, rank, kda, peaks)
             torch.cuda.empty_cache()
             res["variants"] = run_variants(args, ws, kda, peaks)
+        if not args.no_backward and args.only == "all":
+            torch.cuda.empty_cache()
+            res["backward"] = run_backward(args, ws, kda, peaks)
         if rank == 0 and not args.no_cpu and args.only == "all":
             cfg = W.BATCHED
             heads, batch = cfg.H, 2

@@ -91,3 +91,39 @@ def test_backward_without_dh0(kda):
                      host(inp["beta"]), inp["scale"], host(dout), dhT=host(dhT))
     for g, r in zip(got[:5], ref[:5]):
         assert rel(g, r) <= 1e-5
+
+
+def _full_size(kda, cfg, pairs):
+    """GPU backward on the whole workload; oracle on the listed (sequence, head)
+    pairs (each run alone, h0 and dhT sliced)."""
+    inp = W.make_prefill(cfg, "cuda")
+    dout, dhT = _upstream(cfg, inp, 17)
+    got = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
+                        dout, h0=inp["h0"], dhT=dhT)
+    torch.cuda.synchronize()
+    worst = dict.fromkeys(NAMES, 0.0)
+    for n, h in pairs:
+        sl = lambda x: host(x[n:n + 1, :, h:h + 1])
+        st = lambda x: None if x is None else host(x[n:n + 1, h:h + 1])
+        ref = oracle.bwd(sl(inp["q"]), sl(inp["k"]), sl(inp["v"]), sl(inp["log_alpha"]),
+                         sl(inp["beta"]), inp["scale"], sl(dout), h0=st(inp["h0"]), dhT=st(dhT))
+        mine = [sl(g) for g in got[:5]] + [st(got[5])]
+        for name, g, r in zip(NAMES, mine, ref):
+            worst[name] = max(worst[name], rel(g, r))
+    print(f"PARITY bwd {cfg.name} pairs={len(pairs)} " +
+          " ".join(f"{k}={v:.3e}" for k, v in worst.items()))
+    for name, e in worst.items():
+        assert e <= TOL["bf16"][name], (cfg.name, name, e)
+
+
+def test_backward_full_16_head_workload(kda):
+    """B=1, H=16, T=4096, d=128, bf16, h0 ~ N(0, 0.02): all 16 pairs."""
+    _full_size(kda, W.SINGLE, [(0, h) for h in range(W.SINGLE.H)])
+
+
+@pytest.mark.slow
+def test_backward_full_batched_workload_sampled(kda):
+    """B=8, H=32, T=8192, d=128, bf16: 4 sampled (sequence, head) pairs."""
+    rng = np.random.default_rng(2)
+    pairs = [(int(rng.integers(8)), int(rng.integers(32))) for _ in range(4)]
+    _full_size(kda, W.BATCHED, pairs)
