@@ -336,12 +336,12 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     float* sQ = sK + C * DK;          // [C][DK]
     float* sG = sQ + C * DK;          // [C][DK]  cumulative log-decay
     float* sdG = sG + C * DK;         // [C][DK]
-    float* sT = sdG + C * DK;         // [C][C]
-    float* sAp = sT + C * C;          // [C][C]   A', then dA' = diag(beta) dA
-    float* sdT = sAp + C * C;         // [C][C]   dT', then dT = dT' diag(beta)
-    float* sX = sdT + C * C;          // [C][C]   dT T^T, then dA
-    float* sdAqk = sX + C * C;        // [C][C]
-    float* sB = sdAqk + C * C;        // [C]
+    float* sAp = sdG + C * DK;        // [C][C]   A', then dA' = diag(beta) dA
+    float* sdAqk = sAp + C * C;       // [C][C]   dAqk, then scale dAqk
+    float* sT = sdAqk + C * C;        // [C][C]   T          } free after dA: scratch of the
+    float* sdT = sT + C * C;          // [C][C]   dT', dT    } pairwise terms, 2 x [48][DK]
+    float* sX = sdT + C * C;          // [C][C]   dT T^T, dA }
+    float* sB = sX + C * C;           // [C]
     float* sdB = sB + C;              // [C]
 
     const int64_t gc = blockIdx.x;
@@ -415,47 +415,114 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     for (int e = tid; e < C * C; e += kBT) sAp[e] = sB[e / C] * sX[e];
     __syncthreads();
 
-    // pairwise products and elementwise terms, element (i, c)
+    // Pairwise terms, sub-chunk by sub-chunk (16 rows).  For the rows i of sub-chunk p,
+    // with L = scale dAqk:
+    //   X1 = sum_{j<i}  dA'_ij k_j e^{G_i - G_j}     X3 = sum_{j<=i} L_ij k_j e^{G_i - G_j}
+    //   X2 = sum_{j>i}  dA'_ji k_j e^{G_j - G_i}     X4 = sum_{j>=i} L_ji q_j e^{G_j - G_i}
+    // then dk = X1 + X2 + X4, dq = X3, dG = k (X1 - X2 - X4) + q X3.  Off the diagonal
+    // block the exponential splits at the sub-chunk boundary into two factors <= 1,
+    // e^{G_i - G_f} e^{G_f - G_j} (f = first row, j before it) and e^{G_j - G_e} e^{G_e - G_i}
+    // (e = last row, j after it), so those sums are products with Z = k e^{G_f - G},
+    // k e^{G - G_e}, q e^{G - G_e}; inside the diagonal block they are taken pairwise.
     const float* dKG = blk + BW::dKG;
     const float* dQG = blk + BW::dQG;
     const float* dKh = blk + BW::dKh;
     const float* gam = blk + SW::Gam;
-    for (int e = tid; e < C * DK; e += kBT) {
-        const int i = e / DK, c = e % DK;
-        const float gi = sG[e], ki = sK[e], qi = sQ[e];
-        float dk = 0.f, dq = 0.f, dg = 0.f;
-        for (int j = 0; j < C; ++j) {
-            const float kj = sK[j * DK + c], gj = sG[j * DK + c];
-            if (j < i) {
-                const float ex = expf(gi - gj);
-                const float x = sAp[i * C + j] * ex;
-                const float y = scale * sdAqk[i * C + j] * ex;
-                dk += x * kj;
-                dq += y * kj;
-                dg += (x * ki + y * qi) * kj;
-            } else if (j > i) {
-                const float ex = expf(gj - gi);
-                const float x = sAp[j * C + i] * ex;
-                const float y = scale * sdAqk[j * C + i] * ex;
-                const float qj = sQ[j * DK + c];
-                dk += x * kj + y * qj;
-                dg -= (x * kj + y * qj) * ki;
-            } else {
-                const float y = scale * sdAqk[i * C + i];
-                dq += y * ki;
-                dk += y * qi;
+    for (int e = tid; e < C * C; e += kBT) sdAqk[e] *= scale;
+    constexpr int NM = DK / 16;
+    const int ti = tid >> 4, tc = tid & 15;           // row within the sub-chunk, channel group
+    float* Z1 = sT;                                   // [48][DK]
+    float* Z2 = sT + 48 * DK;                         // [48][DK]
+    for (int p = 0; p < 4; ++p) {
+        const int f = 16 * p, el = f + 15, nu = C - 1 - el;
+        const int i = f + ti;
+        float x1[NM], x2[NM], x3[NM], x4[NM];
+        __syncthreads();                              // scratch free, dA', L final
+        for (int e = tid; e < f * DK; e += kBT) {
+            const int c = e % DK;
+            Z1[e] = sK[e] * expf(sG[f * DK + c] - sG[e]);
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NM; ++m) { x1[m] = 0.f; x3[m] = 0.f; }
+        for (int j = 0; j < f; ++j) {
+            const float a1 = sAp[i * C + j], a3 = sdAqk[i * C + j];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const float z = Z1[j * DK + tc + 16 * m];
+                x1[m] += a1 * z;
+                x3[m] += a3 * z;
             }
         }
-        const float eg = expf(gi), egl = expf(sG[(C - 1) * DK + c] - gi);
-        dq += scale * eg * dQG[e];
-        dg += scale * qi * eg * dQG[e];
-        dk += egl * dKh[e] + eg * dKG[e];
-        dg += ki * eg * dKG[e] - ki * egl * dKh[e];
-        sdG[e] = dg;
-        if (i < len) {
-            const int64_t dst = ((t0 + i) * H + h) * DK + c;
-            IO<T>::store((T*)b.dq, dst, dq);
-            IO<T>::store((T*)b.dk, dst, dk);
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+            const int c = tc + 16 * m;
+            const float fac = expf(sG[i * DK + c] - sG[f * DK + c]);
+            x1[m] *= fac;
+            x3[m] *= fac;
+        }
+        for (int j = f; j <= i; ++j) {                // diagonal block, j <= i
+            const float a1 = (j < i) ? sAp[i * C + j] : 0.f, a3 = sdAqk[i * C + j];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const int c = tc + 16 * m;
+                const float kz = sK[j * DK + c] * expf(sG[i * DK + c] - sG[j * DK + c]);
+                x1[m] += a1 * kz;
+                x3[m] += a3 * kz;
+            }
+        }
+        __syncthreads();                              // Z1 is refilled below
+        for (int e = tid; e < nu * DK; e += kBT) {
+            const int j = el + 1 + e / DK, c = e % DK;
+            const float ex = expf(sG[j * DK + c] - sG[el * DK + c]);
+            Z1[e] = sK[j * DK + c] * ex;
+            Z2[e] = sQ[j * DK + c] * ex;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int m = 0; m < NM; ++m) { x2[m] = 0.f; x4[m] = 0.f; }
+        for (int jj = 0; jj < nu; ++jj) {
+            const int j = el + 1 + jj;
+            const float a2 = sAp[j * C + i], a4 = sdAqk[j * C + i];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                x2[m] += a2 * Z1[jj * DK + tc + 16 * m];
+                x4[m] += a4 * Z2[jj * DK + tc + 16 * m];
+            }
+        }
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+            const int c = tc + 16 * m;
+            const float fac = expf(sG[el * DK + c] - sG[i * DK + c]);
+            x2[m] *= fac;
+            x4[m] *= fac;
+        }
+        for (int j = i; j <= el; ++j) {               // diagonal block, j >= i
+            const float a2 = (j > i) ? sAp[j * C + i] : 0.f, a4 = sdAqk[j * C + i];
+#pragma unroll
+            for (int m = 0; m < NM; ++m) {
+                const int c = tc + 16 * m;
+                const float ex = expf(sG[j * DK + c] - sG[i * DK + c]);
+                x2[m] += a2 * sK[j * DK + c] * ex;
+                x4[m] += a4 * sQ[j * DK + c] * ex;
+            }
+        }
+        // gradients of element (i, c): the pairwise part and the elementwise terms
+#pragma unroll
+        for (int m = 0; m < NM; ++m) {
+            const int c = tc + 16 * m, e = i * DK + c;
+            const float gi = sG[e], ki = sK[e], qi = sQ[e];
+            const float eg = expf(gi), egl = expf(sG[(C - 1) * DK + c] - gi);
+            const float dqg = dQG[e], dkg = dKG[e], dkh = dKh[e];
+            const float dk = x1[m] + x2[m] + x4[m] + egl * dkh + eg * dkg;
+            const float dq = x3[m] + scale * eg * dqg;
+            sdG[e] = ki * (x1[m] - x2[m] - x4[m]) + qi * x3[m] + scale * qi * eg * dqg +
+                     ki * eg * dkg - ki * egl * dkh;
+            if (i < len) {
+                const int64_t dst = ((t0 + i) * H + h) * DK + c;
+                IO<T>::store((T*)b.dq, dst, dq);
+                IO<T>::store((T*)b.dk, dst, dk);
+            }
         }
     }
     __syncthreads();
