@@ -33,11 +33,15 @@
 namespace kda {
 
 constexpr int kBT = 256;          // threads of every backward kernel
-constexpr int kTW = 32;           // dv columns per walk tile / dense tile
 
 // ---------------------------------------------------------------------------
 // reverse walk: per (sequence, head, 32-column tile)
 // ---------------------------------------------------------------------------
+constexpr int kAP = 68;           // row pitch of the transposed Aqk
+
+// dS stays in registers across chunks: thread (warp w, lane) owns row c = 32 (w mod DK/32)
+// + lane and NJ consecutive columns of the 32-column tile (NJ = 16 for DK = 128, 8 for 64);
+// it is copied to shared memory once per chunk as the operand of Khat dS'.
 template <typename T, int DK, int DV>
 __global__ void __launch_bounds__(kBT)
 chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
@@ -45,17 +49,18 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     using BW = BwdWs<DK, DV>;
     using SW = SimtWs<DK, DV>;
     constexpr int C = kChunk;
+    constexpr int RG = DK / 32;       // groups of 32 rows
     const SeqInfo& si = b.si;
     const int64_t H = b.H;
-    extern __shared__ float smem[];
+    extern __shared__ __align__(16) float smem[];
     float* sW = smem;                 // [C][DK]
     float* sQG = sW + C * DK;         // [C][DK]
     float* sKh = sQG + C * DK;        // [C][DK]
-    float* sAqk = sKh + C * DK;       // [C][C]
-    float* sdO = sAqk + C * C;        // [C][32]
+    float* sAqkT = sKh + C * DK;      // [C][kAP]  Aqk transposed
+    float* sdO = sAqkT + C * kAP;     // [C][32]
     float* sdE = sdO + C * kTW;       // [C][32]
-    float* sdS = sdE + C * kTW;       // [DK][32]
-    float* sGam = sdS + DK * kTW;     // [DK]
+    float* sdS = sdE + C * kTW;       // [DK][kSP]
+    float* sGam = sdS + DK * kSP;     // [DK]
 
     const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
     const int64_t tiles = DV / kTW;
@@ -72,65 +77,75 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     const int64_t sidx = n * H + h;
     const T* __restrict__ dout = (const T*)b.dout;
 
-    for (int e = tid; e < DK * kTW; e += kBT) {
-        const int c = e / kTW, j = e % kTW;
-        sdS[e] = b.dhT ? b.dhT[sidx * DK * DV + c * DV + j0 + j] : 0.f;
-    }
+    constexpr int NCW = 8 / RG;                       // warps sharing one row group
+    constexpr int NJ = kTW / NCW;                     // columns per thread
+    const int c = 32 * (wrp % RG) + lane;
+    const int jb = NJ * (wrp / RG);
+    float ds[NJ];
+#pragma unroll
+    for (int x = 0; x < NJ; ++x)
+        ds[x] = b.dhT ? b.dhT[sidx * DK * DV + (int64_t)c * DV + j0 + jb + x] : 0.f;
+
     for (int64_t ch = nchunks - 1; ch >= 0; --ch) {
         float* blk = ws + ((gc0 + ch) * Hg + hl) * BW::size;
         const int64_t t0 = bos + ch * C;
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-        __syncthreads();
-        for (int e = tid; e < C * DK; e += kBT) {
-            sW[e] = blk[SW::W + e];
-            sQG[e] = blk[SW::QG + e];
-            sKh[e] = blk[SW::KG + e];
+        __syncthreads();                              // previous chunk's reads are done
+        for (int e = tid; e < C * DK / 4; e += kBT) {
+            reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
+            reinterpret_cast<float4*>(sQG)[e] = reinterpret_cast<const float4*>(blk + SW::QG)[e];
+            reinterpret_cast<float4*>(sKh)[e] = reinterpret_cast<const float4*>(blk + SW::KG)[e];
         }
-        for (int e = tid; e < C * C; e += kBT) sAqk[e] = blk[SW::Aqk + e];
-        for (int c = tid; c < DK; c += kBT) sGam[c] = blk[SW::Gam + c];
+        for (int e = tid; e < C * C; e += kBT) {
+            const int r = e / C, t = e % C;           // Aqk[r][t] -> AqkT[t][r]
+            sAqkT[t * kAP + r] = blk[SW::Aqk + e];
+        }
+        for (int cc = tid; cc < DK; cc += kBT) sGam[cc] = blk[SW::Gam + cc];
         for (int e = tid; e < C * kTW; e += kBT) {
             const int t = e / kTW, j = e % kTW;
             sdO[e] = t < len ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
         }
-        for (int e = tid; e < DK * kTW; e += kBT)          // gradient of this chunk's exit state
-            blk[BW::dSx + (e / kTW) * DV + j0 + (e % kTW)] = sdS[e];
-        __syncthreads();
-        // dE = Aqk^T dO + Khat dS'
-        for (int t = wrp; t < C; t += 8) {
-            float acc = 0.f;
-            for (int s = t; s < C; ++s) acc += sAqk[s * C + t] * sdO[s * kTW + lane];
-            for (int c = 0; c < DK; ++c) acc += sKh[t * DK + c] * sdS[c * kTW + lane];
-            sdE[t * kTW + lane] = acc;
-        }
-        __syncthreads();
-        // dS = Diag(e^{G_last}) dS' + Q_G^T dO - W^T dE
-        for (int c = wrp; c < DK; c += 8) {
-            float acc = sGam[c] * sdS[c * kTW + lane];
-            for (int t = 0; t < C; ++t)
-                acc += sQG[t * DK + c] * sdO[t * kTW + lane] - sW[t * DK + c] * sdE[t * kTW + lane];
-            sdS[c * kTW + lane] = acc;
-        }
-    }
-    __syncthreads();
-    if (b.dh0)
-        for (int e = tid; e < DK * kTW; e += kBT)
-            b.dh0[sidx * DK * DV + (e / kTW) * DV + j0 + (e % kTW)] = sdS[e];
-}
-
-// acc[r] += sum_k A[(row0 + 8 r) * lda + k] * B[k * 32 + lane] (A rows read as
-// 16-byte broadcasts, B columns one per lane), r < 8, K a multiple of 4.
-__device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int lda, int row0,
-                                          const float* B, int K, int lane)
-{
-    for (int k = 0; k < K; k += 4) {
-        const float b0 = B[k * kTW + lane], b1 = B[(k + 1) * kTW + lane];
-        const float b2 = B[(k + 2) * kTW + lane], b3 = B[(k + 3) * kTW + lane];
+        // this chunk's exit-state gradient: to shared memory (for dE) and to the workspace
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const float4 a = *reinterpret_cast<const float4*>(A + (row0 + 8 * r) * lda + k);
-            acc[r] += a.x * b0 + a.y * b1 + a.z * b2 + a.w * b3;
+        for (int x = 0; x < NJ; x += 4) {
+            const float4 v4 = make_float4(ds[x], ds[x + 1], ds[x + 2], ds[x + 3]);
+            *reinterpret_cast<float4*>(sdS + c * kSP + jb + x) = v4;
+            *reinterpret_cast<float4*>(blk + BW::dSx + (int64_t)c * DV + j0 + jb + x) = v4;
+        }
+        __syncthreads();
+        // dE = Aqk^T dO + Khat dS': rows t = w + 8 r, column lane
+        {
+            float acc[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+            rows8_mac<kTW>(acc, sAqkT, kAP, wrp, sdO, C, lane);
+            rows8_mac<kSP>(acc, sKh, DK, wrp, sdS, DK, lane);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) sdE[(wrp + 8 * r) * kTW + lane] = acc[r];
+        }
+        __syncthreads();
+        // dS = Diag(e^{G_last}) dS' + Q_G^T dO - W^T dE  (row c, columns jb .. jb + NJ - 1)
+        {
+            const float gmc = sGam[c];
+#pragma unroll
+            for (int x = 0; x < NJ; ++x) ds[x] *= gmc;
+            for (int t = 0; t < C; ++t) {
+                const float qg = sQG[t * DK + c], wv = sW[t * DK + c];
+#pragma unroll
+                for (int x = 0; x < NJ; x += 4) {
+                    const float4 o4 = *reinterpret_cast<const float4*>(sdO + t * kTW + jb + x);
+                    const float4 e4 = *reinterpret_cast<const float4*>(sdE + t * kTW + jb + x);
+                    ds[x] += qg * o4.x - wv * e4.x;
+                    ds[x + 1] += qg * o4.y - wv * e4.y;
+                    ds[x + 2] += qg * o4.z - wv * e4.z;
+                    ds[x + 3] += qg * o4.w - wv * e4.w;
+                }
+            }
         }
     }
+    if (b.dh0)
+#pragma unroll
+        for (int x = 0; x < NJ; ++x) b.dh0[sidx * DK * DV + (int64_t)c * DV + j0 + jb + x] = ds[x];
 }
 
 // ---------------------------------------------------------------------------
@@ -149,13 +164,15 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
     float* sW = smem;                 // [C][DK]
     float* sKG = sW + C * DK;         // [C][DK]   K e^G
     float* sKh = sKG + C * DK;        // [C][DK]   K e^{G_last - G}
-    float* sAqk = sKh + C * DK;       // [C][C]
-    float* sT = sAqk + C * C;         // [C][C]
-    float* sS = sT + C * C;           // [DK][32]
+    float* sAqkT = sKh + C * DK;      // [C][kAP]  Aqk transposed
+    float* sTT = sAqkT + C * kAP;     // [C][kAP]  diag(beta) T^T
+    float* sS = sTT + C * kAP;        // [DK][32]
     float* sdSn = sS + DK * kTW;      // [DK][32]
     float* sdO = sdSn + DK * kTW;     // [C][32]
     float* sdE = sdO + C * kTW;       // [C][32]
-    float* sB = sdE + C * kTW;        // [C]
+    float* sUt = sdE + C * kTW;       // [C][32]
+    float* sV = sUt + C * kTW;        // [C][32]
+    float* sB = sV + C * kTW;         // [C]
 
     const int64_t gc = blockIdx.x;
     const int hl = blockIdx.y;
@@ -169,16 +186,18 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
     const T* __restrict__ v = (const T*)b.v;
     T* __restrict__ dv = (T*)b.dv;
 
-    for (int e = tid; e < C * DK; e += kBT) {
-        sW[e] = blk[SW::W + e];
-        sKG[e] = blk[BW::KGm + e];
-        sKh[e] = blk[SW::KG + e];
-    }
-    for (int e = tid; e < C * C; e += kBT) {
-        sAqk[e] = blk[SW::Aqk + e];
-        sT[e] = blk[BW::Tm + e];
+    for (int e = tid; e < C * DK / 4; e += kBT) {
+        reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
+        reinterpret_cast<float4*>(sKG)[e] = reinterpret_cast<const float4*>(blk + BW::KGm)[e];
+        reinterpret_cast<float4*>(sKh)[e] = reinterpret_cast<const float4*>(blk + SW::KG)[e];
     }
     for (int t = tid; t < C; t += kBT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
+    __syncthreads();
+    for (int e = tid; e < C * C; e += kBT) {
+        const int r = e / C, t = e % C;               // Aqk[r][t] -> AqkT[t][r]; T likewise,
+        sAqkT[t * kAP + r] = blk[SW::Aqk + e];        // with row t of T^T scaled by beta_t
+        sTT[t * kAP + r] = blk[BW::Tm + e] * sB[t];
+    }
     float glS = 0.f;                                  // thread c < DK: sum_v S[c][v] dS'[c][v]
 
     for (int j0 = 0; j0 < DV; j0 += kTW) {
@@ -190,7 +209,10 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
         }
         for (int e = tid; e < C * kTW; e += kBT) {
             const int t = e / kTW, j = e % kTW;
-            sdO[e] = t < len ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+            const bool ok = t < len;
+            sdO[e] = ok ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+            sV[e] = ok ? IO<T>::load(v, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+            sUt[e] = blk[SW::Ut + t * DV + j0 + j];
         }
         __syncthreads();
         if (tid < DK)
@@ -199,34 +221,31 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
         float e8[8], r8[8], de8[8];
 #pragma unroll
         for (int r = 0; r < 8; ++r) { e8[r] = 0.f; r8[r] = 0.f; de8[r] = 0.f; }
-        rows8_mac(e8, sW, DK, wrp, sS, DK, lane);      // W S
-        rows8_mac(r8, sKG, DK, wrp, sS, DK, lane);     // K_G S
-        rows8_mac(de8, sKh, DK, wrp, sdSn, DK, lane);  // Khat dS'
+        rows8_mac(e8, sW, DK, wrp, sS, DK, lane);        // W S
+        rows8_mac(r8, sKG, DK, wrp, sS, DK, lane);       // K_G S
+        rows8_mac(de8, sKh, DK, wrp, sdSn, DK, lane);    // Khat dS'
+        rows8_mac(de8, sAqkT, kAP, wrp, sdO, C, lane);   // + Aqk^T dO
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
             const int t = wrp + 8 * r;
-            const float ut = blk[SW::Ut + t * DV + j0 + lane];
-            const float vt = t < len ? IO<T>::load(v, ((t0 + t) * H + h) * DV + j0 + lane) : 0.f;
-            e8[r] = ut - e8[r];
-            r8[r] = vt - r8[r];
-            float acc = 0.f;                            // Aqk^T dO
-            for (int s = t; s < C; ++s) acc += sAqk[s * C + t] * sdO[s * kTW + lane];
-            de8[r] += acc;
+            e8[r] = sUt[t * kTW + lane] - e8[r];
+            r8[r] = sV[t * kTW + lane] - r8[r];
             sdE[t * kTW + lane] = de8[r];
             blk[BW::E + t * DV + j0 + lane] = e8[r];
             blk[BW::R + t * DV + j0 + lane] = r8[r];
             blk[BW::dE + t * DV + j0 + lane] = de8[r];
         }
         __syncthreads();
-        // dR = diag(beta) T^T dE  (T lower: T[s][t] != 0 only for s >= t)
+        // dR = diag(beta) T^T dE
+        float dr8[8];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) dr8[r] = 0.f;
+        rows8_mac(dr8, sTT, kAP, wrp, sdE, C, lane);
 #pragma unroll
         for (int r = 0; r < 8; ++r) {
             const int t = wrp + 8 * r;
-            float acc = 0.f;
-            for (int s = t; s < C; ++s) acc += sT[s * C + t] * sdE[s * kTW + lane];
-            acc *= sB[t];
-            blk[BW::dR + t * DV + j0 + lane] = acc;
-            if (t < len) IO<T>::store(dv, ((t0 + t) * H + h) * DV + j0 + lane, acc);
+            blk[BW::dR + t * DV + j0 + lane] = dr8[r];
+            if (t < len) IO<T>::store(dv, ((t0 + t) * H + h) * DV + j0 + lane, dr8[r]);
         }
     }
     if (tid < DK) blk[BW::dGlS + tid] = glS;
@@ -542,9 +561,9 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
 }
 
 template <int DK, int DV>
-constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kChunk + 2 * kChunk * kTW + DK * kTW + DK); }
+constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kAP + 2 * kChunk * kTW + DK * kSP + DK); }
 template <int DK, int DV>
-constexpr size_t bwd_dense1_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + 2 * kChunk * kChunk + 2 * DK * kTW + 2 * kChunk * kTW + kChunk); }
+constexpr size_t bwd_dense1_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + 2 * kChunk * kAP + 2 * DK * kTW + 4 * kChunk * kTW + kChunk); }
 template <int DK, int DV>
 constexpr size_t bwd_param_smem() { return sizeof(float) * (size_t)(4 * kChunk * DK + 5 * kChunk * kChunk + 2 * kChunk); }
 

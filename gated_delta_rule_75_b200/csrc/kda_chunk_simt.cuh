@@ -8,6 +8,27 @@
 
 namespace kda {
 
+constexpr int kTW = 32;           // dv columns per state-walk tile
+constexpr int kSP = 36;           // row pitch of a [DK][32] state tile in shared memory:
+                                  // 16-byte accesses by 8 consecutive rows hit distinct banks
+
+// acc[r] += sum_k A[(row0 + 8 r) * lda + k] * B[k * ldb + lane] (A rows read as
+// 16-byte broadcasts, B columns one per lane), r < 8, K a multiple of 4.
+template <int LDB = kTW>
+__device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int lda, int row0,
+                                          const float* B, int K, int lane)
+{
+    for (int k = 0; k < K; k += 4) {
+        const float b0 = B[k * LDB + lane], b1 = B[(k + 1) * LDB + lane];
+        const float b2 = B[(k + 2) * LDB + lane], b3 = B[(k + 3) * LDB + lane];
+#pragma unroll
+        for (int r = 0; r < 8; ++r) {
+            const float4 a = *reinterpret_cast<const float4*>(A + (row0 + 8 * r) * lda + k);
+            acc[r] += a.x * b0 + a.y * b1 + a.z * b2 + a.w * b3;
+        }
+    }
+}
+
 // Workspace block of one (chunk, head), in floats.
 template <int DK, int DV>
 struct SimtWs {
@@ -51,12 +72,12 @@ struct BwdWs {
 template <int DK, int DV>
 constexpr size_t simt_prep_smem()
 {
-    return sizeof(float) * (size_t)(kChunk * (3 * DK + DV) + 2 * kChunk * kChunk + kChunk);
+    return sizeof(float) * (size_t)(kChunk * (3 * DK + DV) + 2 * kChunk * kChunk + kChunk + 32 * DK + 48 * (DK + 4));
 }
 template <int DK, int DV>
 constexpr size_t simt_state_smem()
 {
-    return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kChunk + kChunk * 32 + DK * 32 + DK);
+    return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kChunk + kChunk * kTW + DK * kSP + DK);
 }
 
 
@@ -79,6 +100,10 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     float* sA = sG + C * DK;          // [C][C]
     float* sT = sA + C * C;           // [C][C]
     float* sB = sT + C * C;           // [C]
+    float* sKin = sB + C;             // [16][DK]  rows of one sub-chunk, referenced to its first row
+    float* sQin = sKin + 16 * DK;     // [16][DK]
+    constexpr int KVP = DK + 4;       // padded row pitch of sKvar (16 rows -> distinct banks)
+    float* sKvar = sQin + 16 * DK;    // [48][KVP] earlier rows, referenced forward to it
 
     const int64_t gc = blockIdx.x;
     const int hl = blockIdx.y;
@@ -110,22 +135,73 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     __syncthreads();
 
     float* blk = ws + (gc * Hg + hl) * (kBwd ? BwdWs<DK, DV>::size : SimtWs<DK, DV>::size);
-    // (b1) A (strictly lower, beta-weighted) and Aqk (lower incl. diagonal)
-    for (int pidx = tid; pidx < C * C; pidx += blockDim.x) {
-        const int i = pidx / C, j = pidx % C;
-        float kk = 0.f, qk = 0.f;
-        if (j <= i) {
-            for (int cc = 0; cc < DK; ++cc) {
-                const int c = (cc + j) % DK;        // rotate to spread banks
-                const float e = expf(sG[i * DK + c] - sG[j * DK + c]);
-                const float kj = sK[j * DK + c] * e;
-                kk += sK[i * DK + c] * kj;
-                qk += sQ[i * DK + c] * kj;
+    // (b1) A (strictly lower, beta-weighted) and Aqk (lower incl. diagonal), one 16-row
+    // sub-chunk of rows i at a time.  For columns j before the sub-chunk (first row f) the
+    // exponential splits into two factors <= 1, e^{G_i - G_f} e^{G_f - G_j}, so the sums are
+    // dot products of precomputed rows; inside the diagonal block it is taken pairwise.
+    for (int e = tid; e < C * C; e += blockDim.x) {
+        sA[e] = 0.f;
+        sT[e] = 0.f;
+        if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + e] = 0.f;
+    }
+    for (int p = 0; p < C / 16; ++p) {
+        const int f = 16 * p;
+        __syncthreads();                          // zeros written, scratch rows free
+        for (int e = tid; e < 16 * DK; e += blockDim.x) {
+            const int i = f + e / DK, c = e % DK;
+            const float x = expf(sG[i * DK + c] - sG[f * DK + c]);
+            sKin[e] = sK[i * DK + c] * x;
+            sQin[e] = sQ[i * DK + c] * x;
+        }
+        for (int e = tid; e < f * DK; e += blockDim.x) {
+            const int j = e / DK, c = e % DK;
+            sKvar[j * KVP + c] = sK[e] * expf(sG[f * DK + c] - sG[e]);
+        }
+        __syncthreads();
+        if (tid < 256) {                          // rows f .. f+15, columns jg + 16 u < f
+            // lanes run along the columns (padded Kvar rows), the row is a broadcast
+            const int r = tid >> 4, jg = tid & 15, i = f + r;
+            float kk[3] = {0.f, 0.f, 0.f}, qk[3] = {0.f, 0.f, 0.f};
+            for (int c = 0; c < DK; c += 4) {
+                const float4 a = *reinterpret_cast<const float4*>(sKin + r * DK + c);
+                const float4 q4 = *reinterpret_cast<const float4*>(sQin + r * DK + c);
+#pragma unroll
+                for (int u = 0; u < 3; ++u) {
+                    if (u < p) {
+                        const float4 kv = *reinterpret_cast<const float4*>(sKvar + (jg + 16 * u) * KVP + c);
+                        kk[u] += a.x * kv.x + a.y * kv.y + a.z * kv.z + a.w * kv.w;
+                        qk[u] += q4.x * kv.x + q4.y * kv.y + q4.z * kv.z + q4.w * kv.w;
+                    }
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < 3; ++u) {
+                if (u < p) {
+                    const int j = jg + 16 * u;
+                    sA[i * C + j] = sB[i] * kk[u];
+                    sT[i * C + j] = scale * qk[u];   // Aqk parked in sT for now
+                    if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = kk[u];
+                }
+            }
+            // diagonal block: pair (i, j = f + jg) when j <= i; lanes differ in j, so the
+            // rotated channel index spreads them over the banks
+            const int j = f + jg;
+            if (j <= i) {
+                float dk_ = 0.f, dq_ = 0.f;
+                for (int cc = 0; cc < DK; ++cc) {
+                    const int c = (cc + j) % DK;    // rotate to spread banks
+                    const float e = expf(sG[i * DK + c] - sG[j * DK + c]);
+                    const float kj = sK[j * DK + c] * e;
+                    dk_ += sK[i * DK + c] * kj;
+                    dq_ += sQ[i * DK + c] * kj;
+                }
+                if (j < i) {
+                    sA[i * C + j] = sB[i] * dk_;
+                    if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = dk_;
+                }
+                sT[i * C + j] = scale * dq_;
             }
         }
-        sA[pidx] = (j < i) ? sB[i] * kk : 0.f;
-        sT[pidx] = (j <= i) ? scale * qk : 0.f;   // Aqk parked in sT for now
-        if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + pidx] = (j < i) ? kk : 0.f;
     }
     __syncthreads();
 
@@ -189,15 +265,15 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     const SeqInfo& si = a.si;
     const int64_t H = a.H;
     T* __restrict__ out = (T*)a.out;
-    constexpr int C = kChunk, TW = 32;
-    extern __shared__ float smem[];
+    constexpr int C = kChunk, TW = kTW;
+    extern __shared__ __align__(16) float smem[];
     float* sW = smem;                 // [C][DK]
     float* sQG = sW + C * DK;         // [C][DK]
     float* sKG = sQG + C * DK;        // [C][DK]
     float* sAqk = sKG + C * DK;       // [C][C]
     float* sU = sAqk + C * C;         // [C][TW]
-    float* sS = sU + C * TW;          // [DK][TW]
-    float* sGam = sS + DK * TW;       // [DK]
+    float* sS = sU + C * TW;          // [DK][kSP]  copy of the entry state
+    float* sGam = sS + DK * kSP;      // [DK]
 
     // blocks run (tile, head)-innermost over sequences ranked longest first
     const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
@@ -216,57 +292,81 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     const int64_t sidx = a.state_index(n, h);
     const float* h0p = (a.h0 && sidx >= 0) ? a.h0 + sidx * DK * DV : nullptr;
     float* hTp = (a.hT && sidx >= 0) ? a.hT + sidx * DK * DV : nullptr;
-    for (int e = tid; e < DK * TW; e += blockDim.x) {
-        const int c = e / TW, j = e % TW;
-        sS[e] = h0p ? h0p[c * DV + j0 + j] : 0.f;
-    }
+    // the state tile lives in registers: thread (warp w, lane) owns row c = 32 (w mod DK/32)
+    // + lane and NJ consecutive columns (NJ = 16 for DK = 128, 8 for DK = 64)
+    constexpr int RG = DK / 32, NJ = TW / (8 / RG);
+    const int c = 32 * (wrp % RG) + lane, jb = NJ * (wrp / RG);
+    float st[NJ];
+#pragma unroll
+    for (int x = 0; x < NJ; ++x) st[x] = h0p ? h0p[(int64_t)c * DV + j0 + jb + x] : 0.f;
+
     for (int64_t ch = 0; ch < nchunks; ++ch) {
         float* blk = ws + ((gc0 + ch) * Hg + hl) * kStride;
         const int64_t t0 = bos + ch * C;
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-        __syncthreads();
-        for (int e = tid; e < C * DK; e += blockDim.x) {
-            sW[e] = blk[SimtWs<DK, DV>::W + e];
-            sQG[e] = blk[SimtWs<DK, DV>::QG + e];
-            sKG[e] = blk[SimtWs<DK, DV>::KG + e];
+        __syncthreads();                          // the previous chunk's reads are done
+        for (int e = tid; e < C * DK / 4; e += blockDim.x) {
+            reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::W)[e];
+            reinterpret_cast<float4*>(sQG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::QG)[e];
+            reinterpret_cast<float4*>(sKG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::KG)[e];
         }
-        for (int e = tid; e < C * C; e += blockDim.x) sAqk[e] = blk[SimtWs<DK, DV>::Aqk + e];
+        for (int e = tid; e < C * C / 4; e += blockDim.x)
+            reinterpret_cast<float4*>(sAqk)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::Aqk)[e];
         for (int e = tid; e < C * TW; e += blockDim.x)
             sU[e] = blk[SimtWs<DK, DV>::Ut + (e / TW) * DV + j0 + (e % TW)];
-        for (int c = tid; c < DK; c += blockDim.x) sGam[c] = blk[SimtWs<DK, DV>::Gam + c];
-        if constexpr (kBwd)
-            for (int e = tid; e < DK * TW; e += blockDim.x)
-                blk[BwdWs<DK, DV>::Sx + (e / TW) * DV + j0 + (e % TW)] = sS[e];
-        __syncthreads();
-        // U = Ut - W S
-        for (int t = wrp; t < C; t += 8) {
-            float acc = 0.f;
-            for (int c = 0; c < DK; ++c) acc += sW[t * DK + c] * sS[c * TW + lane];
-            sU[t * TW + lane] -= acc;
+        for (int cc = tid; cc < DK; cc += blockDim.x) sGam[cc] = blk[SimtWs<DK, DV>::Gam + cc];
+#pragma unroll
+        for (int x = 0; x < NJ; x += 4) {
+            const float4 v4 = make_float4(st[x], st[x + 1], st[x + 2], st[x + 3]);
+            *reinterpret_cast<float4*>(sS + c * kSP + jb + x) = v4;
+            if constexpr (kBwd)
+                *reinterpret_cast<float4*>(blk + BwdWs<DK, DV>::Sx + (int64_t)c * DV + j0 + jb + x) = v4;
         }
         __syncthreads();
-        // O = scale (Q e^G) S + Aqk U   (uses the entry state)
-        for (int t = wrp; !kBwd && t < len; t += 8) {
-            float acc = 0.f;
-            for (int c = 0; c < DK; ++c) acc += sQG[t * DK + c] * sS[c * TW + lane];
-            for (int s = 0; s <= t; ++s) acc += sAqk[t * C + s] * sU[s * TW + lane];
-            IO<T>::store(out, ((t0 + t) * H + h) * DV + j0 + lane, acc);
+        // U = Ut - W S: rows t = w + 8 r, column lane
+        {
+            float acc[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+            rows8_mac<kSP>(acc, sW, DK, wrp, sS, DK, lane);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) sU[(wrp + 8 * r) * TW + lane] -= acc[r];
         }
         __syncthreads();
-        // S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U
-        for (int c = wrp; c < DK; c += 8) {
-            float acc = sGam[c] * sS[c * TW + lane];
-            for (int t = 0; t < C; ++t) acc += sKG[t * DK + c] * sU[t * TW + lane];
-            sS[c * TW + lane] = acc;
+        // O = scale (Q e^G) S + Aqk U   (the entry state; Aqk is zero above the diagonal)
+        if constexpr (!kBwd) {
+            float acc[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) acc[r] = 0.f;
+            rows8_mac<kSP>(acc, sQG, DK, wrp, sS, DK, lane);
+            rows8_mac<TW>(acc, sAqk, C, wrp, sU, C, lane);
+#pragma unroll
+            for (int r = 0; r < 8; ++r) {
+                const int t = wrp + 8 * r;
+                if (t < len) IO<T>::store(out, ((t0 + t) * H + h) * DV + j0 + lane, acc[r]);
+            }
+        }
+        // S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U, in registers
+        {
+            const float gmc = sGam[c];
+#pragma unroll
+            for (int x = 0; x < NJ; ++x) st[x] *= gmc;
+            for (int t = 0; t < C; ++t) {
+                const float kg = sKG[t * DK + c];
+#pragma unroll
+                for (int x = 0; x < NJ; x += 4) {
+                    const float4 u4 = *reinterpret_cast<const float4*>(sU + t * TW + jb + x);
+                    st[x] += kg * u4.x;
+                    st[x + 1] += kg * u4.y;
+                    st[x + 2] += kg * u4.z;
+                    st[x + 3] += kg * u4.w;
+                }
+            }
         }
     }
-    __syncthreads();
-    if (hTp) {
-        for (int e = tid; e < DK * TW; e += blockDim.x) {
-            const int c = e / TW, j = e % TW;
-            hTp[c * DV + j0 + j] = sS[e];
-        }
-    }
+    if (hTp)
+#pragma unroll
+        for (int x = 0; x < NJ; ++x) hTp[(int64_t)c * DV + j0 + jb + x] = st[x];
 }
 
 }  // namespace kda
