@@ -420,7 +420,7 @@ def bwd_kernel_flops(kname, cfg):
         "bwd_state": 6 * C * dk * dv + tri * dv * 2,
         "bwd_dense1": 6 * C * dk * dv + 2 * tri * dv * 2,
         "bwd_dense2": 6 * C * dk * dv + 4 * C * C * dv,
-        "bwd_param": 2 * C ** 3 + C * C * dk * 10,
+        "bwd_param": 2 * C ** 3 + 4 * C * C * dk,   # dA through the inverse; 4 pairwise sums
     }
     return per.get(kname, 0.0) * chunks
 
