@@ -127,3 +127,18 @@ def test_backward_full_batched_workload_sampled(kda):
     rng = np.random.default_rng(2)
     pairs = [(int(rng.integers(8)), int(rng.integers(32))) for _ in range(4)]
     _full_size(kda, W.BATCHED, pairs)
+
+
+def test_backward_empty_inputs(kda):
+    """T = 0: no token gradients, dh0 = dhT; packed batch of empty sequences likewise."""
+    for lengths in (None, [0, 0, 0]):
+        cfg = (W.small_prefill(B=2, T=0, H=2, dk=64, dv=64, io_dtype="f32", seed=1, h0_std=0.1)
+               if lengths is None else
+               W.small_prefill(H=2, dk=64, dv=64, io_dtype="f32", seed=1, h0_std=0.1, lengths=lengths))
+        inp = W.make_prefill(cfg, "cuda")
+        dout, dhT = _upstream(cfg, inp, 3)
+        got = kda.chunk_bwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                            inp["scale"], dout, h0=inp["h0"], dhT=dhT, cu_seqlens=inp["cu_seqlens"])
+        torch.cuda.synchronize()
+        torch.testing.assert_close(got[5], dhT, rtol=0, atol=0)
+        assert all(g.numel() == 0 for g in got[:5])

@@ -187,3 +187,30 @@ def test_context_parallel_pieces(kda, io, d, cuts):
     eo, eh = rel(out, ro), rel(hT, rh)
     print(f"PARITY context_parallel_{io}_d{d}_cuts{len(cuts) - 1} out={eo:.3e} hT={eh:.3e}")
     assert eo <= TOL[io] and eh <= TOL[io]
+
+
+def test_context_parallel_helper_over_nccl_one_rank(kda):
+    """chunk_fwd_context_parallel with the library's own ops and an NCCL process
+    group of one rank (the all-gather runs, the composition has no predecessor):
+    the product path end to end, against the oracle."""
+    import datetime
+    import os
+    import socket
+    import torch.distributed as dist
+    from gated_delta_rule_75_b200.context_parallel import chunk_fwd_context_parallel
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    store = dist.TCPStore("127.0.0.1", port, 1, True, timeout=datetime.timedelta(seconds=30))
+    dist.init_process_group("nccl", store=store, rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60))
+    try:
+        cfg = W.small_prefill(B=2, T=300, H=2, dk=128, dv=128, io_dtype="bf16", seed=15, h0_std=0.02)
+        inp = W.make_prefill(cfg, "cuda")
+        out, hT = chunk_fwd_context_parallel(inp["q"], inp["k"], inp["v"], inp["log_alpha"],
+                                             inp["beta"], inp["scale"], h0=inp["h0"])
+        torch.cuda.synchronize()
+        ro, rh = oracle_prefill(inp)
+        assert rel(out, ro) <= TOL["bf16"] and rel(hT, rh) <= TOL["bf16"]
+    finally:
+        dist.destroy_process_group()
