@@ -323,7 +323,10 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
     if (impl < KDA_PREFILL_AUTO || impl > KDA_PREFILL_TENSORCORE_SEGMENTED)
         return KDA_ERR_INVALID_ARG;
-    const bool tc_shape = io_dtype == KDA_IO_BF16 && dk == 128 && dv == 128;
+    // the tensor-core kernels address token rows with 32-bit TMA coordinates
+    const int64_t T_rows = cu_seqlens ? T : B * T;
+    const bool tc_shape = io_dtype == KDA_IO_BF16 && dk == 128 && dv == 128 &&
+                          T_rows < (int64_t(1) << 31);
     const bool tc_forced = impl != KDA_PREFILL_AUTO && impl != KDA_PREFILL_SIMT;
     if (tc_forced && !tc_shape) return KDA_ERR_UNSUPPORTED;
     const bool use_tc = tc_forced || (impl == KDA_PREFILL_AUTO && tc_shape);

@@ -81,7 +81,7 @@ typedef enum {
 typedef enum {
     KDA_PREFILL_AUTO = 0,      /* tensor cores for bf16 with dk = dv = 128, SIMT otherwise */
     KDA_PREFILL_SIMT = 1,      /* fp32 SIMT chunk kernels (any supported shape / dtype) */
-    KDA_PREFILL_TENSORCORE = 2, /* tcgen05 chunk kernels; bf16, dk = dv = 128 only */
+    KDA_PREFILL_TENSORCORE = 2, /* tcgen05 chunk kernels; bf16, dk = dv = 128, < 2^31 token rows */
     KDA_PREFILL_TENSORCORE_CHAIN = 3,     /* tcgen05, one chain per (sequence, head) */
     KDA_PREFILL_TENSORCORE_SEGMENTED = 4  /* tcgen05, segment-parallel walk */
 } kda_prefill_impl_t;
