@@ -52,12 +52,13 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     constexpr int RG = DK / 32;       // groups of 32 rows
     const SeqInfo& si = b.si;
     const int64_t H = b.H;
+    // Two operand buffers, reloaded between the two phases of a chunk so that two CTAs
+    // fit on an SM: X = Khat then W, Y = Aqk^T (pitch kAP) then Q_G.
     extern __shared__ __align__(16) float smem[];
-    float* sW = smem;                 // [C][DK]
-    float* sQG = sW + C * DK;         // [C][DK]
-    float* sKh = sQG + C * DK;        // [C][DK]
-    float* sAqkT = sKh + C * DK;      // [C][kAP]  Aqk transposed
-    float* sdO = sAqkT + C * kAP;     // [C][32]
+    constexpr int YW = DK > kAP ? DK : kAP;
+    float* sX = smem;                 // [C][DK]
+    float* sY = sX + C * YW;          // [C][YW]
+    float* sdO = sY + C * YW;         // [C][32]
     float* sdE = sdO + C * kTW;       // [C][32]
     float* sdS = sdE + C * kTW;       // [DK][kSP]
     float* sGam = sdS + DK * kSP;     // [DK]
@@ -91,14 +92,11 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         const int64_t t0 = bos + ch * C;
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
         __syncthreads();                              // previous chunk's reads are done
-        for (int e = tid; e < C * DK / 4; e += kBT) {
-            reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
-            reinterpret_cast<float4*>(sQG)[e] = reinterpret_cast<const float4*>(blk + SW::QG)[e];
-            reinterpret_cast<float4*>(sKh)[e] = reinterpret_cast<const float4*>(blk + SW::KG)[e];
-        }
+        for (int e = tid; e < C * DK / 4; e += kBT)
+            reinterpret_cast<float4*>(sX)[e] = reinterpret_cast<const float4*>(blk + SW::KG)[e];
         for (int e = tid; e < C * C; e += kBT) {
             const int r = e / C, t = e % C;           // Aqk[r][t] -> AqkT[t][r]
-            sAqkT[t * kAP + r] = blk[SW::Aqk + e];
+            sY[t * kAP + r] = blk[SW::Aqk + e];
         }
         for (int cc = tid; cc < DK; cc += kBT) sGam[cc] = blk[SW::Gam + cc];
         for (int e = tid; e < C * kTW; e += kBT) {
@@ -118,10 +116,15 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
             float acc[8];
 #pragma unroll
             for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-            rows8_mac<kTW>(acc, sAqkT, kAP, wrp, sdO, C, lane);
-            rows8_mac<kSP>(acc, sKh, DK, wrp, sdS, DK, lane);
+            rows8_mac<kTW>(acc, sY, kAP, wrp, sdO, C, lane);
+            rows8_mac<kSP>(acc, sX, DK, wrp, sdS, DK, lane);
 #pragma unroll
             for (int r = 0; r < 8; ++r) sdE[(wrp + 8 * r) * kTW + lane] = acc[r];
+        }
+        __syncthreads();
+        for (int e = tid; e < C * DK / 4; e += kBT) {
+            reinterpret_cast<float4*>(sX)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
+            reinterpret_cast<float4*>(sY)[e] = reinterpret_cast<const float4*>(blk + SW::QG)[e];
         }
         __syncthreads();
         // dS = Diag(e^{G_last}) dS' + Q_G^T dO - W^T dE  (row c, columns jb .. jb + NJ - 1)
@@ -130,7 +133,7 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
 #pragma unroll
             for (int x = 0; x < NJ; ++x) ds[x] *= gmc;
             for (int t = 0; t < C; ++t) {
-                const float qg = sQG[t * DK + c], wv = sW[t * DK + c];
+                const float qg = sY[t * DK + c], wv = sX[t * DK + c];
 #pragma unroll
                 for (int x = 0; x < NJ; x += 4) {
                     const float4 o4 = *reinterpret_cast<const float4*>(sdO + t * kTW + jb + x);
@@ -561,7 +564,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
 }
 
 template <int DK, int DV>
-constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kAP + 2 * kChunk * kTW + DK * kSP + DK); }
+constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(2 * kChunk * (DK > kAP ? DK : kAP) + 2 * kChunk * kTW + DK * kSP + DK); }
 template <int DK, int DV>
 constexpr size_t bwd_dense1_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + 2 * kChunk * kAP + 2 * DK * kTW + 4 * kChunk * kTW + kChunk); }
 template <int DK, int DV>
@@ -578,7 +581,7 @@ static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaS
                                       (int)simt_prep_smem<DK, DV>())))
             return r;
         if ((r = cudaFuncSetAttribute(chunk_state_simt_kernel<T, DK, DV, true>, (cudaFuncAttribute)mx,
-                                      (int)simt_state_smem<DK, DV>())))
+                                      (int)simt_state_smem<DK, DV, true>())))
             return r;
         if ((r = cudaFuncSetAttribute(chunk_bwd_state_kernel<T, DK, DV>, (cudaFuncAttribute)mx,
                                       (int)bwd_state_smem<DK, DV>())))
@@ -611,7 +614,7 @@ static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaS
         const dim3 gwalk((unsigned)(si.N * hg * (DV / kTW)));
         {
             LaunchScope scope(st, K_STATE_SIMT);
-            chunk_state_simt_kernel<T, DK, DV, true><<<gwalk, 256, simt_state_smem<DK, DV>(), st>>>(
+            chunk_state_simt_kernel<T, DK, DV, true><<<gwalk, 256, simt_state_smem<DK, DV, true>(), st>>>(
                 ws, a, hb, Hg);
             if ((e = cudaGetLastError())) return e;
         }

@@ -74,10 +74,11 @@ constexpr size_t simt_prep_smem()
 {
     return sizeof(float) * (size_t)(kChunk * (3 * DK + DV) + 2 * kChunk * kChunk + kChunk + 32 * DK + 48 * (DK + 4));
 }
-template <int DK, int DV>
+template <int DK, int DV, bool kBwd = false>
 constexpr size_t simt_state_smem()
 {
-    return sizeof(float) * (size_t)(3 * kChunk * DK + kChunk * kChunk + kChunk * kTW + DK * kSP + DK);
+    return sizeof(float) * (size_t)((kBwd ? 2 : 3) * kChunk * DK + (kBwd ? 0 : kChunk * kChunk) +
+                                    kChunk * kTW + DK * kSP + DK);
 }
 
 
@@ -267,13 +268,14 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     T* __restrict__ out = (T*)a.out;
     constexpr int C = kChunk, TW = kTW;
     extern __shared__ __align__(16) float smem[];
-    float* sW = smem;                 // [C][DK]
-    float* sQG = sW + C * DK;         // [C][DK]
-    float* sKG = sQG + C * DK;        // [C][DK]
-    float* sAqk = sKG + C * DK;       // [C][C]
-    float* sU = sAqk + C * C;         // [C][TW]
-    float* sS = sU + C * TW;          // [DK][kSP]  copy of the entry state
-    float* sGam = sS + DK * kSP;      // [DK]
+    // (the backward walk writes no output: no Q e^G, no Aqk, and half the shared memory)
+    float* sW = smem;                                  // [C][DK]
+    float* sKG = sW + C * DK;                          // [C][DK]
+    float* sU = sKG + C * DK;                          // [C][TW]
+    float* sS = sU + C * TW;                           // [DK][kSP]  copy of the entry state
+    float* sGam = sS + DK * kSP;                       // [DK]
+    float* sQG = sGam + DK;                            // [C][DK]    (forward only)
+    float* sAqk = sQG + C * DK;                        // [C][C]     (forward only)
 
     // blocks run (tile, head)-innermost over sequences ranked longest first
     const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
@@ -307,11 +309,13 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
         __syncthreads();                          // the previous chunk's reads are done
         for (int e = tid; e < C * DK / 4; e += blockDim.x) {
             reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::W)[e];
-            reinterpret_cast<float4*>(sQG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::QG)[e];
             reinterpret_cast<float4*>(sKG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::KG)[e];
+            if constexpr (!kBwd)
+                reinterpret_cast<float4*>(sQG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::QG)[e];
         }
-        for (int e = tid; e < C * C / 4; e += blockDim.x)
-            reinterpret_cast<float4*>(sAqk)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::Aqk)[e];
+        if constexpr (!kBwd)
+            for (int e = tid; e < C * C / 4; e += blockDim.x)
+                reinterpret_cast<float4*>(sAqk)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::Aqk)[e];
         for (int e = tid; e < C * TW; e += blockDim.x)
             sU[e] = blk[SimtWs<DK, DV>::Ut + (e / TW) * DV + j0 + (e % TW)];
         for (int cc = tid; cc < DK; cc += blockDim.x) sGam[cc] = blk[SimtWs<DK, DV>::Gam + cc];
