@@ -32,7 +32,9 @@
 
 namespace kda {
 
-constexpr int kBT = 256;          // threads of every backward kernel
+constexpr int kBT = 256;          // threads of the backward kernels
+constexpr int kPT = 512;          // threads of the parameter kernel (one CTA per SM: more warps)
+constexpr int kD1T = 512;         // threads of dense pass 1 (likewise)
 
 // ---------------------------------------------------------------------------
 // reverse walk: per (sequence, head, 32-column tile)
@@ -155,7 +157,7 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
 // dense pass 1: per (chunk, head)
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kBT)
+__global__ void __launch_bounds__(kD1T)
 chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
@@ -189,14 +191,14 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
     const T* __restrict__ v = (const T*)b.v;
     T* __restrict__ dv = (T*)b.dv;
 
-    for (int e = tid; e < C * DK / 4; e += kBT) {
+    for (int e = tid; e < C * DK / 4; e += kD1T) {
         reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
         reinterpret_cast<float4*>(sKG)[e] = reinterpret_cast<const float4*>(blk + BW::KGm)[e];
         reinterpret_cast<float4*>(sKh)[e] = reinterpret_cast<const float4*>(blk + SW::KG)[e];
     }
-    for (int t = tid; t < C; t += kBT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
+    for (int t = tid; t < C; t += kD1T) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
     __syncthreads();
-    for (int e = tid; e < C * C; e += kBT) {
+    for (int e = tid; e < C * C; e += kD1T) {
         const int r = e / C, t = e % C;               // Aqk[r][t] -> AqkT[t][r]; T likewise,
         sAqkT[t * kAP + r] = blk[SW::Aqk + e];        // with row t of T^T scaled by beta_t
         sTT[t * kAP + r] = blk[BW::Tm + e] * sB[t];
@@ -205,12 +207,12 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
 
     for (int j0 = 0; j0 < DV; j0 += kTW) {
         __syncthreads();
-        for (int e = tid; e < DK * kTW; e += kBT) {
+        for (int e = tid; e < DK * kTW; e += kD1T) {
             const int c = e / kTW, j = e % kTW;
             sS[e] = blk[BW::Sx + c * DV + j0 + j];
             sdSn[e] = blk[BW::dSx + c * DV + j0 + j];
         }
-        for (int e = tid; e < C * kTW; e += kBT) {
+        for (int e = tid; e < C * kTW; e += kD1T) {
             const int t = e / kTW, j = e % kTW;
             const bool ok = t < len;
             sdO[e] = ok ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
@@ -220,17 +222,18 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
         __syncthreads();
         if (tid < DK)
             for (int j = 0; j < kTW; ++j) glS += sS[tid * kTW + j] * sdSn[tid * kTW + j];
-        // rows w, w+8, ..., w+56 of this warp; column j0 + lane
-        float e8[8], r8[8], de8[8];
+        // rows w, w + NW, ... of this warp (NW warps); column j0 + lane
+        constexpr int NW = kD1T / 32, NR = C / NW;
+        float e8[NR], r8[NR], de8[NR];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) { e8[r] = 0.f; r8[r] = 0.f; de8[r] = 0.f; }
-        rows8_mac(e8, sW, DK, wrp, sS, DK, lane);        // W S
-        rows8_mac(r8, sKG, DK, wrp, sS, DK, lane);       // K_G S
-        rows8_mac(de8, sKh, DK, wrp, sdSn, DK, lane);    // Khat dS'
-        rows8_mac(de8, sAqkT, kAP, wrp, sdO, C, lane);   // + Aqk^T dO
+        for (int r = 0; r < NR; ++r) { e8[r] = 0.f; r8[r] = 0.f; de8[r] = 0.f; }
+        rows_mac<NR, NW, kTW>(e8, sW, DK, wrp, sS, DK, lane);        // W S
+        rows_mac<NR, NW, kTW>(r8, sKG, DK, wrp, sS, DK, lane);       // K_G S
+        rows_mac<NR, NW, kTW>(de8, sKh, DK, wrp, sdSn, DK, lane);    // Khat dS'
+        rows_mac<NR, NW, kTW>(de8, sAqkT, kAP, wrp, sdO, C, lane);   // + Aqk^T dO
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int t = wrp + 8 * r;
+        for (int r = 0; r < NR; ++r) {
+            const int t = wrp + NW * r;
             e8[r] = sUt[t * kTW + lane] - e8[r];
             r8[r] = sV[t * kTW + lane] - r8[r];
             sdE[t * kTW + lane] = de8[r];
@@ -240,13 +243,13 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
         }
         __syncthreads();
         // dR = diag(beta) T^T dE
-        float dr8[8];
+        float dr8[NR];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) dr8[r] = 0.f;
-        rows8_mac(dr8, sTT, kAP, wrp, sdE, C, lane);
+        for (int r = 0; r < NR; ++r) dr8[r] = 0.f;
+        rows_mac<NR, NW, kTW>(dr8, sTT, kAP, wrp, sdE, C, lane);
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const int t = wrp + 8 * r;
+        for (int r = 0; r < NR; ++r) {
+            const int t = wrp + NW * r;
             blk[BW::dR + t * DV + j0 + lane] = dr8[r];
             if (t < len) IO<T>::store(dv, ((t0 + t) * H + h) * DV + j0 + lane, dr8[r]);
         }
@@ -345,7 +348,7 @@ chunk_bwd_dense2_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
 // parameter gradients: per (chunk, head)
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kBT)
+__global__ void __launch_bounds__(kPT)
 chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
@@ -378,7 +381,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     const T* __restrict__ k = (const T*)b.k;
     const float scale = b.scale;
 
-    for (int e = tid; e < C * DK; e += kBT) {
+    for (int e = tid; e < C * DK; e += kPT) {
         const int t = e / DK, c = e % DK;
         const bool ok = t < len;
         const int64_t src = ((t0 + t) * H + h) * DK + c;
@@ -386,13 +389,13 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
         sG[e] = ok ? b.log_alpha[src] : 0.f;
     }
-    for (int e = tid; e < C * C; e += kBT) {
+    for (int e = tid; e < C * C; e += kPT) {
         sT[e] = blk[BW::Tm + e];
         sAp[e] = blk[BW::Ap + e];
         sdT[e] = blk[BW::dTp + e];
         sdAqk[e] = blk[BW::dAqk + e];
     }
-    for (int t = tid; t < C; t += kBT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
+    for (int t = tid; t < C; t += kPT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
     __syncthreads();
     if (tid < DK) {                                   // G = cumsum(g) per channel
         float run = 0.f;
@@ -405,10 +408,10 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         sdB[tid] = acc;
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += kBT) sdT[e] *= sB[e % C];   // dT = dT' diag(beta)
+    for (int e = tid; e < C * C; e += kPT) sdT[e] *= sB[e % C];   // dT = dT' diag(beta)
     __syncthreads();
     // X = dT T^T:  X[r][j] = sum_m dT[r][m] T[j][m]  (T[j][m] = 0 for m > j)
-    for (int e = tid; e < C * C; e += kBT) {
+    for (int e = tid; e < C * C; e += kPT) {
         const int r = e / C, j = e % C;
         float acc = 0.f;
         for (int m = 0; m <= j; ++m) acc += sdT[r * C + m] * sT[j * C + m];
@@ -416,16 +419,17 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     }
     __syncthreads();
     // dA[i][j] = -sum_r T[r][i] X[r][j]  (i > j; T[r][i] = 0 for r < i)
-    float dA[16];
-    for (int u = 0; u < 16; ++u) {
-        const int e = tid + kBT * u, i = e / C, j = e % C;
+    constexpr int NU = C * C / kPT;
+    float dA[NU];
+    for (int u = 0; u < NU; ++u) {
+        const int e = tid + kPT * u, i = e / C, j = e % C;
         float acc = 0.f;
         if (j < i)
             for (int r = i; r < C; ++r) acc += sT[r * C + i] * sX[r * C + j];
         dA[u] = -acc;
     }
     __syncthreads();
-    for (int u = 0; u < 16; ++u) sX[tid + kBT * u] = dA[u];
+    for (int u = 0; u < NU; ++u) sX[tid + kPT * u] = dA[u];
     __syncthreads();
     // dbeta_i += sum_{j<i} dA[i][j] A'[i][j];  dA' = diag(beta) dA
     if (tid < C) {
@@ -434,7 +438,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         sdB[tid] += acc;
     }
     __syncthreads();
-    for (int e = tid; e < C * C; e += kBT) sAp[e] = sB[e / C] * sX[e];
+    for (int e = tid; e < C * C; e += kPT) sAp[e] = sB[e / C] * sX[e];
     __syncthreads();
 
     // Pairwise terms, sub-chunk by sub-chunk (16 rows).  For the rows i of sub-chunk p,
@@ -450,9 +454,10 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     const float* dQG = blk + BW::dQG;
     const float* dKh = blk + BW::dKh;
     const float* gam = blk + SW::Gam;
-    for (int e = tid; e < C * C; e += kBT) sdAqk[e] *= scale;
-    constexpr int NM = DK / 16;
-    const int ti = tid >> 4, tc = tid & 15;           // row within the sub-chunk, channel group
+    for (int e = tid; e < C * C; e += kPT) sdAqk[e] *= scale;
+    constexpr int NG = kPT / 16;                      // channel groups (lanes along channels)
+    constexpr int NM = DK / NG;                       // channels per thread
+    const int ti = tid / NG, tc = tid % NG;           // row within the sub-chunk, channel group
     float* Z1 = sT;                                   // [48][DK]
     float* Z2 = sT + 48 * DK;                         // [48][DK]
     for (int p = 0; p < 4; ++p) {
@@ -460,7 +465,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         const int i = f + ti;
         float x1[NM], x2[NM], x3[NM], x4[NM];
         __syncthreads();                              // scratch free, dA', L final
-        for (int e = tid; e < f * DK; e += kBT) {
+        for (int e = tid; e < f * DK; e += kPT) {
             const int c = e % DK;
             Z1[e] = sK[e] * expf(sG[f * DK + c] - sG[e]);
         }
@@ -471,14 +476,14 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
             const float a1 = sAp[i * C + j], a3 = sdAqk[i * C + j];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
-                const float z = Z1[j * DK + tc + 16 * m];
+                const float z = Z1[j * DK + tc + NG * m];
                 x1[m] += a1 * z;
                 x3[m] += a3 * z;
             }
         }
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            const int c = tc + 16 * m;
+            const int c = tc + NG * m;
             const float fac = expf(sG[i * DK + c] - sG[f * DK + c]);
             x1[m] *= fac;
             x3[m] *= fac;
@@ -487,14 +492,14 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
             const float a1 = (j < i) ? sAp[i * C + j] : 0.f, a3 = sdAqk[i * C + j];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
-                const int c = tc + 16 * m;
+                const int c = tc + NG * m;
                 const float kz = sK[j * DK + c] * expf(sG[i * DK + c] - sG[j * DK + c]);
                 x1[m] += a1 * kz;
                 x3[m] += a3 * kz;
             }
         }
         __syncthreads();                              // Z1 is refilled below
-        for (int e = tid; e < nu * DK; e += kBT) {
+        for (int e = tid; e < nu * DK; e += kPT) {
             const int j = el + 1 + e / DK, c = e % DK;
             const float ex = expf(sG[j * DK + c] - sG[el * DK + c]);
             Z1[e] = sK[j * DK + c] * ex;
@@ -508,13 +513,13 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
             const float a2 = sAp[j * C + i], a4 = sdAqk[j * C + i];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
-                x2[m] += a2 * Z1[jj * DK + tc + 16 * m];
-                x4[m] += a4 * Z2[jj * DK + tc + 16 * m];
+                x2[m] += a2 * Z1[jj * DK + tc + NG * m];
+                x4[m] += a4 * Z2[jj * DK + tc + NG * m];
             }
         }
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            const int c = tc + 16 * m;
+            const int c = tc + NG * m;
             const float fac = expf(sG[el * DK + c] - sG[i * DK + c]);
             x2[m] *= fac;
             x4[m] *= fac;
@@ -523,7 +528,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
             const float a2 = (j > i) ? sAp[j * C + i] : 0.f, a4 = sdAqk[j * C + i];
 #pragma unroll
             for (int m = 0; m < NM; ++m) {
-                const int c = tc + 16 * m;
+                const int c = tc + NG * m;
                 const float ex = expf(sG[j * DK + c] - sG[i * DK + c]);
                 x2[m] += a2 * sK[j * DK + c] * ex;
                 x4[m] += a4 * sQ[j * DK + c] * ex;
@@ -532,7 +537,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         // gradients of element (i, c): the pairwise part and the elementwise terms
 #pragma unroll
         for (int m = 0; m < NM; ++m) {
-            const int c = tc + 16 * m, e = i * DK + c;
+            const int c = tc + NG * m, e = i * DK + c;
             const float gi = sG[e], ki = sK[e], qi = sQ[e];
             const float eg = expf(gi), egl = expf(sG[(C - 1) * DK + c] - gi);
             const float dqg = dQG[e], dkg = dKG[e], dkh = dKh[e];
@@ -606,7 +611,7 @@ static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaS
         const dim3 gchunk((unsigned)si.chunks_upper, (unsigned)hg);
         if (si.chunks_upper > 0) {
             LaunchScope scope(st, K_PREP_SIMT);
-            chunk_prep_simt_kernel<T, DK, DV, true><<<gchunk, 256, simt_prep_smem<DK, DV>(), st>>>(
+            chunk_prep_simt_kernel<T, DK, DV, true><<<gchunk, kSimtPrepThreads, simt_prep_smem<DK, DV>(), st>>>(
                 (const T*)b.q, (const T*)b.k, (const T*)b.v, b.log_alpha, b.beta, si, b.H, hb, Hg,
                 b.scale, ws, 0);
             if ((e = cudaGetLastError())) return e;
@@ -626,7 +631,7 @@ static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaS
         if (si.chunks_upper > 0) {
             {
                 LaunchScope scope(st, K_BWD_DENSE1);
-                chunk_bwd_dense1_kernel<T, DK, DV><<<gchunk, kBT, bwd_dense1_smem<DK, DV>(), st>>>(
+                chunk_bwd_dense1_kernel<T, DK, DV><<<gchunk, kD1T, bwd_dense1_smem<DK, DV>(), st>>>(
                     ws, b, hb, Hg);
                 if ((e = cudaGetLastError())) return e;
             }
@@ -638,7 +643,7 @@ static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaS
             }
             {
                 LaunchScope scope(st, K_BWD_PARAM);
-                chunk_bwd_param_kernel<T, DK, DV><<<gchunk, kBT, bwd_param_smem<DK, DV>(), st>>>(
+                chunk_bwd_param_kernel<T, DK, DV><<<gchunk, kPT, bwd_param_smem<DK, DV>(), st>>>(
                     ws, b, hb, Hg);
                 if ((e = cudaGetLastError())) return e;
             }

@@ -12,21 +12,29 @@ constexpr int kTW = 32;           // dv columns per state-walk tile
 constexpr int kSP = 36;           // row pitch of a [DK][32] state tile in shared memory:
                                   // 16-byte accesses by 8 consecutive rows hit distinct banks
 
-// acc[r] += sum_k A[(row0 + 8 r) * lda + k] * B[k * ldb + lane] (A rows read as
-// 16-byte broadcasts, B columns one per lane), r < 8, K a multiple of 4.
-template <int LDB = kTW>
-__device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int lda, int row0,
-                                          const float* B, int K, int lane)
+// acc[r] += sum_k A[(row0 + RS r) * lda + k] * B[k * LDB + lane], r < NR (A rows read as
+// 16-byte broadcasts, B columns one per lane), K a multiple of 4.
+template <int NR, int RS, int LDB>
+__device__ __forceinline__ void rows_mac(float (&acc)[NR], const float* A, int lda, int row0,
+                                         const float* B, int K, int lane)
 {
     for (int k = 0; k < K; k += 4) {
         const float b0 = B[k * LDB + lane], b1 = B[(k + 1) * LDB + lane];
         const float b2 = B[(k + 2) * LDB + lane], b3 = B[(k + 3) * LDB + lane];
 #pragma unroll
-        for (int r = 0; r < 8; ++r) {
-            const float4 a = *reinterpret_cast<const float4*>(A + (row0 + 8 * r) * lda + k);
+        for (int r = 0; r < NR; ++r) {
+            const float4 a = *reinterpret_cast<const float4*>(A + (row0 + RS * r) * lda + k);
             acc[r] += a.x * b0 + a.y * b1 + a.z * b2 + a.w * b3;
         }
     }
+}
+
+// The eight-warp form: rows row0 + 8 r, r < 8.
+template <int LDB = kTW>
+__device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int lda, int row0,
+                                          const float* B, int K, int lane)
+{
+    rows_mac<8, 8, LDB>(acc, A, lda, row0, B, K, lane);
 }
 
 // Workspace block of one (chunk, head), in floats.
@@ -85,8 +93,10 @@ constexpr size_t simt_state_smem()
 // ---------------------------------------------------------------------------
 // step a + b: cumulative log-decay and intra-chunk transform
 // ---------------------------------------------------------------------------
+constexpr int kSimtPrepThreads = 256;   // 16 rows x 16 column lanes in the A / Aqk phase
+
 template <typename T, int DK, int DV, bool kBwd = false>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(kSimtPrepThreads)
 chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const float* __restrict__ log_alpha, const float* __restrict__ beta,
                        SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
@@ -159,8 +169,8 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
             sKvar[j * KVP + c] = sK[e] * expf(sG[f * DK + c] - sG[e]);
         }
         __syncthreads();
-        if (tid < 256) {                          // rows f .. f+15, columns jg + 16 u < f
-            // lanes run along the columns (padded Kvar rows), the row is a broadcast
+        {   // rows f .. f+15 (r = tid / 16), columns jg + 16 u < f; lanes run along the
+            // columns (padded Kvar rows), the row is a broadcast
             const int r = tid >> 4, jg = tid & 15, i = f + r;
             float kk[3] = {0.f, 0.f, 0.f}, qk[3] = {0.f, 0.f, 0.f};
             for (int c = 0; c < DK; c += 4) {
