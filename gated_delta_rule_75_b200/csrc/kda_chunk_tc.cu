@@ -21,6 +21,9 @@
 //   off-diagonal blocks by tf32 mma.sync block products; W = T' (K e^G) as a
 //   tcgen05 MMA.  It writes one operand image per (chunk, head), already in the
 //   128B-swizzled shared-memory layout the state kernel's MMAs read.
+// Kernel `chunk_prep_gdn_tc` (Gated DeltaNet, one gate per (token, head)): the same
+//   image from two plain MMAs (k k^T, k q^T) and per-token scalings, since a scalar
+//   decay factors out of the key products; three CTAs per SM.
 // Kernel `chunk_state_tc` (one CTA per (sequence, head), steps c and d): walks
 //   the chunks in order with S^T (dv x dk, fp32) resident in tensor memory and
 //   a bf16 copy in shared memory as the MMA operand; each chunk's image (bulk
@@ -174,11 +177,119 @@ struct PrepMaps {
     CUtensorMap k, q, g;
 };
 
-template <bool kScalarGate>
+// Shared tail of the prep kernels, after A (fp32, strictly lower, beta-scaled rows, pitch
+// AP) is in sA and K e^G (bf16, MN-major image rows) in P_K (sT: room for T, pitch AP): T = (I + A)^{-1}, T' = T diag(beta) as a
+// bf16 K-major image (in P_Q and in the workspace), and W = -T' (K e^G) by one MMA whose
+// completion is phase `parity` of `bar`; W goes to the workspace image.  Returns false when
+// the bounded wait gave up.
+__device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img, float* sA, float* sT,
+                                          const float* sB, uint32_t tmem, uint64_t* bar,
+                                          uint32_t parity, int* err)
+{
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int sp = w & 3;                          // TMEM lane quarter of this warp
+    // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution,
+    // one column per thread, held in registers
+    if (tid < C) {
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+        float tcol[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
+            tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -acc);
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
+    }
+    __syncthreads();
+    // off-diagonal blocks, 32 x 32 recursion (X blocks are parked in the unused
+    // upper blocks of A):
+    //   level 1 (warps 0, 1): T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
+    //   level 2: X = A_21 T_1 (rows 2..3, cols 0..1), then T_21 = -T_2 X
+    {
+        auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
+        auto Tb = [&](int r, int c) { return sT + (16 * r) * AP + 16 * c; };
+        if (w < 2) {
+            const int p = 2 * w + 1, r = 2 * w;
+            float acc[2][4] = {};
+            mma16x16x16_tf32<AP>(acc, Ab(p, r), Tb(r, r), l);
+            store16x16<AP>(Ab(r, p), acc, 1.f, l);
+            __syncwarp();
+            float acc2[2][4] = {};
+            mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
+            store16x16<AP>(Tb(p, r), acc2, -1.f, l);
+        }
+        __syncthreads();
+        if (w < 4) {
+            const int p = 2 + (w >> 1), r = w & 1;       // X_pr = sum_{m=r..1} A_pm T_mr
+            float acc[2][4] = {};
+            for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
+            store16x16<AP>(Ab(r, p), acc, 1.f, l);
+        }
+        __syncthreads();
+        if (w < 4) {
+            const int p = 2 + (w >> 1), r = w & 1;       // T_pr = -sum_{m=2..p} T_pm X_mr
+            float acc[2][4] = {};
+            for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
+            store16x16<AP>(Tb(p, r), acc, -1.f, l);
+        }
+        __syncthreads();
+    }
+    // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
+    for (int e = tid; e < C * 8; e += PT) {
+        const int i = e >> 3, cb = e & 7;
+        float f[8], bt[8];
+        ld8f(sT + i * AP + 8 * cb, f);
+        ld8f(sB + 8 * cb, bt);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * bt[x] : 0.f;
+        const uint4 u = pack8(f);
+        *reinterpret_cast<uint4*>(sm + P_Q + sw128_offset(i, 8 * cb)) = u;
+        *reinterpret_cast<uint4*>(img + IMG_T + sw128_offset(i, 8 * cb)) = u;
+    }
+    fence_smem_to_async();
+    fence_before_sync();
+    __syncthreads();
+
+    // ---- (b3) W = T' (K e^G): M = 64 tokens, N = 128 channels, K = 64 tokens
+    if (tid == 0) {
+        fence_after_sync();
+        const uint32_t idesc = make_idesc_bf16(64, 128, false, true, true);   // -T' (K e^G)
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const uint64_t ad = make_desc(smem_u32(sm + P_Q + ks * 32), 16, 1024);
+            const uint64_t bd = make_desc(smem_u32(sm + P_K + ks * 2048), 8192, 1024);
+            mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
+        }
+        commit(bar);
+    }
+    const bool ok = block_wait(bar, parity, err, 3);
+    fence_after_sync();
+    if (ok) {
+        const int i = 16 * sp + l, half = w >> 2;
+        float f[4][16];
+#pragma unroll
+        for (int cb = 0; cb < 4; ++cb)
+            tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 64 * half + 16 * cb, f[cb]);
+        tmem_wait_ld();
+        if (l < 16) {
+            unsigned char* dst = img + IMG_W + half * 8192;
+#pragma unroll
+            for (int cb = 0; cb < 4; ++cb) {
+                *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
+                *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
+            }
+        }
+    }
+    return ok;
+}
+
 __global__ void __launch_bounds__(PT, 2)
 chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
-                     const float* __restrict__ log_a, SeqInfo si, int64_t H, int64_t h_base,
-                     int64_t Hg, float scale, unsigned char* __restrict__ ws, int* __restrict__ err)
+                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
+                     unsigned char* __restrict__ ws, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -202,28 +313,23 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     float* sB = reinterpret_cast<float*>(sm + P_BETA);
     auto G = [&](int t, int c) -> float& { return *reinterpret_cast<float*>(sGb + g_off(t, c)); };
 
-    float* sGs = sB + C;                           // [64] scalar gates (kScalarGate)
     if (tid == 0) {                                // the input loads go out first
         mbar_init(&bar_in, 1);
         mbar_init(&bar, 1);
         fence_mbar_init();
-        tma::expect_tx(&bar_in, kScalarGate ? P_TX - 32768 : P_TX);
+        tma::expect_tx(&bar_in, P_TX);
         const int32_t y = (int32_t)t0, x = (int32_t)(h * D);
         tma::load_2d(sm + P_K, &maps.k, x, y, &bar_in);
         tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_in);
         tma::load_2d(sm + P_Q, &maps.q, x, y, &bar_in);
         tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_in);
-        if (!kScalarGate) {
 #pragma unroll
-            for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
-        }
+        for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
     }
-    // beta (and the scalar gates) meanwhile: their latency overlaps the TMA loads
+    // beta meanwhile: its latency overlaps the TMA loads
     const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
-    const float gval = (kScalarGate && tid < len) ? log_a[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
     if (tid < C) sB[tid] = bval;
-    if (kScalarGate && tid < C) sGs[tid] = gval;
     fence_before_sync();
     bool ok = block_wait(&bar_in, 0, err, 1);      // also the barrier for sB and the TMEM address
     fence_after_sync();
@@ -250,8 +356,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             float v[32];
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-                v[x] = kScalarGate ? sGs[tb + x]
-                                   : *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
+                v[x] = *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
             float run = 0.f;
 #pragma unroll
             for (int x = 0; x < 32; ++x) {
@@ -420,102 +525,182 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         fence_before_sync();
         __syncthreads();
 
-        // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution,
-        // one column per thread, held in registers
-        if (tid < C) {
-            const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-            float tcol[16];
-#pragma unroll
-            for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
-#pragma unroll
-                for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
-                tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -acc);
-            }
-#pragma unroll
-            for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
+        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 0, err);
+    } else {
+        // the input loads may still be in flight: let them land before leaving
+        mbar_wait(&bar_in, 0, nullptr, 0, 200);
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (w == 0) tmem_dealloc(tmem, 128);
+}
+
+// ---------------------------------------------------------------------------
+// Gated DeltaNet prep: one gate per (token, head)
+// ---------------------------------------------------------------------------
+// With a scalar decay per token the pairwise factor e^{G_i - G_j} is the same for every
+// channel, so ("Kimi Delta Attention: la atencion lineal detras de Kimi K2 y Qwen3",
+// comparison of DeltaNet, Gated DeltaNet and KDA; the gate is per head there)
+//   A_ij = beta_i e^{G_i - G_j} (k_i . k_j),   Aqk_ij = scale e^{G_i - G_j} (q_i . k_j)
+// come from two plain MMAs on the loaded k and q tiles, with one exponential per (i, j) at
+// extraction and every factor <= 1; the image rows are k and q scaled per token.  No
+// per-channel operands are built, so the kernel needs 68 KB of shared memory and few
+// registers: three CTAs per SM.
+constexpr uint32_t GP_K = 0;                        // k (TMA, swizzled), later K e^G   16 KB
+constexpr uint32_t GP_Q = 16384;                    // q (TMA), later the T' image      16 KB
+constexpr uint32_t GP_A = 32768;                    // fp32 A [64][AP]                  17 KB
+constexpr uint32_t GP_T = GP_A + 64 * AP * 4;       // fp32 T [64][AP]                  17 KB
+constexpr uint32_t GP_BETA = GP_T + 64 * AP * 4;    // beta [64], cumulative gate [64]
+constexpr uint32_t GP_BYTES = GP_BETA + 512;
+constexpr uint32_t GP_SMEM = GP_BYTES + 1024;
+
+__global__ void __launch_bounds__(PT, 3)
+chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
+                         const float* __restrict__ log_a, SeqInfo si, int64_t H, int64_t h_base,
+                         int64_t Hg, float scale, unsigned char* __restrict__ ws,
+                         int* __restrict__ err)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ uint64_t bar_in, bar;
+    __shared__ uint32_t tmem_base;
+
+    const int64_t gc = blockIdx.x;
+    const int hl = blockIdx.y;
+    const int64_t h = h_base + hl;
+    int64_t n, t0, len;
+    if (!si.locate(gc, n, t0, len)) return;
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int sp = w & 3;                          // TMEM lane quarter of this warp
+    unsigned char* img = ws + (gc * Hg + hl) * (int64_t)IMG_BYTES;
+    float* sB = reinterpret_cast<float*>(sm + GP_BETA);
+    float* sG = sB + C;                            // [64] cumulative gate, log2 units
+
+    if (tid == 0) {                                // the input loads go out first
+        mbar_init(&bar_in, 1);
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+        tma::expect_tx(&bar_in, 32768);
+        const int32_t y = (int32_t)t0, x = (int32_t)(h * D);
+        tma::load_2d(sm + GP_K, &maps.k, x, y, &bar_in);
+        tma::load_2d(sm + GP_K + 8192, &maps.k, x + 64, y, &bar_in);
+        tma::load_2d(sm + GP_Q, &maps.q, x, y, &bar_in);
+        tma::load_2d(sm + GP_Q + 8192, &maps.q, x + 64, y, &bar_in);
+    }
+    const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
+    const float gval = (tid < len) ? log_a[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
+    if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
+    if (tid < C) {
+        sB[tid] = bval;
+        sG[tid] = kLog2e * gval;
+    }
+    fence_before_sync();
+    bool ok = block_wait(&bar_in, 0, err, 1);      // also the barrier for sB, sG and TMEM
+    fence_after_sync();
+    const uint32_t tmem = tmem_base;
+    if (ok && len < C) {
+        // a partial chunk: tokens past its end (next sequence or zero fill) read as zero
+        for (int e = tid; e < (C - (int)len) * 16; e += PT) {
+            const int t = (int)len + (e >> 4), ch = e & 15;
+            const uint32_t off = (ch >> 3) * 8192 + sw128_offset(t, (8 * ch) & 63);
+            *reinterpret_cast<uint4*>(sm + GP_K + off) = make_uint4(0, 0, 0, 0);
+            *reinterpret_cast<uint4*>(sm + GP_Q + off) = make_uint4(0, 0, 0, 0);
         }
-        __syncthreads();
-        // off-diagonal blocks, 32 x 32 recursion (X blocks are parked in the unused
-        // upper blocks of A):
-        //   level 1 (warps 0, 1): T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
-        //   level 2: X = A_21 T_1 (rows 2..3, cols 0..1), then T_21 = -T_2 X
-        {
-            auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
-            auto Tb = [&](int r, int c) { return sT + (16 * r) * AP + 16 * c; };
-            if (w < 2) {
-                const int p = 2 * w + 1, r = 2 * w;
-                float acc[2][4] = {};
-                mma16x16x16_tf32<AP>(acc, Ab(p, r), Tb(r, r), l);
-                store16x16<AP>(Ab(r, p), acc, 1.f, l);
-                __syncwarp();
-                float acc2[2][4] = {};
-                mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
-                store16x16<AP>(Tb(p, r), acc2, -1.f, l);
-            }
-            __syncthreads();
-            if (w < 4) {
-                const int p = 2 + (w >> 1), r = w & 1;       // X_pr = sum_{m=r..1} A_pm T_mr
-                float acc[2][4] = {};
-                for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
-                store16x16<AP>(Ab(r, p), acc, 1.f, l);
-            }
-            __syncthreads();
-            if (w < 4) {
-                const int p = 2 + (w >> 1), r = w & 1;       // T_pr = -sum_{m=2..p} T_pm X_mr
-                float acc[2][4] = {};
-                for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
-                store16x16<AP>(Tb(p, r), acc, -1.f, l);
-            }
-            __syncthreads();
-        }
-        // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
-        for (int e = tid; e < C * 8; e += PT) {
-            const int i = e >> 3, cb = e & 7;
-            float f[8], bt[8];
-            ld8f(sT + i * AP + 8 * cb, f);
-            ld8f(sB + 8 * cb, bt);
+    }
+    if (ok && w == 0) {                            // cumulative gate: lanes hold tokens l, l + 32
+        float a = sG[l], b = sG[l + 32];
 #pragma unroll
-            for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * bt[x] : 0.f;
-            const uint4 u = pack8(f);
-            *reinterpret_cast<uint4*>(sm + P_Q + sw128_offset(i, 8 * cb)) = u;
-            *reinterpret_cast<uint4*>(img + IMG_T + sw128_offset(i, 8 * cb)) = u;
+        for (int o = 1; o < 32; o <<= 1) {
+            const float ua = __shfl_up_sync(0xffffffffu, a, o), ub = __shfl_up_sync(0xffffffffu, b, o);
+            if (l >= o) { a += ua; b += ub; }
+        }
+        b += __shfl_sync(0xffffffffu, a, 31);
+        sG[l] = a;
+        sG[l + 32] = b;
+    }
+    fence_smem_to_async();
+    fence_before_sync();
+    __syncthreads();
+    if (ok && tid == 0) {                          // D1[j][i] = k_j . k_i, D2[j][i] = k_j . q_i
+        fence_after_sync();
+        const uint32_t idesc = make_idesc_bf16(64, 64, false, false);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t o = (ks >> 2) * 8192 + (ks & 3) * 32;
+            const uint64_t kd = make_desc(smem_u32(sm + GP_K + o), 16, 1024);
+            const uint64_t qd = make_desc(smem_u32(sm + GP_Q + o), 16, 1024);
+            mma_bf16(tmem, kd, kd, idesc, ks > 0 ? 1u : 0u);
+            mma_bf16(tmem + 64, kd, qd, idesc, ks > 0 ? 1u : 0u);
+        }
+        commit(&bar);
+    }
+    // while the MMAs run: scale Q e^G and K e^{G_last - G} into the image, e^{G_last}
+    if (ok) {
+        const float gl = sG[C - 1];
+        for (int e = tid; e < C * 16; e += PT) {
+            const int t = e >> 4, cg = e & 15;
+            const uint32_t off = (cg >> 3) * 8192 + sw128_offset(t, (cg & 7) * 8);
+            float kk[8], qq[8], tmp[8];
+            unpack8(*reinterpret_cast<const uint4*>(sm + GP_K + off), kk);
+            unpack8(*reinterpret_cast<const uint4*>(sm + GP_Q + off), qq);
+            const float eqs = scale * ex2(sG[t]), egl = ex2(gl - sG[t]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) tmp[x] = qq[x] * eqs;
+            *reinterpret_cast<uint4*>(img + IMG_QG + off) = pack8(tmp);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) tmp[x] = kk[x] * egl;
+            *reinterpret_cast<uint4*>(img + IMG_B2 + 8192 + off) = pack8(tmp);
+        }
+        if (tid < D) reinterpret_cast<float*>(img + IMG_GAM)[tid] = ex2(gl);
+    }
+    if (ok) ok = block_wait(&bar, 0, err, 2);
+    fence_after_sync();
+    float* sA = reinterpret_cast<float*>(sm + GP_A);
+    float* sT = reinterpret_cast<float*>(sm + GP_T);
+    if (ok) {
+        // K e^G in place (the MMAs are done with k) for W = -T' (K e^G)
+        for (int e = tid; e < C * 16; e += PT) {
+            const int t = e >> 4, cg = e & 15;
+            const uint32_t off = (cg >> 3) * 8192 + sw128_offset(t, (cg & 7) * 8);
+            float kk[8];
+            unpack8(*reinterpret_cast<const uint4*>(sm + GP_K + off), kk);
+            const float eg = ex2(sG[t]);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) kk[x] *= eg;
+            *reinterpret_cast<uint4*>(sm + GP_K + off) = pack8(kk);
+        }
+        // extraction: thread (warp w, lane l < 16) takes key row j = 16 sp + l and query /
+        // row columns i = 32 (w >> 2) .. +31: A (fp32, for the inverse) and Aqk^T (image)
+        const int j = 16 * sp + l, ib = 32 * (w >> 2);
+        float d1[2][16], d2[2][16];
+        const uint32_t lane = (uint32_t)(32 * sp) << 16;
+        tmem_ld16(tmem + lane + ib, d1[0]);
+        tmem_ld16(tmem + lane + ib + 16, d1[1]);
+        tmem_ld16(tmem + lane + 64 + ib, d2[0]);
+        tmem_ld16(tmem + lane + 64 + ib + 16, d2[1]);
+        tmem_wait_ld();
+        if (l < 16) {
+            const float gj = sG[j];
+            float aq[32];
+#pragma unroll
+            for (int x = 0; x < 2; ++x)
+#pragma unroll
+                for (int cc = 0; cc < 16; ++cc) {
+                    const int i = ib + 16 * x + cc;
+                    const float e = (i >= j) ? ex2(sG[i] - gj) : 0.f;    // <= 1
+                    sA[i * AP + j] = (j < i) ? sB[i] * e * d1[x][cc] : 0.f;
+                    aq[16 * x + cc] = scale * e * d2[x][cc];
+                }
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, ib + 8 * m)) = pack8(aq + 8 * m);
         }
         fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
-
-        // ---- (b3) W = T' (K e^G): M = 64 tokens, N = 128 channels, K = 64 tokens
-        if (tid == 0) {
-            fence_after_sync();
-            const uint32_t idesc = make_idesc_bf16(64, 128, false, true, true);   // -T' (K e^G)
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = make_desc(smem_u32(sm + P_Q + ks * 32), 16, 1024);
-                const uint64_t bd = make_desc(smem_u32(sm + P_K + ks * 2048), 8192, 1024);
-                mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
-            }
-            commit(&bar);
-        }
-        ok = block_wait(&bar, 0, err, 3);
-        fence_after_sync();
-        if (ok) {
-            const int i = 16 * sp + l, half = w >> 2;
-            float f[4][16];
-#pragma unroll
-            for (int cb = 0; cb < 4; ++cb)
-                tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 64 * half + 16 * cb, f[cb]);
-            tmem_wait_ld();
-            if (l < 16) {
-                unsigned char* dst = img + IMG_W + half * 8192;
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
-                }
-            }
-        }
-    } else {
+        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 1, err);
+    } else if (!ok) {
         // the input loads may still be in flight: let them land before leaving
         mbar_wait(&bar_in, 0, nullptr, 0, 200);
     }
@@ -844,11 +1029,11 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     static std::atomic<uint64_t> attrs_done{0};
     cudaError_t e = once_per_device(attrs_done, [] {
         cudaError_t r;
-        if ((r = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<false>,
+        if ((r = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
             return r;
-        if ((r = cudaFuncSetAttribute(tc::chunk_prep_tc_kernel<true>,
-                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::P_SMEM)))
+        if ((r = cudaFuncSetAttribute(tc::chunk_prep_gdn_tc_kernel,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tc::GP_SMEM)))
             return r;
         if ((r = set_state_smem<true, tc::WALK_SEQ>())) return r;
         if ((r = set_state_smem<false, tc::WALK_SEQ>())) return r;
@@ -873,11 +1058,11 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
         LaunchScope scope(s, K_PREP_TC);
         if (a.gate_scalar)
-            tc::chunk_prep_tc_kernel<true><<<gp, tc::PT, tc::P_SMEM, s>>>(
+            tc::chunk_prep_gdn_tc_kernel<<<gp, tc::PT, tc::GP_SMEM, s>>>(
                 maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, a.scale, w, err);
         else
-            tc::chunk_prep_tc_kernel<false><<<gp, tc::PT, tc::P_SMEM, s>>>(
-                maps, a.beta, nullptr, a.si, a.H, hb, Hg, a.scale, w, err);
+            tc::chunk_prep_tc_kernel<<<gp, tc::PT, tc::P_SMEM, s>>>(
+                maps, a.beta, a.si, a.H, hb, Hg, a.scale, w, err);
         return cudaGetLastError();
     };
     SegPlan none;

@@ -1,8 +1,10 @@
 """Gated DeltaNet (one decay per token and head) through kda_gdn_chunk_fwd and
 kda_gdn_recurrent_step, against the fp64 oracle with the gate broadcast over
 the key channels (the oracle pins tie that broadcast to the scalar-gate
-recurrence), and bit-for-bit against the KDA entry points fed the broadcast
-gate (same kernels, same arithmetic)."""
+recurrence).  The SIMT path and the decode step run the KDA arithmetic on the
+broadcast gate, so they also match the KDA entry points bit for bit; the
+tensor-core prefill has its own prep kernel (the scalar decay factors out of
+the key products), checked against the oracle only."""
 import numpy as np
 import pytest
 import torch
@@ -41,13 +43,17 @@ def test_gdn_prefill(kda, io, impl, dk, varlen):
     cu = None if inp["cu_seqlens"] is None else host(inp["cu_seqlens"]).numpy()
     ro, rh = oracle.fwd(host(inp["q"]), host(inp["k"]), host(inp["v"]), host(_expand(log_a, dk)),
                         host(inp["beta"]), inp["scale"], h0=host(inp["h0"]), cu_seqlens=cu)
-    assert rel(out, ro) <= TOL[io] and rel(hT, rh) <= TOL[io]
-    # the KDA entry point with the broadcast gate runs the same arithmetic
+    e_out, e_h = rel(out, ro), rel(hT, rh)
     out2, hT2 = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], _expand(log_a, dk), inp["beta"],
                               inp["scale"], h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], impl=impl)
     torch.cuda.synchronize()
-    torch.testing.assert_close(out, out2, rtol=0, atol=0)
-    torch.testing.assert_close(hT, hT2, rtol=0, atol=0)
+    print(f"PARITY gdn_{io}_{impl}_varlen{int(varlen)} out={e_out:.3e} hT={e_h:.3e} "
+          f"(kda entry on the broadcast gate: out={rel(out2, ro):.3e} hT={rel(hT2, rh):.3e})")
+    assert e_out <= TOL[io] and e_h <= TOL[io]
+    if impl == "simt":
+        # the KDA entry point with the broadcast gate runs the same arithmetic
+        torch.testing.assert_close(out, out2, rtol=0, atol=0)
+        torch.testing.assert_close(hT, hT2, rtol=0, atol=0)
 
 
 @pytest.mark.parametrize("io", ["f32", "bf16"])
