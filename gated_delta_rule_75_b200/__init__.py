@@ -16,7 +16,7 @@ import os
 import torch
 
 __all__ = ["chunk_fwd", "recurrent_step", "gdn_chunk_fwd", "gdn_recurrent_step", "KDAError",
-           "chunk_fwd_segmap", "affine_prefix", "chunk_bwd",
+           "chunk_fwd_segmap", "affine_prefix", "chunk_bwd", "gdn_chunk_bwd",
            "library_path", "version",
            "profiler_enable", "profiler_read",
            "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
@@ -79,6 +79,8 @@ def _load():
     lib.kda_chunk_bwd.argtypes = [vp] * 15 + [i64, i64, i64, i64, i64, ctypes.c_float,
                                               ctypes.c_int, vp]
     lib.kda_chunk_bwd.restype = ctypes.c_int
+    lib.kda_gdn_chunk_bwd.argtypes = lib.kda_chunk_bwd.argtypes
+    lib.kda_gdn_chunk_bwd.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -345,7 +347,7 @@ def affine_prefix(maps, offs, h0=None, out=None):
 
 
 def chunk_bwd(q, k, v, log_alpha, beta, scale, dout, h0=None, dhT=None, cu_seqlens=None,
-              need_dh0=True):
+              need_dh0=True, _gdn=False):
     """Gradients of sum(dout * out) + sum(dhT * hT) for the prefill
     :func:`chunk_fwd` computes on the same inputs (C ABI ``kda_chunk_bwd``).
     dout [B,T,H,dv] in the I/O dtype; dhT [N,H,dk,dv] fp32 or None.  Returns
@@ -359,7 +361,7 @@ def chunk_bwd(q, k, v, log_alpha, beta, scale, dout, h0=None, dhT=None, cu_seqle
     for name, t, shp in (("q", q, (B, T, H, dk)), ("k", k, (B, T, H, dk)), ("v", v, (B, T, H, dv)),
                          ("dout", dout, (B, T, H, dv))):
         _check(t, name, io, shp, dev)
-    _check(log_alpha, "log_alpha", torch.float32, (B, T, H, dk), dev)
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H) if _gdn else (B, T, H, dk), dev)
     _check(beta, "beta", torch.float32, (B, T, H), dev)
     if cu_seqlens is not None:
         if B != 1 or cu_seqlens.dtype != torch.int32 or cu_seqlens.device != dev:
@@ -376,10 +378,18 @@ def chunk_bwd(q, k, v, log_alpha, beta, scale, dout, h0=None, dhT=None, cu_seqle
     dg = torch.empty_like(log_alpha)
     db = torch.empty_like(beta)
     dh0 = torch.empty((N, H, dk, dv), dtype=torch.float32, device=dev) if need_dh0 else None
-    st = _load().kda_chunk_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0),
-                               _ptr(dout), _ptr(dhT), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg),
-                               _ptr(db), _ptr(dh0), _ptr(cu_seqlens), N, T, H, dk, dv,
-                               float(scale), _IO[io], _stream(dev))
+    fn = _load().kda_gdn_chunk_bwd if _gdn else _load().kda_chunk_bwd
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(h0), _ptr(dout),
+            _ptr(dhT), _ptr(dq), _ptr(dk_), _ptr(dv_), _ptr(dg), _ptr(db), _ptr(dh0),
+            _ptr(cu_seqlens), N, T, H, dk, dv, float(scale), _IO[io], _stream(dev))
     if st != KDA_OK:
-        raise KDAError(st, "kda_chunk_bwd")
+        raise KDAError(st, "kda_gdn_chunk_bwd" if _gdn else "kda_chunk_bwd")
     return dq, dk_, dv_, dg, db, dh0
+
+
+def gdn_chunk_bwd(q, k, v, log_a, beta, scale, dout, h0=None, dhT=None, cu_seqlens=None,
+                  need_dh0=True):
+    """Gated DeltaNet gradients (C ABI ``kda_gdn_chunk_bwd``): as :func:`chunk_bwd`
+    with one gate per (token, head), log_a [B,T,H] fp32; returns dlog_a [B,T,H]."""
+    return chunk_bwd(q, k, v, log_a, beta, scale, dout, h0=h0, dhT=dhT, cu_seqlens=cu_seqlens,
+                     need_dh0=need_dh0, _gdn=True)

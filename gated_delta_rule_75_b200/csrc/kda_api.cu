@@ -545,14 +545,15 @@ kda_status_t kda_affine_prefix(const float* maps, const float* offs, const float
 
 }  // extern "C"
 
-extern "C" {
+namespace kda {
 
-kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
-                           const float* beta, const float* h0, const void* dout, const float* dhT,
-                           void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
-                           float* dh0, const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
-                           int64_t dk_, int64_t dv_, float scale, kda_io_dtype_t io_dtype,
-                           cudaStream_t stream)
+static kda_status_t chunk_bwd_impl(const void* q, const void* k, const void* v,
+                                   const float* log_alpha, const float* beta, const float* h0,
+                                   const void* dout, const float* dhT, void* dq, void* dk, void* dv,
+                                   float* dlog_alpha, float* dbeta, float* dh0,
+                                   const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                                   int64_t dk_, int64_t dv_, float scale, kda_io_dtype_t io_dtype,
+                                   bool gate_scalar, cudaStream_t stream)
 {
     if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
@@ -561,9 +562,12 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
     if (B == 0 || H == 0) return KDA_OK;
     const int64_t T_total = cu_seqlens ? T : B * T;
     if (T_total > 0) {
-        const void* ptrs[] = {q, k, v, dout, dq, dk, dv, log_alpha, dlog_alpha};
+        const void* ptrs[] = {q, k, v, dout, dq, dk, dv};
         for (const void* p : ptrs)
             if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+        const void* gates[] = {log_alpha, dlog_alpha};
+        for (const void* p : gates)
+            if (p == nullptr || !(gate_scalar ? aligned4(p) : aligned16(p))) return KDA_ERR_INVALID_ARG;
         if (beta == nullptr || !aligned4(beta) || dbeta == nullptr || !aligned4(dbeta))
             return KDA_ERR_INVALID_ARG;
         // outputs must not alias inputs (or one another)
@@ -588,6 +592,7 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
     b.dout = dout; b.dhT = dhT; b.dq = dq; b.dk = dk; b.dv = dv; b.dlog_alpha = dlog_alpha;
     b.dbeta = dbeta; b.dh0 = dh0; b.H = H; b.dk_ = (int)dk_; b.dv_ = (int)dv_; b.scale = scale;
     b.io = io_dtype;
+    b.gate_scalar = gate_scalar;
     SeqInfo& si = b.si;
     si.cu = cu_seqlens;
     si.chunk_off = nullptr;
@@ -628,6 +633,32 @@ kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const fl
         if (flag & kErrSeqlens) return KDA_ERR_INVALID_ARG;
     }
     return KDA_OK;
+}
+
+}  // namespace kda
+
+extern "C" {
+
+kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v, const float* log_alpha,
+                           const float* beta, const float* h0, const void* dout, const float* dhT,
+                           void* dq, void* dk, void* dv, float* dlog_alpha, float* dbeta,
+                           float* dh0, const int32_t* cu_seqlens, int64_t B, int64_t T, int64_t H,
+                           int64_t dk_, int64_t dv_, float scale, kda_io_dtype_t io_dtype,
+                           cudaStream_t stream)
+{
+    return chunk_bwd_impl(q, k, v, log_alpha, beta, h0, dout, dhT, dq, dk, dv, dlog_alpha, dbeta,
+                          dh0, cu_seqlens, B, T, H, dk_, dv_, scale, io_dtype, false, stream);
+}
+
+kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, const float* log_a,
+                               const float* beta, const float* h0, const void* dout,
+                               const float* dhT, void* dq, void* dk, void* dv, float* dlog_a,
+                               float* dbeta, float* dh0, const int32_t* cu_seqlens, int64_t B,
+                               int64_t T, int64_t H, int64_t dk_, int64_t dv_, float scale,
+                               kda_io_dtype_t io_dtype, cudaStream_t stream)
+{
+    return chunk_bwd_impl(q, k, v, log_a, beta, h0, dout, dhT, dq, dk, dv, dlog_a, dbeta, dh0,
+                          cu_seqlens, B, T, H, dk_, dv_, scale, io_dtype, true, stream);
 }
 
 }  // extern "C"

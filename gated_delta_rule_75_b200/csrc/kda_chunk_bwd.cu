@@ -387,7 +387,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         const int64_t src = ((t0 + t) * H + h) * DK + c;
         sK[e] = ok ? IO<T>::load(k, src) : 0.f;
         sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
-        sG[e] = ok ? b.log_alpha[src] : 0.f;
+        sG[e] = ok ? b.log_alpha[b.gate_scalar ? (t0 + t) * H + h : src] : 0.f;
     }
     for (int e = tid; e < C * C; e += kPT) {
         sT[e] = blk[BW::Tm + e];
@@ -562,7 +562,16 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         float run = acc;
         for (int i = C - 1; i >= 0; --i) {
             run += sdG[i * DK + c];
-            if (i < len) b.dlog_alpha[((t0 + i) * H + h) * DK + c] = run;
+            if (b.gate_scalar) sdG[i * DK + c] = run;
+            else if (i < len) b.dlog_alpha[((t0 + i) * H + h) * DK + c] = run;
+        }
+    }
+    if (b.gate_scalar) {                              // one gate per (token, head): channel sum
+        __syncthreads();
+        if (tid < len) {
+            float acc = 0.f;
+            for (int c = 0; c < DK; ++c) acc += sdG[tid * DK + (c + tid) % DK];
+            b.dlog_alpha[(t0 + tid) * H + h] = acc;
         }
     }
     if (tid < len) b.dbeta[(t0 + tid) * H + h] = sdB[tid];
@@ -613,7 +622,7 @@ static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaS
             LaunchScope scope(st, K_PREP_SIMT);
             chunk_prep_simt_kernel<T, DK, DV, true><<<gchunk, kSimtPrepThreads, simt_prep_smem<DK, DV>(), st>>>(
                 (const T*)b.q, (const T*)b.k, (const T*)b.v, b.log_alpha, b.beta, si, b.H, hb, Hg,
-                b.scale, ws, 0);
+                b.scale, ws, b.gate_scalar ? 1 : 0);
             if ((e = cudaGetLastError())) return e;
         }
         const dim3 gwalk((unsigned)(si.N * hg * (DV / kTW)));

@@ -177,7 +177,7 @@ struct BackwardArgs {
     void* dq;                 // [.., H, dk] io dtype
     void* dk;
     void* dv;                 // [.., H, dv] io dtype
-    float* dlog_alpha;        // [.., H, dk]
+    float* dlog_alpha;        // [.., H, dk] ([.., H] with gate_scalar)
     float* dbeta;             // [.., H]
     float* dh0;               // nullable
     SeqInfo si;
@@ -185,6 +185,9 @@ struct BackwardArgs {
     int dk_, dv_;
     float scale;
     kda_io_dtype_t io;
+    // Gated DeltaNet: log_alpha [.., H] broadcast over the key channels; dlog_alpha [.., H]
+    // receives the channel sum of the per-channel gradient
+    bool gate_scalar;
 };
 
 struct DecodeArgs {

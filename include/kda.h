@@ -308,6 +308,21 @@ KDA_API kda_status_t kda_chunk_bwd(const void* q, const void* k, const void* v,
                                    float scale, kda_io_dtype_t io_dtype, cudaStream_t stream);
 
 /*
+ * kda_gdn_chunk_bwd -- kda_chunk_bwd for the Gated DeltaNet form: log_a
+ * [B, T, H] fp32 (one gate per token and head, as kda_gdn_chunk_fwd takes it);
+ * dlog_a [B, T, H] fp32 receives its gradient, the sum over the key channels of
+ * the per-channel one (the gate multiplies every channel).  Other arguments
+ * as for kda_chunk_bwd; log_a and dlog_a need 4-byte alignment.
+ */
+KDA_API kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v,
+                                       const float* log_a, const float* beta, const float* h0,
+                                       const void* dout, const float* dhT,
+                                       void* dq, void* dk, void* dv, float* dlog_a,
+                                       float* dbeta, float* dh0, const int32_t* cu_seqlens,
+                                       int64_t B, int64_t T, int64_t H, int64_t dk_, int64_t dv_,
+                                       float scale, kda_io_dtype_t io_dtype, cudaStream_t stream);
+
+/*
  * Context parallelism: one long sequence split across GPUs (or across calls).
  *
  * The recurrence is linear in the state, so a run of tokens maps any entry

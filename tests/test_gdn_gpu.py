@@ -72,3 +72,31 @@ def test_gdn_decode(kda, io):
                                 host(x["beta"]), S_ref, scale)
         assert rel(o, ro) <= TOL[io]
         assert rel(S, S_ref) <= 1e-5
+
+
+@pytest.mark.parametrize("io,dk", [("f32", 64), ("bf16", 128)])
+@pytest.mark.parametrize("varlen", [False, True])
+def test_gdn_backward(kda, io, dk, varlen):
+    """kda_gdn_chunk_bwd against the oracle's reverse mode on the broadcast gate;
+    the gate gradient is the channel sum of the per-channel one."""
+    lengths = [100, 1, 64, 150] if varlen else None
+    cfg = W.small_prefill(B=2, T=150, H=2, dk=dk, dv=dk, io_dtype=io, seed=62, h0_std=0.03,
+                          lengths=lengths)
+    inp = W.make_prefill(cfg, "cuda")
+    log_a = W.scalar_gates(cfg.B, cfg.T, cfg.H, seed=62, device="cuda")
+    gen = torch.Generator(device="cuda").manual_seed(63)
+    dout = torch.randn((cfg.B, cfg.T, cfg.H, dk), generator=gen, device="cuda").to(inp["q"].dtype)
+    dhT = torch.randn((cfg.N, cfg.H, dk, dk), generator=gen, device="cuda")
+    got = kda.gdn_chunk_bwd(inp["q"], inp["k"], inp["v"], log_a, inp["beta"], inp["scale"], dout,
+                            h0=inp["h0"], dhT=dhT, cu_seqlens=inp["cu_seqlens"])
+    torch.cuda.synchronize()
+    cu = None if inp["cu_seqlens"] is None else host(inp["cu_seqlens"]).numpy()
+    ref = oracle.bwd(host(inp["q"]), host(inp["k"]), host(inp["v"]), host(_expand(log_a, dk)),
+                     host(inp["beta"]), inp["scale"], host(dout), h0=host(inp["h0"]),
+                     dhT=host(dhT), cu_seqlens=cu)
+    ref = list(ref)
+    ref[3] = ref[3].sum(axis=-1)
+    tol = {"f32": [1e-5] * 6, "bf16": [5e-3, 5e-3, 5e-3, 1e-5, 1e-5, 1e-5]}[io]
+    errs = [rel(g, r) for g, r in zip(got, ref)]
+    print(f"PARITY gdn_bwd_{io}_varlen{int(varlen)} " + " ".join(f"{e:.3e}" for e in errs))
+    assert all(e <= t for e, t in zip(errs, tol)), errs

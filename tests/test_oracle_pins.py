@@ -459,3 +459,25 @@ def test_backward_matches_autograd_of_a_plain_recurrence():
     grads = oracle.bwd(q, k, v, g, b, scale, dout, h0=h0, dhT=dhT, cu_seqlens=cu)
     for t, gx in zip(ts, grads):
         np.testing.assert_allclose(gx, t.grad.numpy(), rtol=1e-10, atol=1e-11)
+
+
+def test_scalar_gate_gradient_is_the_channel_sum():
+    """Gated DeltaNet: with one gate per (token, head) broadcast over the key
+    channels, the gate's gradient (central differences of the loss in the
+    scalar gate) equals the channel sum of oracle.bwd's per-channel gradient."""
+    rng = np.random.default_rng(33)
+    T, H, dk, dv, scale = 20, 1, 4, 3, 0.6
+    q, k, v, _, b, h0, cu = _rand_inputs(rng, 1, T, H, dk, dv)
+    la = -np.log1p(np.exp(rng.standard_normal((1, T, H))))
+    dout = rng.standard_normal((1, T, H, dv))
+    dhT = rng.standard_normal((1, H, dk, dv))
+    g = lambda a: np.repeat(a[..., None], dk, axis=-1)
+    grads = oracle.bwd(q, k, v, g(la), b, scale, dout, h0=h0, dhT=dhT)
+    eps = 1e-6
+    for t in range(T):
+        lp, lm = la.copy(), la.copy()
+        lp[0, t, 0] += eps
+        lm[0, t, 0] -= eps
+        fd = (_loss(q, k, v, g(lp), b, h0, None, scale, dout, dhT) -
+              _loss(q, k, v, g(lm), b, h0, None, scale, dout, dhT)) / (2 * eps)
+        np.testing.assert_allclose(grads[3][0, t, 0].sum(), fd, rtol=1e-6, atol=1e-7)
