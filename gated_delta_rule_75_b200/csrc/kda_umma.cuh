@@ -148,7 +148,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
 
 // Block-wide wait: thread 0 polls `bar` (phase `parity`) with the iteration
 // limit of mbar_wait, the rest of the block sleeps in the barrier, and every
-// thread gets the same verdict.  The barrier orders the observed completion
+// thread gets the same outcome.  The barrier orders the observed completion
 // (and the data it guards) before everything the block does next.
 __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, int* err, int err_bit)
 {

@@ -393,7 +393,7 @@ def test_composed_segment_maps_reproduce_the_sequence(cuts):
 
 
 # --------------------------------------------------------------------------
-# P-grad: the backward pass (training, SURVEY row f-3)
+# P-grad: the backward pass (training)
 # --------------------------------------------------------------------------
 def _loss(q, k, v, g, b, h0, cu, scale, dout, dhT):
     out, hT = oracle.fwd(q, k, v, g, b, scale, h0=h0, cu_seqlens=cu)
