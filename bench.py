@@ -392,10 +392,26 @@ def run_decode(args, ws, rank, kda, peaks):
     bytes_step = per_head * cfg.N * cfg.H
     launches, timed, kms = stats["decode_step"]
     gbs = bytes_step / (kms / max(1, timed) / 1e3) / 1e9
+    # the same chained loop captured once as a CUDA graph and replayed (no per-step launch cost)
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        run_all()                                  # warm the side stream before capture
+    stream.wait_stream(side)
+    with torch.cuda.graph(graph):
+        run_all()
+    graph.replay()
+    torch.cuda.synchronize()
+    barrier(ws)
+    g_ms = max_over_ranks(time_region(graph.replay, 1, stream), ws)
+    del graph
     return {
         "workload": cfg.name, "steps_chained": cfg.steps, "ms_per_step": ms / cfg.steps,
         "tokens_per_s": cfg.N * cfg.steps * ws / (ms / 1e3),
         "state_GBps": bytes_step * cfg.steps * ws / (ms / 1e3) / 1e9,
+        "cuda_graph": {"ms_per_step": g_ms / cfg.steps,
+                       "state_GBps": bytes_step * cfg.steps * ws / (g_ms / 1e3) / 1e9},
         "roofline": {"kernel": "decode_step", "bound": "hbm", "achieved": gbs,
                      "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "traffic": measured_traffic("decode_step", cfg.name),
