@@ -81,6 +81,9 @@ def _load():
     lib.kda_chunk_bwd.restype = ctypes.c_int
     lib.kda_gdn_chunk_bwd.argtypes = lib.kda_chunk_bwd.argtypes
     lib.kda_gdn_chunk_bwd.restype = ctypes.c_int
+    lib.kda_debug_prep_image.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ctypes.c_float,
+                                         ctypes.c_int, vp]
+    lib.kda_debug_prep_image.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -393,3 +396,24 @@ def gdn_chunk_bwd(q, k, v, log_a, beta, scale, dout, h0=None, dhT=None, cu_seqle
     with one gate per (token, head), log_a [B,T,H] fp32; returns dlog_a [B,T,H]."""
     return chunk_bwd(q, k, v, log_a, beta, scale, dout, h0=h0, dhT=dhT, cu_seqlens=cu_seqlens,
                      need_dh0=need_dh0, _gdn=True)
+
+
+IMAGE_BYTES = 66560   # one (chunk, head) operand image of the tensor-core prefill
+
+
+def debug_prep_image(q, k, log_alpha, beta, scale, gate_scalar=False):
+    """Test hook (C ABI ``kda_debug_prep_image``): the tensor-core prep kernel's
+    operand images of a fixed-length bf16 batch, uint8 [B*ceil(T/64)*H, 66560]."""
+    B, T, H, dk = q.shape
+    dev = q.device
+    _check(q, "q", torch.bfloat16, (B, T, H, 128), dev)
+    _check(k, "k", torch.bfloat16, (B, T, H, 128), dev)
+    _check(log_alpha, "log_alpha", torch.float32, (B, T, H) if gate_scalar else (B, T, H, 128), dev)
+    _check(beta, "beta", torch.float32, (B, T, H), dev)
+    n = B * ((T + 63) // 64) * H
+    image = torch.zeros((n, IMAGE_BYTES), dtype=torch.uint8, device=dev)
+    st = _load().kda_debug_prep_image(_ptr(q), _ptr(k), _ptr(log_alpha), _ptr(beta), _ptr(image),
+                                      B, T, H, float(scale), 1 if gate_scalar else 0, _stream(dev))
+    if st != KDA_OK:
+        raise KDAError(st, "kda_debug_prep_image")
+    return image

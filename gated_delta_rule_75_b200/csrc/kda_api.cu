@@ -662,3 +662,34 @@ kda_status_t kda_gdn_chunk_bwd(const void* q, const void* k, const void* v, cons
 }
 
 }  // extern "C"
+
+extern "C" {
+
+kda_status_t kda_debug_prep_image(const void* q, const void* k, const float* log_alpha,
+                                  const float* beta, void* image, int64_t B, int64_t T, int64_t H,
+                                  float scale, int gate_scalar, cudaStream_t stream)
+{
+    if (B < 0 || T < 0 || H < 0 || H > 65535) return KDA_ERR_INVALID_ARG;
+    if (B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;
+    if (B == 0 || T == 0 || H == 0) return KDA_OK;
+    const void* ptrs[] = {q, k, image};
+    for (const void* p : ptrs)
+        if (p == nullptr || !aligned16(p)) return KDA_ERR_INVALID_ARG;
+    if (log_alpha == nullptr || !(gate_scalar ? aligned4(log_alpha) : aligned16(log_alpha)))
+        return KDA_ERR_INVALID_ARG;
+    if (beta == nullptr || !aligned4(beta)) return KDA_ERR_INVALID_ARG;
+    PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
+    a.q = q; a.k = k; a.v = k;                 // v is not read by the prep
+    a.log_alpha = log_alpha; a.beta = beta; a.H = H; a.dk = 128; a.dv = 128;
+    a.scale = scale; a.io = KDA_IO_BF16; a.gate_scalar = gate_scalar != 0; a.tc_what = 2;
+    SeqInfo& si = a.si;
+    si.N = B;
+    si.T_seq = T;
+    si.T_total = B * T;
+    si.nct = (T + kChunk - 1) / kChunk;
+    si.chunks_upper = B * si.nct;
+    return from_cuda(run_prefill_tc(a, static_cast<unsigned char*>(image), H, nullptr, stream));
+}
+
+}  // extern "C"

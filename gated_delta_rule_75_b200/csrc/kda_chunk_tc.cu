@@ -1113,6 +1113,7 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     for (int64_t hb = 0; hb < a.H; hb += Hg) {
         const int64_t hg = (a.H - hb) < Hg ? (a.H - hb) : Hg;
         if ((e = launch_prep(hb, hg, ws, st))) return e;
+        if (a.tc_what == 2) continue;          // operand images only
         if (a.tc_what == 1) {                  // each sequence's (M, B) into the caller's buffers
             if ((e = launch_walk(tc::WALK_VALUE, sp, hb, hg, ws, st))) return e;
             if ((e = launch_walk(tc::WALK_MAP, sp, hb, hg, ws, st))) return e;

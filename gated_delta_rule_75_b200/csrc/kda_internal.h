@@ -145,8 +145,9 @@ struct PrefillArgs {
     // tensor-core path: segment-parallel state walk (len == 0: one chain per
     // (sequence, head)); the buffers are placed by run_prefill_tc
     SegPlan seg;
-    // what the tensor-core state walks produce: outputs and final states (0),
-    // or only each sequence's affine map, into seg.maps / seg.offs (1)
+    // what the tensor-core path produces: outputs and final states (0), only each
+    // sequence's affine map into seg.maps / seg.offs (1), or only the operand images of
+    // the prep kernel, left in the workspace (2; the test hook kda_debug_prep_image)
     int tc_what;
 
 #ifdef __CUDACC__

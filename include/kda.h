@@ -370,6 +370,23 @@ KDA_API kda_status_t kda_affine_prefix(const float* maps, const float* offs, con
                                        float* out, int64_t nseg, int64_t NH, int64_t dk,
                                        int64_t dv, cudaStream_t stream);
 
+/*
+ * kda_debug_prep_image -- test hook, not part of the method: runs only the
+ * tensor-core prep kernel (cumulative decay and intra-chunk transform) of a
+ * fixed-length bf16 batch with dk = dv = 128 and leaves its per-(chunk, head)
+ * operand images in `image` (device, caller-owned, B * ceil(T / 64) * H blocks of
+ * 66560 bytes, block (chunk c of sequence n, head h) at index (n * ceil(T/64) + c)
+ * * H + h), in the 128-byte-swizzled bf16 layout the state kernel reads:
+ * -W | scale Q e^G | [Aqk^T | K e^{G_last - G}] | T diag(beta) | e^{G_last} (fp32).
+ * log_alpha is [B, T, H, dk], or [B, T, H] with gate_scalar != 0 (Gated DeltaNet
+ * prep).  Lets the tests check the intra-chunk kernels against the fp64 chunk
+ * equations one quantity at a time.
+ */
+KDA_API kda_status_t kda_debug_prep_image(const void* q, const void* k, const float* log_alpha,
+                                          const float* beta, void* image, int64_t B, int64_t T,
+                                          int64_t H, float scale, int gate_scalar,
+                                          cudaStream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char* kda_status_string(kda_status_t status);
 
