@@ -45,7 +45,7 @@ constexpr int kAP = 68;           // row pitch of the transposed Aqk
 // + lane and NJ consecutive columns of the 32-column tile (NJ = 16 for DK = 128, 8 for 64);
 // it is copied to shared memory once per chunk as the operand of Khat dS'.
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kBT)
+__global__ void __launch_bounds__(kBT, 2)
 chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
@@ -157,7 +157,7 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
 // dense pass 1: per (chunk, head)
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kD1T)
+__global__ void __launch_bounds__(kD1T, 1)
 chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
@@ -263,7 +263,7 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
 //   3: dT'  =  dE R^T   4: dAqk = dO E^T (kept for m <= i)       (m < C)
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kBT)
+__global__ void __launch_bounds__(kBT, 4)   // four CTAs per SM hide the tile loads
 chunk_bwd_dense2_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
@@ -348,7 +348,7 @@ chunk_bwd_dense2_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
 // parameter gradients: per (chunk, head)
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kPT)
+__global__ void __launch_bounds__(kPT, 1)
 chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;

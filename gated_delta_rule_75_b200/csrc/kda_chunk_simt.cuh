@@ -96,7 +96,7 @@ constexpr size_t simt_state_smem()
 constexpr int kSimtPrepThreads = 256;   // 16 rows x 16 column lanes in the A / Aqk phase
 
 template <typename T, int DK, int DV, bool kBwd = false>
-__global__ void __launch_bounds__(kSimtPrepThreads)
+__global__ void __launch_bounds__(kSimtPrepThreads, 1)
 chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
                        const float* __restrict__ log_alpha, const float* __restrict__ beta,
                        SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
@@ -267,7 +267,7 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
 // steps c + d: sequential state propagation and output, per 32-column dv tile
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV, bool kBwd = false>
-__global__ void __launch_bounds__(256)
+__global__ void __launch_bounds__(256, kBwd ? 2 : 1)   // occupancy set by shared memory
 chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, int64_t Hg)
 {
     // kBwd: backward blocks; every chunk's entry state is saved (Sx) and
