@@ -257,7 +257,7 @@ kda_status_t kda_chunk_fwd_slots(const void* q, const void* k, const void* v,
 namespace kda {
 
 // Streaming multiprocessors of the current device (queried once per device).
-static int64_t sm_count()
+int64_t device_sm_count()
 {
     static std::mutex mu;
     static int cached[64] = {};
@@ -284,7 +284,7 @@ static SegPlan plan_segments(const SeqInfo& si, int64_t H, kda_prefill_impl_t im
     std::memset(&p, 0, sizeof(p));
     if (impl == KDA_PREFILL_TENSORCORE_CHAIN || si.chunks_upper <= 0) return p;
     const bool force = impl == KDA_PREFILL_TENSORCORE_SEGMENTED;
-    const int64_t sms = sm_count();
+    const int64_t sms = device_sm_count();
     const int64_t chains = si.N * H;
     if (!force && chains * 4 > sms) return p;
     if (si.cu == nullptr) {

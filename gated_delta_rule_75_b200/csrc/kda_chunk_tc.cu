@@ -159,12 +159,17 @@ constexpr uint32_t P_KQ = 65536;       // K-major B: [Kin_p; Qin_p] x 4, one K-b
 constexpr uint32_t P_KV = 81920;       // K-major A: Kvar rows (160), one K-block                20 KB
 constexpr uint32_t P_A = 65536;        // fp32 A [64][68] (aliases KQ/KV after the strips)       17 KB
 constexpr uint32_t P_T = P_A + 64 * AP * 4;   // fp32 T [64][68]                                 17 KB
-constexpr uint32_t P_VEC = 102400;     // per-channel vectors: egf[4], eglf[4], dvec[6]          7 KB
-constexpr uint32_t P_BETA = P_VEC + 14 * 512;  // beta [64], then the scalar gates [64]
+constexpr uint32_t P_VEC = 102400;     // per-channel vectors: egf[4], eglf[4], dvec[6]          8 KB
+constexpr int VP = 144;                // floats per vector: 4 pad floats after every 32 channels
+constexpr uint32_t P_BETA = P_VEC + 14 * VP * 4;   // beta [64], then the scalar gates [64]
 constexpr uint32_t P_BYTES = P_BETA + 512;
 constexpr uint32_t P_SMEM = P_BYTES + 1024 + 64;
 constexpr uint32_t P_TX = 16384 + 16384 + 32768;   // bytes the input TMA loads deliver
 static_assert(P_T + 64 * AP * 4 <= P_VEC, "A/T overlap the vectors");
+
+// Index of channel c in a padded per-channel vector: the 8-channel groups that a
+// quarter-warp reads (32 channels apart) fall in distinct banks.
+__device__ __forceinline__ int vidx(int c) { return c + 4 * (c >> 5); }
 
 // Byte offset of G[t][c] in the four 128B-swizzled slabs of 32 fp32 channels.
 __device__ __forceinline__ uint32_t g_off(int t, int c)
@@ -180,11 +185,13 @@ struct PrepMaps {
 // Shared tail of the prep kernels, after A (fp32, strictly lower, beta-scaled rows, pitch
 // AP) is in sA and K e^G (bf16, MN-major image rows) in P_K (sT: room for T, pitch AP): T = (I + A)^{-1}, T' = T diag(beta) as a
 // bf16 K-major image (in P_Q and in the workspace), and W = -T' (K e^G) by one MMA whose
-// completion is phase `parity` of `bar`; W goes to the workspace image.  Returns false when
-// the bounded wait gave up.
+// completion is phase `parity` of `bar`; W goes to the workspace image.  `after_mma()` runs in
+// every thread once that MMA has completed (its operands in P_Q and P_K are no longer read).
+// Returns false when the bounded wait gave up.
+template <typename AfterMma>
 __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img, float* sA, float* sT,
                                           const float* sB, uint32_t tmem, uint64_t* bar,
-                                          uint32_t parity, int* err)
+                                          uint32_t parity, int* err, AfterMma after_mma)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3;                          // TMEM lane quarter of this warp
@@ -268,6 +275,7 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
     const bool ok = block_wait(bar, parity, err, 3);
     fence_after_sync();
     if (ok) {
+        after_mma();                               // P_Q and P_K are free from here on
         const int i = 16 * sp + l, half = w >> 2;
         float f[4][16];
 #pragma unroll
@@ -288,247 +296,299 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
 
 __global__ void __launch_bounds__(PT, 2)
 chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
-                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
+                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, int64_t hg, float scale,
                      unsigned char* __restrict__ ws, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t bar_in, bar;
+    __shared__ uint64_t bar_g, bar_kq, bar;
     __shared__ uint32_t tmem_base;
 
-    const int64_t gc = blockIdx.x;
-    const int hl = blockIdx.y;
-    const int64_t h = h_base + hl;
-    int64_t n, t0, len;
-    if (!si.locate(gc, n, t0, len)) return;
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3;                          // TMEM lane quarter of this warp
-    unsigned char* img = ws + (gc * Hg + hl) * (int64_t)IMG_BYTES;
-
     unsigned char* sGb = sm + P_G;
-    float* egf = reinterpret_cast<float*>(sm + P_VEC);           // [4][128]  e^{G_f}
-    float* eglf = egf + 4 * D;                                    // [4][128]  e^{G_last - G_f}
-    float* dvec = eglf + 4 * D;                                   // [6][128]  e^{G_fp - G_fr}
+    float* egf = reinterpret_cast<float*>(sm + P_VEC);           // [4][VP]  e^{G_f}
+    float* eglf = egf + 4 * VP;                                   // [4][VP]  e^{G_last - G_f}
+    float* dvec = eglf + 4 * VP;                                  // [6][VP]  e^{G_fp - G_fr}
     float* sB = reinterpret_cast<float*>(sm + P_BETA);
     auto G = [&](int t, int c) -> float& { return *reinterpret_cast<float*>(sGb + g_off(t, c)); };
 
-    if (tid == 0) {                                // the input loads go out first
-        mbar_init(&bar_in, 1);
+    // Work items are (chunk, head) pairs, item = chunk * hg + head; this CTA takes
+    // blockIdx.x, blockIdx.x + gridDim.x, ...  The next item's gates are fetched as soon
+    // as the current one's are last read (after the operand build), its k and q once the
+    // W MMA has consumed P_K and P_Q, so the loads overlap the rest of the current item.
+    const int64_t items = si.chunks_upper * hg;
+    auto next_item = [&](int64_t from, int64_t& n_, int64_t& t0_, int64_t& len_) -> int64_t {
+        for (int64_t it = from; it < items; it += gridDim.x)
+            if (si.locate(it / hg, n_, t0_, len_)) return it;
+        return -1;
+    };
+    auto issue_g = [&](int64_t item, int64_t t0_) {               // one thread
+        const int32_t y = (int32_t)t0_, x = (int32_t)((h_base + item % hg) * D);
+        tma::expect_tx(&bar_g, 32768);
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) tma::load_2d(sGb + s4 * 8192, &maps.g, x + 32 * s4, y, &bar_g);
+    };
+    auto issue_kq = [&](int64_t item, int64_t t0_) {              // one thread
+        const int32_t y = (int32_t)t0_, x = (int32_t)((h_base + item % hg) * D);
+        tma::expect_tx(&bar_kq, 32768);
+        tma::load_2d(sm + P_K, &maps.k, x, y, &bar_kq);
+        tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_kq);
+        tma::load_2d(sm + P_Q, &maps.q, x, y, &bar_kq);
+        tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_kq);
+    };
+
+    int64_t n = 0, t0 = 0, len = 0;
+    int64_t cur = next_item(blockIdx.x, n, t0, len);
+    if (tid == 0) {
+        mbar_init(&bar_g, 1);
+        mbar_init(&bar_kq, 1);
         mbar_init(&bar, 1);
         fence_mbar_init();
-        tma::expect_tx(&bar_in, P_TX);
-        const int32_t y = (int32_t)t0, x = (int32_t)(h * D);
-        tma::load_2d(sm + P_K, &maps.k, x, y, &bar_in);
-        tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_in);
-        tma::load_2d(sm + P_Q, &maps.q, x, y, &bar_in);
-        tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_in);
-#pragma unroll
-        for (int s = 0; s < 4; ++s) tma::load_2d(sGb + s * 8192, &maps.g, x + 32 * s, y, &bar_in);
+        if (cur >= 0) {
+            issue_g(cur, t0);
+            issue_kq(cur, t0);
+        }
     }
-    // beta meanwhile: its latency overlaps the TMA loads
-    const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
-    if (tid < C) sB[tid] = bval;
     fence_before_sync();
-    bool ok = block_wait(&bar_in, 0, err, 1);      // also the barrier for sB and the TMEM address
+    __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
-    if (ok && len < C) {
-        // a partial chunk: tokens past its end (next sequence or zero fill) read as zero
-        for (int e = tid; e < (C - (int)len) * 16; e += PT) {
-            const int t = (int)len + (e >> 4), ch = e & 15;
-            const uint32_t off = (ch >> 3) * 8192 + sw128_offset(t, (8 * ch) & 63);
-            *reinterpret_cast<uint4*>(sm + P_K + off) = make_uint4(0, 0, 0, 0);
-            *reinterpret_cast<uint4*>(sm + P_Q + off) = make_uint4(0, 0, 0, 0);
-        }
-        __syncthreads();
-    }
-
-    if (ok) {
-        // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
-        // Threads c and c + 128 scan tokens 0..31 and 32..63 in registers; the second
-        // half then adds the first half's total and derives the per-channel vectors.
-        {
-            const int c = tid & 127, part = tid >> 7, tb = 32 * part;
-            const unsigned char* slab = sGb + (c >> 5) * 8192 + (c & 3) * 4;
-            const int q0 = (c & 31) >> 2;
-            float v[32];
-#pragma unroll
-            for (int x = 0; x < 32; ++x)
-                v[x] = *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
-            float run = 0.f;
-#pragma unroll
-            for (int x = 0; x < 32; ++x) {
-                run += (tb + x < len) ? kLog2e * v[x] : 0.f;
-                v[x] = run;
-            }
-            if (part == 0) {
-#pragma unroll
-                for (int x = 0; x < 32; ++x)
-                    *reinterpret_cast<float*>(const_cast<unsigned char*>(slab) + x * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
-            }
-            __syncthreads();
-            if (part == 1) {
-                const float base = G(31, c);
-#pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    v[x] += base;
-                    *reinterpret_cast<float*>(const_cast<unsigned char*>(slab) + (32 + x) * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
-                }
-                const float Gl = v[31];
-                const float Gf[4] = {G(0, c), G(16, c), v[0], v[16]};
-#pragma unroll
-                for (int p = 0; p < 4; ++p) {
-                    egf[p * D + c] = ex2(Gf[p]);
-                    eglf[p * D + c] = ex2(Gl - Gf[p]);
-                }
-                int idx = 0;
-#pragma unroll
-                for (int p = 1; p < 4; ++p)
-#pragma unroll
-                    for (int r = 0; r < p; ++r) dvec[(idx++) * D + c] = ex2(Gf[p] - Gf[r]);
-                reinterpret_cast<float*>(img + IMG_GAM)[c] = ex2(Gl);
-            }
-        }
-        __syncthreads();
-
-        // ---- (b1) A / Aqk strips: operands built per channel half, MMAs accumulate.
-        // Thread (ch8, tr, p) handles rows 16p + tr and 16p + tr + 8 of channels
-        // c0 .. c0 + 7, so the sub-chunk's reference values are loaded once.
-        const int ch8 = tid & 7, tr = (tid >> 3) & 7, p = tid >> 6;
-        for (int hh = 0; hh < 2 && ok; ++hh) {
-            const int c0 = 64 * hh + 8 * ch8;
-            const unsigned char* slab = sGb + (c0 >> 5) * 8192;
-            const int q0 = (c0 & 31) >> 2;
-            float Gf8[8], eg[8], egl[8];
-            {
-                const int tf = 16 * p;
-                const float4 fa = *reinterpret_cast<const float4*>(slab + tf * 128 + (q0 << 4));
-                const float4 fb = *reinterpret_cast<const float4*>(slab + tf * 128 + ((q0 + 1) << 4));
-                Gf8[0] = fa.x; Gf8[1] = fa.y; Gf8[2] = fa.z; Gf8[3] = fa.w;
-                Gf8[4] = fb.x; Gf8[5] = fb.y; Gf8[6] = fb.z; Gf8[7] = fb.w;
-            }
-            ld8f(egf + p * D + c0, eg);
-            ld8f(eglf + p * D + c0, egl);
-            float egs[8];
-#pragma unroll
-            for (int j = 0; j < 8; ++j) egs[j] = scale * eg[j];
-            float kin[2][8], qin[2][8], kd[2][8];
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int t = 16 * p + tr + 8 * rr;
-                float G8[8], kk[8], qq[8];
-                {
-                    const float4 a = *reinterpret_cast<const float4*>(slab + t * 128 + ((q0 ^ (t & 7)) << 4));
-                    const float4 b = *reinterpret_cast<const float4*>(slab + t * 128 + (((q0 + 1) ^ (t & 7)) << 4));
-                    G8[0] = a.x; G8[1] = a.y; G8[2] = a.z; G8[3] = a.w;
-                    G8[4] = b.x; G8[5] = b.y; G8[6] = b.z; G8[7] = b.w;
-                }
-                const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
-                unpack8(*reinterpret_cast<const uint4*>(sm + P_K + off), kk);
-                unpack8(*reinterpret_cast<const uint4*>(sm + P_Q + off), qq);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float x = G8[j] - Gf8[j];
-                    const float e1 = ex2(x);          // <= 1
-                    const float r1 = ex2(-x);         // >= 1, at most 15 tokens of decay
-                    kin[rr][j] = kk[j] * e1;
-                    qin[rr][j] = qq[j] * e1;          // `scale` is applied to Aqk and Q e^G later
-                    kd[rr][j] = kk[j] * r1;
-                }
-                // operands of the strip MMAs first
-                const int ts = tr + 8 * rr;          // row within the sub-chunk
-                float tmp[8];
-                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + ts, 8 * ch8)) = pack8(kin[rr]);
-                *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * p + 16 + ts, 8 * ch8)) = pack8(qin[rr]);
-                *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[p] + t, 8 * ch8)) = pack8(kd[rr]);
-#pragma unroll
-                for (int pv = 1; pv < 4; ++pv) {
-                    if (pv > p) {
-                        float dv8[8];
-                        ld8f(dvec + ((pv * (pv - 1)) / 2 + p) * D + c0, dv8);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * dv8[j];
-                        *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pv] + t, 8 * ch8)) = pack8(tmp);
-                    }
-                }
-            }
-            fence_smem_to_async();
-            fence_before_sync();
-            __syncthreads();
-            if (tid == 0) {
-                fence_after_sync();
-                const uint32_t idesc = make_idesc_bf16(64, 32, false, false);
-#pragma unroll
-                for (int pp = 0; pp < 4; ++pp)
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        const uint64_t ad = make_desc(smem_u32(sm + P_KV + kVoff[pp] * 128 + ks * 32), 16, 1024);
-                        const uint64_t bd = make_desc(smem_u32(sm + P_KQ + 32 * pp * 128 + ks * 32), 16, 1024);
-                        mma_bf16(tmem + 32 * pp, ad, bd, idesc, (hh > 0 || ks > 0) ? 1u : 0u);
-                    }
-                commit(&bar);
-            }
-            // while the MMAs run: scale Q e^G, K e^{G_last - G} (image) and K e^G (in place)
-#pragma unroll
-            for (int rr = 0; rr < 2; ++rr) {
-                const int t = 16 * p + tr + 8 * rr;
-                const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
-                float tmp[8];
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * egs[j];
-                *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * egl[j];
-                *reinterpret_cast<uint4*>(img + IMG_B2 + (1 + hh) * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) tmp[j] = kin[rr][j] * eg[j];
-                *reinterpret_cast<uint4*>(sm + P_K + off) = pack8(tmp);
-            }
-            ok = block_wait(&bar, hh & 1, err, 2) && ok;
-            fence_after_sync();
-        }
-    }
-
+    // loads issued and waited for per barrier (at most one in flight each), and
+    // completions of the MMA barrier waited for; identical in every thread
+    uint32_t g_issued = cur >= 0 ? 1 : 0, kq_issued = g_issued, g_seen = 0, kq_seen = 0, mph = 0;
+    bool ok = true;
     float* sA = reinterpret_cast<float*>(sm + P_A);
     float* sT = reinterpret_cast<float*>(sm + P_T);
-    if (ok) {
-        // ---- extract A (fp32, for the inverse) and Aqk^T (bf16 image rows);
-        // warps w and w + 4 share a TMEM lane quarter and take two strips each
-        const int j = 16 * sp + l;
-        float kp[2][16], qp[2][16];
+
+    while (cur >= 0 && ok) {
+        const int64_t gc = cur / hg;
+        const int hl = (int)(cur - gc * hg);
+        const int64_t h = h_base + hl;
+        unsigned char* img = ws + (gc * Hg + hl) * (int64_t)IMG_BYTES;
+        int64_t n2 = 0, t02 = 0, len2 = 0;
+        const int64_t nxt = next_item(cur + gridDim.x, n2, t02, len2);
+
+        const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
+        if (tid < C) sB[tid] = bval;
+        fence_before_sync();
+        ok = block_wait(&bar_g, g_seen & 1, err, 1);   // also the barrier for sB
+        fence_after_sync();
+        if (!ok) break;
+        ++g_seen;
+
+        if (ok) {
+            // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
+            // Threads c and c + 128 scan tokens 0..31 and 32..63 in registers; the second
+            // half then adds the first half's total and derives the per-channel vectors.
+            {
+                const int c = tid & 127, part = tid >> 7, tb = 32 * part;
+                const unsigned char* slab = sGb + (c >> 5) * 8192 + (c & 3) * 4;
+                const int q0 = (c & 31) >> 2;
+                float v[32];
 #pragma unroll
-        for (int x = 0; x < 2; ++x) {
-            const int p = 2 * (w >> 2) + x;
-            tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p, kp[x]);
-            tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p + 16, qp[x]);
+                for (int x = 0; x < 32; ++x)
+                    v[x] = *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
+                float run = 0.f;
+#pragma unroll
+                for (int x = 0; x < 32; ++x) {
+                    run += (tb + x < len) ? kLog2e * v[x] : 0.f;
+                    v[x] = run;
+                }
+                if (part == 0) {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x)
+                        *reinterpret_cast<float*>(const_cast<unsigned char*>(slab) + x * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
+                }
+                __syncthreads();
+                if (part == 1) {
+                    const float base = G(31, c);
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        v[x] += base;
+                        *reinterpret_cast<float*>(const_cast<unsigned char*>(slab) + (32 + x) * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
+                    }
+                    const float Gl = v[31];
+                    const float Gf[4] = {G(0, c), G(16, c), v[0], v[16]};
+#pragma unroll
+                    for (int p = 0; p < 4; ++p) {
+                        egf[p * VP + vidx(c)] = ex2(Gf[p]);
+                        eglf[p * VP + vidx(c)] = ex2(Gl - Gf[p]);
+                    }
+                    int idx = 0;
+#pragma unroll
+                    for (int p = 1; p < 4; ++p)
+#pragma unroll
+                        for (int r = 0; r < p; ++r) dvec[(idx++) * VP + vidx(c)] = ex2(Gf[p] - Gf[r]);
+                    reinterpret_cast<float*>(img + IMG_GAM)[c] = ex2(Gl);
+                }
+            }
+            ok = block_wait(&bar_kq, kq_seen & 1, err, 1) && ok;   // also the end of (a)
+            fence_after_sync();
+            if (ok) ++kq_seen;
+            if (ok && len < C) {
+                // a partial chunk: tokens past its end (next sequence or zero fill) read as zero
+                for (int e = tid; e < (C - (int)len) * 16; e += PT) {
+                    const int t = (int)len + (e >> 4), ch = e & 15;
+                    const uint32_t off = (ch >> 3) * 8192 + sw128_offset(t, (8 * ch) & 63);
+                    *reinterpret_cast<uint4*>(sm + P_K + off) = make_uint4(0, 0, 0, 0);
+                    *reinterpret_cast<uint4*>(sm + P_Q + off) = make_uint4(0, 0, 0, 0);
+                }
+                __syncthreads();
+            }
+
+            // ---- (b1) A / Aqk strips: operands built per channel half, MMAs accumulate.
+            // Thread (ch8, tr, p) handles channels c0 .. c0 + 7 of row 16p + tr (sub-chunk
+            // p) and of row 16(3 - p) + tr + 8 (sub-chunk 3 - p): every thread then writes
+            // the same number of later-sub-chunk key variants (three).
+            const int ch8 = tid & 7, tr = (tid >> 3) & 7, p = tid >> 6;
+            for (int hh = 0; hh < 2 && ok; ++hh) {
+                const int c0 = 64 * hh + 8 * ch8;
+                const int vc = vidx(c0);
+                const unsigned char* slab = sGb + (c0 >> 5) * 8192;
+                const int q0 = (c0 & 31) >> 2;
+                float kin[2][8], qin[2][8], kd[2][8];
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int ps = rr == 0 ? p : 3 - p;            // sub-chunk of this row
+                    const int t = 16 * ps + tr + 8 * rr;
+                    float Gf8[8], G8[8], kk[8], qq[8];
+                    {
+                        const int tf = 16 * ps;
+                        const float4 fa = *reinterpret_cast<const float4*>(slab + tf * 128 + (q0 << 4));
+                        const float4 fb = *reinterpret_cast<const float4*>(slab + tf * 128 + ((q0 + 1) << 4));
+                        Gf8[0] = fa.x; Gf8[1] = fa.y; Gf8[2] = fa.z; Gf8[3] = fa.w;
+                        Gf8[4] = fb.x; Gf8[5] = fb.y; Gf8[6] = fb.z; Gf8[7] = fb.w;
+                        const float4 a = *reinterpret_cast<const float4*>(slab + t * 128 + ((q0 ^ (t & 7)) << 4));
+                        const float4 b = *reinterpret_cast<const float4*>(slab + t * 128 + (((q0 + 1) ^ (t & 7)) << 4));
+                        G8[0] = a.x; G8[1] = a.y; G8[2] = a.z; G8[3] = a.w;
+                        G8[4] = b.x; G8[5] = b.y; G8[6] = b.z; G8[7] = b.w;
+                    }
+                    const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
+                    unpack8(*reinterpret_cast<const uint4*>(sm + P_K + off), kk);
+                    unpack8(*reinterpret_cast<const uint4*>(sm + P_Q + off), qq);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) {
+                        const float x = G8[j] - Gf8[j];
+                        const float e1 = ex2(x);          // <= 1
+                        const float r1 = ex2(-x);         // >= 1, at most 15 tokens of decay
+                        kin[rr][j] = kk[j] * e1;
+                        qin[rr][j] = qq[j] * e1;          // `scale` is applied to Aqk and Q e^G later
+                        kd[rr][j] = kk[j] * r1;
+                    }
+                    // operands of the strip MMAs first
+                    const int ts = tr + 8 * rr;          // row within the sub-chunk
+                    float tmp[8];
+                    *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * ps + ts, 8 * ch8)) = pack8(kin[rr]);
+                    *reinterpret_cast<uint4*>(sm + P_KQ + sw128_offset(32 * ps + 16 + ts, 8 * ch8)) = pack8(qin[rr]);
+                    *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[ps] + t, 8 * ch8)) = pack8(kd[rr]);
+#pragma unroll
+                    for (int pv = 1; pv < 4; ++pv) {
+                        if (pv > ps) {
+                            float dv8[8];
+                            ld8f(dvec + ((pv * (pv - 1)) / 2 + ps) * VP + vc, dv8);
+#pragma unroll
+                            for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * dv8[j];
+                            *reinterpret_cast<uint4*>(sm + P_KV + sw128_offset(kVoff[pv] + t, 8 * ch8)) = pack8(tmp);
+                        }
+                    }
+                }
+                fence_smem_to_async();
+                fence_before_sync();
+                __syncthreads();
+                if (tid == 0) {
+                    fence_after_sync();
+                    const uint32_t idesc = make_idesc_bf16(64, 32, false, false);
+#pragma unroll
+                    for (int pp = 0; pp < 4; ++pp)
+#pragma unroll
+                        for (int ks = 0; ks < 4; ++ks) {
+                            const uint64_t ad = make_desc(smem_u32(sm + P_KV + kVoff[pp] * 128 + ks * 32), 16, 1024);
+                            const uint64_t bd = make_desc(smem_u32(sm + P_KQ + 32 * pp * 128 + ks * 32), 16, 1024);
+                            mma_bf16(tmem + 32 * pp, ad, bd, idesc, (hh > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    commit(&bar);
+                    if (hh == 1 && nxt >= 0) issue_g(nxt, t02);   // G is not read again
+                }
+                if (hh == 1 && nxt >= 0) ++g_issued;
+                // while the MMAs run: scale Q e^G, K e^{G_last - G} (image) and K e^G (in place)
+#pragma unroll
+                for (int rr = 0; rr < 2; ++rr) {
+                    const int ps = rr == 0 ? p : 3 - p;
+                    const int t = 16 * ps + tr + 8 * rr;
+                    const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
+                    float eg[8], egl[8], egs[8], tmp[8];
+                    ld8f(egf + ps * VP + vc, eg);
+                    ld8f(eglf + ps * VP + vc, egl);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) egs[j] = scale * eg[j];
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * egs[j];
+                    *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * egl[j];
+                    *reinterpret_cast<uint4*>(img + IMG_B2 + (1 + hh) * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
+#pragma unroll
+                    for (int j = 0; j < 8; ++j) tmp[j] = kin[rr][j] * eg[j];
+                    *reinterpret_cast<uint4*>(sm + P_K + off) = pack8(tmp);
+                }
+                ok = block_wait(&bar, mph & 1, err, 2) && ok;
+                fence_after_sync();
+                ++mph;
+            }
         }
-        tmem_wait_ld();
-        if (l < 16) {
+
+        if (ok) {
+            // ---- extract A (fp32, for the inverse) and Aqk^T (bf16 image rows);
+            // warps w and w + 4 share a TMEM lane quarter and take two strips each
+            const int j = 16 * sp + l;
+            float kp[2][16], qp[2][16];
 #pragma unroll
             for (int x = 0; x < 2; ++x) {
                 const int p = 2 * (w >> 2) + x;
-                float aq[16], bt[16];
-                ld8f(sB + 16 * p, bt);
-                ld8f(sB + 16 * p + 8, bt + 8);
-#pragma unroll
-                for (int cc = 0; cc < 16; ++cc) {
-                    const int i = 16 * p + cc;
-                    sA[i * AP + j] = (j < i) ? bt[cc] * kp[x][cc] : 0.f;
-                    aq[cc] = (j <= i) ? scale * qp[x][cc] : 0.f;
-                }
-                *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
-                *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p + 8)) = pack8(aq + 8);
+                tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p, kp[x]);
+                tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p + 16, qp[x]);
             }
+            tmem_wait_ld();
+            if (l < 16) {
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int p = 2 * (w >> 2) + x;
+                    float aq[16], bt[16];
+                    ld8f(sB + 16 * p, bt);
+                    ld8f(sB + 16 * p + 8, bt + 8);
+#pragma unroll
+                    for (int cc = 0; cc < 16; ++cc) {
+                        const int i = 16 * p + cc;
+                        sA[i * AP + j] = (j < i) ? bt[cc] * kp[x][cc] : 0.f;
+                        aq[cc] = (j <= i) ? scale * qp[x][cc] : 0.f;
+                    }
+                    *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
+                    *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p + 8)) = pack8(aq + 8);
+                }
+            }
+            fence_before_sync();
+            __syncthreads();
+
+            ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, mph & 1, err, [&] {
+                if (tid == 0 && nxt >= 0) issue_kq(nxt, t02);
+                if (nxt >= 0) ++kq_issued;
+            });
+            ++mph;
         }
         fence_before_sync();
-        __syncthreads();
-
-        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 0, err);
-    } else {
-        // the input loads may still be in flight: let them land before leaving
-        mbar_wait(&bar_in, 0, nullptr, 0, 200);
+        __syncthreads();                               // TMEM, sA, sT and sB reads of this item are done
+        cur = nxt;
+        n = n2;
+        t0 = t02;
+        len = len2;
+    }
+    // after an error: let the loads in flight land before the CTA leaves
+    if (tid == 0) {
+        if (g_seen < g_issued) mbar_wait(&bar_g, g_seen & 1, nullptr, 0, 200);
+        if (kq_seen < kq_issued) mbar_wait(&bar_kq, kq_seen & 1, nullptr, 0, 200);
     }
     fence_before_sync();
     __syncthreads();
@@ -699,7 +759,7 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
         fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
-        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 1, err);
+        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 1, err, [] {});
     } else if (!ok) {
         // the input loads may still be in flight: let them land before leaving
         mbar_wait(&bar_in, 0, nullptr, 0, 200);
@@ -1057,12 +1117,16 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         if (a.si.chunks_upper <= 0) return cudaSuccess;
         dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
         LaunchScope scope(s, K_PREP_TC);
-        if (a.gate_scalar)
+        if (a.gate_scalar) {
             tc::chunk_prep_gdn_tc_kernel<<<gp, tc::PT, tc::GP_SMEM, s>>>(
                 maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, a.scale, w, err);
-        else
-            tc::chunk_prep_tc_kernel<<<gp, tc::PT, tc::P_SMEM, s>>>(
-                maps, a.beta, a.si, a.H, hb, Hg, a.scale, w, err);
+        } else {
+            // persistent: two CTAs per SM walk the (chunk, head) items
+            const int64_t items = a.si.chunks_upper * hg;
+            const int64_t slots = 2 * device_sm_count();
+            tc::chunk_prep_tc_kernel<<<(unsigned)(items < slots ? items : slots), tc::PT, tc::P_SMEM, s>>>(
+                maps, a.beta, a.si, a.H, hb, Hg, hg, a.scale, w, err);
+        }
         return cudaGetLastError();
     };
     SegPlan none;

@@ -211,6 +211,9 @@ struct DecodeArgs {
 // Runs `f` (a per-device setup such as raising a kernel's shared-memory
 // limit) once per device: the bit of the current device in `done` is set after
 // the first success.  Devices past 63 run it every time.
+// Streaming multiprocessors of the current device (queried once per device).
+int64_t device_sm_count();
+
 template <typename F>
 inline cudaError_t once_per_device(std::atomic<uint64_t>& done, F f)
 {
