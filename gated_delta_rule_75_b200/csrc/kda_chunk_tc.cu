@@ -164,7 +164,6 @@ constexpr int VP = 144;                // floats per vector: 4 pad floats after 
 constexpr uint32_t P_BETA = P_VEC + 14 * VP * 4;   // beta [64], then the scalar gates [64]
 constexpr uint32_t P_BYTES = P_BETA + 512;
 constexpr uint32_t P_SMEM = P_BYTES + 1024 + 64;
-constexpr uint32_t P_TX = 16384 + 16384 + 32768;   // bytes the input TMA loads deliver
 static_assert(P_T + 64 * AP * 4 <= P_VEC, "A/T overlap the vectors");
 
 // Index of channel c in a padded per-channel vector: the 8-channel groups that a
@@ -304,6 +303,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ uint64_t bar_g, bar_kq, bar;
     __shared__ uint32_t tmem_base;
+    __shared__ int32_t s_next[2][3];              // an item, its first token and length
 
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3;                          // TMEM lane quarter of this warp
@@ -317,21 +317,29 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     // Work items are (chunk, head) pairs, item = chunk * hg + head; this CTA takes
     // blockIdx.x, blockIdx.x + gridDim.x, ...  The next item's gates are fetched as soon
     // as the current one's are last read (after the operand build), its k and q once the
-    // W MMA has consumed P_K and P_Q, so the loads overlap the rest of the current item.
-    const int64_t items = si.chunks_upper * hg;
-    auto next_item = [&](int64_t from, int64_t& n_, int64_t& t0_, int64_t& len_) -> int64_t {
-        for (int64_t it = from; it < items; it += gridDim.x)
-            if (si.locate(it / hg, n_, t0_, len_)) return it;
+    // W MMA has consumed P_K and P_Q, and its beta at the start of the current item, so the
+    // loads overlap the rest of the current item.  One thread finds the next item (items
+    // and token rows fit in 32 bits: the launch checks both).
+    const int32_t items = (int32_t)(si.chunks_upper * hg), hg32 = (int32_t)hg;
+    auto next_item = [&](int32_t from, int32_t& t0_, int32_t& len_) -> int32_t {
+        for (int32_t it = from; it < items; it += (int32_t)gridDim.x) {
+            int64_t n_, t, ln;
+            if (si.locate(it / hg32, n_, t, ln)) {
+                t0_ = (int32_t)t;
+                len_ = (int32_t)ln;
+                return it;
+            }
+        }
         return -1;
     };
-    auto issue_g = [&](int64_t item, int64_t t0_) {               // one thread
-        const int32_t y = (int32_t)t0_, x = (int32_t)((h_base + item % hg) * D);
+    auto issue_g = [&](int32_t item, int32_t t0_) {               // one thread
+        const int32_t y = t0_, x = (int32_t)((h_base + item % hg32) * D);
         tma::expect_tx(&bar_g, 32768);
 #pragma unroll
         for (int s4 = 0; s4 < 4; ++s4) tma::load_2d(sGb + s4 * 8192, &maps.g, x + 32 * s4, y, &bar_g);
     };
-    auto issue_kq = [&](int64_t item, int64_t t0_) {              // one thread
-        const int32_t y = (int32_t)t0_, x = (int32_t)((h_base + item % hg) * D);
+    auto issue_kq = [&](int32_t item, int32_t t0_) {              // one thread
+        const int32_t y = t0_, x = (int32_t)((h_base + item % hg32) * D);
         tma::expect_tx(&bar_kq, 32768);
         tma::load_2d(sm + P_K, &maps.k, x, y, &bar_kq);
         tma::load_2d(sm + P_K + 8192, &maps.k, x + 64, y, &bar_kq);
@@ -339,22 +347,31 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         tma::load_2d(sm + P_Q + 8192, &maps.q, x + 64, y, &bar_kq);
     };
 
-    int64_t n = 0, t0 = 0, len = 0;
-    int64_t cur = next_item(blockIdx.x, n, t0, len);
+    auto load_beta = [&](int32_t item, int32_t t0_, int32_t len_) -> float {
+        return (item >= 0 && tid < len_) ? beta[((int64_t)t0_ + tid) * H + h_base + item % hg32] : 0.f;
+    };
+
     if (tid == 0) {
+        int32_t t_ = 0, l_ = 0;
+        const int32_t it = next_item((int32_t)blockIdx.x, t_, l_);
+        s_next[0][0] = it;
+        s_next[0][1] = t_;
+        s_next[0][2] = l_;
         mbar_init(&bar_g, 1);
         mbar_init(&bar_kq, 1);
         mbar_init(&bar, 1);
         fence_mbar_init();
-        if (cur >= 0) {
-            issue_g(cur, t0);
-            issue_kq(cur, t0);
+        if (it >= 0) {
+            issue_g(it, t_);
+            issue_kq(it, t_);
         }
     }
     if (w == 0) { tmem_alloc(&tmem_base, 128); tmem_relinquish(); }
     fence_before_sync();
     __syncthreads();
     fence_after_sync();
+    int32_t cur = s_next[0][0], t0 = s_next[0][1], len = s_next[0][2];
+    float bnext = load_beta(cur, t0, len);
     const uint32_t tmem = tmem_base;
     // loads issued and waited for per barrier (at most one in flight each), and
     // completions of the MMA barrier waited for; identical in every thread
@@ -364,20 +381,25 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     float* sT = reinterpret_cast<float*>(sm + P_T);
 
     while (cur >= 0 && ok) {
-        const int64_t gc = cur / hg;
-        const int hl = (int)(cur - gc * hg);
-        const int64_t h = h_base + hl;
-        unsigned char* img = ws + (gc * Hg + hl) * (int64_t)IMG_BYTES;
-        int64_t n2 = 0, t02 = 0, len2 = 0;
-        const int64_t nxt = next_item(cur + gridDim.x, n2, t02, len2);
-
-        const float bval = (tid < len) ? beta[(t0 + (tid < C ? tid : 0)) * H + h] : 0.f;
-        if (tid < C) sB[tid] = bval;
+        const int32_t gc = cur / hg32, hl = cur - gc * hg32;
+        unsigned char* img = ws + ((int64_t)gc * Hg + hl) * (int64_t)IMG_BYTES;
+        // item i + 1 goes to s_next[(i + 1) & 1]: the last reads of that entry came before
+        // the previous item's barriers (g_seen counts the items started)
+        int32_t* sn = s_next[(g_seen + 1) & 1];
+        if (tid == 0) {
+            int32_t t_ = 0, l_ = 0;
+            sn[0] = next_item(cur + (int32_t)gridDim.x, t_, l_);
+            sn[1] = t_;
+            sn[2] = l_;
+        }
+        if (tid < C) sB[tid] = bnext;
         fence_before_sync();
-        ok = block_wait(&bar_g, g_seen & 1, err, 1);   // also the barrier for sB
+        ok = block_wait(&bar_g, g_seen & 1, err, 1);   // also the barrier for sB and s_next
         fence_after_sync();
         if (!ok) break;
         ++g_seen;
+        const int32_t nxt = sn[0], t02 = sn[1], len2 = sn[2];
+        bnext = load_beta(nxt, t02, len2);
 
         if (ok) {
             // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
@@ -392,10 +414,18 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 for (int x = 0; x < 32; ++x)
                     v[x] = *reinterpret_cast<const float*>(slab + (tb + x) * 128 + ((q0 ^ (x & 7)) << 4));
                 float run = 0.f;
+                if (len == C) {
 #pragma unroll
-                for (int x = 0; x < 32; ++x) {
-                    run += (tb + x < len) ? kLog2e * v[x] : 0.f;
-                    v[x] = run;
+                    for (int x = 0; x < 32; ++x) {
+                        run += kLog2e * v[x];
+                        v[x] = run;
+                    }
+                } else {
+#pragma unroll
+                    for (int x = 0; x < 32; ++x) {
+                        run += (tb + x < len) ? kLog2e * v[x] : 0.f;
+                        v[x] = run;
+                    }
                 }
                 if (part == 0) {
 #pragma unroll
@@ -552,18 +582,30 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * p + 16, qp[x]);
             }
             tmem_wait_ld();
+            // Rows i of strip p against columns j of block sp (warp-uniform): blocks above
+            // the diagonal are zero in Aqk and never read in A (the inverse reads the strictly
+            // lower part of A and parks scratch blocks above it), so A needs no mask at all.
             if (l < 16) {
 #pragma unroll
                 for (int x = 0; x < 2; ++x) {
-                    const int p = 2 * (w >> 2) + x;
-                    float aq[16], bt[16];
-                    ld8f(sB + 16 * p, bt);
-                    ld8f(sB + 16 * p + 8, bt + 8);
+                    const int p = 2 * (w >> 2) + x, rel = sp - p;
+                    float aq[16];
+                    if (rel <= 0) {
+                        float bt[16];
+                        ld8f(sB + 16 * p, bt);
+                        ld8f(sB + 16 * p + 8, bt + 8);
 #pragma unroll
-                    for (int cc = 0; cc < 16; ++cc) {
-                        const int i = 16 * p + cc;
-                        sA[i * AP + j] = (j < i) ? bt[cc] * kp[x][cc] : 0.f;
-                        aq[cc] = (j <= i) ? scale * qp[x][cc] : 0.f;
+                        for (int cc = 0; cc < 16; ++cc) sA[(16 * p + cc) * AP + j] = bt[cc] * kp[x][cc];
+                    }
+                    if (rel < 0) {
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc) aq[cc] = scale * qp[x][cc];
+                    } else if (rel == 0) {
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc) aq[cc] = (l <= cc) ? scale * qp[x][cc] : 0.f;
+                    } else {
+#pragma unroll
+                        for (int cc = 0; cc < 16; ++cc) aq[cc] = 0.f;
                     }
                     *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p)) = pack8(aq);
                     *reinterpret_cast<uint4*>(img + IMG_B2 + sw128_offset(j, 16 * p + 8)) = pack8(aq + 8);
@@ -581,7 +623,6 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
         fence_before_sync();
         __syncthreads();                               // TMEM, sA, sT and sB reads of this item are done
         cur = nxt;
-        n = n2;
         t0 = t02;
         len = len2;
     }
@@ -1123,6 +1164,7 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         } else {
             // persistent: two CTAs per SM walk the (chunk, head) items
             const int64_t items = a.si.chunks_upper * hg;
+            if (items > INT32_MAX) return cudaErrorInvalidValue;   // items are 32-bit in the kernel
             const int64_t slots = 2 * device_sm_count();
             tc::chunk_prep_tc_kernel<<<(unsigned)(items < slots ? items : slots), tc::PT, tc::P_SMEM, s>>>(
                 maps, a.beta, a.si, a.H, hb, Hg, hg, a.scale, w, err);
