@@ -106,6 +106,12 @@ __device__ __forceinline__ uint32_t tf32(float x)
     return r;
 }
 
+// Barrier `id` (1..15) over the first `count` threads that reach it (whole warps).
+__device__ __forceinline__ void bar_sync_named(int id, int count)
+{
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
 // acc (16x16, m16n8 fragments for the two 8-column halves) += X * Y, where X
 // and Y are 16x16 fp32 blocks in shared memory with a row pitch of P floats.
 template <int P>
@@ -186,16 +192,23 @@ struct PrepMaps {
 // bf16 K-major image (in P_Q and in the workspace), and W = -T' (K e^G) by one MMA whose
 // completion is phase `parity` of `bar`; W goes to the workspace image.  `after_mma()` runs in
 // every thread once that MMA has completed (its operands in P_Q and P_K are no longer read).
+// The inverse runs on warps 0-3; warps 4-7 run `side()` meanwhile (work that touches none of
+// A, T, beta or the operands here), whose result every thread gets in `side_ok`.
 // Returns false when the bounded wait gave up.
-template <typename AfterMma>
+template <typename AfterMma, typename Side>
 __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img, float* sA, float* sT,
                                           const float* sB, uint32_t tmem, uint64_t* bar,
-                                          uint32_t parity, int* err, AfterMma after_mma)
+                                          uint32_t parity, int* err, AfterMma after_mma, Side side,
+                                          bool& side_ok)
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3;                          // TMEM lane quarter of this warp
-    // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution,
-    // one column per thread, held in registers
+    // ---- (b2) T = (I + A)^{-1} on warps 0-3: diagonal 16x16 blocks by forward
+    // substitution, one column per thread, held in registers
+    bool mine = true;
+    if (w >= 4) {
+        mine = side();
+    } else {
     if (tid < C) {
         const int b = tid >> 4, cc = tid & 15, o = 16 * b;
         float tcol[16];
@@ -209,7 +222,7 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
     }
-    __syncthreads();
+    bar_sync_named(1, 128);
     // off-diagonal blocks, 32 x 32 recursion (X blocks are parked in the unused
     // upper blocks of A):
     //   level 1 (warps 0, 1): T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
@@ -227,22 +240,23 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
             mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
             store16x16<AP>(Tb(p, r), acc2, -1.f, l);
         }
-        __syncthreads();
-        if (w < 4) {
+        bar_sync_named(1, 128);
+        {
             const int p = 2 + (w >> 1), r = w & 1;       // X_pr = sum_{m=r..1} A_pm T_mr
             float acc[2][4] = {};
             for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
             store16x16<AP>(Ab(r, p), acc, 1.f, l);
         }
-        __syncthreads();
-        if (w < 4) {
+        bar_sync_named(1, 128);
+        {
             const int p = 2 + (w >> 1), r = w & 1;       // T_pr = -sum_{m=2..p} T_pm X_mr
             float acc[2][4] = {};
             for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
             store16x16<AP>(Tb(p, r), acc, -1.f, l);
         }
-        __syncthreads();
     }
+    }
+    side_ok = __syncthreads_and(mine ? 1 : 0) != 0;
     // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
     for (int e = tid; e < C * 8; e += PT) {
         const int i = e >> 3, cb = e & 7;
@@ -304,6 +318,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     __shared__ uint64_t bar_g, bar_kq, bar;
     __shared__ uint32_t tmem_base;
     __shared__ int32_t s_next[2][3];              // an item, its first token and length
+    __shared__ int s_gates_ok;                    // the next item's gates arrived (warps 4-7)
 
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3;                          // TMEM lane quarter of this warp
@@ -376,16 +391,54 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
     // loads issued and waited for per barrier (at most one in flight each), and
     // completions of the MMA barrier waited for; identical in every thread
     uint32_t g_issued = cur >= 0 ? 1 : 0, kq_issued = g_issued, g_seen = 0, kq_seen = 0, mph = 0;
-    bool ok = true;
+    uint32_t started = 0;                          // items begun
+    bool ok = true, scanned = false;               // scanned: this item's step (a) is done
     float* sA = reinterpret_cast<float*>(sm + P_A);
     float* sT = reinterpret_cast<float*>(sm + P_T);
+
+    // Step (a) for one channel c over all tokens, by one thread (the 128-thread form that
+    // warps 4-7 run for the next item while warps 0-3 invert (I + A) of the current one):
+    // G in place, the per-channel vectors and e^{G_last} into `img_`.
+    auto scan_channel = [&](int c, int len_, unsigned char* img_) {
+        unsigned char* slab = sGb + (c >> 5) * 8192 + (c & 3) * 4;
+        const int q0 = (c & 31) >> 2;
+        float run = 0.f, Gf[4];
+#pragma unroll
+        for (int pq = 0; pq < 4; ++pq) {
+            float v[16];
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+                v[x] = *reinterpret_cast<const float*>(slab + (16 * pq + x) * 128 + ((q0 ^ (x & 7)) << 4));
+#pragma unroll
+            for (int x = 0; x < 16; ++x) {
+                run += (len_ == C || 16 * pq + x < len_) ? kLog2e * v[x] : 0.f;
+                v[x] = run;
+            }
+            Gf[pq] = v[0];
+#pragma unroll
+            for (int x = 0; x < 16; ++x)
+                *reinterpret_cast<float*>(slab + (16 * pq + x) * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
+        }
+        const float Gl = run;
+#pragma unroll
+        for (int pq = 0; pq < 4; ++pq) {
+            egf[pq * VP + vidx(c)] = ex2(Gf[pq]);
+            eglf[pq * VP + vidx(c)] = ex2(Gl - Gf[pq]);
+        }
+        int idx = 0;
+#pragma unroll
+        for (int pq = 1; pq < 4; ++pq)
+#pragma unroll
+            for (int r = 0; r < pq; ++r) dvec[(idx++) * VP + vidx(c)] = ex2(Gf[pq] - Gf[r]);
+        reinterpret_cast<float*>(img_ + IMG_GAM)[c] = ex2(Gl);
+    };
 
     while (cur >= 0 && ok) {
         const int32_t gc = cur / hg32, hl = cur - gc * hg32;
         unsigned char* img = ws + ((int64_t)gc * Hg + hl) * (int64_t)IMG_BYTES;
         // item i + 1 goes to s_next[(i + 1) & 1]: the last reads of that entry came before
-        // the previous item's barriers (g_seen counts the items started)
-        int32_t* sn = s_next[(g_seen + 1) & 1];
+        // the previous item's barriers
+        int32_t* sn = s_next[(started + 1) & 1];
         if (tid == 0) {
             int32_t t_ = 0, l_ = 0;
             sn[0] = next_item(cur + (int32_t)gridDim.x, t_, l_);
@@ -393,15 +446,12 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             sn[2] = l_;
         }
         if (tid < C) sB[tid] = bnext;
-        fence_before_sync();
-        ok = block_wait(&bar_g, g_seen & 1, err, 1);   // also the barrier for sB and s_next
-        fence_after_sync();
-        if (!ok) break;
-        ++g_seen;
-        const int32_t nxt = sn[0], t02 = sn[1], len2 = sn[2];
-        bnext = load_beta(nxt, t02, len2);
-
-        if (ok) {
+        if (!scanned) {
+            fence_before_sync();
+            ok = block_wait(&bar_g, g_seen & 1, err, 1);
+            fence_after_sync();
+            if (!ok) break;
+            ++g_seen;
             // ---- (a) cumulative log-decay per channel in log2 units; rows >= len add nothing.
             // Threads c and c + 128 scan tokens 0..31 and 32..63 in registers; the second
             // half then adds the first half's total and derives the per-channel vectors.
@@ -455,10 +505,15 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                     reinterpret_cast<float*>(img + IMG_GAM)[c] = ex2(Gl);
                 }
             }
-            ok = block_wait(&bar_kq, kq_seen & 1, err, 1) && ok;   // also the end of (a)
-            fence_after_sync();
-            if (ok) ++kq_seen;
-            if (ok && len < C) {
+        }
+        ok = block_wait(&bar_kq, kq_seen & 1, err, 1);   // end of (a); barrier for sB and s_next
+        fence_after_sync();
+        if (!ok) break;
+        ++kq_seen;
+        const int32_t nxt = sn[0], t02 = sn[1], len2 = sn[2];
+        bnext = load_beta(nxt, t02, len2);
+        {
+            if (len < C) {
                 // a partial chunk: tokens past its end (next sequence or zero fill) read as zero
                 for (int e = tid; e < (C - (int)len) * 16; e += PT) {
                     const int t = (int)len + (e >> 4), ch = e & 15;
@@ -614,17 +669,32 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
             fence_before_sync();
             __syncthreads();
 
+            // warps 4-7: step (a) of the next item while warps 0-3 invert
+            bool side_ok = true;
             ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, mph & 1, err, [&] {
                 if (tid == 0 && nxt >= 0) issue_kq(nxt, t02);
                 if (nxt >= 0) ++kq_issued;
-            });
+            }, [&]() -> bool {
+                if (nxt < 0) return true;
+                if (tid == 128) s_gates_ok = mbar_wait(&bar_g, g_seen & 1, err, 1) ? 1 : 0;
+                bar_sync_named(2, 128);
+                if (!s_gates_ok) return false;
+                const int32_t gcn = nxt / hg32;
+                scan_channel(tid - 128, len2,
+                             ws + ((int64_t)gcn * Hg + (nxt - gcn * hg32)) * (int64_t)IMG_BYTES);
+                return true;
+            }, side_ok);
             ++mph;
+            scanned = nxt >= 0 && side_ok;
+            if (scanned) ++g_seen;
+            ok = ok && side_ok;
         }
         fence_before_sync();
         __syncthreads();                               // TMEM, sA, sT and sB reads of this item are done
         cur = nxt;
         t0 = t02;
         len = len2;
+        ++started;
     }
     // after an error: let the loads in flight land before the CTA leaves
     if (tid == 0) {
@@ -800,7 +870,8 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
         fence_smem_to_async();
         fence_before_sync();
         __syncthreads();
-        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 1, err, [] {});
+        bool side_ok;
+        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 1, err, [] {}, [] { return true; }, side_ok);
     } else if (!ok) {
         // the input loads may still be in flight: let them land before leaving
         mbar_wait(&bar_in, 0, nullptr, 0, 200);
