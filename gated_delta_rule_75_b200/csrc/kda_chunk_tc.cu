@@ -195,7 +195,7 @@ struct PrepMaps {
 // The inverse runs on warps 0-3; warps 4-7 run `side()` meanwhile (work that touches none of
 // A, T, beta or the operands here), whose result every thread gets in `side_ok`.
 // Returns false when the bounded wait gave up.
-template <typename AfterMma, typename Side>
+template <bool kSplit, typename AfterMma, typename Side>
 __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img, float* sA, float* sT,
                                           const float* sB, uint32_t tmem, uint64_t* bar,
                                           uint32_t parity, int* err, AfterMma after_mma, Side side,
@@ -203,31 +203,35 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
 {
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int sp = w & 3;                          // TMEM lane quarter of this warp
-    // ---- (b2) T = (I + A)^{-1} on warps 0-3: diagonal 16x16 blocks by forward
-    // substitution, one column per thread, held in registers
+    // barrier of the warps that take part in the inverse: 0-3 with kSplit, else all
+    auto inv_sync = [] {
+        if constexpr (kSplit) bar_sync_named(1, 128);
+        else __syncthreads();
+    };
     bool mine = true;
-    if (w >= 4) {
+    if (kSplit && w >= 4) {
         mine = side();
     } else {
-    if (tid < C) {
-        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-        float tcol[16];
+        // ---- (b2) T = (I + A)^{-1}: diagonal 16x16 blocks by forward substitution,
+        // one column per thread, held in registers
+        if (tid < C) {
+            const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+            float tcol[16];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc = 0.f;
+            for (int r = 0; r < 16; ++r) {
+                float acc = 0.f;
 #pragma unroll
-            for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
-            tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -acc);
+                for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
+                tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -acc);
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
         }
-#pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
-    }
-    bar_sync_named(1, 128);
-    // off-diagonal blocks, 32 x 32 recursion (X blocks are parked in the unused
-    // upper blocks of A):
-    //   level 1 (warps 0, 1): T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
-    //   level 2: X = A_21 T_1 (rows 2..3, cols 0..1), then T_21 = -T_2 X
-    {
+        inv_sync();
+        // off-diagonal blocks, 32 x 32 recursion (X blocks are parked in the unused
+        // upper blocks of A):
+        //   level 1 (warps 0, 1): T_10 = -T_11 A_10 T_00,  T_32 = -T_33 A_32 T_22
+        //   level 2 (warps 0-3): X = A_21 T_1 (rows 2..3, cols 0..1), then T_21 = -T_2 X
         auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
         auto Tb = [&](int r, int c) { return sT + (16 * r) * AP + 16 * c; };
         if (w < 2) {
@@ -240,23 +244,27 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
             mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
             store16x16<AP>(Tb(p, r), acc2, -1.f, l);
         }
-        bar_sync_named(1, 128);
-        {
+        inv_sync();
+        if (w < 4) {
             const int p = 2 + (w >> 1), r = w & 1;       // X_pr = sum_{m=r..1} A_pm T_mr
             float acc[2][4] = {};
             for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
             store16x16<AP>(Ab(r, p), acc, 1.f, l);
         }
-        bar_sync_named(1, 128);
-        {
+        inv_sync();
+        if (w < 4) {
             const int p = 2 + (w >> 1), r = w & 1;       // T_pr = -sum_{m=2..p} T_pm X_mr
             float acc[2][4] = {};
             for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
             store16x16<AP>(Tb(p, r), acc, -1.f, l);
         }
     }
+    if constexpr (kSplit) {
+        side_ok = __syncthreads_and(mine ? 1 : 0) != 0;
+    } else {
+        __syncthreads();
+        side_ok = true;
     }
-    side_ok = __syncthreads_and(mine ? 1 : 0) != 0;
     // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
     for (int e = tid; e < C * 8; e += PT) {
         const int i = e >> 3, cb = e & 7;
@@ -671,7 +679,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
 
             // warps 4-7: step (a) of the next item while warps 0-3 invert
             bool side_ok = true;
-            ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, mph & 1, err, [&] {
+            ok = prep_tail<true>(sm, img, sA, sT, sB, tmem, &bar, mph & 1, err, [&] {
                 if (tid == 0 && nxt >= 0) issue_kq(nxt, t02);
                 if (nxt >= 0) ++kq_issued;
             }, [&]() -> bool {
@@ -871,7 +879,7 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
         fence_before_sync();
         __syncthreads();
         bool side_ok;
-        ok = prep_tail(sm, img, sA, sT, sB, tmem, &bar, 1, err, [] {}, [] { return true; }, side_ok);
+        ok = prep_tail<false>(sm, img, sA, sT, sB, tmem, &bar, 1, err, [] {}, [] { return true; }, side_ok);
     } else if (!ok) {
         // the input loads may still be in flight: let them land before leaving
         mbar_wait(&bar_in, 0, nullptr, 0, 200);
