@@ -30,9 +30,12 @@
 //   copy) and its v tile (TMA) are double-buffered.  Per chunk:
 //     U^T = V^T T'^T + S^T (-W)^T             (fp32 in TMEM)
 //     O^T = S^T (scale Q e^G)^T
-//     [O^T | S^T] += U^T [Aqk^T | K e^{G_last - G}]   (one MMA, N = 64 + 128)
-//   then O goes to HBM, S^T is copied to bf16 for the next chunk and scaled by
-//   the next chunk's e^{G_last} in TMEM.
+//     S^T += U^T (K e^{G_last - G}),  O^T += U^T Aqk^T
+//   then S^T is copied to bf16 for the next chunk and scaled by the next
+//   chunk's e^{G_last} in TMEM, and O leaves through a shared-memory tile (one
+//   tensor store per whole chunk).  Eight worker warps do the TMEM and SIMT work;
+//   one thread of a ninth warp issues every MMA and copy, and the two sides meet
+//   only on mbarriers, so the issuer's waits on the tensor pipe hold back no worker.
 // Every mbarrier wait is bounded; on a timeout the CTA records it in the
 // workspace error word, drains its own copies and frees its TMEM.
 #include <cstring>
@@ -110,6 +113,24 @@ __device__ __forceinline__ uint32_t tf32(float x)
 __device__ __forceinline__ void bar_sync_named(int id, int count)
 {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Barrier `id` over `count` threads that also ANDs `pred` across them: every thread gets the
+// same answer, so a group can leave a loop together.
+__device__ __forceinline__ bool bar_and_named(int id, int count, bool pred)
+{
+    uint32_t r;
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.and.pred q, %2, %3, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t"
+        "}\n"
+        : "=r"(r)
+        : "r"(pred ? 1u : 0u), "r"(id), "r"(count)
+        : "memory");
+    return r != 0;
 }
 
 // acc (16x16, m16n8 fragments for the two 8-column halves) += X * Y, where X
@@ -899,7 +920,7 @@ constexpr uint32_t S_UBF = S_SBF + 32768;                // U^T bf16, K-major A:
 constexpr uint32_t S_BYTES = S_UBF + 16384;
 constexpr uint32_t S_SMEM = S_BYTES + 1024;
 
-constexpr int ST = 256;                                 // state-kernel threads
+constexpr int ST = 288;                                 // state-kernel threads: 8 worker warps + the issuer's
 
 // What one CTA walks (kMode):
 //   WALK_SEQ   a whole sequence from h0 (or zero): outputs and the final state;
@@ -914,6 +935,7 @@ enum { WALK_SEQ = 0, WALK_VALUE = 1, WALK_MAP = 2, WALK_FINAL = 3 };
 template <bool kHasH0, int kMode>
 __global__ void __launch_bounds__(ST, 1)
 chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constant__ CUtensorMap vmap,
+                      const __grid_constant__ CUtensorMap omap,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, SeqInfo si, int64_t H, int64_t h_base, int64_t Hg,
                       const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err,
@@ -924,7 +946,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    __shared__ uint64_t full[2], bar1, bar2;
+    __shared__ uint64_t full[2], bar1, bar2, barO, uready, sready;
     __shared__ uint32_t tmem_base;
 
     // blocks run heads-innermost over sequences ranked longest first (or over
@@ -980,12 +1002,19 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         else return h0p ? h0p[c * D + j] : 0.f;
     };
 
+    // Roles: warps 0-7 (workers) own the TMEM lanes and all SIMT work; one thread of warp 8
+    // (the issuer) issues every MMA and stage copy.  They meet only on mbarriers: the MMA
+    // commits (bar1: U^T of a chunk; bar2: its state update; barO: all of its MMAs), the stage
+    // copies (full), and two worker arrivals per chunk (uready: U^T staged as an operand;
+    // sready: the next state staged), so neither side ever waits for the other's unrelated work.
+    const bool worker = w < 8;
+    const bool issuer = tid == 8 * 32;
     if (nch == 0) {                                      // nothing to walk: final = entry state
-        if (hTp)
+        if (hTp && worker)
             for (int c = 64 * half; c < 64 * half + 64; ++c) hTp[c * D + j] = s_init(c);
         return;
     }
-    auto load_stage = [&](int64_t ch, int s) {          // one thread
+    auto load_stage = [&](int64_t ch, int s) {          // issuer
         unsigned char* st = sm + s * STAGE_BYTES;
         fence_smem_to_async();
         tma::expect_tx(&full[s], kV ? IMG_BYTES + 16384 : IMG_BYTES);
@@ -997,9 +1026,10 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         }
     };
 
-    if (tid == 0) {
+    if (issuer) {
         mbar_init(&full[0], 1); mbar_init(&full[1], 1);
-        mbar_init(&bar1, 1); mbar_init(&bar2, 1);
+        mbar_init(&bar1, 1); mbar_init(&bar2, 1); mbar_init(&barO, 1);
+        mbar_init(&uready, 8); mbar_init(&sready, 8);  // one arrival per worker warp
         fence_mbar_init();
         load_stage(0, 0);
         if (nch > 1) load_stage(1, 1);
@@ -1012,176 +1042,234 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
     const uint32_t lane = (uint32_t)(32 * qt) << 16;
     const uint32_t tU = tmem, tS = tmem + 256;
     auto tO = [&](int64_t ch) { return tmem + 64 + 64 * (uint32_t)(ch & 1); };
-    bool pending[2] = {true, nch > 1};
-
-    // U^T = V^T T'^T + S^T (-W)^T and O^T = S^T (scale Q e^G)^T for chunk ch (one thread)
-    auto issue_mma1 = [&](int64_t ch) {
-        unsigned char* st = sm + (ch & 1) * STAGE_BYTES;
-        fence_after_sync();
-        if constexpr (kV) {
-            const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
-#pragma unroll
-            for (int ks = 0; ks < 4; ++ks)
-                mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
-                         make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
-        }
-        const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
-        const uint32_t to = tO(ch);
-#pragma unroll
-        for (int ks = 0; ks < 8; ++ks) {
-            const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
-            mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1,
-                     (kV || ks > 0) ? 1u : 0u);
-            if constexpr (kOut)
-                mma_bf16(to, ad, make_desc(smem_u32(st + IMG_QG + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, ks > 0);
-        }
-        commit(&bar1);
+    // a worker warp's arrival: its lanes' shared-memory writes visible to the tensor core and
+    // their TMEM accesses ordered before the issuer's next MMA
+    auto warp_arrive = [&](uint64_t* b) {
+        fence_smem_to_async();
+        fence_before_sync();
+        __syncwarp();
+        if (l == 0) mbar_arrive(b);
     };
+    bool ok = true;
 
-    bool ok = __syncthreads_and(mbar_wait(&full[0], 0, err, 4) ? 1 : 0);
-    if (ok) pending[0] = false;
-
-    // initial state: bf16 copy (operand) and gamma_0-scaled fp32 in TMEM; this
-    // thread owns columns 64*half .. +63 of row j of S^T
-    if (ok) {
-        const float* gam = reinterpret_cast<const float*>(sm + IMG_GAM);
-        unsigned char* dst = sm + S_SBF + half * 16384;
-#pragma unroll 1
-        for (int cb = 0; cb < 4; ++cb) {
-            const int c0 = 64 * half + 16 * cb;
-            float f[16];
-#pragma unroll
-            for (int x = 0; x < 16; ++x) f[x] = s_init(c0 + x);
-            *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f);
-            *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f + 8);
-#pragma unroll
-            for (int x = 0; x < 16; ++x) f[x] *= gam[c0 + x];
-            tmem_st16(tS + lane + c0, f);
-        }
-        tmem_wait_st();
-    }
-    fence_smem_to_async();
-    fence_before_sync();
-    __syncthreads();
-    if (ok && tid == 0) issue_mma1(0);
-
-    for (int64_t ch = 0; ok && ch < nch; ++ch) {
-        const int s = (int)(ch & 1);
-        unsigned char* st = sm + s * STAGE_BYTES;
-        const int64_t t0 = bos + ch * C;
-        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-        const uint32_t ph = (uint32_t)(ch & 1);
-        const bool last = (ch + 1 == nch);
-
-        ok = __syncthreads_and(mbar_wait(&bar1, ph, err, 5) ? 1 : 0);
-        fence_after_sync();
-        if (!ok) break;
-
-        // U^T (fp32, TMEM) -> bf16 operand rows; this thread: tokens 32*half .. +31
-        {
-            float f[2][16];
-            tmem_ld16(tU + lane + 32 * half, f[0]);
-            tmem_ld16(tU + lane + 32 * half + 16, f[1]);
-            tmem_wait_ld();
-#pragma unroll
-            for (int x = 0; x < 2; ++x) {
-                const int c = 32 * half + 16 * x;
-                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, c)) = pack8(f[x]);
-                *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, c + 8)) = pack8(f[x] + 8);
-            }
-        }
-        fence_smem_to_async();
-        fence_before_sync();
-        __syncthreads();
-        if (tid == 0) {
+    if (w == 8) {
+        // the issuer's warp: every lane takes the same branches (the waits' outcomes are shared
+        // with __all_sync), lane 0 issues
+        auto wait_all = [&](uint64_t* b, uint32_t parity, int bit) -> bool {
+            return __all_sync(0xffffffffu, mbar_wait(b, parity, err, bit) ? 1 : 0) != 0;
+        };
+        // stage copies issued and waited for per stage (for the drain after an error)
+        uint32_t issued[2] = {1u, nch > 1 ? 1u : 0u}, seen[2] = {0u, 0u};
+        auto wait_stage = [&](int s) -> bool {
+            if (!wait_all(&full[s], seen[s] & 1, 4)) return false;
+            ++seen[s];
+            return true;
+        };
+        // U^T = V^T T'^T + S^T (-W)^T (commit: bar1), then O^T = S^T (scale Q e^G)^T
+        auto issue_mma1 = [&](int64_t ch) {
+            unsigned char* st = sm + (ch & 1) * STAGE_BYTES;
             fence_after_sync();
-            // O^T += U^T Aqk^T (N = 64) ; S^T += U^T (K e^{Gl - G}) (N = 128)
-            const uint32_t idO = make_idesc_bf16(128, 64, false, true);
-            const uint32_t idS = make_idesc_bf16(128, 128, false, true);
+            if constexpr (kV) {
+                const uint32_t id0 = make_idesc_bf16(128, 64, true, false);
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-                const uint64_t ad = make_desc(smem_u32(sm + S_UBF + ks * 32), 16, 1024);
-                if constexpr (kOut)
-                    mma_bf16(tO(ch), ad, make_desc(smem_u32(st + IMG_B2 + ks * 2048), 8192, 1024), idO, 1u);
-                mma_bf16(tS, ad, make_desc(smem_u32(st + IMG_B2 + 8192 + ks * 2048), 8192, 1024), idS, 1u);
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tU, make_desc(smem_u32(st + STAGE_V + ks * 2048), 8192, 1024),
+                             make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
             }
-            commit(&bar2);
-        }
-        ok = __syncthreads_and(mbar_wait(&bar2, ph, err, 5) ? 1 : 0);
-        fence_after_sync();
-        if (!ok) break;
-
-        // the stage is free again: prefetch chunk ch + 2 into it
-        if (ch + 2 < nch) {
-            if (tid == 0) load_stage(ch + 2, s);
-            pending[s] = true;
-        }
-        const float* gam_next = nullptr;
-        if (!last) {
-            ok = __syncthreads_and(mbar_wait(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 4) ? 1 : 0);
-            if (!ok) break;
-            pending[s ^ 1] = false;
-            gam_next = reinterpret_cast<const float*>(sm + (s ^ 1) * STAGE_BYTES + IMG_GAM);
-        }
-
-        // next entry state: bf16 operand copy, then scaled by the next chunk's decay
-        {
-            float f[4][16];
+            const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) tmem_ld16(tS + lane + 64 * half + 16 * cb, f[cb]);
-            tmem_wait_ld();
-            if (last) {
-                if (hTp)
+            for (int ks = 0; ks < 8; ++ks) {
+                const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
+                mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1,
+                         (kV || ks > 0) ? 1u : 0u);
+            }
+            commit(&bar1);
+            if constexpr (kOut) {
+                const uint32_t to = tO(ch);
 #pragma unroll
-                    for (int cb = 0; cb < 4; ++cb)
-#pragma unroll
-                        for (int x = 0; x < 16; ++x) hTp[(64 * half + 16 * cb + x) * D + j] = f[cb][x];
-            } else {
-                unsigned char* dst = sm + S_SBF + half * 16384;
-#pragma unroll
-                for (int cb = 0; cb < 4; ++cb) {
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f[cb]);
-                    *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f[cb] + 8);
-                    float g8[16];
-                    ld8f(gam_next + 64 * half + 16 * cb, g8);
-                    ld8f(gam_next + 64 * half + 16 * cb + 8, g8 + 8);
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) f[cb][x] *= g8[x];
-                    tmem_st16(tS + lane + 64 * half + 16 * cb, f[cb]);
+                for (int ks = 0; ks < 8; ++ks) {
+                    const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
+                    mma_bf16(to, ad, make_desc(smem_u32(st + IMG_QG + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1, ks > 0);
                 }
+            }
+        };
+        ok = wait_all(&sready, 0, 6) && wait_stage(0);               // entry state staged
+        if (ok && l == 0) issue_mma1(0);
+        __syncwarp();
+        for (int64_t ch = 0; ok && ch < nch; ++ch) {
+            const int s = (int)(ch & 1);
+            unsigned char* st = sm + s * STAGE_BYTES;
+            const uint32_t ph = (uint32_t)(ch & 1);
+            if (!(ok = wait_all(&uready, ph, 6))) break;               // U^T staged
+            if (l == 0) {
+                fence_after_sync();
+                // S^T += U^T (K e^{Gl - G}) (N = 128; commit: bar2), then O^T += U^T Aqk^T
+                // (N = 64); barO covers all MMAs of this chunk
+                const uint32_t idO = make_idesc_bf16(128, 64, false, true);
+                const uint32_t idS = make_idesc_bf16(128, 128, false, true);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tS, make_desc(smem_u32(sm + S_UBF + ks * 32), 16, 1024),
+                             make_desc(smem_u32(st + IMG_B2 + 8192 + ks * 2048), 8192, 1024), idS, 1u);
+                commit(&bar2);
+                if constexpr (kOut) {
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tO(ch), make_desc(smem_u32(sm + S_UBF + ks * 32), 16, 1024),
+                                 make_desc(smem_u32(st + IMG_B2 + ks * 2048), 8192, 1024), idO, 1u);
+                }
+                commit(&barO);
+            }
+            __syncwarp();
+            if (ch + 2 < nch) {                                        // the stage takes chunk ch + 2
+                if (!(ok = wait_all(&barO, ph, 5))) break;
+                if (l == 0) load_stage(ch + 2, s);
+                __syncwarp();
+                ++issued[s];
+            }
+            if (ch + 1 < nch) {                                        // next state staged
+                if (!(ok = wait_all(&sready, (uint32_t)((ch + 1) & 1), 6) && wait_stage(s ^ 1))) break;
+                if (l == 0) issue_mma1(ch + 1);
+                __syncwarp();
+            }
+        }
+        if (!ok && l == 0)                                             // drain this CTA's copies
+            for (int s = 0; s < 2; ++s)
+                while (seen[s] < issued[s]) {
+                    mbar_wait(&full[s], seen[s] & 1, nullptr, 0, 200);
+                    ++seen[s];
+                }
+        __syncwarp();
+    } else if (worker) {
+        // every wait of the workers goes through one AND-barrier, so they leave together
+        ok = bar_and_named(1, 256, mbar_wait(&full[0], 0, err, 4));
+        // entry state: bf16 copy (operand) and gamma_0-scaled fp32 in TMEM; this thread owns
+        // columns 64*half .. +63 of row j of S^T
+        if (ok) {
+            const float* gam = reinterpret_cast<const float*>(sm + IMG_GAM);
+            unsigned char* dst = sm + S_SBF + half * 16384;
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                const int c0 = 64 * half + 16 * cb;
+                float f[16];
+#pragma unroll
+                for (int x = 0; x < 16; ++x) f[x] = s_init(c0 + x);
+                *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f);
+                *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f + 8);
+#pragma unroll
+                for (int x = 0; x < 16; ++x) f[x] *= gam[c0 + x];
+                tmem_st16(tS + lane + c0, f);
+            }
+            tmem_wait_st();
+        }
+        warp_arrive(&sready);
+        for (int64_t ch = 0; ok && ch < nch; ++ch) {
+            const int s = (int)(ch & 1);
+            const int64_t t0 = bos + ch * C;
+            const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+            const uint32_t ph = (uint32_t)(ch & 1);
+            const bool last = (ch + 1 == nch);
+
+            // U^T (fp32, TMEM) -> bf16 operand rows; this thread: tokens 32*half .. +31.  The
+            // worker barrier also keeps the previous chunk's output copy-out (same buffer) ahead.
+            if constexpr (kOut) {
+                if (tid == 0) tma::bulk_wait_read();     // the previous chunk's output store
+            }
+            if (!(ok = bar_and_named(1, 256, mbar_wait(&bar1, ph, err, 5)))) break;
+            fence_after_sync();
+            {
+                float f[2][16];
+                tmem_ld16(tU + lane + 32 * half, f[0]);
+                tmem_ld16(tU + lane + 32 * half + 16, f[1]);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 2; ++x) {
+                    const int c = 32 * half + 16 * x;
+                    *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, c)) = pack8(f[x]);
+                    *reinterpret_cast<uint4*>(sm + S_UBF + sw128_offset(j, c + 8)) = pack8(f[x] + 8);
+                }
+            }
+            warp_arrive(&uready);
+
+            // next entry state: bf16 operand copy, then scaled by the next chunk's decay (two
+            // rounds of 32 columns: register budget of nine warps per CTA)
+            if (!(ok = bar_and_named(1, 256, mbar_wait(&bar2, ph, err, 5) &&
+                                               (last || mbar_wait(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 4)))))
+                break;
+            fence_after_sync();
+            const float* gam_next =
+                last ? nullptr : reinterpret_cast<const float*>(sm + (s ^ 1) * STAGE_BYTES + IMG_GAM);
+#pragma unroll
+            for (int rd = 0; rd < 2; ++rd) {
+                float f[2][16];
+#pragma unroll
+                for (int x = 0; x < 2; ++x) tmem_ld16(tS + lane + 64 * half + 32 * rd + 16 * x, f[x]);
+                tmem_wait_ld();
+                if (last) {
+                    if (hTp)
+#pragma unroll
+                        for (int x = 0; x < 2; ++x)
+#pragma unroll
+                            for (int y = 0; y < 16; ++y) hTp[(64 * half + 32 * rd + 16 * x + y) * D + j] = f[x][y];
+                } else {
+                    unsigned char* dst = sm + S_SBF + half * 16384;
+#pragma unroll
+                    for (int x = 0; x < 2; ++x) {
+                        const int cb = 2 * rd + x;
+                        *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb)) = pack8(f[x]);
+                        *reinterpret_cast<uint4*>(dst + sw128_offset(j, 16 * cb + 8)) = pack8(f[x] + 8);
+                        float g8[16];
+                        ld8f(gam_next + 64 * half + 16 * cb, g8);
+                        ld8f(gam_next + 64 * half + 16 * cb + 8, g8 + 8);
+#pragma unroll
+                        for (int y = 0; y < 16; ++y) f[x][y] *= g8[y];
+                        tmem_st16(tS + lane + 64 * half + 16 * cb, f[x]);
+                    }
+                }
+            }
+            if (!last) {
                 tmem_wait_st();
+                warp_arrive(&sready);
             }
-        }
-        fence_smem_to_async();
-        fence_before_sync();
-        __syncthreads();
-        if (!last && tid == 0) issue_mma1(ch + 1);     // overlaps the output write below
 
-        // output rows of this chunk: tokens 32*half .. +31 of column j
-        if constexpr (kOut) {
-            float f[2][16];
-            tmem_ld16(tO(ch) + lane + 32 * half, f[0]);
-            tmem_ld16(tO(ch) + lane + 32 * half + 16, f[1]);
-            tmem_wait_ld();
-            __nv_bfloat16* op = out + (t0 * H + h) * D + j;
+            // output rows of this chunk, staged through the U^T buffer (its MMAs are complete
+            // once barO is) as a [token][dv] bf16 tile: a whole chunk leaves as one tensor store
+            // (thread 0; its source is released before the buffer's next use, at the top of the
+            // loop), a partial one row by row (the rows past it belong to the next sequence)
+            if constexpr (kOut) {
+                if (!(ok = bar_and_named(1, 256, mbar_wait(&barO, ph, err, 5)))) break;
+                fence_after_sync();
+                unsigned char* stg = sm + S_UBF;
+                float f[2][16];
+                tmem_ld16(tO(ch) + lane + 32 * half, f[0]);
+                tmem_ld16(tO(ch) + lane + 32 * half + 16, f[1]);
+                tmem_wait_ld();
 #pragma unroll
-            for (int x = 0; x < 2; ++x)
+                for (int x = 0; x < 2; ++x)
 #pragma unroll
-                for (int y = 0; y < 16; ++y) {
-                    const int t = 32 * half + 16 * x + y;
-                    if (t < len) op[(int64_t)t * H * D] = __float2bfloat16_rn(f[x][y]);
+                    for (int y = 0; y < 16; ++y) {
+                        const int t = 32 * half + 16 * x + y;
+                        *reinterpret_cast<__nv_bfloat16*>(stg + t * 256 + j * 2) = __float2bfloat16_rn(f[x][y]);
+                    }
+                fence_smem_to_async();
+                bar_sync_named(1, 256);
+                if (len == C) {
+                    if (tid == 0) {
+                        tma::store_2d(&omap, (int32_t)(h * D), (int32_t)t0, stg);
+                        tma::bulk_commit();
+                    }
+                } else {
+                    for (int e = tid; e < len * 16; e += 256) {
+                        const int r = e >> 4, c = e & 15;
+                        *reinterpret_cast<uint4*>(out + ((t0 + r) * H + h) * D + 8 * c) =
+                            *reinterpret_cast<const uint4*>(stg + r * 256 + c * 16);
+                    }
                 }
-        }
-        fence_before_sync();
-    }
-    if (!ok) {
-        // drain this CTA's own copies in flight before its shared memory goes away
-        for (int s = 0; s < 2; ++s)
-            if (pending[s]) {
-                mbar_wait(&full[s], 0, nullptr, 0, 200);
-                mbar_wait(&full[s], 1, nullptr, 0, 200);
             }
+            fence_before_sync();
+        }
     }
+    if (kOut && tid == 0) tma::bulk_wait_all();      // the last output store
     fence_before_sync();
     __syncthreads();
     if (w == 0) tmem_dealloc(tmem, 512);
@@ -1232,6 +1320,11 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
     else if ((e = make_tensor_map_2d(&maps.g, a.log_alpha, false, cols, rows, cols * 4, 32, 64, true)))
         return e;
     if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
+    // out as [tokens][H * D] bf16, boxes of one head's 128 columns x 64 tokens, unswizzled
+    // (absent when no walk writes outputs: the segment-map entry point)
+    CUtensorMap omap;
+    memset(&omap, 0, sizeof(omap));
+    if (a.out && (e = make_tensor_map_2d(&omap, a.out, true, cols, rows, cols * 2, tc::D, 64, false))) return e;
 
     auto launch_prep = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
         if (a.si.chunks_upper <= 0) return cudaSuccess;
@@ -1257,10 +1350,10 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         LaunchScope scope(s, K_STATE_TC);
         if (a.h0)
             tc::chunk_state_tc_kernel<true, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
+                w, vmap, omap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
         else
             tc::chunk_state_tc_kernel<false, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
+                w, vmap, omap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
         return cudaGetLastError();
     };
     // one walk over every segment of the plan (grid: segment bound x heads)
@@ -1272,13 +1365,13 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         __nv_bfloat16* o = (__nv_bfloat16*)a.out;
         if (mode == tc::WALK_VALUE)
             tc::chunk_state_tc_kernel<false, tc::WALK_VALUE><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+                w, vmap, omap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
         else if (mode == tc::WALK_MAP)
             tc::chunk_state_tc_kernel<false, tc::WALK_MAP><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+                w, vmap, omap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
         else
             tc::chunk_state_tc_kernel<false, tc::WALK_FINAL><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, nullptr, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+                w, vmap, omap, nullptr, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
         return cudaGetLastError();
     };
 

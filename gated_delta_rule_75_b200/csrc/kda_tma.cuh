@@ -34,6 +34,25 @@ __device__ __forceinline__ void load_bulk(void* dst_smem, const void* src, uint3
         : "memory");
 }
 
+// 2-D tiled store of a box from shared memory to (x, y) of the tensor; rows past the tensor's
+// last row are not written.  Completion is tracked by bulk groups (commit / wait below).
+__device__ __forceinline__ void store_2d(const CUtensorMap* map, int32_t x, int32_t y, const void* src_smem)
+{
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];"
+                 :
+                 : "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y),
+                   "r"(static_cast<uint32_t>(__cvta_generic_to_shared(src_smem)))
+                 : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+
+// Wait until this thread's committed bulk stores have read their shared-memory source.
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// Wait until this thread's committed bulk stores are complete.
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
 // Arm `bar` (arrival count 1) for `bytes` of incoming transfers.
 __device__ __forceinline__ void expect_tx(uint64_t* bar, uint32_t bytes)
 {

@@ -79,6 +79,13 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64
         : "memory");
 }
 
+// One arrival on `bar` (release at CTA scope: this thread's earlier writes are visible to a
+// thread that observes the phase complete).
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar)
+{
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Arrive once on `bar` when every tcgen05.mma this thread issued so far completes.
 __device__ __forceinline__ void commit(uint64_t* bar)
 {
