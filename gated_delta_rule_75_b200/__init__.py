@@ -84,6 +84,8 @@ def _load():
     lib.kda_debug_prep_image.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ctypes.c_float,
                                          ctypes.c_int, vp]
     lib.kda_debug_prep_image.restype = ctypes.c_int
+    lib.kda_debug_bounded_wait.argtypes = [ctypes.c_int32, vp, vp]
+    lib.kda_debug_bounded_wait.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -399,6 +401,16 @@ def gdn_chunk_bwd(q, k, v, log_a, beta, scale, dout, h0=None, dhT=None, cu_seqle
 
 
 IMAGE_BYTES = 66560   # one (chunk, head) operand image of the tensor-core prefill
+
+
+def debug_bounded_wait(polls, device="cuda"):
+    """Self-test (C ABI ``kda_debug_bounded_wait``): a device wait on a barrier that
+    nothing completes, given up after ``polls`` polls.  Returns the status code
+    (KDA_ERR_TIMEOUT expected) and the error word the kernel wrote."""
+    dev = torch.device(device)
+    word = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = _load().kda_debug_bounded_wait(int(polls), _ptr(word), _stream(dev))
+    return st, int(word.item())
 
 
 def debug_prep_image(q, k, log_alpha, beta, scale, gate_scalar=False):

@@ -280,9 +280,14 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
                            cudaStream_t st);
 
 // Device error word bits (workspace header): malformed cu_seqlens, and bounded
-// waits that gave up in the tensor-core kernels.
+// waits that gave up in the tensor-core kernels (bit 1: input copies of the prep;
+// 2, 3: its MMAs; 4: state-walk stage copies; 5: state-walk MMAs; 6: the state
+// walk's worker/issuer hand-offs).
 constexpr int kErrSeqlens = 1 << 0;
-constexpr int kErrTimeoutMask = 0x3e;
+constexpr int kErrTimeoutMask = 0x7e;
+
+// Self-test of the bounded mbarrier wait (kda_selftest.cu).
+cudaError_t launch_bounded_wait_selftest(int* err, uint32_t polls, cudaStream_t st);
 
 // kda_seqinfo.cu.  With seg_off set, also the first segment of each sequence
 // for segments of seg_len chunks (at least one per sequence), capped at seg_cap.

@@ -387,6 +387,19 @@ KDA_API kda_status_t kda_debug_prep_image(const void* q, const void* k, const fl
                                           int64_t H, float scale, int gate_scalar,
                                           cudaStream_t stream);
 
+/*
+ * kda_debug_bounded_wait -- self-test, not part of the method: one CTA waits on
+ * an mbarrier that nothing completes, with the same bounded wait the library's
+ * kernels use on their copies, MMAs and warp hand-offs, giving up after `polls`
+ * suspended polls (each at most ~0.1 ms).  It then sets its bit in `err_word`
+ * (device, caller-owned, 4-byte aligned; zeroed first) and returns with nothing
+ * in flight.  Synchronises `stream`.  Returns KDA_ERR_TIMEOUT when the wait gave
+ * up (the expected outcome), KDA_OK otherwise, KDA_ERR_INVALID_ARG for polls
+ * outside [1, 20000] or a bad pointer.  Lets the tests check that a wait that
+ * runs out is reported and leaves the context usable.
+ */
+KDA_API kda_status_t kda_debug_bounded_wait(int32_t polls, int32_t* err_word, cudaStream_t stream);
+
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char* kda_status_string(kda_status_t status);
 

@@ -102,3 +102,9 @@ def test_python_binding_checks_shapes_on_host():
         kda.chunk_fwd(q, q, q, q, torch.zeros(1, 8, 3), 0.1)
     with pytest.raises(TypeError):
         kda.chunk_fwd(q.double(), q.double(), q.double(), q, torch.zeros(1, 8, 2), 0.1)
+
+
+def test_bounded_wait_selftest_argument_errors(lib):
+    import gated_delta_rule_75_b200 as kda
+    for polls, word in ((0, FAKE), (20001, FAKE), (10, None), (10, FAKE + 2)):
+        assert lib.kda_debug_bounded_wait(polls, word, None) == kda.KDA_ERR_INVALID_ARG
