@@ -1056,7 +1056,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         // the issuer's warp: every lane takes the same branches (the waits' outcomes are shared
         // with __all_sync), lane 0 issues
         auto wait_all = [&](uint64_t* b, uint32_t parity, int bit) -> bool {
-            return __all_sync(0xffffffffu, mbar_wait(b, parity, err, bit) ? 1 : 0) != 0;
+            return __all_sync(0xffffffffu, mbar_wait_spin(b, parity, err, bit) ? 1 : 0) != 0;
         };
         // stage copies issued and waited for per stage (for the drain after an error)
         uint32_t issued[2] = {1u, nch > 1 ? 1u : 0u}, seen[2] = {0u, 0u};
@@ -1142,7 +1142,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
         __syncwarp();
     } else if (worker) {
         // every wait of the workers goes through one AND-barrier, so they leave together
-        ok = bar_and_named(1, 256, mbar_wait(&full[0], 0, err, 4));
+        ok = bar_and_named(1, 256, mbar_wait_spin(&full[0], 0, err, 4));
         // entry state: bf16 copy (operand) and gamma_0-scaled fp32 in TMEM; this thread owns
         // columns 64*half .. +63 of row j of S^T
         if (ok) {
@@ -1175,7 +1175,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             if constexpr (kOut) {
                 if (tid == 0) tma::bulk_wait_read();     // the previous chunk's output store
             }
-            if (!(ok = bar_and_named(1, 256, mbar_wait(&bar1, ph, err, 5)))) break;
+            if (!(ok = bar_and_named(1, 256, mbar_wait_spin(&bar1, ph, err, 5)))) break;
             fence_after_sync();
             {
                 float f[2][16];
@@ -1193,8 +1193,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 
             // next entry state: bf16 operand copy, then scaled by the next chunk's decay (two
             // rounds of 32 columns: register budget of nine warps per CTA)
-            if (!(ok = bar_and_named(1, 256, mbar_wait(&bar2, ph, err, 5) &&
-                                               (last || mbar_wait(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 4)))))
+            if (!(ok = bar_and_named(1, 256, mbar_wait_spin(&bar2, ph, err, 5) &&
+                                               (last || mbar_wait_spin(&full[s ^ 1], (uint32_t)(((ch + 1) >> 1) & 1), err, 4)))))
                 break;
             fence_after_sync();
             const float* gam_next =
@@ -1237,7 +1237,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             // (thread 0; its source is released before the buffer's next use, at the top of the
             // loop), a partial one row by row (the rows past it belong to the next sequence)
             if constexpr (kOut) {
-                if (!(ok = bar_and_named(1, 256, mbar_wait(&barO, ph, err, 5)))) break;
+                if (!(ok = bar_and_named(1, 256, mbar_wait_spin(&barO, ph, err, 5)))) break;
                 fence_after_sync();
                 unsigned char* stg = sm + S_UBF;
                 float f[2][16];

@@ -1,9 +1,10 @@
-// Self-test of the bounded wait that every kernel of this library uses on its
+// Self-test of the two bounded waits the kernels of this library use on their
 // mbarriers (TMA copies, tensor-core MMAs, hand-offs between warps): one CTA waits
-// on a barrier that nothing ever completes.  Thread 0 gives up after `polls`
-// suspended polls, sets its bit in the error word, and the CTA returns with no
-// copy or MMA in flight, so the context stays usable.  Nothing here faults, traps
-// or spins without a limit.
+// on a barrier that nothing ever completes, first with the suspended poll (given up
+// after `polls` polls; error bit 1), then with the spinning poll bounded by elapsed
+// cycles (`polls` x 200000 cycles, about 0.1 ms per poll; error bit 2).  The CTA
+// returns with no copy or MMA in flight, so the context stays usable.  Nothing here
+// faults, traps or spins without a limit.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 #include "kda_umma.cuh"
@@ -19,7 +20,10 @@ __global__ void bounded_wait_selftest_kernel(int* __restrict__ err, uint32_t pol
     }
     __syncthreads();
     int gave_up = 0;
-    if (threadIdx.x == 0) gave_up = umma::mbar_wait(&bar, 0, err, 1, polls) ? 0 : 1;
+    if (threadIdx.x == 0) {
+        gave_up = umma::mbar_wait(&bar, 0, err, 1, polls) ? 0 : 1;
+        gave_up += umma::mbar_wait_spin(&bar, 0, err, 2, (long long)polls * 200000LL) ? 0 : 1;
+    }
     __syncthreads_or(gave_up);
 }
 

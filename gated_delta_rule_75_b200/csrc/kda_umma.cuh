@@ -153,14 +153,41 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* e
     return false;
 }
 
-// Block-wide wait: thread 0 polls `bar` (phase `parity`) with the iteration
-// limit of mbar_wait, the rest of the block sleeps in the barrier, and every
+// The same wait, polled without a suspend hint (each try returns after a short,
+// implementation-defined time) for the low-latency hand-offs of the state walk, where
+// a suspended thread's wake-up would sit on the critical path.  Bounded by elapsed
+// cycles (`limit_cycles`, about 2 s at the B200's clock by default); on a timeout it
+// sets bit `err_bit` in *err and returns false.
+__device__ __forceinline__ bool mbar_wait_spin(uint64_t* bar, uint32_t parity, int* err, int err_bit,
+                                               long long limit_cycles = 4000000000LL)
+{
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t"
+            ".reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.b32 %0, 1, 0, p;\n\t"
+            "}\n"
+            : "=r"(ok)
+            : "r"(smem_u32(bar)), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > limit_cycles) break;
+    }
+    if (err) atomicOr(err, 1 << err_bit);
+    return false;
+}
+
+// Block-wide wait: thread 0 polls `bar` (phase `parity`) without a suspend hint,
+// bounded as mbar_wait_spin, the rest of the block sleeps in the barrier, and every
 // thread gets the same outcome.  The barrier orders the observed completion
 // (and the data it guards) before everything the block does next.
 __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, int* err, int err_bit)
 {
     int ok = 1;
-    if (threadIdx.x == 0) ok = mbar_wait(bar, parity, err, err_bit) ? 1 : 0;
+    if (threadIdx.x == 0) ok = mbar_wait_spin(bar, parity, err, err_bit) ? 1 : 0;
     return __syncthreads_or(ok ? 0 : 1) == 0;
 }
 

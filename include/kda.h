@@ -389,11 +389,12 @@ KDA_API kda_status_t kda_debug_prep_image(const void* q, const void* k, const fl
 
 /*
  * kda_debug_bounded_wait -- self-test, not part of the method: one CTA waits on
- * an mbarrier that nothing completes, with the same bounded wait the library's
- * kernels use on their copies, MMAs and warp hand-offs, giving up after `polls`
- * suspended polls (each at most ~0.1 ms).  It then sets its bit in `err_word`
- * (device, caller-owned, 4-byte aligned; zeroed first) and returns with nothing
- * in flight.  Synchronises `stream`.  Returns KDA_ERR_TIMEOUT when the wait gave
+ * an mbarrier that nothing completes, with the two bounded waits the library's
+ * kernels use on their copies, MMAs and warp hand-offs: `polls` suspended polls
+ * (each at most ~0.1 ms; bit 1 of `err_word` when it gives up), then a spinning
+ * poll bounded at `polls` x 200000 clock cycles (bit 2).  `err_word` is device
+ * memory, caller-owned, 4-byte aligned, zeroed first; the CTA returns with
+ * nothing in flight.  Synchronises `stream`.  Returns KDA_ERR_TIMEOUT when the wait gave
  * up (the expected outcome), KDA_OK otherwise, KDA_ERR_INVALID_ARG for polls
  * outside [1, 20000] or a bad pointer.  Lets the tests check that a wait that
  * runs out is reported and leaves the context usable.
