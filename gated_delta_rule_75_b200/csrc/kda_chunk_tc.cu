@@ -240,10 +240,13 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
             float tcol[16];
 #pragma unroll
             for (int r = 0; r < 16; ++r) {
-                float acc = 0.f;
+                float acc0 = 0.f, acc1 = 0.f;            // two chains: half the dependent adds
 #pragma unroll
-                for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
-                tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -acc);
+                for (int m = 0; m < r; ++m) {
+                    if (m & 1) acc1 += sA[(o + r) * AP + o + m] * tcol[m];
+                    else acc0 += sA[(o + r) * AP + o + m] * tcol[m];
+                }
+                tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -(acc0 + acc1));
             }
 #pragma unroll
             for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
@@ -286,15 +289,20 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
         __syncthreads();
         side_ok = true;
     }
-    // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace
+    // T' = T diag(beta) in bf16: K-major image (rows i, K = j), in smem and in the workspace.
+    // Blocks above the diagonal are zero (never written in sT); the diagonal blocks already
+    // hold zeros above their diagonal, and the blocks below are complete.
     for (int e = tid; e < C * 8; e += PT) {
         const int i = e >> 3, cb = e & 7;
-        float f[8], bt[8];
-        ld8f(sT + i * AP + 8 * cb, f);
-        ld8f(sB + 8 * cb, bt);
+        uint4 u = make_uint4(0, 0, 0, 0);
+        if ((cb >> 1) <= (i >> 4)) {
+            float f[8], bt[8];
+            ld8f(sT + i * AP + 8 * cb, f);
+            ld8f(sB + 8 * cb, bt);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x <= i) ? f[x] * bt[x] : 0.f;
-        const uint4 u = pack8(f);
+            for (int x = 0; x < 8; ++x) f[x] *= bt[x];
+            u = pack8(f);
+        }
         *reinterpret_cast<uint4*>(sm + P_Q + sw128_offset(i, 8 * cb)) = u;
         *reinterpret_cast<uint4*>(img + IMG_T + sw128_offset(i, 8 * cb)) = u;
     }
