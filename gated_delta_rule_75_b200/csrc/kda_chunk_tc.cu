@@ -56,7 +56,7 @@ constexpr int D = 128;     // dk = dv = 128
 constexpr float kLog2e = 1.4426950408889634f;
 
 // Operand image of one (chunk, head), byte offsets (all 1024-aligned).
-constexpr uint32_t IMG_W = 0;          // -W          K-major B: 64 token rows x 128 ch (2 K-blocks)
+constexpr uint32_t IMG_W = 0;          // -W^T        MN-major B: 128 channel rows x 64 tokens
 constexpr uint32_t IMG_QG = 16384;     // scale Q e^G K-major B: same shape
 constexpr uint32_t IMG_B2 = 32768;     // MN-major B, K = 64 token rows: [Aqk^T | K e^{Gl-G}] (3 x 64)
 constexpr uint32_t IMG_T = 57344;      // T' = T diag(beta), K-major: 64 rows x 64
@@ -310,14 +310,16 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
     fence_before_sync();
     __syncthreads();
 
-    // ---- (b3) W = T' (K e^G): M = 64 tokens, N = 128 channels, K = 64 tokens
+    // ---- (b3) -W^T = -(K e^G)^T T'^T: M = 128 channels (every TMEM lane holds a row),
+    // N = 64 tokens, K = 64 tokens; stored as the MN-major [channel][token] tile the state
+    // kernel reads as its B operand
     if (tid == 0) {
         fence_after_sync();
-        const uint32_t idesc = make_idesc_bf16(64, 128, false, true, true);   // -T' (K e^G)
+        const uint32_t idesc = make_idesc_bf16(128, 64, true, false, true);   // -(K e^G)^T T'^T
 #pragma unroll
         for (int ks = 0; ks < 4; ++ks) {
-            const uint64_t ad = make_desc(smem_u32(sm + P_Q + ks * 32), 16, 1024);
-            const uint64_t bd = make_desc(smem_u32(sm + P_K + ks * 2048), 8192, 1024);
+            const uint64_t ad = make_desc(smem_u32(sm + P_K + ks * 2048), 8192, 1024);   // MN-major
+            const uint64_t bd = make_desc(smem_u32(sm + P_Q + ks * 32), 16, 1024);      // K-major
             mma_bf16(tmem, ad, bd, idesc, ks > 0 ? 1u : 0u);
         }
         commit(bar);
@@ -326,19 +328,17 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
     fence_after_sync();
     if (ok) {
         after_mma();                               // P_Q and P_K are free from here on
-        const int i = 16 * sp + l, half = w >> 2;
-        float f[4][16];
-#pragma unroll
-        for (int cb = 0; cb < 4; ++cb)
-            tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 64 * half + 16 * cb, f[cb]);
+        // warp w: channel 32 (w % 4) + lane, tokens 32 (w / 4) .. +31
+        const int c = 32 * sp + l, half = w >> 2;
+        float f[2][16];
+        tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * half, f[0]);
+        tmem_ld16(tmem + ((uint32_t)(32 * sp) << 16) + 32 * half + 16, f[1]);
         tmem_wait_ld();
-        if (l < 16) {
-            unsigned char* dst = img + IMG_W + half * 8192;
+        unsigned char* dst = img + IMG_W;
 #pragma unroll
-            for (int cb = 0; cb < 4; ++cb) {
-                *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb)) = pack8(f[cb]);
-                *reinterpret_cast<uint4*>(dst + sw128_offset(i, 16 * cb + 8)) = pack8(f[cb] + 8);
-            }
+        for (int x = 0; x < 2; ++x) {
+            *reinterpret_cast<uint4*>(dst + sw128_offset(c, 32 * half + 16 * x)) = pack8(f[x]);
+            *reinterpret_cast<uint4*>(dst + sw128_offset(c, 32 * half + 16 * x + 8)) = pack8(f[x] + 8);
         }
     }
     return ok;
@@ -1085,10 +1085,11 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
                              make_desc(smem_u32(st + IMG_T + ks * 32), 16, 1024), id0, ks > 0);
             }
             const uint32_t id1 = make_idesc_bf16(128, 64, false, false);
+            const uint32_t idW = make_idesc_bf16(128, 64, false, true);    // -W^T: MN-major B
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks) {
                 const uint64_t ad = make_desc(smem_u32(sm + S_SBF + (ks >> 2) * 16384 + (ks & 3) * 32), 16, 1024);
-                mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + (ks >> 2) * 8192 + (ks & 3) * 32), 16, 1024), id1,
+                mma_bf16(tU, ad, make_desc(smem_u32(st + IMG_W + ks * 2048), 8192, 1024), idW,
                          (kV || ks > 0) ? 1u : 0u);
             }
             commit(&bar1);

@@ -377,7 +377,8 @@ KDA_API kda_status_t kda_affine_prefix(const float* maps, const float* offs, con
  * operand images in `image` (device, caller-owned, B * ceil(T / 64) * H blocks of
  * 66560 bytes, block (chunk c of sequence n, head h) at index (n * ceil(T/64) + c)
  * * H + h), in the 128-byte-swizzled bf16 layout the state kernel reads:
- * -W | scale Q e^G | [Aqk^T | K e^{G_last - G}] | T diag(beta) | e^{G_last} (fp32).
+ * -W^T ([channel][token]) | scale Q e^G | [Aqk^T | K e^{G_last - G}] | T diag(beta) |
+ * e^{G_last} (fp32).
  * log_alpha is [B, T, H, dk], or [B, T, H] with gate_scalar != 0 (Gated DeltaNet
  * prep).  Lets the tests check the intra-chunk kernels against the fp64 chunk
  * equations one quantity at a time.

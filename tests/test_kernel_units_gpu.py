@@ -43,7 +43,7 @@ def decode(img):
     j = np.arange(C)[:, None]
     i = np.arange(C)[None, :]
     return {
-        "W": -_bf16_at(img, IMG_W + two_blocks),
+        "W": -_bf16_at(img, IMG_W + np.vectorize(_sw)(c, r)),           # -W^T: [channel][token]
         "QG": _bf16_at(img, IMG_QG + two_blocks),
         "AqkT": _bf16_at(img, IMG_B2 + np.vectorize(_sw)(j, i)),          # [j][i] = Aqk[i][j]
         "KGl": _bf16_at(img, IMG_B2 + 8192 + two_blocks),
