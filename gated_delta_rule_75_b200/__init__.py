@@ -81,8 +81,7 @@ def _load():
     lib.kda_chunk_bwd.restype = ctypes.c_int
     lib.kda_gdn_chunk_bwd.argtypes = lib.kda_chunk_bwd.argtypes
     lib.kda_gdn_chunk_bwd.restype = ctypes.c_int
-    lib.kda_debug_prep_image.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ctypes.c_float,
-                                         ctypes.c_int, vp]
+    lib.kda_debug_prep_image.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, ctypes.c_int, vp]
     lib.kda_debug_prep_image.restype = ctypes.c_int
     lib.kda_debug_bounded_wait.argtypes = [ctypes.c_int32, vp, vp]
     lib.kda_debug_bounded_wait.restype = ctypes.c_int
@@ -413,9 +412,10 @@ def debug_bounded_wait(polls, device="cuda"):
     return st, int(word.item())
 
 
-def debug_prep_image(q, k, log_alpha, beta, scale, gate_scalar=False):
+def debug_prep_image(q, k, log_alpha, beta, gate_scalar=False):
     """Test hook (C ABI ``kda_debug_prep_image``): the tensor-core prep kernel's
-    operand images of a fixed-length bf16 batch, uint8 [B*ceil(T/64)*H, 66560]."""
+    operand images of a fixed-length bf16 batch, uint8 [B*ceil(T/64)*H, 66560]
+    (Q e^G and Aqk without the attention scale)."""
     B, T, H, dk = q.shape
     dev = q.device
     _check(q, "q", torch.bfloat16, (B, T, H, 128), dev)
@@ -425,7 +425,7 @@ def debug_prep_image(q, k, log_alpha, beta, scale, gate_scalar=False):
     n = B * ((T + 63) // 64) * H
     image = torch.zeros((n, IMAGE_BYTES), dtype=torch.uint8, device=dev)
     st = _load().kda_debug_prep_image(_ptr(q), _ptr(k), _ptr(log_alpha), _ptr(beta), _ptr(image),
-                                      B, T, H, float(scale), 1 if gate_scalar else 0, _stream(dev))
+                                      B, T, H, 1 if gate_scalar else 0, _stream(dev))
     if st != KDA_OK:
         raise KDAError(st, "kda_debug_prep_image")
     return image

@@ -667,7 +667,7 @@ extern "C" {
 
 kda_status_t kda_debug_prep_image(const void* q, const void* k, const float* log_alpha,
                                   const float* beta, void* image, int64_t B, int64_t T, int64_t H,
-                                  float scale, int gate_scalar, cudaStream_t stream)
+                                  int gate_scalar, cudaStream_t stream)
 {
     if (B < 0 || T < 0 || H < 0 || H > 65535) return KDA_ERR_INVALID_ARG;
     if (B * T >= (int64_t(1) << 31)) return KDA_ERR_UNSUPPORTED;
@@ -682,7 +682,7 @@ kda_status_t kda_debug_prep_image(const void* q, const void* k, const float* log
     std::memset(&a, 0, sizeof(a));
     a.q = q; a.k = k; a.v = k;                 // v is not read by the prep
     a.log_alpha = log_alpha; a.beta = beta; a.H = H; a.dk = 128; a.dv = 128;
-    a.scale = scale; a.io = KDA_IO_BF16; a.gate_scalar = gate_scalar != 0; a.tc_what = 2;
+    a.scale = 1.f; a.io = KDA_IO_BF16; a.gate_scalar = gate_scalar != 0; a.tc_what = 2;
     SeqInfo& si = a.si;
     si.N = B;
     si.T_seq = T;

@@ -8,8 +8,8 @@
 // T' = (I + A)^{-1} diag(beta):
 //
 //   A_ij   = beta_i sum_c k_ic k_jc e^{G_ic - G_jc}   (i > j)
-//   Aqk_ij = scale  sum_c q_ic k_jc e^{G_ic - G_jc}   (i >= j)
-//   W = T' (K e^G),  U = T' V - W S,  O = scale (Q e^G) S + Aqk U,
+//   Aqk_ij = sum_c q_ic k_jc e^{G_ic - G_jc}          (i >= j)
+//   W = T' (K e^G),  U = T' V - W S,  O = scale ((Q e^G) S + Aqk U),
 //   S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U
 //
 // Kernel `chunk_prep_tc` (one CTA per (chunk, head), steps a and b): TMA loads
@@ -29,7 +29,7 @@
 //   a bf16 copy in shared memory as the MMA operand; each chunk's image (bulk
 //   copy) and its v tile (TMA) are double-buffered.  Per chunk:
 //     U^T = V^T T'^T + S^T (-W)^T             (fp32 in TMEM)
-//     O^T = S^T (scale Q e^G)^T
+//     O^T = S^T (Q e^G)^T
 //     S^T += U^T (K e^{G_last - G}),  O^T += U^T Aqk^T
 //   then S^T is copied to bf16 for the next chunk and scaled by the next
 //   chunk's e^{G_last} in TMEM, and O leaves through a shared-memory tile (one
@@ -57,7 +57,7 @@ constexpr float kLog2e = 1.4426950408889634f;
 
 // Operand image of one (chunk, head), byte offsets (all 1024-aligned).
 constexpr uint32_t IMG_W = 0;          // -W^T        MN-major B: 128 channel rows x 64 tokens
-constexpr uint32_t IMG_QG = 16384;     // scale Q e^G K-major B: same shape
+constexpr uint32_t IMG_QG = 16384;     // Q e^G       K-major B: 64 token rows x 128 ch (2 K-blocks)
 constexpr uint32_t IMG_B2 = 32768;     // MN-major B, K = 64 token rows: [Aqk^T | K e^{Gl-G}] (3 x 64)
 constexpr uint32_t IMG_T = 57344;      // T' = T diag(beta), K-major: 64 rows x 64
 constexpr uint32_t IMG_GAM = 65536;    // e^{G_last}, fp32 [128]
@@ -346,7 +346,7 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
 
 __global__ void __launch_bounds__(PT, 2)
 chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
-                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, int64_t hg, float scale,
+                     SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, int64_t hg,
                      unsigned char* __restrict__ ws, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
@@ -597,7 +597,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                         const float e1 = ex2(x);          // <= 1
                         const float r1 = ex2(-x);         // >= 1, at most 15 tokens of decay
                         kin[rr][j] = kk[j] * e1;
-                        qin[rr][j] = qq[j] * e1;          // `scale` is applied to Aqk and Q e^G later
+                        qin[rr][j] = qq[j] * e1;
                         kd[rr][j] = kk[j] * r1;
                     }
                     // operands of the strip MMAs first
@@ -635,19 +635,17 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                     if (hh == 1 && nxt >= 0) issue_g(nxt, t02);   // G is not read again
                 }
                 if (hh == 1 && nxt >= 0) ++g_issued;
-                // while the MMAs run: scale Q e^G, K e^{G_last - G} (image) and K e^G (in place)
+                // while the MMAs run: the image's Q e^G and K e^{G_last - G}, and K e^G (in place)
 #pragma unroll
                 for (int rr = 0; rr < 2; ++rr) {
                     const int ps = rr == 0 ? p : 3 - p;
                     const int t = 16 * ps + tr + 8 * rr;
                     const uint32_t off = hh * 8192 + sw128_offset(t, 8 * ch8);
-                    float eg[8], egl[8], egs[8], tmp[8];
+                    float eg[8], egl[8], tmp[8];
                     ld8f(egf + ps * VP + vc, eg);
                     ld8f(eglf + ps * VP + vc, egl);
 #pragma unroll
-                    for (int j = 0; j < 8; ++j) egs[j] = scale * eg[j];
-#pragma unroll
-                    for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * egs[j];
+                    for (int j = 0; j < 8; ++j) tmp[j] = qin[rr][j] * eg[j];
                     *reinterpret_cast<uint4*>(img + IMG_QG + hh * 8192 + sw128_offset(t, 8 * ch8)) = pack8(tmp);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) tmp[j] = kd[rr][j] * egl[j];
@@ -691,10 +689,10 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                     }
                     if (rel < 0) {
 #pragma unroll
-                        for (int cc = 0; cc < 16; ++cc) aq[cc] = scale * qp[x][cc];
+                        for (int cc = 0; cc < 16; ++cc) aq[cc] = qp[x][cc];
                     } else if (rel == 0) {
 #pragma unroll
-                        for (int cc = 0; cc < 16; ++cc) aq[cc] = (l <= cc) ? scale * qp[x][cc] : 0.f;
+                        for (int cc = 0; cc < 16; ++cc) aq[cc] = (l <= cc) ? qp[x][cc] : 0.f;
                     } else {
 #pragma unroll
                         for (int cc = 0; cc < 16; ++cc) aq[cc] = 0.f;
@@ -749,7 +747,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
 // With a scalar decay per token the pairwise factor e^{G_i - G_j} is the same for every
 // channel, so ("Kimi Delta Attention: la atencion lineal detras de Kimi K2 y Qwen3",
 // comparison of DeltaNet, Gated DeltaNet and KDA; the gate is per head there)
-//   A_ij = beta_i e^{G_i - G_j} (k_i . k_j),   Aqk_ij = scale e^{G_i - G_j} (q_i . k_j)
+//   A_ij = beta_i e^{G_i - G_j} (k_i . k_j),   Aqk_ij = e^{G_i - G_j} (q_i . k_j)
 // come from two plain MMAs on the loaded k and q tiles, with one exponential per (i, j) at
 // extraction and every factor <= 1; the image rows are k and q scaled per token.  No
 // per-channel operands are built, so the kernel needs 68 KB of shared memory and few
@@ -765,8 +763,7 @@ constexpr uint32_t GP_SMEM = GP_BYTES + 1024;
 __global__ void __launch_bounds__(PT, 3)
 chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
                          const float* __restrict__ log_a, SeqInfo si, int64_t H, int64_t h_base,
-                         int64_t Hg, float scale, unsigned char* __restrict__ ws,
-                         int* __restrict__ err)
+                         int64_t Hg, unsigned char* __restrict__ ws, int* __restrict__ err)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -843,7 +840,7 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
         }
         commit(&bar);
     }
-    // while the MMAs run: scale Q e^G and K e^{G_last - G} into the image, e^{G_last}
+    // while the MMAs run: Q e^G and K e^{G_last - G} into the image, e^{G_last}
     if (ok) {
         const float gl = sG[C - 1];
         for (int e = tid; e < C * 16; e += PT) {
@@ -852,7 +849,7 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
             float kk[8], qq[8], tmp[8];
             unpack8(*reinterpret_cast<const uint4*>(sm + GP_K + off), kk);
             unpack8(*reinterpret_cast<const uint4*>(sm + GP_Q + off), qq);
-            const float eqs = scale * ex2(sG[t]), egl = ex2(gl - sG[t]);
+            const float eqs = ex2(sG[t]), egl = ex2(gl - sG[t]);
 #pragma unroll
             for (int x = 0; x < 8; ++x) tmp[x] = qq[x] * eqs;
             *reinterpret_cast<uint4*>(img + IMG_QG + off) = pack8(tmp);
@@ -898,7 +895,7 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
                     const int i = ib + 16 * x + cc;
                     const float e = (i >= j) ? ex2(sG[i] - gj) : 0.f;    // <= 1
                     sA[i * AP + j] = (j < i) ? sB[i] * e * d1[x][cc] : 0.f;
-                    aq[16 * x + cc] = scale * e * d2[x][cc];
+                    aq[16 * x + cc] = e * d2[x][cc];
                 }
 #pragma unroll
             for (int m = 0; m < 4; ++m)
@@ -943,7 +940,7 @@ enum { WALK_SEQ = 0, WALK_VALUE = 1, WALK_MAP = 2, WALK_FINAL = 3 };
 template <bool kHasH0, int kMode>
 __global__ void __launch_bounds__(ST, 1)
 chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constant__ CUtensorMap vmap,
-                      const __grid_constant__ CUtensorMap omap,
+                      const __grid_constant__ CUtensorMap omap, float scale,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, SeqInfo si, int64_t H, int64_t h_base, int64_t Hg,
                       const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err,
@@ -1073,7 +1070,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
             ++seen[s];
             return true;
         };
-        // U^T = V^T T'^T + S^T (-W)^T (commit: bar1), then O^T = S^T (scale Q e^G)^T
+        // U^T = V^T T'^T + S^T (-W)^T (commit: bar1), then O^T = S^T (Q e^G)^T (the output takes
+        // `scale` when it leaves TMEM)
         auto issue_mma1 = [&](int64_t ch) {
             unsigned char* st = sm + (ch & 1) * STAGE_BYTES;
             fence_after_sync();
@@ -1258,7 +1256,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 #pragma unroll
                     for (int y = 0; y < 16; ++y) {
                         const int t = 32 * half + 16 * x + y;
-                        *reinterpret_cast<__nv_bfloat16*>(stg + t * 256 + j * 2) = __float2bfloat16_rn(f[x][y]);
+                        *reinterpret_cast<__nv_bfloat16*>(stg + t * 256 + j * 2) = __float2bfloat16_rn(scale * f[x][y]);
                     }
                 fence_smem_to_async();
                 bar_sync_named(1, 256);
@@ -1341,14 +1339,14 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         LaunchScope scope(s, K_PREP_TC);
         if (a.gate_scalar) {
             tc::chunk_prep_gdn_tc_kernel<<<gp, tc::PT, tc::GP_SMEM, s>>>(
-                maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, a.scale, w, err);
+                maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, w, err);
         } else {
             // persistent: two CTAs per SM walk the (chunk, head) items
             const int64_t items = a.si.chunks_upper * hg;
             if (items > INT32_MAX) return cudaErrorInvalidValue;   // items are 32-bit in the kernel
             const int64_t slots = 2 * device_sm_count();
             tc::chunk_prep_tc_kernel<<<(unsigned)(items < slots ? items : slots), tc::PT, tc::P_SMEM, s>>>(
-                maps, a.beta, a.si, a.H, hb, Hg, hg, a.scale, w, err);
+                maps, a.beta, a.si, a.H, hb, Hg, hg, w, err);
         }
         return cudaGetLastError();
     };
@@ -1359,10 +1357,10 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         LaunchScope scope(s, K_STATE_TC);
         if (a.h0)
             tc::chunk_state_tc_kernel<true, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
+                w, vmap, omap, a.scale, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
         else
             tc::chunk_state_tc_kernel<false, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
+                w, vmap, omap, a.scale, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
         return cudaGetLastError();
     };
     // one walk over every segment of the plan (grid: segment bound x heads)
@@ -1374,13 +1372,13 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         __nv_bfloat16* o = (__nv_bfloat16*)a.out;
         if (mode == tc::WALK_VALUE)
             tc::chunk_state_tc_kernel<false, tc::WALK_VALUE><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+                w, vmap, omap, a.scale, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
         else if (mode == tc::WALK_MAP)
             tc::chunk_state_tc_kernel<false, tc::WALK_MAP><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+                w, vmap, omap, a.scale, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
         else
             tc::chunk_state_tc_kernel<false, tc::WALK_FINAL><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, nullptr, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+                w, vmap, omap, a.scale, nullptr, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
         return cudaGetLastError();
     };
 

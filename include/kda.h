@@ -377,16 +377,15 @@ KDA_API kda_status_t kda_affine_prefix(const float* maps, const float* offs, con
  * operand images in `image` (device, caller-owned, B * ceil(T / 64) * H blocks of
  * 66560 bytes, block (chunk c of sequence n, head h) at index (n * ceil(T/64) + c)
  * * H + h), in the 128-byte-swizzled bf16 layout the state kernel reads:
- * -W^T ([channel][token]) | scale Q e^G | [Aqk^T | K e^{G_last - G}] | T diag(beta) |
- * e^{G_last} (fp32).
- * log_alpha is [B, T, H, dk], or [B, T, H] with gate_scalar != 0 (Gated DeltaNet
- * prep).  Lets the tests check the intra-chunk kernels against the fp64 chunk
- * equations one quantity at a time.
+ * -W^T ([channel][token]) | Q e^G | [Aqk^T | K e^{G_last - G}] | T diag(beta) |
+ * e^{G_last} (fp32).  Q e^G and Aqk carry no `scale`: the state kernel applies it
+ * to the output.  log_alpha is [B, T, H, dk], or [B, T, H] with gate_scalar != 0
+ * (Gated DeltaNet prep).  Lets the tests check the intra-chunk kernels against the
+ * fp64 chunk equations one quantity at a time.
  */
 KDA_API kda_status_t kda_debug_prep_image(const void* q, const void* k, const float* log_alpha,
                                           const float* beta, void* image, int64_t B, int64_t T,
-                                          int64_t H, float scale, int gate_scalar,
-                                          cudaStream_t stream);
+                                          int64_t H, int gate_scalar, cudaStream_t stream);
 
 /*
  * kda_debug_bounded_wait -- self-test, not part of the method: one CTA waits on

@@ -1,5 +1,5 @@
 """Per-kernel parity of the tensor-core prep (steps a and b): the operand image
-it writes for each (chunk, head) -- -W, scale Q e^G, Aqk^T, K e^{G_last - G},
+it writes for each (chunk, head) -- -W^T, Q e^G, Aqk^T, K e^{G_last - G},
 T diag(beta) and e^{G_last} -- decoded from its 128-byte-swizzled bf16 layout and
 compared quantity by quantity with the fp64 chunk equations of
 tests/test_chunk_algebra.py on the same rounded inputs; and T (I + A) = I with
@@ -64,7 +64,7 @@ def test_prep_image_matches_chunk_equations(kda, gdn):
     log_a = W.scalar_gates(cfg.B, cfg.T, cfg.H, seed=90, device="cuda") if gdn else None
     g = log_a.unsqueeze(-1).expand(*log_a.shape, 128).contiguous() if gdn else inp["log_alpha"]
     imgs = kda.debug_prep_image(inp["q"], inp["k"], log_a if gdn else inp["log_alpha"], inp["beta"],
-                                inp["scale"], gate_scalar=gdn)
+                                gate_scalar=gdn)
     torch.cuda.synchronize()
     imgs = imgs.cpu().numpy()
     h = lambda x: x.detach().cpu().double().numpy()
@@ -78,7 +78,7 @@ def test_prep_image_matches_chunk_equations(kda, gdn):
             for hd in range(cfg.H):
                 pad = lambda x: np.concatenate([x[n, t0:t0 + L, hd], np.zeros((C - L,) + x.shape[3:])])
                 ref = chunk_intra(pad(q), pad(k), np.zeros((C, 128)), pad(gg),
-                                  np.concatenate([b[n, t0:t0 + L, hd], np.zeros(C - L)]), inp["scale"])
+                                  np.concatenate([b[n, t0:t0 + L, hd], np.zeros(C - L)]), 1.0)   # the image is unscaled
                 got = decode(imgs[(n * nct + ch) * cfg.H + hd])
                 bb = np.concatenate([b[n, t0:t0 + L, hd], np.zeros(C - L)])
                 pairs = {"W": (got["W"], ref["W"]), "QG": (got["QG"], ref["QG"]),
