@@ -34,7 +34,6 @@ int64_t simt_ws_floats_per_chunk(int dk, int dv)
 template <typename T, int DK, int DV>
 static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaStream_t st)
 {
-    constexpr int C = kChunk;
     const size_t smem_prep = simt_prep_smem<DK, DV>();
     const size_t smem_state = simt_state_smem<DK, DV>();
     static std::atomic<uint64_t> attrs_done{0};

@@ -37,7 +37,7 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(kPrefixThreads)
+__global__ void __launch_bounds__(kPrefixThreads, 1)   // one CTA per SM: registers uncapped
 affine_prefix_kernel(PrefixArgs p)
 {
     extern __shared__ __align__(16) float msm[];               // 2 x [128][kMPitch]

@@ -42,13 +42,13 @@ kda_status_t kda_debug_bounded_wait(int32_t polls, int32_t* err_word, cudaStream
     if (polls < 1 || polls > 20000 || err_word == nullptr ||
         (reinterpret_cast<uintptr_t>(err_word) & 3) != 0)
         return KDA_ERR_INVALID_ARG;
-    cudaError_t e;
-    if ((e = cudaMemsetAsync(err_word, 0, sizeof(int32_t), stream))) return KDA_ERR_CUDA;
-    if ((e = kda::launch_bounded_wait_selftest(err_word, (uint32_t)polls, stream))) return KDA_ERR_CUDA;
-    int32_t flag = 0;
-    if ((e = cudaMemcpyAsync(&flag, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, stream)))
+    if (cudaMemsetAsync(err_word, 0, sizeof(int32_t), stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (kda::launch_bounded_wait_selftest(err_word, (uint32_t)polls, stream) != cudaSuccess)
         return KDA_ERR_CUDA;
-    if ((e = cudaStreamSynchronize(stream))) return KDA_ERR_CUDA;
+    int32_t flag = 0;
+    if (cudaMemcpyAsync(&flag, err_word, sizeof(int32_t), cudaMemcpyDeviceToHost, stream) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return KDA_ERR_CUDA;
     return (flag & kda::kErrTimeoutMask) ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 

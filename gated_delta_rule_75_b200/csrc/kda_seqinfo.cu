@@ -19,7 +19,7 @@
 
 namespace kda {
 
-constexpr int kScanThreads = 1024;
+constexpr int kScanThreads = 512;    // 57 registers: no spill (1024 threads cap them at 64)
 
 __global__ void __launch_bounds__(kScanThreads)
 chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total, int64_t cap,
