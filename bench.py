@@ -299,18 +299,24 @@ def run_prefill(args, ws, rank, kda, peaks):
     return res, inp, step, (out, hT)
 
 
-KERNEL_SOURCE = {"chunk_prep_tc": "kda_chunk_tc.cu", "chunk_state_tc": "kda_chunk_tc.cu",
-                 "chunk_prep_simt": "kda_chunk_simt.cu", "chunk_state_simt": "kda_chunk_simt.cu",
-                 "decode_step": "kda_decode.cu"}
+_TC_SOURCES = ("kda_chunk_tc.cu", "kda_umma.cuh", "kda_tma.cuh")
+_SIMT_SOURCES = ("kda_chunk_simt.cu", "kda_chunk_simt.cuh")
+KERNEL_SOURCE = {"chunk_prep_tc": _TC_SOURCES, "chunk_state_tc": _TC_SOURCES,
+                 "chunk_prep_gdn_tc": _TC_SOURCES,
+                 "chunk_prep_simt": _SIMT_SOURCES, "chunk_state_simt": _SIMT_SOURCES,
+                 "decode_step": ("kda_decode.cu",)}
 
 
 def kernel_source_sha(kname):
+    """SHA-256 prefix of the source files that define kernel `kname` (concatenated)."""
     import hashlib
-    f = KERNEL_SOURCE.get(kname)
-    if f is None:
+    files = KERNEL_SOURCE.get(kname)
+    if files is None:
         return None
-    path = os.path.join(ROOT, "gated_delta_rule_75_b200", "csrc", f)
-    return hashlib.sha256(open(path, "rb").read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "gated_delta_rule_75_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
 
 
 def measured_traffic(kname, workload):

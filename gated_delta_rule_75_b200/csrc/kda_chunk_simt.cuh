@@ -12,6 +12,21 @@ constexpr int kTW = 32;           // dv columns per state-walk tile
 constexpr int kSP = 36;           // row pitch of a [DK][32] state tile in shared memory:
                                   // 16-byte accesses by 8 consecutive rows hit distinct banks
 
+// 16-byte global -> shared copies that complete asynchronously (cp.async, L2 only),
+// grouped by commit and waited for per thread: every thread's own copies are done
+// after async_wait<N>() with at most N newer groups pending; a barrier after it makes
+// them visible to the block.
+__device__ __forceinline__ void async16(float* dst, const float* src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     static_cast<uint32_t>(__cvta_generic_to_shared(dst))),
+                 "l"(src)
+                 : "memory");
+}
+__device__ __forceinline__ void async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
 // acc[r] += sum_k A[(row0 + RS r) * lda + k] * B[k * LDB + lane], r < NR (A rows read as
 // 16-byte broadcasts, B columns one per lane), K a multiple of 4.
 template <int NR, int RS, int LDB>
@@ -86,7 +101,7 @@ template <int DK, int DV, bool kBwd = false>
 constexpr size_t simt_state_smem()
 {
     return sizeof(float) * (size_t)((kBwd ? 2 : 3) * kChunk * DK + (kBwd ? 0 : kChunk * kChunk) +
-                                    kChunk * kTW + DK * kSP + DK);
+                                    2 * kChunk * kTW + DK * kSP + DK);
 }
 
 
@@ -95,6 +110,55 @@ constexpr size_t simt_state_smem()
 // ---------------------------------------------------------------------------
 constexpr int kSimtPrepThreads = 256;   // 16 rows x 16 column lanes in the A / Aqk phase
 
+// One 16-byte global load of I/O elements, widened to fp32.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int N = 4;
+    using Raw = float4;
+    static __device__ __forceinline__ void widen(const float4& r, float (&o)[4]) {
+        o[0] = r.x; o[1] = r.y; o[2] = r.z; o[3] = r.w;
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    using Raw = uint4;
+    static __device__ __forceinline__ void widen(const uint4& r, float (&o)[8]) {
+        const uint32_t w[4] = {r.x, r.y, r.z, r.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {          // a bf16 is the high half of its fp32 value
+            o[2 * i] = __uint_as_float(w[i] << 16);
+            o[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+    }
+};
+
+// Rows [C][D] of one (chunk, head) into shared memory as fp32: every 16-byte
+// load of the thread is issued before the first one is used.
+template <typename T, int D, int NT>
+__device__ __forceinline__ void load_rows(float* dst, const T* __restrict__ src, int64_t t0,
+                                          int len, int64_t H, int64_t h, int tid)
+{
+    using V = Vec16<T>;
+    constexpr int PER_ROW = D / V::N, NV = kChunk * PER_ROW / NT;
+    static_assert(kChunk * PER_ROW % NT == 0, "rows split evenly over the block");
+    typename V::Raw r[NV];
+#pragma unroll
+    for (int x = 0; x < NV; ++x) {
+        const int e = tid + x * NT, t = e / PER_ROW, c = (e % PER_ROW) * V::N;
+        if (t < len) r[x] = *reinterpret_cast<const typename V::Raw*>(src + ((t0 + t) * H + h) * D + c);
+        else r[x] = typename V::Raw{};
+    }
+#pragma unroll
+    for (int x = 0; x < NV; ++x) {
+        const int e = tid + x * NT, t = e / PER_ROW, c = (e % PER_ROW) * V::N;
+        float o[V::N];
+        V::widen(r[x], o);
+#pragma unroll
+        for (int i = 0; i < V::N; i += 4)
+            *reinterpret_cast<float4*>(dst + t * D + c + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
+    }
+}
+
 template <typename T, int DK, int DV, bool kBwd = false>
 __global__ void __launch_bounds__(kSimtPrepThreads, 1)
 chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T* __restrict__ v,
@@ -102,8 +166,8 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                        SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
                        float* __restrict__ ws, int gate_scalar)
 {
-    constexpr int C = kChunk;
-    extern __shared__ float smem[];
+    constexpr int C = kChunk, NT = kSimtPrepThreads;
+    extern __shared__ __align__(16) float smem[];
     float* sK = smem;                 // [C][DK]
     float* sQ = sK + C * DK;          // [C][DK], later beta K e^G
     float* sV = sQ + C * DK;          // [C][DV], later beta V
@@ -119,23 +183,23 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     const int64_t gc = blockIdx.x;
     const int hl = blockIdx.y;
     const int64_t h = h_base + hl;
-    int64_t n, t0, len;
-    if (!si.locate(gc, n, t0, len)) return;
-    const int tid = threadIdx.x;
+    int64_t n, t0, len64;
+    if (!si.locate(gc, n, t0, len64)) return;
+    const int len = (int)len64;
+    const int tid = threadIdx.x, lane = tid & 31;
 
-    for (int e = tid; e < C * DK; e += blockDim.x) {
-        const int t = e / DK, c = e % DK;
-        const bool ok = t < len;
-        const int64_t src = ((t0 + t) * H + h) * DK + c;
-        sK[e] = ok ? IO<T>::load(k, src) : 0.f;
-        sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
-        sG[e] = ok ? log_alpha[gate_scalar ? (t0 + t) * H + h : src] : 0.f;
+    load_rows<T, DK, NT>(sK, k, t0, len, H, h, tid);
+    load_rows<T, DK, NT>(sQ, q, t0, len, H, h, tid);
+    load_rows<T, DV, NT>(sV, v, t0, len, H, h, tid);
+    if (gate_scalar) {
+        for (int e = tid; e < C * DK; e += NT) {
+            const int t = e / DK;
+            sG[e] = t < len ? log_alpha[(t0 + t) * H + h] : 0.f;
+        }
+    } else {
+        load_rows<float, DK, NT>(sG, log_alpha, t0, len, H, h, tid);
     }
-    for (int e = tid; e < C * DV; e += blockDim.x) {
-        const int t = e / DV, c = e % DV;
-        sV[e] = t < len ? IO<T>::load(v, ((t0 + t) * H + h) * DV + c) : 0.f;
-    }
-    for (int t = tid; t < C; t += blockDim.x) sB[t] = t < len ? beta[(t0 + t) * H + h] : 0.f;
+    for (int t = tid; t < C; t += NT) sB[t] = t < len ? beta[(t0 + t) * H + h] : 0.f;
     __syncthreads();
 
     // (a) inclusive cumulative sum of log-decay per channel within the chunk
@@ -150,27 +214,40 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     // sub-chunk of rows i at a time.  For columns j before the sub-chunk (first row f) the
     // exponential splits into two factors <= 1, e^{G_i - G_f} e^{G_f - G_j}, so the sums are
     // dot products of precomputed rows; inside the diagonal block it is taken pairwise.
-    for (int e = tid; e < C * C; e += blockDim.x) {
+    for (int e = tid; e < C * C; e += NT) {
         sA[e] = 0.f;
         sT[e] = 0.f;
         if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + e] = 0.f;
     }
+    // diagonal-block work split: threads 0..239 take the 120 pairs i > j of a 16-row
+    // block, two threads per pair (one channel half each, partner = lane ^ 1); threads
+    // 240..255 take the 16 diagonal entries of Aqk, where the decay factor is 1
+    constexpr int kPairThreads = 240, HALF = DK / 2;
+    int pi = 0, pj = 0;
+    if (tid < kPairThreads) {
+        int m = tid >> 1;
+        pi = 1;
+        while (m >= pi) { m -= pi; ++pi; }
+        pj = m;
+    } else {
+        pi = pj = tid - kPairThreads;
+    }
     for (int p = 0; p < C / 16; ++p) {
         const int f = 16 * p;
         __syncthreads();                          // zeros written, scratch rows free
-        for (int e = tid; e < 16 * DK; e += blockDim.x) {
+        for (int e = tid; e < 16 * DK; e += NT) {
             const int i = f + e / DK, c = e % DK;
             const float x = expf(sG[i * DK + c] - sG[f * DK + c]);
             sKin[e] = sK[i * DK + c] * x;
             sQin[e] = sQ[i * DK + c] * x;
         }
-        for (int e = tid; e < f * DK; e += blockDim.x) {
+        for (int e = tid; e < f * DK; e += NT) {
             const int j = e / DK, c = e % DK;
             sKvar[j * KVP + c] = sK[e] * expf(sG[f * DK + c] - sG[e]);
         }
         __syncthreads();
-        {   // rows f .. f+15 (r = tid / 16), columns jg + 16 u < f; lanes run along the
-            // columns (padded Kvar rows), the row is a broadcast
+        if (p > 0) {   // rows f .. f+15 (r = tid / 16), columns jg + 16 u < f; lanes run along
+                       // the columns (padded Kvar rows), the row is a broadcast
             const int r = tid >> 4, jg = tid & 15, i = f + r;
             float kk[3] = {0.f, 0.f, 0.f}, qk[3] = {0.f, 0.f, 0.f};
             for (int c = 0; c < DK; c += 4) {
@@ -194,72 +271,188 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                     if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = kk[u];
                 }
             }
-            // diagonal block: pair (i, j = f + jg) when j <= i; lanes differ in j, so the
-            // rotated channel index spreads them over the banks
-            const int j = f + jg;
-            if (j <= i) {
-                float dk_ = 0.f, dq_ = 0.f;
-                for (int cc = 0; cc < DK; ++cc) {
-                    const int c = (cc + j) % DK;    // rotate to spread banks
-                    const float e = expf(sG[i * DK + c] - sG[j * DK + c]);
-                    const float kj = sK[j * DK + c] * e;
+        }
+        {   // diagonal block, pairwise; the channel order is rotated by the lane so that
+            // the 32 lanes of a warp hit 32 distinct banks
+            const int i = f + pi, j = f + pj;
+            float dk_ = 0.f, dq_ = 0.f;
+            if (tid < kPairThreads) {
+                const int c0 = (tid & 1) * HALF;
+                for (int cc = 0; cc < HALF; ++cc) {
+                    const int c = c0 + (cc + lane) % HALF;
+                    const float kj = sK[j * DK + c] * expf(sG[i * DK + c] - sG[j * DK + c]);
                     dk_ += sK[i * DK + c] * kj;
                     dq_ += sQ[i * DK + c] * kj;
                 }
-                if (j < i) {
+            } else {
+                for (int cc = 0; cc < DK; ++cc) {
+                    const int c = (cc + lane) % DK;
+                    dq_ += sQ[i * DK + c] * sK[i * DK + c];
+                }
+            }
+            const float ok = __shfl_xor_sync(0xffffffffu, dk_, 1);
+            const float oq = __shfl_xor_sync(0xffffffffu, dq_, 1);
+            if (tid < kPairThreads) {
+                if ((tid & 1) == 0) {
+                    dk_ += ok;
+                    dq_ += oq;
                     sA[i * C + j] = sB[i] * dk_;
+                    sT[i * C + j] = scale * dq_;
                     if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = dk_;
                 }
-                sT[i * C + j] = scale * dq_;
+            } else {
+                sT[i * C + i] = scale * dq_;
             }
         }
     }
     __syncthreads();
 
-    for (int e = tid; e < C * C; e += blockDim.x) blk[SimtWs<DK, DV>::Aqk + e] = sT[e];
+    for (int e = tid; e < C * C; e += NT) blk[SimtWs<DK, DV>::Aqk + e] = sT[e];
     // Q e^G (scaled), K e^{G_last - G}, e^{G_last}
-    for (int e = tid; e < C * DK; e += blockDim.x) {
-        const int c = e % DK;
-        const float G = sG[e], Gl = sG[(C - 1) * DK + c];
-        blk[SimtWs<DK, DV>::QG + e] = scale * sQ[e] * expf(G);
-        blk[SimtWs<DK, DV>::KG + e] = sK[e] * expf(Gl - G);
+    for (int e4 = tid; e4 < C * DK / 4; e4 += NT) {
+        const int e = 4 * e4, c = e % DK;
+        const float4 G = *reinterpret_cast<const float4*>(sG + e);
+        const float4 Gl = *reinterpret_cast<const float4*>(sG + (C - 1) * DK + c);
+        const float4 q4 = *reinterpret_cast<const float4*>(sQ + e);
+        const float4 k4 = *reinterpret_cast<const float4*>(sK + e);
+        *reinterpret_cast<float4*>(blk + SimtWs<DK, DV>::QG + e) =
+            make_float4(scale * q4.x * expf(G.x), scale * q4.y * expf(G.y),
+                        scale * q4.z * expf(G.z), scale * q4.w * expf(G.w));
+        *reinterpret_cast<float4*>(blk + SimtWs<DK, DV>::KG + e) =
+            make_float4(k4.x * expf(Gl.x - G.x), k4.y * expf(Gl.y - G.y),
+                        k4.z * expf(Gl.z - G.z), k4.w * expf(Gl.w - G.w));
     }
-    for (int c = tid; c < DK; c += blockDim.x) blk[SimtWs<DK, DV>::Gam + c] = expf(sG[(C - 1) * DK + c]);
+    for (int c = tid; c < DK; c += NT) blk[SimtWs<DK, DV>::Gam + c] = expf(sG[(C - 1) * DK + c]);
     __syncthreads();
 
-    // (b2) T = (I + A)^{-1}: column c by forward substitution
-    if (tid < C) {
-        const int c = tid;
-        for (int i = 0; i < C; ++i) sT[i * C + c] = (i == c) ? 1.f : 0.f;
-        for (int i = c + 1; i < C; ++i) {
+    // (b2) T = (I + A)^{-1} by 16 x 16 blocks.  Diagonal blocks: one column per thread
+    // (threads 0..63), forward substitution in registers; the other threads clear the
+    // blocks above the diagonal and scale K e^G and V by beta.
+    if (tid < 64) {
+        const int f = 16 * (tid >> 4), c = tid & 15;
+        float col[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
             float acc = 0.f;
-            for (int j = c; j < i; ++j) acc += sA[i * C + j] * sT[j * C + c];
-            sT[i * C + c] = -acc;
+#pragma unroll
+            for (int j = 0; j < i; ++j) acc += sA[(f + i) * C + f + j] * col[j];
+            col[i] = (i == c) ? 1.f : -acc;       // zero above the diagonal (acc = 0 there)
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sT[(f + i) * C + f + c] = col[i];
+    } else {
+        for (int e = tid - 64; e < C * C; e += NT - 64) {
+            const int i = e / C, j = e % C;
+            if ((j >> 4) > (i >> 4)) sT[e] = 0.f;
+        }
+        // beta K e^G into sQ, beta V in place
+        for (int e = tid - 64; e < C * DK; e += NT - 64) sQ[e] = sB[e / DK] * sK[e] * expf(sG[e]);
+        for (int e = tid - 64; e < C * DV; e += NT - 64) sV[e] *= sB[e / DV];
+    }
+    // Off-diagonal blocks by distance d = p - r: T_pr = -T_pp sum_{m=r}^{p-1} A_pm T_mr,
+    // whose factors all lie at distances below d.  Thread (a, b) owns entry (a, b) of each
+    // block of the level; the partial sums go through sKin.
+    {
+        const int a = tid >> 4, b = tid & 15;
+        float* sX = sKin;                         // [3][16][16]
+        for (int d = 1; d < 4; ++d) {
+            __syncthreads();                      // level d - 1 (or the diagonal) written
+            for (int r = 0; r + d < 4; ++r) {
+                const int p = r + d;
+                float x = 0.f;
+                for (int m = r; m < p; ++m) {
+#pragma unroll
+                    for (int l = 0; l < 16; l += 4) {
+                        const float4 av = *reinterpret_cast<const float4*>(sA + (16 * p + a) * C + 16 * m + l);
+                        x += av.x * sT[(16 * m + l) * C + 16 * r + b] + av.y * sT[(16 * m + l + 1) * C + 16 * r + b] +
+                             av.z * sT[(16 * m + l + 2) * C + 16 * r + b] + av.w * sT[(16 * m + l + 3) * C + 16 * r + b];
+                    }
+                }
+                sX[r * 256 + a * 16 + b] = x;
+            }
+            __syncthreads();
+            for (int r = 0; r + d < 4; ++r) {
+                const int p = r + d;
+                float y = 0.f;
+#pragma unroll
+                for (int l = 0; l < 16; l += 4) {
+                    const float4 tv = *reinterpret_cast<const float4*>(sT + (16 * p + a) * C + 16 * p + l);
+                    y += tv.x * sX[r * 256 + l * 16 + b] + tv.y * sX[r * 256 + (l + 1) * 16 + b] +
+                         tv.z * sX[r * 256 + (l + 2) * 16 + b] + tv.w * sX[r * 256 + (l + 3) * 16 + b];
+                }
+                sT[(16 * p + a) * C + 16 * r + b] = -y;
+            }
         }
     }
-    // beta K e^G into sQ, beta V in place
-    for (int e = tid; e < C * DK; e += blockDim.x) sQ[e] = sB[e / DK] * sK[e] * expf(sG[e]);
-    for (int e = tid; e < C * DV; e += blockDim.x) sV[e] *= sB[e / DV];
     __syncthreads();
 
     if constexpr (kBwd) {                       // T and K e^G for the backward
-        for (int e = tid; e < C * C; e += blockDim.x) blk[BwdWs<DK, DV>::Tm + e] = sT[e];
-        for (int e = tid; e < C * DK; e += blockDim.x)
+        for (int e = tid; e < C * C; e += NT) blk[BwdWs<DK, DV>::Tm + e] = sT[e];
+        for (int e = tid; e < C * DK; e += NT)
             blk[BwdWs<DK, DV>::KGm + e] = sK[e] * expf(sG[e]);
     }
 
-    // (b3) W = T (beta K e^G), Ut = T (beta V)
-    for (int e = tid; e < C * DK; e += blockDim.x) {
-        const int i = e / DK, c = e % DK;
-        float acc = 0.f;
-        for (int j = 0; j <= i; ++j) acc += sT[i * C + j] * sQ[j * DK + c];
-        blk[SimtWs<DK, DV>::W + e] = acc;
-    }
-    for (int e = tid; e < C * DV; e += blockDim.x) {
-        const int i = e / DV, c = e % DV;
-        float acc = 0.f;
-        for (int j = 0; j <= i; ++j) acc += sT[i * C + j] * sV[j * DV + c];
-        blk[SimtWs<DK, DV>::Ut + e] = acc;
+    // (b3) [W | Ut] = T [beta K e^G | beta V], register-tiled: thread (g, cg) owns rows
+    // 2g, 2g+1 (which need columns j <= 2g+1 of T) and 62-2g, 63-2g (j <= 63-2g), so all
+    // threads do the same number of products, and 16-byte column groups 4 cg + 64 u.
+    {
+        constexpr int NU = (DK + DV) / 64;
+        const int g = tid >> 4, cg = tid & 15;
+        const int row[4] = {2 * g, 2 * g + 1, 62 - 2 * g, 63 - 2 * g};
+        const int jl = (2 * g + 2 + 3) & ~3;
+        const int jh = (64 - 2 * g + 3) & ~3;
+        float4 acc[4][NU];
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int u = 0; u < NU; ++u) acc[rr][u] = make_float4(0.f, 0.f, 0.f, 0.f);
+        auto bcol = [&](int u, int j) -> float4 {
+            return 64 * u < DK ? *reinterpret_cast<const float4*>(sQ + j * DK + 64 * u + 4 * cg)
+                               : *reinterpret_cast<const float4*>(sV + j * DV + 64 * u - DK + 4 * cg);
+        };
+        auto step = [&](int j, const float (&tj)[4][4], int r0) {
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj)
+#pragma unroll
+                for (int u = 0; u < NU; ++u) {
+                    const float4 bv = bcol(u, j + jj);
+#pragma unroll
+                    for (int rr = 0; rr < 4; ++rr) {
+                        if (rr < r0) continue;
+                        const float t = tj[rr][jj];
+                        acc[rr][u].x += t * bv.x;
+                        acc[rr][u].y += t * bv.y;
+                        acc[rr][u].z += t * bv.z;
+                        acc[rr][u].w += t * bv.w;
+                    }
+                }
+        };
+        for (int j = 0; j < jl; j += 4) {
+            float tj[4][4];
+#pragma unroll
+            for (int rr = 0; rr < 4; ++rr) {
+                const float4 t4 = *reinterpret_cast<const float4*>(sT + row[rr] * C + j);
+                tj[rr][0] = t4.x; tj[rr][1] = t4.y; tj[rr][2] = t4.z; tj[rr][3] = t4.w;
+            }
+            step(j, tj, 0);
+        }
+        for (int j = jl; j < jh; j += 4) {
+            float tj[4][4] = {};
+#pragma unroll
+            for (int rr = 2; rr < 4; ++rr) {
+                const float4 t4 = *reinterpret_cast<const float4*>(sT + row[rr] * C + j);
+                tj[rr][0] = t4.x; tj[rr][1] = t4.y; tj[rr][2] = t4.z; tj[rr][3] = t4.w;
+            }
+            step(j, tj, 2);
+        }
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+            for (int u = 0; u < NU; ++u) {
+                float* dst = 64 * u < DK ? blk + SimtWs<DK, DV>::W + row[rr] * DK + 64 * u + 4 * cg
+                                         : blk + SimtWs<DK, DV>::Ut + row[rr] * DV + 64 * u - DK + 4 * cg;
+                *reinterpret_cast<float4*>(dst) = acc[rr][u];
+            }
     }
 }
 
@@ -276,13 +469,13 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     const SeqInfo& si = a.si;
     const int64_t H = a.H;
     T* __restrict__ out = (T*)a.out;
-    constexpr int C = kChunk, TW = kTW;
+    constexpr int C = kChunk, TW = kTW, NT = 256;
     extern __shared__ __align__(16) float smem[];
-    // (the backward walk writes no output: no Q e^G, no Aqk, and half the shared memory)
+    // (the backward walk writes no output: no Q e^G, no Aqk, and less shared memory)
     float* sW = smem;                                  // [C][DK]
     float* sKG = sW + C * DK;                          // [C][DK]
-    float* sU = sKG + C * DK;                          // [C][TW]
-    float* sS = sU + C * TW;                           // [DK][kSP]  copy of the entry state
+    float* sUb = sKG + C * DK;                         // 2 x [C][TW]  (chunk ch in buffer ch & 1)
+    float* sS = sUb + 2 * C * TW;                      // [DK][kSP]  copy of the entry state
     float* sGam = sS + DK * kSP;                       // [DK]
     float* sQG = sGam + DK;                            // [C][DK]    (forward only)
     float* sAqk = sQG + C * DK;                        // [C][C]     (forward only)
@@ -300,6 +493,36 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
     const int64_t nchunks = si.chunk_count(n, eos - bos);
     const int64_t gc0 = si.chunk_start(n);
+    auto block_of = [&](int64_t ch) { return ws + ((gc0 + ch) * Hg + hl) * kStride; };
+
+    // Each buffer is refilled by cp.async as soon as its last reader of the previous
+    // chunk is past a barrier, so the loads of chunk ch + 1 run under chunk ch's work:
+    //   group U:  K e^{G_last-G}, e^{G_last} of ch and the Ut tile of ch + 1   (top of ch)
+    //   group W:  W of ch + 1                                           (after U = Ut - W S)
+    //   group QA: Q e^G and Aqk of ch + 1                               (after the output)
+    // Every wait is "all but the newest group", and each is followed by a barrier.
+    auto load_ut = [&](int64_t ch) {
+        const float* src = block_of(ch) + SimtWs<DK, DV>::Ut + j0;
+        float* dst = sUb + (ch & 1) * C * TW;
+        for (int e = tid; e < C * TW / 4; e += NT)
+            async16(dst + 4 * e, src + (e / (TW / 4)) * DV + 4 * (e % (TW / 4)));
+    };
+    auto load_kg = [&](int64_t ch) {
+        const float* b = block_of(ch);
+        for (int e = tid; e < C * DK / 4; e += NT) async16(sKG + 4 * e, b + SimtWs<DK, DV>::KG + 4 * e);
+        for (int e = tid; e < DK / 4; e += NT) async16(sGam + 4 * e, b + SimtWs<DK, DV>::Gam + 4 * e);
+    };
+    auto load_w = [&](int64_t ch) {
+        const float* b = block_of(ch) + SimtWs<DK, DV>::W;
+        for (int e = tid; e < C * DK / 4; e += NT) async16(sW + 4 * e, b + 4 * e);
+    };
+    auto load_qa = [&](int64_t ch) {
+        if constexpr (!kBwd) {
+            const float* b = block_of(ch);
+            for (int e = tid; e < C * DK / 4; e += NT) async16(sQG + 4 * e, b + SimtWs<DK, DV>::QG + 4 * e);
+            for (int e = tid; e < C * C / 4; e += NT) async16(sAqk + 4 * e, b + SimtWs<DK, DV>::Aqk + 4 * e);
+        }
+    };
 
     const int64_t sidx = a.state_index(n, h);
     const float* h0p = (a.h0 && sidx >= 0) ? a.h0 + sidx * DK * DV : nullptr;
@@ -312,23 +535,20 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
 #pragma unroll
     for (int x = 0; x < NJ; ++x) st[x] = h0p ? h0p[(int64_t)c * DV + j0 + jb + x] : 0.f;
 
+    if (nchunks > 0) {
+        load_ut(0);
+        load_w(0);
+    }
+    async_commit();
+    if (nchunks > 0) load_qa(0);
+    async_commit();
+
     for (int64_t ch = 0; ch < nchunks; ++ch) {
-        float* blk = ws + ((gc0 + ch) * Hg + hl) * kStride;
+        float* blk = block_of(ch);
+        float* sU = sUb + (ch & 1) * C * TW;
         const int64_t t0 = bos + ch * C;
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-        __syncthreads();                          // the previous chunk's reads are done
-        for (int e = tid; e < C * DK / 4; e += blockDim.x) {
-            reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::W)[e];
-            reinterpret_cast<float4*>(sKG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::KG)[e];
-            if constexpr (!kBwd)
-                reinterpret_cast<float4*>(sQG)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::QG)[e];
-        }
-        if constexpr (!kBwd)
-            for (int e = tid; e < C * C / 4; e += blockDim.x)
-                reinterpret_cast<float4*>(sAqk)[e] = reinterpret_cast<const float4*>(blk + SimtWs<DK, DV>::Aqk)[e];
-        for (int e = tid; e < C * TW; e += blockDim.x)
-            sU[e] = blk[SimtWs<DK, DV>::Ut + (e / TW) * DV + j0 + (e % TW)];
-        for (int cc = tid; cc < DK; cc += blockDim.x) sGam[cc] = blk[SimtWs<DK, DV>::Gam + cc];
+        async_wait<1>();                          // Ut and W of this chunk
 #pragma unroll
         for (int x = 0; x < NJ; x += 4) {
             const float4 v4 = make_float4(st[x], st[x + 1], st[x + 2], st[x + 3]);
@@ -336,7 +556,10 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
             if constexpr (kBwd)
                 *reinterpret_cast<float4*>(blk + BwdWs<DK, DV>::Sx + (int64_t)c * DV + j0 + jb + x) = v4;
         }
-        __syncthreads();
+        __syncthreads();                          // also: the previous chunk's state update is done
+        load_kg(ch);
+        if (ch + 1 < nchunks) load_ut(ch + 1);
+        async_commit();
         // U = Ut - W S: rows t = w + 8 r, column lane
         {
             float acc[8];
@@ -346,7 +569,10 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
 #pragma unroll
             for (int r = 0; r < 8; ++r) sU[(wrp + 8 * r) * TW + lane] -= acc[r];
         }
+        async_wait<1>();                          // Q e^G and Aqk of this chunk
         __syncthreads();
+        if (ch + 1 < nchunks) load_w(ch + 1);
+        async_commit();
         // O = scale (Q e^G) S + Aqk U   (the entry state; Aqk is zero above the diagonal)
         if constexpr (!kBwd) {
             float acc[8];
@@ -360,6 +586,10 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
                 if (t < len) IO<T>::store(out, ((t0 + t) * H + h) * DV + j0 + lane, acc[r]);
             }
         }
+        async_wait<1>();                          // K e^{G_last - G} and e^{G_last} of this chunk
+        __syncthreads();
+        if (ch + 1 < nchunks) load_qa(ch + 1);
+        async_commit();
         // S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U, in registers
         {
             const float gmc = sGam[c];
@@ -377,7 +607,9 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
                 }
             }
         }
+        // the next chunk's barrier (after its Ut / W wait) orders these reads before any refill
     }
+    async_wait<0>();
     if (hTp)
 #pragma unroll
         for (int x = 0; x < NJ; ++x) hTp[(int64_t)c * DV + j0 + jb + x] = st[x];
