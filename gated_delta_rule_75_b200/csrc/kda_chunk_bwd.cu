@@ -220,8 +220,11 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
             sUt[e] = blk[SW::Ut + t * DV + j0 + j];
         }
         __syncthreads();
-        if (tid < DK)
-            for (int j = 0; j < kTW; ++j) glS += sS[tid * kTW + j] * sdSn[tid * kTW + j];
+        if (tid < DK)                                 // (column order rotated by the row: no bank conflicts)
+            for (int jj = 0; jj < kTW; ++jj) {
+                const int j = (jj + tid) % kTW;
+                glS += sS[tid * kTW + j] * sdSn[tid * kTW + j];
+            }
         // rows w, w + NW, ... of this warp (NW warps); column j0 + lane
         constexpr int NW = kD1T / 32, NR = C / NW;
         float e8[NR], r8[NR], de8[NR];
@@ -364,8 +367,9 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     float* sdG = sG + C * DK;         // [C][DK]
     float* sAp = sdG + C * DK;        // [C][C]   A', then dA' = diag(beta) dA
     float* sdAqk = sAp + C * C;       // [C][C]   dAqk, then scale dAqk
-    float* sT = sdAqk + C * C;        // [C][C]   T          } free after dA: scratch of the
-    float* sdT = sT + C * C;          // [C][C]   dT', dT    } pairwise terms, 2 x [48][DK]
+    constexpr int TP = C + 1;         // row pitch of T: column walks over rows hit distinct banks
+    float* sT = sdAqk + C * C;        // [C][TP]  T          } free after dA: scratch of the
+    float* sdT = sT + C * TP;         // [C][C]   dT', dT    } pairwise terms, 2 x [48][DK]
     float* sX = sdT + C * C;          // [C][C]   dT T^T, dA }
     float* sB = sX + C * C;           // [C]
     float* sdB = sB + C;              // [C]
@@ -391,7 +395,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
         sG[e] = ok ? b.log_alpha[b.gate_scalar ? (t0 + t) * H + h : src] : 0.f;
     }
     for (int e = tid; e < C * C; e += kPT) {
-        sT[e] = blk[BW::Tm + e];
+        sT[(e / C) * TP + e % C] = blk[BW::Tm + e];
         sAp[e] = blk[BW::Ap + e];
         sdT[e] = blk[BW::dTp + e];
         sdAqk[e] = blk[BW::dAqk + e];
@@ -405,7 +409,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     // dbeta_i = sum_r T[r][i] dT'[r][i]
     if (tid < C) {
         float acc = 0.f;
-        for (int r = tid; r < C; ++r) acc += sT[r * C + tid] * sdT[r * C + tid];
+        for (int r = tid; r < C; ++r) acc += sT[r * TP + tid] * sdT[r * C + tid];
         sdB[tid] = acc;
     }
     __syncthreads();
@@ -415,21 +419,23 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     for (int e = tid; e < C * C; e += kPT) {
         const int r = e / C, j = e % C;
         float acc = 0.f;
-        for (int m = 0; m <= j; ++m) acc += sdT[r * C + m] * sT[j * C + m];
+        for (int m = 0; m <= j; ++m) acc += sdT[r * C + m] * sT[j * TP + m];
         sX[e] = acc;
     }
     __syncthreads();
     // dA[i][j] = -sum_r T[r][i] X[r][j]  (i > j; T[r][i] = 0 for r < i)
     constexpr int NU = C * C / kPT;
     float dA[NU];
+#pragma unroll
     for (int u = 0; u < NU; ++u) {
         const int e = tid + kPT * u, i = e / C, j = e % C;
         float acc = 0.f;
         if (j < i)
-            for (int r = i; r < C; ++r) acc += sT[r * C + i] * sX[r * C + j];
+            for (int r = i; r < C; ++r) acc += sT[r * TP + i] * sX[r * C + j];
         dA[u] = -acc;
     }
     __syncthreads();
+#pragma unroll
     for (int u = 0; u < NU; ++u) sX[tid + kPT * u] = dA[u];
     __syncthreads();
     // dbeta_i += sum_{j<i} dA[i][j] A'[i][j];  dA' = diag(beta) dA
@@ -583,7 +589,7 @@ constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(2 * kChunk *
 template <int DK, int DV>
 constexpr size_t bwd_dense1_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + 2 * kChunk * kAP + 2 * DK * kTW + 4 * kChunk * kTW + kChunk); }
 template <int DK, int DV>
-constexpr size_t bwd_param_smem() { return sizeof(float) * (size_t)(4 * kChunk * DK + 5 * kChunk * kChunk + 2 * kChunk); }
+constexpr size_t bwd_param_smem() { return sizeof(float) * (size_t)(4 * kChunk * DK + 5 * kChunk * kChunk + 3 * kChunk); }
 
 template <typename T, int DK, int DV>
 static cudaError_t run_bwd_t(const BackwardArgs& b, float* ws, int64_t Hg, cudaStream_t st)

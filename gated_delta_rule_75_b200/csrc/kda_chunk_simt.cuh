@@ -52,6 +52,28 @@ __device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int l
     rows_mac<8, 8, LDB>(acc, A, lda, row0, B, K, lane);
 }
 
+// acc[i][x] += sum_k A[(row0 + i) * LDA + k] * B[k * LDB + 2 cp + x], i < 4, x < 2, K a
+// multiple of 4: four rows by two columns per thread.  With the lanes of a warp split
+// into two row groups (row0 four rows apart) and 16 column pairs, each 16-byte row load
+// serves 16 lanes and each 8-byte column load two, so a k step costs two shared-memory
+// wavefronts for eight FMAs when LDA keeps the two row groups on different banks.
+template <int LDA, int LDB>
+__device__ __forceinline__ void tile42_mac(float (&acc)[4][2], const float* A, int row0,
+                                           const float* B, int K, int cp)
+{
+    for (int k = 0; k < K; k += 4) {
+        float2 b[4];
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk) b[kk] = *reinterpret_cast<const float2*>(B + (k + kk) * LDB + 2 * cp);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            const float4 a = *reinterpret_cast<const float4*>(A + (row0 + i) * LDA + k);
+            acc[i][0] += a.x * b[0].x + a.y * b[1].x + a.z * b[2].x + a.w * b[3].x;
+            acc[i][1] += a.x * b[0].y + a.y * b[1].y + a.z * b[2].y + a.w * b[3].y;
+        }
+    }
+}
+
 // Workspace block of one (chunk, head), in floats.
 template <int DK, int DV>
 struct SimtWs {
@@ -95,13 +117,13 @@ struct BwdWs {
 template <int DK, int DV>
 constexpr size_t simt_prep_smem()
 {
-    return sizeof(float) * (size_t)(kChunk * (3 * DK + DV) + 2 * kChunk * kChunk + kChunk + 32 * DK + 48 * (DK + 4));
+    return sizeof(float) * (size_t)(kChunk * (3 * DK + DV) + 2 * kChunk * kChunk + kChunk + 32 * DK + 64 * (DK + 4));
 }
 template <int DK, int DV, bool kBwd = false>
 constexpr size_t simt_state_smem()
 {
-    return sizeof(float) * (size_t)((kBwd ? 2 : 3) * kChunk * DK + (kBwd ? 0 : kChunk * kChunk) +
-                                    2 * kChunk * kTW + DK * kSP + DK);
+    return sizeof(float) * (size_t)((kBwd ? 1 : 2) * kChunk * (DK + 4) + kChunk * DK +
+                                    (kBwd ? 0 : kChunk * (kChunk + 4)) + 2 * kChunk * kTW + DK * kSP + DK);
 }
 
 
@@ -178,7 +200,7 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     float* sKin = sB + C;             // [16][DK]  rows of one sub-chunk, referenced to its first row
     float* sQin = sKin + 16 * DK;     // [16][DK]
     constexpr int KVP = DK + 4;       // padded row pitch of sKvar (16 rows -> distinct banks)
-    float* sKvar = sQin + 16 * DK;    // [48][KVP] earlier rows, referenced forward to it
+    float* sKvar = sQin + 16 * DK;    // [64][KVP] earlier rows (and the sub-chunk's own), referenced to it
 
     const int64_t gc = blockIdx.x;
     const int hl = blockIdx.y;
@@ -211,9 +233,12 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
 
     float* blk = ws + (gc * Hg + hl) * (kBwd ? BwdWs<DK, DV>::size : SimtWs<DK, DV>::size);
     // (b1) A (strictly lower, beta-weighted) and Aqk (lower incl. diagonal), one 16-row
-    // sub-chunk of rows i at a time.  For columns j before the sub-chunk (first row f) the
-    // exponential splits into two factors <= 1, e^{G_i - G_f} e^{G_f - G_j}, so the sums are
-    // dot products of precomputed rows; inside the diagonal block it is taken pairwise.
+    // sub-chunk of rows i at a time.  The exponential splits at the sub-chunk's first row f,
+    // e^{G_i - G_f} e^{G_f - G_j}, so the sums are dot products of precomputed rows.  For
+    // columns j before the sub-chunk both factors are <= 1.  Inside the diagonal block the
+    // second factor is >= 1, bounded by the block's decay; where some channel decays by more
+    // than 64 nats across the block (e^64 ~ 6e27, its inverse still a normal fp32 number)
+    // that block is taken pairwise, e^{G_i - G_j} per channel, so any decay rate is exact.
     for (int e = tid; e < C * C; e += NT) {
         sA[e] = 0.f;
         sT[e] = 0.f;
@@ -232,30 +257,36 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     } else {
         pi = pj = tid - kPairThreads;
     }
+    constexpr float kMaxBlockDecay = 64.f;
     for (int p = 0; p < C / 16; ++p) {
         const int f = 16 * p;
-        __syncthreads();                          // zeros written, scratch rows free
+        // (this barrier also: zeros written, scratch rows free)
+        const int pairwise = __syncthreads_or(
+            tid < DK && fabsf(sG[f * DK + tid] - sG[(f + 15) * DK + tid]) > kMaxBlockDecay);
         for (int e = tid; e < 16 * DK; e += NT) {
             const int i = f + e / DK, c = e % DK;
-            const float x = expf(sG[i * DK + c] - sG[f * DK + c]);
+            const float d = sG[i * DK + c] - sG[f * DK + c];
+            const float x = expf(d);
             sKin[e] = sK[i * DK + c] * x;
             sQin[e] = sQ[i * DK + c] * x;
+            if (!pairwise) sKvar[i * KVP + c] = sK[i * DK + c] * expf(-d);
         }
         for (int e = tid; e < f * DK; e += NT) {
             const int j = e / DK, c = e % DK;
             sKvar[j * KVP + c] = sK[e] * expf(sG[f * DK + c] - sG[e]);
         }
         __syncthreads();
-        if (p > 0) {   // rows f .. f+15 (r = tid / 16), columns jg + 16 u < f; lanes run along
+        const int nu = pairwise ? p : p + 1;      // column blocks taken as dot products
+        if (nu > 0) {  // rows f .. f+15 (r = tid / 16), columns jg + 16 u; lanes run along
                        // the columns (padded Kvar rows), the row is a broadcast
             const int r = tid >> 4, jg = tid & 15, i = f + r;
-            float kk[3] = {0.f, 0.f, 0.f}, qk[3] = {0.f, 0.f, 0.f};
+            float kk[4] = {0.f, 0.f, 0.f, 0.f}, qk[4] = {0.f, 0.f, 0.f, 0.f};
             for (int c = 0; c < DK; c += 4) {
                 const float4 a = *reinterpret_cast<const float4*>(sKin + r * DK + c);
                 const float4 q4 = *reinterpret_cast<const float4*>(sQin + r * DK + c);
 #pragma unroll
-                for (int u = 0; u < 3; ++u) {
-                    if (u < p) {
+                for (int u = 0; u < 4; ++u) {
+                    if (u < nu) {
                         const float4 kv = *reinterpret_cast<const float4*>(sKvar + (jg + 16 * u) * KVP + c);
                         kk[u] += a.x * kv.x + a.y * kv.y + a.z * kv.z + a.w * kv.w;
                         qk[u] += q4.x * kv.x + q4.y * kv.y + q4.z * kv.z + q4.w * kv.w;
@@ -263,17 +294,19 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                 }
             }
 #pragma unroll
-            for (int u = 0; u < 3; ++u) {
-                if (u < p) {
-                    const int j = jg + 16 * u;
-                    sA[i * C + j] = sB[i] * kk[u];
+            for (int u = 0; u < 4; ++u) {
+                const int j = jg + 16 * u;
+                if (u < nu && j <= i) {           // (the diagonal block: its lower half only)
+                    if (j < i) {
+                        sA[i * C + j] = sB[i] * kk[u];
+                        if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = kk[u];
+                    }
                     sT[i * C + j] = scale * qk[u];   // Aqk parked in sT for now
-                    if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = kk[u];
                 }
             }
         }
-        {   // diagonal block, pairwise; the channel order is rotated by the lane so that
-            // the 32 lanes of a warp hit 32 distinct banks
+        if (pairwise) {   // diagonal block, pairwise; the channel order is rotated by the lane
+                          // so that the 32 lanes of a warp hit 32 distinct banks
             const int i = f + pi, j = f + pj;
             float dk_ = 0.f, dq_ = 0.f;
             if (tid < kPairThreads) {
@@ -472,13 +505,16 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     constexpr int C = kChunk, TW = kTW, NT = 256;
     extern __shared__ __align__(16) float smem[];
     // (the backward walk writes no output: no Q e^G, no Aqk, and less shared memory)
-    float* sW = smem;                                  // [C][DK]
-    float* sKG = sW + C * DK;                          // [C][DK]
+    // row pitches DK + 4 and C + 4: the two row groups of a warp in tile42_mac (four rows
+    // apart) land on different banks
+    constexpr int WP = DK + 4, AP = C + 4;
+    float* sW = smem;                                  // [C][WP]
+    float* sKG = sW + C * WP;                          // [C][DK]
     float* sUb = sKG + C * DK;                         // 2 x [C][TW]  (chunk ch in buffer ch & 1)
     float* sS = sUb + 2 * C * TW;                      // [DK][kSP]  copy of the entry state
     float* sGam = sS + DK * kSP;                       // [DK]
-    float* sQG = sGam + DK;                            // [C][DK]    (forward only)
-    float* sAqk = sQG + C * DK;                        // [C][C]     (forward only)
+    float* sQG = sGam + DK;                            // [C][WP]    (forward only)
+    float* sAqk = sQG + C * WP;                        // [C][AP]    (forward only)
 
     // blocks run (tile, head)-innermost over sequences ranked longest first
     const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
@@ -514,13 +550,16 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     };
     auto load_w = [&](int64_t ch) {
         const float* b = block_of(ch) + SimtWs<DK, DV>::W;
-        for (int e = tid; e < C * DK / 4; e += NT) async16(sW + 4 * e, b + 4 * e);
+        for (int e = tid; e < C * DK / 4; e += NT)
+            async16(sW + (e / (DK / 4)) * WP + 4 * (e % (DK / 4)), b + 4 * e);
     };
     auto load_qa = [&](int64_t ch) {
         if constexpr (!kBwd) {
             const float* b = block_of(ch);
-            for (int e = tid; e < C * DK / 4; e += NT) async16(sQG + 4 * e, b + SimtWs<DK, DV>::QG + 4 * e);
-            for (int e = tid; e < C * C / 4; e += NT) async16(sAqk + 4 * e, b + SimtWs<DK, DV>::Aqk + 4 * e);
+            for (int e = tid; e < C * DK / 4; e += NT)
+                async16(sQG + (e / (DK / 4)) * WP + 4 * (e % (DK / 4)), b + SimtWs<DK, DV>::QG + 4 * e);
+            for (int e = tid; e < C * C / 4; e += NT)
+                async16(sAqk + (e / (C / 4)) * AP + 4 * (e % (C / 4)), b + SimtWs<DK, DV>::Aqk + 4 * e);
         }
     };
 
@@ -560,14 +599,18 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
         load_kg(ch);
         if (ch + 1 < nchunks) load_ut(ch + 1);
         async_commit();
-        // U = Ut - W S: rows t = w + 8 r, column lane
+        // U = Ut - W S: thread (warp w, lane) takes rows 8 w + 4 (lane / 16) + i, i < 4,
+        // and columns 2 (lane mod 16) + x, x < 2
+        const int row0 = 8 * wrp + 4 * (lane >> 4), cp = lane & 15;
         {
-            float acc[8];
+            float acc[4][2] = {};
+            tile42_mac<WP, kSP>(acc, sW, row0, sS, DK, cp);
 #pragma unroll
-            for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-            rows8_mac<kSP>(acc, sW, DK, wrp, sS, DK, lane);
-#pragma unroll
-            for (int r = 0; r < 8; ++r) sU[(wrp + 8 * r) * TW + lane] -= acc[r];
+            for (int i = 0; i < 4; ++i) {
+                float2* u2 = reinterpret_cast<float2*>(sU + (row0 + i) * TW + 2 * cp);
+                const float2 u = *u2;
+                *u2 = make_float2(u.x - acc[i][0], u.y - acc[i][1]);
+            }
         }
         async_wait<1>();                          // Q e^G and Aqk of this chunk
         __syncthreads();
@@ -575,15 +618,17 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
         async_commit();
         // O = scale (Q e^G) S + Aqk U   (the entry state; Aqk is zero above the diagonal)
         if constexpr (!kBwd) {
-            float acc[8];
+            float acc[4][2] = {};
+            tile42_mac<WP, kSP>(acc, sQG, row0, sS, DK, cp);
+            tile42_mac<AP, TW>(acc, sAqk, row0, sU, C, cp);
 #pragma unroll
-            for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-            rows8_mac<kSP>(acc, sQG, DK, wrp, sS, DK, lane);
-            rows8_mac<TW>(acc, sAqk, C, wrp, sU, C, lane);
-#pragma unroll
-            for (int r = 0; r < 8; ++r) {
-                const int t = wrp + 8 * r;
-                if (t < len) IO<T>::store(out, ((t0 + t) * H + h) * DV + j0 + lane, acc[r]);
+            for (int i = 0; i < 4; ++i) {
+                const int t = row0 + i;
+                if (t < len) {
+                    const int64_t o = ((t0 + t) * H + h) * DV + j0 + 2 * cp;
+                    IO<T>::store(out, o, acc[i][0]);
+                    IO<T>::store(out, o + 1, acc[i][1]);
+                }
             }
         }
         async_wait<1>();                          // K e^{G_last - G} and e^{G_last} of this chunk

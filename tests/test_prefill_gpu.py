@@ -65,6 +65,19 @@ def test_tensorcore_fast_and_slow_decay(kda, shift):
     check_full(kda, cfg, "tensorcore")
 
 
+@pytest.mark.parametrize("shift", [-4.0, 3.0, 3.6, 8.0])
+def test_simt_decay_rates_fp32(kda, shift):
+    """fp32 I/O at mean per-token decays from e^-0.02 to e^-8: the SIMT prep factors
+    each 16-row diagonal block through its first row while every channel's decay
+    across the block stays within 64 nats and takes it pairwise past that.  Over 15
+    tokens the channels decay by ~46 nats at shift 3 (factored blocks), ~55 at 3.6
+    (the largest of 128 channels passes 64 in about half the blocks: both kinds in
+    one chunk) and ~120 at 8 (pairwise blocks); parity holds at the fp32 bar throughout."""
+    cfg = W.small_prefill(B=1, T=200, H=2, dk=128, dv=128, io_dtype="f32", seed=11,
+                          gate_shift=shift, h0_std=0.05)
+    check_full(kda, cfg, "simt")
+
+
 def test_tensorcore_refuses_unsupported_shapes(kda):
     cfg = W.small_prefill(B=1, T=64, H=1, dk=64, dv=64, io_dtype="bf16", seed=1)
     inp = W.make_prefill(cfg, "cuda")
