@@ -43,35 +43,40 @@ constexpr int kAP = 68;           // row pitch of the transposed Aqk
 
 // dS stays in registers across chunks: thread (warp w, lane) owns row c = 32 (w mod DK/32)
 // + lane and NJ consecutive columns of the 32-column tile (NJ = 16 for DK = 128, 8 for 64);
-// it is copied to shared memory once per chunk as the operand of Khat dS'.
+// it is copied to shared memory once per chunk as the operand of Khat dS'.  Each operand
+// has its own buffer, refilled by cp.async while the other phase of the chunk runs:
+//   group A (Khat, Aqk of chunk ch - 1): issued after dE of chunk ch, used by dE of ch - 1
+//   group B (W, Q_G, e^{G_last} of ch):  issued when chunk ch starts, used by its dS update
+// and the dO tile of the next chunk is fetched into registers one chunk ahead.
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kBT, 2)
+__global__ void __launch_bounds__(kBT, 1)
 chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
     using SW = SimtWs<DK, DV>;
-    constexpr int C = kChunk;
+    using V = Vec16<T>;
+    constexpr int C = kChunk, TW = kTW;
     constexpr int RG = DK / 32;       // groups of 32 rows
+    constexpr int KP = DK + 4;        // row pitch of Khat (two row groups of tile42_mac on distinct banks)
     const SeqInfo& si = b.si;
     const int64_t H = b.H;
-    // Two operand buffers, reloaded between the two phases of a chunk so that two CTAs
-    // fit on an SM: X = Khat then W, Y = Aqk^T (pitch kAP) then Q_G.
     extern __shared__ __align__(16) float smem[];
-    constexpr int YW = DK > kAP ? DK : kAP;
-    float* sX = smem;                 // [C][DK]
-    float* sY = sX + C * YW;          // [C][YW]
-    float* sdO = sY + C * YW;         // [C][32]
-    float* sdE = sdO + C * kTW;       // [C][32]
-    float* sdS = sdE + C * kTW;       // [DK][kSP]
-    float* sGam = sdS + DK * kSP;     // [DK]
+    float* sKh = smem;                // [C][KP]   K e^{G_last - G}
+    float* sAqk = sKh + C * KP;       // [C][C]    Aqk (row r, column t), read as Aqk^T
+    float* sW = sAqk + C * C;         // [C][DK]
+    float* sQG = sW + C * DK;         // [C][DK]
+    float* sGam = sQG + C * DK;       // [DK]
+    float* sdO = sGam + DK;           // [C][TW]
+    float* sdE = sdO + C * TW;        // [C][TW]
+    float* sdS = sdE + C * TW;        // [DK][kSP]
 
     const int64_t hg = (H - h_base) < Hg ? (H - h_base) : Hg;
-    const int64_t tiles = DV / kTW;
+    const int64_t tiles = DV / TW;
     const int64_t bid = blockIdx.x;
     const int64_t n = bid / (hg * tiles);
     const int hl = (int)((bid / tiles) % hg);
     const int64_t h = h_base + hl;
-    const int j0 = (int)(bid % tiles) * kTW;
+    const int j0 = (int)(bid % tiles) * TW;
     const int tid = threadIdx.x, lane = tid & 31, wrp = tid >> 5;
     int64_t bos, eos;
     seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
@@ -79,9 +84,41 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     const int64_t gc0 = si.chunk_start(n);
     const int64_t sidx = n * H + h;
     const T* __restrict__ dout = (const T*)b.dout;
+    auto block_of = [&](int64_t ch) { return ws + ((gc0 + ch) * Hg + hl) * BW::size; };
+
+    auto load_a = [&](int64_t ch) {
+        const float* blk = block_of(ch);
+        for (int e = tid; e < C * DK / 4; e += kBT)
+            async16(sKh + (e / (DK / 4)) * KP + 4 * (e % (DK / 4)), blk + SW::KG + 4 * e);
+        for (int e = tid; e < C * C / 4; e += kBT) async16(sAqk + 4 * e, blk + SW::Aqk + 4 * e);
+    };
+    auto load_b = [&](int64_t ch) {
+        const float* blk = block_of(ch);
+        for (int e = tid; e < C * DK / 4; e += kBT) {
+            async16(sW + 4 * e, blk + SW::W + 4 * e);
+            async16(sQG + 4 * e, blk + SW::QG + 4 * e);
+        }
+        for (int e = tid; e < DK / 4; e += kBT) async16(sGam + 4 * e, blk + SW::Gam + 4 * e);
+    };
+    // the dO tile [C][TW] of one chunk: NV 16-byte loads per thread, rows past the end as zeros
+    constexpr int PER_ROW = TW / V::N, NV = C * PER_ROW / kBT;
+    static_assert(C * PER_ROW % kBT == 0, "the dO tile splits evenly over the block");
+    typename V::Raw rdo[NV];
+    auto fetch_do = [&](int64_t ch) {
+        const int64_t t0 = bos + ch * C;
+        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
+#pragma unroll
+        for (int x = 0; x < NV; ++x) {
+            const int e = tid + x * kBT, t = e / PER_ROW, j = (e % PER_ROW) * V::N;
+            if (t < len)
+                rdo[x] = *reinterpret_cast<const typename V::Raw*>(dout + ((t0 + t) * H + h) * DV + j0 + j);
+            else
+                rdo[x] = typename V::Raw{};
+        }
+    };
 
     constexpr int NCW = 8 / RG;                       // warps sharing one row group
-    constexpr int NJ = kTW / NCW;                     // columns per thread
+    constexpr int NJ = TW / NCW;                      // columns per thread
     const int c = 32 * (wrp % RG) + lane;
     const int jb = NJ * (wrp / RG);
     float ds[NJ];
@@ -89,57 +126,60 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     for (int x = 0; x < NJ; ++x)
         ds[x] = b.dhT ? b.dhT[sidx * DK * DV + (int64_t)c * DV + j0 + jb + x] : 0.f;
 
+    if (nchunks > 0) {
+        load_a(nchunks - 1);
+        fetch_do(nchunks - 1);
+    }
+    async_commit();
+    const int row0 = 8 * wrp + 4 * (lane >> 4), cp = lane & 15;   // tile42 rows and column pair
     for (int64_t ch = nchunks - 1; ch >= 0; --ch) {
-        float* blk = ws + ((gc0 + ch) * Hg + hl) * BW::size;
-        const int64_t t0 = bos + ch * C;
-        const int len = (int)((eos - t0) < C ? (eos - t0) : C);
-        __syncthreads();                              // previous chunk's reads are done
-        for (int e = tid; e < C * DK / 4; e += kBT)
-            reinterpret_cast<float4*>(sX)[e] = reinterpret_cast<const float4*>(blk + SW::KG)[e];
-        for (int e = tid; e < C * C; e += kBT) {
-            const int r = e / C, t = e % C;           // Aqk[r][t] -> AqkT[t][r]
-            sY[t * kAP + r] = blk[SW::Aqk + e];
+        float* blk = block_of(ch);
+        async_wait<0>();                              // Khat and Aqk of this chunk
+        // this chunk's dO tile and exit-state gradient into shared memory (dS' also to the
+        // workspace)
+#pragma unroll
+        for (int x = 0; x < NV; ++x) {
+            const int e = tid + x * kBT, t = e / PER_ROW, j = (e % PER_ROW) * V::N;
+            float o[V::N];
+            V::widen(rdo[x], o);
+#pragma unroll
+            for (int i = 0; i < V::N; i += 4)
+                *reinterpret_cast<float4*>(sdO + t * TW + j + i) = make_float4(o[i], o[i + 1], o[i + 2], o[i + 3]);
         }
-        for (int cc = tid; cc < DK; cc += kBT) sGam[cc] = blk[SW::Gam + cc];
-        for (int e = tid; e < C * kTW; e += kBT) {
-            const int t = e / kTW, j = e % kTW;
-            sdO[e] = t < len ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
-        }
-        // this chunk's exit-state gradient: to shared memory (for dE) and to the workspace
 #pragma unroll
         for (int x = 0; x < NJ; x += 4) {
             const float4 v4 = make_float4(ds[x], ds[x + 1], ds[x + 2], ds[x + 3]);
             *reinterpret_cast<float4*>(sdS + c * kSP + jb + x) = v4;
             *reinterpret_cast<float4*>(blk + BW::dSx + (int64_t)c * DV + j0 + jb + x) = v4;
         }
-        __syncthreads();
-        // dE = Aqk^T dO + Khat dS': rows t = w + 8 r, column lane
+        __syncthreads();                              // also: the previous chunk's dS update is done
+        load_b(ch);
+        async_commit();
+        if (ch > 0) fetch_do(ch - 1);
+        // dE = Aqk^T dO + Khat dS': 4 x 2 register tiles
         {
-            float acc[8];
+            float acc[4][2] = {};
+            tile42t_mac<C, TW>(acc, sAqk, row0, sdO, C, cp);
+            tile42_mac<KP, kSP>(acc, sKh, row0, sdS, DK, cp);
 #pragma unroll
-            for (int r = 0; r < 8; ++r) acc[r] = 0.f;
-            rows8_mac<kTW>(acc, sY, kAP, wrp, sdO, C, lane);
-            rows8_mac<kSP>(acc, sX, DK, wrp, sdS, DK, lane);
-#pragma unroll
-            for (int r = 0; r < 8; ++r) sdE[(wrp + 8 * r) * kTW + lane] = acc[r];
+            for (int i = 0; i < 4; ++i)
+                *reinterpret_cast<float2*>(sdE + (row0 + i) * TW + 2 * cp) = make_float2(acc[i][0], acc[i][1]);
         }
+        async_wait<0>();                              // W, Q_G, e^{G_last} of this chunk
         __syncthreads();
-        for (int e = tid; e < C * DK / 4; e += kBT) {
-            reinterpret_cast<float4*>(sX)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
-            reinterpret_cast<float4*>(sY)[e] = reinterpret_cast<const float4*>(blk + SW::QG)[e];
-        }
-        __syncthreads();
+        if (ch > 0) load_a(ch - 1);
+        async_commit();
         // dS = Diag(e^{G_last}) dS' + Q_G^T dO - W^T dE  (row c, columns jb .. jb + NJ - 1)
         {
             const float gmc = sGam[c];
 #pragma unroll
             for (int x = 0; x < NJ; ++x) ds[x] *= gmc;
             for (int t = 0; t < C; ++t) {
-                const float qg = sY[t * DK + c], wv = sX[t * DK + c];
+                const float qg = sQG[t * DK + c], wv = sW[t * DK + c];
 #pragma unroll
                 for (int x = 0; x < NJ; x += 4) {
-                    const float4 o4 = *reinterpret_cast<const float4*>(sdO + t * kTW + jb + x);
-                    const float4 e4 = *reinterpret_cast<const float4*>(sdE + t * kTW + jb + x);
+                    const float4 o4 = *reinterpret_cast<const float4*>(sdO + t * TW + jb + x);
+                    const float4 e4 = *reinterpret_cast<const float4*>(sdE + t * TW + jb + x);
                     ds[x] += qg * o4.x - wv * e4.x;
                     ds[x + 1] += qg * o4.y - wv * e4.y;
                     ds[x + 2] += qg * o4.z - wv * e4.z;
@@ -147,7 +187,9 @@ chunk_bwd_state_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
                 }
             }
         }
+        __syncthreads();                              // dO and dE reads done before the next chunk's writes
     }
+    async_wait<0>();
     if (b.dh0)
 #pragma unroll
         for (int x = 0; x < NJ; ++x) b.dh0[sidx * DK * DV + (int64_t)c * DV + j0 + jb + x] = ds[x];
@@ -585,7 +627,7 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
 }
 
 template <int DK, int DV>
-constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(2 * kChunk * (DK > kAP ? DK : kAP) + 2 * kChunk * kTW + DK * kSP + DK); }
+constexpr size_t bwd_state_smem() { return sizeof(float) * (size_t)(kChunk * (DK + 4) + kChunk * kChunk + 2 * kChunk * DK + DK + 2 * kChunk * kTW + DK * kSP); }
 template <int DK, int DV>
 constexpr size_t bwd_dense1_smem() { return sizeof(float) * (size_t)(3 * kChunk * DK + 2 * kChunk * kAP + 2 * DK * kTW + 4 * kChunk * kTW + kChunk); }
 template <int DK, int DV>

@@ -74,6 +74,23 @@ __device__ __forceinline__ void tile42_mac(float (&acc)[4][2], const float* A, i
     }
 }
 
+// The same with A read transposed: acc[i][x] += sum_k A[k * LDA + row0 + i] * B[k * LDB + 2 cp + x]
+// (the four rows of a thread are one 16-byte load per k).
+template <int LDA, int LDB>
+__device__ __forceinline__ void tile42t_mac(float (&acc)[4][2], const float* A, int row0,
+                                            const float* B, int K, int cp)
+{
+#pragma unroll 4
+    for (int k = 0; k < K; ++k) {
+        const float2 bv = *reinterpret_cast<const float2*>(B + k * LDB + 2 * cp);
+        const float4 a = *reinterpret_cast<const float4*>(A + k * LDA + row0);
+        acc[0][0] += a.x * bv.x; acc[0][1] += a.x * bv.y;
+        acc[1][0] += a.y * bv.x; acc[1][1] += a.y * bv.y;
+        acc[2][0] += a.z * bv.x; acc[2][1] += a.z * bv.y;
+        acc[3][0] += a.w * bv.x; acc[3][1] += a.w * bv.y;
+    }
+}
+
 // Workspace block of one (chunk, head), in floats.
 template <int DK, int DV>
 struct SimtWs {
