@@ -147,7 +147,7 @@ constexpr size_t simt_state_smem()
 // ---------------------------------------------------------------------------
 // step a + b: cumulative log-decay and intra-chunk transform
 // ---------------------------------------------------------------------------
-constexpr int kSimtPrepThreads = 256;   // 16 rows x 16 column lanes in the A / Aqk phase
+constexpr int kSimtPrepThreads = 512;   // 16 warps: one CTA per SM (shared memory), so more warps hide latency
 
 // One 16-byte global load of I/O elements, widened to fp32.
 template <typename T> struct Vec16;
@@ -261,9 +261,9 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
         sT[e] = 0.f;
         if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + e] = 0.f;
     }
-    // diagonal-block work split: threads 0..239 take the 120 pairs i > j of a 16-row
-    // block, two threads per pair (one channel half each, partner = lane ^ 1); threads
-    // 240..255 take the 16 diagonal entries of Aqk, where the decay factor is 1
+    // pairwise diagonal blocks: threads 0..239 take the 120 pairs i > j of a 16-row block,
+    // two threads per pair (one channel half each, partner = lane ^ 1); threads 240..255
+    // take the 16 diagonal entries of Aqk, where the decay factor is 1; the rest idle
     constexpr int kPairThreads = 240, HALF = DK / 2;
     int pi = 0, pj = 0;
     if (tid < kPairThreads) {
@@ -271,7 +271,7 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
         pi = 1;
         while (m >= pi) { m -= pi; ++pi; }
         pj = m;
-    } else {
+    } else if (tid < 256) {
         pi = pj = tid - kPairThreads;
     }
     constexpr float kMaxBlockDecay = 64.f;
@@ -294,11 +294,12 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
         }
         __syncthreads();
         const int nu = pairwise ? p : p + 1;      // column blocks taken as dot products
-        if (nu > 0) {  // rows f .. f+15 (r = tid / 16), columns jg + 16 u; lanes run along
-                       // the columns (padded Kvar rows), the row is a broadcast
-            const int r = tid >> 4, jg = tid & 15, i = f + r;
+        if (nu > 0) {  // row f + w of warp w, columns jg + 16 u (lane = 16 half + jg); lanes run
+                       // along the columns (padded Kvar rows), the row is a broadcast; the two
+                       // half-warps take one channel half each and meet by a shuffle
+            const int r = tid >> 5, jg = lane & 15, i = f + r, c0 = (lane >> 4) * (DK / 2);
             float kk[4] = {0.f, 0.f, 0.f, 0.f}, qk[4] = {0.f, 0.f, 0.f, 0.f};
-            for (int c = 0; c < DK; c += 4) {
+            for (int c = c0; c < c0 + DK / 2; c += 4) {
                 const float4 a = *reinterpret_cast<const float4*>(sKin + r * DK + c);
                 const float4 q4 = *reinterpret_cast<const float4*>(sQin + r * DK + c);
 #pragma unroll
@@ -312,8 +313,13 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
             }
 #pragma unroll
             for (int u = 0; u < 4; ++u) {
+                kk[u] += __shfl_xor_sync(0xffffffffu, kk[u], 16);
+                qk[u] += __shfl_xor_sync(0xffffffffu, qk[u], 16);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
                 const int j = jg + 16 * u;
-                if (u < nu && j <= i) {           // (the diagonal block: its lower half only)
+                if (lane < 16 && u < nu && j <= i) {   // (the diagonal block: its lower half only)
                     if (j < i) {
                         sA[i * C + j] = sB[i] * kk[u];
                         if constexpr (kBwd) blk[BwdWs<DK, DV>::Ap + i * C + j] = kk[u];
@@ -322,8 +328,8 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                 }
             }
         }
-        if (pairwise) {   // diagonal block, pairwise; the channel order is rotated by the lane
-                          // so that the 32 lanes of a warp hit 32 distinct banks
+        if (pairwise && tid < 256) {   // diagonal block, pairwise; the channel order is rotated
+                                       // by the lane so that the 32 lanes of a warp hit 32 banks
             const int i = f + pi, j = f + pj;
             float dk_ = 0.f, dq_ = 0.f;
             if (tid < kPairThreads) {
@@ -400,14 +406,15 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
         for (int e = tid - 64; e < C * DV; e += NT - 64) sV[e] *= sB[e / DV];
     }
     // Off-diagonal blocks by distance d = p - r: T_pr = -T_pp sum_{m=r}^{p-1} A_pm T_mr,
-    // whose factors all lie at distances below d.  Thread (a, b) owns entry (a, b) of each
-    // block of the level; the partial sums go through sKin.
+    // whose factors all lie at distances below d.  Thread (a, b) < 256 owns entry (a, b) of
+    // each block of the level; the partial sums go through sKin.
     {
-        const int a = tid >> 4, b = tid & 15;
+        const int a = (tid >> 4) & 15, b = tid & 15;
+        const bool act = tid < 256;
         float* sX = sKin;                         // [3][16][16]
         for (int d = 1; d < 4; ++d) {
             __syncthreads();                      // level d - 1 (or the diagonal) written
-            for (int r = 0; r + d < 4; ++r) {
+            for (int r = 0; act && r + d < 4; ++r) {
                 const int p = r + d;
                 float x = 0.f;
                 for (int m = r; m < p; ++m) {
@@ -421,7 +428,7 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                 sX[r * 256 + a * 16 + b] = x;
             }
             __syncthreads();
-            for (int r = 0; r + d < 4; ++r) {
+            for (int r = 0; act && r + d < 4; ++r) {
                 const int p = r + d;
                 float y = 0.f;
 #pragma unroll
@@ -443,31 +450,31 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
     }
 
     // (b3) [W | Ut] = T [beta K e^G | beta V], register-tiled: thread (g, cg) owns rows
-    // 2g, 2g+1 (which need columns j <= 2g+1 of T) and 62-2g, 63-2g (j <= 63-2g), so all
-    // threads do the same number of products, and 16-byte column groups 4 cg + 64 u.
+    // g (which needs columns j <= g of T) and 63 - g (j <= 63 - g), so all threads do the
+    // same number of products, and 16-byte column groups 4 cg + 64 u.
     {
         constexpr int NU = (DK + DV) / 64;
         const int g = tid >> 4, cg = tid & 15;
-        const int row[4] = {2 * g, 2 * g + 1, 62 - 2 * g, 63 - 2 * g};
-        const int jl = (2 * g + 2 + 3) & ~3;
-        const int jh = (64 - 2 * g + 3) & ~3;
-        float4 acc[4][NU];
+        const int row[2] = {g, 63 - g};
+        const int jl = (g + 1 + 3) & ~3;
+        const int jh = (64 - g + 3) & ~3;
+        float4 acc[2][NU];
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
+        for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
             for (int u = 0; u < NU; ++u) acc[rr][u] = make_float4(0.f, 0.f, 0.f, 0.f);
         auto bcol = [&](int u, int j) -> float4 {
             return 64 * u < DK ? *reinterpret_cast<const float4*>(sQ + j * DK + 64 * u + 4 * cg)
                                : *reinterpret_cast<const float4*>(sV + j * DV + 64 * u - DK + 4 * cg);
         };
-        auto step = [&](int j, const float (&tj)[4][4], int r0) {
+        auto step = [&](int j, const float (&tj)[2][4], int r0) {
 #pragma unroll
             for (int jj = 0; jj < 4; ++jj)
 #pragma unroll
                 for (int u = 0; u < NU; ++u) {
                     const float4 bv = bcol(u, j + jj);
 #pragma unroll
-                    for (int rr = 0; rr < 4; ++rr) {
+                    for (int rr = 0; rr < 2; ++rr) {
                         if (rr < r0) continue;
                         const float t = tj[rr][jj];
                         acc[rr][u].x += t * bv.x;
@@ -478,25 +485,22 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                 }
         };
         for (int j = 0; j < jl; j += 4) {
-            float tj[4][4];
+            float tj[2][4];
 #pragma unroll
-            for (int rr = 0; rr < 4; ++rr) {
+            for (int rr = 0; rr < 2; ++rr) {
                 const float4 t4 = *reinterpret_cast<const float4*>(sT + row[rr] * C + j);
                 tj[rr][0] = t4.x; tj[rr][1] = t4.y; tj[rr][2] = t4.z; tj[rr][3] = t4.w;
             }
             step(j, tj, 0);
         }
         for (int j = jl; j < jh; j += 4) {
-            float tj[4][4] = {};
-#pragma unroll
-            for (int rr = 2; rr < 4; ++rr) {
-                const float4 t4 = *reinterpret_cast<const float4*>(sT + row[rr] * C + j);
-                tj[rr][0] = t4.x; tj[rr][1] = t4.y; tj[rr][2] = t4.z; tj[rr][3] = t4.w;
-            }
-            step(j, tj, 2);
+            float tj[2][4] = {};
+            const float4 t4 = *reinterpret_cast<const float4*>(sT + row[1] * C + j);
+            tj[1][0] = t4.x; tj[1][1] = t4.y; tj[1][2] = t4.z; tj[1][3] = t4.w;
+            step(j, tj, 1);
         }
 #pragma unroll
-        for (int rr = 0; rr < 4; ++rr)
+        for (int rr = 0; rr < 2; ++rr)
 #pragma unroll
             for (int u = 0; u < NU; ++u) {
                 float* dst = 64 * u < DK ? blk + SimtWs<DK, DV>::W + row[rr] * DK + 64 * u + 4 * cg
