@@ -233,6 +233,27 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
     const T* __restrict__ v = (const T*)b.v;
     T* __restrict__ dv = (T*)b.dv;
 
+    // the per-tile operands (S, dS', dO, V, Ut columns j0 .. j0 + 31) go through registers
+    // one tile ahead, so their loads run under the previous tile's products
+    constexpr int NS = DK * kTW / kD1T, NO = C * kTW / kD1T;
+    float rS[NS], rdS[NS], rdO[NO], rV[NO], rU[NO];
+    auto fetch = [&](int j0) {
+#pragma unroll
+        for (int x = 0; x < NS; ++x) {
+            const int e = tid + x * kD1T, c = e / kTW, j = e % kTW;
+            rS[x] = blk[BW::Sx + c * DV + j0 + j];
+            rdS[x] = blk[BW::dSx + c * DV + j0 + j];
+        }
+#pragma unroll
+        for (int x = 0; x < NO; ++x) {
+            const int e = tid + x * kD1T, t = e / kTW, j = e % kTW;
+            const bool ok = t < len;
+            rdO[x] = ok ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+            rV[x] = ok ? IO<T>::load(v, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
+            rU[x] = blk[SW::Ut + t * DV + j0 + j];
+        }
+    };
+    fetch(0);
     for (int e = tid; e < C * DK / 4; e += kD1T) {
         reinterpret_cast<float4*>(sW)[e] = reinterpret_cast<const float4*>(blk + SW::W)[e];
         reinterpret_cast<float4*>(sKG)[e] = reinterpret_cast<const float4*>(blk + BW::KGm)[e];
@@ -247,21 +268,22 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
     }
     float glS = 0.f;                                  // thread c < DK: sum_v S[c][v] dS'[c][v]
 
+#pragma unroll 1
     for (int j0 = 0; j0 < DV; j0 += kTW) {
         __syncthreads();
-        for (int e = tid; e < DK * kTW; e += kD1T) {
-            const int c = e / kTW, j = e % kTW;
-            sS[e] = blk[BW::Sx + c * DV + j0 + j];
-            sdSn[e] = blk[BW::dSx + c * DV + j0 + j];
+#pragma unroll
+        for (int x = 0; x < NS; ++x) {
+            sS[tid + x * kD1T] = rS[x];
+            sdSn[tid + x * kD1T] = rdS[x];
         }
-        for (int e = tid; e < C * kTW; e += kD1T) {
-            const int t = e / kTW, j = e % kTW;
-            const bool ok = t < len;
-            sdO[e] = ok ? IO<T>::load(dout, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
-            sV[e] = ok ? IO<T>::load(v, ((t0 + t) * H + h) * DV + j0 + j) : 0.f;
-            sUt[e] = blk[SW::Ut + t * DV + j0 + j];
+#pragma unroll
+        for (int x = 0; x < NO; ++x) {
+            sdO[tid + x * kD1T] = rdO[x];
+            sV[tid + x * kD1T] = rV[x];
+            sUt[tid + x * kD1T] = rU[x];
         }
         __syncthreads();
+        if (j0 + kTW < DV) fetch(j0 + kTW);
         if (tid < DK)                                 // (column order rotated by the row: no bank conflicts)
             for (int jj = 0; jj < kTW; ++jj) {
                 const int j = (jj + tid) % kTW;
