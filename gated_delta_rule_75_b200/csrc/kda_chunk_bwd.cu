@@ -330,8 +330,7 @@ chunk_bwd_dense1_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
 //   3: dT'  =  dE R^T   4: dAqk = dO E^T (kept for m <= i)       (m < C)
 // ---------------------------------------------------------------------------
 template <typename T, int DK, int DV>
-__global__ void __launch_bounds__(kBT, 4)   // four CTAs per SM hide the tile loads (64 registers;
-                                             // an 8-byte spill, still the fastest bound measured)
+__global__ void __launch_bounds__(kBT, 4)   // four CTAs per SM hide the tile loads (64 registers)
 chunk_bwd_dense2_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, int64_t Hg)
 {
     using BW = BwdWs<DK, DV>;
@@ -373,16 +372,27 @@ chunk_bwd_dense2_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, 
 
     for (int v0 = 0; v0 < DV; v0 += kTW) {
         __syncthreads();
-        for (int e = tid; e < C * kTW; e += kBT) {
-            const int i = e / kTW, j = e % kTW;
-            float x;
-            if (a_is_dO) x = i < len ? IO<T>::load(dout, ((t0 + i) * H + h) * DV + v0 + j) : 0.f;
-            else x = Ag[i * DV + v0 + j];
-            sA[i * P + j] = x;
+        // 16-byte loads (four columns), scattered into the padded rows
+        for (int e4 = tid; e4 < C * kTW / 4; e4 += kBT) {
+            const int i = e4 / (kTW / 4), j = 4 * (e4 % (kTW / 4));
+            float4 x;
+            if (a_is_dO) {
+                const bool ok = i < len;
+                const int64_t o = ((t0 + i) * H + h) * DV + v0 + j;
+                x = ok ? make_float4(IO<T>::load(dout, o), IO<T>::load(dout, o + 1),
+                                     IO<T>::load(dout, o + 2), IO<T>::load(dout, o + 3))
+                       : make_float4(0.f, 0.f, 0.f, 0.f);
+            } else {
+                x = *reinterpret_cast<const float4*>(Ag + i * DV + v0 + j);
+            }
+            float* d = sA + i * P + j;
+            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
         }
-        for (int e = tid; e < M * kTW; e += kBT) {
-            const int m = e / kTW, j = e % kTW;
-            sBm[m * P + j] = Bg[m * DV + v0 + j];
+        for (int e4 = tid; e4 < M * kTW / 4; e4 += kBT) {
+            const int m = e4 / (kTW / 4), j = 4 * (e4 % (kTW / 4));
+            const float4 x = *reinterpret_cast<const float4*>(Bg + m * DV + v0 + j);
+            float* d = sBm + m * P + j;
+            d[0] = x.x; d[1] = x.y; d[2] = x.z; d[3] = x.w;
         }
         __syncthreads();
         for (int j = 0; j < kTW; ++j) {
@@ -450,19 +460,37 @@ chunk_bwd_param_kernel(float* __restrict__ ws, BackwardArgs b, int64_t h_base, i
     const T* __restrict__ k = (const T*)b.k;
     const float scale = b.scale;
 
-    for (int e = tid; e < C * DK; e += kPT) {
-        const int t = e / DK, c = e % DK;
-        const bool ok = t < len;
-        const int64_t src = ((t0 + t) * H + h) * DK + c;
-        sK[e] = ok ? IO<T>::load(k, src) : 0.f;
-        sQ[e] = ok ? IO<T>::load(q, src) : 0.f;
-        sG[e] = ok ? b.log_alpha[b.gate_scalar ? (t0 + t) * H + h : src] : 0.f;
+    // inputs by 16-byte loads, all of a thread's issued before the first is used
+    load_rows<T, DK, kPT>(sK, k, t0, len, H, h, tid);
+    load_rows<T, DK, kPT>(sQ, q, t0, len, H, h, tid);
+    if (b.gate_scalar) {
+        for (int e = tid; e < C * DK; e += kPT) {
+            const int t = e / DK;
+            sG[e] = t < len ? b.log_alpha[(t0 + t) * H + h] : 0.f;
+        }
+    } else {
+        load_rows<float, DK, kPT>(sG, b.log_alpha, t0, len, H, h, tid);
     }
-    for (int e = tid; e < C * C; e += kPT) {
-        sT[(e / C) * TP + e % C] = blk[BW::Tm + e];
-        sAp[e] = blk[BW::Ap + e];
-        sdT[e] = blk[BW::dTp + e];
-        sdAqk[e] = blk[BW::dAqk + e];
+    {
+        constexpr int N4 = C * C / 4 / kPT;
+        float4 rt[N4], ra[N4], rd[N4], rq[N4];
+#pragma unroll
+        for (int x = 0; x < N4; ++x) {
+            const int e4 = tid + x * kPT;
+            rt[x] = reinterpret_cast<const float4*>(blk + BW::Tm)[e4];
+            ra[x] = reinterpret_cast<const float4*>(blk + BW::Ap)[e4];
+            rd[x] = reinterpret_cast<const float4*>(blk + BW::dTp)[e4];
+            rq[x] = reinterpret_cast<const float4*>(blk + BW::dAqk)[e4];
+        }
+#pragma unroll
+        for (int x = 0; x < N4; ++x) {
+            const int e = 4 * (tid + x * kPT), r = e / C, c = e % C;
+            sT[r * TP + c] = rt[x].x; sT[r * TP + c + 1] = rt[x].y;
+            sT[r * TP + c + 2] = rt[x].z; sT[r * TP + c + 3] = rt[x].w;
+            reinterpret_cast<float4*>(sAp)[e / 4] = ra[x];
+            reinterpret_cast<float4*>(sdT)[e / 4] = rd[x];
+            reinterpret_cast<float4*>(sdAqk)[e / 4] = rq[x];
+        }
     }
     for (int t = tid; t < C; t += kPT) sB[t] = t < len ? b.beta[(t0 + t) * H + h] : 0.f;
     __syncthreads();
