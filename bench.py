@@ -367,6 +367,12 @@ def kernel_algorithmic_bytes(kname, cfg):
 TC_WS_BYTES_PER_CHUNK = 66560         # per (chunk, head) operand image of the tensor-core path
 
 
+def decode_bytes_per_head_step(cfg):
+    """Bytes one decode step must move per (sequence, head): the fp32 state read and
+    written, q and k (bf16), v (bf16), log_alpha (fp32), beta, and the bf16 output."""
+    return 2 * cfg.dk * cfg.dv * 4 + 2 * cfg.dk * 2 + cfg.dv * 2 + cfg.dk * 4 + 4 + cfg.dv * 2
+
+
 def run_decode(args, ws, rank, kda, peaks):
     cfg = W.DECODE
     if args.decode_steps != cfg.steps:
@@ -394,8 +400,7 @@ def run_decode(args, ws, rank, kda, peaks):
     kda.profiler_enable(False)
     stats = kda.profiler_read(reset=True)
     ms = max_over_ranks(ms, ws)
-    per_head = 2 * cfg.dk * cfg.dv * 4 + 2 * cfg.dk * 2 + cfg.dv * 2 + cfg.dk * 4 + 4 + cfg.dv * 2
-    bytes_step = per_head * cfg.N * cfg.H
+    bytes_step = decode_bytes_per_head_step(cfg) * cfg.N * cfg.H
     launches, timed, kms = stats["decode_step"]
     gbs = bytes_step / (kms / max(1, timed) / 1e3) / 1e9
     # the same chained loop captured once as a CUDA graph and replayed (no per-step launch cost)
