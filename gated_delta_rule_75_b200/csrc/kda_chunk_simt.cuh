@@ -587,13 +587,17 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     const int64_t sidx = a.state_index(n, h);
     const float* h0p = (a.h0 && sidx >= 0) ? a.h0 + sidx * DK * DV : nullptr;
     float* hTp = (a.hT && sidx >= 0) ? a.hT + sidx * DK * DV : nullptr;
-    // the state tile lives in registers: thread (warp w, lane) owns row c = 32 (w mod DK/32)
-    // + lane and NJ consecutive columns (NJ = 16 for DK = 128, 8 for DK = 64)
-    constexpr int RG = DK / 32, NJ = TW / (8 / RG);
-    const int c = 32 * (wrp % RG) + lane, jb = NJ * (wrp / RG);
-    float st[NJ];
+    // the state tile lives in registers: thread (warp w, lane) owns rows c_r = 64 (w mod DK/64)
+    // + lane + 32 r, r < 2, and NJ consecutive columns (NJ = 8 for DK = 128, 4 for DK = 64):
+    // per token of the update two key loads and NJ / 4 broadcast loads of U feed 2 NJ FMAs
+    constexpr int RG = DK / 64, NJ = TW / (8 / RG);
+    const int cb = 64 * (wrp % RG) + lane, jb = NJ * (wrp / RG);
+    const int crow[2] = {cb, cb + 32};
+    float st[2][NJ];
 #pragma unroll
-    for (int x = 0; x < NJ; ++x) st[x] = h0p ? h0p[(int64_t)c * DV + j0 + jb + x] : 0.f;
+    for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int x = 0; x < NJ; ++x) st[r][x] = h0p ? h0p[(int64_t)crow[r] * DV + j0 + jb + x] : 0.f;
 
     if (nchunks > 0) {
         load_ut(0);
@@ -610,12 +614,14 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
         const int len = (int)((eos - t0) < C ? (eos - t0) : C);
         async_wait<1>();                          // Ut and W of this chunk
 #pragma unroll
-        for (int x = 0; x < NJ; x += 4) {
-            const float4 v4 = make_float4(st[x], st[x + 1], st[x + 2], st[x + 3]);
-            *reinterpret_cast<float4*>(sS + c * kSP + jb + x) = v4;
-            if constexpr (kBwd)
-                *reinterpret_cast<float4*>(blk + BwdWs<DK, DV>::Sx + (int64_t)c * DV + j0 + jb + x) = v4;
-        }
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int x = 0; x < NJ; x += 4) {
+                const float4 v4 = make_float4(st[r][x], st[r][x + 1], st[r][x + 2], st[r][x + 3]);
+                *reinterpret_cast<float4*>(sS + crow[r] * kSP + jb + x) = v4;
+                if constexpr (kBwd)
+                    *reinterpret_cast<float4*>(blk + BwdWs<DK, DV>::Sx + (int64_t)crow[r] * DV + j0 + jb + x) = v4;
+            }
         __syncthreads();                          // also: the previous chunk's state update is done
         load_kg(ch);
         if (ch + 1 < nchunks) load_ut(ch + 1);
@@ -658,18 +664,25 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
         async_commit();
         // S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U, in registers
         {
-            const float gmc = sGam[c];
 #pragma unroll
-            for (int x = 0; x < NJ; ++x) st[x] *= gmc;
+            for (int r = 0; r < 2; ++r) {
+                const float gmc = sGam[crow[r]];
+#pragma unroll
+                for (int x = 0; x < NJ; ++x) st[r][x] *= gmc;
+            }
             for (int t = 0; t < C; ++t) {
-                const float kg = sKG[t * DK + c];
+                const float kg0 = sKG[t * DK + crow[0]], kg1 = sKG[t * DK + crow[1]];
 #pragma unroll
                 for (int x = 0; x < NJ; x += 4) {
                     const float4 u4 = *reinterpret_cast<const float4*>(sU + t * TW + jb + x);
-                    st[x] += kg * u4.x;
-                    st[x + 1] += kg * u4.y;
-                    st[x + 2] += kg * u4.z;
-                    st[x + 3] += kg * u4.w;
+                    st[0][x] += kg0 * u4.x;
+                    st[0][x + 1] += kg0 * u4.y;
+                    st[0][x + 2] += kg0 * u4.z;
+                    st[0][x + 3] += kg0 * u4.w;
+                    st[1][x] += kg1 * u4.x;
+                    st[1][x + 1] += kg1 * u4.y;
+                    st[1][x + 2] += kg1 * u4.z;
+                    st[1][x + 3] += kg1 * u4.w;
                 }
             }
         }
@@ -678,7 +691,9 @@ chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, i
     async_wait<0>();
     if (hTp)
 #pragma unroll
-        for (int x = 0; x < NJ; ++x) hTp[(int64_t)c * DV + j0 + jb + x] = st[x];
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int x = 0; x < NJ; ++x) hTp[(int64_t)crow[r] * DV + j0 + jb + x] = st[r][x];
 }
 
 }  // namespace kda
