@@ -18,10 +18,11 @@
 // WY/UT transform, parallel over (chunk, head)) writes W, Ut, Aqk, Q e^G,
 // K e^{G_last-G} and e^{G_last} to an fp32 workspace; `state` (steps c and d)
 // walks the chunks of one (sequence, head, 32-column dv tile) in order with the
-// state tile in shared memory and writes the output.  Exponentials here are
-// taken pairwise (e^{G_i - G_j}), so this path has no limit on the decay rate.
-// It is the reference-quality GPU path: fp32 I/O and the bisection baseline of
-// the tensor-core kernels.
+// state tile in registers and writes the output.  Every exponential is either a
+// factor <= 1 or, inside a 16-token diagonal block, bounded by 64 nats of decay;
+// blocks that decay faster are taken pairwise (e^{G_i - G_j}), so this path has
+// no limit on the decay rate.  It is the reference-quality GPU path: fp32 I/O
+// and the bisection baseline of the tensor-core kernels.
 #include "kda_chunk_simt.cuh"
 
 namespace kda {
