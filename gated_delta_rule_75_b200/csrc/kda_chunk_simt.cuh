@@ -44,14 +44,6 @@ __device__ __forceinline__ void rows_mac(float (&acc)[NR], const float* A, int l
     }
 }
 
-// The eight-warp form: rows row0 + 8 r, r < 8.
-template <int LDB = kTW>
-__device__ __forceinline__ void rows8_mac(float (&acc)[8], const float* A, int lda, int row0,
-                                          const float* B, int K, int lane)
-{
-    rows_mac<8, 8, LDB>(acc, A, lda, row0, B, K, lane);
-}
-
 // acc[i][x] += sum_k A[(row0 + i) * LDA + k] * B[k * LDB + 2 cp + x], i < 4, x < 2, K a
 // multiple of 4: four rows by two columns per thread.  With the lanes of a warp split
 // into two row groups (row0 four rows apart) and 16 column pairs, each 16-byte row load
