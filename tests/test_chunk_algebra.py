@@ -262,3 +262,111 @@ def test_chunk_backward_equals_oracle(L):
     ref = [r[0, :, 0] for r in ref[:5]] + [ref[5][0, 0]]
     for a, r in zip(got, ref):
         np.testing.assert_allclose(a, r, rtol=1e-9, atol=1e-10)
+
+
+# --------------------------------------------------------------------------
+# Exponent references of the fused tensor-core prep (what it multiplies out)
+# --------------------------------------------------------------------------
+# The pairwise factor e^{G_ic - G_jc} of A and Aqk becomes a matrix product once
+# it is split as e^{G_ic - R_c} e^{R_c - G_jc} around a reference row R.  The
+# fused prep takes one reference for the whole chunk, the last token of its
+# first half (row 31), whenever every |G_tc - R_c| stays within RANGE_LOG2
+# (log2 units; the margin below the fp32 exponent range keeps the factors <= 1
+# of small key components normal).  Otherwise it takes the lower triangle
+# level by level: at level l the chunk is cut into blocks of 2s rows
+# (s = 32, 16, ..., 1); a pair i > j belongs to the level where i is in the
+# upper half of a block and j in its lower half, and both factors are
+# referenced to the first row f of that upper half, so e^{G_i - G_f} <= 1 and
+# e^{G_f - G_j} <= 1 for every channel, at any decay rate.  One product per level
+# covers every block (entries across blocks are not used), and a last product
+# without exponents gives the diagonal of Aqk.
+RANGE_LOG2 = 100.0
+REF_FAST = 31
+
+
+def _pairwise(qc, kc, gc):
+    G = np.cumsum(gc, axis=0)
+    E = np.exp(G[:, None, :] - G[None, :, :])
+    Akk = np.einsum("ic,jc,ijc->ij", kc, kc, E)
+    Aqk = np.einsum("ic,jc,ijc->ij", qc, kc, E)
+    return np.tril(Akk, -1), np.tril(Aqk, 0)
+
+
+def _fast_needs_fallback(gc):
+    G = np.cumsum(gc, axis=0)
+    return np.abs(G - G[REF_FAST]).max() / np.log(2.0) > RANGE_LOG2
+
+
+def _single_reference(qc, kc, gc, dtype=np.float64):
+    G = np.cumsum(gc, axis=0)
+    x = (G - G[REF_FAST]).astype(dtype)
+    Kin, Qin, Kd = kc * np.exp(x), qc * np.exp(x), kc * np.exp(-x)
+    return np.tril(Kin @ Kd.T, -1), np.tril(Qin @ Kd.T, 0), (Kin, Qin, Kd)
+
+
+def _level_passes(qc, kc, gc, dtype=np.float64):
+    """The fallback: returns A (strictly lower), Aqk (lower) and the exponents
+    of every factor used."""
+    G = np.cumsum(gc, axis=0)
+    t = np.arange(C)
+    Akk = np.zeros((C, C))
+    Aqk = np.zeros((C, C))
+    exps = []
+    s = C // 2
+    while s >= 1:
+        upper = (t % (2 * s)) >= s
+        f = (t // (2 * s)) * 2 * s + s                       # first row of the block's upper half
+        x = (G - G[f]).astype(dtype)
+        Kin = np.where(upper[:, None], kc * np.exp(x), 0.0)
+        Qin = np.where(upper[:, None], qc * np.exp(x), 0.0)
+        Kd = np.where(upper[:, None], 0.0, kc * np.exp(-x))
+        Dk, Dq = Kin @ Kd.T, Qin @ Kd.T
+        pair = upper[:, None] & ~upper[None, :] & ((t // (2 * s))[:, None] == (t // (2 * s))[None, :])
+        Akk[pair] = Dk[pair]
+        Aqk[pair] = Dq[pair]
+        exps += [x[upper], -x[~upper]]
+        s //= 2
+    Aqk[t, t] = np.einsum("ic,ic->i", qc, kc)                # diagonal: no exponent
+    return np.tril(Akk, -1), Aqk, exps
+
+
+@pytest.mark.parametrize("shift", [-2.0, 0.0])
+def test_single_reference_reproduces_pairs(shift):
+    """The workload's gate distributions stay inside the one-reference range
+    and the factored products equal the pairwise sums."""
+    rng = np.random.default_rng(50)
+    q, k, v, g, b = _inputs(rng, C, 128, 4, gate_shift=shift)
+    assert not _fast_needs_fallback(g)
+    A_ref, Aqk_ref = _pairwise(q, k, g)
+    A, Aqk, _ = _single_reference(q, k, g)
+    np.testing.assert_allclose(A, A_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Aqk, Aqk_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("shift", [8.0, 40.0])
+def test_level_fallback_under_fast_decay(shift):
+    """About 8 (and 40) nats of decay per token: the one-reference factors
+    leave the fp32 range, so the prep must switch; every factor of the level
+    passes is <= 1, and their products still equal the pairwise sums."""
+    rng = np.random.default_rng(51)
+    q, k, v, g, b = _inputs(rng, C, 128, 4, gate_shift=shift)
+    assert _fast_needs_fallback(g)
+    with np.errstate(over="ignore"):
+        _, _, f32 = _single_reference(q, k, g, dtype=np.float32)
+    assert not all(np.all(np.isfinite(f)) for f in f32)
+    with np.errstate(under="ignore"):
+        A_ref, Aqk_ref = _pairwise(q, k, g)
+        A, Aqk, exps = _level_passes(q, k, g)
+    assert all(np.all(x <= 0.0) for x in exps)
+    np.testing.assert_allclose(A, A_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Aqk, Aqk_ref, rtol=0, atol=1e-12)
+
+
+def test_level_fallback_slow_decay():
+    """The level passes are exact at slow decay too, and cover each pair once."""
+    rng = np.random.default_rng(52)
+    q, k, v, g, b = _inputs(rng, C, 32, 4, gate_shift=-4.0)
+    A_ref, Aqk_ref = _pairwise(q, k, g)
+    A, Aqk, _ = _level_passes(q, k, g)
+    np.testing.assert_allclose(A, A_ref, rtol=0, atol=1e-12)
+    np.testing.assert_allclose(Aqk, Aqk_ref, rtol=0, atol=1e-12)
