@@ -26,7 +26,7 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_NO_MEMOR
     KDA_ERR_TIMEOUT = range(6)
 _IO = {torch.float32: 0, torch.bfloat16: 1}
 _IMPL = {"auto": 0, "simt": 1, "tensorcore": 2, "tensorcore_chain": 3,
-         "tensorcore_segmented": 4}
+         "tensorcore_segmented": 4, "tensorcore_fused": 5}
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libkda.so")
 

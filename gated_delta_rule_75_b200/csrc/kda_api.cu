@@ -282,8 +282,12 @@ static SegPlan plan_segments(const SeqInfo& si, int64_t H, kda_prefill_impl_t im
 {
     SegPlan p;
     std::memset(&p, 0, sizeof(p));
-    if (impl == KDA_PREFILL_TENSORCORE_CHAIN || si.chunks_upper <= 0) return p;
-    const bool force = impl == KDA_PREFILL_TENSORCORE_SEGMENTED;
+    if (impl == KDA_PREFILL_TENSORCORE_CHAIN || impl == KDA_PREFILL_TENSORCORE_FUSED ||
+        si.chunks_upper <= 0)
+        return p;
+    // AUTO and TENSORCORE run the fused kernel; only an explicit request segments
+    if (impl != KDA_PREFILL_TENSORCORE_SEGMENTED) return p;
+    const bool force = true;
     const int64_t sms = device_sm_count();
     const int64_t chains = si.N * H;
     if (!force && chains * 4 > sms) return p;
@@ -321,7 +325,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if (B < 0 || T < 0 || H < 0) return KDA_ERR_INVALID_ARG;
     if (io_dtype != KDA_IO_F32 && io_dtype != KDA_IO_BF16) return KDA_ERR_UNSUPPORTED;
     if (!head_ok(dk) || !head_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (impl < KDA_PREFILL_AUTO || impl > KDA_PREFILL_TENSORCORE_SEGMENTED)
+    if (impl < KDA_PREFILL_AUTO || impl > KDA_PREFILL_TENSORCORE_FUSED)
         return KDA_ERR_INVALID_ARG;
     // the tensor-core kernels address token rows with 32-bit TMA coordinates
     const int64_t T_rows = cu_seqlens ? T : B * T;
@@ -394,12 +398,17 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         if (plan.upper > 0x7fffffffLL / H) std::memset(&plan, 0, sizeof(plan));
     }
     const bool seg_table = use_tc && !segmap && plan.len > 0 && cu_seqlens != nullptr;
+    // the fused kernel (KDA form, outputs wanted, tokens present, no segmentation): it
+    // builds every chunk's operands on chip, so it needs no per-chunk workspace
+    const bool use_fused = use_tc && !segmap && !gate_scalar && T_total > 0 && plan.len == 0 &&
+                           impl != KDA_PREFILL_TENSORCORE_CHAIN;
 
     // workspace: [1 KiB header (error word) | chunk offsets (+ length order,
     // + segment offsets) | per head group: per-(chunk, head) blocks, segment
     // buffers | SIMT segmap extras]
     const int64_t blk_bytes =
-        use_tc ? tc_ws_bytes_per_chunk()
+        use_fused ? 0
+        : use_tc ? tc_ws_bytes_per_chunk()
                : simt_ws_floats_per_chunk((int)dk, (int)(segmap && dk > dv ? dk : dv)) *
                      (int64_t)sizeof(float);
     const bool ordered = cu_seqlens != nullptr && B <= kMaxOrderedSeqs && !seg_table;
@@ -407,7 +416,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         cu_seqlens ? ((B + 1) * 8 + (ordered ? B * 4 : 0) + (seg_table ? (B + 1) * 8 : 0) + 1023) /
                          1024 * 1024
                    : 0;
-    const int64_t seg_bytes = (use_tc && !segmap) ? tc_seg_bytes_per_head(plan) : 0;
+    const int64_t seg_bytes = (use_tc && !segmap && !use_fused) ? tc_seg_bytes_per_head(plan) : 0;
     const int64_t per_head = blk_bytes * (si.chunks_upper > 0 ? si.chunks_upper : 1) + seg_bytes;
     // SIMT segmap: zero values [T, H, dk], scratch outputs [T, H, max(dk, dv)],
     // identity initial states [N, H, dk, dk]
@@ -421,7 +430,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         extra = ex_eye + B * H * dk * dk * 4;
     }
     const int64_t budget = workspace_budget() - 1024 - off_bytes - extra;
-    int64_t Hg = budget / per_head;
+    int64_t Hg = per_head > 0 ? budget / per_head : H;
     if (Hg < 1) Hg = 1;
     if (Hg > H) Hg = H;
     const int64_t ws_bytes = 1024 + off_bytes + Hg * per_head + (extra ? extra + 1024 : 0);
@@ -445,7 +454,9 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         plan.seg_off = seg_off;
     }
     unsigned char* ws = reinterpret_cast<unsigned char*>(base + 1024 + off_bytes);
-    if (use_tc) {
+    if (use_fused) {
+        e = run_prefill_fused(a, err_flag, stream);
+    } else if (use_tc) {
         e = run_prefill_tc(a, ws, Hg, err_flag, stream);
     } else if (!segmap) {
         e = run_prefill_simt(a, reinterpret_cast<float*>(ws), Hg, stream);

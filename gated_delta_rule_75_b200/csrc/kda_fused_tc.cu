@@ -1,0 +1,961 @@
+// Fused chunkwise KDA prefill on the sm_100a tensor cores (bf16 I/O, dk = dv = 128).
+//
+// The chunk equations are those of the two-kernel path (derived by unrolling the
+// per-token step of "Kimi Delta Attention: la atencion lineal detras de Kimi K2 y
+// Qwen3", section "Como funciona Kimi Delta Attention paso a paso"; the chunkwise
+// form is the one "Kimi Linear acaba de superar a la atencion completa en sus
+// propios terminos" says the method trains with), with T' = (I + A)^{-1} diag(beta):
+//
+//   A_ij   = beta_i sum_c k_ic k_jc e^{G_ic - G_jc}   (i > j)
+//   Aqk_ij = sum_c q_ic k_jc e^{G_ic - G_jc}          (i >= j)
+//   W = T' (K e^G),  U = T' V - W S,  O = scale ((Q e^G) S + Aqk U),
+//   S <- Diag(e^{G_last}) S + (K e^{G_last - G})^T U
+//
+// One CTA per SM walks (sequence, head) chains, heads innermost, and computes
+// every chunk's operands on chip: nothing but the inputs, the outputs and the
+// final states crosses HBM.  Roles (448 threads):
+//   warps 0-7   prep: thread (channel c, token half) -- cumulative decay in
+//               registers, the exponential factors, the operand tiles [c][t]
+//               (token-contiguous, 128B-swizzled), the A / Aqk read-out, the
+//               blocked inverse of (I + A), T' and the -W^T read-out;
+//   warps 8-11  walk: thread = value column j (a TMEM lane of S^T) -- the
+//               state's decay scaling, the U^T / S^T bf16 copies (kept in
+//               tensor memory as MMA operands), the output tile;
+//   warp 12     one thread issues the prep's TMA loads and MMAs;
+//   warp 13     one thread issues the walk's MMAs and v loads.
+// Per chunk, k and q land by TMA as [t][c] tiles and are transposed into tensor
+// memory by an MMA with the identity (exact), so each prep thread owns one
+// channel's tokens.  The decay factors e^{G_i - G_j} are split around one
+// reference row for the whole chunk when every factor stays within 2^100, so
+// A and Aqk are one MMA; otherwise the lower triangle is taken level by level
+// (blocks of 64, 32, ..., 2 rows; each pair i > j at the level where i and j
+// fall in different halves, both factors referenced to the first row of the
+// upper half and so <= 1), plus one product for the diagonal: exact at any
+// decay rate.  The state walk of chunk c (U^T = V^T T'^T + S^T (-W^T),
+// O^T = S^T (Q e^G)^T + U^T Aqk^T, S^T += U^T (K e^{Gl - G})) overlaps the prep
+// of chunk c + 1; the operands whose producer and consumer overlap are
+// double-buffered, the rest are handed over on mbarriers.  Every wait is
+// bounded; a wait that gives up sets a bit in the error word and makes every
+// role leave its loop, after which the CTA drains its copies and MMAs and
+// frees its tensor memory.
+#include <cstring>
+
+#include "kda_common.cuh"
+#include "kda_internal.h"
+#include "kda_tc_util.cuh"
+#include "kda_tma.cuh"
+#include "kda_umma.cuh"
+
+namespace kda {
+
+using namespace umma;
+using namespace tcu;
+
+namespace fz {
+
+constexpr int C = 64;
+constexpr int D = 128;
+constexpr int NT = 448;
+constexpr int AP = 68;                      // row pitch (floats) of the fp32 A and T
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kRange = 100.f;             // one-reference factors stay within 2^+-100
+constexpr long long kWaitCycles = 4000000000LL;
+
+constexpr int W_WALK = 8;                   // walk warps 8-11
+constexpr int W_PI = 12;                    // prep issuer
+constexpr int W_WI = 13;                    // walk issuer
+
+constexpr int NB_PAIR = 1;                  // 1..4: prep warps w and w + 4
+constexpr int NB_PREP = 5;                  // prep warps 0-7
+constexpr int NB_INV = 6;                   // prep warps 0-3
+constexpr int NB_WALK = 7;                  // walk warps
+
+// Shared memory (bytes from a 1024-aligned base).  [c][t] tiles: 128 channel rows of
+// 64 tokens (128 B), 128B-swizzled -- K-major when the tokens are the reduction index,
+// MN-major when they are the M/N index.
+constexpr uint32_t F_ID = 0;                // identity 64 x 64 bf16                       8 KB
+constexpr uint32_t F_KQ = 8192;             // k | q [t][c] (TMA), then Kin^T | Qin^T       32 KB
+constexpr uint32_t F_KD = 40960;            // Kd^T, then T fp32 [64][AP]                  17 KB
+constexpr uint32_t F_KG = 58368;            // (K e^G)^T                                   16 KB
+constexpr uint32_t F_QG = 74752;            // (Q e^G)^T x 2; after use the output tile    32 KB
+constexpr uint32_t F_KL = 107520;           // (K e^{Gl - G})^T x 2                        32 KB
+constexpr uint32_t F_AQ = 140288;           // Aqk [i][j] x 2                              16 KB
+constexpr uint32_t F_TP = 156672;           // T' [i][j]                                    8 KB
+constexpr uint32_t F_W = 164864;            // A fp32 [64][AP] for the inverse, then -W^T  17 KB
+constexpr uint32_t F_V = 182272;            // v [t][dv] (TMA) x 2                         32 KB
+constexpr uint32_t F_GAM = 215040;          // e^{G_last} x 2
+constexpr uint32_t F_BETA = 216064;         // beta of the chunk
+constexpr uint32_t F_XCH = 216320;          // half sums of the decay [3][128]
+constexpr uint32_t F_BYTES = F_XCH + 3 * 128 * 4;
+constexpr uint32_t F_SMEM = F_BYTES + 1024;
+static_assert(F_KD + 64 * AP * 4 <= F_KG, "T scratch overlaps (K e^G)^T");
+static_assert(F_W + 64 * AP * 4 <= F_V, "A scratch overlaps v");
+
+// Tensor memory columns (512 allocated)
+constexpr uint32_t TM_KT = 0;               // k^T fp32 (prep), then -W^T
+constexpr uint32_t TM_QT = 64;              // q^T fp32
+constexpr uint32_t TM_WT = 0;
+constexpr uint32_t TM_S = 128;              // S^T fp32 (state)
+constexpr uint32_t TM_U = 256;              // U^T fp32; its first 32 columns then hold U^T bf16
+constexpr uint32_t TM_O = 320;              // O^T fp32
+constexpr uint32_t TM_SB = 384;             // S^T bf16 (operand)
+constexpr uint32_t TM_D = 448;              // [Kin; Qin] Kd^T
+
+struct Bars {
+    uint64_t kq, tr, ops, a, t, w, img;     // prep pipeline
+    uint64_t v[2], u, s, o, ur, sc, sr, orr, go;   // walk pipeline
+    uint64_t m1, fr[2];                     // walk -> prep: MMA1 done, image slot free
+    uint64_t fin_p, fin_w;                  // issuers' final drains
+};
+
+__device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile(
+        "{\n\t"
+        ".reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.b32 %0, 1, 0, p;\n\t"
+        "}\n"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded poll of one phase; gives up when another role has given up (abort) or after
+// about 2 s, then sets bit `bit` in *err and the abort flag.
+__device__ __forceinline__ bool fwait(uint64_t* bar, uint32_t parity, int* err, int bit,
+                                      volatile int* abort)
+{
+    const long long t0 = clock64();
+    for (uint32_t i = 1;; ++i) {
+        if (mbar_test(bar, parity)) return true;
+        if ((i & 31u) == 0) {
+            if (*abort) return false;
+            if (clock64() - t0 > kWaitCycles) {
+                if (err) atomicOr(err, 1 << bit);
+                *abort = 1;
+                return false;
+            }
+        }
+    }
+}
+
+// A group's wait: `leader` polls, the group's barrier shares the outcome.
+__device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, bool leader, int barid,
+                                      int count, int* err, int bit, volatile int* abort)
+{
+    bool ok = true;
+    if (leader) ok = fwait(bar, parity, err, bit, abort);
+    return bar_and_named(barid, count, ok);
+}
+
+// The chunks of one CTA: chains b, b + G, b + 2G, ... of the (sequence rank, head)
+// list, heads innermost; sequences ranked longest first when an order is known.
+// Chains without tokens are skipped (their final states are written separately).
+struct Items {
+    int64_t r, rstep, rend, H;
+    int64_t n, h, bos, eos, nch, c, sidx;
+    bool ok;
+
+    __device__ __forceinline__ void init(int64_t b, int64_t step, const SeqInfo& si, int64_t H_,
+                                         const int32_t* slots, int64_t P)
+    {
+        r = b;
+        rstep = step;
+        rend = si.N * H_;
+        H = H_;
+        load(si, slots, P);
+    }
+    __device__ __forceinline__ void load(const SeqInfo& si, const int32_t* slots, int64_t P)
+    {
+        ok = false;
+        while (r < rend) {
+            const int64_t sr = r / H;
+            h = r - sr * H;
+            n = si.seq_of(sr);
+            seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
+            nch = (eos - bos + C - 1) / C;
+            if (nch > 0) {
+                c = 0;
+                sidx = n * H + h;
+                if (slots) {
+                    const int64_t sl = slots[n];
+                    sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
+                }
+                ok = true;
+                return;
+            }
+            r += rstep;
+        }
+    }
+    __device__ __forceinline__ void next(const SeqInfo& si, const int32_t* slots, int64_t P)
+    {
+        if (++c >= nch) {
+            r += rstep;
+            load(si, slots, P);
+        }
+    }
+    __device__ __forceinline__ int64_t t0() const { return bos + c * C; }
+    __device__ __forceinline__ int len() const
+    {
+        const int64_t l = eos - t0();
+        return (int)(l < C ? l : C);
+    }
+    __device__ __forceinline__ bool first() const { return c == 0; }
+    __device__ __forceinline__ bool last() const { return c + 1 == nch; }
+};
+
+// Byte offset of token t of channel row c in a [c][t] tile.
+__device__ __forceinline__ uint32_t ct_off(int c, int t)
+{
+    return (uint32_t)c * 128u + ((uint32_t)(((t >> 3) ^ c) & 7) << 4);
+}
+
+// T = (I + A)^{-1} for the strictly lower A (fp32, pitch AP): 16 x 16 diagonal blocks
+// by forward substitution (threads 0-63, one column each), then the blocks below by
+// tf32 block products in two levels (warps 0-3; scratch blocks parked above the
+// diagonal of A).  T's blocks above the diagonal are not written.
+__device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, int tid)
+{
+    const int w = tid >> 5, l = tid & 31;
+    if (tid < C) {
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
+        float tcol[16];
+#pragma unroll
+        for (int r = 0; r < 16; ++r) {
+            float acc0 = 0.f, acc1 = 0.f;
+#pragma unroll
+            for (int m = 0; m < r; ++m) {
+                if (m & 1) acc1 += sA[(o + r) * AP + o + m] * tcol[m];
+                else acc0 += sA[(o + r) * AP + o + m] * tcol[m];
+            }
+            tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -(acc0 + acc1));
+        }
+#pragma unroll
+        for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
+    }
+    bar_sync_named(NB_INV, 128);
+    auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
+    auto Tb = [&](int r, int c) { return sT + (16 * r) * AP + 16 * c; };
+    if (w < 2) {                                  // T_10 = -T_11 A_10 T_00, T_32 = -T_33 A_32 T_22
+        const int p = 2 * w + 1, r = 2 * w;
+        float acc[2][4] = {};
+        mma16x16x16_tf32<AP>(acc, Ab(p, r), Tb(r, r), l);
+        store16x16<AP>(Ab(r, p), acc, 1.f, l);
+        __syncwarp();
+        float acc2[2][4] = {};
+        mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
+        store16x16<AP>(Tb(p, r), acc2, -1.f, l);
+    }
+    bar_sync_named(NB_INV, 128);
+    {                                             // X_pr = sum_{m = r..1} A_pm T_mr
+        const int p = 2 + (w >> 1), r = w & 1;
+        float acc[2][4] = {};
+        for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
+        store16x16<AP>(Ab(r, p), acc, 1.f, l);
+    }
+    bar_sync_named(NB_INV, 128);
+    {                                             // T_pr = -sum_{m = 2..p} T_pm X_mr
+        const int p = 2 + (w >> 1), r = w & 1;
+        float acc[2][4] = {};
+        for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
+        store16x16<AP>(Tb(p, r), acc, -1.f, l);
+    }
+}
+
+// Level-pass selection of the exact fallback: pair (i, j) is taken at pass `pass`
+// (0..5: blocks of 2s rows, s = 32 >> pass) when i is in the upper half of its block
+// and j in the lower half of the same block; pass 6 takes the diagonal (Aqk only).
+__device__ __forceinline__ bool pass_pair(int pass, int i, int j)
+{
+    if (pass == 6) return i == j;
+    const int s = 32 >> pass;
+    const int f = (i & ~(2 * s - 1)) + s;       // first row of i's upper half
+    return (i & (2 * s - 1)) >= s && j >= f - s && j < f;
+}
+
+__global__ void __launch_bounds__(NT, 1)
+chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
+                      const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                      const float* __restrict__ log_alpha, const float* __restrict__ beta,
+                      const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
+                      float* __restrict__ hT, float scale, SeqInfo si, int64_t H,
+                      const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err)
+{
+    extern __shared__ unsigned char smem_raw[];
+    unsigned char* sm = reinterpret_cast<unsigned char*>(
+        (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    __shared__ Bars bars;
+    __shared__ uint32_t tmem_base;
+    __shared__ int s_npass;
+    __shared__ int s_abort_raw;
+    volatile int* abort = &s_abort_raw;
+
+    const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    Items it0;
+    it0.init(blockIdx.x, gridDim.x, si, H, slots, P);
+
+    if (tid == W_PI * 32) {
+        mbar_init(&bars.kq, 1); mbar_init(&bars.tr, 1); mbar_init(&bars.ops, 8);
+        mbar_init(&bars.a, 1); mbar_init(&bars.t, 8); mbar_init(&bars.w, 1); mbar_init(&bars.img, 8);
+        mbar_init(&bars.v[0], 1); mbar_init(&bars.v[1], 1);
+        mbar_init(&bars.u, 1); mbar_init(&bars.s, 1); mbar_init(&bars.o, 1);
+        mbar_init(&bars.ur, 4); mbar_init(&bars.sc, 4); mbar_init(&bars.sr, 4); mbar_init(&bars.orr, 4);
+        mbar_init(&bars.go, 1); mbar_init(&bars.m1, 1); mbar_init(&bars.fr[0], 1); mbar_init(&bars.fr[1], 1);
+        mbar_init(&bars.fin_p, 1); mbar_init(&bars.fin_w, 1);
+        fence_mbar_init();
+        s_abort_raw = 0;
+        s_npass = 1;
+    }
+    if (w < 8) {                                  // the identity operand of the transposes
+        for (int e = tid; e < 512; e += 256) {
+            const int r = e >> 3, cb = e & 7;
+            float f[8];
+#pragma unroll
+            for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x == r) ? 1.f : 0.f;
+            *reinterpret_cast<uint4*>(sm + F_ID + sw128_offset(r, 8 * cb)) = pack8(f);
+        }
+        fence_smem_to_async();
+    }
+    if (w == W_PI) { tmem_alloc(&tmem_base, 512); tmem_relinquish(); }
+    fence_before_sync();
+    __syncthreads();
+    fence_after_sync();
+    const uint32_t tmem = tmem_base;
+
+    if (w < 8) {
+        // ------------------------------------------------------------------ prep
+        const int q4 = w & 3, ph = w >> 2;
+        const int pc = 32 * q4 + l;               // channel (TMEM lane of k^T, q^T, -W^T)
+        const uint32_t lane = (uint32_t)(32 * q4) << 16;
+        const bool leader = tid == 0;
+        float* sB = reinterpret_cast<float*>(sm + F_BETA);
+        float* xch = reinterpret_cast<float*>(sm + F_XCH);
+        float* sA = reinterpret_cast<float*>(sm + F_W);
+        float* sT = reinterpret_cast<float*>(sm + F_KD);
+        const int64_t rs = H * D;                 // floats between token rows of log_alpha
+
+        // this thread's 32 gates of an item (natural log; zero past its end) and, for the
+        // first 64 channels' threads, beta of row pc
+        auto load_inputs = [&](const Items& x, float* g, float& b) {
+            const int64_t t0 = x.t0();
+            const int len = x.len();
+            const float* base = log_alpha + (t0 + 32 * ph) * rs + x.h * D + pc;
+#pragma unroll
+            for (int y = 0; y < 32; ++y) g[y] = (32 * ph + y < len) ? __ldg(base + y * rs) : 0.f;
+            b = (q4 < 2 && pc < len) ? __ldg(beta + (t0 + pc) * H + x.h) : 0.f;
+        };
+
+        Items it = it0;
+        float gv[32], bv = 0.f;
+        if (it.ok) load_inputs(it, gv, bv);
+        uint32_t n_a = 0;                         // completions of bars.a seen
+        for (uint32_t k = 0; it.ok; ++k) {
+            const int s = (int)(k & 1);
+            const int len = it.len();
+            // ---- (a) cumulative decay of channel pc over this half's tokens, log2 units
+            float G[32];
+            float run = 0.f;
+#pragma unroll
+            for (int y = 0; y < 32; ++y) {
+                run += kLog2e * gv[y];
+                G[y] = run;
+            }
+            xch[ph * 128 + pc] = run;
+            if (ph == 1) xch[256 + pc] = G[0];
+            bar_sync_named(NB_PAIR + q4, 64);
+            const float s0 = xch[pc], s1 = xch[128 + pc];
+            const float G32 = s0 + xch[256 + pc];
+            if (ph == 1) {
+#pragma unroll
+                for (int y = 0; y < 32; ++y) G[y] += s0;
+            }
+            const float Gm = s0, Gl = s0 + s1;    // reference row 31, last row
+            float mx = 0.f;
+#pragma unroll
+            for (int y = 0; y < 32; ++y) mx = fmaxf(mx, fabsf(G[y] - Gm));
+            const float bcur = bv;
+            Items nx = it;
+            nx.next(si, slots, P);
+            if (nx.ok) load_inputs(nx, gv, bv);   // in flight during this chunk
+
+            // k^T, q^T of this chunk in TMEM; image slot s free (chunk k - 2 walked);
+            // T', -W^T and the A scratch free (MMA1 of chunk k - 1 done)
+            bool ok = true;
+            if (leader) {
+                ok = fwait(&bars.tr, k & 1, err, 1, abort);
+                if (ok && k >= 2) ok = fwait(&bars.fr[s], ((k - 2) >> 1) & 1, err, 6, abort);
+                if (ok && k >= 1) ok = fwait(&bars.m1, (k - 1) & 1, err, 6, abort);
+            }
+            if (!bar_and_named(NB_PREP, 256, ok)) break;
+            fence_after_sync();
+            const bool fast = bar_and_named(NB_PREP, 256, !(mx > kRange));
+            if (leader) s_npass = fast ? 1 : 7;
+
+            unsigned char* qg = sm + F_QG + s * 16384;
+            unsigned char* kl = sm + F_KL + s * 16384;
+            unsigned char* aq = sm + F_AQ + s * 8192;
+            auto load_kq = [&](int hb, float* kf, float* qf) {
+                tmem_ld16(tmem + lane + TM_KT + 32 * ph + 16 * hb, kf);
+                tmem_ld16(tmem + lane + TM_QT + 32 * ph + 16 * hb, qf);
+                tmem_wait_ld();
+                if (len < C) {
+#pragma unroll
+                    for (int y = 0; y < 16; ++y)
+                        if (32 * ph + 16 * hb + y >= len) kf[y] = qf[y] = 0.f;
+                }
+            };
+            auto ops_arrive = [&] {
+                fence_smem_to_async();
+                fence_before_sync();
+                __syncwarp();
+                if (l == 0) mbar_arrive(&bars.ops);
+            };
+            auto wait_a = [&]() -> bool {
+                bool o2 = true;
+                if (leader) o2 = fwait(&bars.a, n_a & 1, err, 2, abort);
+                ++n_a;
+                o2 = bar_and_named(NB_PREP, 256, o2);
+                fence_after_sync();
+                return o2;
+            };
+
+            if (fast) {
+                // ---- (b1) one reference: Kin = k e^{G - Gm}, Qin, Kd = k e^{Gm - G}, and the
+                // image tiles K e^G = Kin e^{Gm}, Q e^G, K e^{Gl - G} = Kd e^{Gl - Gm}
+                const float Em = ex2(Gm), Egl = ex2(Gl - Gm);
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {
+                    float kf[16], qf[16];
+                    load_kq(hb, kf, qf);
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) {
+                        float kin[8], qin[8], kd[8], t1[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int y = 8 * m + e;
+                            const float x = G[16 * hb + y] - Gm;
+                            const float e1 = ex2(x), e2 = ex2(-x);
+                            kin[e] = kf[y] * e1;
+                            qin[e] = qf[y] * e1;
+                            kd[e] = kf[y] * e2;
+                        }
+                        const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
+                        *reinterpret_cast<uint4*>(sm + F_KQ + off) = pack8(kin);
+                        *reinterpret_cast<uint4*>(sm + F_KQ + 16384 + off) = pack8(qin);
+                        *reinterpret_cast<uint4*>(sm + F_KD + off) = pack8(kd);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) t1[e] = kin[e] * Em;
+                        *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(t1);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) t1[e] = qin[e] * Em;
+                        *reinterpret_cast<uint4*>(qg + off) = pack8(t1);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) t1[e] = kd[e] * Egl;
+                        *reinterpret_cast<uint4*>(kl + off) = pack8(t1);
+                    }
+                }
+                if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
+                ops_arrive();
+                if (!wait_a()) break;
+                // ---- A (fp32, beta-scaled rows, for the inverse) and Aqk (bf16 image)
+                float d[32];
+                tmem_ld16(tmem + lane + TM_D + 32 * ph, d);
+                tmem_ld16(tmem + lane + TM_D + 32 * ph + 16, d + 16);
+                tmem_wait_ld();
+                if (q4 < 2) {
+                    const int i = pc;
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) {
+                        const int j = 32 * ph + y;
+                        sA[i * AP + j] = (j < i) ? bcur * d[y] : 0.f;
+                    }
+                    if (ph == 0) sB[i] = bcur;
+                } else {
+                    const int i = pc - 64;
+#pragma unroll
+                    for (int m = 0; m < 4; ++m) {
+                        float a8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) a8[e] = (32 * ph + 8 * m + e <= i) ? d[8 * m + e] : 0.f;
+                        *reinterpret_cast<uint4*>(aq + sw128_offset(i, 32 * ph + 8 * m)) = pack8(a8);
+                    }
+                }
+            } else {
+                // ---- (b1') the level passes: every factor <= 1 (log_alpha <= 0)
+                for (int e = tid; e < 64 * AP / 4; e += 256)
+                    reinterpret_cast<float4*>(sA)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
+                for (int e = tid; e < 512; e += 256)
+                    reinterpret_cast<uint4*>(aq)[e] = make_uint4(0, 0, 0, 0);
+                if (q4 < 2 && ph == 0) sB[pc] = bcur;
+                float Gs[32];                     // indexed at run time (local memory)
+#pragma unroll
+                for (int y = 0; y < 32; ++y) Gs[y] = G[y];
+#pragma unroll
+                for (int hb = 0; hb < 2; ++hb) {  // image tiles from e^G and e^{Gl - G} directly
+                    float kf[16], qf[16];
+                    load_kq(hb, kf, qf);
+#pragma unroll
+                    for (int m = 0; m < 2; ++m) {
+                        float a8[8], b8[8], c8[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int y = 8 * m + e;
+                            const float eg = ex2(G[16 * hb + y]), egl = ex2(Gl - G[16 * hb + y]);
+                            a8[e] = kf[y] * eg;
+                            b8[e] = qf[y] * eg;
+                            c8[e] = kf[y] * egl;
+                        }
+                        const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
+                        *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(a8);
+                        *reinterpret_cast<uint4*>(qg + off) = pack8(b8);
+                        *reinterpret_cast<uint4*>(kl + off) = pack8(c8);
+                    }
+                }
+                if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
+                bar_sync_named(NB_PREP, 256);     // zeroed A / Aqk before any pass writes
+                bool pok = true;
+                for (int pass = 0; pass < 7 && pok; ++pass) {
+                    const int hs = 32 >> pass;    // half block of this level (pass < 6)
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb) {
+                        float kf[16], qf[16];
+                        load_kq(hb, kf, qf);
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            float kin[8], qin[8], kd[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const int y = 8 * m + e, t = 32 * ph + 16 * hb + y;
+                                if (pass == 6) {
+                                    kin[e] = kf[y]; qin[e] = qf[y]; kd[e] = kf[y];
+                                } else {
+                                    const bool up = (t & (2 * hs - 1)) >= hs;
+                                    const int f = (t & ~(2 * hs - 1)) + hs;
+                                    const float Gf = (hs == 32) ? G32 : Gs[f - 32 * ph];
+                                    const float x = G[16 * hb + y] - Gf;   // <= 0 up, >= 0 below
+                                    const float ef = ex2(up ? x : -x);
+                                    kin[e] = up ? kf[y] * ef : 0.f;
+                                    qin[e] = up ? qf[y] * ef : 0.f;
+                                    kd[e] = up ? 0.f : kf[y] * ef;
+                                }
+                            }
+                            const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
+                            *reinterpret_cast<uint4*>(sm + F_KQ + off) = pack8(kin);
+                            *reinterpret_cast<uint4*>(sm + F_KQ + 16384 + off) = pack8(qin);
+                            *reinterpret_cast<uint4*>(sm + F_KD + off) = pack8(kd);
+                        }
+                    }
+                    ops_arrive();
+                    if (!(pok = wait_a())) break;
+                    float d[32];
+                    tmem_ld16(tmem + lane + TM_D + 32 * ph, d);
+                    tmem_ld16(tmem + lane + TM_D + 32 * ph + 16, d + 16);
+                    tmem_wait_ld();
+                    if (q4 < 2) {
+                        const int i = pc;
+                        if (pass < 6)
+                            for (int y = 0; y < 32; ++y)
+                                if (pass_pair(pass, i, 32 * ph + y)) sA[i * AP + 32 * ph + y] = bcur * d[y];
+                    } else {
+                        const int i = pc - 64;
+                        for (int y = 0; y < 32; ++y)
+                            if (pass_pair(pass, i, 32 * ph + y))
+                                *reinterpret_cast<__nv_bfloat16*>(aq + sw128_offset(i, 32 * ph + y)) =
+                                    __float2bfloat16_rn(d[y]);
+                    }
+                    fence_before_sync();          // TMEM reads before the next pass's MMA
+                }
+                if (!pok) break;
+            }
+            fence_smem_to_async();                // Aqk: read by the walk's MMAs
+            bar_sync_named(NB_PREP, 256);         // A complete
+            // ---- (b2) T = (I + A)^{-1} (warps 0-3)
+            if (w < 4) invert_unit_lower(sA, sT, tid);
+            bar_sync_named(NB_PREP, 256);
+            // T' = T diag(beta), bf16 [i][j]; blocks above the diagonal are zero
+            for (int e = tid; e < C * 8; e += 256) {
+                const int i = e >> 3, cb = e & 7;
+                uint4 u = make_uint4(0, 0, 0, 0);
+                if ((cb >> 1) <= (i >> 4)) {
+                    float f[8], bt[8];
+                    ld8f(sT + i * AP + 8 * cb, f);
+                    ld8f(sB + 8 * cb, bt);
+#pragma unroll
+                    for (int x = 0; x < 8; ++x) f[x] *= bt[x];
+                    u = pack8(f);
+                }
+                *reinterpret_cast<uint4*>(sm + F_TP + sw128_offset(i, 8 * cb)) = u;
+            }
+            fence_smem_to_async();
+            fence_before_sync();
+            __syncwarp();
+            if (l == 0) mbar_arrive(&bars.t);
+            // ---- (b3) -W^T = -(K e^G)^T T'^T from TMEM into the image, [c][i]
+            ok = true;
+            if (leader) ok = fwait(&bars.w, k & 1, err, 3, abort);
+            if (!bar_and_named(NB_PREP, 256, ok)) break;
+            fence_after_sync();
+            {
+                float f[32];
+                tmem_ld16(tmem + lane + TM_WT + 32 * ph, f);
+                tmem_ld16(tmem + lane + TM_WT + 32 * ph + 16, f + 16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int m = 0; m < 4; ++m)
+                    *reinterpret_cast<uint4*>(sm + F_W + sw128_offset(pc, 32 * ph + 8 * m)) = pack8(f + 8 * m);
+            }
+            fence_smem_to_async();
+            fence_before_sync();
+            __syncwarp();
+            if (l == 0) mbar_arrive(&bars.img);
+            it = nx;
+        }
+    } else if (w < W_PI) {
+        // ------------------------------------------------------------------ walk
+        const int q4 = w & 3;
+        const int j = 32 * q4 + l;                // value column = TMEM lane of S^T, U^T, O^T
+        const uint32_t lane = (uint32_t)(32 * q4) << 16;
+        const bool wlead = tid == W_WALK * 32;
+        // chains without tokens: final state = initial state
+        for (int64_t r = blockIdx.x; hT && r < si.N * H; r += gridDim.x) {
+            const int64_t sr = r / H, h = r - sr * H, n = si.seq_of(sr);
+            int64_t bos, eos;
+            seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
+            if (eos > bos) continue;
+            int64_t sidx = n * H + h;
+            if (slots) {
+                const int64_t sl = slots[n];
+                sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
+            }
+            if (sidx < 0) continue;
+            for (int c = 0; c < D; ++c)
+                hT[sidx * D * D + c * D + j] = h0 ? h0[sidx * D * D + c * D + j] : 0.f;
+        }
+        auto arrive4 = [&](uint64_t* b) {
+            fence_before_sync();
+            __syncwarp();
+            if (l == 0) mbar_arrive(b);
+        };
+        auto wwait = [&](uint64_t* b, uint32_t par, int bit) -> bool {
+            const bool o = gwait(b, par, wlead, NB_WALK, 128, err, bit, abort);
+            fence_after_sync();
+            return o;
+        };
+        Items it = it0;
+        for (uint32_t k = 0; it.ok; ++k) {
+            const int s = (int)(k & 1);
+            if (slots && it.first() && wlead && err) {
+                const int64_t sl = slots[it.n];
+                if (sl >= P) atomicOr(err, 1);
+            }
+            if (it.first()) {                     // entry state: fp32 and its bf16 operand copy
+                const float* hp = (h0 && it.sidx >= 0) ? h0 + it.sidx * D * D : nullptr;
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    float f[32];
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) f[y] = hp ? hp[(32 * cb + y) * D + j] : 0.f;
+                    tmem_st16(tmem + lane + TM_S + 32 * cb, f);
+                    tmem_st16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
+                    uint32_t u[16];
+#pragma unroll
+                    for (int y = 0; y < 16; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
+                    tmem_st16u(tmem + lane + TM_SB + 16 * cb, u);
+                }
+                tmem_wait_st();
+                arrive4(&bars.sr);
+            }
+            // the state decays by this chunk's e^{G_last} once MMA1 (which reads only the
+            // bf16 copy) is issued; MMA2 accumulates onto the scaled state
+            if (!wwait(&bars.go, k & 1, 6)) break;
+            {
+                const float* gam = reinterpret_cast<const float*>(sm + F_GAM + s * 512);
+#pragma unroll 1
+                for (int cb = 0; cb < 8; ++cb) {
+                    float f[16], g8[16];
+                    tmem_ld16(tmem + lane + TM_S + 16 * cb, f);
+                    ld8f(gam + 16 * cb, g8);
+                    ld8f(gam + 16 * cb + 8, g8 + 8);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int y = 0; y < 16; ++y) f[y] *= g8[y];
+                    tmem_st16(tmem + lane + TM_S + 16 * cb, f);
+                }
+                tmem_wait_st();
+                arrive4(&bars.sc);
+            }
+            // U^T -> bf16 operand (first 32 columns of its own TMEM range)
+            if (!wwait(&bars.u, k & 1, 5)) break;
+            {
+                float f[64];
+#pragma unroll
+                for (int x = 0; x < 4; ++x) tmem_ld16(tmem + lane + TM_U + 16 * x, f + 16 * x);
+                tmem_wait_ld();
+                uint32_t u[32];
+#pragma unroll
+                for (int y = 0; y < 32; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
+                tmem_st16u(tmem + lane + TM_U, u);
+                tmem_st16u(tmem + lane + TM_U + 16, u + 16);
+                tmem_wait_st();
+                arrive4(&bars.ur);
+            }
+            // next entry state -> bf16 operand, or the final state
+            if (!wwait(&bars.s, k & 1, 5)) break;
+            if (!it.last()) {
+#pragma unroll 1
+                for (int cb = 0; cb < 4; ++cb) {
+                    float f[32];
+                    tmem_ld16(tmem + lane + TM_S + 32 * cb, f);
+                    tmem_ld16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
+                    tmem_wait_ld();
+                    uint32_t u[16];
+#pragma unroll
+                    for (int y = 0; y < 16; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
+                    tmem_st16u(tmem + lane + TM_SB + 16 * cb, u);
+                }
+                tmem_wait_st();
+                arrive4(&bars.sr);
+            } else if (hT && it.sidx >= 0) {
+                float* hp = hT + it.sidx * D * D;
+#pragma unroll 1
+                for (int cb = 0; cb < 8; ++cb) {
+                    float f[16];
+                    tmem_ld16(tmem + lane + TM_S + 16 * cb, f);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int y = 0; y < 16; ++y) hp[(16 * cb + y) * D + j] = f[y];
+                }
+            }
+            // output rows: [t][dv] bf16 tile in the consumed (Q e^G)^T slot, one tensor store
+            if (!wwait(&bars.o, k & 1, 5)) break;
+            unsigned char* stg = sm + F_QG + s * 16384;
+            {
+#pragma unroll 1
+                for (int x = 0; x < 4; ++x) {
+                    float f[16];
+                    tmem_ld16(tmem + lane + TM_O + 16 * x, f);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int y = 0; y < 16; ++y)
+                        *reinterpret_cast<__nv_bfloat16*>(stg + (16 * x + y) * 256 + 2 * j) =
+                            __float2bfloat16_rn(scale * f[y]);
+                }
+            }
+            arrive4(&bars.orr);
+            fence_smem_to_async();
+            bar_sync_named(NB_WALK, 128);
+            const int len = it.len();
+            const int64_t t0 = it.t0();
+            if (len == C) {
+                if (wlead) {
+                    tma::store_2d(&omap, (int32_t)(it.h * D), (int32_t)t0, stg);
+                    tma::bulk_commit();
+                    tma::bulk_wait_read();
+                    mbar_arrive(&bars.fr[s]);
+                }
+            } else {
+                for (int e = tid - W_WALK * 32; e < len * 16; e += 128) {
+                    const int r = e >> 4, c = e & 15;
+                    *reinterpret_cast<uint4*>(out + ((t0 + r) * H + it.h) * D + 8 * c) =
+                        *reinterpret_cast<const uint4*>(stg + r * 256 + c * 16);
+                }
+                bar_sync_named(NB_WALK, 128);
+                if (wlead) mbar_arrive(&bars.fr[s]);
+            }
+            it.next(si, slots, P);
+        }
+        if (wlead) tma::bulk_wait_all();
+    } else if (w == W_PI) {
+        // ------------------------------------------------------------------ prep issuer
+        if (l == 0) {
+            auto issue_kq = [&](const Items& x) {
+                const int32_t y = (int32_t)x.t0(), xc = (int32_t)(x.h * D);
+                tma::expect_tx(&bars.kq, 32768);
+                tma::load_2d(sm + F_KQ, &kmap, xc, y, &bars.kq);
+                tma::load_2d(sm + F_KQ + 8192, &kmap, xc + 64, y, &bars.kq);
+                tma::load_2d(sm + F_KQ + 16384, &qmap, xc, y, &bars.kq);
+                tma::load_2d(sm + F_KQ + 24576, &qmap, xc + 64, y, &bars.kq);
+            };
+            Items it = it0;
+            uint32_t n_ops = 0, kq_issued = 0, kq_seen = 0;
+            if (it.ok) { issue_kq(it); ++kq_issued; }
+            for (uint32_t k = 0; it.ok; ++k) {
+                Items nx = it;
+                nx.next(si, slots, P);
+                if (!fwait(&bars.kq, k & 1, err, 1, abort)) break;
+                ++kq_seen;
+                if (k > 0 && !fwait(&bars.img, (k - 1) & 1, err, 6, abort)) break;
+                fence_after_sync();
+                {                                 // k^T, q^T = [t][c]^T I (exact)
+                    const uint32_t id = make_idesc_bf16(128, 64, true, false);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tmem + TM_KT, make_desc(smem_u32(sm + F_KQ + ks * 2048), 8192, 1024),
+                                 make_desc(smem_u32(sm + F_ID + ks * 32), 16, 1024), id, ks > 0);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tmem + TM_QT, make_desc(smem_u32(sm + F_KQ + 16384 + ks * 2048), 8192, 1024),
+                                 make_desc(smem_u32(sm + F_ID + ks * 32), 16, 1024), id, ks > 0);
+                    commit(&bars.tr);
+                }
+                bool ok = true;
+                int np = 1;
+                for (int p = 0; p < np; ++p) {    // [Kin; Qin] Kd^T, once per pass
+                    if (!(ok = fwait(&bars.ops, n_ops & 1, err, 6, abort))) break;
+                    ++n_ops;
+                    if (p == 0) np = *reinterpret_cast<volatile int*>(&s_npass);
+                    fence_after_sync();
+                    const uint32_t id = make_idesc_bf16(128, 64, true, true);
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(tmem + TM_D, make_desc(smem_u32(sm + F_KQ + ks * 2048), 16384, 1024),
+                                 make_desc(smem_u32(sm + F_KD + ks * 2048), 16384, 1024), id, ks > 0);
+                    commit(&bars.a);
+                }
+                if (!ok) break;
+                // the k / q buffer is free once the last pass has read its operands
+                if (!fwait(&bars.a, (n_ops - 1) & 1, err, 2, abort)) break;
+                if (nx.ok) { issue_kq(nx); ++kq_issued; }
+                if (!fwait(&bars.t, k & 1, err, 6, abort)) break;
+                fence_after_sync();
+                {                                 // -W^T = -(K e^G)^T T'^T
+                    const uint32_t id = make_idesc_bf16(128, 64, false, false, true);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ++ks)
+                        mma_bf16(tmem + TM_WT, make_desc(smem_u32(sm + F_KG + ks * 32), 16, 1024),
+                                 make_desc(smem_u32(sm + F_TP + ks * 32), 16, 1024), id, ks > 0);
+                    commit(&bars.w);
+                }
+                it = nx;
+            }
+            // drain: this thread's MMAs and copies
+            commit(&bars.fin_p);
+            mbar_wait(&bars.fin_p, 0, nullptr, 0, 200);
+            while (kq_seen < kq_issued) {
+                mbar_wait(&bars.kq, kq_seen & 1, nullptr, 0, 200);
+                ++kq_seen;
+            }
+        }
+        __syncwarp();
+    } else {
+        // ------------------------------------------------------------------ walk issuer
+        if (l == 0) {
+            auto issue_v = [&](const Items& x, int slot) {
+                const int32_t y = (int32_t)x.t0(), xc = (int32_t)(x.h * D);
+                tma::expect_tx(&bars.v[slot], 16384);
+                tma::load_2d(sm + F_V + slot * 16384, &vmap, xc, y, &bars.v[slot]);
+                tma::load_2d(sm + F_V + slot * 16384 + 8192, &vmap, xc + 64, y, &bars.v[slot]);
+            };
+            Items it = it0;
+            uint32_t v_issued[2] = {0, 0}, v_seen[2] = {0, 0};
+            {
+                Items i1 = it;
+                if (i1.ok) { issue_v(i1, 0); ++v_issued[0]; i1.next(si, slots, P); }
+                if (i1.ok) { issue_v(i1, 1); ++v_issued[1]; }
+            }
+            const uint32_t id_v = make_idesc_bf16(128, 64, true, false);   // V^T T'^T
+            const uint32_t id_n = make_idesc_bf16(128, 64, false, true);   // S^T x MN-major B
+            const uint32_t id_s = make_idesc_bf16(128, 128, false, false); // U^T (K e^{Gl-G})
+            const uint32_t id_o = make_idesc_bf16(128, 64, false, false);  // U^T Aqk^T
+            for (uint32_t k = 0; it.ok; ++k) {
+                const int s = (int)(k & 1);
+                Items n2 = it;
+                n2.next(si, slots, P);
+                if (n2.ok) n2.next(si, slots, P);
+                if (!fwait(&bars.img, k & 1, err, 6, abort)) break;
+                if (!fwait(&bars.v[s], (k >> 1) & 1, err, 4, abort)) break;
+                ++v_seen[s];
+                if (!fwait(&bars.sr, k & 1, err, 6, abort)) break;
+                if (k > 0 && !fwait(&bars.o, (k - 1) & 1, err, 5, abort)) break;
+                fence_after_sync();
+                // U^T = V^T T'^T + S^T (-W^T)
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + TM_U, make_desc(smem_u32(sm + F_V + s * 16384 + ks * 2048), 8192, 1024),
+                             make_desc(smem_u32(sm + F_TP + ks * 32), 16, 1024), id_v, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * ks,
+                                make_desc(smem_u32(sm + F_W + ks * 2048), 16384, 1024), id_n, 1u);
+                commit(&bars.u);
+                mbar_arrive(&bars.go);
+                // O^T = S^T (Q e^G)^T (the output tile of the previous chunk has left TMEM)
+                if (k > 0 && !fwait(&bars.orr, (k - 1) & 1, err, 6, abort)) break;
+                fence_after_sync();
+#pragma unroll
+                for (int ks = 0; ks < 8; ++ks)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * ks,
+                                make_desc(smem_u32(sm + F_QG + s * 16384 + ks * 2048), 16384, 1024), id_n,
+                                ks > 0);
+                if (!fwait(&bars.u, k & 1, err, 5, abort)) break;
+                mbar_arrive(&bars.m1);            // T', -W^T and this v slot are free
+                if (n2.ok) { issue_v(n2, s); ++v_issued[s]; }
+                if (!fwait(&bars.ur, k & 1, err, 6, abort)) break;
+                if (!fwait(&bars.sc, k & 1, err, 6, abort)) break;
+                fence_after_sync();
+                // S^T += U^T (K e^{Gl - G});  O^T += U^T Aqk^T
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tmem + TM_S, tmem + TM_U + 8 * ks,
+                                make_desc(smem_u32(sm + F_KL + s * 16384 + ks * 32), 16, 1024), id_s, 1u);
+                commit(&bars.s);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_U + 8 * ks,
+                                make_desc(smem_u32(sm + F_AQ + s * 8192 + ks * 32), 16, 1024), id_o, 1u);
+                commit(&bars.o);
+                it.next(si, slots, P);
+            }
+            commit(&bars.fin_w);
+            mbar_wait(&bars.fin_w, 0, nullptr, 0, 200);
+            for (int s = 0; s < 2; ++s)
+                while (v_seen[s] < v_issued[s]) {
+                    mbar_wait(&bars.v[s], v_seen[s] & 1, nullptr, 0, 200);
+                    ++v_seen[s];
+                }
+        }
+        __syncwarp();
+    }
+    fence_before_sync();
+    __syncthreads();
+    if (w == W_PI) tmem_dealloc(tmem, 512);
+}
+
+}  // namespace fz
+
+cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st)
+{
+    static std::atomic<uint64_t> attrs_done{0};
+    cudaError_t e = once_per_device(attrs_done, [] {
+        return cudaFuncSetAttribute(fz::chunk_fused_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    (int)fz::F_SMEM);
+    });
+    if (e) return e;
+    const int64_t chains = a.si.N * a.H;
+    if (chains <= 0 || a.si.T_total <= 0) {
+        // no tokens: the final states are the initial ones
+        if (a.hT && chains > 0) {
+            // handled by the kernel's empty-chain pass (one CTA per SM at most)
+        } else {
+            return cudaSuccess;
+        }
+    }
+    const uint64_t rows = (uint64_t)(a.si.T_total > 0 ? a.si.T_total : 1), cols = (uint64_t)a.H * fz::D;
+    CUtensorMap kmap, qmap, vmap, omap;
+    if ((e = make_tensor_map_2d(&kmap, a.k, true, cols, rows, cols * 2, 64, 64, true))) return e;
+    if ((e = make_tensor_map_2d(&qmap, a.q, true, cols, rows, cols * 2, 64, 64, true))) return e;
+    if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
+    if ((e = make_tensor_map_2d(&omap, a.out, true, cols, rows, cols * 2, fz::D, 64, false))) return e;
+    const int64_t sms = device_sm_count();
+    const unsigned grid = (unsigned)(chains < sms ? chains : sms);
+    LaunchScope scope(st, K_FUSED_TC);
+    fz::chunk_fused_tc_kernel<<<grid, fz::NT, fz::F_SMEM, st>>>(
+        kmap, qmap, vmap, omap, a.log_alpha, a.beta, a.h0, (__nv_bfloat16*)a.out, a.hT, a.scale, a.si,
+        a.H, a.slots, a.P, err);
+    return cudaGetLastError();
+}
+
+}  // namespace kda

@@ -242,6 +242,7 @@ enum KernelId {
     K_BWD_DENSE1,
     K_BWD_DENSE2,
     K_BWD_PARAM,
+    K_FUSED_TC,
     K_KERNEL_COUNT
 };
 
@@ -278,6 +279,10 @@ int64_t tc_ws_bytes_per_chunk();
 int64_t tc_seg_bytes_per_head(const SegPlan& p);
 cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, int* err,
                            cudaStream_t st);
+
+// kda_fused_tc.cu (bf16, dk = dv = 128, T_total > 0): the whole prefill in one
+// kernel, no workspace beyond the error word.
+cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st);
 
 // Device error word bits (workspace header): malformed cu_seqlens, and bounded
 // waits that gave up in the tensor-core kernels (bit 1: input copies of the prep;

@@ -16,7 +16,7 @@ namespace kda {
 static const char* const kKernelNames[K_KERNEL_COUNT] = {
     "chunk_offsets", "chunk_prep_simt", "chunk_state_simt", "decode_step",
     "chunk_prep_tc", "chunk_state_tc", "chunk_state_seg_tc", "affine_prefix", "fill",
-    "bwd_state", "bwd_dense1", "bwd_dense2", "bwd_param",
+    "bwd_state", "bwd_dense1", "bwd_dense2", "bwd_param", "chunk_fused_tc",
 };
 
 namespace {

@@ -29,11 +29,12 @@
  *    in its warning on key normalisation); the kernels do not renormalise.
  *  - `scale` multiplies q once, at the read (configurations use 1/sqrt(dk)).
  *  - log_alpha is the natural log of the per-channel decay, finite and <= 0.
- *    The tensor-core prefill path additionally assumes that, within each
- *    64-token chunk, no key channel decays by more than e^-80 over 16
- *    consecutive tokens (its exponential factors are referenced to 16-token
- *    sub-chunk starts and would leave the fp32 range beyond that); the SIMT
- *    paths have no such limit.
+ *    The default tensor-core prefill (the fused kernel) and the SIMT paths
+ *    hold at any decay rate.  The two-kernel tensor-core forms, reached only
+ *    through KDA_PREFILL_TENSORCORE_CHAIN or _SEGMENTED, assume that within
+ *    each 64-token chunk no key channel decays by more than e^-80 over 16
+ *    consecutive tokens (their exponential factors are referenced to 16-token
+ *    sub-chunk starts and would leave the fp32 range beyond that).
  *  - Supported head sizes: dk, dv in {64, 128}.  Anything else returns
  *    KDA_ERR_UNSUPPORTED.
  */
@@ -75,15 +76,22 @@ typedef enum {
  * parallel: a segment maps its entry state affinely (S -> M S + B, the
  * recurrence being linear in S), so each segment's M and B are computed
  * independently, the entry states follow from a short composition, and a last
- * parallel walk writes the outputs.  AUTO and TENSORCORE choose between the
- * two by the chain count; the last two values force one or the other.
+ * parallel walk writes the outputs.  AUTO and TENSORCORE run the fused kernel:
+ * one CTA per SM walks chains and builds each chunk's operands on chip while
+ * the previous chunk's state update runs, so only the inputs, the outputs and
+ * the states cross device memory (no workspace per chunk), and it is exact at
+ * any decay rate.  The last three values force one form; the two-kernel forms
+ * (CHAIN, SEGMENTED) keep the decay-range limit stated above.
  */
 typedef enum {
     KDA_PREFILL_AUTO = 0,      /* tensor cores for bf16 with dk = dv = 128, SIMT otherwise */
     KDA_PREFILL_SIMT = 1,      /* fp32 SIMT chunk kernels (any supported shape / dtype) */
     KDA_PREFILL_TENSORCORE = 2, /* tcgen05 chunk kernels; bf16, dk = dv = 128, < 2^31 token rows */
-    KDA_PREFILL_TENSORCORE_CHAIN = 3,     /* tcgen05, one chain per (sequence, head) */
-    KDA_PREFILL_TENSORCORE_SEGMENTED = 4  /* tcgen05, segment-parallel walk */
+    KDA_PREFILL_TENSORCORE_CHAIN = 3,     /* tcgen05, two kernels (operand image in
+                                             workspace), one chain per (sequence, head) */
+    KDA_PREFILL_TENSORCORE_SEGMENTED = 4, /* tcgen05, segment-parallel walk */
+    KDA_PREFILL_TENSORCORE_FUSED = 5      /* tcgen05, one kernel: every chunk's operands
+                                             built on chip next to the state walk */
 } kda_prefill_impl_t;
 
 /*

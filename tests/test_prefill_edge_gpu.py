@@ -27,10 +27,11 @@ def kda(cuda_ok):
     return kda
 
 
-@pytest.mark.parametrize("impl", ["simt", "tensorcore"])
+@pytest.mark.parametrize("impl", ["simt", "tensorcore_chain", "tensorcore_fused"])
 def test_head_groups_with_small_workspace(cuda_ok, impl):
-    """64 MiB budget: 512 chunks per head need about 34 MB (tensor cores) or
-    76 MB (SIMT), so the three heads run in separate groups."""
+    """64 MiB budget: 512 chunks per head need about 34 MB (two-kernel tensor-core
+    path) or 76 MB (SIMT), so the three heads run in separate groups; the fused
+    kernel needs no per-chunk workspace and runs them in one launch."""
     code = textwrap.dedent(f"""
         import sys; sys.path.insert(0, {ROOT!r}); sys.path.insert(0, {os.path.join(ROOT, 'tests')!r})
         import workloads as W, gated_delta_rule_75_b200 as kda, torch
@@ -51,7 +52,8 @@ def test_head_groups_with_small_workspace(cuda_ok, impl):
     assert r.returncode == 0, r.stdout + r.stderr
 
 
-@pytest.mark.parametrize("impl,io", [("simt", "f32"), ("tensorcore", "bf16")])
+@pytest.mark.parametrize("impl,io", [("simt", "f32"), ("tensorcore", "bf16"),
+                                     ("tensorcore_chain", "bf16")])
 def test_final_state_written_over_initial_state(kda, impl, io):
     cfg = W.small_prefill(B=2, T=130, H=2, dk=128, dv=128, io_dtype=io, seed=32, h0_std=0.05)
     inp = W.make_prefill(cfg, "cuda")
@@ -64,7 +66,7 @@ def test_final_state_written_over_initial_state(kda, impl, io):
     assert rel(out, ro) <= TOL[io] and rel(state, rh) <= TOL[io]
 
 
-@pytest.mark.parametrize("impl", ["simt", "tensorcore"])
+@pytest.mark.parametrize("impl", ["simt", "tensorcore", "tensorcore_chain"])
 @pytest.mark.parametrize("cu", [[0, 100, 50, 200], [0, 200, 0, 200], [0, 64, 300, 200], [5, 64, 128, 200]])
 def test_malformed_offsets_are_reported_not_faulted(kda, impl, cu):
     cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype="bf16", seed=33, lengths=[64, 64, 72])

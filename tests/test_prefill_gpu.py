@@ -13,7 +13,10 @@ from kda_testutil import TOL, host, oracle_pairs, oracle_prefill, rel
 
 pytestmark = pytest.mark.gpu
 
-IMPLS = ["simt", "tensorcore"]        # tensor cores: bf16 with dk = dv = 128 only
+# tensor cores: bf16 with dk = dv = 128 only; "tensorcore_fused" is the one-kernel prefill
+# (what AUTO runs with enough chains), "tensorcore_chain" the two-kernel one
+IMPLS = ["simt", "tensorcore_fused", "tensorcore_chain"]
+TC_IMPLS = ["tensorcore_fused", "tensorcore_chain"]
 
 
 @pytest.fixture(scope="module")
@@ -56,13 +59,51 @@ def test_bf16_d128_ragged(kda, impl, T):
     check_full(kda, cfg, impl)
 
 
+@pytest.mark.parametrize("impl", TC_IMPLS)
 @pytest.mark.parametrize("shift", [3.0, -4.0])
-def test_tensorcore_fast_and_slow_decay(kda, shift):
-    """Mean per-token decay e^-3.1 (fast) and e^-0.02 (slow): the sub-chunk
+def test_tensorcore_fast_and_slow_decay(kda, shift, impl):
+    """Mean per-token decay e^-3.1 (fast) and e^-0.02 (slow): the exponent
     references keep the tensor-core factors in range; parity holds."""
     cfg = W.small_prefill(B=1, T=256, H=2, dk=128, dv=128, io_dtype="bf16", seed=4,
                           gate_shift=shift, h0_std=0.02)
-    check_full(kda, cfg, "tensorcore")
+    check_full(kda, cfg, impl)
+
+
+@pytest.mark.parametrize("impl", ["auto", "tensorcore_fused"])
+@pytest.mark.parametrize("shift", [8.0, 40.0])
+def test_fused_exact_at_any_decay(kda, shift, impl):
+    """Mean per-token decay about e^-8 and e^-40 in bf16 at d = 128 through the
+    default path: the one-reference factors would leave the fp32 range, so every
+    chunk takes the level passes (all factors <= 1); parity holds."""
+    cfg = W.small_prefill(B=2, T=200, H=2, dk=128, dv=128, io_dtype="bf16", seed=12,
+                          gate_shift=shift, h0_std=0.05)
+    check_full(kda, cfg, impl)
+
+
+def test_fused_mixed_fast_and_fallback_chunks(kda):
+    """Chunks of both kinds in one call (fast decay in one sequence, slow in the
+    other, packed): the per-chunk choice of factors is independent."""
+    slow = W.small_prefill(B=1, T=190, H=2, dk=128, dv=128, io_dtype="bf16", seed=13, h0_std=0.05)
+    fast = W.small_prefill(B=1, T=130, H=2, dk=128, dv=128, io_dtype="bf16", seed=14,
+                           gate_shift=8.0, h0_std=0.05)
+    a, b = W.make_prefill(slow, "cuda"), W.make_prefill(fast, "cuda")
+    inp = {k: (torch.cat([a[k], b[k]], dim=1) if k in ("q", "k", "v", "log_alpha", "beta") else a[k])
+           for k in a}
+    inp["h0"] = torch.cat([a["h0"], b["h0"]], dim=0)
+    inp["cu_seqlens"] = torch.tensor([0, 190, 320], dtype=torch.int32, device="cuda")
+    out, hT = run(kda, inp, "tensorcore_fused")
+    ro, rh = oracle_prefill(inp)
+    eo, eh = rel(out, ro), rel(hT, rh)
+    print(f"PARITY mixed-decay fused out={eo:.3e} hT={eh:.3e}")
+    assert eo <= TOL["bf16"] and eh <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("impl", TC_IMPLS)
+def test_more_chains_than_sms(kda, impl):
+    """160 (sequence, head) chains: the fused kernel's persistent CTAs take
+    several chains each (the grid has one CTA per SM)."""
+    cfg = W.small_prefill(B=5, T=130, H=32, dk=128, dv=128, io_dtype="bf16", seed=15, h0_std=0.02)
+    check_full(kda, cfg, impl)
 
 
 @pytest.mark.parametrize("shift", [-4.0, 3.0, 3.6, 8.0])
@@ -96,14 +137,16 @@ def test_head_sizes_ragged_tail(kda, dk, dv, io):
     check_full(kda, cfg, "simt")
 
 
-@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "simt"), ("bf16", "tensorcore")])
+@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "simt"), ("bf16", "tensorcore_fused"),
+                                     ("bf16", "tensorcore_chain")])
 def test_packed_variable_lengths(kda, io, impl):
     lens = [1, 63, 64, 65, 0, 130, 200, 7]
     cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype=io, seed=7, h0_std=0.05, lengths=lens)
     check_full(kda, cfg, impl)
 
 
-@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "tensorcore")])
+@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "tensorcore_fused"),
+                                     ("bf16", "tensorcore_chain")])
 def test_packed_equals_separate_calls(kda, io, impl):
     lens = [70, 1, 129]
     cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype=io, seed=8, h0_std=0.05, lengths=lens)
@@ -123,7 +166,8 @@ def test_packed_equals_separate_calls(kda, io, impl):
 
 
 @pytest.mark.parametrize("t1", [64, 100])
-@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "tensorcore")])
+@pytest.mark.parametrize("io,impl", [("f32", "simt"), ("bf16", "tensorcore_fused"),
+                                     ("bf16", "tensorcore_chain")])
 def test_continuation_across_calls(kda, t1, io, impl):
     """[0, t1) then [t1, T) with h0 = hT of the first call equals one pass
     (on and off a chunk boundary): the state layout survives the hand-over."""

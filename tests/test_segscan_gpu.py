@@ -2,8 +2,7 @@
 C ABI, against the fp64 oracle.
 
 * the tensor-core prefill with every (sequence, head) chain cut into segments
-  (value walk, map walk, composition, final walk) -- forced, and chosen
-  automatically when the chains are too few to fill the GPU;
+  (value walk, map walk, composition, final walk), on request;
 * kda_chunk_fwd_segmap: (M, B) of each (sequence, head) vs oracle.segment_map;
 * kda_affine_prefix vs oracle.compose;
 * a sequence split into consecutive pieces run one after another on one GPU
@@ -101,19 +100,23 @@ def test_segmented_walk_on_pool_slots(kda):
 
 
 def test_automatic_choice(kda):
-    """Few chains (1 sequence x 2 heads): the walk is segmented; many chains
-    (8 x 32): one chain per (sequence, head)."""
+    """AUTO runs the fused one-kernel prefill for few chains (1 sequence x 2
+    heads) and for many (8 x 32); the segmented walk runs only when asked for."""
     kda.profiler_read(reset=True)
     cfg = W.small_prefill(B=1, T=2048, H=2, dk=128, dv=128, io_dtype="bf16", seed=11,
                           h0_std=0.02)
     _check(kda, cfg, "auto")
     st = kda.profiler_read(reset=True)
-    assert st["chunk_state_seg_tc"][0] == 2 and st["affine_prefix"][0] == 1, st
+    assert st["chunk_fused_tc"][0] == 1 and st["chunk_state_seg_tc"][0] == 0, st
     cfg = W.small_prefill(B=8, T=100, H=32, dk=128, dv=128, io_dtype="bf16", seed=12)
     inp = W.make_prefill(cfg, "cuda")
     _run(kda, inp, "auto")
     st = kda.profiler_read(reset=True)
-    assert st["chunk_state_seg_tc"][0] == 0 and st["chunk_state_tc"][0] == 1, st
+    assert st["chunk_fused_tc"][0] == 1 and st["chunk_state_tc"][0] == 0, st
+    _check(kda, W.small_prefill(B=1, T=2048, H=2, dk=128, dv=128, io_dtype="bf16", seed=11,
+                                h0_std=0.02), "tensorcore_segmented")
+    st = kda.profiler_read(reset=True)
+    assert st["chunk_state_seg_tc"][0] == 2 and st["affine_prefix"][0] == 1, st
 
 
 @pytest.mark.parametrize("io,d", [("bf16", 128), ("f32", 64), ("bf16", 64), ("f32", 128)])
