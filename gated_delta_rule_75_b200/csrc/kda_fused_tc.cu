@@ -25,16 +25,18 @@
 //   warp 13     one thread issues the walk's MMAs and v loads.
 // Per chunk, k and q land by TMA as [t][c] tiles and are transposed into tensor
 // memory by an MMA with the identity (exact), so each prep thread owns one
-// channel's tokens.  The decay factors e^{G_i - G_j} are split around one
-// reference row for the whole chunk when every factor stays within 2^100, so
-// A and Aqk are one MMA; otherwise the lower triangle is taken level by level
-// (blocks of 64, 32, ..., 2 rows; each pair i > j at the level where i and j
-// fall in different halves, both factors referenced to the first row of the
-// upper half and so <= 1), plus one product for the diagonal: exact at any
-// decay rate.  The state walk of chunk c (U^T = V^T T'^T + S^T (-W^T),
+// channel's tokens.  The decay factors e^{G_i - G_j} are split as e^{G_i} e^{-G_j}
+// when every |G| of the chunk stays within 2^100: the row operands of A and Aqk
+// are then the image tiles K e^G and Q e^G themselves, the column operand is
+// K e^{-G}, and A and Aqk are one MMA.  Otherwise the lower triangle is taken
+// level by level (blocks of 64, 32, ..., 2 rows; each pair i > j at the level
+// where i and j fall in different halves, both factors referenced to the first
+// row of the upper half and so <= 1), plus one product for the diagonal: exact
+// at any decay rate.  The state walk of chunk c (U^T = V^T T'^T + S^T (-W^T),
 // O^T = S^T (Q e^G)^T + U^T Aqk^T, S^T += U^T (K e^{Gl - G})) overlaps the prep
-// of chunk c + 1; the operands whose producer and consumer overlap are
-// double-buffered, the rest are handed over on mbarriers.  Every wait is
+// of chunk c + 1; the state's decay by the next chunk's e^{G_last} is applied
+// as the walk copies the state for that chunk.  Operands whose producer and
+// consumer overlap are double-buffered, the rest are handed over on mbarriers.  Every wait is
 // bounded; a wait that gives up sets a bit in the error word and makes every
 // role leave its loop, after which the CTA drains its copies and MMAs and
 // frees its tensor memory.
@@ -58,7 +60,7 @@ constexpr int D = 128;
 constexpr int NT = 448;
 constexpr int AP = 68;                      // row pitch (floats) of the fp32 A and T
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRange = 100.f;             // one-reference factors stay within 2^+-100
+constexpr float kRange = 100.f;             // fast path: every |G| (log2) within 100
 constexpr long long kWaitCycles = 4000000000LL;
 
 constexpr int W_WALK = 8;                   // walk warps 8-11
@@ -73,19 +75,20 @@ constexpr int NB_WALK = 7;                  // walk warps
 // Shared memory (bytes from a 1024-aligned base).  [c][t] tiles: 128 channel rows of
 // 64 tokens (128 B), 128B-swizzled -- K-major when the tokens are the reduction index,
 // MN-major when they are the M/N index.
-constexpr uint32_t F_ID = 0;                // identity 64 x 64 bf16                       8 KB
-constexpr uint32_t F_KQ = 8192;             // k | q [t][c] (TMA), then Kin^T | Qin^T       32 KB
-constexpr uint32_t F_KD = 40960;            // Kd^T, then T fp32 [64][AP]                  17 KB
-constexpr uint32_t F_KG = 58368;            // (K e^G)^T                                   16 KB
-constexpr uint32_t F_QG = 74752;            // (Q e^G)^T x 2; after use the output tile    32 KB
-constexpr uint32_t F_KL = 107520;           // (K e^{Gl - G})^T x 2                        32 KB
-constexpr uint32_t F_AQ = 140288;           // Aqk [i][j] x 2                              16 KB
-constexpr uint32_t F_TP = 156672;           // T' [i][j]                                    8 KB
-constexpr uint32_t F_W = 164864;            // A fp32 [64][AP] for the inverse, then -W^T  17 KB
-constexpr uint32_t F_V = 182272;            // v [t][dv] (TMA) x 2                         32 KB
-constexpr uint32_t F_GAM = 215040;          // e^{G_last} x 2
-constexpr uint32_t F_BETA = 216064;         // beta of the chunk
-constexpr uint32_t F_XCH = 216320;          // half sums of the decay [3][128]
+constexpr uint32_t F_ID = 0;                // identity 16 x 16 bf16 (16 rows of 128 B)     2 KB
+constexpr uint32_t F_G = 2048;              // log_alpha [t][c] fp32 (TMA, unswizzled)     32 KB
+constexpr uint32_t F_KQ = 34816;            // k | q [t][c] (TMA)                          32 KB
+constexpr uint32_t F_KD = 67584;            // (K e^{-G})^T, then T fp32 [64][AP]          17 KB
+constexpr uint32_t F_KG = 84992;            // (K e^G)^T                                   16 KB
+constexpr uint32_t F_QG = 101376;           // (Q e^G)^T x 2; after use the output tile    32 KB
+constexpr uint32_t F_KL = 134144;           // (K e^{Gl - G})^T x 2                        32 KB
+constexpr uint32_t F_AQ = 166912;           // Aqk [i][j] x 2                              16 KB
+constexpr uint32_t F_TP = 183296;           // T' [i][j]                                    8 KB
+constexpr uint32_t F_W = 191488;            // A fp32 [64][AP] for the inverse, then -W^T  17 KB
+constexpr uint32_t F_V = 208896;            // v [t][dv] (TMA)                             16 KB
+constexpr uint32_t F_GAM = 225280;          // e^{G_last} x 2
+constexpr uint32_t F_BETA = 226304;         // beta of the chunk
+constexpr uint32_t F_XCH = 226560;          // half sums of the decay [3][128]
 constexpr uint32_t F_BYTES = F_XCH + 3 * 128 * 4;
 constexpr uint32_t F_SMEM = F_BYTES + 1024;
 static_assert(F_KD + 64 * AP * 4 <= F_KG, "T scratch overlaps (K e^G)^T");
@@ -99,11 +102,11 @@ constexpr uint32_t TM_S = 128;              // S^T fp32 (state)
 constexpr uint32_t TM_U = 256;              // U^T fp32; its first 32 columns then hold U^T bf16
 constexpr uint32_t TM_O = 320;              // O^T fp32
 constexpr uint32_t TM_SB = 384;             // S^T bf16 (operand)
-constexpr uint32_t TM_D = 448;              // [Kin; Qin] Kd^T
+constexpr uint32_t TM_D = 448;              // [K e^G; Q e^G] (K e^{-G})^T
 
 struct Bars {
-    uint64_t kq, tr, ops, a, t, w, img;     // prep pipeline
-    uint64_t v[2], u, s, o, ur, sc, sr, orr, go;   // walk pipeline
+    uint64_t g, gc, kq, tr, ops, gam, a, t, w, img;   // prep pipeline
+    uint64_t v, u, s, o, ur, sr, orr;          // walk pipeline
     uint64_t m1, fr[2];                     // walk -> prep: MMA1 done, image slot free
     uint64_t fin_p, fin_w;                  // issuers' final drains
 };
@@ -151,35 +154,31 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, bool leade
     return bar_and_named(barid, count, ok);
 }
 
-// The chunks of one CTA: chains b, b + G, b + 2G, ... of the (sequence rank, head)
-// list, heads innermost; sequences ranked longest first when an order is known.
+// The chunks of one CTA: chains blockIdx.x, + gridDim.x, ... of the (sequence rank,
+// head) list, heads innermost; sequences ranked longest first when an order is known.
 // Chains without tokens are skipped (their final states are written separately).
+// Token rows and chain indices fit 32 bits (the launch checks both).
 struct Items {
-    int64_t r, rstep, rend, H;
-    int64_t n, h, bos, eos, nch, c, sidx;
+    int32_t r, h, n, bos, eos, nch, c;
+    int64_t sidx;                               // state index, -1: none
     bool ok;
 
-    __device__ __forceinline__ void init(int64_t b, int64_t step, const SeqInfo& si, int64_t H_,
-                                         const int32_t* slots, int64_t P)
-    {
-        r = b;
-        rstep = step;
-        rend = si.N * H_;
-        H = H_;
-        load(si, slots, P);
-    }
-    __device__ __forceinline__ void load(const SeqInfo& si, const int32_t* slots, int64_t P)
+    __device__ __forceinline__ void load(const SeqInfo& si, int32_t H, const int32_t* slots, int64_t P)
     {
         ok = false;
+        const int32_t rend = (int32_t)si.N * H;
         while (r < rend) {
-            const int64_t sr = r / H;
+            const int32_t sr = r / H;
             h = r - sr * H;
-            n = si.seq_of(sr);
-            seq_range(si.cu, n, si.T_seq, si.T_total, bos, eos);
+            n = (int32_t)si.seq_of(sr);
+            int64_t b, e;
+            seq_range(si.cu, n, si.T_seq, si.T_total, b, e);
+            bos = (int32_t)b;
+            eos = (int32_t)e;
             nch = (eos - bos + C - 1) / C;
             if (nch > 0) {
                 c = 0;
-                sidx = n * H + h;
+                sidx = (int64_t)n * H + h;
                 if (slots) {
                     const int64_t sl = slots[n];
                     sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
@@ -187,21 +186,26 @@ struct Items {
                 ok = true;
                 return;
             }
-            r += rstep;
+            r += (int32_t)gridDim.x;
         }
     }
-    __device__ __forceinline__ void next(const SeqInfo& si, const int32_t* slots, int64_t P)
+    __device__ __forceinline__ void init(const SeqInfo& si, int32_t H, const int32_t* slots, int64_t P)
+    {
+        r = (int32_t)blockIdx.x;
+        load(si, H, slots, P);
+    }
+    __device__ __forceinline__ void next(const SeqInfo& si, int32_t H, const int32_t* slots, int64_t P)
     {
         if (++c >= nch) {
-            r += rstep;
-            load(si, slots, P);
+            r += (int32_t)gridDim.x;
+            load(si, H, slots, P);
         }
     }
-    __device__ __forceinline__ int64_t t0() const { return bos + c * C; }
+    __device__ __forceinline__ int32_t t0() const { return bos + c * C; }
     __device__ __forceinline__ int len() const
     {
-        const int64_t l = eos - t0();
-        return (int)(l < C ? l : C);
+        const int32_t l = eos - t0();
+        return l < C ? l : C;
     }
     __device__ __forceinline__ bool first() const { return c == 0; }
     __device__ __forceinline__ bool last() const { return c + 1 == nch; }
@@ -279,6 +283,7 @@ __device__ __forceinline__ bool pass_pair(int pass, int i, int j)
 __global__ void __launch_bounds__(NT, 1)
 chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap qmap,
                       const __grid_constant__ CUtensorMap vmap, const __grid_constant__ CUtensorMap omap,
+                      const __grid_constant__ CUtensorMap gmap,
                       const float* __restrict__ log_alpha, const float* __restrict__ beta,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, float scale, SeqInfo si, int64_t H,
@@ -294,24 +299,25 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     volatile int* abort = &s_abort_raw;
 
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
+    const int32_t H32 = (int32_t)H;
     Items it0;
-    it0.init(blockIdx.x, gridDim.x, si, H, slots, P);
+    it0.init(si, H32, slots, P);
 
     if (tid == W_PI * 32) {
-        mbar_init(&bars.kq, 1); mbar_init(&bars.tr, 1); mbar_init(&bars.ops, 8);
+        mbar_init(&bars.g, 1); mbar_init(&bars.gc, 8);
+        mbar_init(&bars.kq, 1); mbar_init(&bars.tr, 1); mbar_init(&bars.ops, 8); mbar_init(&bars.gam, 8);
         mbar_init(&bars.a, 1); mbar_init(&bars.t, 8); mbar_init(&bars.w, 1); mbar_init(&bars.img, 8);
-        mbar_init(&bars.v[0], 1); mbar_init(&bars.v[1], 1);
-        mbar_init(&bars.u, 1); mbar_init(&bars.s, 1); mbar_init(&bars.o, 1);
-        mbar_init(&bars.ur, 4); mbar_init(&bars.sc, 4); mbar_init(&bars.sr, 4); mbar_init(&bars.orr, 4);
-        mbar_init(&bars.go, 1); mbar_init(&bars.m1, 1); mbar_init(&bars.fr[0], 1); mbar_init(&bars.fr[1], 1);
+        mbar_init(&bars.v, 1); mbar_init(&bars.u, 1); mbar_init(&bars.s, 1); mbar_init(&bars.o, 1);
+        mbar_init(&bars.ur, 4); mbar_init(&bars.sr, 4); mbar_init(&bars.orr, 4);
+        mbar_init(&bars.m1, 1); mbar_init(&bars.fr[0], 1); mbar_init(&bars.fr[1], 1);
         mbar_init(&bars.fin_p, 1); mbar_init(&bars.fin_w, 1);
         fence_mbar_init();
         s_abort_raw = 0;
         s_npass = 1;
     }
     if (w < 8) {                                  // the identity operand of the transposes
-        for (int e = tid; e < 512; e += 256) {
-            const int r = e >> 3, cb = e & 7;
+        if (tid < 128) {
+            const int r = tid >> 3, cb = tid & 7;
             float f[8];
 #pragma unroll
             for (int x = 0; x < 8; ++x) f[x] = (8 * cb + x == r) ? 1.f : 0.f;
@@ -337,32 +343,29 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         float* sT = reinterpret_cast<float*>(sm + F_KD);
         const int64_t rs = H * D;                 // floats between token rows of log_alpha
 
-        // this thread's 32 gates of an item (natural log; zero past its end) and, for the
-        // first 64 channels' threads, beta of row pc
-        auto load_inputs = [&](const Items& x, float* g, float& b) {
-            const int64_t t0 = x.t0();
-            const int len = x.len();
-            const float* base = log_alpha + (t0 + 32 * ph) * rs + x.h * D + pc;
-#pragma unroll
-            for (int y = 0; y < 32; ++y) g[y] = (32 * ph + y < len) ? __ldg(base + y * rs) : 0.f;
-            b = (q4 < 2 && pc < len) ? __ldg(beta + (t0 + pc) * H + x.h) : 0.f;
-        };
-
+        const float* sg = reinterpret_cast<const float*>(sm + F_G);
         Items it = it0;
-        float gv[32], bv = 0.f;
-        if (it.ok) load_inputs(it, gv, bv);
         uint32_t n_a = 0;                         // completions of bars.a seen
         for (uint32_t k = 0; it.ok; ++k) {
             const int s = (int)(k & 1);
             const int len = it.len();
+            // beta of row pc (threads of the first 64 channels), read at the extraction
+            const float bcur = (q4 < 2 && pc < len) ? __ldg(beta + ((int64_t)it.t0() + pc) * H + it.h) : 0.f;
             // ---- (a) cumulative decay of channel pc over this half's tokens, log2 units
+            // (rows past the chunk's end add nothing)
+            bool ok = true;
+            if (leader) ok = fwait(&bars.g, k & 1, err, 1, abort);
+            if (!bar_and_named(NB_PREP, 256, ok)) break;
             float G[32];
             float run = 0.f;
 #pragma unroll
             for (int y = 0; y < 32; ++y) {
-                run += kLog2e * gv[y];
+                const float gy = sg[(32 * ph + y) * D + pc];
+                run += (32 * ph + y < len) ? kLog2e * gy : 0.f;
                 G[y] = run;
             }
+            __syncwarp();
+            if (l == 0) mbar_arrive(&bars.gc);    // the gate tile may take the next chunk's
             xch[ph * 128 + pc] = run;
             if (ph == 1) xch[256 + pc] = G[0];
             bar_sync_named(NB_PAIR + q4, 64);
@@ -372,25 +375,25 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 #pragma unroll
                 for (int y = 0; y < 32; ++y) G[y] += s0;
             }
-            const float Gm = s0, Gl = s0 + s1;    // reference row 31, last row
+            const float Gl = s0 + s1;             // last row
             float mx = 0.f;
 #pragma unroll
-            for (int y = 0; y < 32; ++y) mx = fmaxf(mx, fabsf(G[y] - Gm));
-            const float bcur = bv;
-            Items nx = it;
-            nx.next(si, slots, P);
-            if (nx.ok) load_inputs(nx, gv, bv);   // in flight during this chunk
+            for (int y = 0; y < 32; ++y) mx = fmaxf(mx, fabsf(G[y]));
 
-            // k^T, q^T of this chunk in TMEM; image slot s free (chunk k - 2 walked);
-            // T', -W^T and the A scratch free (MMA1 of chunk k - 1 done)
-            bool ok = true;
+            // k^T, q^T of this chunk in TMEM; image slot s free (chunk k - 2 walked)
             if (leader) {
                 ok = fwait(&bars.tr, k & 1, err, 1, abort);
                 if (ok && k >= 2) ok = fwait(&bars.fr[s], ((k - 2) >> 1) & 1, err, 6, abort);
-                if (ok && k >= 1) ok = fwait(&bars.m1, (k - 1) & 1, err, 6, abort);
             }
             if (!bar_and_named(NB_PREP, 256, ok)) break;
             fence_after_sync();
+            // T', -W^T and the A scratch (all in place of the previous chunk's): free once
+            // MMA1 of chunk k - 1 has completed
+            auto wait_m1 = [&]() -> bool {
+                bool o = true;
+                if (leader && k >= 1) o = fwait(&bars.m1, (k - 1) & 1, err, 6, abort);
+                return bar_and_named(NB_PREP, 256, o);
+            };
             const bool fast = bar_and_named(NB_PREP, 256, !(mx > kRange));
             if (leader) s_npass = fast ? 1 : 7;
 
@@ -407,11 +410,11 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                         if (32 * ph + 16 * hb + y >= len) kf[y] = qf[y] = 0.f;
                 }
             };
-            auto ops_arrive = [&] {
+            auto warp_arrive = [&](uint64_t* b) {
                 fence_smem_to_async();
                 fence_before_sync();
                 __syncwarp();
-                if (l == 0) mbar_arrive(&bars.ops);
+                if (l == 0) mbar_arrive(b);
             };
             auto wait_a = [&]() -> bool {
                 bool o2 = true;
@@ -421,44 +424,41 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 fence_after_sync();
                 return o2;
             };
+            auto put_gamma = [&] {
+                if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
+            };
 
             if (fast) {
-                // ---- (b1) one reference: Kin = k e^{G - Gm}, Qin, Kd = k e^{Gm - G}, and the
-                // image tiles K e^G = Kin e^{Gm}, Q e^G, K e^{Gl - G} = Kd e^{Gl - Gm}
-                const float Em = ex2(Gm), Egl = ex2(Gl - Gm);
+                // ---- (b1) e^{G_i - G_j} = e^{G_i} e^{-G_j}: the image tiles K e^G, Q e^G are the
+                // row operands of A and Aqk, K e^{-G} the column operand; K e^{Gl - G} = K e^{-G} e^{Gl}
+                const float Egl = ex2(Gl);
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
                     float kf[16], qf[16];
                     load_kq(hb, kf, qf);
 #pragma unroll
                     for (int m = 0; m < 2; ++m) {
-                        float kin[8], qin[8], kd[8], t1[8];
+                        float a8[8], b8[8], c8[8], d8[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int y = 8 * m + e;
-                            const float x = G[16 * hb + y] - Gm;
-                            const float e1 = ex2(x), e2 = ex2(-x);
-                            kin[e] = kf[y] * e1;
-                            qin[e] = qf[y] * e1;
-                            kd[e] = kf[y] * e2;
+                            const float e1 = ex2(G[16 * hb + y]), e2 = ex2(-G[16 * hb + y]);
+                            a8[e] = kf[y] * e1;
+                            b8[e] = qf[y] * e1;
+                            c8[e] = kf[y] * e2;
+                            d8[e] = c8[e] * Egl;
                         }
                         const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
-                        *reinterpret_cast<uint4*>(sm + F_KQ + off) = pack8(kin);
-                        *reinterpret_cast<uint4*>(sm + F_KQ + 16384 + off) = pack8(qin);
-                        *reinterpret_cast<uint4*>(sm + F_KD + off) = pack8(kd);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) t1[e] = kin[e] * Em;
-                        *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(t1);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) t1[e] = qin[e] * Em;
-                        *reinterpret_cast<uint4*>(qg + off) = pack8(t1);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) t1[e] = kd[e] * Egl;
-                        *reinterpret_cast<uint4*>(kl + off) = pack8(t1);
+                        *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(a8);
+                        *reinterpret_cast<uint4*>(qg + off) = pack8(b8);
+                        *reinterpret_cast<uint4*>(sm + F_KD + off) = pack8(c8);
+                        *reinterpret_cast<uint4*>(kl + off) = pack8(d8);
                     }
                 }
-                if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
-                ops_arrive();
+                put_gamma();
+                warp_arrive(&bars.ops);
+                warp_arrive(&bars.gam);
+                if (!wait_m1()) break;
                 if (!wait_a()) break;
                 // ---- A (fp32, beta-scaled rows, for the inverse) and Aqk (bf16 image)
                 float d[32];
@@ -484,7 +484,9 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                     }
                 }
             } else {
-                // ---- (b1') the level passes: every factor <= 1 (log_alpha <= 0)
+                // ---- (b1') the level passes: every factor <= 1 (log_alpha <= 0).  The image
+                // tiles K e^G and Q e^G hold each pass's row operands and are written last.
+                if (!wait_m1()) break;
                 for (int e = tid; e < 64 * AP / 4; e += 256)
                     reinterpret_cast<float4*>(sA)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
                 for (int e = tid; e < 512; e += 256)
@@ -494,30 +496,24 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 #pragma unroll
                 for (int y = 0; y < 32; ++y) Gs[y] = G[y];
 #pragma unroll
-                for (int hb = 0; hb < 2; ++hb) {  // image tiles from e^G and e^{Gl - G} directly
+                for (int hb = 0; hb < 2; ++hb) {  // K e^{Gl - G} (<= 1) and e^{G_last}
                     float kf[16], qf[16];
                     load_kq(hb, kf, qf);
 #pragma unroll
                     for (int m = 0; m < 2; ++m) {
-                        float a8[8], b8[8], c8[8];
+                        float c8[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int y = 8 * m + e;
-                            const float eg = ex2(G[16 * hb + y]), egl = ex2(Gl - G[16 * hb + y]);
-                            a8[e] = kf[y] * eg;
-                            b8[e] = qf[y] * eg;
-                            c8[e] = kf[y] * egl;
-                        }
-                        const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
-                        *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(a8);
-                        *reinterpret_cast<uint4*>(qg + off) = pack8(b8);
-                        *reinterpret_cast<uint4*>(kl + off) = pack8(c8);
+                        for (int e = 0; e < 8; ++e) c8[e] = kf[8 * m + e] * ex2(Gl - G[16 * hb + 8 * m + e]);
+                        *reinterpret_cast<uint4*>(kl + ct_off(pc, 32 * ph + 16 * hb + 8 * m)) = pack8(c8);
                     }
                 }
-                if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
+                put_gamma();
+                warp_arrive(&bars.gam);
                 bar_sync_named(NB_PREP, 256);     // zeroed A / Aqk before any pass writes
                 bool pok = true;
-                for (int pass = 0; pass < 7 && pok; ++pass) {
+                for (int pass = 0; pass < 8 && pok; ++pass) {
+                    // passes 0-5: the levels; 6: the diagonal; 7: the image tiles K e^G, Q e^G
+                    // (no MMA)
                     const int hs = 32 >> pass;    // half block of this level (pass < 6)
 #pragma unroll
                     for (int hb = 0; hb < 2; ++hb) {
@@ -529,8 +525,9 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 #pragma unroll
                             for (int e = 0; e < 8; ++e) {
                                 const int y = 8 * m + e, t = 32 * ph + 16 * hb + y;
-                                if (pass == 6) {
-                                    kin[e] = kf[y]; qin[e] = qf[y]; kd[e] = kf[y];
+                                if (pass >= 6) {
+                                    const float eg = pass == 7 ? ex2(G[16 * hb + y]) : 1.f;
+                                    kin[e] = kf[y] * eg; qin[e] = qf[y] * eg; kd[e] = kf[y];
                                 } else {
                                     const bool up = (t & (2 * hs - 1)) >= hs;
                                     const int f = (t & ~(2 * hs - 1)) + hs;
@@ -543,12 +540,13 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                                 }
                             }
                             const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
-                            *reinterpret_cast<uint4*>(sm + F_KQ + off) = pack8(kin);
-                            *reinterpret_cast<uint4*>(sm + F_KQ + 16384 + off) = pack8(qin);
-                            *reinterpret_cast<uint4*>(sm + F_KD + off) = pack8(kd);
+                            *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(kin);
+                            *reinterpret_cast<uint4*>(qg + off) = pack8(qin);
+                            if (pass < 7) *reinterpret_cast<uint4*>(sm + F_KD + off) = pack8(kd);
                         }
                     }
-                    ops_arrive();
+                    if (pass == 7) break;
+                    warp_arrive(&bars.ops);
                     if (!(pok = wait_a())) break;
                     float d[32];
                     tmem_ld16(tmem + lane + TM_D + 32 * ph, d);
@@ -570,7 +568,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 }
                 if (!pok) break;
             }
-            fence_smem_to_async();                // Aqk: read by the walk's MMAs
+            fence_smem_to_async();                // Aqk, K e^G, Q e^G: read by the async proxy
             bar_sync_named(NB_PREP, 256);         // A complete
             // ---- (b2) T = (I + A)^{-1} (warps 0-3)
             if (w < 4) invert_unit_lower(sA, sT, tid);
@@ -589,10 +587,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 }
                 *reinterpret_cast<uint4*>(sm + F_TP + sw128_offset(i, 8 * cb)) = u;
             }
-            fence_smem_to_async();
-            fence_before_sync();
-            __syncwarp();
-            if (l == 0) mbar_arrive(&bars.t);
+            warp_arrive(&bars.t);
             // ---- (b3) -W^T = -(K e^G)^T T'^T from TMEM into the image, [c][i]
             ok = true;
             if (leader) ok = fwait(&bars.w, k & 1, err, 3, abort);
@@ -607,11 +602,8 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 for (int m = 0; m < 4; ++m)
                     *reinterpret_cast<uint4*>(sm + F_W + sw128_offset(pc, 32 * ph + 8 * m)) = pack8(f + 8 * m);
             }
-            fence_smem_to_async();
-            fence_before_sync();
-            __syncwarp();
-            if (l == 0) mbar_arrive(&bars.img);
-            it = nx;
+            warp_arrive(&bars.img);
+            it.next(si, H32, slots, P);
         }
     } else if (w < W_PI) {
         // ------------------------------------------------------------------ walk
@@ -644,80 +636,90 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             fence_after_sync();
             return o;
         };
+        // S^T fp32 -> bf16 operand copy; the fp32 state then decays by the next chunk's
+        // e^{G_last} (slot g) before its update MMA accumulates onto it.  `src` (nullable:
+        // zeros) replaces the TMEM state when a chain starts.
+        auto stage_state = [&](const float* src, int g) {
+            const float* gam = reinterpret_cast<const float*>(sm + F_GAM + g * 512);
+#pragma unroll 1
+            for (int cb = 0; cb < 4; ++cb) {
+                float f[32];
+                if (src) {
+#pragma unroll
+                    for (int y = 0; y < 32; ++y) f[y] = src[(32 * cb + y) * D + j];
+                } else {
+                    tmem_ld16(tmem + lane + TM_S + 32 * cb, f);
+                    tmem_ld16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
+                    tmem_wait_ld();
+                }
+                uint32_t u[16];
+#pragma unroll
+                for (int y = 0; y < 16; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
+                tmem_st16u(tmem + lane + TM_SB + 16 * cb, u);
+                float g8[32];
+#pragma unroll
+                for (int y = 0; y < 32; y += 8) ld8f(gam + 32 * cb + y, g8 + y);
+#pragma unroll
+                for (int y = 0; y < 32; ++y) f[y] *= g8[y];
+                tmem_st16(tmem + lane + TM_S + 32 * cb, f);
+                tmem_st16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
+            }
+            tmem_wait_st();
+            arrive4(&bars.sr);
+        };
         Items it = it0;
         for (uint32_t k = 0; it.ok; ++k) {
             const int s = (int)(k & 1);
-            if (slots && it.first() && wlead && err) {
-                const int64_t sl = slots[it.n];
-                if (sl >= P) atomicOr(err, 1);
-            }
-            if (it.first()) {                     // entry state: fp32 and its bf16 operand copy
-                const float* hp = (h0 && it.sidx >= 0) ? h0 + it.sidx * D * D : nullptr;
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
+            if (it.first()) {                     // entry state (h0 or zeros), decayed by this chunk
+                if (slots && wlead && err) {
+                    const int64_t sl = slots[it.n];
+                    if (sl >= P) atomicOr(err, 1);
+                }
+                if (!wwait(&bars.gam, k & 1, 6)) break;
+                if (h0 && it.sidx >= 0) {
+                    stage_state(h0 + it.sidx * D * D, s);
+                } else {
                     float f[32];
 #pragma unroll
-                    for (int y = 0; y < 32; ++y) f[y] = hp ? hp[(32 * cb + y) * D + j] : 0.f;
-                    tmem_st16(tmem + lane + TM_S + 32 * cb, f);
-                    tmem_st16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
-                    uint32_t u[16];
-#pragma unroll
-                    for (int y = 0; y < 16; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
-                    tmem_st16u(tmem + lane + TM_SB + 16 * cb, u);
-                }
-                tmem_wait_st();
-                arrive4(&bars.sr);
-            }
-            // the state decays by this chunk's e^{G_last} once MMA1 (which reads only the
-            // bf16 copy) is issued; MMA2 accumulates onto the scaled state
-            if (!wwait(&bars.go, k & 1, 6)) break;
-            {
-                const float* gam = reinterpret_cast<const float*>(sm + F_GAM + s * 512);
+                    for (int y = 0; y < 32; ++y) f[y] = 0.f;
 #pragma unroll 1
-                for (int cb = 0; cb < 8; ++cb) {
-                    float f[16], g8[16];
-                    tmem_ld16(tmem + lane + TM_S + 16 * cb, f);
-                    ld8f(gam + 16 * cb, g8);
-                    ld8f(gam + 16 * cb + 8, g8 + 8);
-                    tmem_wait_ld();
+                    for (int cb = 0; cb < 4; ++cb) {
+                        tmem_st16(tmem + lane + TM_S + 32 * cb, f);
+                        tmem_st16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
+                        uint32_t u[16];
 #pragma unroll
-                    for (int y = 0; y < 16; ++y) f[y] *= g8[y];
-                    tmem_st16(tmem + lane + TM_S + 16 * cb, f);
+                        for (int y = 0; y < 16; ++y) u[y] = 0u;
+                        tmem_st16u(tmem + lane + TM_SB + 16 * cb, u);
+                    }
+                    tmem_wait_st();
+                    arrive4(&bars.sr);
                 }
-                tmem_wait_st();
-                arrive4(&bars.sc);
             }
             // U^T -> bf16 operand (first 32 columns of its own TMEM range)
             if (!wwait(&bars.u, k & 1, 5)) break;
             {
-                float f[64];
-#pragma unroll
-                for (int x = 0; x < 4; ++x) tmem_ld16(tmem + lane + TM_U + 16 * x, f + 16 * x);
+                // all 64 columns are read before the packed halves overwrite the first 32
+                float f[32], g[32];
+                tmem_ld16(tmem + lane + TM_U, f);
+                tmem_ld16(tmem + lane + TM_U + 16, f + 16);
+                tmem_ld16(tmem + lane + TM_U + 32, g);
+                tmem_ld16(tmem + lane + TM_U + 48, g + 16);
                 tmem_wait_ld();
-                uint32_t u[32];
+                uint32_t u[16];
 #pragma unroll
-                for (int y = 0; y < 32; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
+                for (int y = 0; y < 16; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
                 tmem_st16u(tmem + lane + TM_U, u);
-                tmem_st16u(tmem + lane + TM_U + 16, u + 16);
+#pragma unroll
+                for (int y = 0; y < 16; ++y) u[y] = pack_bf16(g[2 * y], g[2 * y + 1]);
+                tmem_st16u(tmem + lane + TM_U + 16, u);
                 tmem_wait_st();
                 arrive4(&bars.ur);
             }
-            // next entry state -> bf16 operand, or the final state
+            // next entry state -> bf16 operand and decay, or the final state
             if (!wwait(&bars.s, k & 1, 5)) break;
             if (!it.last()) {
-#pragma unroll 1
-                for (int cb = 0; cb < 4; ++cb) {
-                    float f[32];
-                    tmem_ld16(tmem + lane + TM_S + 32 * cb, f);
-                    tmem_ld16(tmem + lane + TM_S + 32 * cb + 16, f + 16);
-                    tmem_wait_ld();
-                    uint32_t u[16];
-#pragma unroll
-                    for (int y = 0; y < 16; ++y) u[y] = pack_bf16(f[2 * y], f[2 * y + 1]);
-                    tmem_st16u(tmem + lane + TM_SB + 16 * cb, u);
-                }
-                tmem_wait_st();
-                arrive4(&bars.sr);
+                if (!wwait(&bars.gam, (k + 1) & 1, 6)) break;
+                stage_state(nullptr, s ^ 1);
             } else if (hT && it.sidx >= 0) {
                 float* hp = hT + it.sidx * D * D;
 #pragma unroll 1
@@ -730,21 +732,19 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 }
             }
             // output rows: [t][dv] bf16 tile in the consumed (Q e^G)^T slot, one tensor store
+            // per whole chunk; the image slot is released once the store has read it
             if (!wwait(&bars.o, k & 1, 5)) break;
             unsigned char* stg = sm + F_QG + s * 16384;
             {
-#pragma unroll 1
-                for (int x = 0; x < 4; ++x) {
-                    float f[16];
-                    tmem_ld16(tmem + lane + TM_O + 16 * x, f);
-                    tmem_wait_ld();
+                float f[64];
 #pragma unroll
-                    for (int y = 0; y < 16; ++y)
-                        *reinterpret_cast<__nv_bfloat16*>(stg + (16 * x + y) * 256 + 2 * j) =
-                            __float2bfloat16_rn(scale * f[y]);
-                }
+                for (int x = 0; x < 4; ++x) tmem_ld16(tmem + lane + TM_O + 16 * x, f + 16 * x);
+                tmem_wait_ld();
+                arrive4(&bars.orr);
+#pragma unroll
+                for (int t = 0; t < 64; ++t)
+                    *reinterpret_cast<__nv_bfloat16*>(stg + t * 256 + 2 * j) = __float2bfloat16_rn(scale * f[t]);
             }
-            arrive4(&bars.orr);
             fence_smem_to_async();
             bar_sync_named(NB_WALK, 128);
             const int len = it.len();
@@ -765,12 +765,16 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 bar_sync_named(NB_WALK, 128);
                 if (wlead) mbar_arrive(&bars.fr[s]);
             }
-            it.next(si, slots, P);
+            it.next(si, H32, slots, P);
         }
         if (wlead) tma::bulk_wait_all();
     } else if (w == W_PI) {
         // ------------------------------------------------------------------ prep issuer
         if (l == 0) {
+            auto issue_g = [&](const Items& x) {
+                tma::expect_tx(&bars.g, 32768);
+                tma::load_2d(sm + F_G, &gmap, (int32_t)(x.h * D), (int32_t)x.t0(), &bars.g);
+            };
             auto issue_kq = [&](const Items& x) {
                 const int32_t y = (int32_t)x.t0(), xc = (int32_t)(x.h * D);
                 tma::expect_tx(&bars.kq, 32768);
@@ -780,45 +784,50 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 tma::load_2d(sm + F_KQ + 24576, &qmap, xc + 64, y, &bars.kq);
             };
             Items it = it0;
-            uint32_t n_ops = 0, kq_issued = 0, kq_seen = 0;
-            if (it.ok) { issue_kq(it); ++kq_issued; }
+            uint32_t n_ops = 0, kq_issued = 0, kq_seen = 0, g_issued = 0;
+            if (it.ok) { issue_g(it); ++g_issued; issue_kq(it); ++kq_issued; }
             for (uint32_t k = 0; it.ok; ++k) {
                 Items nx = it;
-                nx.next(si, slots, P);
+                nx.next(si, H32, slots, P);
                 if (!fwait(&bars.kq, k & 1, err, 1, abort)) break;
                 ++kq_seen;
                 if (k > 0 && !fwait(&bars.img, (k - 1) & 1, err, 6, abort)) break;
                 fence_after_sync();
-                {                                 // k^T, q^T = [t][c]^T I (exact)
-                    const uint32_t id = make_idesc_bf16(128, 64, true, false);
+                {                                 // k^T, q^T: each 16-token block times I16 (exact)
+                    const uint32_t id = make_idesc_bf16(128, 16, true, false);
+                    const uint64_t bi = make_desc(smem_u32(sm + F_ID), 16, 1024);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(tmem + TM_KT, make_desc(smem_u32(sm + F_KQ + ks * 2048), 8192, 1024),
-                                 make_desc(smem_u32(sm + F_ID + ks * 32), 16, 1024), id, ks > 0);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(tmem + TM_QT, make_desc(smem_u32(sm + F_KQ + 16384 + ks * 2048), 8192, 1024),
-                                 make_desc(smem_u32(sm + F_ID + ks * 32), 16, 1024), id, ks > 0);
+                    for (int ks = 0; ks < 4; ++ks) {
+                        mma_bf16(tmem + TM_KT + 16 * ks, make_desc(smem_u32(sm + F_KQ + ks * 2048), 8192, 1024),
+                                 bi, id, 0u);
+                        mma_bf16(tmem + TM_QT + 16 * ks,
+                                 make_desc(smem_u32(sm + F_KQ + 16384 + ks * 2048), 8192, 1024), bi, id, 0u);
+                    }
                     commit(&bars.tr);
                 }
+                // the k / q buffer is free once the transposes have read it, the gate tile once
+                // the prep threads have scanned it
+                if (!fwait(&bars.tr, k & 1, err, 1, abort)) break;
+                if (nx.ok) { issue_kq(nx); ++kq_issued; }
+                if (!fwait(&bars.gc, k & 1, err, 6, abort)) break;
+                if (nx.ok) { issue_g(nx); ++g_issued; }
+                const uint32_t s = k & 1;
                 bool ok = true;
                 int np = 1;
-                for (int p = 0; p < np; ++p) {    // [Kin; Qin] Kd^T, once per pass
+                for (int p = 0; p < np; ++p) {    // [K e^G; Q e^G] (K e^{-G})^T, once per pass
                     if (!(ok = fwait(&bars.ops, n_ops & 1, err, 6, abort))) break;
                     ++n_ops;
                     if (p == 0) np = *reinterpret_cast<volatile int*>(&s_npass);
                     fence_after_sync();
                     const uint32_t id = make_idesc_bf16(128, 64, true, true);
+                    const uint32_t lbo = F_QG + s * 16384 - F_KG;    // K e^G -> Q e^G block
 #pragma unroll
                     for (int ks = 0; ks < 8; ++ks)
-                        mma_bf16(tmem + TM_D, make_desc(smem_u32(sm + F_KQ + ks * 2048), 16384, 1024),
+                        mma_bf16(tmem + TM_D, make_desc(smem_u32(sm + F_KG + ks * 2048), lbo, 1024),
                                  make_desc(smem_u32(sm + F_KD + ks * 2048), 16384, 1024), id, ks > 0);
                     commit(&bars.a);
                 }
                 if (!ok) break;
-                // the k / q buffer is free once the last pass has read its operands
-                if (!fwait(&bars.a, (n_ops - 1) & 1, err, 2, abort)) break;
-                if (nx.ok) { issue_kq(nx); ++kq_issued; }
                 if (!fwait(&bars.t, k & 1, err, 6, abort)) break;
                 fence_after_sync();
                 {                                 // -W^T = -(K e^G)^T T'^T
@@ -838,50 +847,47 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 mbar_wait(&bars.kq, kq_seen & 1, nullptr, 0, 200);
                 ++kq_seen;
             }
+            // gate tiles: the prep threads wait for each one they scan; at most the one issued
+            // for a chunk that was never started is left in flight
+            if (*abort) mbar_wait(&bars.g, (g_issued - 1) & 1, nullptr, 0, 200);
         }
         __syncwarp();
     } else {
         // ------------------------------------------------------------------ walk issuer
         if (l == 0) {
-            auto issue_v = [&](const Items& x, int slot) {
+            auto issue_v = [&](const Items& x) {
                 const int32_t y = (int32_t)x.t0(), xc = (int32_t)(x.h * D);
-                tma::expect_tx(&bars.v[slot], 16384);
-                tma::load_2d(sm + F_V + slot * 16384, &vmap, xc, y, &bars.v[slot]);
-                tma::load_2d(sm + F_V + slot * 16384 + 8192, &vmap, xc + 64, y, &bars.v[slot]);
+                tma::expect_tx(&bars.v, 16384);
+                tma::load_2d(sm + F_V, &vmap, xc, y, &bars.v);
+                tma::load_2d(sm + F_V + 8192, &vmap, xc + 64, y, &bars.v);
             };
             Items it = it0;
-            uint32_t v_issued[2] = {0, 0}, v_seen[2] = {0, 0};
-            {
-                Items i1 = it;
-                if (i1.ok) { issue_v(i1, 0); ++v_issued[0]; i1.next(si, slots, P); }
-                if (i1.ok) { issue_v(i1, 1); ++v_issued[1]; }
-            }
+            uint32_t v_issued = 0, v_seen = 0;
+            if (it.ok) { issue_v(it); ++v_issued; }
             const uint32_t id_v = make_idesc_bf16(128, 64, true, false);   // V^T T'^T
             const uint32_t id_n = make_idesc_bf16(128, 64, false, true);   // S^T x MN-major B
             const uint32_t id_s = make_idesc_bf16(128, 128, false, false); // U^T (K e^{Gl-G})
             const uint32_t id_o = make_idesc_bf16(128, 64, false, false);  // U^T Aqk^T
             for (uint32_t k = 0; it.ok; ++k) {
                 const int s = (int)(k & 1);
-                Items n2 = it;
-                n2.next(si, slots, P);
-                if (n2.ok) n2.next(si, slots, P);
+                Items nx = it;
+                nx.next(si, H32, slots, P);
                 if (!fwait(&bars.img, k & 1, err, 6, abort)) break;
-                if (!fwait(&bars.v[s], (k >> 1) & 1, err, 4, abort)) break;
-                ++v_seen[s];
+                if (!fwait(&bars.v, k & 1, err, 4, abort)) break;
+                ++v_seen;
                 if (!fwait(&bars.sr, k & 1, err, 6, abort)) break;
                 if (k > 0 && !fwait(&bars.o, (k - 1) & 1, err, 5, abort)) break;
                 fence_after_sync();
                 // U^T = V^T T'^T + S^T (-W^T)
 #pragma unroll
                 for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + TM_U, make_desc(smem_u32(sm + F_V + s * 16384 + ks * 2048), 8192, 1024),
+                    mma_bf16(tmem + TM_U, make_desc(smem_u32(sm + F_V + ks * 2048), 8192, 1024),
                              make_desc(smem_u32(sm + F_TP + ks * 32), 16, 1024), id_v, ks > 0);
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
                     mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * ks,
                                 make_desc(smem_u32(sm + F_W + ks * 2048), 16384, 1024), id_n, 1u);
                 commit(&bars.u);
-                mbar_arrive(&bars.go);
                 // O^T = S^T (Q e^G)^T (the output tile of the previous chunk has left TMEM)
                 if (k > 0 && !fwait(&bars.orr, (k - 1) & 1, err, 6, abort)) break;
                 fence_after_sync();
@@ -891,10 +897,9 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                                 make_desc(smem_u32(sm + F_QG + s * 16384 + ks * 2048), 16384, 1024), id_n,
                                 ks > 0);
                 if (!fwait(&bars.u, k & 1, err, 5, abort)) break;
-                mbar_arrive(&bars.m1);            // T', -W^T and this v slot are free
-                if (n2.ok) { issue_v(n2, s); ++v_issued[s]; }
+                mbar_arrive(&bars.m1);            // T', -W^T and the v tile are free
+                if (nx.ok) { issue_v(nx); ++v_issued; }
                 if (!fwait(&bars.ur, k & 1, err, 6, abort)) break;
-                if (!fwait(&bars.sc, k & 1, err, 6, abort)) break;
                 fence_after_sync();
                 // S^T += U^T (K e^{Gl - G});  O^T += U^T Aqk^T
 #pragma unroll
@@ -907,15 +912,14 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                     mma_bf16_ts(tmem + TM_O, tmem + TM_U + 8 * ks,
                                 make_desc(smem_u32(sm + F_AQ + s * 8192 + ks * 32), 16, 1024), id_o, 1u);
                 commit(&bars.o);
-                it.next(si, slots, P);
+                it = nx;
             }
             commit(&bars.fin_w);
             mbar_wait(&bars.fin_w, 0, nullptr, 0, 200);
-            for (int s = 0; s < 2; ++s)
-                while (v_seen[s] < v_issued[s]) {
-                    mbar_wait(&bars.v[s], v_seen[s] & 1, nullptr, 0, 200);
-                    ++v_seen[s];
-                }
+            while (v_seen < v_issued) {
+                mbar_wait(&bars.v, v_seen & 1, nullptr, 0, 200);
+                ++v_seen;
+            }
         }
         __syncwarp();
     }
@@ -949,11 +953,13 @@ cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st)
     if ((e = make_tensor_map_2d(&qmap, a.q, true, cols, rows, cols * 2, 64, 64, true))) return e;
     if ((e = make_tensor_map_2d(&vmap, a.v, true, cols, rows, cols * 2, 64, 64, true))) return e;
     if ((e = make_tensor_map_2d(&omap, a.out, true, cols, rows, cols * 2, fz::D, 64, false))) return e;
+    CUtensorMap gmap;                             // log_alpha [tokens][H * D] fp32, 128 x 64 boxes
+    if ((e = make_tensor_map_2d(&gmap, a.log_alpha, false, cols, rows, cols * 4, fz::D, 64, false))) return e;
     const int64_t sms = device_sm_count();
     const unsigned grid = (unsigned)(chains < sms ? chains : sms);
     LaunchScope scope(st, K_FUSED_TC);
     fz::chunk_fused_tc_kernel<<<grid, fz::NT, fz::F_SMEM, st>>>(
-        kmap, qmap, vmap, omap, a.log_alpha, a.beta, a.h0, (__nv_bfloat16*)a.out, a.hT, a.scale, a.si,
+        kmap, qmap, vmap, omap, gmap, a.log_alpha, a.beta, a.h0, (__nv_bfloat16*)a.out, a.hT, a.scale, a.si,
         a.H, a.slots, a.P, err);
     return cudaGetLastError();
 }
