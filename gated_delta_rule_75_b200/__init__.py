@@ -85,6 +85,10 @@ def _load():
     lib.kda_debug_prep_image.restype = ctypes.c_int
     lib.kda_debug_bounded_wait.argtypes = [ctypes.c_int32, vp, vp]
     lib.kda_debug_bounded_wait.restype = ctypes.c_int
+    lib.kda_workspace_high_water.argtypes = [ctypes.POINTER(ctypes.c_int64), ctypes.c_int]
+    lib.kda_workspace_high_water.restype = ctypes.c_int
+    lib.kda_get_error.argtypes = [vp, ctypes.POINTER(ctypes.c_int32)]
+    lib.kda_get_error.restype = ctypes.c_int
     lib.kda_profiler_enable.argtypes = [ctypes.c_int]
     lib.kda_profiler_enable.restype = None
     lib.kda_profiler_read.argtypes = [ctypes.POINTER(_KernelStat), ctypes.c_int, ctypes.c_int]
@@ -402,11 +406,41 @@ def gdn_chunk_bwd(q, k, v, log_a, beta, scale, dout, h0=None, dhT=None, cu_seqle
 IMAGE_BYTES = 66560   # one (chunk, head) operand image of the tensor-core prefill
 
 
-def debug_bounded_wait(polls, device="cuda"):
+def get_error(device="cuda") -> int:
+    """C ABI ``kda_get_error``: takes (reads and clears) the device's error word
+    after the work queued on the current stream; bit 0 = malformed cu_seqlens or a
+    slot out of range, bits 1-6 = a bounded device wait gave up."""
+    dev = torch.device(device)
+    word = ctypes.c_int32(0)
+    with torch.cuda.device(dev):
+        st = _load().kda_get_error(_stream(dev), ctypes.byref(word))
+    if st != 0:
+        raise KDAError(st, "kda_get_error")
+    return int(word.value)
+
+
+def workspace_high_water(reset=False, device="cuda") -> int:
+    """C ABI ``kda_workspace_high_water``: the most workspace bytes the library had
+    allocated at once on ``device`` since the last reset; ``reset`` restarts it."""
+    v = ctypes.c_int64(0)
+    with torch.cuda.device(torch.device(device)):
+        st = _load().kda_workspace_high_water(ctypes.byref(v), 1 if reset else 0)
+    if st != 0:
+        raise KDAError(st, "kda_workspace_high_water")
+    return int(v.value)
+
+
+def debug_bounded_wait(polls, device="cuda", to_library_word=False):
     """Self-test (C ABI ``kda_debug_bounded_wait``): a device wait on a barrier that
     nothing completes, given up after ``polls`` polls.  Returns the status code
-    (KDA_ERR_TIMEOUT expected) and the error word the kernel wrote."""
+    (KDA_ERR_TIMEOUT expected) and the error word the kernel wrote; with
+    ``to_library_word`` the bits go to the library's error word instead (read them
+    with ``get_error``) and the word returned is None."""
     dev = torch.device(device)
+    if to_library_word:
+        with torch.cuda.device(dev):
+            st = _load().kda_debug_bounded_wait(int(polls), None, _stream(dev))
+        return st, None
     word = torch.zeros(1, dtype=torch.int32, device=dev)
     st = _load().kda_debug_bounded_wait(int(polls), _ptr(word), _stream(dev))
     return st, int(word.item())

@@ -12,7 +12,7 @@
 
 namespace kda {
 
-static bool debug_mode()
+bool debug_mode_on()
 {
     static const bool on = [] {
         const char* s = std::getenv("KDA_DEBUG");
@@ -20,6 +20,8 @@ static bool debug_mode()
     }();
     return on;
 }
+
+static bool debug_mode() { return debug_mode_on(); }
 
 static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static bool aligned4(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
@@ -113,6 +115,25 @@ using namespace kda;
 
 extern "C" {
 
+kda_status_t kda_workspace_high_water(int64_t* bytes, int reset)
+{
+    if (bytes == nullptr) return KDA_ERR_INVALID_ARG;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KDA_ERR_CUDA;
+    cudaMemPool_t pool = workspace_pool(dev);
+    if (!pool) return KDA_ERR_CUDA;
+    uint64_t v = 0;
+    if (cudaMemPoolGetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &v) != cudaSuccess)
+        return KDA_ERR_CUDA;
+    *bytes = (int64_t)v;
+    if (reset) {
+        uint64_t zero = 0;
+        if (cudaMemPoolSetAttribute(pool, cudaMemPoolAttrUsedMemHigh, &zero) != cudaSuccess)
+            return KDA_ERR_CUDA;
+    }
+    return KDA_OK;
+}
+
 const char* kda_status_string(kda_status_t s)
 {
     switch (s) {
@@ -131,9 +152,6 @@ int kda_version(void) { return 100; }
 }  // extern "C"
 
 namespace kda {
-
-// Error word for debug-mode checks of the decode step (which has no workspace).
-static __device__ int g_decode_err;
 
 static kda_status_t recurrent_step_impl(const void* q, const void* k, const void* v,
                                         const float* log_alpha, const float* beta, float* state,
@@ -160,20 +178,13 @@ static kda_status_t recurrent_step_impl(const void* q, const void* k, const void
     a.scale = scale; a.io = io_dtype; a.slots = slots; a.err = nullptr;
     a.gate_scalar = gate_scalar;
     cudaError_t e = cudaSuccess;
-    if (debug_mode() && slots) {
-        void* ep = nullptr;
-        if ((e = cudaGetSymbolAddress(&ep, g_decode_err))) return from_cuda(e);
-        a.err = static_cast<int*>(ep);
-        if ((e = cudaMemsetAsync(a.err, 0, sizeof(int), stream))) return from_cuda(e);
-    }
+    // only a slot out of range sets a bit here
+    if (slots && (e = library_error_word(&a.err))) return from_cuda(e);
     e = launch_decode(a, stream);
     if (e == cudaSuccess && debug_mode()) {
-        e = cudaStreamSynchronize(stream);
-        if (e == cudaSuccess && a.err) {
-            int flag = 0;
-            e = cudaMemcpy(&flag, a.err, sizeof(int), cudaMemcpyDeviceToHost);
-            if (e == cudaSuccess && flag) return KDA_ERR_INVALID_ARG;
-        }
+        int flag = 0;
+        if ((e = take_error_word(stream, &flag))) return from_cuda(e);
+        return status_from_error_bits(flag);
     }
     return from_cuda(e);
 }
@@ -403,7 +414,7 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     const bool use_fused = use_tc && !segmap && !gate_scalar && T_total > 0 && plan.len == 0 &&
                            impl != KDA_PREFILL_TENSORCORE_CHAIN;
 
-    // workspace: [1 KiB header (error word) | chunk offsets (+ length order,
+    // workspace: [1 KiB header (reserved) | chunk offsets (+ length order,
     // + segment offsets) | per head group: per-(chunk, head) blocks, segment
     // buffers | SIMT segmap extras]
     const int64_t blk_bytes =
@@ -439,9 +450,9 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     cudaError_t e = buf.alloc((size_t)ws_bytes, stream);
     if (e) return from_cuda(e);
     char* base = static_cast<char*>(buf.ptr);
-    int* err_flag = reinterpret_cast<int*>(base);
+    int* err_flag = nullptr;
+    if ((e = library_error_word(&err_flag))) return from_cuda(e);
     a.err = err_flag;
-    if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
         int32_t* order = ordered ? reinterpret_cast<int32_t*>(chunk_off + B + 1) : nullptr;
@@ -481,11 +492,8 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     if (e) return from_cuda(e);
     if (debug_mode()) {
         int flag = 0;
-        if ((e = cudaMemcpyAsync(&flag, err_flag, sizeof(int), cudaMemcpyDeviceToHost, stream)))
-            return from_cuda(e);
-        if ((e = cudaStreamSynchronize(stream))) return from_cuda(e);
-        if (flag & kErrTimeoutMask) return KDA_ERR_TIMEOUT;
-        if (flag & kErrSeqlens) return KDA_ERR_INVALID_ARG;
+        if ((e = take_error_word(stream, &flag))) return from_cuda(e);
+        return status_from_error_bits(flag);
     }
     return KDA_OK;
 }
@@ -614,7 +622,7 @@ static kda_status_t chunk_bwd_impl(const void* q, const void* k, const void* v,
     si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
     si.order = nullptr;
 
-    // workspace: [1 KiB header (error word) | chunk offsets | per-(chunk, head) backward blocks]
+    // workspace: [1 KiB header (reserved) | chunk offsets | per-(chunk, head) backward blocks]
     const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 1023) / 1024 * 1024 : 0;
     const int64_t per_head = bwd_ws_floats_per_chunk((int)dk_, (int)dv_) * (int64_t)sizeof(float) *
                              (si.chunks_upper > 0 ? si.chunks_upper : 1);
@@ -625,8 +633,8 @@ static kda_status_t chunk_bwd_impl(const void* q, const void* k, const void* v,
     cudaError_t e = buf.alloc((size_t)(1024 + off_bytes + Hg * per_head), stream);
     if (e) return from_cuda(e);
     char* base = static_cast<char*>(buf.ptr);
-    int* err_flag = reinterpret_cast<int*>(base);
-    if ((e = cudaMemsetAsync(err_flag, 0, 256, stream))) return from_cuda(e);
+    int* err_flag = nullptr;
+    if ((e = library_error_word(&err_flag))) return from_cuda(e);
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 1024);
         if ((e = launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, nullptr,
@@ -638,10 +646,8 @@ static kda_status_t chunk_bwd_impl(const void* q, const void* k, const void* v,
     if (e) return from_cuda(e);
     if (debug_mode()) {
         int flag = 0;
-        if ((e = cudaMemcpyAsync(&flag, err_flag, sizeof(int), cudaMemcpyDeviceToHost, stream)))
-            return from_cuda(e);
-        if ((e = cudaStreamSynchronize(stream))) return from_cuda(e);
-        if (flag & kErrSeqlens) return KDA_ERR_INVALID_ARG;
+        if ((e = take_error_word(stream, &flag))) return from_cuda(e);
+        return status_from_error_bits(flag);
     }
     return KDA_OK;
 }

@@ -291,6 +291,16 @@ cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st);
 constexpr int kErrSeqlens = 1 << 0;
 constexpr int kErrTimeoutMask = 0x7e;
 
+// kda_errors.cu: the library's per-GPU device error word (the current device's),
+// taking it (read and clear, ordered on `st`, waits for `st`), and the status its
+// bits map to in debug mode.
+cudaError_t library_error_word(int** out);
+cudaError_t take_error_word(cudaStream_t st, int* host_out);
+kda_status_t status_from_error_bits(int bits);
+// KDA_DEBUG=1 in the environment (read once): every call waits for its stream and
+// returns the status of the error bits it finds (kda_api.cu).
+bool debug_mode_on();
+
 // Self-test of the bounded mbarrier wait (kda_selftest.cu).
 cudaError_t launch_bounded_wait_selftest(int* err, uint32_t polls, cudaStream_t st);
 

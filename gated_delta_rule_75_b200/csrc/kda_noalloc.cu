@@ -22,6 +22,7 @@
 //    before any stream capture.
 #include <cuda_runtime.h>
 
+#include <cstring>
 #include <mutex>
 
 #include "kda.h"
@@ -86,6 +87,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     if (B * H * 4 > 0x7fffffffLL) return KDA_ERR_UNSUPPORTED;
 
     PrefillArgs a;
+    std::memset(&a, 0, sizeof(a));
     a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.h0 = h0;
     a.out = out; a.hT = hT; a.H = H; a.dk = (int)dk; a.dv = (int)dv; a.scale = scale;
     a.io = io_dtype;
@@ -103,7 +105,7 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     si.chunks_upper = cu_seqlens ? (T / kChunk + B) : B * si.nct;
     si.order = nullptr;
 
-    // scratch layout: [256 B error word | chunk offsets | per-(chunk, head) blocks];
+    // scratch layout: [256 B reserved | chunk offsets | per-(chunk, head) blocks];
     // at least one head's chunks must fit, heads then run in groups that fit
     const int64_t blk = simt_ws_floats_per_chunk((int)dk, (int)dv) * (int64_t)sizeof(float);
     const int64_t off_bytes = cu_seqlens ? ((B + 1) * 8 + 255) / 256 * 256 : 0;
@@ -117,11 +119,11 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     cudaError_t e = noalloc_scratch_ptr(&base_v);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     char* base = static_cast<char*>(base_v);
-    int* err_flag = reinterpret_cast<int*>(base);
+    // errors go to the library's device error word (kda_get_error); offsets and
+    // blocks are fully written by the kernels before they are read
+    int* err_flag = nullptr;
+    if (library_error_word(&err_flag) != cudaSuccess) return KDA_ERR_CUDA;
     a.err = err_flag;
-    // the error word must start at zero; offsets and blocks are fully written
-    // by the kernels before they are read
-    if (cudaMemsetAsync(err_flag, 0, 256, stream) != cudaSuccess) return KDA_ERR_CUDA;
     if (cu_seqlens) {
         int64_t* chunk_off = reinterpret_cast<int64_t*>(base + 256);
         if (launch_chunk_offsets(cu_seqlens, B, T_total, si.chunks_upper, chunk_off, nullptr,
@@ -131,5 +133,10 @@ extern "C" KDA_API kda_status_t kda_chunk_fwd_noalloc(
     }
     float* ws = reinterpret_cast<float*>(base + 256 + off_bytes);
     if (run_prefill_simt(a, ws, Hg, stream) != cudaSuccess) return KDA_ERR_CUDA;
+    if (debug_mode_on()) {
+        int flag = 0;
+        if (take_error_word(stream, &flag) != cudaSuccess) return KDA_ERR_CUDA;
+        return status_from_error_bits(flag);
+    }
     return KDA_OK;
 }

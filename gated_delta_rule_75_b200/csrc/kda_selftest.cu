@@ -39,9 +39,15 @@ extern "C" {
 
 kda_status_t kda_debug_bounded_wait(int32_t polls, int32_t* err_word, cudaStream_t stream)
 {
-    if (polls < 1 || polls > 20000 || err_word == nullptr ||
-        (reinterpret_cast<uintptr_t>(err_word) & 3) != 0)
+    if (polls < 1 || polls > 20000 || (reinterpret_cast<uintptr_t>(err_word) & 3) != 0)
         return KDA_ERR_INVALID_ARG;
+    if (err_word == nullptr) {                   // report into the library's error word
+        int* lib_word = nullptr;
+        if (kda::library_error_word(&lib_word) != cudaSuccess) return KDA_ERR_CUDA;
+        if (kda::launch_bounded_wait_selftest(lib_word, (uint32_t)polls, stream) != cudaSuccess)
+            return KDA_ERR_CUDA;
+        return cudaStreamSynchronize(stream) == cudaSuccess ? KDA_OK : KDA_ERR_CUDA;
+    }
     if (cudaMemsetAsync(err_word, 0, sizeof(int32_t), stream) != cudaSuccess) return KDA_ERR_CUDA;
     if (kda::launch_bounded_wait_selftest(err_word, (uint32_t)polls, stream) != cudaSuccess)
         return KDA_ERR_CUDA;

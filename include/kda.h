@@ -20,10 +20,15 @@
  *    caller owns all of them.
  *  - Calls are asynchronous on `stream` (0 = legacy default stream).  Argument
  *    errors are detected on the host and returned before anything is launched;
- *    a failed launch returns KDA_ERR_CUDA.  No entry point synchronises the
- *    device unless KDA_DEBUG=1 is set in the environment, in which case the
- *    call synchronises `stream` at the end and also reports device-side input
- *    errors (malformed cu_seqlens) as KDA_ERR_INVALID_ARG.
+ *    a failed launch returns KDA_ERR_CUDA.  What only the device can see (a
+ *    malformed cu_seqlens array, a state slot out of range, a bounded wait
+ *    that gave up) is ORed into the library's device error word, one per GPU
+ *    and shared by all calls on it, and stays there until kda_get_error takes
+ *    it; see kda_get_error for the bits.  No entry point synchronises the
+ *    device unless KDA_DEBUG=1 is set in the environment, in which case every
+ *    call takes the error word itself after its own work (so it synchronises
+ *    `stream`) and returns KDA_ERR_TIMEOUT or KDA_ERR_INVALID_ARG for the bits
+ *    it finds.
  *  - q and k are expected to be L2-normalised per (token, head) by the caller
  *    (the delta rule is only stable for normalised keys, as the same page notes
  *    in its warning on key normalisation); the kernels do not renormalise.
@@ -61,7 +66,7 @@ typedef enum {
     KDA_ERR_UNSUPPORTED = 2,   /* head size or dtype not implemented */
     KDA_ERR_CUDA = 3,          /* a CUDA runtime call or launch failed */
     KDA_ERR_NO_MEMORY = 4,     /* workspace could not be allocated */
-    KDA_ERR_TIMEOUT = 5        /* reserved: a bounded device-side wait gave up */
+    KDA_ERR_TIMEOUT = 5        /* a bounded device-side wait gave up (debug) */
 } kda_status_t;
 
 typedef enum {
@@ -118,7 +123,8 @@ typedef enum {
  *              cu_seqlens[B] = T, and N = B.  Empty sequences are allowed
  *              (their hT equals h0).  Offsets are clamped into [0, T] on the
  *              device, so a malformed array never causes an out-of-bounds
- *              access (its results are then unspecified; KDA_DEBUG=1 reports it).
+ *              access (its results are then unspecified; bit 0 of the error
+ *              word reports it).
  *              With NULL, every one of the N = B sequences has length T.
  * Memory: the call allocates stream-ordered workspace from a library-owned
  * CUDA memory pool (bounded, reused across calls); KDA_ERR_NO_MEMORY if that
@@ -254,8 +260,8 @@ KDA_API kda_status_t kda_gdn_recurrent_step(const void* q, const void* k, const 
  *  slots       DEVICE int32 [N]: sequence n uses pool slot slots[n].  A negative
  *              slot means "no cached state": zero initial state, final state
  *              not stored (decode: output row set to 0, nothing else touched).
- *              Slots >= P are not accessed (reported as KDA_ERR_INVALID_ARG in
- *              KDA_DEBUG mode).  Two sequences of one call must not share a
+ *              Slots >= P are not accessed (bit 0 of the error word reports
+ *              them).  Two sequences of one call must not share a
  *              slot (their updates would race).
  *
  * kda_chunk_fwd_slots -- kda_chunk_fwd_ex with h0 = hT = state_pool[slots[n]];
@@ -401,13 +407,46 @@ KDA_API kda_status_t kda_debug_prep_image(const void* q, const void* k, const fl
  * kernels use on their copies, MMAs and warp hand-offs: `polls` suspended polls
  * (each at most ~0.1 ms; bit 1 of `err_word` when it gives up), then a spinning
  * poll bounded at `polls` x 200000 clock cycles (bit 2).  `err_word` is device
- * memory, caller-owned, 4-byte aligned, zeroed first; the CTA returns with
- * nothing in flight.  Synchronises `stream`.  Returns KDA_ERR_TIMEOUT when the wait gave
- * up (the expected outcome), KDA_OK otherwise, KDA_ERR_INVALID_ARG for polls
- * outside [1, 20000] or a bad pointer.  Lets the tests check that a wait that
+ * memory, caller-owned, 4-byte aligned, zeroed first; or NULL, and then the
+ * bits go to the library's error word (taken with kda_get_error) and the call
+ * returns KDA_OK.  The CTA returns with nothing in flight.  Synchronises
+ * `stream`.  Returns KDA_ERR_TIMEOUT when the wait gave up on `err_word` (the
+ * expected outcome), KDA_OK otherwise, KDA_ERR_INVALID_ARG for polls outside
+ * [1, 20000] or a misaligned pointer.  Lets the tests check that a wait that
  * runs out is reported and leaves the context usable.
  */
 KDA_API kda_status_t kda_debug_bounded_wait(int32_t polls, int32_t* err_word, cudaStream_t stream);
+
+/*
+ * kda_get_error -- takes the current device's error word: reads it and clears
+ * it in one atomic exchange queued on `stream`, then waits for `stream` and
+ * stores the bits in *word (host memory).  The word collects the bits of every
+ * call made on this device since the last take, from any stream; bits of work
+ * still running on another stream may land after the exchange (and are then
+ * returned by the next take).  No kernel reads the word, so bits left in it
+ * never change what a later call computes.
+ *   bit 0      a malformed cu_seqlens array, or a state slot >= P
+ *   bits 1-6   a bounded device-side wait gave up (1: input copies, 2-3: the
+ *              operand MMAs, 4: state copies, 5: state-walk MMAs, 6: hand-offs
+ *              between warps); the kernel stopped that work without faulting
+ *              and its outputs are unspecified
+ * Returns KDA_ERR_INVALID_ARG for word == NULL, KDA_ERR_CUDA if a CUDA call
+ * failed, KDA_OK otherwise.
+ */
+KDA_API kda_status_t kda_get_error(cudaStream_t stream, int32_t* word);
+
+/*
+ * kda_workspace_high_water -- the most bytes of workspace that calls on the
+ * current device had allocated at once from the library's pool since the last
+ * reset (the pool's used-memory high-water mark; allocations are counted as
+ * the pool rounds them), stored in *bytes; reset != 0 then restarts the mark
+ * at the bytes in use now.  The tensor-core prefill needs a fixed 1 KiB (plus
+ * at most 20 bytes per sequence with cu_seqlens) whatever T is; the two-kernel and SIMT
+ * forms grow with the number of chunks up to the workspace budget, beyond
+ * which heads run in groups; the decode step allocates nothing.
+ * KDA_ERR_INVALID_ARG for bytes == NULL, KDA_ERR_CUDA if a CUDA call failed.
+ */
+KDA_API kda_status_t kda_workspace_high_water(int64_t* bytes, int reset);
 
 /* Static, NUL-terminated description of a status code. */
 KDA_API const char* kda_status_string(kda_status_t status);

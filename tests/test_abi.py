@@ -106,5 +106,13 @@ def test_python_binding_checks_shapes_on_host():
 
 def test_bounded_wait_selftest_argument_errors(lib):
     import gated_delta_rule_75_b200 as kda
-    for polls, word in ((0, FAKE), (20001, FAKE), (10, None), (10, FAKE + 2)):
+    # (a NULL word is valid: the bits then go to the library's error word)
+    for polls, word in ((0, FAKE), (20001, FAKE), (0, None), (10, FAKE + 2)):
         assert lib.kda_debug_bounded_wait(polls, word, None) == kda.KDA_ERR_INVALID_ARG
+
+
+def test_error_word_and_high_water_argument_errors(lib):
+    import gated_delta_rule_75_b200 as kda
+    # NULL destinations are refused before any CUDA call
+    assert lib.kda_get_error(None, None) == kda.KDA_ERR_INVALID_ARG
+    assert lib.kda_workspace_high_water(None, 0) == kda.KDA_ERR_INVALID_ARG
