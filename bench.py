@@ -269,15 +269,8 @@ def run_prefill(args, ws, rank, kda, peaks):
     algo_flop_step = FLOP_PER_HEAD_TOKEN * head_tokens_per_step
     path_gbs = algo_bytes_step / (ms_max / args.steps / 1e3) / 1e9
     path_tflops = algo_flop_step / (ms_max / args.steps / 1e3) / 1e12
-    kbytes = kernel_algorithmic_bytes(kname, cfg) / max(1.0, launches_per_step)
-    roof = {"kernel": kname, "bound": "hbm", "achieved": kbytes / (k_ms_per_launch / 1e3) / 1e9,
-            "peak": peaks["hbm_gbs"], "unit": "GB/s",
-            "frac": None, "traffic": None, "launches_per_step": launches_per_step,
-            "ms_per_launch": k_ms_per_launch, "share_of_step": k_ms_per_step / (ms_max / args.steps),
-            "algorithmic_bytes_per_launch": kbytes, "peak_source": peaks["source"] + " (burst copy)"}
-    roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = measured_traffic(kname, cfg.name)
-    roof["traffic_source"] = "profiles/dram_traffic.md (ncu dram__bytes_read.sum + dram__bytes_write.sum)"
+    roof = prefill_roofline(kname, cfg, k_ms_per_launch, launches_per_step, peaks)
+    roof["share_of_step"] = k_ms_per_step / (ms_max / args.steps)
     res = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": ws, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_max / args.steps, "higher_is_better": True,
@@ -286,6 +279,7 @@ def run_prefill(args, ws, rank, kda, peaks):
         "prefill_impl": args.prefill_impl,
         "tc_frac": path_tflops / (peaks["bf16_tflops"]),
         "hbm_frac": path_gbs / peaks["hbm_gbs"],
+        "binding_frac": binding_frac(value / ws, cfg, peaks),
         "path": {"algorithmic_GBps": path_gbs, "algorithmic_TFLOPs": path_tflops,
                  "bytes_per_head_token": BYTES_PER_HEAD_TOKEN,
                  "flop_per_head_token": FLOP_PER_HEAD_TOKEN,
@@ -299,9 +293,56 @@ def run_prefill(args, ws, rank, kda, peaks):
     return res, inp, step, (out, hT)
 
 
-_TC_SOURCES = ("kda_chunk_tc.cu", "kda_umma.cuh", "kda_tma.cuh")
+def path_bytes_per_head_token(cfg):
+    """The path's minimal I/O per (token, head): q, k, v read and out written in the
+    I/O dtype, log_alpha fp32, beta fp32 (1540 B at d = 128 with bf16 I/O)."""
+    io = 2 if cfg.io_dtype == "bf16" else 4
+    return (2 * cfg.dk + 2 * cfg.dv) * io + cfg.dk * 4 + 4
+
+
+def path_flop_per_head_token(cfg):
+    """Chunk-form flops per (token, head): 2C(3dk + 2dv) + 6 dk dv (180,224 at C = 64, d = 128)."""
+    return 2 * CHUNK * (3 * cfg.dk + 2 * cfg.dv) + 6 * cfg.dk * cfg.dv
+
+
+def prefill_roofline(kname, cfg, ms_per_launch, launches_per_step, peaks):
+    """HBM roofline of the dominant prefill kernel.  `achieved` counts only the
+    path's minimal bytes: 1540 B (at d = 128, bf16) x the head-tokens one launch
+    processes, over that launch's event time, so bytes a kernel moves beyond the
+    path minimum (an intermediate image, re-reads) earn nothing; `kernel_io_frac`
+    is the kernel's own algorithmic I/O over the same time."""
+    ht_launch = cfg.tokens * cfg.H / max(1.0, launches_per_step)
+    algo = path_bytes_per_head_token(cfg) * ht_launch
+    kbytes = kernel_algorithmic_bytes(kname, cfg) / max(1.0, launches_per_step)
+    sec = ms_per_launch / 1e3
+    roof = {"kernel": kname, "bound": "hbm", "achieved": algo / sec / 1e9,
+            "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": algo / sec / 1e9 / peaks["hbm_gbs"],
+            "traffic": measured_traffic(kname, cfg.name),
+            "algorithmic_bytes_per_launch": algo,
+            "bytes_per_head_token": path_bytes_per_head_token(cfg),
+            "head_tokens_per_launch": ht_launch, "launches_per_step": launches_per_step,
+            "ms_per_launch": ms_per_launch,
+            "kernel_io_bytes_per_launch": kbytes,
+            "kernel_io_frac": kbytes / sec / 1e9 / peaks["hbm_gbs"],
+            "peak_source": peaks["source"] + " (burst copy)",
+            "traffic_source": "profiles/dram_traffic.json (ncu dram__bytes_read.sum + "
+                              "dram__bytes_write.sum per launch)"}
+    return roof
+
+
+def binding_frac(tokens_per_s, cfg, peaks):
+    """tokens/s over the lower of the tensor-bound and the HBM-bound tokens/s at the
+    path's minimal I/O (HBM binds: 117 flop/B against a ridge near 250)."""
+    tc_bound = peaks["bf16_tflops"] * 1e12 / (cfg.H * path_flop_per_head_token(cfg))
+    hbm_bound = peaks["hbm_gbs"] * 1e9 / (cfg.H * path_bytes_per_head_token(cfg))
+    return tokens_per_s / min(tc_bound, hbm_bound)
+
+
+_TC_SOURCES = ("kda_chunk_tc.cu", "kda_tc_util.cuh", "kda_umma.cuh", "kda_tma.cuh")
+_FUSED_SOURCES = ("kda_fused_tc.cu", "kda_tc_util.cuh", "kda_umma.cuh", "kda_tma.cuh")
 _SIMT_SOURCES = ("kda_chunk_simt.cu", "kda_chunk_simt.cuh")
-KERNEL_SOURCE = {"chunk_prep_tc": _TC_SOURCES, "chunk_state_tc": _TC_SOURCES,
+KERNEL_SOURCE = {"chunk_fused_tc": _FUSED_SOURCES,
+                 "chunk_prep_tc": _TC_SOURCES, "chunk_state_tc": _TC_SOURCES,
                  "chunk_prep_gdn_tc": _TC_SOURCES,
                  "chunk_prep_simt": _SIMT_SOURCES, "chunk_state_simt": _SIMT_SOURCES,
                  "decode_step": ("kda_decode.cu",)}
@@ -319,22 +360,21 @@ def kernel_source_sha(kname):
     return h.hexdigest()[:16]
 
 
-def measured_traffic(kname, workload):
+TRAFFIC_PATH = os.path.join(ROOT, "profiles", "dram_traffic.json")
+
+
+def measured_traffic(kname, workload, path=TRAFFIC_PATH):
     """DRAM bytes (read + write) per launch of `kname` on `workload` from the
-    committed ncu table profiles/dram_traffic.md, or None when the table has no
-    row for this kernel source (the kernel changed since the capture)."""
-    path = os.path.join(ROOT, "profiles", "dram_traffic.md")
+    committed ncu capture table, or None when no entry matches the kernel's current
+    source hash (the kernel changed since the capture).  An entry captured on a
+    smaller case of the same kernel carries `scale` = the workload's units per
+    launch over the capture's, and its bytes are scaled by it."""
     if not os.path.exists(path):
         return None
     sha = kernel_source_sha(kname)
-    for line in open(path):
-        cells = [c.strip().strip("`") for c in line.strip().strip("|").split("|")]
-        if len(cells) >= 7 and cells[0] == kname and cells[1] == workload and cells[2] == sha:
-            try:
-                launches = float(cells[3])
-                return (float(cells[4]) + float(cells[5])) / launches
-            except ValueError:
-                return None
+    for e in json.load(open(path))["entries"]:
+        if e["kernel"] == kname and e["workload"] == workload and e["source_sha256"] == sha:
+            return (e["dram_read_bytes"] + e["dram_write_bytes"]) / e["launches"] * e.get("scale", 1.0)
     return None
 
 
@@ -358,6 +398,9 @@ def kernel_algorithmic_bytes(kname, cfg):
         return ht * (2 * dk * io + dk * 4 + 4) + chunks * TC_WS_BYTES_PER_CHUNK
     if kname == "chunk_state_tc":        # reads the image and v; writes out and hT
         return chunks * TC_WS_BYTES_PER_CHUNK + ht * 2 * dv * io + cfg.N * cfg.H * dk * dv * 4
+    if kname == "chunk_fused_tc":        # reads q,k,v,g,beta (and h0); writes out and hT
+        states = cfg.N * cfg.H * dk * dv * 4
+        return qkvgb + ht * dv * io + states * (2 if cfg.h0_std > 0 else 1)
     if kname == "chunk_state_seg_tc":    # value walk (image, v) + map walk (image), per step;
         # the per-segment (M, B) matrices they write are not counted
         return 2 * chunks * TC_WS_BYTES_PER_CHUNK + ht * dv * io
@@ -570,6 +613,76 @@ def run_variants(args, ws, kda, peaks):
     return res
 
 
+L2_FLUSH_BYTES = 256 << 20          # twice the 126 MB L2
+
+
+def run_workload(kda, cfg, reps, warmup, peaks, ws, flush):
+    """One prefill workload through kda_chunk_fwd (AUTO): `warmup` untimed calls, then
+    `reps` calls each bracketed by its own CUDA events on the launching stream (with
+    `flush`, a 256 MB buffer is written before every rep, outside the events, so a
+    workload that fits in L2 is read from HBM); the median rep is reported, max over
+    ranks, with the dominant kernel's roofline and every kernel's time per call."""
+    inp = W.make_prefill(cfg, "cuda")
+    io = torch.bfloat16 if cfg.io_dtype == "bf16" else torch.float32
+    out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=io, device="cuda")
+    hT = torch.empty((cfg.N, cfg.H, cfg.dk, cfg.dv), dtype=torch.float32, device="cuda")
+    stream = torch.cuda.current_stream()
+    fbuf = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda") if flush else None
+
+    def step():
+        kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
+                      h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], out=out, hT=hT)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    kda.profiler_read(reset=True)
+    kda.profiler_enable(True)
+    barrier(ws)
+    times = []
+    for _ in range(reps):
+        if fbuf is not None:
+            fbuf.fill_(1.0)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        step()
+        e1.record(stream)
+        e1.synchronize()
+        times.append(e0.elapsed_time(e1))
+    barrier(ws)
+    kda.profiler_enable(False)
+    stats = kda.profiler_read(reset=True)
+    ms = max_over_ranks(statistics.median(times), ws)
+    kname, (_, ktimed, kms) = max(stats.items(), key=lambda kv: kv[1][2])
+    launches_per_step = ktimed / reps
+    roof = prefill_roofline(kname, cfg, kms / max(1, ktimed), launches_per_step, peaks)
+    roof["share_of_step"] = kms / reps / ms
+    res = {"workload": cfg.name, "tokens_per_s": cfg.tokens * ws / (ms / 1e3), "ms": ms,
+           "reps": reps, "statistic": "median", "io": cfg.io_dtype, "dk": cfg.dk, "H": cfg.H,
+           "l2": ("256 MB buffer written before every rep (the inputs fit in L2)" if flush
+                  else "inputs larger than L2"),
+           "binding_frac": binding_frac(cfg.tokens / (ms / 1e3), cfg, peaks),
+           "roofline": roof,
+           "kernels": {k: {"launches_per_call": v[0] / reps, "ms_per_call": v[2] / reps}
+                       for k, v in stats.items() if v[0]},
+           "gpu_launches_per_call": sum(v[0] for v in stats.values()) / reps}
+    del inp, out, hT, fbuf
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_workloads(args, ws, kda, peaks):
+    """The other prefill configurations, each through the default entry point: the
+    tiny fp32 case (B=1, H=2, T=256, d=64), one head group (B=1, H=16, T=4096), and
+    the long-context packed batch (16 sequences, 2^20 tokens, H=32)."""
+    res = {}
+    for key, cfg, reps, flush in (("tiny", W.TINY, 10, True), ("single", W.SINGLE, 10, True),
+                                  ("varlen", W.varlen_config(), 5, False)):
+        res[key] = run_workload(kda, cfg, reps, args.warmup, peaks, ws, flush)
+    return res
+
+
 def run_e2e(args, ws, kda, inp, bufs, steps):
     """Same metric through the public API with host (pinned) buffers: every
     step copies its inputs host->device and its output device->host inside the
@@ -650,6 +763,8 @@ def main():
     ap.add_argument("--bwd-steps", type=int, default=3,
                     help="timed steps of the backward leg (at most --steps)")
     ap.add_argument("--no-backward", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the tiny, single-head-group and varlen prefill workloads")
     ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
                     help="restrict the run (profiling of one kernel family)")
     ap.add_argument("--decode-steps", type=int, default=W.DECODE.steps)
@@ -696,6 +811,9 @@ def main():
         if not args.no_backward and args.only == "all":
             torch.cuda.empty_cache()
             res["backward"] = run_backward(args, ws, kda, peaks)
+        if not args.no_workloads and args.only == "all":
+            torch.cuda.empty_cache()
+            res["workloads"] = run_workloads(args, ws, kda, peaks)
         if rank == 0 and not args.no_cpu and args.only == "all":
             cfg = W.BATCHED
             heads, batch = cfg.H, 2
