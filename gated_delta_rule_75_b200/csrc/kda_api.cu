@@ -289,16 +289,17 @@ int64_t device_sm_count()
 // the SMs the walk is latency-bound on its longest chain; cutting the chains
 // into segments costs about three walks' worth of work (value, map, final) but
 // runs them side by side.  The plan aims at about one segment-CTA per SM.
-static SegPlan plan_segments(const SeqInfo& si, int64_t H, kda_prefill_impl_t impl)
+// Segment plan of the two-kernel tensor-core form: forced by SEGMENTED; under AUTO and
+// TENSORCORE (`guarded`: the two-kernel form with the fused kernel as its fallback)
+// only when there are few chains (at most a quarter of the SMs) and, for fixed-length
+// batches, at least four segments per chain.
+static SegPlan plan_segments(const SeqInfo& si, int64_t H, kda_prefill_impl_t impl, bool guarded)
 {
     SegPlan p;
     std::memset(&p, 0, sizeof(p));
-    if (impl == KDA_PREFILL_TENSORCORE_CHAIN || impl == KDA_PREFILL_TENSORCORE_FUSED ||
-        si.chunks_upper <= 0)
-        return p;
-    // AUTO and TENSORCORE run the fused kernel; only an explicit request segments
-    if (impl != KDA_PREFILL_TENSORCORE_SEGMENTED) return p;
-    const bool force = true;
+    if (si.chunks_upper <= 0) return p;
+    if (impl != KDA_PREFILL_TENSORCORE_SEGMENTED && !guarded) return p;
+    const bool force = impl == KDA_PREFILL_TENSORCORE_SEGMENTED;
     const int64_t sms = device_sm_count();
     const int64_t chains = si.N * H;
     if (!force && chains * 4 > sms) return p;
@@ -404,17 +405,25 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         plan.offs = offs;
         plan.hstride = H;
         plan.abs_head = true;
-    } else if (use_tc) {
-        plan = plan_segments(si, H, impl);
+    }
+    // AUTO / TENSORCORE (KDA form, outputs wanted, tokens present): the fused kernel,
+    // which builds every chunk's operands on chip (no per-chunk workspace) and is exact
+    // at any decay rate.  With few chains (at most half the SMs) the two-kernel form,
+    // whose prep spreads over every SM, goes first: its prep flags any 16-token block
+    // outside its decay range, its walks then do nothing, and the fused kernel launched
+    // after them computes the call only in that case.
+    const bool auto_tc = use_tc && !segmap && !gate_scalar && T_total > 0 &&
+                         (impl == KDA_PREFILL_AUTO || impl == KDA_PREFILL_TENSORCORE);
+    const bool guarded = auto_tc && si.N * H * 2 <= device_sm_count();
+    if (use_tc && !segmap) {
+        plan = plan_segments(si, H, impl, guarded);
         if (plan.upper > 0x7fffffffLL / H) std::memset(&plan, 0, sizeof(plan));
     }
     const bool seg_table = use_tc && !segmap && plan.len > 0 && cu_seqlens != nullptr;
-    // the fused kernel (KDA form, outputs wanted, tokens present, no segmentation): it
-    // builds every chunk's operands on chip, so it needs no per-chunk workspace
-    const bool use_fused = use_tc && !segmap && !gate_scalar && T_total > 0 && plan.len == 0 &&
-                           impl != KDA_PREFILL_TENSORCORE_CHAIN;
+    const bool use_fused = auto_tc ? !guarded : (impl == KDA_PREFILL_TENSORCORE_FUSED && !gate_scalar &&
+                                                 !segmap && T_total > 0);
 
-    // workspace: [1 KiB header (reserved) | chunk offsets (+ length order,
+    // workspace: [1 KiB header (words 64, 65: see below) | chunk offsets (+ length order,
     // + segment offsets) | per head group: per-(chunk, head) blocks, segment
     // buffers | SIMT segmap extras]
     const int64_t blk_bytes =
@@ -465,8 +474,16 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
         plan.seg_off = seg_off;
     }
     unsigned char* ws = reinterpret_cast<unsigned char*>(base + 1024 + off_bytes);
+    // header words: 64, the fused kernel's chain tickets (packed sequences); 65, the
+    // two-kernel form's decay-range flag
+    int* ticket = cu_seqlens ? reinterpret_cast<int*>(base) + 64 : nullptr;
     if (use_fused) {
-        e = run_prefill_fused(a, err_flag, stream);
+        e = run_prefill_fused(a, err_flag, ticket, nullptr, stream);
+    } else if (guarded) {
+        a.range_flag = reinterpret_cast<int*>(base) + 65;
+        e = cudaMemsetAsync(a.range_flag, 0, sizeof(int), stream);
+        if (!e) e = run_prefill_tc(a, ws, Hg, err_flag, stream);
+        if (!e) e = run_prefill_fused(a, err_flag, ticket, a.range_flag, stream);
     } else if (use_tc) {
         e = run_prefill_tc(a, ws, Hg, err_flag, stream);
     } else if (!segmap) {

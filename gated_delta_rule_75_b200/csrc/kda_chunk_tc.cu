@@ -56,6 +56,10 @@ namespace tc {
 constexpr int C = 64;
 constexpr int D = 128;     // dk = dv = 128
 constexpr float kLog2e = 1.4426950408889634f;
+// Decay range of the 16-token references (log2 units): a factor e^{G_f - G_j} with j in
+// the 16-token block that starts at f stays below 2^116 when no channel decays by more
+// than e^-80 over the block's 15 steps (the prep reports a block past this).
+constexpr float kRangeLog2 = 80.f * kLog2e;
 
 // Operand image of one (chunk, head), byte offsets (all 1024-aligned).
 constexpr uint32_t IMG_W = 0;          // -W^T        MN-major B: 128 channel rows x 64 tokens
@@ -241,7 +245,7 @@ __device__ __forceinline__ bool prep_tail(unsigned char* sm, unsigned char* img,
 __global__ void __launch_bounds__(PT, 2)
 chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restrict__ beta,
                      SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, int64_t hg,
-                     unsigned char* __restrict__ ws, int* __restrict__ err)
+                     unsigned char* __restrict__ ws, int* __restrict__ err, int* __restrict__ range_flag)
 {
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -346,6 +350,7 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                 v[x] = run;
             }
             Gf[pq] = v[0];
+            if (range_flag && v[0] - v[15] > kRangeLog2) atomicOr(range_flag, 1);
 #pragma unroll
             for (int x = 0; x < 16; ++x)
                 *reinterpret_cast<float*>(slab + (16 * pq + x) * 128 + ((q0 ^ (x & 7)) << 4)) = v[x];
@@ -408,6 +413,8 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                         v[x] = run;
                     }
                 }
+                if (range_flag && (v[0] - v[15] > kRangeLog2 || v[16] - v[31] > kRangeLog2))
+                    atomicOr(range_flag, 1);
                 if (part == 0) {
 #pragma unroll
                     for (int x = 0; x < 32; ++x)
@@ -842,6 +849,7 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 {
     constexpr bool kOut = kMode == WALK_SEQ || kMode == WALK_FINAL;   // outputs written
     constexpr bool kV = kMode != WALK_MAP;                            // v tiles used
+    if (sp.skip && *sp.skip) return;               // the fused kernel takes this call over
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -1240,12 +1248,13 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
             if (items > INT32_MAX) return cudaErrorInvalidValue;   // items are 32-bit in the kernel
             const int64_t slots = 2 * device_sm_count();
             tc::chunk_prep_tc_kernel<<<(unsigned)(items < slots ? items : slots), tc::PT, tc::P_SMEM, s>>>(
-                maps, a.beta, a.si, a.H, hb, Hg, hg, w, err);
+                maps, a.beta, a.si, a.H, hb, Hg, hg, w, err, a.range_flag);
         }
         return cudaGetLastError();
     };
     SegPlan none;
     memset(&none, 0, sizeof(none));
+    none.skip = a.range_flag;
     auto launch_state = [&](int64_t hb, int64_t hg, unsigned char* w, cudaStream_t s) -> cudaError_t {
         dim3 gs((unsigned)(a.si.N * hg));
         LaunchScope scope(s, K_STATE_TC);
@@ -1278,6 +1287,7 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
 
     // segment buffers sit after the operand images of one head group
     SegPlan sp = a.seg;
+    sp.skip = a.tc_what == 0 ? a.range_flag : nullptr;
     if (a.tc_what == 0 && sp.len > 0) {
         const int64_t mat = (int64_t)tc::D * tc::D;
         float* segbuf = reinterpret_cast<float*>(

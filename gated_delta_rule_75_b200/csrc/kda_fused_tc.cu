@@ -154,51 +154,123 @@ __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, bool leade
     return bar_and_named(barid, count, ok);
 }
 
-// The chunks of one CTA: chains blockIdx.x, + gridDim.x, ... of the (sequence rank,
-// head) list, heads innermost; sequences ranked longest first when an order is known.
-// Chains without tokens are skipped (their final states are written separately).
-// Token rows and chain indices fit 32 bits (the launch checks both).
+// Where a CTA's chains come from.  Static: blockIdx.x, + gridDim.x, ... of the
+// (sequence rank, head) list.  Dynamic (packed sequences of mixed lengths): chain
+// blockIdx.x first, then whatever chain a ticket from the global counter names
+// (gridDim.x + ticket), so the CTAs that finish early take the remaining chains and,
+// with the sequences ranked longest first, the long chains start first.  In dynamic
+// mode one thread (the prep issuer, the role furthest ahead) takes the tickets and
+// publishes each chain it starts, in order, in a ring in shared memory; every other
+// role reads the ring at the same position.
+constexpr int kRing = 16;
+struct Sched {
+    int* ticket;                                // global counter (zeroed) or null: static
+    volatile int* ring_val;                     // [kRing] chain index, -1: no more chains
+    volatile int* ring_seq;                     // [kRing] position the entry was written for
+};
+
+// The chunks of one CTA, chain by chain, heads innermost; sequences ranked longest
+// first when an order is known.  Chains without tokens are skipped (their final
+// states are written separately).  Token rows and chain indices fit 32 bits (the
+// launch checks both).
 struct Items {
     int32_t r, h, n, bos, eos, nch, c;
     int64_t sidx;                               // state index, -1: none
+    uint32_t q;                                 // chains started before this one
     bool ok;
 
-    __device__ __forceinline__ void load(const SeqInfo& si, int32_t H, const int32_t* slots, int64_t P)
+    // Chain r's fields; false when r is past the end or the chain has no tokens.
+    __device__ __forceinline__ bool set(int32_t r_, const SeqInfo& si, int32_t H, const int32_t* slots,
+                                        int64_t P)
     {
-        ok = false;
+        r = r_;
+        if (r < 0 || r >= (int32_t)si.N * H) return false;
+        const int32_t sr = r / H;
+        h = r - sr * H;
+        n = (int32_t)si.seq_of(sr);
+        int64_t b, e;
+        seq_range(si.cu, n, si.T_seq, si.T_total, b, e);
+        bos = (int32_t)b;
+        eos = (int32_t)e;
+        nch = (eos - bos + C - 1) / C;
+        c = 0;
+        sidx = (int64_t)n * H + h;
+        if (slots) {
+            const int64_t sl = slots[n];
+            sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
+        }
+        return nch > 0;
+    }
+    // The first chain with tokens from candidate `r` on, in the source's order, or -1.
+    __device__ __forceinline__ int32_t resolve(int32_t r_, const Sched& sc, const SeqInfo& si, int32_t H,
+                                               const int32_t* slots, int64_t P)
+    {
         const int32_t rend = (int32_t)si.N * H;
-        while (r < rend) {
-            const int32_t sr = r / H;
-            h = r - sr * H;
-            n = (int32_t)si.seq_of(sr);
-            int64_t b, e;
-            seq_range(si.cu, n, si.T_seq, si.T_total, b, e);
-            bos = (int32_t)b;
-            eos = (int32_t)e;
-            nch = (eos - bos + C - 1) / C;
-            if (nch > 0) {
-                c = 0;
-                sidx = (int64_t)n * H + h;
-                if (slots) {
-                    const int64_t sl = slots[n];
-                    sidx = (sl >= 0 && sl < P) ? sl * H + h : -1;
-                }
-                ok = true;
-                return;
+        while (r_ < rend) {
+            if (set(r_, si, H, slots, P)) return r_;
+            r_ = sc.ticket ? (int32_t)gridDim.x + atomicAdd(sc.ticket, 1) : r_ + (int32_t)gridDim.x;
+        }
+        return -1;
+    }
+    // Publisher: ring entry q (dynamic mode).
+    __device__ __forceinline__ void publish(const Sched& sc, uint32_t qq, int32_t val)
+    {
+        sc.ring_val[qq % kRing] = val;
+        __threadfence_block();
+        sc.ring_seq[qq % kRing] = (int)qq;
+    }
+    // Reader: ring entry q, polled with the same bounds as the mbarrier waits.
+    __device__ __forceinline__ int32_t read(const Sched& sc, uint32_t qq, int* err, volatile int* abort)
+    {
+        const long long t0 = clock64();
+        for (uint32_t i = 1;; ++i) {
+            if (sc.ring_seq[qq % kRing] == (int)qq) {
+                __threadfence_block();
+                return sc.ring_val[qq % kRing];
             }
-            r += (int32_t)gridDim.x;
+            if ((i & 31u) == 0) {
+                if (*abort) return -1;
+                if (clock64() - t0 > kWaitCycles) {
+                    if (err) atomicOr(err, 1 << 6);
+                    *abort = 1;
+                    return -1;
+                }
+            }
         }
     }
-    __device__ __forceinline__ void init(const SeqInfo& si, int32_t H, const int32_t* slots, int64_t P)
+    // Chain number q from the source: the publisher resolves and publishes it, the
+    // other roles read it (dynamic) or resolve it themselves (static).
+    __device__ __forceinline__ void take(int32_t cand, bool publisher, const Sched& sc, const SeqInfo& si,
+                                         int32_t H, const int32_t* slots, int64_t P, int* err,
+                                         volatile int* abort)
     {
-        r = (int32_t)blockIdx.x;
-        load(si, H, slots, P);
+        int32_t got;
+        if (!sc.ticket || publisher) {
+            got = resolve(cand, sc, si, H, slots, P);
+            if (sc.ticket) publish(sc, q, got);
+        } else {
+            got = read(sc, q, err, abort);
+        }
+        ok = got >= 0 && set(got, si, H, slots, P);
     }
-    __device__ __forceinline__ void next(const SeqInfo& si, int32_t H, const int32_t* slots, int64_t P)
+    __device__ __forceinline__ void init(bool publisher, const Sched& sc, const SeqInfo& si, int32_t H,
+                                         const int32_t* slots, int64_t P, int* err, volatile int* abort)
+    {
+        q = 0;
+        take((int32_t)blockIdx.x, publisher, sc, si, H, slots, P, err, abort);
+    }
+    __device__ __forceinline__ void next(bool publisher, const Sched& sc, const SeqInfo& si, int32_t H,
+                                         const int32_t* slots, int64_t P, int* err, volatile int* abort)
     {
         if (++c >= nch) {
-            r += (int32_t)gridDim.x;
-            load(si, H, slots, P);
+            ++q;
+            if (sc.ticket && !publisher) {
+                take(-1, false, sc, si, H, slots, P, err, abort);
+                return;
+            }
+            const int32_t cand = sc.ticket ? (int32_t)gridDim.x + atomicAdd(sc.ticket, 1)
+                                           : r + (int32_t)gridDim.x;
+            take(cand, publisher, sc, si, H, slots, P, err, abort);
         }
     }
     __device__ __forceinline__ int32_t t0() const { return bos + c * C; }
@@ -287,8 +359,10 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                       const float* __restrict__ log_alpha, const float* __restrict__ beta,
                       const float* __restrict__ h0, __nv_bfloat16* __restrict__ out,
                       float* __restrict__ hT, float scale, SeqInfo si, int64_t H,
-                      const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err)
+                      const int32_t* __restrict__ slots, int64_t P, int* __restrict__ err,
+                      int* __restrict__ ticket, const int* __restrict__ run_if)
 {
+    if (run_if && *run_if == 0) return;           // the two-kernel form computed this call
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -296,12 +370,14 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     __shared__ uint32_t tmem_base;
     __shared__ int s_npass;
     __shared__ int s_abort_raw;
+    __shared__ int s_ring_val[kRing], s_ring_seq[kRing];
     volatile int* abort = &s_abort_raw;
 
     const int tid = threadIdx.x, w = tid >> 5, l = tid & 31;
     const int32_t H32 = (int32_t)H;
-    Items it0;
-    it0.init(si, H32, slots, P);
+    const Sched sc{ticket, s_ring_val, s_ring_seq};
+    const bool publisher = tid == W_PI * 32;
+    if (tid < kRing) s_ring_seq[tid] = -1;
 
     if (tid == W_PI * 32) {
         mbar_init(&bars.g, 1); mbar_init(&bars.gc, 8);
@@ -330,6 +406,11 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
     __syncthreads();
     fence_after_sync();
     const uint32_t tmem = tmem_base;
+    // every role's first chain (the publisher's entry is written before anyone reads it)
+    Items it0;
+    if (publisher) it0.init(true, sc, si, H32, slots, P, err, abort);
+    __syncthreads();
+    if (!publisher) it0.init(false, sc, si, H32, slots, P, err, abort);
 
     if (w < 8) {
         // ------------------------------------------------------------------ prep
@@ -603,7 +684,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                     *reinterpret_cast<uint4*>(sm + F_W + sw128_offset(pc, 32 * ph + 8 * m)) = pack8(f + 8 * m);
             }
             warp_arrive(&bars.img);
-            it.next(si, H32, slots, P);
+            it.next(false, sc, si, H32, slots, P, err, abort);
         }
     } else if (w < W_PI) {
         // ------------------------------------------------------------------ walk
@@ -765,7 +846,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 bar_sync_named(NB_WALK, 128);
                 if (wlead) mbar_arrive(&bars.fr[s]);
             }
-            it.next(si, H32, slots, P);
+            it.next(false, sc, si, H32, slots, P, err, abort);
         }
         if (wlead) tma::bulk_wait_all();
     } else if (w == W_PI) {
@@ -788,7 +869,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             if (it.ok) { issue_g(it); ++g_issued; issue_kq(it); ++kq_issued; }
             for (uint32_t k = 0; it.ok; ++k) {
                 Items nx = it;
-                nx.next(si, H32, slots, P);
+                nx.next(true, sc, si, H32, slots, P, err, abort);
                 if (!fwait(&bars.kq, k & 1, err, 1, abort)) break;
                 ++kq_seen;
                 if (k > 0 && !fwait(&bars.img, (k - 1) & 1, err, 6, abort)) break;
@@ -871,7 +952,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             for (uint32_t k = 0; it.ok; ++k) {
                 const int s = (int)(k & 1);
                 Items nx = it;
-                nx.next(si, H32, slots, P);
+                nx.next(false, sc, si, H32, slots, P, err, abort);
                 if (!fwait(&bars.img, k & 1, err, 6, abort)) break;
                 if (!fwait(&bars.v, k & 1, err, 4, abort)) break;
                 ++v_seen;
@@ -930,7 +1011,8 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 
 }  // namespace fz
 
-cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st)
+cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, int* ticket, const int* run_if,
+                              cudaStream_t st)
 {
     static std::atomic<uint64_t> attrs_done{0};
     cudaError_t e = once_per_device(attrs_done, [] {
@@ -957,10 +1039,13 @@ cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st)
     if ((e = make_tensor_map_2d(&gmap, a.log_alpha, false, cols, rows, cols * 4, fz::D, 64, false))) return e;
     const int64_t sms = device_sm_count();
     const unsigned grid = (unsigned)(chains < sms ? chains : sms);
+    // packed sequences of mixed lengths: chains handed out by tickets (the counter is
+    // zeroed here, in stream order); equal-length chains: the static order balances
+    if (ticket && (e = cudaMemsetAsync(ticket, 0, sizeof(int), st))) return e;
     LaunchScope scope(st, K_FUSED_TC);
     fz::chunk_fused_tc_kernel<<<grid, fz::NT, fz::F_SMEM, st>>>(
         kmap, qmap, vmap, omap, gmap, a.log_alpha, a.beta, a.h0, (__nv_bfloat16*)a.out, a.hT, a.scale, a.si,
-        a.H, a.slots, a.P, err);
+        a.H, a.slots, a.P, err, ticket, run_if);
     return cudaGetLastError();
 }
 

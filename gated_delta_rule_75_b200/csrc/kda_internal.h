@@ -93,6 +93,10 @@ struct SegPlan {
     float* starts;
     int64_t hstride;
     bool abs_head;
+    // device word or nullptr: when it is nonzero at launch, the state walks do nothing
+    // (the prep found a chunk outside the two-kernel form's decay range and the fused
+    // kernel, launched after them, computes the whole call instead)
+    const int* skip;
 
 #ifdef __CUDACC__
     // Segment g -> (sequence n, index s within it, segments of n); false past the end.
@@ -145,6 +149,9 @@ struct PrefillArgs {
     // tensor-core path: segment-parallel state walk (len == 0: one chain per
     // (sequence, head)); the buffers are placed by run_prefill_tc
     SegPlan seg;
+    // two-kernel tensor-core path: device word the prep sets (bit 0) when a 16-token
+    // block of some channel decays by more than its exponent range allows, or nullptr
+    int* range_flag;
     // what the tensor-core path produces: outputs and final states (0), only each
     // sequence's affine map into seg.maps / seg.offs (1), or only the operand images of
     // the prep kernel, left in the workspace (2; the test hook kda_debug_prep_image)
@@ -281,8 +288,11 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
                            cudaStream_t st);
 
 // kda_fused_tc.cu (bf16, dk = dv = 128, T_total > 0): the whole prefill in one
-// kernel, no workspace beyond the error word.
-cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, cudaStream_t st);
+// kernel.  `ticket` (device int, or null): the counter that hands out chains to
+// CTAs as they free up (zeroed by the call); null keeps the static order.
+// `run_if` (device int, or null): the kernel does nothing unless it is nonzero at launch.
+cudaError_t run_prefill_fused(const PrefillArgs& a, int* err, int* ticket, const int* run_if,
+                              cudaStream_t st);
 
 // Device error word bits (workspace header): malformed cu_seqlens, and bounded
 // waits that gave up in the tensor-core kernels (bit 1: input copies of the prep;

@@ -34,8 +34,8 @@
  *    in its warning on key normalisation); the kernels do not renormalise.
  *  - `scale` multiplies q once, at the read (configurations use 1/sqrt(dk)).
  *  - log_alpha is the natural log of the per-channel decay, finite and <= 0.
- *    The default tensor-core prefill (the fused kernel) and the SIMT paths
- *    hold at any decay rate.  The two-kernel tensor-core forms, reached only
+ *    The default tensor-core prefill (AUTO / TENSORCORE) and the SIMT paths
+ *    hold at any decay rate.  The two-kernel tensor-core forms, when forced
  *    through KDA_PREFILL_TENSORCORE_CHAIN or _SEGMENTED, assume that within
  *    each 64-token chunk no key channel decays by more than e^-80 over 16
  *    consecutive tokens (their exponential factors are referenced to 16-token
@@ -85,8 +85,16 @@ typedef enum {
  * one CTA per SM walks chains and builds each chunk's operands on chip while
  * the previous chunk's state update runs, so only the inputs, the outputs and
  * the states cross device memory (no workspace per chunk), and it is exact at
- * any decay rate.  The last three values force one form; the two-kernel forms
- * (CHAIN, SEGMENTED) keep the decay-range limit stated above.
+ * any decay rate.  With packed sequences its CTAs take chains from a shared
+ * counter as they free up, longest sequences first.  When there are few chains
+ * (at most half the SMs), AUTO and TENSORCORE first run the two-kernel form
+ * (operand images in the workspace, prepared on every SM; segmented when there
+ * are at most a quarter of the SMs' chains); its prep checks every 16-token
+ * block against the two-kernel decay range, and if any block is past it the
+ * walks do nothing and the fused kernel, launched after them, computes the
+ * whole call -- so AUTO stays exact at any decay rate.  The last three values
+ * force one form; the forced two-kernel forms (CHAIN, SEGMENTED) keep the
+ * decay-range limit stated above.
  */
 typedef enum {
     KDA_PREFILL_AUTO = 0,      /* tensor cores for bf16 with dk = dv = 128, SIMT otherwise */
@@ -440,10 +448,11 @@ KDA_API kda_status_t kda_get_error(cudaStream_t stream, int32_t* word);
  * current device had allocated at once from the library's pool since the last
  * reset (the pool's used-memory high-water mark; allocations are counted as
  * the pool rounds them), stored in *bytes; reset != 0 then restarts the mark
- * at the bytes in use now.  The tensor-core prefill needs a fixed 1 KiB (plus
- * at most 20 bytes per sequence with cu_seqlens) whatever T is; the two-kernel and SIMT
- * forms grow with the number of chunks up to the workspace budget, beyond
- * which heads run in groups; the decode step allocates nothing.
+ * at the bytes in use now.  The fused tensor-core prefill (the default when the
+ * chains outnumber half the SMs) needs a fixed 1 KiB (plus at most 20 bytes per
+ * sequence with cu_seqlens) whatever T is; the two-kernel and SIMT forms grow
+ * with the number of chunks up to the workspace budget, beyond which heads run
+ * in groups; the decode step allocates nothing.
  * KDA_ERR_INVALID_ARG for bytes == NULL, KDA_ERR_CUDA if a CUDA call failed.
  */
 KDA_API kda_status_t kda_workspace_high_water(int64_t* bytes, int reset);

@@ -106,6 +106,21 @@ def test_more_chains_than_sms(kda, impl):
     check_full(kda, cfg, impl)
 
 
+@pytest.mark.parametrize("impl", ["auto", "tensorcore_fused"])
+def test_packed_chains_handed_out_by_tickets(kda, impl):
+    """Packed sequences: after its first chain each CTA takes the next one from a
+    global ticket counter, and the other roles of the CTA read it from the issuer's
+    ring.  400 sequences of 0 to 150 tokens (empty ones included, sorted longest first
+    on the device) at H = 2: 800 chains over one CTA per SM, with initial states."""
+    rng = np.random.default_rng(16)
+    lengths = [int(x) for x in rng.integers(0, 151, size=400)]
+    lengths[3] = 0
+    lengths[-1] = 0
+    cfg = W.small_prefill(H=2, dk=128, dv=128, io_dtype="bf16", seed=16, h0_std=0.02,
+                          lengths=lengths)
+    check_full(kda, cfg, impl)
+
+
 @pytest.mark.parametrize("shift", [-4.0, 3.0, 3.6, 8.0])
 def test_simt_decay_rates_fp32(kda, shift):
     """fp32 I/O at mean per-token decays from e^-0.02 to e^-8: the SIMT prep factors

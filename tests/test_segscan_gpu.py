@@ -100,23 +100,66 @@ def test_segmented_walk_on_pool_slots(kda):
 
 
 def test_automatic_choice(kda):
-    """AUTO runs the fused one-kernel prefill for few chains (1 sequence x 2
-    heads) and for many (8 x 32); the segmented walk runs only when asked for."""
+    """AUTO with few chains (1 sequence x 2 heads) runs the two-kernel form with the
+    segment-parallel walk, then launches the fused kernel, which does nothing when no
+    chunk left the two-kernel decay range; with half the SMs' worth of chains (2 x 32)
+    the one-chain-per-(sequence, head) walk; with many chains (8 x 32) only the fused
+    kernel; the segmented walk runs on request too."""
     kda.profiler_read(reset=True)
     cfg = W.small_prefill(B=1, T=2048, H=2, dk=128, dv=128, io_dtype="bf16", seed=11,
                           h0_std=0.02)
     _check(kda, cfg, "auto")
     st = kda.profiler_read(reset=True)
-    assert st["chunk_fused_tc"][0] == 1 and st["chunk_state_seg_tc"][0] == 0, st
+    assert st["chunk_prep_tc"][0] == 1 and st["chunk_state_seg_tc"][0] == 2, st
+    assert st["affine_prefix"][0] == 1 and st["chunk_fused_tc"][0] == 1, st
+    _check(kda, W.small_prefill(B=2, T=200, H=32, dk=128, dv=128, io_dtype="bf16", seed=14,
+                                h0_std=0.02), "auto")
+    st = kda.profiler_read(reset=True)
+    assert st["chunk_state_tc"][0] == 1 and st["chunk_state_seg_tc"][0] == 0, st
     cfg = W.small_prefill(B=8, T=100, H=32, dk=128, dv=128, io_dtype="bf16", seed=12)
     inp = W.make_prefill(cfg, "cuda")
     _run(kda, inp, "auto")
     st = kda.profiler_read(reset=True)
     assert st["chunk_fused_tc"][0] == 1 and st["chunk_state_tc"][0] == 0, st
+    assert st["chunk_prep_tc"][0] == 0, st
     _check(kda, W.small_prefill(B=1, T=2048, H=2, dk=128, dv=128, io_dtype="bf16", seed=11,
                                 h0_std=0.02), "tensorcore_segmented")
     st = kda.profiler_read(reset=True)
     assert st["chunk_state_seg_tc"][0] == 2 and st["affine_prefix"][0] == 1, st
+
+
+@pytest.mark.parametrize("shape", [(1, 2048, 2, None), (2, 200, 32, None),
+                                   (1, 0, 2, [900, 0, 130, 1000])])
+@pytest.mark.parametrize("shift", [8.0, 40.0])
+def test_automatic_choice_falls_back_past_the_decay_range(kda, shape, shift):
+    """Few chains under AUTO with fast decay (about e^-8 and e^-40 per token): the
+    two-kernel prep flags the 16-token blocks past its range, its walks do nothing and
+    the fused kernel computes the call: parity at the bf16 bar, segmented, one chain
+    per (sequence, head), and packed."""
+    B, T, H, lengths = shape
+    cfg = W.small_prefill(B=B, T=T, H=H, dk=128, dv=128, io_dtype="bf16", seed=15,
+                          gate_shift=shift, h0_std=0.02, lengths=lengths)
+    _check(kda, cfg, "auto")
+
+
+def test_automatic_choice_one_fast_sequence_moves_the_whole_call(kda):
+    """One packed sequence past the range among slow ones: the whole call goes to the
+    fused kernel, and the slow sequences' results are still right."""
+    slow = W.small_prefill(H=2, dk=128, dv=128, io_dtype="bf16", seed=16, h0_std=0.02,
+                           lengths=[700, 64])
+    fast = W.small_prefill(B=1, T=300, H=2, dk=128, dv=128, io_dtype="bf16", seed=17,
+                           gate_shift=8.0, h0_std=0.02)
+    a, b = W.make_prefill(slow, "cuda"), W.make_prefill(fast, "cuda")
+    inp = {k: (torch.cat([a[k], b[k]], dim=1) if k in ("q", "k", "v", "log_alpha", "beta") else a[k])
+           for k in a}
+    inp["h0"] = torch.cat([a["h0"], b["h0"]], dim=0)
+    inp["cu_seqlens"] = torch.tensor([0, 700, 764, 1064], dtype=torch.int32, device="cuda")
+    kda.profiler_read(reset=True)
+    out, hT = _run(kda, inp, "auto")
+    st = kda.profiler_read(reset=True)
+    assert st["chunk_prep_tc"][0] == 1 and st["chunk_fused_tc"][0] == 1, st
+    ro, rh = oracle_prefill(inp)
+    assert rel(out, ro) <= TOL["bf16"] and rel(hT, rh) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("io,d", [("bf16", 128), ("f32", 64), ("bf16", 64), ("f32", 128)])
