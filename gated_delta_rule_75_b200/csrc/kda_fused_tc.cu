@@ -95,20 +95,19 @@ static_assert(F_KD + 64 * AP * 4 <= F_KG, "T scratch overlaps (K e^G)^T");
 static_assert(F_W + 64 * AP * 4 <= F_V, "A scratch overlaps v");
 
 // Tensor memory columns (512 allocated)
-constexpr uint32_t TM_KT = 0;               // k^T fp32 (prep), then -W^T
+constexpr uint32_t TM_KT = 0;               // k^T fp32 (prep)
 constexpr uint32_t TM_QT = 64;              // q^T fp32
-constexpr uint32_t TM_WT = 0;
 constexpr uint32_t TM_S = 128;              // S^T fp32 (state)
 constexpr uint32_t TM_U = 256;              // U^T fp32; its first 32 columns then hold U^T bf16
 constexpr uint32_t TM_O = 320;              // O^T fp32
 constexpr uint32_t TM_SB = 384;             // S^T bf16 (operand)
-constexpr uint32_t TM_D = 448;              // [K e^G; Q e^G] (K e^{-G})^T
+constexpr uint32_t TM_D = 448;              // [K e^G; Q e^G] (K e^{-G})^T, then -W^T
 
 struct Bars {
-    uint64_t g, gc, kq, tr, ops, gam, a, t, w, img;   // prep pipeline
+    uint64_t g, gc, kq, tr, ktf, gam, a, w, img;   // prep pipeline
     uint64_t v, u, s, o, ur, sr, orr;          // walk pipeline
     uint64_t m1, fr[2];                     // walk -> prep: MMA1 done, image slot free
-    uint64_t fin_p, fin_w;                  // issuers' final drains
+    uint64_t fin_p, fin_w, fin_q;           // issuers' and the prep leader's final drains
 };
 
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)
@@ -289,11 +288,39 @@ __device__ __forceinline__ uint32_t ct_off(int c, int t)
     return (uint32_t)c * 128u + ((uint32_t)(((t >> 3) ^ c) & 7) << 4);
 }
 
+// Byte offset of element (i, j) in the 128B-swizzled [i][j] bf16 T' tile (64 x 64).
+__device__ __forceinline__ uint32_t tp_off(int i, int j)
+{
+    return sw128_offset(i, j & ~7) + 2u * (uint32_t)(j & 7);
+}
+
+// A 16 x 16 block of T (mma.sync accumulator layout, times `s`) at block (p, r): to the
+// fp32 T (pitch AP) and, scaled by beta_j, to the bf16 T' tile.
+__device__ __forceinline__ void store_t_block(float* sT, unsigned char* tp, const float* sB, int p, int r,
+                                              const float (&acc)[2][4], float s, int lane)
+{
+    store16x16<AP>(sT + (16 * p) * AP + 16 * r, acc, s, lane);
+    const int g = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int nh = 0; nh < 2; ++nh) {
+        const int j = 16 * r + 8 * nh + 2 * q;
+        const float b0 = sB[j], b1 = sB[j + 1];
+        *reinterpret_cast<uint32_t*>(tp + tp_off(16 * p + g, j)) =
+            pack_bf16(s * acc[nh][0] * b0, s * acc[nh][1] * b1);
+        *reinterpret_cast<uint32_t*>(tp + tp_off(16 * p + g + 8, j)) =
+            pack_bf16(s * acc[nh][2] * b0, s * acc[nh][3] * b1);
+    }
+}
+
 // T = (I + A)^{-1} for the strictly lower A (fp32, pitch AP): 16 x 16 diagonal blocks
 // by forward substitution (threads 0-63, one column each), then the blocks below by
 // tf32 block products in two levels (warps 0-3; scratch blocks parked above the
-// diagonal of A).  T's blocks above the diagonal are not written.
-__device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, int tid)
+// diagonal of A).  Every block of T on or below the diagonal is written twice: in fp32
+// to sT (the later levels read it) and as T' = T diag(beta) to the bf16 tile `tp`
+// (the diagonal blocks by warps 2-3 while warps 0-1 take the first level), whose blocks
+// above the diagonal stay zero (written once, when the kernel starts).
+__device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, unsigned char* tp, const float* sB,
+                                                  int tid)
 {
     const int w = tid >> 5, l = tid & 31;
     if (tid < C) {
@@ -323,7 +350,18 @@ __device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, int tid)
         __syncwarp();
         float acc2[2][4] = {};
         mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
-        store16x16<AP>(Tb(p, r), acc2, -1.f, l);
+        store_t_block(sT, tp, sB, p, r, acc2, -1.f, l);
+    } else {                                      // meanwhile, T' of the diagonal blocks
+        const int t = tid - 64, o = 16 * (t >> 4), i = o + (t & 15);
+        float f[8], bt[8];
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+            ld8f(sT + i * AP + o + 8 * hlf, f);
+            ld8f(sB + o + 8 * hlf, bt);
+#pragma unroll
+            for (int x = 0; x < 8; ++x) f[x] *= bt[x];
+            *reinterpret_cast<uint4*>(tp + sw128_offset(i, o + 8 * hlf)) = pack8(f);
+        }
     }
     bar_sync_named(NB_INV, 128);
     {                                             // X_pr = sum_{m = r..1} A_pm T_mr
@@ -337,7 +375,7 @@ __device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, int tid)
         const int p = 2 + (w >> 1), r = w & 1;
         float acc[2][4] = {};
         for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
-        store16x16<AP>(Tb(p, r), acc, -1.f, l);
+        store_t_block(sT, tp, sB, p, r, acc, -1.f, l);
     }
 }
 
@@ -368,7 +406,6 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     __shared__ Bars bars;
     __shared__ uint32_t tmem_base;
-    __shared__ int s_npass;
     __shared__ int s_abort_raw;
     __shared__ int s_ring_val[kRing], s_ring_seq[kRing];
     volatile int* abort = &s_abort_raw;
@@ -381,17 +418,18 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 
     if (tid == W_PI * 32) {
         mbar_init(&bars.g, 1); mbar_init(&bars.gc, 8);
-        mbar_init(&bars.kq, 1); mbar_init(&bars.tr, 1); mbar_init(&bars.ops, 8); mbar_init(&bars.gam, 8);
-        mbar_init(&bars.a, 1); mbar_init(&bars.t, 8); mbar_init(&bars.w, 1); mbar_init(&bars.img, 8);
+        mbar_init(&bars.kq, 1); mbar_init(&bars.tr, 1); mbar_init(&bars.ktf, 8); mbar_init(&bars.gam, 8);
+        mbar_init(&bars.a, 1); mbar_init(&bars.w, 1); mbar_init(&bars.img, 8);
         mbar_init(&bars.v, 1); mbar_init(&bars.u, 1); mbar_init(&bars.s, 1); mbar_init(&bars.o, 1);
         mbar_init(&bars.ur, 4); mbar_init(&bars.sr, 4); mbar_init(&bars.orr, 4);
         mbar_init(&bars.m1, 1); mbar_init(&bars.fr[0], 1); mbar_init(&bars.fr[1], 1);
-        mbar_init(&bars.fin_p, 1); mbar_init(&bars.fin_w, 1);
+        mbar_init(&bars.fin_p, 1); mbar_init(&bars.fin_w, 1); mbar_init(&bars.fin_q, 1);
         fence_mbar_init();
         s_abort_raw = 0;
-        s_npass = 1;
     }
     if (w < 8) {                                  // the identity operand of the transposes
+        for (int e = tid; e < 512; e += 256)      // T' tile: blocks above the diagonal stay 0
+            reinterpret_cast<uint4*>(sm + F_TP)[e] = make_uint4(0, 0, 0, 0);
         if (tid < 128) {
             const int r = tid >> 3, cb = tid & 7;
             float f[8];
@@ -425,8 +463,37 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         const int64_t rs = H * D;                 // floats between token rows of log_alpha
 
         const float* sg = reinterpret_cast<const float*>(sm + F_G);
+        // operand descriptors (the leader issues the prep's MMAs): A and Aqk take the rows
+        // [K e^G; Q e^G] (the Q e^G block of slot s one LBO step after K e^G) against the
+        // columns K e^{-G}; -W^T = -(K e^G)^T T'^T
+        const uint64_t dRow0 = make_desc(smem_u32(sm + F_KG), F_QG - F_KG, 1024);
+        const uint64_t dRow1 = make_desc(smem_u32(sm + F_KG), F_QG + 16384 - F_KG, 1024);
+        const uint64_t dCol = make_desc(smem_u32(sm + F_KD), 16384, 1024);
+        const uint64_t dKgT = make_desc(smem_u32(sm + F_KG), 16, 1024);
+        const uint64_t dTp = make_desc(smem_u32(sm + F_TP), 16, 1024);
+        constexpr uint32_t idA = make_idesc_bf16(128, 64, true, true);
+        constexpr uint32_t idW = make_idesc_bf16(128, 64, false, false, true);
         Items it = it0;
         uint32_t n_a = 0;                         // completions of bars.a seen
+        // -W^T of chunk kk from TMEM into the image, [c][i]; then the image is complete
+        auto read_w = [&](uint32_t kk) -> bool {
+            bool o = true;
+            if (leader) o = fwait(&bars.w, kk & 1, err, 3, abort);
+            if (!bar_and_named(NB_PREP, 256, o)) return false;
+            fence_after_sync();
+            float f[32];
+            tmem_ld16(tmem + lane + TM_D + 32 * ph, f);
+            tmem_ld16(tmem + lane + TM_D + 32 * ph + 16, f + 16);
+            tmem_wait_ld();
+#pragma unroll
+            for (int m = 0; m < 4; ++m)
+                *reinterpret_cast<uint4*>(sm + F_W + sw128_offset(pc, 32 * ph + 8 * m)) = pack8(f + 8 * m);
+            fence_smem_to_async();
+            fence_before_sync();
+            __syncwarp();
+            if (l == 0) mbar_arrive(&bars.img);
+            return true;
+        };
         for (uint32_t k = 0; it.ok; ++k) {
             const int s = (int)(k & 1);
             const int len = it.len();
@@ -476,7 +543,6 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 return bar_and_named(NB_PREP, 256, o);
             };
             const bool fast = bar_and_named(NB_PREP, 256, !(mx > kRange));
-            if (leader) s_npass = fast ? 1 : 7;
 
             unsigned char* qg = sm + F_QG + s * 16384;
             unsigned char* kl = sm + F_KL + s * 16384;
@@ -508,6 +574,19 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             auto put_gamma = [&] {
                 if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
             };
+            // the operand tiles are complete: the leader issues [K e^G; Q e^G] (K e^{-G})^T
+            auto issue_a = [&] {
+                fence_smem_to_async();
+                fence_before_sync();
+                bar_sync_named(NB_PREP, 256);
+                if (leader) {
+                    fence_after_sync();
+#pragma unroll
+                    for (int ks = 0; ks < 8; ++ks)
+                        mma_bf16(tmem + TM_D, (s ? dRow1 : dRow0) + 128u * ks, dCol + 128u * ks, idA, ks > 0);
+                    commit(&bars.a);
+                }
+            };
 
             if (fast) {
                 // ---- (b1) e^{G_i - G_j} = e^{G_i} e^{-G_j}: the image tiles K e^G, Q e^G are the
@@ -537,8 +616,9 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                     }
                 }
                 put_gamma();
-                warp_arrive(&bars.ops);
                 warp_arrive(&bars.gam);
+                warp_arrive(&bars.ktf);           // k^T, q^T read: the next chunk's may land
+                issue_a();
                 if (!wait_m1()) break;
                 if (!wait_a()) break;
                 // ---- A (fp32, beta-scaled rows, for the inverse) and Aqk (bf16 image)
@@ -549,9 +629,14 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 if (q4 < 2) {
                     const int i = pc;
 #pragma unroll
-                    for (int y = 0; y < 32; ++y) {
-                        const int j = 32 * ph + y;
-                        sA[i * AP + j] = (j < i) ? bcur * d[y] : 0.f;
+                    for (int m = 0; m < 8; ++m) {
+                        float4 v4;
+                        const int j = 32 * ph + 4 * m;
+                        v4.x = (j + 0 < i) ? bcur * d[4 * m + 0] : 0.f;
+                        v4.y = (j + 1 < i) ? bcur * d[4 * m + 1] : 0.f;
+                        v4.z = (j + 2 < i) ? bcur * d[4 * m + 2] : 0.f;
+                        v4.w = (j + 3 < i) ? bcur * d[4 * m + 3] : 0.f;
+                        *reinterpret_cast<float4*>(sA + i * AP + j) = v4;
                     }
                     if (ph == 0) sB[i] = bcur;
                 } else {
@@ -627,7 +712,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                         }
                     }
                     if (pass == 7) break;
-                    warp_arrive(&bars.ops);
+                    issue_a();
                     if (!(pok = wait_a())) break;
                     float d[32];
                     tmem_ld16(tmem + lane + TM_D + 32 * ph, d);
@@ -648,43 +733,31 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                     fence_before_sync();          // TMEM reads before the next pass's MMA
                 }
                 if (!pok) break;
+                warp_arrive(&bars.ktf);           // k^T, q^T read (pass 7 was the last)
             }
             fence_smem_to_async();                // Aqk, K e^G, Q e^G: read by the async proxy
             bar_sync_named(NB_PREP, 256);         // A complete
-            // ---- (b2) T = (I + A)^{-1} (warps 0-3)
-            if (w < 4) invert_unit_lower(sA, sT, tid);
+            // ---- (b2) T = (I + A)^{-1} and the bf16 T' = T diag(beta) (warps 0-3)
+            if (w < 4) invert_unit_lower(sA, sT, sm + F_TP, sB, tid);
+            // ---- (b3) -W^T = -(K e^G)^T T'^T: the leader's MMA into the A / Aqk columns
+            // (read out above)
+            fence_smem_to_async();
+            fence_before_sync();
             bar_sync_named(NB_PREP, 256);
-            // T' = T diag(beta), bf16 [i][j]; blocks above the diagonal are zero
-            for (int e = tid; e < C * 8; e += 256) {
-                const int i = e >> 3, cb = e & 7;
-                uint4 u = make_uint4(0, 0, 0, 0);
-                if ((cb >> 1) <= (i >> 4)) {
-                    float f[8], bt[8];
-                    ld8f(sT + i * AP + 8 * cb, f);
-                    ld8f(sB + 8 * cb, bt);
+            if (leader) {
+                fence_after_sync();
 #pragma unroll
-                    for (int x = 0; x < 8; ++x) f[x] *= bt[x];
-                    u = pack8(f);
-                }
-                *reinterpret_cast<uint4*>(sm + F_TP + sw128_offset(i, 8 * cb)) = u;
+                for (int ks = 0; ks < 4; ++ks)
+                    mma_bf16(tmem + TM_D, dKgT + 2u * ks, dTp + 2u * ks, idW, ks > 0);
+                commit(&bars.w);
             }
-            warp_arrive(&bars.t);
-            // ---- (b3) -W^T = -(K e^G)^T T'^T from TMEM into the image, [c][i]
-            ok = true;
-            if (leader) ok = fwait(&bars.w, k & 1, err, 3, abort);
-            if (!bar_and_named(NB_PREP, 256, ok)) break;
-            fence_after_sync();
-            {
-                float f[32];
-                tmem_ld16(tmem + lane + TM_WT + 32 * ph, f);
-                tmem_ld16(tmem + lane + TM_WT + 32 * ph + 16, f + 16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int m = 0; m < 4; ++m)
-                    *reinterpret_cast<uint4*>(sm + F_W + sw128_offset(pc, 32 * ph + 8 * m)) = pack8(f + 8 * m);
-            }
-            warp_arrive(&bars.img);
+            if (!read_w(k)) break;
             it.next(false, sc, si, H32, slots, P, err, abort);
+        }
+        // the leader's MMAs have completed before the CTA frees its tensor memory
+        if (leader) {
+            commit(&bars.fin_q);
+            mbar_wait(&bars.fin_q, 0, nullptr, 0, 200);
         }
     } else if (w < W_PI) {
         // ------------------------------------------------------------------ walk
@@ -865,60 +938,33 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 tma::load_2d(sm + F_KQ + 24576, &qmap, xc + 64, y, &bars.kq);
             };
             Items it = it0;
-            uint32_t n_ops = 0, kq_issued = 0, kq_seen = 0, g_issued = 0;
+            uint32_t kq_issued = 0, kq_seen = 0, g_issued = 0;
+            // k^T, q^T: each 16-token block of the [t][c] tiles times I16 (exact)
+            const uint32_t idT = make_idesc_bf16(128, 16, true, false);
+            const uint64_t dI = make_desc(smem_u32(sm + F_ID), 16, 1024);
+            const uint64_t dK = make_desc(smem_u32(sm + F_KQ), 8192, 1024);
+            const uint64_t dQ = make_desc(smem_u32(sm + F_KQ + 16384), 8192, 1024);
             if (it.ok) { issue_g(it); ++g_issued; issue_kq(it); ++kq_issued; }
             for (uint32_t k = 0; it.ok; ++k) {
                 Items nx = it;
                 nx.next(true, sc, si, H32, slots, P, err, abort);
                 if (!fwait(&bars.kq, k & 1, err, 1, abort)) break;
                 ++kq_seen;
-                if (k > 0 && !fwait(&bars.img, (k - 1) & 1, err, 6, abort)) break;
+                // the prep threads have read chunk k - 1's k^T, q^T
+                if (k > 0 && !fwait(&bars.ktf, (k - 1) & 1, err, 6, abort)) break;
                 fence_after_sync();
-                {                                 // k^T, q^T: each 16-token block times I16 (exact)
-                    const uint32_t id = make_idesc_bf16(128, 16, true, false);
-                    const uint64_t bi = make_desc(smem_u32(sm + F_ID), 16, 1024);
 #pragma unroll
-                    for (int ks = 0; ks < 4; ++ks) {
-                        mma_bf16(tmem + TM_KT + 16 * ks, make_desc(smem_u32(sm + F_KQ + ks * 2048), 8192, 1024),
-                                 bi, id, 0u);
-                        mma_bf16(tmem + TM_QT + 16 * ks,
-                                 make_desc(smem_u32(sm + F_KQ + 16384 + ks * 2048), 8192, 1024), bi, id, 0u);
-                    }
-                    commit(&bars.tr);
+                for (int ks = 0; ks < 4; ++ks) {
+                    mma_bf16(tmem + TM_KT + 16 * ks, dK + 128u * ks, dI, idT, 0u);
+                    mma_bf16(tmem + TM_QT + 16 * ks, dQ + 128u * ks, dI, idT, 0u);
                 }
+                commit(&bars.tr);
                 // the k / q buffer is free once the transposes have read it, the gate tile once
                 // the prep threads have scanned it
                 if (!fwait(&bars.tr, k & 1, err, 1, abort)) break;
                 if (nx.ok) { issue_kq(nx); ++kq_issued; }
                 if (!fwait(&bars.gc, k & 1, err, 6, abort)) break;
                 if (nx.ok) { issue_g(nx); ++g_issued; }
-                const uint32_t s = k & 1;
-                bool ok = true;
-                int np = 1;
-                for (int p = 0; p < np; ++p) {    // [K e^G; Q e^G] (K e^{-G})^T, once per pass
-                    if (!(ok = fwait(&bars.ops, n_ops & 1, err, 6, abort))) break;
-                    ++n_ops;
-                    if (p == 0) np = *reinterpret_cast<volatile int*>(&s_npass);
-                    fence_after_sync();
-                    const uint32_t id = make_idesc_bf16(128, 64, true, true);
-                    const uint32_t lbo = F_QG + s * 16384 - F_KG;    // K e^G -> Q e^G block
-#pragma unroll
-                    for (int ks = 0; ks < 8; ++ks)
-                        mma_bf16(tmem + TM_D, make_desc(smem_u32(sm + F_KG + ks * 2048), lbo, 1024),
-                                 make_desc(smem_u32(sm + F_KD + ks * 2048), 16384, 1024), id, ks > 0);
-                    commit(&bars.a);
-                }
-                if (!ok) break;
-                if (!fwait(&bars.t, k & 1, err, 6, abort)) break;
-                fence_after_sync();
-                {                                 // -W^T = -(K e^G)^T T'^T
-                    const uint32_t id = make_idesc_bf16(128, 64, false, false, true);
-#pragma unroll
-                    for (int ks = 0; ks < 4; ++ks)
-                        mma_bf16(tmem + TM_WT, make_desc(smem_u32(sm + F_KG + ks * 32), 16, 1024),
-                                 make_desc(smem_u32(sm + F_TP + ks * 32), 16, 1024), id, ks > 0);
-                    commit(&bars.w);
-                }
                 it = nx;
             }
             // drain: this thread's MMAs and copies
@@ -949,8 +995,18 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             const uint32_t id_n = make_idesc_bf16(128, 64, false, true);   // S^T x MN-major B
             const uint32_t id_s = make_idesc_bf16(128, 128, false, false); // U^T (K e^{Gl-G})
             const uint32_t id_o = make_idesc_bf16(128, 64, false, false);  // U^T Aqk^T
+            const uint64_t dV = make_desc(smem_u32(sm + F_V), 8192, 1024);
+            const uint64_t dTp = make_desc(smem_u32(sm + F_TP), 16, 1024);
+            const uint64_t dWt = make_desc(smem_u32(sm + F_W), 16384, 1024);
+            // per image slot: the descriptors of slot 1 are those of slot 0 plus the slot
+            // stride (16 KB for Q e^G and K e^{Gl - G}, 8 KB for Aqk) in 16-byte units
+            const uint64_t dQg0 = make_desc(smem_u32(sm + F_QG), 16384, 1024);
+            const uint64_t dKl0 = make_desc(smem_u32(sm + F_KL), 16, 1024);
+            const uint64_t dAq0 = make_desc(smem_u32(sm + F_AQ), 16, 1024);
             for (uint32_t k = 0; it.ok; ++k) {
                 const int s = (int)(k & 1);
+                const uint64_t dQg = dQg0 + (s ? 1024u : 0u), dKl = dKl0 + (s ? 1024u : 0u);
+                const uint64_t dAq = dAq0 + (s ? 512u : 0u);
                 Items nx = it;
                 nx.next(false, sc, si, H32, slots, P, err, abort);
                 if (!fwait(&bars.img, k & 1, err, 6, abort)) break;
@@ -961,22 +1017,16 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 fence_after_sync();
                 // U^T = V^T T'^T + S^T (-W^T)
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16(tmem + TM_U, make_desc(smem_u32(sm + F_V + ks * 2048), 8192, 1024),
-                             make_desc(smem_u32(sm + F_TP + ks * 32), 16, 1024), id_v, ks > 0);
+                for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + TM_U, dV + 128u * ks, dTp + 2u * ks, id_v, ks > 0);
 #pragma unroll
-                for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * ks,
-                                make_desc(smem_u32(sm + F_W + ks * 2048), 16384, 1024), id_n, 1u);
+                for (int ks = 0; ks < 8; ++ks) mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * ks, dWt + 128u * ks, id_n, 1u);
                 commit(&bars.u);
                 // O^T = S^T (Q e^G)^T (the output tile of the previous chunk has left TMEM)
                 if (k > 0 && !fwait(&bars.orr, (k - 1) & 1, err, 6, abort)) break;
                 fence_after_sync();
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * ks,
-                                make_desc(smem_u32(sm + F_QG + s * 16384 + ks * 2048), 16384, 1024), id_n,
-                                ks > 0);
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * ks, dQg + 128u * ks, id_n, ks > 0);
                 if (!fwait(&bars.u, k & 1, err, 5, abort)) break;
                 mbar_arrive(&bars.m1);            // T', -W^T and the v tile are free
                 if (nx.ok) { issue_v(nx); ++v_issued; }
@@ -984,14 +1034,10 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 fence_after_sync();
                 // S^T += U^T (K e^{Gl - G});  O^T += U^T Aqk^T
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TM_S, tmem + TM_U + 8 * ks,
-                                make_desc(smem_u32(sm + F_KL + s * 16384 + ks * 32), 16, 1024), id_s, 1u);
+                for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(tmem + TM_S, tmem + TM_U + 8 * ks, dKl + 2u * ks, id_s, 1u);
                 commit(&bars.s);
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks)
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_U + 8 * ks,
-                                make_desc(smem_u32(sm + F_AQ + s * 8192 + ks * 32), 16, 1024), id_o, 1u);
+                for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(tmem + TM_O, tmem + TM_U + 8 * ks, dAq + 2u * ks, id_o, 1u);
                 commit(&bars.o);
                 it = nx;
             }
