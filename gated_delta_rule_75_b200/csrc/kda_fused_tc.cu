@@ -17,11 +17,13 @@
 //   warps 0-7   prep: thread (channel c, token half) -- cumulative decay in
 //               registers, the exponential factors, the operand tiles [c][t]
 //               (token-contiguous, 128B-swizzled), the A / Aqk read-out, the
-//               blocked inverse of (I + A), T' and the -W^T read-out;
+//               blocked inverse of (I + A) (which also writes T') and the -W^T
+//               read-out; thread 0 issues the A / Aqk and -W^T MMAs itself;
 //   warps 8-11  walk: thread = value column j (a TMEM lane of S^T) -- the
 //               state's decay scaling, the U^T / S^T bf16 copies (kept in
 //               tensor memory as MMA operands), the output tile;
-//   warp 12     one thread issues the prep's TMA loads and MMAs;
+//   warp 12     one thread issues the prep's TMA loads and the k / q transposes,
+//               and (packed sequences) takes each CTA's next chain by ticket;
 //   warp 13     one thread issues the walk's MMAs and v loads.
 // Per chunk, k and q land by TMA as [t][c] tiles and are transposed into tensor
 // memory by an MMA with the identity (exact), so each prep thread owns one
@@ -107,7 +109,7 @@ struct Bars {
     uint64_t g, gc, kq, tr, ktf, gam, a, w, img;   // prep pipeline
     uint64_t v, u, s, o, ur, sr, orr;          // walk pipeline
     uint64_t m1, fr[2];                     // walk -> prep: MMA1 done, image slot free
-    uint64_t fin_p, fin_w, fin_q;           // issuers' and the prep leader's final drains
+    uint64_t fin_p, fin_w, fin_q;           // final drains: prep issuer, walk issuer, prep leader
 };
 
 __device__ __forceinline__ bool mbar_test(uint64_t* bar, uint32_t parity)

@@ -1,6 +1,7 @@
 """The library's prefill and decode calls captured in CUDA graphs (stream-ordered
 workspace from the library's pool becomes graph allocation nodes): replays give
-bit-for-bit the eager results.  Runs in a child process without KDA_DEBUG, whose
+bit-for-bit the eager results -- for a fixed-length batch, packed sequences
+(chains handed out by tickets) and few chains (AUTO's guarded two-kernel form).  Runs in a child process without KDA_DEBUG, whose
 synchronising checks cannot be captured."""
 import os
 import subprocess
@@ -37,6 +38,29 @@ out.zero_(); hT.zero_()
 g.replay(); g.replay()
 torch.cuda.synchronize()
 assert torch.equal(out, ref_out) and torch.equal(hT, ref_hT), "prefill replay differs"
+
+# packed sequences (the fused kernel hands chains out by tickets: the counter is zeroed inside
+# the graph) and few chains (AUTO's two-kernel form with its decay-range flag, then the fused
+# kernel returning at once): replays match the eager calls bit for bit
+for cfg in (W.small_prefill(H=24, dk=128, dv=128, io_dtype="bf16", seed=72, h0_std=0.02,
+                            lengths=[300, 0, 130, 64, 1, 250]),
+            W.small_prefill(B=1, T=700, H=2, dk=128, dv=128, io_dtype="bf16", seed=73, h0_std=0.02)):
+    inp = W.make_prefill(cfg, "cuda")
+    args = (inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"])
+    kw = dict(h0=inp["h0"], cu_seqlens=inp["cu_seqlens"])
+    ref_out, ref_hT = kda.chunk_fwd(*args, **kw)
+    out = torch.empty_like(ref_out); hT = torch.empty_like(ref_hT)
+    with torch.cuda.stream(side):
+        kda.chunk_fwd(*args, out=out, hT=hT, **kw)
+    torch.cuda.current_stream().wait_stream(side)
+    g3 = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g3):
+        kda.chunk_fwd(*args, out=out, hT=hT, **kw)
+    out.zero_(); hT.zero_()
+    g3.replay(); g3.replay()
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref_out) and torch.equal(hT, ref_hT), "replay differs: " + cfg.name
+    del g3
 
 # decode: 5 chained steps captured once
 dcfg = W.DecodeConfig("graph", N=8, H=4, dk=128, dv=128, steps=5, seed=71)
