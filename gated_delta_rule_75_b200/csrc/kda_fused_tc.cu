@@ -71,7 +71,6 @@ constexpr int W_WI = 13;                    // walk issuer
 
 constexpr int NB_PAIR = 1;                  // 1..4: prep warps w and w + 4
 constexpr int NB_PREP = 5;                  // prep warps 0-7
-constexpr int NB_INV = 6;                   // prep warps 0-3
 constexpr int NB_WALK = 7;                  // walk warps
 
 // Shared memory (bytes from a 1024-aligned base).  [c][t] tiles: 128 channel rows of
@@ -296,31 +295,59 @@ __device__ __forceinline__ uint32_t tp_off(int i, int j)
     return sw128_offset(i, j & ~7) + 2u * (uint32_t)(j & 7);
 }
 
-// A 16 x 16 block of T (mma.sync accumulator layout, times `s`) at block (p, r): to the
-// fp32 T (pitch AP) and, scaled by beta_j, to the bf16 T' tile.
-__device__ __forceinline__ void store_t_block(float* sT, unsigned char* tp, const float* sB, int p, int r,
-                                              const float (&acc)[2][4], float s, int lane)
+// Columns 8 nh .. 8 nh + 7 of the 16 x 16 product X Y (fp32 blocks of pitch AP, tf32
+// operands, fp32 accumulation): one m16n8k8 accumulator per k-step pair.
+__device__ __forceinline__ void mma16x8x16_tf32(float (&acc)[4], const float* X, const float* Y, int nh,
+                                                int lane)
 {
-    store16x16<AP>(sT + (16 * p) * AP + 16 * r, acc, s, lane);
     const int g = lane >> 2, q = lane & 3;
 #pragma unroll
-    for (int nh = 0; nh < 2; ++nh) {
-        const int j = 16 * r + 8 * nh + 2 * q;
-        const float b0 = sB[j], b1 = sB[j + 1];
-        *reinterpret_cast<uint32_t*>(tp + tp_off(16 * p + g, j)) =
-            pack_bf16(s * acc[nh][0] * b0, s * acc[nh][1] * b1);
-        *reinterpret_cast<uint32_t*>(tp + tp_off(16 * p + g + 8, j)) =
-            pack_bf16(s * acc[nh][2] * b0, s * acc[nh][3] * b1);
+    for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t a0 = tf32(X[g * AP + 8 * ks + q]);
+        const uint32_t a1 = tf32(X[(g + 8) * AP + 8 * ks + q]);
+        const uint32_t a2 = tf32(X[g * AP + 8 * ks + q + 4]);
+        const uint32_t a3 = tf32(X[(g + 8) * AP + 8 * ks + q + 4]);
+        const uint32_t b0 = tf32(Y[(8 * ks + q) * AP + 8 * nh + g]);
+        const uint32_t b1 = tf32(Y[(8 * ks + q + 4) * AP + 8 * nh + g]);
+        asm volatile(
+            "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 "
+            "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+            : "+f"(acc[0]), "+f"(acc[1]), "+f"(acc[2]), "+f"(acc[3])
+            : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
     }
 }
 
-// T = (I + A)^{-1} for the strictly lower A (fp32, pitch AP): 16 x 16 diagonal blocks
-// by forward substitution (threads 0-63, one column each), then the blocks below by
-// tf32 block products in two levels (warps 0-3; scratch blocks parked above the
-// diagonal of A).  Every block of T on or below the diagonal is written twice: in fp32
-// to sT (the later levels read it) and as T' = T diag(beta) to the bf16 tile `tp`
-// (the diagonal blocks by warps 2-3 while warps 0-1 take the first level), whose blocks
-// above the diagonal stay zero (written once, when the kernel starts).
+// Stores columns 8 nh .. + 7 of a 16 x 16 block (accumulator layout, times `s`) to Z.
+__device__ __forceinline__ void store16x8(float* Z, const float (&acc)[4], float s, int nh, int lane)
+{
+    const int g = lane >> 2, q = lane & 3;
+    Z[g * AP + 8 * nh + 2 * q] = s * acc[0];
+    Z[g * AP + 8 * nh + 2 * q + 1] = s * acc[1];
+    Z[(g + 8) * AP + 8 * nh + 2 * q] = s * acc[2];
+    Z[(g + 8) * AP + 8 * nh + 2 * q + 1] = s * acc[3];
+}
+
+// Columns 8 nh .. + 7 of block (p, r) of T (times `s`): to the fp32 T (pitch AP) and,
+// scaled by beta_j, to the bf16 T' tile.
+__device__ __forceinline__ void store_t_half(float* sT, unsigned char* tp, const float* sB, int p, int r,
+                                             int nh, const float (&acc)[4], float s, int lane)
+{
+    store16x8(sT + (16 * p) * AP + 16 * r, acc, s, nh, lane);
+    const int g = lane >> 2, q = lane & 3;
+    const int j = 16 * r + 8 * nh + 2 * q;
+    const float b0 = sB[j], b1 = sB[j + 1];
+    *reinterpret_cast<uint32_t*>(tp + tp_off(16 * p + g, j)) = pack_bf16(s * acc[0] * b0, s * acc[1] * b1);
+    *reinterpret_cast<uint32_t*>(tp + tp_off(16 * p + g + 8, j)) = pack_bf16(s * acc[2] * b0, s * acc[3] * b1);
+}
+
+// T = (I + A)^{-1} for the strictly lower A (fp32, pitch AP), by all eight prep warps:
+// 16 x 16 diagonal blocks by forward substitution (threads 0-63, one column each), then
+// the blocks below by tf32 block products in three levels, each 16 x 16 product split
+// into its two 8-column halves on two warps (scratch blocks parked above the diagonal
+// of A).  Every block of T on or below the diagonal is written twice: in fp32 to sT (the
+// later levels read it) and as T' = T diag(beta) to the bf16 tile `tp` (the diagonal
+// blocks by warps 4-7 during the first level), whose blocks above the diagonal stay zero
+// (written once, when the kernel starts).
 __device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, unsigned char* tp, const float* sB,
                                                   int tid)
 {
@@ -341,43 +368,39 @@ __device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, unsigned
 #pragma unroll
         for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
     }
-    bar_sync_named(NB_INV, 128);
+    bar_sync_named(NB_PREP, 256);
     auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
     auto Tb = [&](int r, int c) { return sT + (16 * r) * AP + 16 * c; };
-    if (w < 2) {                                  // T_10 = -T_11 A_10 T_00, T_32 = -T_33 A_32 T_22
-        const int p = 2 * w + 1, r = 2 * w;
-        float acc[2][4] = {};
-        mma16x16x16_tf32<AP>(acc, Ab(p, r), Tb(r, r), l);
-        store16x16<AP>(Ab(r, p), acc, 1.f, l);
+    if (w < 4) {                                  // T_10 = -T_11 A_10 T_00, T_32 = -T_33 A_32 T_22
+        const int p = 2 * (w & 1) + 1, r = p - 1, nh = w >> 1;
+        float acc[4] = {};
+        mma16x8x16_tf32(acc, Ab(p, r), Tb(r, r), nh, l);
+        store16x8(Ab(r, p), acc, 1.f, nh, l);
         __syncwarp();
-        float acc2[2][4] = {};
-        mma16x16x16_tf32<AP>(acc2, Tb(p, p), Ab(r, p), l);
-        store_t_block(sT, tp, sB, p, r, acc2, -1.f, l);
+        float acc2[4] = {};
+        mma16x8x16_tf32(acc2, Tb(p, p), Ab(r, p), nh, l);
+        store_t_half(sT, tp, sB, p, r, nh, acc2, -1.f, l);
     } else {                                      // meanwhile, T' of the diagonal blocks
-        const int t = tid - 64, o = 16 * (t >> 4), i = o + (t & 15);
+        const int t = tid - 128, o = 16 * (t >> 5), i = o + ((t >> 1) & 15), hlf = t & 1;
         float f[8], bt[8];
+        ld8f(sT + i * AP + o + 8 * hlf, f);
+        ld8f(sB + o + 8 * hlf, bt);
 #pragma unroll
-        for (int hlf = 0; hlf < 2; ++hlf) {
-            ld8f(sT + i * AP + o + 8 * hlf, f);
-            ld8f(sB + o + 8 * hlf, bt);
-#pragma unroll
-            for (int x = 0; x < 8; ++x) f[x] *= bt[x];
-            *reinterpret_cast<uint4*>(tp + sw128_offset(i, o + 8 * hlf)) = pack8(f);
-        }
+        for (int x = 0; x < 8; ++x) f[x] *= bt[x];
+        *reinterpret_cast<uint4*>(tp + sw128_offset(i, o + 8 * hlf)) = pack8(f);
     }
-    bar_sync_named(NB_INV, 128);
+    bar_sync_named(NB_PREP, 256);
+    const int p = 2 + ((w >> 1) & 1), r = w & 1, nh = w >> 2;
     {                                             // X_pr = sum_{m = r..1} A_pm T_mr
-        const int p = 2 + (w >> 1), r = w & 1;
-        float acc[2][4] = {};
-        for (int m = r; m < 2; ++m) mma16x16x16_tf32<AP>(acc, Ab(p, m), Tb(m, r), l);
-        store16x16<AP>(Ab(r, p), acc, 1.f, l);
+        float acc[4] = {};
+        for (int m = r; m < 2; ++m) mma16x8x16_tf32(acc, Ab(p, m), Tb(m, r), nh, l);
+        store16x8(Ab(r, p), acc, 1.f, nh, l);
     }
-    bar_sync_named(NB_INV, 128);
+    bar_sync_named(NB_PREP, 256);
     {                                             // T_pr = -sum_{m = 2..p} T_pm X_mr
-        const int p = 2 + (w >> 1), r = w & 1;
-        float acc[2][4] = {};
-        for (int m = 2; m <= p; ++m) mma16x16x16_tf32<AP>(acc, Tb(p, m), Ab(r, m), l);
-        store_t_block(sT, tp, sB, p, r, acc, -1.f, l);
+        float acc[4] = {};
+        for (int m = 2; m <= p; ++m) mma16x8x16_tf32(acc, Tb(p, m), Ab(r, m), nh, l);
+        store_t_half(sT, tp, sB, p, r, nh, acc, -1.f, l);
     }
 }
 
@@ -740,7 +763,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             fence_smem_to_async();                // Aqk, K e^G, Q e^G: read by the async proxy
             bar_sync_named(NB_PREP, 256);         // A complete
             // ---- (b2) T = (I + A)^{-1} and the bf16 T' = T diag(beta) (warps 0-3)
-            if (w < 4) invert_unit_lower(sA, sT, sm + F_TP, sB, tid);
+            invert_unit_lower(sA, sT, sm + F_TP, sB, tid);
             // ---- (b3) -W^T = -(K e^G)^T T'^T: the leader's MMA into the A / Aqk columns
             // (read out above)
             fence_smem_to_async();
