@@ -341,7 +341,7 @@ __device__ __forceinline__ void store_t_half(float* sT, unsigned char* tp, const
 }
 
 // T = (I + A)^{-1} for the strictly lower A (fp32, pitch AP), by all eight prep warps:
-// 16 x 16 diagonal blocks by forward substitution (threads 0-63, one column each), then
+// 16 x 16 diagonal blocks from their 8 x 8 halves (threads 0-63), then
 // the blocks below by tf32 block products in three levels, each 16 x 16 product split
 // into its two 8-column halves on two warps (scratch blocks parked above the diagonal
 // of A).  Every block of T on or below the diagonal is written twice: in fp32 to sT (the
@@ -353,20 +353,44 @@ __device__ __forceinline__ void invert_unit_lower(float* sA, float* sT, unsigned
 {
     const int w = tid >> 5, l = tid & 31;
     if (tid < C) {
-        const int b = tid >> 4, cc = tid & 15, o = 16 * b;
-        float tcol[16];
+        // each 16 x 16 diagonal block (16 threads of one warp): its two 8 x 8 diagonal
+        // blocks by forward substitution (one column per thread), then the 8 x 8 block
+        // below them, L = -T_hi A_lo,hi-lo T_lo, by two fp32 products; Y = A T_lo is parked
+        // in the block's unused upper-right 8 x 8 quarter
+        const int b = tid >> 4, cc = tid & 15, o = 16 * b + 8 * (cc >> 3), c8 = cc & 7;
+        float tcol[8];
 #pragma unroll
-        for (int r = 0; r < 16; ++r) {
-            float acc0 = 0.f, acc1 = 0.f;
+        for (int r = 0; r < 8; ++r) {
+            float acc = 0.f;
 #pragma unroll
-            for (int m = 0; m < r; ++m) {
-                if (m & 1) acc1 += sA[(o + r) * AP + o + m] * tcol[m];
-                else acc0 += sA[(o + r) * AP + o + m] * tcol[m];
-            }
-            tcol[r] = (r == cc) ? 1.f : ((r < cc) ? 0.f : -(acc0 + acc1));
+            for (int m = 0; m < r; ++m) acc += sA[(o + r) * AP + o + m] * tcol[m];
+            tcol[r] = (r == c8) ? 1.f : ((r < c8) ? 0.f : -acc);
         }
 #pragma unroll
-        for (int r = 0; r < 16; ++r) sT[(o + r) * AP + o + cc] = tcol[r];
+        for (int r = 0; r < 8; ++r) sT[(o + r) * AP + o + c8] = tcol[r];
+        __syncwarp();
+        const int ob = 16 * b, i = cc >> 1, j0 = 4 * (cc & 1);   // this thread: row i, columns j0..j0+3
+        float y[4];
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {               // Y = A[8+i][0..7] T_lo[.][j]
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc += sA[(ob + 8 + i) * AP + ob + m] * sT[(ob + m) * AP + ob + j0 + x];
+            y[x] = acc;
+        }
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sA[(ob + i) * AP + ob + 8 + j0 + x] = y[x];
+        __syncwarp();
+#pragma unroll
+        for (int x = 0; x < 4; ++x) {               // L = -T_hi Y  (T_hi unit lower)
+            float acc = 0.f;
+#pragma unroll
+            for (int m = 0; m < 8; ++m) acc += sT[(ob + 8 + i) * AP + ob + 8 + m] * sA[(ob + m) * AP + ob + 8 + j0 + x];
+            sT[(ob + 8 + i) * AP + ob + j0 + x] = -acc;
+        }
+        // T's upper-right 8 x 8 quarter of the block is zero
+#pragma unroll
+        for (int x = 0; x < 4; ++x) sT[(ob + i) * AP + ob + 8 + j0 + x] = 0.f;
     }
     bar_sync_named(NB_PREP, 256);
     auto Ab = [&](int r, int c) { return sA + (16 * r) * AP + 16 * c; };
