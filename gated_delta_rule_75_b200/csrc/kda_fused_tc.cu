@@ -624,8 +624,9 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 if (ph == 0) reinterpret_cast<float*>(sm + F_GAM + s * 512)[pc] = ex2(Gl);
             };
             // the operand tiles are complete: the leader issues [K e^G; Q e^G] (K e^{-G})^T
-            auto issue_a = [&] {
-                fence_smem_to_async();
+            // (`fenced`: this thread's tile writes already passed a proxy fence)
+            auto issue_a = [&](bool fenced) {
+                if (!fenced) fence_smem_to_async();
                 fence_before_sync();
                 bar_sync_named(NB_PREP, 256);
                 if (leader) {
@@ -665,9 +666,16 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                     }
                 }
                 put_gamma();
-                warp_arrive(&bars.gam);
-                warp_arrive(&bars.ktf);           // k^T, q^T read: the next chunk's may land
-                issue_a();
+                // one proxy fence for the tiles; e^{G_last} is read by the walk warps (generic)
+                // and k^T, q^T have been read (the next chunk's may land)
+                fence_smem_to_async();
+                fence_before_sync();
+                __syncwarp();
+                if (l == 0) {
+                    mbar_arrive(&bars.gam);
+                    mbar_arrive(&bars.ktf);
+                }
+                issue_a(true);
                 if (!wait_m1()) break;
                 if (!wait_a()) break;
                 // ---- A (fp32, beta-scaled rows, for the inverse) and Aqk (bf16 image)
@@ -761,7 +769,7 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                         }
                     }
                     if (pass == 7) break;
-                    issue_a();
+                    issue_a(false);
                     if (!(pok = wait_a())) break;
                     float d[32];
                     tmem_ld16(tmem + lane + TM_D + 32 * ph, d);
@@ -784,9 +792,18 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 if (!pok) break;
                 warp_arrive(&bars.ktf);           // k^T, q^T read (pass 7 was the last)
             }
-            fence_smem_to_async();                // Aqk, K e^G, Q e^G: read by the async proxy
-            bar_sync_named(NB_PREP, 256);         // A complete
-            // ---- (b2) T = (I + A)^{-1} and the bf16 T' = T diag(beta) (warps 0-3)
+            if (fast) {
+                // the inverse starts with the diagonal 16 x 16 blocks: warp 0 solves rows and
+                // columns 0-31, which it extracted itself; warp 1 solves 32-63, extracted by
+                // warp 5 (the image tiles reach the async proxy through the fence after the
+                // inverse; the inverse's first barrier completes A for the later levels)
+                if (q4 == 1) bar_sync_named(NB_PAIR + 1, 64);
+                else if (w == 0) __syncwarp();
+            } else {
+                fence_smem_to_async();            // Aqk, K e^G, Q e^G: read by the async proxy
+                bar_sync_named(NB_PREP, 256);     // A complete
+            }
+            // ---- (b2) T = (I + A)^{-1} and the bf16 T' = T diag(beta)
             invert_unit_lower(sA, sT, sm + F_TP, sB, tid);
             // ---- (b3) -W^T = -(K e^G)^T T'^T: the leader's MMA into the A / Aqk columns
             // (read out above)
