@@ -671,13 +671,13 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 fence_smem_to_async();
                 fence_before_sync();
                 __syncwarp();
-                if (l == 0) {
-                    mbar_arrive(&bars.gam);
-                    mbar_arrive(&bars.ktf);
-                }
+                if (l == 0) mbar_arrive(&bars.gam);
                 issue_a(true);
                 if (!wait_m1()) break;
                 if (!wait_a()) break;
+                // k^T, q^T were read before A was issued; signalled only now so that the next
+                // chunk's transposes do not queue ahead of A on the tensor pipe
+                if (l == 0) mbar_arrive(&bars.ktf);
                 // ---- A (fp32, beta-scaled rows, for the inverse) and Aqk (bf16 image)
                 float d[32];
                 tmem_ld16(tmem + lane + TM_D + 32 * ph, d);
