@@ -17,8 +17,9 @@
 //   warps 0-7   prep: thread (channel c, token half) -- cumulative decay in
 //               registers, the exponential factors, the operand tiles [c][t]
 //               (token-contiguous, 128B-swizzled), the A / Aqk read-out, the
-//               blocked inverse of (I + A) (which also writes T') and the -W^T
-//               read-out; thread 0 issues the A / Aqk and -W^T MMAs itself;
+//               blocked inverse of (I + A) (its block products split over all
+//               eight warps; it also writes T') and the -W^T read-out; thread 0
+//               issues the A / Aqk and -W^T MMAs itself;
 //   warps 8-11  walk: thread = value column j (a TMEM lane of S^T) -- the
 //               state's decay scaling, the U^T / S^T bf16 copies (kept in
 //               tensor memory as MMA operands), the output tile;
@@ -27,7 +28,9 @@
 //   warp 13     one thread issues the walk's MMAs and v loads.
 // Per chunk, k and q land by TMA as [t][c] tiles and are transposed into tensor
 // memory by an MMA with the identity (exact), so each prep thread owns one
-// channel's tokens.  The decay factors e^{G_i - G_j} are split as e^{G_i} e^{-G_j}
+// channel's tokens; the next chunk's transposes are released only once the A / Aqk
+// MMA of this one has completed, so that they never queue ahead of it on the tensor
+// pipe.  The decay factors e^{G_i - G_j} are split as e^{G_i} e^{-G_j}
 // when every |G| of the chunk stays within 2^100: the row operands of A and Aqk
 // are then the image tiles K e^G and Q e^G themselves, the column operand is
 // K e^{-G}, and A and Aqk are one MMA.  Otherwise the lower triangle is taken
