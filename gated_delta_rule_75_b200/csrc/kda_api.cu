@@ -414,10 +414,26 @@ static kda_status_t chunk_fwd_impl(const void* q, const void* k, const void* v,
     // after them computes the call only in that case.
     const bool auto_tc = use_tc && !segmap && !gate_scalar && T_total > 0 &&
                          (impl == KDA_PREFILL_AUTO || impl == KDA_PREFILL_TENSORCORE);
-    const bool guarded = auto_tc && si.N * H * 2 <= device_sm_count();
+    bool guarded = auto_tc && si.N * H * 2 <= device_sm_count();
     if (use_tc && !segmap) {
         plan = plan_segments(si, H, impl, guarded);
         if (plan.upper > 0x7fffffffLL / H) std::memset(&plan, 0, sizeof(plan));
+    }
+    // ... and only when every head fits one head group: with several groups, a group's walks
+    // finish (writing hT, which may alias h0) before a later group's prep can flag a block,
+    // and the fused kernel would then start those heads from overwritten states
+    if (guarded) {
+        const bool st = plan.len > 0 && cu_seqlens != nullptr;
+        const int64_t ob =
+            cu_seqlens ? ((B + 1) * 8 + (st ? (B + 1) * 8 : (B <= kMaxOrderedSeqs ? B * 4 : 0)) + 1023) /
+                             1024 * 1024
+                       : 0;
+        const int64_t ph = tc_ws_bytes_per_chunk() * (si.chunks_upper > 0 ? si.chunks_upper : 1) +
+                           tc_seg_bytes_per_head(plan);
+        if ((workspace_budget() - 1024 - ob) / ph < H) {
+            guarded = false;
+            std::memset(&plan, 0, sizeof(plan));
+        }
     }
     const bool seg_table = use_tc && !segmap && plan.len > 0 && cu_seqlens != nullptr;
     const bool use_fused = auto_tc ? !guarded : (impl == KDA_PREFILL_TENSORCORE_FUSED && !gate_scalar &&

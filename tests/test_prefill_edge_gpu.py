@@ -27,22 +27,33 @@ def kda(cuda_ok):
     return kda
 
 
-@pytest.mark.parametrize("impl", ["simt", "tensorcore_chain", "tensorcore_fused"])
-def test_head_groups_with_small_workspace(cuda_ok, impl):
+@pytest.mark.parametrize("impl,shift", [("simt", 0.0), ("tensorcore_chain", 0.0),
+                                        ("tensorcore_fused", 0.0), ("auto", 8.0)])
+def test_head_groups_with_small_workspace(cuda_ok, impl, shift):
     """64 MiB budget: 512 chunks per head need about 34 MB (two-kernel tensor-core
     path) or 76 MB (SIMT), so the three heads run in separate groups; the fused
-    kernel needs no per-chunk workspace and runs them in one launch."""
+    kernel needs no per-chunk workspace and runs them in one launch.  AUTO with its
+    12 chains would take the two-kernel form first, but not when the heads need
+    several groups: here, at a decay (about e^-8 per token) that form's prep would
+    flag, with the final states written over the initial ones in place, it runs the
+    fused kernel alone."""
     code = textwrap.dedent(f"""
         import sys; sys.path.insert(0, {ROOT!r}); sys.path.insert(0, {os.path.join(ROOT, 'tests')!r})
         import workloads as W, gated_delta_rule_75_b200 as kda, torch
         from kda_testutil import TOL, oracle_prefill, rel
-        cfg = W.small_prefill(B=4, T=8192, H=3, dk=128, dv=128, io_dtype="bf16", seed=31, h0_std=0.02)
+        cfg = W.small_prefill(B=4, T=8192, H=3, dk=128, dv=128, io_dtype="bf16", seed=31, h0_std=0.02,
+                              gate_shift={shift!r})
         inp = W.make_prefill(cfg, "cuda")
-        out, hT = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
-                                inp["scale"], h0=inp["h0"], impl={impl!r})
-        torch.cuda.synchronize()
         ro, rh = oracle_prefill(inp)
-        eo, eh = rel(out, ro), rel(hT, rh)
+        state = inp["h0"].clone()
+        kda.profiler_read(reset=True)
+        out, hT = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                                inp["scale"], h0=state, hT=state, impl={impl!r})
+        torch.cuda.synchronize()
+        st = kda.profiler_read(reset=True)
+        if {impl!r} == "auto":
+            assert st.get("chunk_prep_tc", (0,))[0] == 0 and st["chunk_fused_tc"][0] == 1, st
+        eo, eh = rel(out, ro), rel(state, rh)
         print(eo, eh)
         assert eo <= TOL["bf16"] and eh <= TOL["bf16"], (eo, eh)
     """)

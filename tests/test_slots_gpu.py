@@ -130,6 +130,39 @@ def test_negative_slot_means_no_cached_state(kda, impl):
     torch.testing.assert_close(pool[2], before[2], rtol=0, atol=0)
 
 
+@pytest.mark.parametrize("lengths", [[300, 130, 0, 200], [700]])
+def test_pool_prefill_past_the_two_kernel_decay_range(kda, lengths):
+    """AUTO with few chains on a state pool at about e^-8 of decay per token: the two-kernel
+    form's prep flags the blocks, its walks leave the pool untouched, and the fused kernel
+    continues every sequence from its slot and returns it there (pooled states read and
+    written in place); unused slots stay as they were."""
+    H, d = 2, 128
+    cfg = W.small_prefill(H=H, dk=d, dv=d, io_dtype="bf16", seed=54, gate_shift=8.0,
+                          lengths=lengths)
+    inp = W.make_prefill(cfg, "cuda")
+    N = len(lengths)
+    P = N + 2
+    pool = torch.randn((P, H, d, d), device="cuda") * 0.05
+    before = pool.clone()
+    slot_list = [P - 1 - n for n in range(N)]
+    slots = torch.tensor(slot_list, dtype=torch.int32, device="cuda")
+    kda.profiler_read(reset=True)
+    out, _ = kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"],
+                           inp["scale"], cu_seqlens=inp["cu_seqlens"], state_pool=pool, slots=slots)
+    torch.cuda.synchronize()
+    st = kda.profiler_read(reset=True)
+    assert st["chunk_prep_tc"][0] >= 1 and st["chunk_fused_tc"][0] == 1, st
+    h0 = before[slot_list]
+    ro, rh = oracle.fwd(host(inp["q"]), host(inp["k"]), host(inp["v"]), host(inp["log_alpha"]),
+                        host(inp["beta"]), inp["scale"], h0=host(h0),
+                        cu_seqlens=host(inp["cu_seqlens"]).numpy())
+    assert rel(out, ro) <= TOL["bf16"]
+    for n, sl in enumerate(slot_list):
+        assert rel(pool[sl], rh[n]) <= TOL["bf16"], n
+    for sl in range(P - N):
+        torch.testing.assert_close(pool[sl], before[sl], rtol=0, atol=0)
+
+
 @pytest.mark.parametrize("impl", ["simt", "tensorcore"])
 def test_slot_beyond_pool_is_reported(kda, impl):
     H, d = 2, 128
