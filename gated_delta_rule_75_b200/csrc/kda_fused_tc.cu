@@ -38,7 +38,9 @@
 // where i and j fall in different halves, both factors referenced to the first
 // row of the upper half and so <= 1), plus one product for the diagonal: exact
 // at any decay rate.  The state walk of chunk c (U^T = V^T T'^T + S^T (-W^T),
-// O^T = S^T (Q e^G)^T + U^T Aqk^T, S^T += U^T (K e^{Gl - G})) overlaps the prep
+// O^T = S^T (Q e^G)^T + U^T Aqk^T, S^T += U^T (K e^{Gl - G}), as three MMA groups:
+// [O^T | U^T] = S^T [(Q e^G)^T | -W^T] with N = 128, U^T += V^T T'^T, and
+// [S^T | O^T] += U^T [K e^{Gl - G} ; Aqk] with N = 192) overlaps the prep
 // of chunk c + 1; the state's decay by the next chunk's e^{G_last} is applied
 // as the walk copies the state for that chunk.  Operands whose producer and
 // consumer overlap are double-buffered, the rest are handed over on mbarriers.  Every wait is
@@ -85,8 +87,7 @@ constexpr uint32_t F_KQ = 34816;            // k | q [t][c] (TMA)               
 constexpr uint32_t F_KD = 67584;            // (K e^{-G})^T, then T fp32 [64][AP]          17 KB
 constexpr uint32_t F_KG = 84992;            // (K e^G)^T                                   16 KB
 constexpr uint32_t F_QG = 101376;           // (Q e^G)^T x 2; after use the output tile    32 KB
-constexpr uint32_t F_KL = 134144;           // (K e^{Gl - G})^T x 2                        32 KB
-constexpr uint32_t F_AQ = 166912;           // Aqk [i][j] x 2                              16 KB
+constexpr uint32_t F_KLAQ = 134144;         // per slot: (K e^{Gl - G})^T, then Aqk [i][j]  48 KB
 constexpr uint32_t F_TP = 183296;           // T' [i][j]                                    8 KB
 constexpr uint32_t F_W = 191488;            // A fp32 [64][AP] for the inverse, then -W^T  17 KB
 constexpr uint32_t F_V = 208896;            // v [t][dv] (TMA)                             16 KB
@@ -102,8 +103,9 @@ static_assert(F_W + 64 * AP * 4 <= F_V, "A scratch overlaps v");
 constexpr uint32_t TM_KT = 0;               // k^T fp32 (prep)
 constexpr uint32_t TM_QT = 64;              // q^T fp32
 constexpr uint32_t TM_S = 128;              // S^T fp32 (state)
-constexpr uint32_t TM_U = 256;              // U^T fp32; its first 32 columns then hold U^T bf16
-constexpr uint32_t TM_O = 320;              // O^T fp32
+constexpr uint32_t TM_O = 256;              // O^T fp32 (right after S^T: one N = 192 update)
+constexpr uint32_t TM_U = 320;              // U^T fp32 (right after O^T: one N = 128 product);
+                                            // its first 32 columns then hold U^T bf16
 constexpr uint32_t TM_SB = 384;             // S^T bf16 (operand)
 constexpr uint32_t TM_D = 448;              // [K e^G; Q e^G] (K e^{-G})^T, then -W^T
 
@@ -512,7 +514,6 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
         float* xch = reinterpret_cast<float*>(sm + F_XCH);
         float* sA = reinterpret_cast<float*>(sm + F_W);
         float* sT = reinterpret_cast<float*>(sm + F_KD);
-        const int64_t rs = H * D;                 // floats between token rows of log_alpha
 
         const float* sg = reinterpret_cast<const float*>(sm + F_G);
         // operand descriptors (the leader issues the prep's MMAs): A and Aqk take the rows
@@ -597,8 +598,8 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             const bool fast = bar_and_named(NB_PREP, 256, !(mx > kRange));
 
             unsigned char* qg = sm + F_QG + s * 16384;
-            unsigned char* kl = sm + F_KL + s * 16384;
-            unsigned char* aq = sm + F_AQ + s * 8192;
+            unsigned char* kl = sm + F_KLAQ + s * 24576;
+            unsigned char* aq = kl + 16384;
             auto load_kq = [&](int hb, float* kf, float* qf) {
                 tmem_ld16(tmem + lane + TM_KT + 32 * ph + 16 * hb, kf);
                 tmem_ld16(tmem + lane + TM_QT + 32 * ph + 16 * hb, qf);
@@ -1061,21 +1062,20 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             uint32_t v_issued = 0, v_seen = 0;
             if (it.ok) { issue_v(it); ++v_issued; }
             const uint32_t id_v = make_idesc_bf16(128, 64, true, false);   // V^T T'^T
-            const uint32_t id_n = make_idesc_bf16(128, 64, false, true);   // S^T x MN-major B
-            const uint32_t id_s = make_idesc_bf16(128, 128, false, false); // U^T (K e^{Gl-G})
-            const uint32_t id_o = make_idesc_bf16(128, 64, false, false);  // U^T Aqk^T
             const uint64_t dV = make_desc(smem_u32(sm + F_V), 8192, 1024);
             const uint64_t dTp = make_desc(smem_u32(sm + F_TP), 16, 1024);
-            const uint64_t dWt = make_desc(smem_u32(sm + F_W), 16384, 1024);
             // per image slot: the descriptors of slot 1 are those of slot 0 plus the slot
             // stride (16 KB for Q e^G and K e^{Gl - G}, 8 KB for Aqk) in 16-byte units
-            const uint64_t dQg0 = make_desc(smem_u32(sm + F_QG), 16384, 1024);
-            const uint64_t dKl0 = make_desc(smem_u32(sm + F_KL), 16, 1024);
-            const uint64_t dAq0 = make_desc(smem_u32(sm + F_AQ), 16, 1024);
+            // [(Q e^G)^T | -W^T] as one MN-major B of N = 128 (the -W^T block one LBO step
+            // after the slot's Q e^G), [K e^{Gl - G} ; Aqk] as one K-major B of N = 192
+            const uint64_t dQW0 = make_desc(smem_u32(sm + F_QG), F_W - F_QG, 1024);
+            const uint64_t dQW1 = make_desc(smem_u32(sm + F_QG + 16384), F_W - F_QG - 16384, 1024);
+            const uint64_t dKA0 = make_desc(smem_u32(sm + F_KLAQ), 16, 1024);
+            const uint32_t id_uo = make_idesc_bf16(128, 128, false, true);
+            const uint32_t id_so = make_idesc_bf16(128, 192, false, false);
             for (uint32_t k = 0; it.ok; ++k) {
                 const int s = (int)(k & 1);
-                const uint64_t dQg = dQg0 + (s ? 1024u : 0u), dKl = dKl0 + (s ? 1024u : 0u);
-                const uint64_t dAq = dAq0 + (s ? 512u : 0u);
+                const uint64_t dQW = s ? dQW1 : dQW0, dKA = dKA0 + (s ? 1536u : 0u);
                 Items nx = it;
                 nx.next(false, sc, si, H32, slots, P, err, abort);
                 if (!fwait(&bars.img, k & 1, err, 6, abort)) break;
@@ -1083,30 +1083,25 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 ++v_seen;
                 if (!fwait(&bars.sr, k & 1, err, 6, abort)) break;
                 if (k > 0 && !fwait(&bars.o, (k - 1) & 1, err, 5, abort)) break;
-                fence_after_sync();
-                // U^T = V^T T'^T + S^T (-W^T)
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + TM_U, dV + 128u * ks, dTp + 2u * ks, id_v, ks > 0);
-#pragma unroll
-                for (int ks = 0; ks < 8; ++ks) mma_bf16_ts(tmem + TM_U, tmem + TM_SB + 8 * ks, dWt + 128u * ks, id_n, 1u);
-                commit(&bars.u);
-                // O^T = S^T (Q e^G)^T (the output tile of the previous chunk has left TMEM)
+                // the output tile of the previous chunk has left TMEM
                 if (k > 0 && !fwait(&bars.orr, (k - 1) & 1, err, 6, abort)) break;
                 fence_after_sync();
+                // [O^T | U^T] = S^T [(Q e^G)^T | -W^T], then U^T += V^T T'^T
 #pragma unroll
                 for (int ks = 0; ks < 8; ++ks)
-                    mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * ks, dQg + 128u * ks, id_n, ks > 0);
+                    mma_bf16_ts(tmem + TM_O, tmem + TM_SB + 8 * ks, dQW + 128u * ks, id_uo, ks > 0);
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) mma_bf16(tmem + TM_U, dV + 128u * ks, dTp + 2u * ks, id_v, 1u);
+                commit(&bars.u);
                 if (!fwait(&bars.u, k & 1, err, 5, abort)) break;
                 mbar_arrive(&bars.m1);            // T', -W^T and the v tile are free
                 if (nx.ok) { issue_v(nx); ++v_issued; }
                 if (!fwait(&bars.ur, k & 1, err, 6, abort)) break;
                 fence_after_sync();
-                // S^T += U^T (K e^{Gl - G});  O^T += U^T Aqk^T
+                // [S^T | O^T] += U^T [K e^{Gl - G} ; Aqk]
 #pragma unroll
-                for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(tmem + TM_S, tmem + TM_U + 8 * ks, dKl + 2u * ks, id_s, 1u);
+                for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(tmem + TM_S, tmem + TM_U + 8 * ks, dKA + 2u * ks, id_so, 1u);
                 commit(&bars.s);
-#pragma unroll
-                for (int ks = 0; ks < 4; ++ks) mma_bf16_ts(tmem + TM_O, tmem + TM_U + 8 * ks, dAq + 2u * ks, id_o, 1u);
                 commit(&bars.o);
                 it = nx;
             }
