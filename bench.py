@@ -621,7 +621,9 @@ def run_workload(kda, cfg, reps, warmup, peaks, ws, flush):
     `reps` calls each bracketed by its own CUDA events on the launching stream (with
     `flush`, a 256 MB buffer is written before every rep, outside the events, so a
     workload that fits in L2 is read from HBM); the median rep is reported, max over
-    ranks, with the dominant kernel's roofline and every kernel's time per call."""
+    ranks.  The library's per-kernel events are off in those reps (they would sit
+    between the call's launches); a second set of `reps` calls with them on gives the
+    dominant kernel's roofline and every kernel's time per call."""
     inp = W.make_prefill(cfg, "cuda")
     io = torch.bfloat16 if cfg.io_dtype == "bf16" else torch.float32
     out = torch.empty((cfg.B, cfg.T, cfg.H, cfg.dv), dtype=io, device="cuda")
@@ -633,32 +635,38 @@ def run_workload(kda, cfg, reps, warmup, peaks, ws, flush):
         kda.chunk_fwd(inp["q"], inp["k"], inp["v"], inp["log_alpha"], inp["beta"], inp["scale"],
                       h0=inp["h0"], cu_seqlens=inp["cu_seqlens"], out=out, hT=hT)
 
+    def timed_reps():
+        t = []
+        for _ in range(reps):
+            if fbuf is not None:
+                fbuf.fill_(1.0)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record(stream)
+            step()
+            e1.record(stream)
+            e1.synchronize()
+            t.append(e0.elapsed_time(e1))
+        return t
+
     for _ in range(warmup):
         step()
     torch.cuda.synchronize()
+    barrier(ws)
+    times = timed_reps()
+    barrier(ws)
     kda.profiler_read(reset=True)
     kda.profiler_enable(True)
-    barrier(ws)
-    times = []
-    for _ in range(reps):
-        if fbuf is not None:
-            fbuf.fill_(1.0)
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        step()
-        e1.record(stream)
-        e1.synchronize()
-        times.append(e0.elapsed_time(e1))
-    barrier(ws)
+    profiled = timed_reps()
     kda.profiler_enable(False)
     stats = kda.profiler_read(reset=True)
     ms = max_over_ranks(statistics.median(times), ws)
     kname, (_, ktimed, kms) = max(stats.items(), key=lambda kv: kv[1][2])
     launches_per_step = ktimed / reps
     roof = prefill_roofline(kname, cfg, kms / max(1, ktimed), launches_per_step, peaks)
-    roof["share_of_step"] = kms / reps / ms
+    roof["share_of_step"] = kms / reps / statistics.median(profiled)
     res = {"workload": cfg.name, "tokens_per_s": cfg.tokens * ws / (ms / 1e3), "ms": ms,
+           "ms_profiled": statistics.median(profiled),
            "reps": reps, "statistic": "median", "io": cfg.io_dtype, "dk": cfg.dk, "H": cfg.H,
            "l2": ("256 MB buffer written before every rep (the inputs fit in L2)" if flush
                   else "inputs larger than L2"),

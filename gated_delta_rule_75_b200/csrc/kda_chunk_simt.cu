@@ -52,17 +52,17 @@ static cudaError_t run_simt_t(const PrefillArgs& a, float* ws, int64_t Hg, cudaS
         if (a.si.chunks_upper > 0) {
             dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
             LaunchScope scope(st, K_PREP_SIMT);
-            chunk_prep_simt_kernel<T, DK, DV><<<gp, kSimtPrepThreads, smem_prep, st>>>(
-                (const T*)a.q, (const T*)a.k, (const T*)a.v, a.log_alpha, a.beta, a.si, a.H, hb,
-                Hg, a.scale, ws, a.gate_scalar ? 1 : 0);
-            if ((e = cudaGetLastError())) return e;
+            e = launch_pdl(chunk_prep_simt_kernel<T, DK, DV>, gp, dim3(kSimtPrepThreads), smem_prep, st,
+                           (const T*)a.q, (const T*)a.k, (const T*)a.v, a.log_alpha, a.beta, a.si, a.H, hb,
+                           Hg, a.scale, ws, a.gate_scalar ? 1 : 0);
+            if (e) return e;
         }
         dim3 gs((unsigned)(a.si.N * hg * (DV / 32)));
         {
             LaunchScope scope(st, K_STATE_SIMT);
-            chunk_state_simt_kernel<T, DK, DV><<<gs, 256, smem_state, st>>>(ws, a, hb, Hg);
+            e = launch_pdl(chunk_state_simt_kernel<T, DK, DV>, gs, dim3(256), smem_state, st, ws, a, hb, Hg);
         }
-        if ((e = cudaGetLastError())) return e;
+        if (e) return e;
     }
     return cudaSuccess;
 }

@@ -197,6 +197,8 @@ chunk_prep_simt_kernel(const T* __restrict__ q, const T* __restrict__ k, const T
                        SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, float scale,
                        float* __restrict__ ws, int gate_scalar)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     constexpr int C = kChunk, NT = kSimtPrepThreads;
     extern __shared__ __align__(16) float smem[];
     float* sK = smem;                 // [C][DK]
@@ -509,6 +511,8 @@ template <typename T, int DK, int DV, bool kBwd = false>
 __global__ void __launch_bounds__(256, kBwd ? 2 : 1)   // occupancy set by shared memory
 chunk_state_simt_kernel(float* __restrict__ ws, PrefillArgs a, int64_t h_base, int64_t Hg)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     // kBwd: backward blocks; every chunk's entry state is saved (Sx) and
     // no output is written
     constexpr int64_t kStride = kBwd ? BwdWs<DK, DV>::size : SimtWs<DK, DV>::size;

@@ -247,6 +247,8 @@ chunk_prep_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __restr
                      SeqInfo si, int64_t H, int64_t h_base, int64_t Hg, int64_t hg,
                      unsigned char* __restrict__ ws, int* __restrict__ err, int* __restrict__ range_flag)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -666,6 +668,8 @@ chunk_prep_gdn_tc_kernel(const __grid_constant__ PrepMaps maps, const float* __r
                          const float* __restrict__ log_a, SeqInfo si, int64_t H, int64_t h_base,
                          int64_t Hg, unsigned char* __restrict__ ws, int* __restrict__ err)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -849,6 +853,8 @@ chunk_state_tc_kernel(const unsigned char* __restrict__ ws, const __grid_constan
 {
     constexpr bool kOut = kMode == WALK_SEQ || kMode == WALK_FINAL;   // outputs written
     constexpr bool kV = kMode != WALK_MAP;                            // v tiles used
+    griddep_wait();
+    griddep_launch_dependents();
     if (sp.skip && *sp.skip) return;               // the fused kernel takes this call over
     extern __shared__ unsigned char smem_raw[];
     unsigned char* sm = reinterpret_cast<unsigned char*>(
@@ -1240,17 +1246,17 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         dim3 gp((unsigned)a.si.chunks_upper, (unsigned)hg);
         LaunchScope scope(s, K_PREP_TC);
         if (a.gate_scalar) {
-            tc::chunk_prep_gdn_tc_kernel<<<gp, tc::PT, tc::GP_SMEM, s>>>(
-                maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, w, err);
+            return launch_pdl(tc::chunk_prep_gdn_tc_kernel, gp, dim3(tc::PT), tc::GP_SMEM, s,
+                              maps, a.beta, a.log_alpha, a.si, a.H, hb, Hg, w, err);
         } else {
             // persistent: two CTAs per SM walk the (chunk, head) items
             const int64_t items = a.si.chunks_upper * hg;
             if (items > INT32_MAX) return cudaErrorInvalidValue;   // items are 32-bit in the kernel
             const int64_t slots = 2 * device_sm_count();
-            tc::chunk_prep_tc_kernel<<<(unsigned)(items < slots ? items : slots), tc::PT, tc::P_SMEM, s>>>(
-                maps, a.beta, a.si, a.H, hb, Hg, hg, w, err, a.range_flag);
+            return launch_pdl(tc::chunk_prep_tc_kernel, dim3((unsigned)(items < slots ? items : slots)),
+                              dim3(tc::PT), tc::P_SMEM, s, maps, a.beta, a.si, a.H, hb, Hg, hg, w, err,
+                              a.range_flag);
         }
-        return cudaGetLastError();
     };
     SegPlan none;
     memset(&none, 0, sizeof(none));
@@ -1259,12 +1265,12 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         dim3 gs((unsigned)(a.si.N * hg));
         LaunchScope scope(s, K_STATE_TC);
         if (a.h0)
-            tc::chunk_state_tc_kernel<true, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, a.scale, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
-        else
-            tc::chunk_state_tc_kernel<false, tc::WALK_SEQ><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, a.scale, nullptr, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, none);
-        return cudaGetLastError();
+            return launch_pdl(tc::chunk_state_tc_kernel<true, tc::WALK_SEQ>, gs, dim3(tc::ST), tc::S_SMEM, s,
+                              w, vmap, omap, a.scale, a.h0, (__nv_bfloat16*)a.out, a.hT, a.si, a.H, hb, Hg,
+                              a.slots, a.P, err, none);
+        return launch_pdl(tc::chunk_state_tc_kernel<false, tc::WALK_SEQ>, gs, dim3(tc::ST), tc::S_SMEM, s,
+                          w, vmap, omap, a.scale, (const float*)nullptr, (__nv_bfloat16*)a.out, a.hT, a.si,
+                          a.H, hb, Hg, a.slots, a.P, err, none);
     };
     // one walk over every segment of the plan (grid: segment bound x heads)
     auto launch_walk = [&](int mode, const SegPlan& sp, int64_t hb, int64_t hg, unsigned char* w,
@@ -1273,16 +1279,16 @@ cudaError_t run_prefill_tc(const PrefillArgs& a, unsigned char* ws, int64_t Hg, 
         dim3 gs((unsigned)(sp.upper * hg));
         LaunchScope scope(s, mode == tc::WALK_FINAL ? K_STATE_TC : K_STATE_SEG_TC);
         __nv_bfloat16* o = (__nv_bfloat16*)a.out;
+        const float* no_h0 = nullptr;
+        float* no_hT = nullptr;
         if (mode == tc::WALK_VALUE)
-            tc::chunk_state_tc_kernel<false, tc::WALK_VALUE><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, a.scale, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
-        else if (mode == tc::WALK_MAP)
-            tc::chunk_state_tc_kernel<false, tc::WALK_MAP><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, a.scale, nullptr, o, nullptr, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
-        else
-            tc::chunk_state_tc_kernel<false, tc::WALK_FINAL><<<gs, tc::ST, tc::S_SMEM, s>>>(
-                w, vmap, omap, a.scale, nullptr, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
-        return cudaGetLastError();
+            return launch_pdl(tc::chunk_state_tc_kernel<false, tc::WALK_VALUE>, gs, dim3(tc::ST), tc::S_SMEM, s,
+                              w, vmap, omap, a.scale, no_h0, o, no_hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+        if (mode == tc::WALK_MAP)
+            return launch_pdl(tc::chunk_state_tc_kernel<false, tc::WALK_MAP>, gs, dim3(tc::ST), tc::S_SMEM, s,
+                              w, vmap, omap, a.scale, no_h0, o, no_hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
+        return launch_pdl(tc::chunk_state_tc_kernel<false, tc::WALK_FINAL>, gs, dim3(tc::ST), tc::S_SMEM, s,
+                          w, vmap, omap, a.scale, no_h0, o, a.hT, a.si, a.H, hb, Hg, a.slots, a.P, err, sp);
     };
 
     // segment buffers sit after the operand images of one head group

@@ -11,6 +11,20 @@ namespace kda {
 constexpr int kChunk = 64;       // tokens per chunk of the chunkwise prefill
 constexpr int kSubChunk = 16;    // sub-chunk used for exponent references
 
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization (launch_pdl) may be scheduled while the kernel before it on the
+// stream is still running or draining.  griddep_wait() holds the calling thread
+// until every grid that this one depends on has completed and its memory writes
+// are visible, so each such kernel calls it before its first global-memory access;
+// griddep_launch_dependents() lets the next kernel's CTAs be scheduled as SMs free
+// up (they still wait for this grid to complete).  Both do nothing in a kernel
+// launched without the attribute.
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void griddep_launch_dependents()
+{
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // I/O element access: fp32 or bf16 storage, fp32 arithmetic.
 template <typename T> struct IO;
 template <> struct IO<float> {

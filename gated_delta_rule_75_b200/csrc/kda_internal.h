@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include <atomic>
+#include <utility>
 
 #include "kda.h"
 
@@ -252,6 +253,29 @@ enum KernelId {
     K_FUSED_TC,
     K_KERNEL_COUNT
 };
+
+// Launch with programmatic stream serialization: the grid may start while the
+// previous kernel on `st` drains (the kernel itself calls griddep_wait before it
+// touches global memory).  Used for the launches of one prefill call, which
+// follow each other back to back on one stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       Args&&... args)
+{
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = grid;
+    cfg.blockDim = block;
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+    const cudaError_t g = cudaGetLastError();   // clears the launch error it may have set
+    return e != cudaSuccess ? e : g;
+}
 
 // Opened around every kernel launch: counts it and, while the profiler is
 // enabled, records start/stop CUDA events on the launching stream.

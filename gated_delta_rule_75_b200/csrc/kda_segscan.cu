@@ -12,19 +12,27 @@
 // columns of X stay in shared memory across the segments (columns of the
 // state never mix).  Each M_s is staged in shared memory by asynchronous
 // 16-byte copies (all threads, coalesced), double-buffered so that M_{s+1}
-// arrives while X_{s+1} = M_s X_s + B_s is computed.  Each thread owns a 4 x 4
-// register tile of the product (rows r, r+32, r+64, r+96; 4 columns), so every
-// 16-byte shared-memory load feeds 16 FMAs; rows of the staged M are padded to
-// 132 floats so that the 8 consecutive rows a warp reads fall in distinct banks.
+// arrives while X_{s+1} = M_s X_s + B_s is computed.  The contraction over the
+// dk rows of X is split four ways: four groups of 128 threads (four warps per
+// scheduler, so the shared-memory loads of one warp hide behind the FMAs of
+// the others) each take a quarter of the rows, and group 0 adds the other
+// three partial products from shared memory.  In every group a thread owns a
+// 4 x 4 register tile of the product (rows r, r+32, r+64, r+96; 4 columns), so
+// every 16-byte shared-memory load feeds 16 FMAs; rows of the staged M are
+// padded to 132 floats so that the 8 consecutive rows a warp reads fall in
+// distinct banks.
 #include "kda_common.cuh"
 #include "kda_internal.h"
 
 namespace kda {
 
-constexpr int kPrefixThreads = 128;
+constexpr int kPrefixGroups = 4;                               // split of the contraction
+constexpr int kPrefixThreads = 128 * kPrefixGroups;
 constexpr int kPrefixCols = 16;
 constexpr int kMPitch = 132;                                   // floats per staged row
-constexpr int kPrefixSmem = 2 * 128 * kMPitch * (int)sizeof(float);
+constexpr int kMapFloats = 2 * 128 * kMPitch;                  // the double-buffered M_s
+constexpr int kPartFloats = (kPrefixGroups - 1) * 128 * kPrefixCols;
+constexpr int kPrefixSmem = (kMapFloats + kPartFloats) * (int)sizeof(float);
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src)
 {
@@ -37,10 +45,13 @@ __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commi
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-__global__ void __launch_bounds__(kPrefixThreads, 1)   // one CTA per SM: registers uncapped
+__global__ void __launch_bounds__(kPrefixThreads, 1)   // one CTA per SM
 affine_prefix_kernel(PrefixArgs p)
 {
-    extern __shared__ __align__(16) float msm[];               // 2 x [128][kMPitch]
+    griddep_wait();
+    griddep_launch_dependents();
+    extern __shared__ __align__(16) float msm[];               // 2 x [128][kMPitch], partials
+    float* part = msm + kMapFloats;                            // [groups - 1][128][kPrefixCols]
     __shared__ __align__(16) float X[128][kPrefixCols];
     const int64_t chain = blockIdx.x;
     const int64_t n = chain / p.hg;
@@ -48,8 +59,10 @@ affine_prefix_kernel(PrefixArgs p)
     const int64_t h = p.h_base + hl;
     const int64_t head = p.abs_head ? h : hl;
     const int tid = threadIdx.x;
-    // this thread: rows rg + 32 i (i < dk / 32) and columns j0 + 4 cg .. +3
-    const int cg = tid & 3, rg = tid >> 2;
+    // this thread: rows rg + 32 i (i < dk / 32) and columns j0 + 4 cg .. +3 of the product,
+    // summed over rows kg dk / 4 .. (kg + 1) dk / 4 - 1 of X; group 0 holds X_s
+    const int kg = tid >> 7, gt = tid & 127;
+    const int cg = gt & 3, rg = gt >> 2;
     const int j = blockIdx.y * kPrefixCols + 4 * cg;
     const int nr = p.dk >> 5;
     const int64_t dkdk = (int64_t)p.dk * p.dk, dkdv = (int64_t)p.dk * p.dv;
@@ -86,7 +99,7 @@ affine_prefix_kernel(PrefixArgs p)
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
         x[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (i < nr) {
+        if (kg == 0 && i < nr) {
             const int r = rg + 32 * i;
             if (p.h0 && sidx >= 0)
                 x[i] = *reinterpret_cast<const float4*>(p.h0 + sidx * dkdv + (int64_t)r * p.dv + j);
@@ -96,7 +109,7 @@ affine_prefix_kernel(PrefixArgs p)
 
     for (int64_t s = 0; s < count; ++s) {
         const int64_t idx = (base + s) * p.hstride + head;
-        if (p.starts) {
+        if (p.starts && kg == 0) {
 #pragma unroll
             for (int i = 0; i < 4; ++i)
                 if (i < nr)
@@ -107,7 +120,7 @@ affine_prefix_kernel(PrefixArgs p)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {                          // B_s: in flight during the wait
             acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (i < nr)
+            if (kg == 0 && i < nr)
                 acc[i] = *reinterpret_cast<const float4*>(p.offs + idx * dkdv +
                                                           (int64_t)(rg + 32 * i) * p.dv + j);
         }
@@ -127,7 +140,7 @@ affine_prefix_kernel(PrefixArgs p)
         };
         if (nr == 4) {
 #pragma unroll 2
-            for (int k = 0; k < 128; k += 4) {
+            for (int k = 32 * kg; k < 32 * kg + 32; k += 4) {
                 float4 m[4];
 #pragma unroll
                 for (int i = 0; i < 4; ++i) m[i] = *reinterpret_cast<const float4*>(mb + 32 * i * kMPitch + k);
@@ -141,7 +154,7 @@ affine_prefix_kernel(PrefixArgs p)
             }
         } else {
 #pragma unroll 2
-            for (int k = 0; k < 64; k += 4) {
+            for (int k = 16 * kg; k < 16 * kg + 16; k += 4) {
                 float4 m[2];
 #pragma unroll
                 for (int i = 0; i < 2; ++i) m[i] = *reinterpret_cast<const float4*>(mb + 32 * i * kMPitch + k);
@@ -154,16 +167,32 @@ affine_prefix_kernel(PrefixArgs p)
                 }
             }
         }
-        __syncthreads();                                       // every read of X_s and M_s is done
+        if (kg > 0) {
+            float* pp = part + (kg - 1) * 128 * kPrefixCols;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            if (i < nr) {
-                x[i] = acc[i];
-                *reinterpret_cast<float4*>(&X[rg + 32 * i][4 * cg]) = acc[i];
+            for (int i = 0; i < 4; ++i)
+                if (i < nr) *reinterpret_cast<float4*>(pp + (rg + 32 * i) * kPrefixCols + 4 * cg) = acc[i];
+        }
+        __syncthreads();                                       // partials written; X_s, M_s read
+        if (kg == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (i < nr) {
+                    const int r = rg + 32 * i;
+#pragma unroll
+                    for (int g = 0; g < kPrefixGroups - 1; ++g) {
+                        const float4 v = *reinterpret_cast<const float4*>(part + (g * 128 + r) * kPrefixCols + 4 * cg);
+                        acc[i].x += v.x; acc[i].y += v.y; acc[i].z += v.z; acc[i].w += v.w;
+                    }
+                    x[i] = acc[i];
+                    *reinterpret_cast<float4*>(&X[r][4 * cg]) = acc[i];
+                }
             }
         }
+        // the next step's first barrier orders X_{s+1} before its reads, and this step's
+        // partial reads before the next partial writes
     }
-    if (p.out && sidx >= 0) {
+    if (p.out && sidx >= 0 && kg == 0) {
 #pragma unroll
         for (int i = 0; i < 4; ++i)
             if (i < nr)
@@ -173,7 +202,7 @@ affine_prefix_kernel(PrefixArgs p)
 
 cudaError_t launch_affine_prefix(const PrefixArgs& p, cudaStream_t st)
 {
-    if (p.dk > 128 || p.dv % kPrefixCols != 0 || p.dk % 4 != 0) return cudaErrorInvalidValue;
+    if ((p.dk != 64 && p.dk != 128) || p.dv % kPrefixCols != 0) return cudaErrorInvalidValue;
     if (p.N * p.hg == 0) return cudaSuccess;
     static std::atomic<uint64_t> attr_done{0};
     cudaError_t e = once_per_device(attr_done, [] {
@@ -183,8 +212,7 @@ cudaError_t launch_affine_prefix(const PrefixArgs& p, cudaStream_t st)
     if (e) return e;
     dim3 grid((unsigned)(p.N * p.hg), (unsigned)(p.dv / kPrefixCols));
     LaunchScope scope(st, K_AFFINE_PREFIX);
-    affine_prefix_kernel<<<grid, kPrefixThreads, kPrefixSmem, st>>>(p);
-    return cudaGetLastError();
+    return launch_pdl(affine_prefix_kernel, grid, dim3(kPrefixThreads), kPrefixSmem, st, p);
 }
 
 __global__ void fill_identity_kernel(float* __restrict__ dst, int64_t total, int d)

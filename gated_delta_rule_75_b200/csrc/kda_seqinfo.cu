@@ -27,6 +27,8 @@ chunk_offsets_kernel(const int32_t* __restrict__ cu, int64_t N, int64_t T_total,
                      int* __restrict__ err, int64_t seg_len, int64_t seg_cap,
                      int64_t* __restrict__ seg_off)
 {
+    griddep_wait();
+    griddep_launch_dependents();
     using Scan = cub::BlockScan<int64_t, kScanThreads>;
     __shared__ typename Scan::TempStorage tmp;
     __shared__ int64_t carry;
@@ -97,9 +99,8 @@ cudaError_t launch_chunk_offsets(const int32_t* cu, int64_t N, int64_t T_total, 
 {
     if (seg_off != nullptr && seg_len < 1) return cudaErrorInvalidValue;
     LaunchScope scope(st, K_CHUNK_OFFSETS);
-    chunk_offsets_kernel<<<1, kScanThreads, 0, st>>>(cu, N, T_total, cap, chunk_off, order,
-                                                     err_flag, seg_len, seg_cap, seg_off);
-    return cudaGetLastError();
+    return launch_pdl(chunk_offsets_kernel, dim3(1), dim3(kScanThreads), 0, st, cu, N, T_total, cap,
+                      chunk_off, order, err_flag, seg_len, seg_cap, seg_off);
 }
 
 }  // namespace kda
