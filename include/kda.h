@@ -29,6 +29,14 @@
  *    call takes the error word itself after its own work (so it synchronises
  *    `stream`) and returns KDA_ERR_TIMEOUT or KDA_ERR_INVALID_ARG for the bits
  *    it finds.
+ *  - The prefill's kernels are launched with programmatic stream
+ *    serialization and let the next grid on `stream` be scheduled early; each
+ *    of them waits for the previous grid to complete before it touches memory.
+ *    Ordinary launches, copies and events after a call are ordered as usual.
+ *    A kernel the caller launches after a call WITH programmatic stream
+ *    serialization must wait for its dependency (cudaGridDependencySynchronize
+ *    or griddepcontrol.wait) before it reads the call's outputs, as that
+ *    launch mode requires of every consumer.
  *  - q and k are expected to be L2-normalised per (token, head) by the caller
  *    (the delta rule is only stable for normalised keys, as the same page notes
  *    in its warning on key normalisation); the kernels do not renormalise.
