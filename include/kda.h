@@ -29,9 +29,10 @@
  *    call takes the error word itself after its own work (so it synchronises
  *    `stream`) and returns KDA_ERR_TIMEOUT or KDA_ERR_INVALID_ARG for the bits
  *    it finds.
- *  - The prefill's kernels are launched with programmatic stream
- *    serialization and let the next grid on `stream` be scheduled early; each
- *    of them waits for the previous grid to complete before it touches memory.
+ *  - The prefill's kernels other than the fused tensor-core kernel are
+ *    launched with programmatic stream serialization and let the next grid on
+ *    `stream` be scheduled early; each of them waits for the previous grid to
+ *    complete before it touches memory.
  *    Ordinary launches, copies and events after a call are ordered as usual.
  *    A kernel the caller launches after a call WITH programmatic stream
  *    serialization must wait for its dependency (cudaGridDependencySynchronize
