@@ -577,9 +577,12 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 for (int y = 0; y < 32; ++y) G[y] += s0;
             }
             const float Gl = s0 + s1;             // last row
-            float mx = 0.f;
+            float mx = 0.f, mxw = 0.f;            // largest |G| and |G - s0| of these tokens
 #pragma unroll
-            for (int y = 0; y < 32; ++y) mx = fmaxf(mx, fabsf(G[y]));
+            for (int y = 0; y < 32; ++y) {
+                mx = fmaxf(mx, fabsf(G[y]));
+                mxw = fmaxf(mxw, fabsf(G[y] - s0));
+            }
 
             // k^T, q^T of this chunk in TMEM; image slot s free (chunk k - 2 walked)
             if (leader) {
@@ -595,7 +598,13 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 if (leader && k >= 1) o = fwait(&bars.m1, (k - 1) & 1, err, 6, abort);
                 return bar_and_named(NB_PREP, 256, o);
             };
-            const bool fast = bar_and_named(NB_PREP, 256, !(mx > kRange));
+            // one exponent reference per chunk and channel: the chunk start while every |G|
+            // is within kRange, else the first half's total s0 while every |G - s0| is (a
+            // chunk decaying by up to twice the range); past that, the level passes
+            bool fast = bar_and_named(NB_PREP, 256, !(mx > kRange));
+            const bool wide = !fast && bar_and_named(NB_PREP, 256, !(mxw > kRange));
+            fast = fast || wide;
+            const float rref = wide ? s0 : 0.f;
 
             unsigned char* qg = sm + F_QG + s * 16384;
             unsigned char* kl = sm + F_KLAQ + s * 24576;
@@ -643,9 +652,11 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
             };
 
             if (fast) {
-                // ---- (b1) e^{G_i - G_j} = e^{G_i} e^{-G_j}: the image tiles K e^G, Q e^G are the
-                // row operands of A and Aqk, K e^{-G} the column operand; K e^{Gl - G} = K e^{-G} e^{Gl}
-                const float Egl = ex2(Gl);
+                // ---- (b1) e^{G_i - G_j} = e^{G_i - r} e^{r - G_j} with the reference r = 0 or s0:
+                // K e^{G - r}, Q e^{G - r} (with r = 0 the image tiles K e^G, Q e^G) are the row
+                // operands of A and Aqk, K e^{r - G} the column operand; K e^{Gl - G} =
+                // K e^{r - G} e^{Gl - r}
+                const float Egl = ex2(Gl - rref);
 #pragma unroll
                 for (int hb = 0; hb < 2; ++hb) {
                     float kf[16], qf[16];
@@ -656,7 +667,8 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int y = 8 * m + e;
-                            const float e1 = ex2(G[16 * hb + y]), e2 = ex2(-G[16 * hb + y]);
+                            const float gg = G[16 * hb + y] - rref;
+                            const float e1 = ex2(gg), e2 = ex2(-gg);
                             a8[e] = kf[y] * e1;
                             b8[e] = qf[y] * e1;
                             c8[e] = kf[y] * e2;
@@ -679,8 +691,32 @@ chunk_fused_tc_kernel(const __grid_constant__ CUtensorMap kmap, const __grid_con
                 issue_a(true);
                 if (!wait_m1()) break;
                 if (!wait_a()) break;
-                // k^T, q^T were read before A was issued; signalled only now so that the next
-                // chunk's transposes do not queue ahead of A on the tensor pipe
+                if (wide) {
+                    // A has read the s0-referenced rows: the image tiles K e^G, Q e^G are
+                    // written again at the chunk start (from k^T, q^T, still in TMEM), as the
+                    // chunk-start reference writes them
+#pragma unroll
+                    for (int hb = 0; hb < 2; ++hb) {
+                        float kf[16], qf[16];
+                        load_kq(hb, kf, qf);
+#pragma unroll
+                        for (int m = 0; m < 2; ++m) {
+                            float a8[8], b8[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) {
+                                const float e1 = ex2(G[16 * hb + 8 * m + e]);
+                                a8[e] = kf[8 * m + e] * e1;
+                                b8[e] = qf[8 * m + e] * e1;
+                            }
+                            const uint32_t off = ct_off(pc, 32 * ph + 16 * hb + 8 * m);
+                            *reinterpret_cast<uint4*>(sm + F_KG + off) = pack8(a8);
+                            *reinterpret_cast<uint4*>(qg + off) = pack8(b8);
+                        }
+                    }
+                }
+                // k^T, q^T were read before A was issued (and again just above for a chunk
+                // referenced to s0); signalled only now so that the next chunk's transposes
+                // do not queue ahead of A on the tensor pipe
                 if (l == 0) mbar_arrive(&bars.ktf);
                 // ---- A (fp32, beta-scaled rows, for the inverse) and Aqk (bf16 image)
                 float d[32];

@@ -80,6 +80,18 @@ def test_fused_exact_at_any_decay(kda, shift, impl):
     check_full(kda, cfg, impl)
 
 
+@pytest.mark.parametrize("shift", [0.3, 0.8])
+def test_fused_mid_chunk_reference(kda, shift):
+    """Mean per-token decay about e^-1.0 and e^-1.3: many (0.3) or all (0.8) chunks
+    decay past the chunk-start reference's range (2^100 over 64 tokens) but within
+    2^100 of the first half's decay sum, so the fused kernel takes one A/Aqk MMA
+    with factors referenced there and writes the image rows back at the chunk start;
+    parity holds, the partial last chunk included."""
+    cfg = W.small_prefill(B=2, T=300, H=2, dk=128, dv=128, io_dtype="bf16", seed=15,
+                          gate_shift=shift, h0_std=0.05)
+    check_full(kda, cfg, "tensorcore_fused")
+
+
 def test_fused_mixed_fast_and_fallback_chunks(kda):
     """Chunks of both kinds in one call (fast decay in one sequence, slow in the
     other, packed): the per-chunk choice of factors is independent."""
