@@ -279,6 +279,11 @@ def test_chunk_backward_equals_oracle(L):
 # e^{G_i - G_f} <= 1 and e^{G_f - G_j} <= 1 for every channel, at any decay rate.
 # One product per level covers every block (entries across blocks are not used),
 # and a last product without exponents gives the diagonal of Aqk.
+# Between the two, a chunk whose every |G_tc - G_31,c| stays within RANGE_LOG2
+# (G_31 = the channel's decay over the first 32 tokens) is split as
+# e^{G_ic - G_31,c} e^{G_31,c - G_jc}: still one product, for chunks decaying by up to
+# twice the range; its row operands differ from the image tiles, which the prep then
+# writes again at the chunk start.
 RANGE_LOG2 = 100.0
 
 
@@ -293,6 +298,24 @@ def _pairwise(qc, kc, gc):
 def _fast_needs_fallback(gc):
     G = np.cumsum(gc, axis=0)
     return np.abs(G).max() / np.log(2.0) > RANGE_LOG2
+
+
+def _reference_choice(gc):
+    """Which form the fused prep takes for one chunk: 'start', 'mid' or 'levels'."""
+    G = np.cumsum(gc, axis=0) / np.log(2.0)
+    if np.abs(G).max() <= RANGE_LOG2:
+        return "start"
+    if np.abs(G - G[min(31, len(G) - 1)]).max() <= RANGE_LOG2:
+        return "mid"
+    return "levels"
+
+
+def _mid_reference(qc, kc, gc):
+    """The mid-chunk split: A (strictly lower), Aqk (lower) and every factor's exponent."""
+    G = np.cumsum(gc, axis=0)
+    x = G - G[min(31, len(G) - 1)]
+    KG, QG, Kn = kc * np.exp(x), qc * np.exp(x), kc * np.exp(-x)
+    return np.tril(KG @ Kn.T, -1), np.tril(QG @ Kn.T, 0), x
 
 
 def _single_reference(qc, kc, gc, dtype=np.float64):
@@ -330,10 +353,10 @@ def _level_passes(qc, kc, gc, dtype=np.float64):
 @pytest.mark.parametrize("shift", [-2.0, 0.0])
 def test_single_reference_reproduces_pairs(shift):
     """The workload's gate distributions stay inside the e^{+-G} range (a chunk
-    of the e^-0.8-per-token workloads decays by about 74 log2 units, so about
-    one chunk in 600 exceeds 100 and takes the level passes) and the factored
-    products equal the pairwise sums; the row operands are the image tiles
-    K e^G and Q e^G."""
+    of the e^-0.8-per-token workloads decays by about 74 log2 units on average; a
+    channel exceeds 100 about once in 20,000, so about one chunk-head in 170 takes
+    the mid-chunk split instead) and the factored products equal the pairwise
+    sums; the row operands are the image tiles K e^G and Q e^G."""
     rng = np.random.default_rng(50)
     q, k, v, g, b = _inputs(rng, C, 128, 4, gate_shift=shift)
     assert not _fast_needs_fallback(g)
@@ -370,3 +393,39 @@ def test_level_fallback_slow_decay():
     A, Aqk, _ = _level_passes(q, k, g)
     np.testing.assert_allclose(A, A_ref, rtol=0, atol=1e-12)
     np.testing.assert_allclose(Aqk, Aqk_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("shift", [0.3, 0.8])
+def test_mid_reference_reproduces_pairs(shift):
+    """About e^-1.0 and e^-1.3 of decay per token: a chunk decays past the
+    chunk-start split's range but every factor of the mid-chunk split stays within
+    2^+-100, and its products equal the pairwise sums (ragged chunk included)."""
+    rng = np.random.default_rng(53)
+    for L in (C, 44):
+        q, k, v, g, b = _inputs(rng, L, 128, 4, gate_shift=shift)
+        if L == C:
+            assert _reference_choice(g) == "mid"
+        if _reference_choice(g) == "levels":
+            continue
+        A_ref, Aqk_ref = _pairwise(q, k, g)
+        A, Aqk, x = _mid_reference(q, k, g)
+        assert np.abs(x).max() / np.log(2.0) <= RANGE_LOG2
+        np.testing.assert_allclose(A, A_ref, rtol=0, atol=1e-12)
+        np.testing.assert_allclose(Aqk, Aqk_ref, rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("shift", [-2.0, 0.0])
+def test_workload_gates_never_need_the_level_passes(shift):
+    """At both workloads' gate distributions (log_alpha = -softplus(N(0, 1) + shift),
+    per channel and token), 4000 chunk-heads of 128 channels all take one of the two
+    single-product splits; at shift 0 some take the mid-chunk one."""
+    rng = np.random.default_rng(54)
+    x = rng.standard_normal((4000, C, 128)) + shift
+    G = np.cumsum(np.log1p(np.exp(x)), axis=1) / np.log(2.0)     # |G| in log2 units
+    start = np.abs(G).max(axis=(1, 2)) <= RANGE_LOG2
+    mid = np.abs(G - G[:, 31:32, :]).max(axis=(1, 2)) <= RANGE_LOG2
+    assert np.all(start | mid)
+    if shift == 0.0:
+        assert not np.all(start)
+    else:
+        assert np.all(start)
