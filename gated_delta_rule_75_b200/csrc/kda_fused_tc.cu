@@ -33,11 +33,13 @@
 // pipe.  The decay factors e^{G_i - G_j} are split as e^{G_i} e^{-G_j}
 // when every |G| of the chunk stays within 2^100: the row operands of A and Aqk
 // are then the image tiles K e^G and Q e^G themselves, the column operand is
-// K e^{-G}, and A and Aqk are one MMA.  Otherwise the lower triangle is taken
-// level by level (blocks of 64, 32, ..., 2 rows; each pair i > j at the level
-// where i and j fall in different halves, both factors referenced to the first
-// row of the upper half and so <= 1), plus one product for the diagonal: exact
-// at any decay rate.  The state walk of chunk c (U^T = V^T T'^T + S^T (-W^T),
+// K e^{-G}, and A and Aqk are one MMA.  When instead every |G - s0| does (s0 = the
+// channel's decay over the first 32 tokens), the same MMA takes e^{G_i - s0} and
+// e^{s0 - G_j}, and the image rows are written again at the chunk start once it has
+// completed.  Past that the lower triangle is taken level by level (blocks of 64,
+// 32, ..., 2 rows; each pair i > j at the level where i and j fall in different
+// halves, both factors referenced to the first row of the upper half and so <= 1),
+// plus one product for the diagonal: exact at any decay rate.  The state walk of chunk c (U^T = V^T T'^T + S^T (-W^T),
 // O^T = S^T (Q e^G)^T + U^T Aqk^T, S^T += U^T (K e^{Gl - G}), as three MMA groups:
 // [O^T | U^T] = S^T [(Q e^G)^T | -W^T] with N = 128, U^T += V^T T'^T, and
 // [S^T | O^T] += U^T [K e^{Gl - G} ; Aqk] with N = 192) overlaps the prep
