@@ -69,7 +69,7 @@ constexpr int D = 128;
 constexpr int NT = 448;
 constexpr int AP = 68;                      // row pitch (floats) of the fp32 A and T
 constexpr float kLog2e = 1.4426950408889634f;
-constexpr float kRange = 100.f;             // fast path: every |G| (log2) within 100
+constexpr float kRange = 100.f;             // one-product forms: every |G| or |G - s0| (log2) within
 constexpr long long kWaitCycles = 4000000000LL;
 
 constexpr int W_WALK = 8;                   // walk warps 8-11
